@@ -1,0 +1,113 @@
+"""Pins for the oracle's cross-layer consistency scoring (StreamCacheVGGT page,
+sections 2.1.1 to 2.1.4): closed forms, a library variance, exact sums."""
+import math
+import statistics
+from fractions import Fraction
+
+import numpy as np
+
+from oracle import OracleConfig, StreamOracle, to_f32
+
+
+def _orc(T, lam=0.5, window=5, layers=8):
+    cfg = OracleConfig(num_layers=layers, num_heads=1, head_dim=4, tokens_per_frame=T, num_special_tokens=1,
+                       page_size=4, window_frames=0, scale_frames=0, kv_dtype="bf16", softmax_scale=0.125,
+                       budget_tokens=10 ** 6, lam=lam, rank_window=window, residual_dim=8)
+    return StreamOracle(cfg)
+
+
+def _residual_with_norms(norms, dim=8):
+    r = np.zeros((len(norms), dim))
+    r[:, 0] = norms
+    return r
+
+
+def test_constant_rank_gives_cons_one_and_fifty_percent_bonus():
+    T = 12
+    orc = _orc(T)
+    norms = np.arange(1, T + 1, dtype=np.float64) * 0.75
+    for l in range(7):
+        sh = orc.score(l, 0, _residual_with_norms(norms))
+        # ranks never move -> sigma = 0 -> Cons = 1 -> s_hat = fp32(s * 1.5)
+        np.testing.assert_array_equal(sh, to_f32(to_f32(norms) * 1.5))
+
+
+def test_lambda_zero_returns_raw_score():
+    rng = np.random.default_rng(0)
+    orc = _orc(50, lam=0.0)
+    for l in range(6):
+        r = rng.standard_normal((50, 8))
+        sh = orc.score(l, 0, r)
+        exact = np.array([math.sqrt(math.fsum(float(v) ** 2 for v in row)) for row in r])
+        np.testing.assert_array_equal(sh, to_f32(exact))
+
+
+def test_opposite_ranks_over_two_layers_give_cons_zero():
+    # token 0 is best at layer 0 and worst at layer 1: normalised ranks 0 and 1,
+    # population sigma = 0.5 > 1/sqrt(12) -> Cons = max(0, 1 - 0.5*sqrt(12)) = 0
+    T = 10
+    orc = _orc(T)
+    n0 = np.linspace(1, 2, T)[::-1].copy()   # token 0 largest
+    orc.score(0, 0, _residual_with_norms(n0))
+    n1 = np.linspace(1, 2, T)                # token 0 smallest
+    sh = orc.score(1, 0, _residual_with_norms(n1))
+    assert sh[0] == float(np.float32(n1[0]))                 # no bonus for token 0
+    # a middle token that keeps rank ~ (T-1)/2 on both layers gets a bonus > 0
+    assert sh[T // 2] > float(np.float32(n1[T // 2]))
+
+
+def test_sigma_matches_library_population_variance():
+    rng = np.random.default_rng(1)
+    T = 40
+    orc = _orc(T, lam=0.5, window=5)
+    ranks = []
+    for l in range(8):
+        r = rng.standard_normal((T, 8))
+        s = to_f32(np.sqrt((r * r).sum(axis=1)))
+        # library ranking: stable argsort of -s gives ties to the lower index
+        order = np.argsort(-s, kind="stable")
+        R = np.empty(T, int); R[order] = np.arange(T)
+        ranks.append(R)
+        sh = orc.score(l, 0, r)
+        win = ranks[max(0, l - 4): l + 1]
+        for i in range(T):
+            vals = [Fraction(int(w[i]), T - 1) for w in win]
+            var = statistics.pvariance(vals)                       # exact rational variance
+            sigma = math.sqrt(var)
+            cons = max(0.0, 1.0 - sigma * math.sqrt(12.0))
+            want = float(s[i]) * (1.0 + 0.5 * cons)
+            # the oracle evaluates sigma from the exact integer D in its own order;
+            # agree to fp32 rounding of nearly equal fp64 values
+            assert abs(sh[i] - want) <= 2 ** -22 * abs(want), (l, i, sh[i], want)
+
+
+def test_ties_break_to_lower_slot_and_window_and_reset():
+    T = 6
+    orc = _orc(T)
+    # all equal norms: ranks are the slot order at every layer -> Cons = 1
+    r = np.ones((T, 8))
+    for l in range(3):
+        sh = orc.score(l, 0, r)
+    assert np.all(sh == to_f32(to_f32(np.sqrt(8.0)) * 1.5))
+    # window: two wild layers, then five constant layers -> only the last five count
+    orc = _orc(T)
+    rng = np.random.default_rng(5)
+    orc.score(0, 1, _residual_with_norms(rng.permutation(T) + 1.0))
+    orc.score(1, 1, _residual_with_norms(rng.permutation(T) + 1.0))
+    base = np.arange(T, dtype=float) + 1.0
+    for l in range(2, 7):
+        sh = orc.score(l, 1, _residual_with_norms(base))
+    np.testing.assert_array_equal(sh, to_f32(to_f32(base) * 1.5))
+    # history resets at a new frame: layer 0 of frame 2 alone -> n = 1 -> Cons = 1
+    sh = orc.score(0, 2, _residual_with_norms(rng.permutation(T) + 1.0))
+    s = sh / 1.5
+    assert np.all(np.abs(sh - to_f32(s * 1.5)) == 0)
+
+
+def test_raw_score_is_fp32_of_exact_norm():
+    rng = np.random.default_rng(2)
+    r = (rng.standard_normal((300, 1024)) * np.exp(rng.standard_normal(300))[:, None]).astype(np.float32)
+    orc = _orc(300, lam=0.0)
+    sh = orc.score(0, 0, r.astype(np.float64))
+    exact = np.array([math.sqrt(math.fsum(float(v) * float(v) for v in row)) for row in r])
+    np.testing.assert_array_equal(sh, to_f32(exact))

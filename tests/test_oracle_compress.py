@@ -1,0 +1,137 @@
+"""Pins for the oracle's keep / merge / drop compression: properties that any correct
+implementation has, each checked with a routine other than the oracle's own."""
+import math
+
+import numpy as np
+import pytest
+import torch
+from scipy.spatial.distance import cdist
+
+from kvc_streams import WORKLOADS, FrameStream
+from oracle import OracleConfig, StreamOracle, bf16_round
+
+
+def _small_wl(**kw):
+    base = dict(tokens_per_frame=8, num_special_tokens=1, num_heads=2, head_dim=4, page_size=4,
+                budget_tokens=40, num_layers=2, residual_dim=16)
+    base.update(kw)
+    return WORKLOADS["vggt_budget_16k"].replace(**base)
+
+
+def _np(x):
+    return x.to(torch.float64).numpy()
+
+
+def _drive(wl, frames, seed=0, on_event=None):
+    st = FrameStream(wl, seed=seed)
+    orc = StreamOracle(OracleConfig.from_workload(wl))
+    events = 0
+    for t in range(frames):
+        for l in range(wl.num_layers):
+            q, k, v = (_np(x) for x in st.frame(l, t))
+            orc.append(l, t, k, v, True)
+            orc.attend(l, q)
+            before_k, before_v, before_ids = orc.gather(l)
+            ids_b, cnt_b, sh_b = orc.token_meta(l)
+            orc.score(l, t, _np(st.residual(l, t)))
+            ids_b, cnt_b, sh_b = orc.token_meta(l)
+            res = orc.compress(l)
+            if res is not None:
+                events += 1
+                if on_event:
+                    on_event(orc, l, res, before_k, before_v, ids_b, cnt_b, sh_b)
+    return orc, events
+
+
+def test_compression_properties():
+    wl = _small_wl()
+    n_keep = math.floor(float(np.float32(wl.keep_frac)) * wl.budget_tokens)
+    n_merge = wl.budget_tokens - n_keep
+    seen = []
+
+    def check(orc, l, res, Kb, Vb, ids_b, cnt_b, sh_b):
+        seen.append(1)
+        N = ids_b.size
+        H, D = wl.num_heads, wl.head_dim
+        kept = res["kept_ids"]
+        src, dst = res["merge_src"], res["merge_dst"]
+        drop = res["dropped_ids"]
+        # tiers partition the cache; sizes as stated
+        assert len(kept) == n_keep and np.all(np.diff(kept) > 0)
+        if res["n_protected"] < n_keep:
+            assert len(src) == min(n_merge, N - n_keep)
+        else:
+            assert len(src) == 0          # no eligible target: the merge tier is dropped
+        allids = np.sort(np.concatenate([kept, src, drop]))
+        assert np.array_equal(allids, np.sort(ids_b))
+        pos = {int(i): p for p, i in enumerate(ids_b)}
+        T = wl.tokens_per_frame
+        prot = {int(i) for i in ids_b if (i // T == 0) or (i % T) < wl.num_special_tokens}
+        assert prot <= set(kept.tolist())
+        # order by s_hat: kept (non-protected) >= merged >= dropped, ties to lower id
+        key = lambda i: (-sh_b[pos[int(i)]], int(i))
+        kept_np = [i for i in kept if int(i) not in prot]
+        if kept_np and len(src):
+            assert max(key(i) for i in kept_np) < min(key(i) for i in src)
+        if len(src) and len(drop):
+            assert max(key(i) for i in src) < min(key(i) for i in drop)
+        # targets: kept, not protected, maximal cosine (scipy), lowest id among ties
+        Kf = Kb.reshape(N, H * D)
+        elig = sorted(int(i) for i in kept_np)
+        E = Kf[[pos[i] for i in elig]]
+        for s_id, d_id in zip(src, dst):
+            assert int(d_id) in elig
+            dist = cdist(Kf[[pos[int(s_id)]]], E, metric="cosine")[0]
+            assert abs(dist[elig.index(int(d_id))] - dist.min()) <= 1e-12
+        # counts conserved: after = keep + merged before
+        Ka, Va, ids_a = orc.gather(l)
+        ida, cnta, sha = orc.token_meta(l)
+        assert np.array_equal(ida, kept)
+        keep_merge = set(kept.tolist()) | set(src.tolist())
+        assert cnta.sum() == sum(int(cnt_b[pos[i]]) for i in keep_merge)
+        # protected tokens unchanged bit for bit; untargeted kept tokens unchanged
+        targets = set(dst.tolist())
+        for p_after, i in enumerate(ida):
+            if int(i) not in targets:
+                assert np.array_equal(Ka[p_after], Kb[pos[int(i)]])
+                assert np.array_equal(Va[p_after], Vb[pos[int(i)]])
+        # merged values = count-weighted mean (numpy average), rounded to bf16
+        for j in targets:
+            srcs = [int(s) for s, d in zip(src, dst) if int(d) == j]
+            members = [j] + srcs
+            w = np.array([cnt_b[pos[m]] for m in members], float)
+            for before, after in ((Kb, Ka), (Vb, Va)):
+                stack = np.stack([before[pos[m]].reshape(-1) for m in members])
+                mean = np.average(stack, axis=0, weights=w)
+                got = after[list(ida).index(j)].reshape(-1)
+                ulp = np.abs(bf16_round(mean) - bf16_round(mean * (1 + 2 ** -8)))
+                assert np.all(np.abs(got - bf16_round(mean)) <= ulp + 1e-300)
+        # compaction packs P per page in ascending id, into the lowest free pages
+        pt = orc.page_table(l)
+        assert np.all(pt[:, 0] == -1)
+        assert pt[:, 3].sum() == n_keep and np.all(pt[:-1, 3] == wl.page_size)
+
+    orc, events = _drive(wl, 9, on_event=check)
+    assert events >= 4 and len(seen) == events
+
+
+def test_full_protected_keep_tier_drops_merge_tier():
+    wl = _small_wl(budget_tokens=20)      # floor(0.6*20) = 12 = 8 (frame 0) + 4 specials by frame 4
+    got = []
+    _drive(wl, 5, on_event=lambda orc, l, res, *a: got.append(res))
+    assert got and got[-1]["n_protected"] == 12 and got[-1]["merge_src"].size == 0
+
+
+def test_protected_overflow_raises():
+    wl = _small_wl(budget_tokens=12, tokens_per_frame=8, num_special_tokens=4)
+    # frame 0 alone is 8 protected tokens > floor(0.6 * 12) = 7
+    with pytest.raises(OverflowError):
+        _drive(wl, 3)
+
+
+def test_no_compression_below_budget():
+    wl = _small_wl(budget_tokens=1000)
+    orc, events = _drive(wl, 5)
+    assert events == 0
+    ids, cnt, sh = orc.token_meta(0)
+    assert ids.size == 5 * wl.tokens_per_frame and np.all(cnt == 1)
