@@ -1,0 +1,245 @@
+/*
+ * kvc.h -- C ABI of libkvc, a B200 (sm_100a) paged KV cache for streaming
+ * visual-geometry transformers: per-frame, frame-causal attention of a new
+ * frame's tokens over a bounded paged cache, plus the cache maintenance around
+ * it (page-aligned append, sliding-window eviction with pinned scale frames,
+ * keyframe skip-append, FP8 quantisation, importance-scored compression).
+ *
+ * Sources, cited by page title and section:
+ *   [GCT]  "How GCTStream Implements Streaming 3D Reconstruction with KV Cache"
+ *   [LBM]  "Can LingBot-Map Achieve 20 FPS Streaming 3D Reconstruction?"
+ *   [SCV]  StreamCacheVGGT (cross-layer consistency scoring + hybrid compression)
+ *   [IVG]  "InfiniteVGGT: Visual Geometry Grounded Transformer for Endless Streams"
+ *   [XSV]  "XStreamVGGT: Extremely Memory-Efficient Streaming Vision Geometry
+ *          Grounded Transformer with KV Cache Compression" (abstract)
+ *
+ * Conventions for every call:
+ *   - Device pointers are caller-owned and must stay valid until the cache's
+ *     stream has executed the call. Host pointers are read or written before
+ *     the call returns.
+ *   - Q, K, V and O are token-major [T, H, D] tensors (T = tokens_per_frame,
+ *     H = num_heads, D = head_dim), densely packed, in the configured I/O dtype
+ *     (fp32 or bf16). D*element_size must be a multiple of 16 bytes and device
+ *     pointers 16-byte aligned.
+ *   - The library allocates all device memory (page pools, page tables,
+ *     scratch) in kvc_create and nothing afterwards, so cache memory is
+ *     constant for the life of a stream ([GCT] Sliding Window Eviction: O(1)
+ *     memory).
+ *   - Calls enqueue work on the cache's stream and return without waiting for
+ *     the GPU, except kvc_page_table, kvc_token_meta, kvc_last_merge,
+ *     kvc_export_pages, kvc_step_host and kvc_synchronize, which synchronise.
+ *   - Errors are status codes; kvc_last_error() gives a message. A status other
+ *     than KVC_OK leaves the cache state unchanged unless stated otherwise.
+ *     A device-side failure (a bounded wait that gave up, an exhausted page
+ *     pool) is latched in a device error word and reported by the next
+ *     synchronising call as KVC_ERR_TIMEOUT or KVC_ERR_DEVICE; the CUDA
+ *     context stays usable.
+ *   - A kvc_cache is not thread-safe; use one per thread or serialise.
+ */
+#ifndef KVC_H_
+#define KVC_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KVC_VERSION 1
+
+/* Every entry point is exported with default visibility; internals stay hidden. */
+#if defined(__GNUC__)
+#define KVC_API __attribute__((visibility("default")))
+#else
+#define KVC_API
+#endif
+
+typedef enum {
+  KVC_OK = 0,
+  KVC_ERR_ARG = 1,          /* invalid argument or unsupported shape */
+  KVC_ERR_OOM = 2,          /* device allocation failed in kvc_create */
+  KVC_ERR_CUDA = 3,         /* a CUDA runtime call failed */
+  KVC_ERR_STATE = 4,        /* call out of order (e.g. attend with nothing pending) */
+  KVC_ERR_BUDGET = 5,       /* protected tokens exceed the keep tier */
+  KVC_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up */
+  KVC_ERR_DEVICE = 7,       /* device-side consistency check failed */
+  KVC_ERR_UNSUPPORTED = 8   /* configuration valid but not implemented on this path */
+} kvc_status;
+
+typedef enum { KVC_F32 = 0, KVC_BF16 = 1, KVC_FP8_E4M3 = 2 } kvc_dtype;
+
+/* Cache configuration; all fields are read once by kvc_create.
+ *
+ * Eviction ([LBM] Sliding-Window Eviction Strategy; [GCT] Sliding Window
+ * Eviction): with window_frames = W > 0 the committed cache of each layer is
+ * the first scale_frames = S committed frames plus the last W committed frames.
+ *
+ * Compression ([SCV] sections 2.1-2.2): with budget_tokens = B > 0 (and
+ * window_frames <= 0) kvc_compress keeps floor(keep_frac * B) tokens, merges
+ * the next B - floor(keep_frac * B) into kept tokens and drops the rest
+ * whenever a layer holds more than B committed tokens.
+ */
+typedef struct {
+  int32_t num_layers;           /* independent per-layer caches */
+  int32_t num_heads;            /* H */
+  int32_t head_dim;             /* D */
+  int32_t tokens_per_frame;     /* T (e.g. 1004 = 37*27 patches + 1 camera + 4 register) */
+  int32_t num_special_tokens;   /* leading camera/register tokens of each frame (protected) */
+  int32_t page_size;            /* P tokens per page; each frame starts on a fresh page */
+  int32_t window_frames;        /* W; <= 0: no sliding window */
+  int32_t scale_frames;         /* S pinned first frames */
+  int32_t io_dtype;             /* kvc_dtype of Q, K, V, O: KVC_F32 or KVC_BF16 */
+  int32_t kv_dtype;             /* storage: same as io_dtype, or KVC_FP8_E4M3 with bf16 I/O */
+  float softmax_scale;          /* logits = softmax_scale * q . k */
+  int32_t budget_tokens;        /* B; 0: no compression */
+  float keep_frac;              /* keep tier fraction (0.6) */
+  float lambda_;                /* consistency weight lambda (0.5) */
+  int32_t rank_window;          /* layers in the rank window (5) */
+  int32_t residual_dim;         /* R, columns of the residual given to kvc_compress */
+  int32_t protect_first_frame;  /* 1: every token of frame 0 is always kept */
+  int32_t max_frames;           /* cap on cached frames when W <= 0 and B == 0 */
+  int32_t kv_splits;            /* KV splits per query tile in attention; 0 = automatic */
+  int32_t reserved[7];          /* must be zero */
+} kvc_config;
+
+/* Cache statistics ([GCT] Cache Monitoring: occupancy, memory use, eviction status). */
+typedef struct {
+  int64_t tokens;               /* committed tokens in the layer */
+  int64_t pages_used;           /* pages held (committed + pending) */
+  int64_t pages_total;          /* pool pages of the layer */
+  int64_t pool_bytes;           /* device bytes of the layer's page pool */
+  int64_t high_water_pages;     /* max pages ever held at once by the layer */
+  int64_t frames_appended;      /* kvc_append_frame calls on the layer */
+  int64_t frames_committed;     /* keyframes committed */
+  int64_t frames_skipped;       /* non-keyframes released after attention */
+  int64_t frames_evicted;       /* frames removed by the sliding window */
+  int64_t compress_events;      /* compressions performed */
+  int64_t device_error;         /* latched device error word (0 = none) */
+  int64_t kernel_launches;      /* kernels this cache has launched (all layers) */
+} kvc_info;
+
+typedef struct kvc_cache kvc_cache;
+
+/* Create a cache on the current CUDA device. `stream` is a cudaStream_t (NULL:
+ * the legacy default stream) on which all later work is enqueued. Allocates the
+ * page pools sized for the configuration (window: (S + W + 1) frames of pages
+ * per layer; budget: 2*ceil(B/P) + (ceil(B/T) + 2) frames of pages), page
+ * tables and scratch, and zero-fills them. On success *out owns everything;
+ * release with kvc_destroy. Errors: KVC_ERR_ARG (bad config), KVC_ERR_OOM. */
+KVC_API kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out);
+
+/* Synchronise the stream and free everything the cache owns. NULL is a no-op. */
+KVC_API kvc_status kvc_destroy(kvc_cache* c);
+
+/* Change the stream used by later calls. */
+KVC_API kvc_status kvc_set_stream(kvc_cache* c, void* stream);
+
+/* Empty every layer (page tables, free lists, rank history, counters) between
+ * videos, keeping the pool memory ([GCT] Cache Initialization and Cleanup,
+ * clean_kv_cache). Stream-ordered. */
+KVC_API kvc_status kvc_reset(kvc_cache* c);
+
+/* Page-aligned append of frame `frame_idx` to `layer` ([LBM] Page-Aligned
+ * Tensor Layout; [GCT] AggregatorStream with Paged KV Cache). The device
+ * allocates ceil(T/P) lowest-free pages and writes k_dev, v_dev ([T, H, D],
+ * io dtype) into them as pool layout [page][head][slot][dim]; slots past T in
+ * the last page are zero. With kv_dtype FP8 each (page, head) block of K and V
+ * is quantised with its own absmax scale: scale = fp32(amax / 448), code =
+ * E4M3 round-to-nearest-even saturating of fp32(x / scale) ([XSV] abstract).
+ * The frame is *pending* until kvc_attend: `is_keyframe` = 0 makes attention
+ * release it afterwards ([GCT] Selective Frame Caching with Skip Append).
+ * Frame indices must increase per layer. Errors: KVC_ERR_STATE if a frame is
+ * already pending on the layer. */
+KVC_API kvc_status kvc_append_frame(kvc_cache* c, int32_t layer, int32_t frame_idx,
+                            const void* k_dev, const void* v_dev, int32_t is_keyframe);
+
+/* Frame attention of the pending frame's queries q_dev [T, H, D] over every
+ * token of `layer` (committed + pending), writing o_dev [T, H, D]:
+ * O[i,h] = sum_j softmax_j(softmax_scale * q_i . k_j) v_j, no mask
+ * ([GCT] Frame-by-Frame Causal Processing; [IVG] Causal Attention). Then the
+ * pending frame is committed (keyframe; frames outside the first S and last W
+ * committed are evicted and their pages freed) or released (non-keyframe).
+ * bf16 with D = 64 runs on tcgen05 tensor cores (fp32 accumulation); fp32 I/O
+ * runs fp32 FMA arithmetic. Errors: KVC_ERR_STATE if nothing is pending. */
+KVC_API kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_dev);
+
+/* Importance scoring and, when the committed cache of `layer` holds more than
+ * B tokens, keep/merge/drop compression ([SCV] 2.1.1-2.1.4, 2). Must follow
+ * kvc_attend of the same frame; within a frame layers are scored in ascending
+ * order (the rank history covers the last rank_window layers of this frame and
+ * is reset when a new frame starts). residual_dev [T, R] fp32 gives the raw
+ * score s_i = fp32(sqrt(sum_c r_ic^2)) (fp64 sum, ascending c). Scores:
+ * rank R (s descending, ties lower slot), sigma from the population variance
+ * of R/(T-1) over the window, Cons = max(0, 1 - sigma sqrt(12)),
+ * s_hat = fp32(s (1 + lambda Cons)) evaluated in fp64. Compression: protected
+ * tokens (frame 0 if protect_first_frame, and the first num_special_tokens of
+ * every frame) are kept; the others by s_hat descending (ties lower id) fill
+ * the keep tier; the next B - floor(keep_frac B) are each merged into the kept
+ * non-protected token of highest full-key cosine (ties lower id) as a
+ * count-weighted mean rounded once to bf16; the rest are dropped; kept tokens
+ * are rewritten in ascending id into the lowest free pages. *fired_out (host,
+ * may be NULL) receives 1 when a compression ran. bf16 caches only.
+ * Errors: KVC_ERR_ARG (B == 0 or NULL residual), KVC_ERR_STATE (order),
+ * KVC_ERR_BUDGET (protected tokens exceed the keep tier). */
+KVC_API kvc_status kvc_compress(kvc_cache* c, int32_t layer, const float* residual_dev, int32_t* fired_out);
+
+/* Synchronise and copy the page table of `layer` to host: rows of 4 int32
+ * (owner, page_in_owner, phys_page, valid_tokens) in cache order; owner is the
+ * frame index, or -1 for pages written by compaction. Writes at most
+ * `capacity` rows; *n_rows receives the full count. `info` (may be NULL)
+ * receives the layer's statistics. */
+KVC_API kvc_status kvc_page_table(kvc_cache* c, int32_t layer, int32_t* rows_host, int32_t capacity,
+                          int32_t* n_rows, kvc_info* info);
+
+/* Synchronise and copy per-token metadata of `layer` in cache order: token id
+ * (frame * T + slot), merge count, and enhanced score s_hat. Any output pointer
+ * may be NULL. */
+KVC_API kvc_status kvc_token_meta(kvc_cache* c, int32_t layer, int64_t* ids_host, int32_t* counts_host,
+                          float* shat_host, int32_t capacity, int32_t* n_out);
+
+/* Synchronise and copy the (source id, target id) pairs of the last
+ * compression of `layer`, in ascending source id. */
+KVC_API kvc_status kvc_last_merge(kvc_cache* c, int32_t layer, int64_t* src_host, int64_t* dst_host,
+                          int32_t capacity, int32_t* n_out);
+
+/* Synchronise and copy the raw pool contents of page-table rows
+ * [first_row, first_row + n_rows) of `layer`: K and V pages as stored
+ * ([H][P][D] per page, storage dtype; FP8: codes), and for FP8 the per-(page,
+ * head) scales [n_rows][H] fp32 (scale pointers may be NULL otherwise). */
+KVC_API kvc_status kvc_export_pages(kvc_cache* c, int32_t layer, int32_t first_row, int32_t n_rows,
+                            void* k_host, void* v_host, float* k_scale_host, float* v_scale_host);
+
+/* One whole frame step of `layer` from HOST buffers: copy q, k, v [T, H, D]
+ * host -> device, append, attend (+ commit/evict), copy O device -> host,
+ * and wait for the copy. Pinned host memory gives full copy bandwidth. */
+KVC_API kvc_status kvc_step_host(kvc_cache* c, int32_t layer, int32_t frame_idx, int32_t is_keyframe,
+                         const void* q_host, const void* k_host, const void* v_host, void* o_host);
+
+/* Wait for all work of the cache and report any latched device error. */
+KVC_API kvc_status kvc_synchronize(kvc_cache* c);
+
+/* Message for the last failing call on `c` (never NULL). */
+KVC_API const char* kvc_last_error(const kvc_cache* c);
+
+/* Name of a status code. */
+KVC_API const char* kvc_status_string(kvc_status s);
+
+/* KVC_VERSION of the built library. */
+KVC_API int32_t kvc_version(void);
+
+/* Test hooks for failure handling, tested without any GPU fault:
+ *   kvc_debug_fail_allocs(n): the n-th next device allocation inside
+ *     kvc_create reports failure (n = 0 disables), which must surface as
+ *     KVC_ERR_OOM with nothing leaked.
+ *   kvc_debug_bounded_wait(c, timeout_us): launches one kernel that waits on a
+ *     device flag nobody sets, with the given bound; the wait gives up, the
+ *     kernel records KVC_ERR_TIMEOUT in the device error word and returns,
+ *     which kvc_synchronize then reports. */
+KVC_API kvc_status kvc_debug_fail_allocs(int32_t n);
+KVC_API kvc_status kvc_debug_bounded_wait(kvc_cache* c, int32_t timeout_us);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVC_H_ */

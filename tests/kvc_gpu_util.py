@@ -1,0 +1,109 @@
+"""Helpers shared by the GPU parity tests: drive the CUDA library and the oracle over
+the same seeded stream and compare them."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from kvc_streams import FrameStream, keyframe_schedule
+from oracle import OracleConfig, StreamOracle
+
+BF16_MAX_ABS = 2e-2
+BF16_MEAN_ABS = 2e-3
+F32_MAX_ABS = 1e-4
+
+
+def np64(x: torch.Tensor) -> np.ndarray:
+    return x.detach().to(torch.float64).cpu().numpy()
+
+
+def sample_rows(T: int, n: int = 64, seed: int = 0) -> np.ndarray:
+    """Seeded query rows, always including rows 0-4 and the last row."""
+    rng = np.random.default_rng(seed)
+    fixed = [r for r in (0, 1, 2, 3, 4, T - 1) if r < T]
+    rest = [r for r in rng.permutation(T).tolist() if r not in fixed][: max(0, n - len(fixed))]
+    return np.array(sorted(set(fixed + rest)))
+
+
+def compare_out(got: np.ndarray, ref: np.ndarray, io_dtype: str, what: str = ""):
+    err = np.abs(got - ref)
+    if io_dtype == "f32":
+        assert err.max() <= F32_MAX_ABS, f"{what}: max abs {err.max():.3e} > {F32_MAX_ABS}"
+    else:
+        assert err.max() <= BF16_MAX_ABS, f"{what}: max abs {err.max():.3e} > {BF16_MAX_ABS}"
+        assert err.mean() <= BF16_MEAN_ABS, f"{what}: mean abs {err.mean():.3e} > {BF16_MEAN_ABS}"
+    return float(err.max()), float(err.mean())
+
+
+def run_parity(kvc, wl, frames, *, check_frames=None, rows=None, seed=0, layers=None, kv_splits=0,
+               check_pages=False, record=None):
+    """Stream `frames` frames through the library and the oracle; compare page tables at
+    every step and outputs on `check_frames` (all if None) for `rows` (all if None)."""
+    dev = torch.device("cuda")
+    cfg = kvc.config_from_workload(wl, kv_splits=kv_splits)
+    h = kvc.kvc_create(cfg)
+    try:
+        st = FrameStream(wl, seed=seed, device=dev)
+        orc = StreamOracle(OracleConfig.from_workload(wl))
+        layers = range(wl.num_layers) if layers is None else layers
+        T, H, D = wl.tokens_per_frame, wl.num_heads, wl.head_dim
+        out = torch.empty((T, H, D), dtype=q_dtype(wl), device=dev)
+        stats = []
+        for t in range(frames):
+            key = keyframe_schedule(t, wl.scale_frames, wl.keyframe_interval)
+            for l in layers:
+                q, k, v = st.frame(l, t)
+                kvc.kvc_append_frame(h, l, t, k, v, key)
+                kvc.kvc_attend(h, l, q, out)
+                orc.append(l, t, np64(k), np64(v), key)
+                do_check = check_frames is None or t in check_frames
+                if do_check:
+                    ref = orc.attend(l, np64(q), rows=rows)
+                else:
+                    orc.commit(l)
+                if do_check:
+                    torch.cuda.synchronize()
+                    got = np64(out)
+                    got = got if rows is None else got[rows]
+                    stats.append((t, l) + compare_out(got, ref, wl.io_dtype, f"frame {t} layer {l}"))
+                pt, info = kvc.kvc_page_table(h, l)
+                want = orc.page_table(l)
+                assert np.array_equal(pt, want), f"page table differs at frame {t} layer {l}"
+                assert info["device_error"] == 0
+                if check_pages and do_check:
+                    check_page_bytes(kvc, h, l, wl, orc)
+            if record is not None:
+                record(t, h, orc)
+        return stats
+    finally:
+        kvc.kvc_destroy(h)
+
+
+def q_dtype(wl):
+    return torch.float32 if wl.io_dtype == "f32" else torch.bfloat16
+
+
+def check_page_bytes(kvc, h, layer, wl, orc):
+    """Stored pages are bit-exact: bf16/f32 values equal the inputs (zeros in masked
+    slots); FP8 codes and scales equal the oracle's."""
+    pt = orc.page_table(layer)
+    n = len(pt)
+    H, P, D = wl.num_heads, wl.page_size, wl.head_dim
+    fp8 = wl.kv_dtype == "fp8_e4m3"
+    elem = 1 if fp8 else (4 if wl.kv_dtype == "f32" else 2)
+    kb, vb, ks, vs = kvc.kvc_export_pages(h, layer, 0, n, H * P * D * elem, H, fp8)
+    if fp8:
+        kc, vc, kso, vso = orc.fp8_pages(layer)
+        assert np.array_equal(kb.reshape(n, H, P, D), kc), "FP8 K codes differ"
+        assert np.array_equal(vb.reshape(n, H, P, D), vc), "FP8 V codes differ"
+        assert np.array_equal(ks.astype(np.float64), kso), "FP8 K scales differ"
+        assert np.array_equal(vs.astype(np.float64), vso), "FP8 V scales differ"
+    else:
+        dt = torch.float32 if elem == 4 else torch.bfloat16
+        L = orc.layers[layer]
+        for i, (pid, owner, g, nv) in enumerate(L.entries):
+            pg = L.pages[pid]
+            kk = torch.from_numpy(kb[i].copy()).view(dt).view(H, P, D).to(torch.float64).numpy()
+            vv = torch.from_numpy(vb[i].copy()).view(dt).view(H, P, D).to(torch.float64).numpy()
+            assert np.array_equal(kk[:, :nv], pg.k[:, :nv]) and np.array_equal(vv[:, :nv], pg.v[:, :nv])
+            assert not kk[:, nv:].any() and not vv[:, nv:].any(), "masked slots must be zero"

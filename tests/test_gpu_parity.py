@@ -1,0 +1,213 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the same
+seeded inputs. Page tables and stored pages are compared bit for bit; attention outputs
+within max-abs 2e-2 / mean-abs 2e-3 (bf16) or 1e-4 (fp32)."""
+import numpy as np
+import pytest
+import torch
+
+from kvc_gpu_util import run_parity, sample_rows, compare_out, np64
+from kvc_streams import WORKLOADS, FrameStream, keyframe_schedule
+from oracle import OracleConfig, StreamOracle
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kvc():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    import transformer_kv_cache_b200 as m
+    return m
+
+
+def test_tiny_f32_full_stream(kvc):
+    wl = WORKLOADS["tiny_f32"]
+    stats = run_parity(kvc, wl, wl.num_frames, check_pages=True)
+    assert len(stats) == wl.num_frames
+
+
+@pytest.mark.parametrize("T,H,W,S,frames,splits", [
+    (300, 4, 6, 2, 12, 0),      # 3 q tiles with a ragged 44-row tail, eviction active
+    (300, 4, 6, 2, 12, 1),      # no KV split
+    (300, 4, 6, 2, 12, 5),      # forced split count
+    (37, 2, 3, 1, 8, 0),        # one ragged q tile, 3 pages/frame, last page 5 valid
+    (5, 2, 2, 0, 6, 0),         # T < P: every page partial
+    (256, 2, 2, 1, 6, 3),       # T a multiple of the page size and of the q tile
+])
+def test_bf16_tensor_core_small(kvc, T, H, W, S, frames, splits):
+    wl = WORKLOADS["vggt_518x378"].replace(tokens_per_frame=T, num_heads=H, window_frames=W, scale_frames=S,
+                                            num_special_tokens=min(5, T))
+    run_parity(kvc, wl, frames, kv_splits=splits, check_pages=True)
+
+
+def test_bf16_keyframes_two_layers(kvc):
+    wl = WORKLOADS["vggt_24layer_k4"].replace(num_layers=2, tokens_per_frame=200, num_heads=4,
+                                               window_frames=4, scale_frames=2)
+    run_parity(kvc, wl, 16, check_pages=True)
+
+
+def test_fp8_small_codes_and_outputs(kvc):
+    wl = WORKLOADS["vggt_518x518_fp8"].replace(tokens_per_frame=150, num_heads=4, window_frames=4, scale_frames=2)
+    run_parity(kvc, wl, 9, check_pages=True)
+
+
+def test_vggt_full_size_steady_state_sampled(kvc):
+    """The 518x378 workload at full size past the window (eviction running), sampled rows."""
+    wl = WORKLOADS["vggt_518x378"]
+    rows = sample_rows(wl.tokens_per_frame, 64, seed=1)
+    frames = wl.scale_frames + wl.window_frames + 4
+    check = {0, 1, wl.scale_frames, wl.scale_frames + wl.window_frames - 1, wl.scale_frames + wl.window_frames,
+             frames - 1}
+    stats = run_parity(kvc, wl, frames, check_frames=check, rows=rows)
+    assert len(stats) == len(check)
+
+
+def test_split_counts_agree(kvc):
+    """Different KV split counts give the same answer within fp32 reassociation."""
+    wl = WORKLOADS["vggt_518x378"].replace(tokens_per_frame=500, num_heads=2, window_frames=10, scale_frames=2)
+    dev = torch.device("cuda")
+    outs = []
+    for splits in (1, 2, 7):
+        h = kvc.kvc_create(kvc.config_from_workload(wl, kv_splits=splits))
+        st = FrameStream(wl, seed=3, device=dev)
+        o = torch.empty((wl.tokens_per_frame, wl.num_heads, wl.head_dim), dtype=torch.bfloat16, device=dev)
+        for t in range(12):
+            q, k, v = st.frame(0, t)
+            kvc.kvc_append_frame(h, 0, t, k, v, True)
+            kvc.kvc_attend(h, 0, q, o)
+        torch.cuda.synchronize()
+        outs.append(np64(o))
+        kvc.kvc_destroy(h)
+    for o in outs[1:]:
+        assert np.abs(o - outs[0]).max() <= 2 * 2 ** -8
+
+
+def test_reset_replays_bit_exact(kvc):
+    wl = WORKLOADS["vggt_518x378"].replace(tokens_per_frame=300, num_heads=2, window_frames=4, scale_frames=1)
+    dev = torch.device("cuda")
+    h = kvc.kvc_create(kvc.config_from_workload(wl))
+    res = []
+    for rep in range(2):
+        st = FrameStream(wl, seed=4, device=dev)
+        o = torch.empty((300, 2, 64), dtype=torch.bfloat16, device=dev)
+        outs = []
+        for t in range(8):
+            q, k, v = st.frame(0, t)
+            kvc.kvc_append_frame(h, 0, t, k, v, True)
+            kvc.kvc_attend(h, 0, q, o)
+            outs.append(o.clone())
+        torch.cuda.synchronize()
+        res.append(outs)
+        pt, info = kvc.kvc_page_table(h, 0)
+        kvc.kvc_reset(h)
+        pt2, info2 = kvc.kvc_page_table(h, 0)
+        assert len(pt2) == 0 and info2["tokens"] == 0
+    for a, b in zip(*res):
+        assert torch.equal(a, b)
+    kvc.kvc_destroy(h)
+
+
+def test_host_buffer_step_matches_device_path(kvc):
+    wl = WORKLOADS["vggt_518x378"].replace(tokens_per_frame=300, num_heads=4, window_frames=4, scale_frames=1)
+    dev = torch.device("cuda")
+    h1 = kvc.kvc_create(kvc.config_from_workload(wl))
+    h2 = kvc.kvc_create(kvc.config_from_workload(wl))
+    st = FrameStream(wl, seed=5, device=dev)
+    o = torch.empty((300, 4, 64), dtype=torch.bfloat16, device=dev)
+    oh = torch.empty((300, 4, 64), dtype=torch.bfloat16).pin_memory()
+    for t in range(7):
+        q, k, v = st.frame(0, t)
+        kvc.kvc_append_frame(h1, 0, t, k, v, True)
+        kvc.kvc_attend(h1, 0, q, o)
+        qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+        kvc.kvc_step_host(h2, 0, t, True, qh, kh, vh, oh)
+        torch.cuda.synchronize()
+        assert torch.equal(o.cpu(), oh)
+    kvc.kvc_destroy(h1)
+    kvc.kvc_destroy(h2)
+
+
+def test_memory_constant_over_long_stream(kvc):
+    wl = WORKLOADS["vggt_518x378"].replace(tokens_per_frame=200, num_heads=2, window_frames=3, scale_frames=1)
+    dev = torch.device("cuda")
+    h = kvc.kvc_create(kvc.config_from_workload(wl))
+    st = FrameStream(wl, seed=6, device=dev)
+    o = torch.empty((200, 2, 64), dtype=torch.bfloat16, device=dev)
+    free0 = None
+    ppf = -(-200 // 16)
+    for t in range(60):
+        q, k, v = st.frame(0, t)
+        kvc.kvc_append_frame(h, 0, t, k, v, True)
+        kvc.kvc_attend(h, 0, q, o)
+        if t == 10:
+            torch.cuda.synchronize()
+            free0 = torch.cuda.mem_get_info()[0]
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    pt, info = kvc.kvc_page_table(h, 0)
+    assert info["high_water_pages"] == (1 + 3 + 1) * ppf
+    assert info["frames_evicted"] == 60 - 4
+    kvc.kvc_destroy(h)
+
+
+def test_error_states(kvc):
+    wl = WORKLOADS["vggt_518x378"].replace(tokens_per_frame=64, num_heads=2, window_frames=2, scale_frames=0)
+    h = kvc.kvc_create(kvc.config_from_workload(wl))
+    dev = torch.device("cuda")
+    x = torch.zeros((64, 2, 64), dtype=torch.bfloat16, device=dev)
+    with pytest.raises(kvc.KVCError) as e:
+        kvc.kvc_attend(h, 0, x, x)
+    assert e.value.status_name == "KVC_ERR_STATE"
+    kvc.kvc_append_frame(h, 0, 0, x, x, True)
+    with pytest.raises(kvc.KVCError) as e:
+        kvc.kvc_append_frame(h, 0, 1, x, x, True)
+    assert e.value.status_name == "KVC_ERR_STATE"
+    with pytest.raises(kvc.KVCError) as e:
+        kvc.kvc_attend(h, 5, x, x)
+    assert e.value.status_name == "KVC_ERR_ARG"
+    kvc.kvc_attend(h, 0, x, x)
+    with pytest.raises(kvc.KVCError) as e:
+        kvc.kvc_append_frame(h, 0, 0, x, x, True)       # frame index must increase
+    assert e.value.status_name == "KVC_ERR_STATE"
+    with pytest.raises(kvc.KVCError) as e:
+        kvc.kvc_compress(h, 0, x)                        # no budget configured
+    assert e.value.status_name == "KVC_ERR_ARG"
+    kvc.kvc_destroy(h)
+    bad = kvc.config_from_workload(wl)
+    bad.head_dim = 48
+    with pytest.raises(kvc.KVCError):
+        kvc.kvc_create(bad)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(kvc):
+    wl = WORKLOADS["vggt_518x378"].replace(tokens_per_frame=64, num_heads=2, window_frames=2, scale_frames=0)
+    h = kvc.kvc_create(kvc.config_from_workload(wl))
+    kvc.kvc_debug_bounded_wait(h, 20000)      # 20 ms on a flag nobody sets
+    with pytest.raises(kvc.KVCError) as e:
+        kvc.kvc_synchronize(h)
+    assert e.value.status_name == "KVC_ERR_TIMEOUT"
+    kvc.kvc_reset(h)
+    kvc.kvc_synchronize(h)
+    x = torch.randn((64, 2, 64), device="cuda").to(torch.bfloat16)
+    o = torch.empty_like(x)
+    kvc.kvc_append_frame(h, 0, 0, x, x, True)
+    kvc.kvc_attend(h, 0, x, o)
+    kvc.kvc_synchronize(h)
+    assert torch.isfinite(o.float()).all()
+    kvc.kvc_destroy(h)
+
+
+def test_allocation_failure_is_reported_without_leak(kvc):
+    wl = WORKLOADS["vggt_518x378"].replace(tokens_per_frame=300, num_heads=4, window_frames=4, scale_frames=1)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for n in (1, 2, 4, 6):
+        kvc.kvc_debug_fail_allocs(n)
+        with pytest.raises(kvc.KVCError) as e:
+            kvc.kvc_create(kvc.config_from_workload(wl))
+        assert e.value.status_name == "KVC_ERR_OOM"
+    kvc.kvc_debug_fail_allocs(0)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    h = kvc.kvc_create(kvc.config_from_workload(wl))
+    kvc.kvc_destroy(h)

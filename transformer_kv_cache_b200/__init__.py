@@ -1,0 +1,287 @@
+"""Python binding of libkvc: the paged KV cache hot path for streaming visual-geometry
+transformers on B200 (sm_100a).
+
+Argument marshalling only: every function here has the name of the C entry point it
+calls (include/kvc.h) and converts torch tensors to device pointers and statuses to
+exceptions. All computation happens in the CUDA library; importing this package fails
+loudly when the built library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvc.so")
+
+KVC_F32, KVC_BF16, KVC_FP8_E4M3 = 0, 1, 2
+DTYPES = {"f32": KVC_F32, "bf16": KVC_BF16, "fp8_e4m3": KVC_FP8_E4M3}
+STATUS = ["KVC_OK", "KVC_ERR_ARG", "KVC_ERR_OOM", "KVC_ERR_CUDA", "KVC_ERR_STATE", "KVC_ERR_BUDGET",
+          "KVC_ERR_TIMEOUT", "KVC_ERR_DEVICE", "KVC_ERR_UNSUPPORTED"]
+
+# every symbol include/kvc.h declares
+EXPORTS = ["kvc_create", "kvc_destroy", "kvc_set_stream", "kvc_reset", "kvc_append_frame", "kvc_attend",
+           "kvc_compress", "kvc_page_table", "kvc_token_meta", "kvc_last_merge", "kvc_export_pages",
+           "kvc_step_host", "kvc_synchronize", "kvc_last_error", "kvc_status_string", "kvc_version",
+           "kvc_debug_fail_allocs", "kvc_debug_bounded_wait"]
+
+
+class kvc_config(ctypes.Structure):
+    _fields_ = [("num_layers", ctypes.c_int32), ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("tokens_per_frame", ctypes.c_int32), ("num_special_tokens", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("window_frames", ctypes.c_int32), ("scale_frames", ctypes.c_int32),
+                ("io_dtype", ctypes.c_int32), ("kv_dtype", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+                ("budget_tokens", ctypes.c_int32), ("keep_frac", ctypes.c_float), ("lambda_", ctypes.c_float),
+                ("rank_window", ctypes.c_int32), ("residual_dim", ctypes.c_int32),
+                ("protect_first_frame", ctypes.c_int32), ("max_frames", ctypes.c_int32),
+                ("kv_splits", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
+
+
+class kvc_info(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "tokens", "pages_used", "pages_total", "pool_bytes", "high_water_pages", "frames_appended",
+        "frames_committed", "frames_skipped", "frames_evicted", "compress_events", "device_error",
+        "kernel_launches")]
+
+    def as_dict(self):
+        return {n: int(getattr(self, n)) for n, _ in self._fields_}
+
+
+class KVCError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        self.status_name = STATUS[status] if 0 <= status < len(STATUS) else str(status)
+        super().__init__(f"{self.status_name}: {message}")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libkvc.so is not built ({LIB_PATH}); run `python transformer_kv_cache_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64p, i32p, fp = ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(ctypes.c_int64), \
+        ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_float)
+    sig = {
+        "kvc_create": ([ctypes.POINTER(kvc_config), vp, ctypes.POINTER(vp)], i32),
+        "kvc_destroy": ([vp], i32),
+        "kvc_set_stream": ([vp, vp], i32),
+        "kvc_reset": ([vp], i32),
+        "kvc_append_frame": ([vp, i32, i32, vp, vp, i32], i32),
+        "kvc_attend": ([vp, i32, vp, vp], i32),
+        "kvc_compress": ([vp, i32, vp, i32p], i32),
+        "kvc_page_table": ([vp, i32, i32p, i32, i32p, ctypes.POINTER(kvc_info)], i32),
+        "kvc_token_meta": ([vp, i32, i64p, i32p, fp, i32, i32p], i32),
+        "kvc_last_merge": ([vp, i32, i64p, i64p, i32, i32p], i32),
+        "kvc_export_pages": ([vp, i32, i32, i32, vp, vp, fp, fp], i32),
+        "kvc_step_host": ([vp, i32, i32, i32, vp, vp, vp, vp], i32),
+        "kvc_synchronize": ([vp], i32),
+        "kvc_last_error": ([vp], ctypes.c_char_p),
+        "kvc_status_string": ([i32], ctypes.c_char_p),
+        "kvc_version": ([], i32),
+        "kvc_debug_fail_allocs": ([i32], i32),
+        "kvc_debug_bounded_wait": ([vp, i32], i32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def _ptr(x) -> Optional[int]:
+    """Device/host pointer of a torch tensor, numpy array, or an int."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if isinstance(x, np.ndarray):
+        return x.ctypes.data
+    return x.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(handle, st: int):
+    if st != 0:
+        msg = _lib.kvc_last_error(handle).decode() if handle else ""
+        raise KVCError(st, msg)
+
+
+def make_config(num_layers, num_heads, head_dim, tokens_per_frame, num_special_tokens, page_size,
+                window_frames, scale_frames, io_dtype="bf16", kv_dtype="bf16", softmax_scale=0.125,
+                budget_tokens=0, keep_frac=0.6, lam=0.5, rank_window=5, residual_dim=1024,
+                protect_first_frame=1, max_frames=0, kv_splits=0) -> kvc_config:
+    c = kvc_config()
+    c.num_layers, c.num_heads, c.head_dim = num_layers, num_heads, head_dim
+    c.tokens_per_frame, c.num_special_tokens, c.page_size = tokens_per_frame, num_special_tokens, page_size
+    c.window_frames, c.scale_frames = window_frames, scale_frames
+    c.io_dtype = DTYPES[io_dtype] if isinstance(io_dtype, str) else io_dtype
+    c.kv_dtype = DTYPES[kv_dtype] if isinstance(kv_dtype, str) else kv_dtype
+    c.softmax_scale = softmax_scale
+    c.budget_tokens, c.keep_frac, c.lambda_ = budget_tokens, keep_frac, lam
+    c.rank_window, c.residual_dim, c.protect_first_frame = rank_window, residual_dim, protect_first_frame
+    c.max_frames, c.kv_splits = max_frames, kv_splits
+    return c
+
+
+def config_from_workload(wl, **over) -> kvc_config:
+    d = dict(num_layers=wl.num_layers, num_heads=wl.num_heads, head_dim=wl.head_dim,
+             tokens_per_frame=wl.tokens_per_frame, num_special_tokens=wl.num_special_tokens,
+             page_size=wl.page_size, window_frames=wl.window_frames, scale_frames=wl.scale_frames,
+             io_dtype=wl.io_dtype, kv_dtype=wl.kv_dtype, softmax_scale=wl.softmax_scale,
+             budget_tokens=wl.budget_tokens, keep_frac=wl.keep_frac, lam=wl.lam, rank_window=wl.rank_window,
+             residual_dim=wl.residual_dim, protect_first_frame=wl.protect_first_frame)
+    d.update(over)
+    return make_config(**d)
+
+
+# ---------------------------------------------------------------- entry points (same names as the C ABI)
+
+def kvc_version() -> int:
+    return int(_lib.kvc_version())
+
+
+def kvc_create(cfg: kvc_config, stream=None) -> int:
+    h = ctypes.c_void_p()
+    st = _lib.kvc_create(ctypes.byref(cfg), _stream(stream), ctypes.byref(h))
+    if st != 0:
+        raise KVCError(st, "kvc_create failed")
+    return h.value
+
+
+def kvc_destroy(handle) -> None:
+    _check(handle, _lib.kvc_destroy(handle))
+
+
+def kvc_set_stream(handle, stream) -> None:
+    _check(handle, _lib.kvc_set_stream(handle, _stream(stream)))
+
+
+def kvc_reset(handle) -> None:
+    _check(handle, _lib.kvc_reset(handle))
+
+
+def kvc_append_frame(handle, layer: int, frame_idx: int, k, v, is_keyframe: bool = True) -> None:
+    _check(handle, _lib.kvc_append_frame(handle, layer, frame_idx, _ptr(k), _ptr(v), int(bool(is_keyframe))))
+
+
+def kvc_attend(handle, layer: int, q, o) -> None:
+    _check(handle, _lib.kvc_attend(handle, layer, _ptr(q), _ptr(o)))
+
+
+def kvc_compress(handle, layer: int, residual) -> bool:
+    fired = ctypes.c_int32(0)
+    _check(handle, _lib.kvc_compress(handle, layer, _ptr(residual), ctypes.byref(fired)))
+    return bool(fired.value)
+
+
+def kvc_page_table(handle, layer: int):
+    """(rows int32 [n, 4] = owner, page_in_owner, phys_page, valid; info dict)"""
+    n = ctypes.c_int32(0)
+    info = kvc_info()
+    _check(handle, _lib.kvc_page_table(handle, layer, None, 0, ctypes.byref(n), ctypes.byref(info)))
+    rows = np.zeros((max(n.value, 1), 4), np.int32)
+    _check(handle, _lib.kvc_page_table(handle, layer, rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                       n.value, ctypes.byref(n), ctypes.byref(info)))
+    return rows[: n.value], info.as_dict()
+
+
+def kvc_token_meta(handle, layer: int, capacity: int = 1 << 22):
+    ids = np.zeros(capacity, np.int64)
+    cnt = np.zeros(capacity, np.int32)
+    sh = np.zeros(capacity, np.float32)
+    n = ctypes.c_int32(0)
+    _check(handle, _lib.kvc_token_meta(handle, layer, ids.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                       cnt.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                       sh.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), capacity,
+                                       ctypes.byref(n)))
+    k = n.value
+    return ids[:k], cnt[:k], sh[:k]
+
+
+def kvc_last_merge(handle, layer: int, capacity: int = 1 << 20):
+    src = np.zeros(capacity, np.int64)
+    dst = np.zeros(capacity, np.int64)
+    n = ctypes.c_int32(0)
+    _check(handle, _lib.kvc_last_merge(handle, layer, src.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                       dst.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), capacity,
+                                       ctypes.byref(n)))
+    return src[: n.value], dst[: n.value]
+
+
+def kvc_export_pages(handle, layer: int, first_row: int, n_rows: int, page_bytes: int, num_heads: int,
+                     fp8: bool = False):
+    """Raw page bytes of rows [first_row, first_row + n_rows): (k uint8 [n, page_bytes], v, k_scale, v_scale)."""
+    k = np.zeros((n_rows, page_bytes), np.uint8)
+    v = np.zeros((n_rows, page_bytes), np.uint8)
+    ks = np.zeros((n_rows, num_heads), np.float32) if fp8 else None
+    vs = np.zeros((n_rows, num_heads), np.float32) if fp8 else None
+    fptr = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_float)) if a is not None else None
+    _check(handle, _lib.kvc_export_pages(handle, layer, first_row, n_rows, k.ctypes.data, v.ctypes.data,
+                                         fptr(ks), fptr(vs)))
+    return k, v, ks, vs
+
+
+def kvc_step_host(handle, layer: int, frame_idx: int, is_keyframe: bool, q_host, k_host, v_host, o_host) -> None:
+    _check(handle, _lib.kvc_step_host(handle, layer, frame_idx, int(bool(is_keyframe)), _ptr(q_host),
+                                      _ptr(k_host), _ptr(v_host), _ptr(o_host)))
+
+
+def kvc_synchronize(handle) -> None:
+    _check(handle, _lib.kvc_synchronize(handle))
+
+
+def kvc_last_error(handle) -> str:
+    return _lib.kvc_last_error(handle).decode()
+
+
+def kvc_status_string(status: int) -> str:
+    return _lib.kvc_status_string(status).decode()
+
+
+def kvc_debug_fail_allocs(n: int) -> None:
+    _lib.kvc_debug_fail_allocs(n)
+
+
+def kvc_debug_bounded_wait(handle, timeout_us: int) -> None:
+    _check(handle, _lib.kvc_debug_bounded_wait(handle, timeout_us))
+
+
+@dataclass
+class KVCache:
+    """Owning wrapper: creates the cache and destroys it when closed."""
+    cfg: kvc_config
+    handle: int = 0
+
+    def __post_init__(self):
+        self.handle = kvc_create(self.cfg)
+
+    def close(self):
+        if self.handle:
+            kvc_destroy(self.handle)
+            self.handle = 0
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

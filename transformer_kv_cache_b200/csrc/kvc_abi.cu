@@ -1,0 +1,562 @@
+// kvc_abi.cu -- the extern "C" entry points of libkvc (declared in include/kvc.h).
+//
+// Host code here validates arguments, keeps the per-layer bookkeeping that decides *what*
+// happens (how many pages a frame takes, which frame the sliding window evicts, whether
+// compression fires) and enqueues the kernels that do it on the device: the page-table
+// manager picks the physical pages and moves entries, the append / attention kernels move
+// and combine the data. Nothing on this path computes on the CPU.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "kvc_internal.h"
+#include "sm100_ptx.cuh"
+
+using namespace kvc;
+
+namespace {
+
+int g_fail_allocs = 0;  // test hook: the n-th next allocation in kvc_create fails
+
+cudaError_t dev_alloc(void** p, size_t bytes) {
+  *p = nullptr;
+  if (g_fail_allocs > 0 && --g_fail_allocs == 0) return cudaErrorMemoryAllocation;
+  if (bytes == 0) bytes = 16;
+  return cudaMalloc(p, bytes);
+}
+
+template <typename T>
+cudaError_t dev_alloc_t(T** p, size_t bytes) {
+  void* v = nullptr;
+  cudaError_t e = dev_alloc(&v, bytes);
+  *p = static_cast<T*>(v);
+  return e;
+}
+
+void free_all(kvc_cache* c) {
+  void* ptrs[] = {c->k_pool,   c->v_pool,   c->k_scale,  c->v_scale, c->entries,  c->bitmap,
+                  c->d_err,    c->tok_id,   c->tok_cnt,  c->tok_shat, c->cmp_scratch, c->part_o,
+                  c->part_lse, c->stage_q,  c->stage_k,  c->stage_v, c->stage_o,  c->rank_hist};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+}
+
+kvc_status fail(kvc_cache* c, kvc_status s, const char* msg) {
+  if (c) c->last_error = msg;
+  return s;
+}
+
+kvc_status cuda_fail(kvc_cache* c, cudaError_t e, const char* where) {
+  if (c) {
+    c->last_error = std::string(where) + ": " + cudaGetErrorString(e);
+  }
+  return KVC_ERR_CUDA;
+}
+
+size_t dtype_bytes(int dt) { return dt == KVC_F32 ? 4 : (dt == KVC_BF16 ? 2 : 1); }
+
+Entry* layer_entries(kvc_cache* c, int layer) { return c->entries + static_cast<size_t>(layer) * c->pool_pages; }
+uint32_t* layer_bitmap(kvc_cache* c, int layer) {
+  return c->bitmap + static_cast<size_t>(layer) * c->bitmap_words;
+}
+uint8_t* layer_pool(kvc_cache* c, uint8_t* pool, int layer) {
+  return pool + static_cast<size_t>(layer) * c->pool_pages * c->page_bytes_kv;
+}
+float* layer_scale(kvc_cache* c, float* sc, int layer) {
+  return sc ? sc + static_cast<size_t>(layer) * c->pool_pages * c->cfg.num_heads : nullptr;
+}
+
+kvc_status check_device_error(kvc_cache* c) {
+  int err = 0;
+  cudaError_t e = cudaMemcpy(&err, c->d_err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(c, e, "reading the device error word");
+  if (err == DERR_TIMEOUT) return fail(c, KVC_ERR_TIMEOUT, "a bounded device-side wait gave up");
+  if (err != 0) return fail(c, KVC_ERR_DEVICE, "device-side consistency check failed (error word set)");
+  return KVC_OK;
+}
+
+kvc_status sync_and_check(kvc_cache* c) {
+  cudaError_t e = cudaStreamSynchronize(c->stream);
+  if (e != cudaSuccess) return cuda_fail(c, e, "cudaStreamSynchronize");
+  return check_device_error(c);
+}
+
+bool valid_layer(kvc_cache* c, int layer) { return layer >= 0 && layer < c->cfg.num_layers; }
+
+// Remove page-table entries [a, b) of a layer (frees their pages, closes the gap).
+kvc_status remove_entries(kvc_cache* c, int layer, int a, int b) {
+  LayerHost& L = c->L[layer];
+  cudaError_t e = launch_mgr_remove(c->stream, layer_entries(c, layer), layer_bitmap(c, layer), L.n_entries, a, b,
+                                    c->d_err);
+  if (e != cudaSuccess) return cuda_fail(c, e, "page-table remove");
+  c->launches++;
+  const int n = b - a;
+  L.n_entries -= n;
+  for (FrameRec& f : L.frames)
+    if (f.first_entry >= b) f.first_entry -= n;
+  return KVC_OK;
+}
+
+}  // namespace
+
+namespace kvc {
+// Budget-mode helpers live in kvc_compress.cu.
+kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_t* fired);
+kvc_status init_token_meta(kvc_cache* c, int layer, int first_entry, int n_pages, int frame);
+size_t compress_scratch_bytes(const kvc_config& cfg, int pool_pages);
+}  // namespace kvc
+
+extern "C" {
+
+int32_t kvc_version(void) { return KVC_VERSION; }
+
+const char* kvc_status_string(kvc_status s) {
+  switch (s) {
+    case KVC_OK: return "KVC_OK";
+    case KVC_ERR_ARG: return "KVC_ERR_ARG";
+    case KVC_ERR_OOM: return "KVC_ERR_OOM";
+    case KVC_ERR_CUDA: return "KVC_ERR_CUDA";
+    case KVC_ERR_STATE: return "KVC_ERR_STATE";
+    case KVC_ERR_BUDGET: return "KVC_ERR_BUDGET";
+    case KVC_ERR_TIMEOUT: return "KVC_ERR_TIMEOUT";
+    case KVC_ERR_DEVICE: return "KVC_ERR_DEVICE";
+    case KVC_ERR_UNSUPPORTED: return "KVC_ERR_UNSUPPORTED";
+  }
+  return "KVC_STATUS_UNKNOWN";
+}
+
+const char* kvc_last_error(const kvc_cache* c) { return c ? c->last_error.c_str() : "null cache"; }
+
+kvc_status kvc_debug_fail_allocs(int32_t n) {
+  g_fail_allocs = n < 0 ? 0 : n;
+  return KVC_OK;
+}
+
+kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
+  if (!cfg || !out) return KVC_ERR_ARG;
+  *out = nullptr;
+  const kvc_config& g = *cfg;
+  for (int i = 0; i < 7; ++i)
+    if (g.reserved[i] != 0) return KVC_ERR_ARG;
+  const bool dims_ok = g.num_layers >= 1 && g.num_heads >= 1 && g.tokens_per_frame >= 1 && g.page_size >= 1 &&
+                       g.num_special_tokens >= 0 && g.num_special_tokens <= g.tokens_per_frame &&
+                       g.scale_frames >= 0 && g.budget_tokens >= 0 &&
+                       (g.head_dim == 16 || g.head_dim == 32 || g.head_dim == 64 || g.head_dim == 128);
+  if (!dims_ok) return KVC_ERR_ARG;
+  if (g.io_dtype != KVC_F32 && g.io_dtype != KVC_BF16) return KVC_ERR_ARG;
+  if (!(g.kv_dtype == g.io_dtype || (g.kv_dtype == KVC_FP8_E4M3 && g.io_dtype == KVC_BF16))) return KVC_ERR_ARG;
+  if (g.kv_dtype == KVC_FP8_E4M3 && g.page_size * g.head_dim > 2048) return KVC_ERR_ARG;
+  if (!(g.softmax_scale > 0.f) || !std::isfinite(g.softmax_scale)) return KVC_ERR_ARG;
+  if (g.window_frames > 0 && g.budget_tokens > 0) return KVC_ERR_ARG;
+  if (g.budget_tokens > 0) {
+    if (g.kv_dtype != KVC_BF16 || !(g.keep_frac > 0.f && g.keep_frac <= 1.f) || g.rank_window < 1 ||
+        g.residual_dim < 1 || !(g.lambda_ >= 0.f) || g.budget_tokens > (1 << 24))
+      return KVC_ERR_ARG;
+  }
+  if (g.window_frames <= 0 && g.budget_tokens == 0 && g.max_frames < 1) return KVC_ERR_ARG;
+  if (g.kv_splits < 0) return KVC_ERR_ARG;
+
+  kvc_cache* c = new (std::nothrow) kvc_cache();
+  if (!c) return KVC_ERR_OOM;
+  c->cfg = g;
+  c->stream = static_cast<cudaStream_t>(stream);
+  cudaGetDevice(&c->device);
+  cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device);
+  const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads, D = g.head_dim;
+  c->ppf = (T + P - 1) / P;
+  if (g.window_frames > 0) {
+    c->pool_pages = (g.scale_frames + g.window_frames + 1) * c->ppf;
+  } else if (g.budget_tokens > 0) {
+    const int B = g.budget_tokens;
+    c->pool_pages = 2 * ((B + P - 1) / P) + ((B + T - 1) / T + 2) * c->ppf;
+  } else {
+    c->pool_pages = (g.max_frames + 1) * c->ppf;
+  }
+  c->bitmap_words = (c->pool_pages + 31) / 32;
+  c->elem_io = dtype_bytes(g.io_dtype);
+  c->elem_kv = dtype_bytes(g.kv_dtype);
+  if ((D * c->elem_io) % 16 != 0) {
+    delete c;
+    return KVC_ERR_ARG;
+  }
+  c->page_elems = static_cast<size_t>(H) * P * D;
+  c->page_bytes_kv = c->page_elems * c->elem_kv;
+  const size_t L = g.num_layers;
+  const size_t frame_bytes = static_cast<size_t>(T) * H * D * c->elem_io;
+  c->tc_path = g.io_dtype == KVC_BF16 && g.kv_dtype == KVC_BF16 && D == 64 && P == 16;
+  const int q_tiles = (T + 127) / 128;
+  c->part_rows = static_cast<size_t>(q_tiles) * H * 16;
+
+  cudaError_t e = cudaSuccess;
+  auto A = [&](cudaError_t r) {
+    if (e == cudaSuccess) e = r;
+  };
+  A(dev_alloc_t(&c->k_pool, L * c->pool_pages * c->page_bytes_kv));
+  A(dev_alloc_t(&c->v_pool, L * c->pool_pages * c->page_bytes_kv));
+  if (g.kv_dtype == KVC_FP8_E4M3) {
+    A(dev_alloc_t(&c->k_scale, L * c->pool_pages * H * sizeof(float)));
+    A(dev_alloc_t(&c->v_scale, L * c->pool_pages * H * sizeof(float)));
+  }
+  A(dev_alloc_t(&c->entries, L * c->pool_pages * sizeof(Entry)));
+  A(dev_alloc_t(&c->bitmap, L * c->bitmap_words * sizeof(uint32_t)));
+  A(dev_alloc_t(&c->d_err, 4 * sizeof(int)));
+  if (c->tc_path) {
+    A(dev_alloc_t(&c->part_o, c->part_rows * 128 * 64 * sizeof(float)));
+    A(dev_alloc_t(&c->part_lse, c->part_rows * 128 * sizeof(float)));
+  }
+  A(dev_alloc_t(&c->stage_q, frame_bytes));
+  A(dev_alloc_t(&c->stage_k, frame_bytes));
+  A(dev_alloc_t(&c->stage_v, frame_bytes));
+  A(dev_alloc_t(&c->stage_o, frame_bytes));
+  if (g.budget_tokens > 0) {
+    const size_t slots = L * c->pool_pages * P;
+    A(dev_alloc_t(&c->tok_id, slots * sizeof(int64_t)));
+    A(dev_alloc_t(&c->tok_cnt, slots * sizeof(int32_t)));
+    A(dev_alloc_t(&c->tok_shat, slots * sizeof(float)));
+    A(dev_alloc_t(&c->rank_hist, static_cast<size_t>(g.rank_window) * T * sizeof(int32_t)));
+    c->cmp_scratch_bytes = compress_scratch_bytes(g, c->pool_pages);
+    A(dev_alloc(&c->cmp_scratch, c->cmp_scratch_bytes));
+  }
+  if (e != cudaSuccess) {
+    free_all(c);
+    delete c;
+    cudaGetLastError();
+    return KVC_ERR_OOM;
+  }
+  // zero everything once so masked slots and unused pages never hold non-finite bytes
+  A(cudaMemsetAsync(c->k_pool, 0, L * c->pool_pages * c->page_bytes_kv, c->stream));
+  A(cudaMemsetAsync(c->v_pool, 0, L * c->pool_pages * c->page_bytes_kv, c->stream));
+  if (c->k_scale) A(cudaMemsetAsync(c->k_scale, 0, L * c->pool_pages * H * sizeof(float), c->stream));
+  if (c->v_scale) A(cudaMemsetAsync(c->v_scale, 0, L * c->pool_pages * H * sizeof(float), c->stream));
+  A(cudaMemsetAsync(c->entries, 0, L * c->pool_pages * sizeof(Entry), c->stream));
+  A(cudaMemsetAsync(c->bitmap, 0, L * c->bitmap_words * sizeof(uint32_t), c->stream));
+  A(cudaMemsetAsync(c->d_err, 0, 4 * sizeof(int), c->stream));
+  if (c->tok_id) {
+    const size_t slots = L * c->pool_pages * P;
+    A(cudaMemsetAsync(c->tok_id, 0, slots * sizeof(int64_t), c->stream));
+    A(cudaMemsetAsync(c->tok_cnt, 0, slots * sizeof(int32_t), c->stream));
+    A(cudaMemsetAsync(c->tok_shat, 0, slots * sizeof(float), c->stream));
+  }
+  A(cudaStreamSynchronize(c->stream));
+  if (e != cudaSuccess) {
+    free_all(c);
+    delete c;
+    cudaGetLastError();
+    return KVC_ERR_CUDA;
+  }
+  if (c->tc_path) {
+    c->tmap_k.resize(1);
+    c->tmap_v.resize(1);
+    const size_t rows = L * c->pool_pages * H * P;
+    if (!encode_pool_tmap(&c->tmap_k[0], c->k_pool, rows, D, P, 2, true) ||
+        !encode_pool_tmap(&c->tmap_v[0], c->v_pool, rows, D, P, 2, true)) {
+      free_all(c);
+      delete c;
+      return KVC_ERR_CUDA;
+    }
+  }
+  c->L.assign(g.num_layers, LayerHost());
+  *out = c;
+  return KVC_OK;
+}
+
+kvc_status kvc_destroy(kvc_cache* c) {
+  if (!c) return KVC_OK;
+  cudaStreamSynchronize(c->stream);
+  free_all(c);
+  delete c;
+  return KVC_OK;
+}
+
+kvc_status kvc_set_stream(kvc_cache* c, void* stream) {
+  if (!c) return KVC_ERR_ARG;
+  c->stream = static_cast<cudaStream_t>(stream);
+  return KVC_OK;
+}
+
+kvc_status kvc_reset(kvc_cache* c) {
+  if (!c) return KVC_ERR_ARG;
+  const size_t L = c->cfg.num_layers;
+  cudaError_t e = cudaMemsetAsync(c->entries, 0, L * c->pool_pages * sizeof(Entry), c->stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->bitmap, 0, L * c->bitmap_words * sizeof(uint32_t), c->stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->d_err, 0, 4 * sizeof(int), c->stream);
+  if (e != cudaSuccess) return cuda_fail(c, e, "kvc_reset");
+  c->L.assign(c->cfg.num_layers, LayerHost());
+  c->hist_frame = -1;
+  c->hist_next_layer = 0;
+  return KVC_OK;
+}
+
+kvc_status kvc_append_frame(kvc_cache* c, int32_t layer, int32_t frame_idx, const void* k_dev, const void* v_dev,
+                            int32_t is_keyframe) {
+  if (!c) return KVC_ERR_ARG;
+  if (!valid_layer(c, layer) || !k_dev || !v_dev || frame_idx < 0)
+    return fail(c, KVC_ERR_ARG, "kvc_append_frame: bad layer, pointer or frame index");
+  if ((reinterpret_cast<uintptr_t>(k_dev) | reinterpret_cast<uintptr_t>(v_dev)) & 15)
+    return fail(c, KVC_ERR_ARG, "kvc_append_frame: K and V must be 16-byte aligned");
+  LayerHost& L = c->L[layer];
+  if (L.has_pending) return fail(c, KVC_ERR_STATE, "kvc_append_frame: a frame is already pending on this layer");
+  if (frame_idx <= L.last_frame) return fail(c, KVC_ERR_STATE, "kvc_append_frame: frame indices must increase");
+  const kvc_config& g = c->cfg;
+  const int n = c->ppf;
+  int used = 0;
+  used = L.n_entries;
+  if (used + n > c->pool_pages) return fail(c, KVC_ERR_STATE, "kvc_append_frame: page pool full");
+  const int T = g.tokens_per_frame, P = g.page_size;
+  Entry* E = layer_entries(c, layer);
+  cudaError_t e = launch_mgr_alloc(c->stream, E, layer_bitmap(c, layer), c->bitmap_words, c->pool_pages,
+                                   L.n_entries, n, frame_idx, P, T - (n - 1) * P, c->d_err);
+  if (e != cudaSuccess) return cuda_fail(c, e, "page allocation");
+  c->launches++;
+  if (g.kv_dtype == KVC_FP8_E4M3) {
+    e = launch_append_fp8(c->stream, k_dev, v_dev, layer_pool(c, c->k_pool, layer), layer_pool(c, c->v_pool, layer),
+                          layer_scale(c, c->k_scale, layer), layer_scale(c, c->v_scale, layer), E + L.n_entries, n, T,
+                          g.num_heads, g.head_dim, P);
+  } else {
+    e = launch_append(c->stream, static_cast<int>(c->elem_kv), k_dev, v_dev, layer_pool(c, c->k_pool, layer),
+                      layer_pool(c, c->v_pool, layer), E + L.n_entries, n, T, g.num_heads, g.head_dim, P);
+  }
+  if (e != cudaSuccess) return cuda_fail(c, e, "append");
+  c->launches++;
+  if (g.budget_tokens > 0) {
+    kvc_status st = init_token_meta(c, layer, L.n_entries, n, frame_idx);
+    if (st != KVC_OK) return st;
+  }
+  L.pending.frame = frame_idx;
+  L.pending.first_entry = L.n_entries;
+  L.pending.n_entries = n;
+  L.has_pending = true;
+  L.pending_key = is_keyframe != 0;
+  L.n_entries += n;
+  L.high_water = std::max<int64_t>(L.high_water, L.n_entries);
+  L.appended++;
+  L.last_frame = frame_idx;
+  return KVC_OK;
+}
+
+kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_dev) {
+  if (!c) return KVC_ERR_ARG;
+  if (!valid_layer(c, layer) || !q_dev || !o_dev) return fail(c, KVC_ERR_ARG, "kvc_attend: bad layer or pointer");
+  if ((reinterpret_cast<uintptr_t>(q_dev) | reinterpret_cast<uintptr_t>(o_dev)) & 15)
+    return fail(c, KVC_ERR_ARG, "kvc_attend: Q and O must be 16-byte aligned");
+  LayerHost& L = c->L[layer];
+  if (!L.has_pending) return fail(c, KVC_ERR_STATE, "kvc_attend: no frame pending on this layer");
+  const kvc_config& g = c->cfg;
+  const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads, D = g.head_dim;
+  Entry* E = layer_entries(c, layer);
+  cudaError_t e;
+  if (c->tc_path) {
+    TcAttnArgs a{};
+    a.q = q_dev;
+    a.o = o_dev;
+    a.entries = E;
+    a.n_pages = L.n_entries;
+    a.T = T;
+    a.H = H;
+    a.P = P;
+    a.page_base = static_cast<long long>(layer) * c->pool_pages;
+    a.softmax_scale = g.softmax_scale;
+    a.splits = g.kv_splits;
+    a.tmap_k = &c->tmap_k[0];
+    a.tmap_v = &c->tmap_v[0];
+    a.fp8 = false;
+    a.part_o = c->part_o;
+    a.part_lse = c->part_lse;
+    a.part_rows = c->part_rows;
+    a.sm_count = c->sm_count;
+    a.err = c->d_err;
+    int launched = 0;
+    e = launch_attn_tc(c->stream, a, nullptr, &launched);
+    c->launches += launched;
+  } else {
+    e = launch_attn_simt(c->stream, g.io_dtype, g.kv_dtype, q_dev, o_dev, layer_pool(c, c->k_pool, layer),
+                         layer_pool(c, c->v_pool, layer), layer_scale(c, c->k_scale, layer),
+                         layer_scale(c, c->v_scale, layer), E, L.n_entries, T, H, D, P, g.softmax_scale);
+    if (e == cudaSuccess) c->launches++;
+  }
+  if (e != cudaSuccess) return cuda_fail(c, e, "attention launch");
+  // commit / evict, or release the skipped frame
+  if (L.pending_key) {
+    L.frames.push_back(L.pending);
+    L.tokens += T;
+    L.committed++;
+    if (g.budget_tokens > 0) {
+      const bool first = L.pending.frame == 0 && g.protect_first_frame;
+      L.protected_tokens += first ? T : std::min(g.num_special_tokens, T);
+    }
+    if (g.window_frames > 0) {
+      const size_t S = static_cast<size_t>(g.scale_frames), W = static_cast<size_t>(g.window_frames);
+      while (L.frames.size() > S + W) {
+        const FrameRec f = L.frames[S];
+        L.frames.erase(L.frames.begin() + S);
+        kvc_status st = remove_entries(c, layer, f.first_entry, f.first_entry + f.n_entries);
+        if (st != KVC_OK) return st;
+        L.tokens -= T;
+        L.evicted++;
+      }
+    }
+  } else {
+    kvc_status st = remove_entries(c, layer, L.pending.first_entry, L.pending.first_entry + L.pending.n_entries);
+    if (st != KVC_OK) return st;
+    L.skipped++;
+  }
+  L.has_pending = false;
+  return KVC_OK;
+}
+
+kvc_status kvc_compress(kvc_cache* c, int32_t layer, const float* residual_dev, int32_t* fired_out) {
+  if (!c) return KVC_ERR_ARG;
+  if (fired_out) *fired_out = 0;
+  if (!valid_layer(c, layer)) return fail(c, KVC_ERR_ARG, "kvc_compress: bad layer");
+  if (c->cfg.budget_tokens <= 0) return fail(c, KVC_ERR_ARG, "kvc_compress: budget_tokens is 0");
+  if (!residual_dev) return fail(c, KVC_ERR_ARG, "kvc_compress: residual is NULL");
+  return compress_layer(c, layer, residual_dev, fired_out);
+}
+
+kvc_status kvc_page_table(kvc_cache* c, int32_t layer, int32_t* rows_host, int32_t capacity, int32_t* n_rows,
+                          kvc_info* info) {
+  if (!c) return KVC_ERR_ARG;
+  if (!valid_layer(c, layer)) return fail(c, KVC_ERR_ARG, "kvc_page_table: bad layer");
+  kvc_status st = sync_and_check(c);
+  if (st != KVC_OK) return st;
+  LayerHost& L = c->L[layer];
+  const int n = L.n_entries;
+  if (n_rows) *n_rows = n;
+  if (rows_host && capacity > 0 && n > 0) {
+    std::vector<Entry> tmp(n);
+    cudaError_t e = cudaMemcpy(tmp.data(), layer_entries(c, layer), n * sizeof(Entry), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(c, e, "kvc_page_table copy");
+    const int m = std::min(n, capacity);
+    for (int i = 0; i < m; ++i) {
+      rows_host[4 * i + 0] = tmp[i].y;
+      rows_host[4 * i + 1] = tmp[i].z;
+      rows_host[4 * i + 2] = tmp[i].x;
+      rows_host[4 * i + 3] = tmp[i].w;
+    }
+  }
+  if (info) {
+    int derr = 0;
+    cudaMemcpy(&derr, c->d_err, sizeof(int), cudaMemcpyDeviceToHost);
+    info->tokens = L.tokens;
+    info->pages_used = L.n_entries;
+    info->pages_total = c->pool_pages;
+    info->pool_bytes = static_cast<int64_t>(c->pool_pages) * c->page_bytes_kv * 2;
+    info->high_water_pages = L.high_water;
+    info->frames_appended = L.appended;
+    info->frames_committed = L.committed;
+    info->frames_skipped = L.skipped;
+    info->frames_evicted = L.evicted;
+    info->compress_events = L.compressions;
+    info->device_error = derr;
+    info->kernel_launches = c->launches;
+  }
+  return KVC_OK;
+}
+
+kvc_status kvc_token_meta(kvc_cache* c, int32_t layer, int64_t* ids_host, int32_t* counts_host, float* shat_host,
+                          int32_t capacity, int32_t* n_out) {
+  if (!c) return KVC_ERR_ARG;
+  if (!valid_layer(c, layer)) return fail(c, KVC_ERR_ARG, "kvc_token_meta: bad layer");
+  if (!c->tok_id) return fail(c, KVC_ERR_UNSUPPORTED, "kvc_token_meta: token metadata exists in budget mode only");
+  kvc_status st = sync_and_check(c);
+  if (st != KVC_OK) return st;
+  LayerHost& L = c->L[layer];
+  const int n = L.n_entries;
+  std::vector<Entry> ent(n);
+  if (n > 0 &&
+      cudaMemcpy(ent.data(), layer_entries(c, layer), n * sizeof(Entry), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return fail(c, KVC_ERR_CUDA, "kvc_token_meta copy");
+  const int P = c->cfg.page_size;
+  const size_t base = static_cast<size_t>(layer) * c->pool_pages * P;
+  std::vector<int64_t> ids(static_cast<size_t>(c->pool_pages) * P);
+  std::vector<int32_t> cnt(ids.size());
+  std::vector<float> sh(ids.size());
+  cudaMemcpy(ids.data(), c->tok_id + base, ids.size() * sizeof(int64_t), cudaMemcpyDeviceToHost);
+  cudaMemcpy(cnt.data(), c->tok_cnt + base, cnt.size() * sizeof(int32_t), cudaMemcpyDeviceToHost);
+  cudaMemcpy(sh.data(), c->tok_shat + base, sh.size() * sizeof(float), cudaMemcpyDeviceToHost);
+  int k = 0;
+  for (int i = 0; i < n; ++i) {
+    for (int s = 0; s < ent[i].w; ++s, ++k) {
+      if (k >= capacity) continue;
+      const size_t slot = static_cast<size_t>(ent[i].x) * P + s;
+      if (ids_host) ids_host[k] = ids[slot];
+      if (counts_host) counts_host[k] = cnt[slot];
+      if (shat_host) shat_host[k] = sh[slot];
+    }
+  }
+  if (n_out) *n_out = k;
+  return KVC_OK;
+}
+
+kvc_status kvc_export_pages(kvc_cache* c, int32_t layer, int32_t first_row, int32_t n_rows, void* k_host,
+                            void* v_host, float* k_scale_host, float* v_scale_host) {
+  if (!c) return KVC_ERR_ARG;
+  if (!valid_layer(c, layer)) return fail(c, KVC_ERR_ARG, "kvc_export_pages: bad layer");
+  kvc_status st = sync_and_check(c);
+  if (st != KVC_OK) return st;
+  LayerHost& L = c->L[layer];
+  if (first_row < 0 || n_rows < 0 || first_row + n_rows > L.n_entries)
+    return fail(c, KVC_ERR_ARG, "kvc_export_pages: row range outside the page table");
+  std::vector<Entry> ent(n_rows);
+  if (n_rows > 0 && cudaMemcpy(ent.data(), layer_entries(c, layer) + first_row, n_rows * sizeof(Entry),
+                               cudaMemcpyDeviceToHost) != cudaSuccess)
+    return fail(c, KVC_ERR_CUDA, "kvc_export_pages copy");
+  const int H = c->cfg.num_heads;
+  for (int i = 0; i < n_rows; ++i) {
+    const size_t phys = ent[i].x;
+    const size_t off = phys * c->page_bytes_kv;
+    if (k_host)
+      cudaMemcpy(static_cast<uint8_t*>(k_host) + i * c->page_bytes_kv, layer_pool(c, c->k_pool, layer) + off,
+                 c->page_bytes_kv, cudaMemcpyDeviceToHost);
+    if (v_host)
+      cudaMemcpy(static_cast<uint8_t*>(v_host) + i * c->page_bytes_kv, layer_pool(c, c->v_pool, layer) + off,
+                 c->page_bytes_kv, cudaMemcpyDeviceToHost);
+    if (k_scale_host && c->k_scale)
+      cudaMemcpy(k_scale_host + static_cast<size_t>(i) * H, layer_scale(c, c->k_scale, layer) + phys * H,
+                 H * sizeof(float), cudaMemcpyDeviceToHost);
+    if (v_scale_host && c->v_scale)
+      cudaMemcpy(v_scale_host + static_cast<size_t>(i) * H, layer_scale(c, c->v_scale, layer) + phys * H,
+                 H * sizeof(float), cudaMemcpyDeviceToHost);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(c, e, "kvc_export_pages");
+  return KVC_OK;
+}
+
+kvc_status kvc_step_host(kvc_cache* c, int32_t layer, int32_t frame_idx, int32_t is_keyframe, const void* q_host,
+                         const void* k_host, const void* v_host, void* o_host) {
+  if (!c) return KVC_ERR_ARG;
+  if (!q_host || !k_host || !v_host || !o_host) return fail(c, KVC_ERR_ARG, "kvc_step_host: NULL host buffer");
+  const kvc_config& g = c->cfg;
+  const size_t bytes = static_cast<size_t>(g.tokens_per_frame) * g.num_heads * g.head_dim * c->elem_io;
+  cudaError_t e = cudaMemcpyAsync(c->stage_q, q_host, bytes, cudaMemcpyHostToDevice, c->stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->stage_k, k_host, bytes, cudaMemcpyHostToDevice, c->stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->stage_v, v_host, bytes, cudaMemcpyHostToDevice, c->stream);
+  if (e != cudaSuccess) return cuda_fail(c, e, "kvc_step_host upload");
+  kvc_status st = kvc_append_frame(c, layer, frame_idx, c->stage_k, c->stage_v, is_keyframe);
+  if (st != KVC_OK) return st;
+  st = kvc_attend(c, layer, c->stage_q, c->stage_o);
+  if (st != KVC_OK) return st;
+  e = cudaMemcpyAsync(o_host, c->stage_o, bytes, cudaMemcpyDeviceToHost, c->stream);
+  if (e != cudaSuccess) return cuda_fail(c, e, "kvc_step_host download");
+  e = cudaStreamSynchronize(c->stream);
+  if (e != cudaSuccess) return cuda_fail(c, e, "kvc_step_host sync");
+  return KVC_OK;
+}
+
+kvc_status kvc_synchronize(kvc_cache* c) {
+  if (!c) return KVC_ERR_ARG;
+  return sync_and_check(c);
+}
+
+kvc_status kvc_debug_bounded_wait(kvc_cache* c, int32_t timeout_us) {
+  if (!c || timeout_us < 0) return KVC_ERR_ARG;
+  cudaError_t e = launch_debug_wait(c->stream, c->d_err + 1, c->d_err, static_cast<long long>(timeout_us) * 1000);
+  if (e != cudaSuccess) return cuda_fail(c, e, "kvc_debug_bounded_wait");
+  c->launches++;
+  return KVC_OK;
+}
+
+}  // extern "C"

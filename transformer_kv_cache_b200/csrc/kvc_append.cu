@@ -1,0 +1,149 @@
+// kvc_append.cu -- page-aligned append of one frame's K and V, optionally with FP8 E4M3
+// absmax quantisation per (page, head).
+//
+// Layout ("Can LingBot-Map Achieve 20 FPS", Page-Aligned Tensor Layout): the caller's
+// token-major [T, H, D] tensors are written straight into pool pages laid out as
+// [page][head][slot][dim], so each (page, head) block is P*D contiguous elements: one
+// TMA box for attention. Slot j of the frame goes to page j / P, offset j % P; slots past
+// T in the frame's last page are written as zeros so masked columns never hold garbage.
+//
+// HBM-bound: every byte is read once and written once with 16-byte vector accesses,
+// iterated in destination order so stores are fully coalesced and each source row of
+// D elements is read by consecutive threads.
+#include <cuda_bf16.h>
+
+#include "kvc_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace kvc {
+
+// One 16-byte chunk per thread-iteration; `vec` = elements per chunk.
+__global__ void append_kernel(const uint4* __restrict__ k_in, const uint4* __restrict__ v_in, uint4* k_pool,
+                              uint4* v_pool, const Entry* __restrict__ entries, int n_pages, int T, int H,
+                              int chunks_per_row, int P) {
+  const long long per_tensor = static_cast<long long>(n_pages) * H * P * chunks_per_row;
+  const long long total = 2 * per_tensor;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const bool is_v = idx >= per_tensor;
+    long long r = is_v ? idx - per_tensor : idx;
+    const int c = static_cast<int>(r % chunks_per_row);
+    r /= chunks_per_row;
+    const int slot = static_cast<int>(r % P);
+    r /= P;
+    const int h = static_cast<int>(r % H);
+    const int g = static_cast<int>(r / H);
+    const int tok = g * P + slot;
+    const int phys = __ldg(&entries[g].x);
+    uint4 val = make_uint4(0, 0, 0, 0);
+    const uint4* src = is_v ? v_in : k_in;
+    if (tok < T) val = __ldg(&src[(static_cast<long long>(tok) * H + h) * chunks_per_row + c]);
+    uint4* dst = is_v ? v_pool : k_pool;
+    dst[((static_cast<long long>(phys) * H + h) * P + slot) * chunks_per_row + c] = val;
+  }
+}
+
+// Two fp32 values -> two E4M3 codes, round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// One warp per (page, head, tensor). The block of valid tokens x D dims is reduced to its
+// absolute maximum; scale = fp32(amax / 448) with an IEEE-rounded division; each code is
+// the E4M3 rounding of the IEEE-rounded fp32 quotient x / scale; an all-zero block has
+// scale 0 and codes 0 ("XStreamVGGT" abstract: KV cache quantisation; OCP FP8 E4M3).
+// Requires D % 8 == 0 and P * D <= 32 * 64.
+__global__ void append_fp8_kernel(const __nv_bfloat16* __restrict__ k_in, const __nv_bfloat16* __restrict__ v_in,
+                                  uint8_t* k_pool, uint8_t* v_pool, float* k_scale, float* v_scale,
+                                  const Entry* __restrict__ entries, int n_pages, int T, int H, int D, int P) {
+  const int warps_per_block = blockDim.x / 32;
+  const int gw = blockIdx.x * warps_per_block + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  const int n_items = n_pages * H * 2;
+  if (gw >= n_items) return;
+  const int tensor = gw % 2;
+  const int ph = gw / 2;
+  const int h = ph % H;
+  const int g = ph / H;
+  const int phys = __ldg(&entries[g].x);
+  const __nv_bfloat16* src = tensor ? v_in : k_in;
+  uint8_t* dst = (tensor ? v_pool : k_pool) + (static_cast<long long>(phys) * H + h) * P * D;
+  float* sc = (tensor ? v_scale : k_scale) + static_cast<long long>(phys) * H + h;
+  const int vec_per_row = D / 8;
+  const int n_vec = P * vec_per_row;     // 8-element groups in the block
+  // each lane handles groups lane, lane + 32, ... (at most 8 for P*D <= 2048)
+  float x[8][8];
+  int nmine = 0;
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int v = lane + 32 * k;
+    if (v < n_vec) {
+      const int slot = v / vec_per_row, c = v % vec_per_row;
+      const int tok = g * P + slot;
+      if (tok < T) {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src + (static_cast<long long>(tok) * H + h) * D) + c);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(b2[e]);
+          x[k][2 * e] = f.x;
+          x[k][2 * e + 1] = f.y;
+          amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[k][e] = 0.f;
+      }
+      nmine = k + 1;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 0.f;
+  if (lane == 0) *sc = scale;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    if (k < nmine) {
+      const int v = lane + 32 * k;
+      uint2 packed = make_uint2(0, 0);
+      if (scale > 0.f) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w[e] = e4m3x2(__fdiv_rn(x[k][2 * e], scale), __fdiv_rn(x[k][2 * e + 1], scale));
+        packed.x = w[0] | (w[1] << 16);
+        packed.y = w[2] | (w[3] << 16);
+      }
+      reinterpret_cast<uint2*>(dst)[v] = packed;
+    }
+  }
+}
+
+cudaError_t launch_append(cudaStream_t s, int elem_bytes, const void* k, const void* v, void* k_pool,
+                          void* v_pool, const Entry* entries, int n_pages, int T, int H, int D, int P) {
+  const int chunks_per_row = D * elem_bytes / 16;
+  const long long total = 2LL * n_pages * H * P * chunks_per_row;
+  const int threads = 256;
+  long long blocks = (total + threads - 1) / threads;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks < 1) blocks = 1;
+  append_kernel<<<static_cast<int>(blocks), threads, 0, s>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_pool),
+      static_cast<uint4*>(v_pool), entries, n_pages, T, H, chunks_per_row, P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_fp8(cudaStream_t s, const void* k, const void* v, uint8_t* k_pool, uint8_t* v_pool,
+                              float* k_scale, float* v_scale, const Entry* entries, int n_pages, int T, int H,
+                              int D, int P) {
+  const int items = n_pages * H * 2;
+  const int warps = 8;
+  append_fp8_kernel<<<(items + warps - 1) / warps, warps * 32, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), k_pool, v_pool, k_scale, v_scale,
+      entries, n_pages, T, H, D, P);
+  return cudaGetLastError();
+}
+
+}  // namespace kvc

@@ -1,0 +1,148 @@
+// kvc_internal.h -- host-side state of a kvc_cache and the launchers of every kernel.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/kvc.h"
+
+namespace kvc {
+
+// A committed frame's pages are a contiguous run of entries in the layer's page list.
+struct FrameRec {
+  int32_t frame = -1;
+  int32_t first_entry = 0;
+  int32_t n_entries = 0;
+};
+
+struct LayerHost {
+  int32_t n_entries = 0;          // entries in the device page list (block + frames + pending)
+  int32_t block_entries = 0;      // leading entries written by compaction (owner -1)
+  int64_t block_tokens = 0;
+  std::vector<FrameRec> frames;   // committed frames after the block, in cache order
+  bool has_pending = false;
+  bool pending_key = false;
+  FrameRec pending;
+  int32_t last_frame = -1;
+  int64_t tokens = 0;             // committed tokens
+  int64_t high_water = 0;
+  int64_t appended = 0, committed = 0, skipped = 0, evicted = 0, compressions = 0;
+  bool seen_frame0 = false;       // frame 0 committed (its tokens are protected)
+  int64_t protected_tokens = 0;   // committed protected tokens (compression)
+  int32_t last_merge_n = 0;
+  int32_t scored_frame = -1;      // frame whose residual was last scored on this layer
+};
+
+// Device page-table entry: x = physical page, y = owner frame (-1: compaction block),
+// z = page index within the owner, w = valid tokens in the page.
+using Entry = int4;
+
+struct Cache {
+  kvc_config cfg{};
+  cudaStream_t stream = nullptr;
+  int device = 0;
+  int sm_count = 148;
+  int ppf = 0;                      // pages per frame
+  int pool_pages = 0;               // pages per layer
+  int bitmap_words = 0;
+  size_t elem_io = 4, elem_kv = 4;  // bytes
+  size_t page_elems = 0;            // H * P * D
+  size_t page_bytes_kv = 0;         // one tensor (K or V) page
+  // device memory (one allocation each, all layers)
+  uint8_t* k_pool = nullptr;        // [layers][pool_pages][H][P][D]
+  uint8_t* v_pool = nullptr;
+  float* k_scale = nullptr;         // FP8: [layers][pool_pages][H]
+  float* v_scale = nullptr;
+  Entry* entries = nullptr;         // [layers][pool_pages]
+  uint32_t* bitmap = nullptr;       // [layers][bitmap_words]
+  int* d_err = nullptr;             // [0] error word, [1] a flag nobody sets
+  // compression metadata, budget mode only: [layers][pool_pages][P]
+  int64_t* tok_id = nullptr;
+  int32_t* tok_cnt = nullptr;
+  float* tok_shat = nullptr;
+  // compression scratch
+  void* cmp_scratch = nullptr;
+  size_t cmp_scratch_bytes = 0;
+  // attention split scratch (partial O and log-sum-exp)
+  float* part_o = nullptr;
+  float* part_lse = nullptr;
+  size_t part_rows = 0;             // capacity in 128-row partial tiles
+  // host-buffer step staging
+  uint8_t* stage_q = nullptr;
+  uint8_t* stage_k = nullptr;
+  uint8_t* stage_v = nullptr;
+  uint8_t* stage_o = nullptr;
+  // tensor maps of each layer's K and V pools (bf16 tensor-core path)
+  std::vector<CUtensorMap> tmap_k, tmap_v;
+  bool tc_path = false;
+  std::vector<LayerHost> L;
+  std::string last_error;
+  // rank history of the frame being scored (compression): [rank_window][T] int32
+  int32_t* rank_hist = nullptr;
+  int32_t hist_frame = -1;
+  int32_t hist_next_layer = 0;
+  int64_t launches = 0;             // kernels launched by this cache
+};
+
+}  // namespace kvc
+
+// The opaque handle of the C ABI is the host-side cache state.
+struct kvc_cache : public kvc::Cache {};
+
+namespace kvc {
+
+// ------------------------------------------------------------------ launchers
+// Page-table manager (one CTA).
+cudaError_t launch_mgr_alloc(cudaStream_t s, Entry* entries, uint32_t* bitmap, int words, int pool_pages,
+                             int start, int n_new, int owner, int valid_full, int valid_last, int* err);
+cudaError_t launch_mgr_remove(cudaStream_t s, Entry* entries, uint32_t* bitmap, int n_entries, int a, int b,
+                              int* err);
+cudaError_t launch_debug_wait(cudaStream_t s, int* flag, int* err, long long timeout_ns);
+
+// Append (same dtype in and out): K, V [T,H,D] -> pages of entries [0, n_pages).
+cudaError_t launch_append(cudaStream_t s, int elem_bytes, const void* k, const void* v, void* k_pool,
+                          void* v_pool, const Entry* entries, int n_pages, int T, int H, int D, int P);
+// Append with FP8 E4M3 absmax quantisation per (page, head); bf16 input.
+cudaError_t launch_append_fp8(cudaStream_t s, const void* k, const void* v, uint8_t* k_pool, uint8_t* v_pool,
+                              float* k_scale, float* v_scale, const Entry* entries, int n_pages, int T, int H,
+                              int D, int P);
+
+// SIMT attention (fp32 arithmetic) over pages [0, n_pages) of a layer.
+cudaError_t launch_attn_simt(cudaStream_t s, int io_dtype, int kv_dtype, const void* q, void* o,
+                             const void* k_pool, const void* v_pool, const float* k_scale, const float* v_scale,
+                             const Entry* entries, int n_pages, int T, int H, int D, int P, float softmax_scale);
+
+// Tensor-core attention (bf16 or FP8 storage, D = 64).
+struct TcAttnArgs {
+  const void* q;
+  void* o;
+  const Entry* entries;
+  int n_pages, T, H, P;
+  long long page_base;              // first pool page of the layer (layer * pool_pages)
+  float softmax_scale;
+  int splits;                       // 0: choose automatically
+  const CUtensorMap* tmap_k;
+  const CUtensorMap* tmap_v;
+  const float* k_scale;             // FP8 only
+  const float* v_scale;
+  bool fp8;
+  float* part_o;
+  float* part_lse;
+  size_t part_rows;
+  int sm_count;
+  int* err;
+};
+// Returns the number of kernels launched through *launched.
+cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used, int* launched);
+int choose_splits(int units, int tiles, int slots);
+
+// Tensor map for a pool: rows of D elements, box of P rows.
+bool encode_pool_tmap(CUtensorMap* map, void* base, size_t rows, int D, int P, int elem_bytes, bool swizzle128);
+
+// Compression kernels.
+cudaError_t launch_score(cudaStream_t s, const float* residual, int T, int R, int layer_slot, int n_hist,
+                         int32_t* rank_hist, int window, float lam, float* shat_out);
+}  // namespace kvc
