@@ -486,13 +486,16 @@ class StreamOracle:
         eligible = sorted(kept_other)          # targets: kept tokens that are not protected
         targets = {}
         if eligible and merged:
+            # cos(K_m, K_j) = K_m . K_j / (|K_j| |K_m|) for every (merge, eligible) pair, as
+            # one matrix product; argmax takes the first maximum = the lowest id on ties
             E = Kf[eligible]
             En = np.sqrt((E * E).sum(axis=1))
-            for m in merged:
-                km = Kf[m]
-                cos = (E @ km) / (En * math.sqrt(float(km @ km)))
-                best = int(np.argmax(cos))      # first maximum = lowest id among ties
-                targets[m] = eligible[best]
+            M = Kf[merged]
+            Mn = np.sqrt((M * M).sum(axis=1))
+            cos = (M @ E.T) / (En[None, :] * Mn[:, None])
+            best = np.argmax(cos, axis=1)
+            for r, m in enumerate(merged):
+                targets[m] = eligible[int(best[r])]
         else:
             dropped = sorted(dropped + merged)
             merged = []

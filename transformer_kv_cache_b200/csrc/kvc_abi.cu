@@ -152,6 +152,7 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   if (g.window_frames > 0 && g.budget_tokens > 0) return KVC_ERR_ARG;
   if (g.budget_tokens > 0) {
     if (g.kv_dtype != KVC_BF16 || !(g.keep_frac > 0.f && g.keep_frac <= 1.f) || g.rank_window < 1 ||
+        g.rank_window > 32 || g.tokens_per_frame > 12288 ||
         g.residual_dim < 1 || !(g.lambda_ >= 0.f) || g.budget_tokens > (1 << 24))
       return KVC_ERR_ARG;
   }
@@ -286,6 +287,7 @@ kvc_status kvc_reset(kvc_cache* c) {
   c->L.assign(c->cfg.num_layers, LayerHost());
   c->hist_frame = -1;
   c->hist_next_layer = 0;
+  c->hist_layers.clear();
   return KVC_OK;
 }
 

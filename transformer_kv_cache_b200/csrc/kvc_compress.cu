@@ -1,16 +1,751 @@
-// kvc_compress.cu -- importance scoring and keep/merge/drop compression (budget mode).
+// kvc_compress.cu -- importance scoring and keep / merge / drop compression (budget mode).
+//
+// Scoring follows the StreamCacheVGGT page, sections 2.1.1-2.1.4: the raw score of a token
+// is the L2 norm of its FFN residual; at every layer the frame's tokens are ranked by it
+// (0 = largest); over a window of the last W layers of the same frame the normalised ranks
+// R/(N-1) have a population standard deviation sigma, compared with the uniform-null
+// spread 1/sqrt(12): Cons = max(0, 1 - sigma*sqrt(12)); s_hat = s * (1 + lambda * Cons).
+// The rank history is kept per frame and reset when a new frame starts.
+//
+// Compression follows section 2 of that page (keep the core, merge the middle into the
+// core, drop the rest); sizes, the merge rule and the protected set follow the budgeted
+// workload's statement: keep floor(keep_frac * B) tokens (protected ones first), merge the
+// next B - floor(keep_frac * B) into the kept non-protected token of highest full-key
+// cosine as count-weighted means, drop the remainder, then rewrite the kept tokens in
+// ascending id into fresh pages.
+//
+// Every step whose result is an integer (ranks, tiers, targets) or a stored value is
+// computed in fp64 with the operation order written next to it, so the results match an
+// fp64 reference bit for bit; the fp64 helpers below use explicitly rounded intrinsics so
+// the compiler cannot contract them into fused multiply-adds.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cmath>
+
 #include "kvc_internal.h"
 #include "sm100_ptx.cuh"
 
 namespace kvc {
 
-size_t compress_scratch_bytes(const kvc_config& cfg, int pool_pages) { return 16; }
+namespace {
 
-kvc_status init_token_meta(kvc_cache* c, int layer, int first_entry, int n_pages, int frame) { return KVC_OK; }
+constexpr int kCosTile = 64;     // sources x targets per CTA in the cosine kernel
+constexpr int kCosK = 32;        // dims per shared-memory stage
+
+struct Scratch {
+  int64_t* ids;
+  float* shat;
+  int32_t* slot;
+  int32_t* cnt;
+  uint8_t* prot;
+  int32_t* rank;
+  int32_t* keep;
+  int32_t* elig;
+  int32_t* merge;
+  int32_t* counts;     // [0] N, [1] keep, [2] elig, [3] merge
+  int32_t* target;     // index into elig, per merge source
+  int32_t* order;      // merge sources sorted by (target, source)
+  float* ks;
+  float* ke;
+  double* ns;
+  double* ne;
+  double* best_v;
+  int32_t* best_j;
+  float* s_raw;        // raw scores of the frame being scored [T]
+  int64_t* last_src;   // [layers][merge cap]
+  int64_t* last_dst;
+};
+
+struct Caps {
+  size_t n_max, n_keep, n_merge, hd, tiles;
+};
+
+Caps caps_of(const kvc_config& g) {
+  Caps c;
+  const size_t B = g.budget_tokens;
+  c.n_max = B + g.tokens_per_frame;
+  c.n_keep = static_cast<size_t>(std::floor(static_cast<double>(g.keep_frac) * static_cast<double>(B)));
+  if (c.n_keep < 1) c.n_keep = 1;
+  c.n_merge = B > c.n_keep ? B - c.n_keep : 1;
+  c.hd = static_cast<size_t>(g.num_heads) * g.head_dim;
+  c.tiles = (c.n_keep + kCosTile - 1) / kCosTile;
+  return c;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Lays out the scratch regions; with base == nullptr only the total size is computed.
+size_t carve(const kvc_config& g, uint8_t* base, Scratch* s) {
+  const Caps c = caps_of(g);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> uint8_t* {
+    uint8_t* p = base ? base + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  Scratch t;
+  t.ids = reinterpret_cast<int64_t*>(take(c.n_max * 8));
+  t.shat = reinterpret_cast<float*>(take(c.n_max * 4));
+  t.slot = reinterpret_cast<int32_t*>(take(c.n_max * 4));
+  t.cnt = reinterpret_cast<int32_t*>(take(c.n_max * 4));
+  t.prot = take(c.n_max);
+  t.rank = reinterpret_cast<int32_t*>(take(c.n_max * 4));
+  t.keep = reinterpret_cast<int32_t*>(take(c.n_max * 4));
+  t.elig = reinterpret_cast<int32_t*>(take(c.n_max * 4));
+  t.merge = reinterpret_cast<int32_t*>(take(c.n_max * 4));
+  t.counts = reinterpret_cast<int32_t*>(take(16 * 4));
+  t.target = reinterpret_cast<int32_t*>(take(c.n_merge * 4));
+  t.order = reinterpret_cast<int32_t*>(take(c.n_merge * 4));
+  t.ks = reinterpret_cast<float*>(take(c.n_merge * c.hd * 4));
+  t.ke = reinterpret_cast<float*>(take(c.n_keep * c.hd * 4));
+  t.ns = reinterpret_cast<double*>(take(c.n_merge * 8));
+  t.ne = reinterpret_cast<double*>(take(c.n_keep * 8));
+  t.best_v = reinterpret_cast<double*>(take(c.n_merge * c.tiles * 8));
+  t.best_j = reinterpret_cast<int32_t*>(take(c.n_merge * c.tiles * 4));
+  t.s_raw = reinterpret_cast<float*>(take(static_cast<size_t>(g.tokens_per_frame) * 4));
+  t.last_src = reinterpret_cast<int64_t*>(take(static_cast<size_t>(g.num_layers) * c.n_merge * 8));
+  t.last_dst = reinterpret_cast<int64_t*>(take(static_cast<size_t>(g.num_layers) * c.n_merge * 8));
+  if (s) *s = t;
+  return off;
+}
+
+// fp64 -> bf16, round to nearest even, one rounding (written from the format's
+// definition: 8 significant bits, subnormal quantum 2^-133, overflow to infinity).
+__device__ __forceinline__ __nv_bfloat16 f64_to_bf16_rne(double x) {
+  if (x == 0.0 || isnan(x) || isinf(x)) return __float2bfloat16_rn(static_cast<float>(x));
+  int e = ilogb(x);                    // |x| in [2^e, 2^(e+1))
+  int qe = e - 7;                      // quantum of 8 significant bits
+  if (qe < -133) qe = -133;
+  const double y = ldexp(rint(ldexp(x, -qe)), qe);   // exact scaling; rint = ties to even
+  if (fabs(y) > 3.3895313892515355e38) return __float2bfloat16_rn(y > 0 ? INFINITY : -INFINITY);
+  return __float2bfloat16_rn(static_cast<float>(y));  // y is a bf16 value: exact
+}
+
+// ------------------------------------------------------------------ scoring
+// s_i = fp32(sqrt(sum_c r_ic^2)); the squares (exact in fp64) are summed in ascending c.
+__global__ void residual_norm_kernel(const float* __restrict__ r, int T, int R, float* __restrict__ s_out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= T) return;
+  const float* row = r + static_cast<long long>(i) * R;
+  double acc = 0.0;
+  for (int c = 0; c < R; ++c) {
+    const double x = static_cast<double>(__ldg(&row[c]));
+    acc = __dadd_rn(acc, __dmul_rn(x, x));
+  }
+  s_out[i] = __double2float_rn(__dsqrt_rn(acc));
+}
+
+// Ranks of the frame's T tokens (s descending, ties to the lower slot), stored in the
+// history slot of this layer; then, over the window layers in `mask`, the population
+// variance of the normalised ranks gives Cons and s_hat, written next to the tokens.
+__global__ void __launch_bounds__(1024) clces_kernel(const float* __restrict__ s, int T, int32_t* hist, int slot,
+                                                      uint32_t mask, int n_win, float lam,
+                                                      const Entry* __restrict__ frame_pages, int P,
+                                                      float* __restrict__ tok_shat_layer) {
+  extern __shared__ float s_sm[];
+  for (int i = threadIdx.x; i < T; i += blockDim.x) s_sm[i] = s[i];
+  __syncthreads();
+  for (int i = threadIdx.x; i < T; i += blockDim.x) {
+    const float si = s_sm[i];
+    int r = 0;
+    for (int j = 0; j < T; ++j) {
+      const float sj = s_sm[j];
+      r += (sj > si) || (sj == si && j < i);
+    }
+    hist[slot * T + i] = r;
+  }
+  __syncthreads();
+  const double sqrt12 = __dsqrt_rn(12.0);
+  const double lamd = static_cast<double>(lam);
+  for (int i = threadIdx.x; i < T; i += blockDim.x) {
+    long long sr = 0, sr2 = 0;
+    for (int k = 0; k < 32; ++k) {
+      if (mask & (1u << k)) {
+        const long long v = hist[k * T + i];
+        sr += v;
+        sr2 += v * v;
+      }
+    }
+    const long long Dv = static_cast<long long>(n_win) * sr2 - sr * sr;
+    const double sigma = __ddiv_rn(__dsqrt_rn(static_cast<double>(Dv)),
+                                   __dmul_rn(static_cast<double>(n_win), static_cast<double>(T - 1)));
+    double cons = __dsub_rn(1.0, __dmul_rn(sigma, sqrt12));
+    if (cons < 0.0) cons = 0.0;
+    const double w = __dmul_rn(static_cast<double>(s_sm[i]), __dadd_rn(1.0, __dmul_rn(lamd, cons)));
+    const int g = i / P;
+    const int phys = frame_pages[g].x;
+    tok_shat_layer[static_cast<long long>(phys) * P + (i % P)] = __double2float_rn(w);
+  }
+}
+
+// Metadata of a freshly appended frame: id = frame * T + slot, count 1, score 0.
+__global__ void meta_init_kernel(int64_t* tok_id, int32_t* tok_cnt, float* tok_shat, const Entry* pages, int n_pages,
+                                 int P, int T, int frame) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n_pages * P) return;
+  const int g = idx / P, s = idx % P;
+  const int tok = g * P + s;
+  const long long phys = pages[g].x;
+  const long long k = phys * P + s;
+  tok_id[k] = tok < T ? static_cast<int64_t>(frame) * T + tok : -1;
+  tok_cnt[k] = tok < T ? 1 : 0;
+  tok_shat[k] = 0.f;
+}
+
+// ------------------------------------------------------------------ tiering
+// Flatten the cache into position order (page-table order, valid slots only; positions
+// ascend with token id) with the metadata each later step needs.
+__global__ void __launch_bounds__(1024) gather_meta_kernel(const Entry* __restrict__ entries, int n_entries, int P,
+                                                            const int64_t* __restrict__ tok_id,
+                                                            const int32_t* __restrict__ tok_cnt,
+                                                            const float* __restrict__ tok_shat, int T, int specials,
+                                                            int protect_first, Scratch sc) {
+  __shared__ int s_warp[32];
+  __shared__ int s_base;
+  if (threadIdx.x == 0) s_base = 0;
+  __syncthreads();
+  for (int chunk = 0; chunk < n_entries; chunk += blockDim.x) {
+    const int e = chunk + threadIdx.x;
+    const int v = e < n_entries ? entries[e].w : 0;
+    // block exclusive scan of v
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = lane < static_cast<int>(blockDim.x >> 5) ? s_warp[lane] : 0;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      s_warp[lane] = w;
+    }
+    __syncthreads();
+    const int pos0 = s_base + (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
+    const int total = s_warp[(blockDim.x >> 5) - 1];
+    if (e < n_entries) {
+      const int phys = entries[e].x;
+      for (int s = 0; s < v; ++s) {
+        const int pos = pos0 + s;
+        const long long k = static_cast<long long>(phys) * P + s;
+        const int64_t id = tok_id[k];
+        sc.ids[pos] = id;
+        sc.shat[pos] = tok_shat[k];
+        sc.cnt[pos] = tok_cnt[k];
+        sc.slot[pos] = static_cast<int32_t>(k);
+        const int64_t frame = id / T, tslot = id % T;
+        sc.prot[pos] = (tslot < specials) || (protect_first && frame == 0);
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) s_base += total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) sc.counts[0] = s_base;
+}
+
+// Order of the non-protected tokens by (s_hat descending, id ascending), as a rank found
+// by counting: positions ascend with id, so (key, position) is a strict total order.
+__device__ __forceinline__ uint32_t desc_key(float f) {
+  // maps larger floats to smaller unsigned keys (total order on finite values)
+  uint32_t u = __float_as_uint(f);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ~u;
+}
+
+__global__ void tier_rank_kernel(Scratch sc, int N) {
+  extern __shared__ uint32_t keys_sm[];   // [chunk]
+  uint8_t* prot_sm = reinterpret_cast<uint8_t*>(keys_sm + 2048);
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const bool mine = i < N && !sc.prot[i];
+  const uint32_t ki = i < N ? desc_key(sc.shat[i]) : 0u;
+  int r = 0;
+  for (int base = 0; base < N; base += 2048) {
+    const int n = min(2048, N - base);
+    __syncthreads();
+    for (int j = threadIdx.x; j < n; j += blockDim.x) {
+      keys_sm[j] = desc_key(sc.shat[base + j]);
+      prot_sm[j] = sc.prot[base + j];
+    }
+    __syncthreads();
+    if (mine) {
+      for (int j = 0; j < n; ++j) {
+        const uint32_t kj = keys_sm[j];
+        const int pj = base + j;
+        r += !prot_sm[j] && (kj < ki || (kj == ki && pj < i));
+      }
+    }
+  }
+  if (i < N) sc.rank[i] = mine ? r : -1;
+}
+
+// Tier lists in position order: keep (protected or rank < n_keep_other), eligible
+// targets (kept, not protected) and merge sources (next n_merge ranks).
+__global__ void __launch_bounds__(1024) tier_lists_kernel(Scratch sc, int N, int n_keep_other, int n_merge) {
+  __shared__ int s_warp[3][32];
+  __shared__ int s_base[3];
+  if (threadIdx.x < 3) s_base[threadIdx.x] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int chunk = 0; chunk < N; chunk += blockDim.x) {
+    const int i = chunk + threadIdx.x;
+    int f[3] = {0, 0, 0};
+    if (i < N) {
+      const bool p = sc.prot[i];
+      const int r = sc.rank[i];
+      f[0] = p || (r < n_keep_other);
+      f[1] = !p && r < n_keep_other;
+      f[2] = !p && r >= n_keep_other && r < n_keep_other + n_merge;
+    }
+    int x[3];
+    for (int q = 0; q < 3; ++q) {
+      x[q] = f[q];
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x[q], o);
+        if (lane >= o) x[q] += y;
+      }
+      if (lane == 31) s_warp[q][warp] = x[q];
+    }
+    __syncthreads();
+    if (warp == 0) {
+      for (int q = 0; q < 3; ++q) {
+        int w = lane < nw ? s_warp[q][lane] : 0;
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, w, o);
+          if (lane >= o) w += y;
+        }
+        s_warp[q][lane] = w;
+      }
+    }
+    __syncthreads();
+    int* lists[3] = {sc.keep, sc.elig, sc.merge};
+    for (int q = 0; q < 3; ++q) {
+      if (f[q]) lists[q][s_base[q] + (warp > 0 ? s_warp[q][warp - 1] : 0) + x[q] - 1] = i;
+    }
+    __syncthreads();
+    if (threadIdx.x < 3) s_base[threadIdx.x] += s_warp[threadIdx.x][nw - 1];
+    __syncthreads();
+  }
+  if (threadIdx.x < 3) sc.counts[1 + threadIdx.x] = s_base[threadIdx.x];
+}
+
+// ------------------------------------------------------------------ merge targets
+// Full H*D keys of listed tokens as fp32 (bf16 values, exact) and their fp64 norms.
+__global__ void gather_keys_kernel(const int32_t* __restrict__ list, const int32_t* __restrict__ count, int cap,
+                                   const int32_t* __restrict__ slot, const __nv_bfloat16* __restrict__ k_pool,
+                                   int H, int P, int D, float* __restrict__ out, double* __restrict__ norms) {
+  const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n = min(*count, cap);
+  if (w >= n) return;
+  const int pos = list[w];
+  const long long k = slot[pos];
+  const long long phys = k / P, s = k % P;
+  const int HD = H * D;
+  double acc = 0.0;
+  for (int c = lane; c < HD; c += 32) {
+    const int h = c / D, d = c % D;
+    const float x = __bfloat162float(k_pool[((phys * H + h) * P + s) * D + d]);
+    out[static_cast<long long>(w) * HD + c] = x;
+    acc = fma(static_cast<double>(x), static_cast<double>(x), acc);
+  }
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) norms[w] = sqrt(acc);
+}
+
+// Cosine of every (source, eligible target) pair in fp64 (dot products accumulated in
+// ascending dimension order); each CTA reduces its 64x64 tile to the best target per
+// source (largest cosine, lowest target index on ties).
+__global__ void __launch_bounds__(256) cos_tile_kernel(const float* __restrict__ ks, const double* __restrict__ ns,
+                                                        const float* __restrict__ ke, const double* __restrict__ ne,
+                                                        const int32_t* __restrict__ counts, int cap_src, int cap_elig,
+                                                        int HD, double* __restrict__ best_v,
+                                                        int32_t* __restrict__ best_j, int tiles) {
+  __shared__ float a_sm[kCosK][kCosTile + 1];
+  __shared__ float b_sm[kCosK][kCosTile + 1];
+  __shared__ double red_v[kCosTile][16];
+  __shared__ int red_j[kCosTile][16];
+  const int n_src = min(counts[3], cap_src);
+  const int n_elig = min(counts[2], cap_elig);
+  const int s0 = blockIdx.y * kCosTile, e0 = blockIdx.x * kCosTile;
+  if (s0 >= n_src || e0 >= n_elig) return;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;   // 16 x 16 threads, 4 x 4 each
+  double acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+  for (int k0 = 0; k0 < HD; k0 += kCosK) {
+    for (int idx = threadIdx.x; idx < kCosK * kCosTile; idx += blockDim.x) {
+      const int r = idx / kCosK, c = idx % kCosK;
+      const int si = s0 + r, ei = e0 + r;
+      a_sm[c][r] = si < n_src ? ks[static_cast<long long>(si) * HD + k0 + c] : 0.f;
+      b_sm[c][r] = ei < n_elig ? ke[static_cast<long long>(ei) * HD + k0 + c] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int c = 0; c < kCosK; ++c) {
+      double av[4], bv[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) av[a] = a_sm[c][ty * 4 + a];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) bv[b] = b_sm[c][tx * 4 + b];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = fma(av[a], bv[b], acc[a][b]);
+    }
+    __syncthreads();
+  }
+  // per source row: best over this thread's 4 targets, then over the 16 threads of the row
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int si = s0 + ty * 4 + a;
+    double bv = -INFINITY;
+    int bj = 0x7fffffff;
+    if (si < n_src) {
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int ei = e0 + tx * 4 + b;
+        if (ei < n_elig) {
+          const double cv = acc[a][b] / (ne[ei] * ns[si]);
+          if (cv > bv) {
+            bv = cv;
+            bj = ei;
+          }
+        }
+      }
+    }
+    red_v[ty * 4 + a][tx] = bv;
+    red_j[ty * 4 + a][tx] = bj;
+  }
+  __syncthreads();
+  if (threadIdx.x < kCosTile) {
+    const int r = threadIdx.x;
+    double bv = -INFINITY;
+    int bj = 0x7fffffff;
+    for (int t = 0; t < 16; ++t) {
+      const double v = red_v[r][t];
+      const int j = red_j[r][t];
+      if (v > bv || (v == bv && j < bj)) {
+        bv = v;
+        bj = j;
+      }
+    }
+    const int si = s0 + r;
+    if (si < n_src) {
+      best_v[static_cast<long long>(si) * tiles + blockIdx.x] = bv;
+      best_j[static_cast<long long>(si) * tiles + blockIdx.x] = bj;
+    }
+  }
+}
+
+__global__ void argmax_reduce_kernel(const double* __restrict__ best_v, const int32_t* __restrict__ best_j,
+                                     const int32_t* __restrict__ counts, int cap_src, int cap_elig, int tiles,
+                                     int32_t* __restrict__ target) {
+  const int si = blockIdx.x * blockDim.x + threadIdx.x;
+  const int n_src = min(counts[3], cap_src);
+  const int n_elig = min(counts[2], cap_elig);
+  if (si >= n_src) return;
+  const int nt = (n_elig + kCosTile - 1) / kCosTile;
+  double bv = -INFINITY;
+  int bj = 0;
+  for (int t = 0; t < nt; ++t) {
+    const double v = best_v[static_cast<long long>(si) * tiles + t];
+    const int j = best_j[static_cast<long long>(si) * tiles + t];
+    if (v > bv || (v == bv && j < bj)) {
+      bv = v;
+      bj = j;
+    }
+  }
+  target[si] = bj;
+}
+
+// Merge sources sorted by (target, source): rank by counting.
+__global__ void merge_order_kernel(const int32_t* __restrict__ target, const int32_t* __restrict__ counts, int cap,
+                                   int32_t* __restrict__ order) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int n = min(counts[3], cap);
+  if (i >= n) return;
+  const long long ki = (static_cast<long long>(target[i]) << 32) | i;
+  int r = 0;
+  for (int j = 0; j < n; ++j) r += ((static_cast<long long>(target[j]) << 32) | j) < ki;
+  order[r] = i;
+}
+
+// For every eligible target with at least one source: acc = c_j x_j, then acc += c_m x_m
+// for its sources in ascending id, all in fp64; x_j = bf16(acc / sum of counts), for
+// every dimension of K and V; the count becomes the sum. Sources are read before any
+// target is written because no token is both.
+__global__ void merge_apply_kernel(Scratch sc, int cap_src, int cap_elig, __nv_bfloat16* k_pool,
+                                   __nv_bfloat16* v_pool, int H, int P, int D) {
+  const int e = blockIdx.x;
+  const int n_src = min(sc.counts[3], cap_src);
+  const int n_elig = min(sc.counts[2], cap_elig);
+  if (e >= n_elig) return;
+  // binary search the sorted (target, source) order for target e
+  int lo = 0, hi = n_src;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (sc.target[sc.order[mid]] < e) lo = mid + 1; else hi = mid;
+  }
+  const int begin = lo;
+  hi = n_src;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (sc.target[sc.order[mid]] <= e) lo = mid + 1; else hi = mid;
+  }
+  const int end = lo;
+  if (begin == end) return;
+  const int jpos = sc.elig[e];
+  const long long kj = sc.slot[jpos];
+  const int cj = sc.cnt[jpos];
+  int tot = cj;
+  for (int q = begin; q < end; ++q) tot += sc.cnt[sc.merge[sc.order[q]]];
+  const int HD = H * D;
+  for (int c = threadIdx.x; c < 2 * HD; c += blockDim.x) {
+    __nv_bfloat16* pool = c < HD ? k_pool : v_pool;
+    const int cc = c < HD ? c : c - HD;
+    const int h = cc / D, d = cc % D;
+    auto addr = [&](long long k) { return ((k / P * H + h) * P + k % P) * D + d; };
+    double acc = __dmul_rn(static_cast<double>(cj), static_cast<double>(__bfloat162float(pool[addr(kj)])));
+    for (int q = begin; q < end; ++q) {
+      const int mpos = sc.merge[sc.order[q]];
+      const double xm = static_cast<double>(__bfloat162float(pool[addr(sc.slot[mpos])]));
+      acc = __dadd_rn(acc, __dmul_rn(static_cast<double>(sc.cnt[mpos]), xm));
+    }
+    pool[addr(kj)] = f64_to_bf16_rne(__ddiv_rn(acc, static_cast<double>(tot)));
+  }
+  if (threadIdx.x == 0) sc.cnt[jpos] = tot;
+}
+
+__global__ void record_merges_kernel(Scratch sc, int cap_src, int64_t* last_src, int64_t* last_dst) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int n = min(sc.counts[3], cap_src);
+  if (i >= n) return;
+  last_src[i] = sc.ids[sc.merge[i]];
+  last_dst[i] = sc.ids[sc.elig[sc.target[i]]];
+}
+
+// Rewrite kept tokens, in position (= id) order, into the freshly allocated pages:
+// K, V (one warp per token, 16-byte rows) and the metadata; tail slots are zeroed.
+__global__ void compact_kernel(Scratch sc, int cap_keep, const Entry* __restrict__ new_pages, int n_new_pages,
+                               __nv_bfloat16* k_pool, __nv_bfloat16* v_pool, int64_t* tok_id, int32_t* tok_cnt,
+                               float* tok_shat, int H, int P, int D) {
+  const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_keep = min(sc.counts[1], cap_keep);
+  if (w >= n_new_pages * P) return;
+  const long long nphys = new_pages[w / P].x;
+  const int ns = w % P;
+  const long long nk = nphys * P + ns;
+  const int chunks = D / 8;   // 16-byte chunks per head row
+  if (w < n_keep) {
+    const int pos = sc.keep[w];
+    const long long ok = sc.slot[pos];
+    const long long ophys = ok / P, os = ok % P;
+    for (int c = lane; c < H * chunks; c += 32) {
+      const int h = c / chunks, q = c % chunks;
+      const long long src = ((ophys * H + h) * P + os) * D + q * 8;
+      const long long dst = ((nphys * H + h) * P + ns) * D + q * 8;
+      *reinterpret_cast<uint4*>(k_pool + dst) = *reinterpret_cast<const uint4*>(k_pool + src);
+      *reinterpret_cast<uint4*>(v_pool + dst) = *reinterpret_cast<const uint4*>(v_pool + src);
+    }
+    if (lane == 0) {
+      tok_id[nk] = sc.ids[pos];
+      tok_cnt[nk] = sc.cnt[pos];
+      tok_shat[nk] = sc.shat[pos];
+    }
+  } else {
+    for (int c = lane; c < H * chunks; c += 32) {
+      const int h = c / chunks, q = c % chunks;
+      const long long dst = ((nphys * H + h) * P + ns) * D + q * 8;
+      *reinterpret_cast<uint4*>(k_pool + dst) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(v_pool + dst) = make_uint4(0, 0, 0, 0);
+    }
+    if (lane == 0) {
+      tok_id[nk] = -1;
+      tok_cnt[nk] = 0;
+      tok_shat[nk] = 0.f;
+    }
+  }
+}
+
+__global__ void check_counts_kernel(const int32_t* counts, int n, int keep, int elig, int merge, int* err) {
+  if (counts[0] != n || counts[1] != keep || counts[2] != elig || counts[3] != merge) latch_error(err, DERR_BOUNDS);
+}
+
+}  // namespace
+
+size_t compress_scratch_bytes(const kvc_config& cfg, int pool_pages) { return carve(cfg, nullptr, nullptr); }
+
+kvc_status init_token_meta(kvc_cache* c, int layer, int first_entry, int n_pages, int frame) {
+  const int P = c->cfg.page_size;
+  const size_t base = static_cast<size_t>(layer) * c->pool_pages * P;
+  const Entry* pages = c->entries + static_cast<size_t>(layer) * c->pool_pages + first_entry;
+  const int n = n_pages * P;
+  meta_init_kernel<<<(n + 255) / 256, 256, 0, c->stream>>>(c->tok_id + base, c->tok_cnt + base, c->tok_shat + base,
+                                                           pages, n_pages, P, c->cfg.tokens_per_frame, frame);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    c->last_error = std::string("token metadata: ") + cudaGetErrorString(e);
+    return KVC_ERR_CUDA;
+  }
+  c->launches++;
+  return KVC_OK;
+}
 
 kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_t* fired) {
-  c->last_error = "kvc_compress: not built yet";
-  return KVC_ERR_UNSUPPORTED;
+  const kvc_config& g = c->cfg;
+  LayerHost& L = c->L[layer];
+  if (L.has_pending || L.frames.empty() || L.frames.back().frame != L.last_frame) {
+    c->last_error = "kvc_compress: call after kvc_attend of the frame, before the next append";
+    return KVC_ERR_STATE;
+  }
+  const int t = L.last_frame;
+  if (L.scored_frame == t) {
+    c->last_error = "kvc_compress: this layer's frame was already scored";
+    return KVC_ERR_STATE;
+  }
+  // rank history of the current frame: layers must come in ascending order
+  if (c->hist_frame != t) {
+    c->hist_frame = t;
+    c->hist_next_layer = 0;
+    c->hist_layers.clear();
+  }
+  if (layer < c->hist_next_layer) {
+    c->last_error = "kvc_compress: layers of a frame must be scored in ascending order";
+    return KVC_ERR_STATE;
+  }
+  Scratch sc;
+  carve(g, static_cast<uint8_t*>(c->cmp_scratch), &sc);
+  const Caps cp = caps_of(g);
+  const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads, D = g.head_dim;
+  const int RW = g.rank_window;
+  const size_t lay_slots = static_cast<size_t>(layer) * c->pool_pages * P;
+  Entry* E = c->entries + static_cast<size_t>(layer) * c->pool_pages;
+  cudaStream_t s = c->stream;
+  cudaError_t e = cudaSuccess;
+  auto ok = [&]() {
+    cudaError_t r = cudaGetLastError();
+    if (r != cudaSuccess && e == cudaSuccess) e = r;
+    c->launches++;
+  };
+
+  // ---- scoring of the frame just committed
+  c->hist_layers.push_back(layer);
+  uint32_t mask = 0;
+  int n_win = 0;
+  for (int l : c->hist_layers)
+    if (l > layer - RW && l <= layer) {
+      mask |= 1u << (l % RW);
+      ++n_win;
+    }
+  residual_norm_kernel<<<(T + 127) / 128, 128, 0, s>>>(residual, T, g.residual_dim, sc.s_raw);
+  ok();
+  const FrameRec& fr = L.frames.back();
+  clces_kernel<<<1, 1024, T * sizeof(float), s>>>(sc.s_raw, T, c->rank_hist, layer % RW, mask, n_win, g.lambda_,
+                                                  E + fr.first_entry, P, c->tok_shat + lay_slots);
+  ok();
+  c->hist_next_layer = layer + 1;
+  L.scored_frame = t;
+  if (e != cudaSuccess) {
+    c->last_error = std::string("kvc_compress scoring: ") + cudaGetErrorString(e);
+    return KVC_ERR_CUDA;
+  }
+  const int B = g.budget_tokens;
+  if (L.tokens <= B) return KVC_OK;
+
+  // ---- compression
+  const int N = static_cast<int>(L.tokens);
+  const int n_keep = static_cast<int>(cp.n_keep);
+  const int n_merge_cap = B - n_keep;
+  const int n_prot = static_cast<int>(L.protected_tokens);
+  if (n_prot > n_keep) {
+    c->last_error = "kvc_compress: protected tokens exceed the keep tier";
+    return KVC_ERR_BUDGET;
+  }
+  const int n_keep_other = n_keep - n_prot;
+  int n_merge = std::min(n_merge_cap, N - n_keep);
+  if (n_keep_other == 0) n_merge = 0;   // no eligible target: the merge tier is dropped
+  __nv_bfloat16* kp = reinterpret_cast<__nv_bfloat16*>(c->k_pool) + static_cast<size_t>(layer) * c->pool_pages * c->page_elems;
+  __nv_bfloat16* vp = reinterpret_cast<__nv_bfloat16*>(c->v_pool) + static_cast<size_t>(layer) * c->pool_pages * c->page_elems;
+
+  gather_meta_kernel<<<1, 1024, 0, s>>>(E, L.n_entries, P, c->tok_id + lay_slots, c->tok_cnt + lay_slots,
+                                        c->tok_shat + lay_slots, T, g.num_special_tokens, g.protect_first_frame, sc);
+  ok();
+  tier_rank_kernel<<<(N + 255) / 256, 256, 2048 * 5, s>>>(sc, N);
+  ok();
+  tier_lists_kernel<<<1, 1024, 0, s>>>(sc, N, n_keep_other, n_merge);
+  ok();
+  check_counts_kernel<<<1, 1, 0, s>>>(sc.counts, N, n_keep, n_keep_other, n_merge, c->d_err);
+  ok();
+  const int HD = H * D;
+  int64_t* lsrc = sc.last_src + static_cast<size_t>(layer) * cp.n_merge;
+  int64_t* ldst = sc.last_dst + static_cast<size_t>(layer) * cp.n_merge;
+  if (n_merge > 0) {
+    gather_keys_kernel<<<(n_merge * 32 + 255) / 256, 256, 0, s>>>(sc.merge, sc.counts + 3, static_cast<int>(cp.n_merge),
+                                                                   sc.slot, kp, H, P, D, sc.ks, sc.ns);
+    ok();
+    gather_keys_kernel<<<(n_keep_other * 32 + 255) / 256, 256, 0, s>>>(
+        sc.elig, sc.counts + 2, static_cast<int>(cp.n_keep), sc.slot, kp, H, P, D, sc.ke, sc.ne);
+    ok();
+    dim3 grid((n_keep_other + kCosTile - 1) / kCosTile, (n_merge + kCosTile - 1) / kCosTile);
+    cos_tile_kernel<<<grid, 256, 0, s>>>(sc.ks, sc.ns, sc.ke, sc.ne, sc.counts, static_cast<int>(cp.n_merge),
+                                         static_cast<int>(cp.n_keep), HD, sc.best_v, sc.best_j,
+                                         static_cast<int>(cp.tiles));
+    ok();
+    argmax_reduce_kernel<<<(n_merge + 255) / 256, 256, 0, s>>>(sc.best_v, sc.best_j, sc.counts,
+                                                                static_cast<int>(cp.n_merge),
+                                                                static_cast<int>(cp.n_keep),
+                                                                static_cast<int>(cp.tiles), sc.target);
+    ok();
+    merge_order_kernel<<<(n_merge + 255) / 256, 256, 0, s>>>(sc.target, sc.counts, static_cast<int>(cp.n_merge),
+                                                              sc.order);
+    ok();
+    merge_apply_kernel<<<n_keep_other, 256, 0, s>>>(sc, static_cast<int>(cp.n_merge), static_cast<int>(cp.n_keep),
+                                                    kp, vp, H, P, D);
+    ok();
+    record_merges_kernel<<<(n_merge + 255) / 256, 256, 0, s>>>(sc, static_cast<int>(cp.n_merge), lsrc, ldst);
+    ok();
+  }
+  // compaction into the lowest free pages, then release every old page
+  const int n_old = L.n_entries;
+  const int n_new = (n_keep + P - 1) / P;
+  if (n_old + n_new > c->pool_pages) {
+    c->last_error = "kvc_compress: page pool too small for compaction";
+    return KVC_ERR_STATE;
+  }
+  e = e != cudaSuccess ? e : launch_mgr_alloc(s, E, c->bitmap + static_cast<size_t>(layer) * c->bitmap_words,
+                                              c->bitmap_words, c->pool_pages, n_old, n_new, -1, P,
+                                              n_keep - (n_new - 1) * P, c->d_err);
+  c->launches++;
+  compact_kernel<<<(n_new * P * 32 + 255) / 256, 256, 0, s>>>(sc, static_cast<int>(cp.n_keep), E + n_old, n_new, kp, vp,
+                                                              c->tok_id + lay_slots, c->tok_cnt + lay_slots,
+                                                              c->tok_shat + lay_slots, H, P, D);
+  ok();
+  e = e != cudaSuccess ? e : launch_mgr_remove(s, E, c->bitmap + static_cast<size_t>(layer) * c->bitmap_words,
+                                               n_old + n_new, 0, n_old, c->d_err);
+  c->launches++;
+  if (e != cudaSuccess) {
+    c->last_error = std::string("kvc_compress: ") + cudaGetErrorString(e);
+    return KVC_ERR_CUDA;
+  }
+  L.n_entries = n_new;
+  L.frames.clear();
+  L.block_entries = n_new;
+  L.block_tokens = n_keep;
+  L.tokens = n_keep;
+  L.compressions++;
+  L.last_merge_n = n_merge;
+  L.high_water = std::max<int64_t>(L.high_water, n_old + n_new);
+  if (fired) *fired = 1;
+  return KVC_OK;
 }
 
 }  // namespace kvc
@@ -19,5 +754,28 @@ extern "C" kvc_status kvc_last_merge(kvc_cache* c, int32_t layer, int64_t* src_h
                                      int32_t capacity, int32_t* n_out) {
   if (!c) return KVC_ERR_ARG;
   if (n_out) *n_out = 0;
+  if (layer < 0 || layer >= c->cfg.num_layers) {
+    c->last_error = "kvc_last_merge: bad layer";
+    return KVC_ERR_ARG;
+  }
+  if (c->cfg.budget_tokens <= 0) {
+    c->last_error = "kvc_last_merge: budget_tokens is 0";
+    return KVC_ERR_ARG;
+  }
+  cudaError_t e = cudaStreamSynchronize(c->stream);
+  if (e != cudaSuccess) {
+    c->last_error = cudaGetErrorString(e);
+    return KVC_ERR_CUDA;
+  }
+  kvc::Scratch sc;
+  kvc::carve(c->cfg, static_cast<uint8_t*>(c->cmp_scratch), &sc);
+  const kvc::Caps cp = kvc::caps_of(c->cfg);
+  const int n = c->L[layer].last_merge_n;
+  const int m = std::min(n, capacity);
+  if (m > 0) {
+    if (src_host) cudaMemcpy(src_host, sc.last_src + static_cast<size_t>(layer) * cp.n_merge, m * 8, cudaMemcpyDeviceToHost);
+    if (dst_host) cudaMemcpy(dst_host, sc.last_dst + static_cast<size_t>(layer) * cp.n_merge, m * 8, cudaMemcpyDeviceToHost);
+  }
+  if (n_out) *n_out = n;
   return KVC_OK;
 }

@@ -84,6 +84,7 @@ struct Cache {
   int32_t* rank_hist = nullptr;
   int32_t hist_frame = -1;
   int32_t hist_next_layer = 0;
+  std::vector<int> hist_layers;     // layers scored so far in the current frame
   int64_t launches = 0;             // kernels launched by this cache
 };
 
