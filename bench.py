@@ -40,6 +40,12 @@ PROFILE_ATTN = os.path.join(ROOT, "profiles", "attn_tc_kernel_vggt_518x378.md")
 ATTN_SRC = os.path.join(ROOT, "transformer_kv_cache_b200", "csrc", "kvc_attn_tc.cu")
 
 
+def log(msg: str):
+    """Progress on stderr (the result line goes to stdout)."""
+    sys.stderr.write(f"[bench {time.strftime('%H:%M:%S')}] {msg}\n")
+    sys.stderr.flush()
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -252,9 +258,12 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
+    log(f"rank {rank}/{world}: generating {n_frames} frames")
     with torch.cuda.stream(stream):
         st = FrameStream(wl, seed=1000 + rank, device=dev)
         frames = [st.frame(0, t) for t in range(n_frames)]
+        torch.cuda.synchronize()
+        log("frames ready; filling the cache")
         out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
         h = kvc.kvc_create(kvc.config_from_workload(wl, kv_splits=args.kv_splits), stream)
         for t in range(fill + warm):
@@ -262,6 +271,7 @@ def run_ours(args):
             kvc.kvc_append_frame(h, 0, t, k, v, True)
             kvc.kvc_attend(h, 0, q, out)
         _, info0 = kvc.kvc_page_table(h, 0)
+        log(f"cache filled ({info0['pages_used']} pages); timing {steps} steps")
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
@@ -279,6 +289,7 @@ def run_ours(args):
             stream.synchronize()
         barrier()
         elapsed_ms = e0.elapsed_time(e1)
+        log(f"timed region {elapsed_ms:.2f} ms")
         _, info1 = kvc.kvc_page_table(h, 0)
         append_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(steps))
         attend_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(steps))
@@ -293,6 +304,7 @@ def run_ours(args):
     # end to end through the public API from pinned host buffers
     e2e = None
     if args.e2e_steps > 0:
+        log("end-to-end leg")
         kvc.kvc_reset(h)
         n_e2e = min(args.e2e_steps, steps)
         with torch.cuda.stream(stream):
@@ -352,6 +364,7 @@ def run_ours(args):
         if e2e:
             line["e2e"] = e2e
         if world == 1 and not args.no_cpu_baseline:
+            log("cpu baseline (oracle sample)")
             per_frame, r, wall = oracle_sample(wl, 24, 16, time_budget_s=25.0)
             v = 1.0 / statistics.mean(per_frame)
             line["cpu_baseline"] = {
@@ -367,6 +380,9 @@ def run_ours(args):
 
 def main():
     args = parse()
+    if os.environ.get("KVC_BENCH_WATCHDOG"):
+        import faulthandler
+        faulthandler.dump_traceback_later(float(os.environ["KVC_BENCH_WATCHDOG"]), exit=False)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -25,13 +25,24 @@ def sample_rows(T: int, n: int = 64, seed: int = 0) -> np.ndarray:
     return np.array(sorted(set(fixed + rest)))
 
 
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Half the bf16 spacing at |x| (the largest error of rounding x to bf16)."""
+    _, e = np.frexp(np.abs(x))                 # |x| in [2^(e-1), 2^e): spacing 2^(e-8)
+    return np.where(x == 0, 0.0, np.ldexp(1.0, np.maximum(e - 9, -134)))
+
+
 def compare_out(got: np.ndarray, ref: np.ndarray, io_dtype: str, what: str = ""):
+    """fp32 outputs: max-abs <= 1e-4. bf16 outputs: mean-abs <= 2e-3, and max-abs <= 2e-2
+    for the error beyond the rounding of the exact value to the bf16 output format
+    (half a bf16 ulp, which alone exceeds 2e-2 once |O| >= 8)."""
     err = np.abs(got - ref)
     if io_dtype == "f32":
         assert err.max() <= F32_MAX_ABS, f"{what}: max abs {err.max():.3e} > {F32_MAX_ABS}"
-    else:
-        assert err.max() <= BF16_MAX_ABS, f"{what}: max abs {err.max():.3e} > {BF16_MAX_ABS}"
-        assert err.mean() <= BF16_MEAN_ABS, f"{what}: mean abs {err.mean():.3e} > {BF16_MEAN_ABS}"
+        return float(err.max()), float(err.mean())
+    beyond = err - bf16_half_ulp(ref)
+    assert beyond.max() <= BF16_MAX_ABS, \
+        f"{what}: max abs {err.max():.3e} ({beyond.max():.3e} beyond bf16 output rounding) > {BF16_MAX_ABS}"
+    assert err.mean() <= BF16_MEAN_ABS, f"{what}: mean abs {err.mean():.3e} > {BF16_MEAN_ABS}"
     return float(err.max()), float(err.mean())
 
 
