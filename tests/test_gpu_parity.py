@@ -211,3 +211,29 @@ def test_allocation_failure_is_reported_without_leak(kvc):
     assert torch.cuda.mem_get_info()[0] == free0
     h = kvc.kvc_create(kvc.config_from_workload(wl))
     kvc.kvc_destroy(h)
+
+
+def test_rescale_in_some_rows_of_a_warp(kvc):
+    """Rows whose running max jumps by more than 2^8 in the last KV tile rescale O while
+    most rows of their warp do not; the warp must stay converged and the result exact.
+    The last frame plants keys k[200] = 6 q[5] and k[230] = 6 q[70] (per head): rows 5
+    and 70 then see logits near 6|q|^2/8 ~ 48 only in the final tile."""
+    wl = WORKLOADS["vggt_518x378"].replace(tokens_per_frame=256, num_heads=2, window_frames=6, scale_frames=1)
+    dev = torch.device("cuda")
+    h = kvc.kvc_create(kvc.config_from_workload(wl, kv_splits=1))
+    orc = StreamOracle(OracleConfig.from_workload(wl))
+    g = torch.Generator(device=dev).manual_seed(7)
+    o = torch.empty((256, 2, 64), dtype=torch.bfloat16, device=dev)
+    for t in range(5):
+        q, k, v = (torch.randn((256, 2, 64), generator=g, device=dev) for _ in range(3))
+        if t == 4:
+            k[200] = 6.0 * q[5]
+            k[230] = 6.0 * q[70]
+        q, k, v = (x.to(torch.bfloat16) for x in (q, k, v))
+        kvc.kvc_append_frame(h, 0, t, k, v, True)
+        kvc.kvc_attend(h, 0, q, o)
+        orc.append(0, t, np64(k), np64(v), True)
+        ref = orc.attend(0, np64(q))
+        torch.cuda.synchronize()
+        compare_out(np64(o), ref, "bf16", f"frame {t}")
+    kvc.kvc_destroy(h)

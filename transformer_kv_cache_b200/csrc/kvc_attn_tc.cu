@@ -42,6 +42,7 @@ constexpr int kThreads = 192;
 constexpr int kTmemCols = 256;
 constexpr int kColS = 0, kColP = 128, kColO = 192;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kPolyCols = 32;                 // of the 128 columns, exponentiated on the FMA pipe
 constexpr size_t kSmemBytes = 1024 + kQBytes + 2 * kStages * kTileBytes + 256;
 }  // namespace tc
 
@@ -66,6 +67,54 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ---- packed fp32 pairs (sm_100a f32x2 arithmetic) and a 3-input max
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void up2(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x on the FMA pipe for a pair, x <= 8 (lazy rescaling bounds the exponent): x is
+// split as n + f with n = round(x) (adding and subtracting 1.5 * 2^23) and |f| <= 1/2;
+// 2^f comes from a degree-3 polynomial whose coefficients were fitted for this kernel
+// (relative minimax on [-1/2, 1/2], max relative error 7.6e-5, far below the 2^-9
+// rounding of P to bf16); 2^n is applied by adding n to the exponent field. Inputs
+// below -125 are clamped so the result stays a normal number (2^-125 ~ 0 for P).
+__device__ __forceinline__ void exp2_poly_pair(float& x0, float& x1) {
+  constexpr float kC0 = 0.9999281764030457f, kC1 = 0.6932609677314758f, kC2 = 0.2426096349954605f,
+                  kC3 = 0.055170949548482895f, kMagic = 12582912.0f;
+  const uint64_t x = pk2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = add2(x, pk2(kMagic, kMagic));
+  const uint64_t n = add2(t, pk2(-kMagic, -kMagic));
+  const uint64_t f = fma2(n, pk2(-1.f, -1.f), x);
+  uint64_t q = fma2(pk2(kC3, kC3), f, pk2(kC2, kC2));
+  q = fma2(q, f, pk2(kC1, kC1));
+  q = fma2(q, f, pk2(kC0, kC0));
+  float q0, q1, t0, t1;
+  up2(q, q0, q1);
+  up2(t, t0, t1);
+  x0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  x1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 // Wait without the abort shortcut, used only to drain a CTA's own in-flight work.
@@ -234,7 +283,8 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
       float m = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < n_tiles; ++j) {
-        if (!mbar_wait_bounded(s_full, j & 1, abort_flag, p.err)) {
+        // tcgen05.ld/st are .sync.aligned: every branch around them is kept warp-uniform
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_full, j & 1, abort_flag, p.err))) {
           ok = false;
           break;
         }
@@ -265,7 +315,8 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
         }
         float mx = -INFINITY;
 #pragma unroll
-        for (int cc = 0; cc < kBN; ++cc) mx = fmaxf(mx, __uint_as_float(s[cc / 32][cc % 32]));
+        for (int cc = 0; cc < kBN; cc += 2)
+          mx = max3(mx, __uint_as_float(s[cc / 32][cc % 32]), __uint_as_float(s[cc / 32][cc % 32 + 1]));
         const float mx_s = mx * c;
         float m_new = m;
         bool rescale = false;
@@ -275,23 +326,51 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           m_new = mx_s;
           rescale = true;
         }
-        float rs = 0.f;
+        // P = 2^(s*c - m): pairs scaled with one packed FMA; the first kBN - kPolyCols
+        // columns use the MUFU ex2, the last kPolyCols the FMA-pipe polynomial
+        const uint64_t c2 = pk2(c, c), nm2 = pk2(-m_new, -m_new);
 #pragma unroll
-        for (int cc = 0; cc < kBN; ++cc) {
-          const float pv = ex2(fmaf(__uint_as_float(s[cc / 32][cc % 32]), c, -m_new));
-          rs += pv;
-          s[cc / 32][cc % 32] = __float_as_uint(pv);
+        for (int cc = 0; cc < kBN; cc += 2) {
+          float x0, x1;
+          up2(fma2(pk2(__uint_as_float(s[cc / 32][cc % 32]), __uint_as_float(s[cc / 32][cc % 32 + 1])), c2, nm2),
+              x0, x1);
+          if (cc >= kBN - kPolyCols) {
+            exp2_poly_pair(x0, x1);
+          } else {
+            x0 = ex2(x0);
+            x1 = ex2(x1);
+          }
+          s[cc / 32][cc % 32] = __float_as_uint(x0);
+          s[cc / 32][cc % 32 + 1] = __float_as_uint(x1);
         }
+        if (need_mask) {
+          // the polynomial maps -inf to 2^-125, not 0: clear masked columns explicitly
+#pragma unroll
+          for (int cc = kBN - kPolyCols; cc < kBN; ++cc)
+            if ((cc % P) >= vcnt[cc / P]) s[cc / 32][cc % 32] = 0u;
+        }
+        uint64_t acc0 = pk2(0.f, 0.f), acc1 = pk2(0.f, 0.f);
+#pragma unroll
+        for (int cc = 0; cc < kBN; cc += 4) {
+          acc0 = add2(acc0, pk2(__uint_as_float(s[cc / 32][cc % 32]), __uint_as_float(s[cc / 32][cc % 32 + 1])));
+          acc1 = add2(acc1,
+                      pk2(__uint_as_float(s[cc / 32][cc % 32 + 2]), __uint_as_float(s[cc / 32][cc % 32 + 3])));
+        }
+        float a0, a1, b0, b1;
+        up2(acc0, a0, a1);
+        up2(acc1, b0, b1);
+        const float rs = (a0 + a1) + (b0 + b1);
         if (j > 0) {
-          if (!mbar_wait_bounded(pv_done, (j - 1) & 1, abort_flag, p.err)) {
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(pv_done, (j - 1) & 1, abort_flag, p.err))) {
             ok = false;
             break;
           }
           tc_fence_after();
         }
-        if (rescale) {
-          // O row *= 2^(m_old - m_new), 16 columns at a time to keep registers for P
-          const float corr = ex2(m - m_new);
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O row *= 2^(m_old - m_new), 16 columns at a time to keep registers for P; the
+          // whole warp takes this branch, rows that keep their reference max scale by 1
+          const float corr = rescale ? ex2(m - m_new) : 1.0f;
           l *= corr;
 #pragma unroll
           for (int q4 = 0; q4 < kHD / 16; ++q4) {
@@ -320,7 +399,7 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
       }
-      if (ok && mbar_wait_bounded(pv_done, (n_tiles - 1) & 1, abort_flag, p.err)) {
+      if (__all_sync(0xffffffffu, ok && mbar_wait_bounded(pv_done, (n_tiles - 1) & 1, abort_flag, p.err))) {
         tc_fence_after();
         uint32_t o0[32], o1[32];
         tmem_ld32(tO, o0);
