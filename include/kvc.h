@@ -227,6 +227,34 @@ KVC_API const char* kvc_status_string(kvc_status s);
 /* KVC_VERSION of the built library. */
 KVC_API int32_t kvc_version(void);
 
+/* Frame attention for callers that cannot allocate device memory: code running
+ * inside a CUDA-graph capture it does not own, embedded runtimes without a device
+ * allocator, plug-ins whose host process forbids allocation after start-up. The pages
+ * have no counterpart to this call; it exists only for such callers.
+ *
+ * Computes the same attention as kvc_attend, with the same tensor-core kernel, over
+ * caller-owned buffers: q_dev and o_dev [tokens, num_heads, 64] bf16; k_pool_dev and
+ * v_pool_dev [pool_pages][num_heads][16][64] bf16 (the layout kvc_append_frame writes);
+ * page_table_dev int32 [n_pages][4] device rows (phys_page, 0, 0, valid_tokens) listing
+ * the pages to attend in any order, each with 1..16 valid leading slots (masked slots
+ * must hold finite values). head_dim must be 64 and page_size 16; kv_splits >= 1 splits
+ * the KV sequence across CTAs. Enqueued on `stream`; nothing is allocated or freed.
+ *
+ * Split partials live in one file-scope device array of 480 partial tiles (128 query
+ * rows x 64 dims fp32 + one log-sum-exp per row, 15.97 MB) that every GPU loading the
+ * library holds until the process exits. Calls with (ceil(tokens/128) * num_heads *
+ * effective splits) > 480 and kv_splits > 1 are rejected with KVC_ERR_ARG. The first
+ * call on a device looks the array's device address up (cudaGetSymbolAddress); make
+ * that first call before any stream capture. All calls share the array: calls whose
+ * kernels overlap on the GPU race on it. Nothing in it needs to start at zero. A wait in
+ * the kernel that gives up (bounded) ends the kernel without an error report here.
+ * Errors: KVC_ERR_ARG (shapes, alignment, sizes beyond the array), KVC_ERR_CUDA. */
+KVC_API kvc_status kvc_attend_paged_noalloc(const void* q_dev, void* o_dev, const void* k_pool_dev,
+                                            const void* v_pool_dev, int64_t pool_pages,
+                                            const int32_t* page_table_dev, int32_t n_pages, int32_t tokens,
+                                            int32_t num_heads, int32_t head_dim, int32_t page_size,
+                                            float softmax_scale, int32_t kv_splits, void* stream);
+
 /* Test hooks for failure handling, tested without any GPU fault:
  *   kvc_debug_fail_allocs(n): the n-th next device allocation inside
  *     kvc_create reports failure (n = 0 disables), which must surface as

@@ -27,7 +27,7 @@ STATUS = ["KVC_OK", "KVC_ERR_ARG", "KVC_ERR_OOM", "KVC_ERR_CUDA", "KVC_ERR_STATE
 EXPORTS = ["kvc_create", "kvc_destroy", "kvc_set_stream", "kvc_reset", "kvc_append_frame", "kvc_attend",
            "kvc_compress", "kvc_page_table", "kvc_token_meta", "kvc_last_merge", "kvc_export_pages",
            "kvc_step_host", "kvc_synchronize", "kvc_last_error", "kvc_status_string", "kvc_version",
-           "kvc_debug_fail_allocs", "kvc_debug_bounded_wait"]
+           "kvc_debug_fail_allocs", "kvc_debug_bounded_wait", "kvc_attend_paged_noalloc"]
 
 
 class kvc_config(ctypes.Structure):
@@ -83,6 +83,8 @@ def _load():
         "kvc_version": ([], i32),
         "kvc_debug_fail_allocs": ([i32], i32),
         "kvc_debug_bounded_wait": ([vp, i32], i32),
+        "kvc_attend_paged_noalloc": ([vp, vp, vp, vp, ctypes.c_int64, vp, i32, i32, i32, i32, i32, ctypes.c_float,
+                                      i32, vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -258,6 +260,17 @@ def kvc_debug_fail_allocs(n: int) -> None:
 
 def kvc_debug_bounded_wait(handle, timeout_us: int) -> None:
     _check(handle, _lib.kvc_debug_bounded_wait(handle, timeout_us))
+
+
+def kvc_attend_paged_noalloc(q, o, k_pool, v_pool, pool_pages: int, page_table, n_pages: int, tokens: int,
+                             num_heads: int, head_dim: int, page_size: int, softmax_scale: float,
+                             kv_splits: int = 1, stream=None) -> None:
+    """Attention over caller-owned pools with no device allocation (see include/kvc.h)."""
+    st = _lib.kvc_attend_paged_noalloc(_ptr(q), _ptr(o), _ptr(k_pool), _ptr(v_pool), pool_pages, _ptr(page_table),
+                                       n_pages, tokens, num_heads, head_dim, page_size, softmax_scale, kv_splits,
+                                       _stream(stream))
+    if st != 0:
+        raise KVCError(st, "kvc_attend_paged_noalloc failed")
 
 
 @dataclass
