@@ -236,8 +236,8 @@ KVC_API int32_t kvc_version(void);
  * caller-owned buffers: q_dev and o_dev [tokens, num_heads, 64] bf16; k_pool_dev and
  * v_pool_dev [pool_pages][num_heads][16][64] bf16 (the layout kvc_append_frame writes);
  * page_table_dev int32 [n_pages][4] device rows (phys_page, 0, 0, valid_tokens) listing
- * the pages to attend in any order, each with 1..16 valid leading slots (masked slots
- * must hold finite values). head_dim must be 64 and page_size 16; kv_splits >= 1 splits
+ * the pages to attend in any order, each with 1..16 valid leading slots (slots past
+ * valid_tokens must hold zeros in both K and V, as kvc_append_frame writes them). head_dim must be 64 and page_size 16; kv_splits >= 1 splits
  * the KV sequence across CTAs. Enqueued on `stream`; nothing is allocated or freed.
  *
  * Split partials live in one file-scope device array of 480 partial tiles (128 query

@@ -359,6 +359,7 @@ kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_de
     a.H = H;
     a.P = P;
     a.page_base = static_cast<long long>(layer) * c->pool_pages;
+    a.pool_rows = static_cast<long long>(g.num_layers) * c->pool_pages * H * P;
     a.softmax_scale = g.softmax_scale;
     a.splits = g.kv_splits;
     a.tmap_k = &c->tmap_k[0];

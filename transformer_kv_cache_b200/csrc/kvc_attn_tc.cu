@@ -11,15 +11,24 @@
 //   warp 1 (one lane)   MMA issuer: S = Q K^T (tcgen05.mma kind::f16, M=128, N=128,
 //                       4 K-steps of 16) into TMEM; O += P V with P read from TMEM
 //                       (M=128, N=64, 8 K-steps) and V as an MN-major operand.
-//   warps 2..5          softmax: thread = query row = TMEM lane; S row to registers
-//                       (tcgen05.ld), masking of the partial last page of each frame,
-//                       online max with lazy rescaling (the running reference max only
-//                       moves when the tile max exceeds it by 2^8, which keeps the result
-//                       exact after the final normalisation), P = 2^(s - m) as bf16 back
-//                       into TMEM (tcgen05.st), O rescaled in TMEM when the max moves.
+//   warps 2..9          softmax: two warps per TMEM lane quadrant, thread = query row =
+//                       TMEM lane, each warp of a pair owning 64 of the tile's 128
+//                       columns; S half-row to registers (tcgen05.ld), row max
+//                       exchanged with the partner warp through shared memory, online
+//                       max with lazy
+//                       rescaling (the running reference max only moves when the tile max
+//                       exceeds it by 2^8, which keeps the result exact after the final
+//                       normalisation), P = 2^(s - m) as bf16 back into TMEM (tcgen05.st),
+//                       the warp's 32 O columns rescaled in TMEM when the max moves.
+//
+// Partial pages need no per-column mask: slots past a page's valid count hold K = V = 0
+// (the append and compaction kernels write zeros there, and pages past the end of the
+// list are read out of bounds so TMA fills zeros), so each scores exactly 0, adds nothing
+// to O and exactly 2^-m to the row sum, which is subtracted once per tile.
 //
 // TMEM (256 columns): S [0,128), P [128,192) (bf16 pairs), O [192,256). Two CTAs fit per
-// SM (TMEM 2 x 256 columns, shared memory 2 x ~82 KB), so one CTA's MMAs overlap the
+// SM (TMEM 2 x 256 columns, shared memory 2 x ~85 KB, 96 registers per thread), which puts
+// four softmax warps on every SM sub-partition and lets one CTA's MMAs overlap the
 // other's softmax. The KV sequence can be split across CTAs; partial outputs carry the
 // log2-sum-exp and a combine kernel merges them. Every barrier wait is bounded: on
 // timeout the CTA records KVC_ERR_TIMEOUT in the error word, drains its own copies and
@@ -38,12 +47,13 @@ constexpr int kHD = 64;                       // head dim (one 128-byte swizzle 
 constexpr int kStages = 2;
 constexpr int kTileBytes = kBN * kHD * 2;     // 16 KB
 constexpr int kQBytes = kBM * kHD * 2;        // 16 KB
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;                 // producer, MMA, 8 softmax warps
 constexpr int kTmemCols = 256;
 constexpr int kColS = 0, kColP = 128, kColO = 192;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kPolyCols = 32;                 // of the 128 columns, exponentiated on the FMA pipe
-constexpr size_t kSmemBytes = 1024 + kQBytes + 2 * kStages * kTileBytes + 256;
+constexpr int kPolyCols = 0;                  // of each warp's 64 columns, exponentiated on the FMA pipe
+                                              // (0: measured fastest; the MUFU is not the limit)                 // of each warp's 64 columns, exponentiated on the FMA pipe
+constexpr size_t kSmemBytes = 1024 + kQBytes + 2 * kStages * kTileBytes + 256 + 2 * 2 * kBM * 4;
 }  // namespace tc
 
 struct TcParams {
@@ -51,6 +61,7 @@ struct TcParams {
   int n_pages, T, H;
   int q_tiles, splits, tiles_per_split, total_tiles;
   long long page_base;          // layer * pool_pages: first pool page of the layer
+  int pool_rows;                // rows of the pool tensor maps (a row index past the end reads zeros)
   float scale_log2;
   __nv_bfloat16* out;
   float* part_o;
@@ -69,52 +80,30 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// ---- packed fp32 pairs (sm_100a f32x2 arithmetic) and a 3-input max
-__device__ __forceinline__ uint64_t pk2(float a, float b) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void up2(uint64_t r, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
+// 3-input max (sm_100a)
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
 
-// 2^x on the FMA pipe for a pair, x <= 8 (lazy rescaling bounds the exponent): x is
-// split as n + f with n = round(x) (adding and subtracting 1.5 * 2^23) and |f| <= 1/2;
-// 2^f comes from a degree-3 polynomial whose coefficients were fitted for this kernel
-// (relative minimax on [-1/2, 1/2], max relative error 7.6e-5, far below the 2^-9
-// rounding of P to bf16); 2^n is applied by adding n to the exponent field. Inputs
-// below -125 are clamped so the result stays a normal number (2^-125 ~ 0 for P).
-__device__ __forceinline__ void exp2_poly_pair(float& x0, float& x1) {
+// 2^x on the FMA pipe for x <= 8 (lazy rescaling bounds the exponent): x is split as
+// n + f with n = round(x) (adding and subtracting 1.5 * 2^23) and |f| <= 1/2; 2^f comes
+// from a degree-3 polynomial whose coefficients were fitted for this kernel (relative
+// minimax on [-1/2, 1/2], max relative error 7.6e-5, far below the 2^-9 rounding of P to
+// bf16); 2^n is applied by adding n to the exponent field. Inputs below -125 are clamped
+// so the result stays a normal number. Used for the last kPolyCols columns of a half.
+__device__ __forceinline__ float exp2_poly(float x) {
   constexpr float kC0 = 0.9999281764030457f, kC1 = 0.6932609677314758f, kC2 = 0.2426096349954605f,
                   kC3 = 0.055170949548482895f, kMagic = 12582912.0f;
-  const uint64_t x = pk2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-  const uint64_t t = add2(x, pk2(kMagic, kMagic));
-  const uint64_t n = add2(t, pk2(-kMagic, -kMagic));
-  const uint64_t f = fma2(n, pk2(-1.f, -1.f), x);
-  uint64_t q = fma2(pk2(kC3, kC3), f, pk2(kC2, kC2));
-  q = fma2(q, f, pk2(kC1, kC1));
-  q = fma2(q, f, pk2(kC0, kC0));
-  float q0, q1, t0, t1;
-  up2(q, q0, q1);
-  up2(t, t0, t1);
-  x0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  x1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+  x = fmaxf(x, -125.f);
+  const float t = x + kMagic;
+  const float n = t - kMagic;
+  const float f = x - n;
+  float q = fmaf(kC3, f, kC2);
+  q = fmaf(q, f, kC1);
+  q = fmaf(q, f, kC0);
+  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
 }
 
 // Wait without the abort shortcut, used only to drain a CTA's own in-flight work.
@@ -144,8 +133,10 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
   uint64_t* p_full = s_full + 2;
   uint64_t* pv_done = s_full + 3;
   uint64_t* mma_final = s_full + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
+  uint64_t* xchg = s_full + 5;                // [4] one per TMEM lane quadrant (softmax warp pair)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xchg + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* red = reinterpret_cast<float*>(bars + 32);   // [2 parity][2 halves][128 rows] row values
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x % p.q_tiles;
@@ -164,8 +155,9 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 4);
-    mbar_init(p_full, 4);
+    mbar_init(s_free, 8);
+    mbar_init(p_full, 8);
+    for (int i = 0; i < 4; ++i) mbar_init(&xchg[i], 64);
     mbar_init(pv_done, 1);
     mbar_init(mma_final, 1);
     *abort_flag = 0;
@@ -201,18 +193,19 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           mbar_arrive_expect_tx(&k_full[st], kTileBytes);
 #pragma unroll
           for (int g = 0; g < kPPT; ++g) {
-            int idx = gt * kPPT + g;
-            if (idx >= p.n_pages) idx = gt * kPPT;   // masked; any valid page keeps the data finite
-            const long long phys = p.page_base + __ldg(&p.entries[idx].x);
-            tma_load_2d(kd + g * P * 128, &tmap_k, &k_full[st], 0, static_cast<int>((phys * p.H + h) * P));
+            const int idx = gt * kPPT + g;
+            // pages past the list end are read past the end of the pool: TMA fills zeros
+            const int row = idx < p.n_pages ? static_cast<int>(((p.page_base + __ldg(&p.entries[idx].x)) * p.H + h) * P)
+                                            : p.pool_rows;
+            tma_load_2d(kd + g * P * 128, &tmap_k, &k_full[st], 0, row);
           }
           mbar_arrive_expect_tx(&v_full[st], kTileBytes);
 #pragma unroll
           for (int g = 0; g < kPPT; ++g) {
-            int idx = gt * kPPT + g;
-            if (idx >= p.n_pages) idx = gt * kPPT;
-            const long long phys = p.page_base + __ldg(&p.entries[idx].x);
-            tma_load_2d(vd + g * P * 128, &tmap_v, &v_full[st], 0, static_cast<int>((phys * p.H + h) * P));
+            const int idx = gt * kPPT + g;
+            const int row = idx < p.n_pages ? static_cast<int>(((p.page_base + __ldg(&p.entries[idx].x)) * p.H + h) * P)
+                                            : p.pool_rows;
+            tma_load_2d(vd + g * P * 128, &tmap_v, &v_full[st], 0, row);
           }
           last[st] = j;
         }
@@ -275,48 +268,71 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
       }
     } else {
       // ------------------------------------------------------------------ softmax warps
-      const int wq = warp & 3;                      // TMEM lane quadrant this warp may access
-      const int r = wq * 32 + lane;                 // query row within the tile
+      // Eight warps. Warp w may only access TMEM lane quadrant w % 4 (its 32 query rows);
+      // the two warps sharing a quadrant split each 128-column S tile into halves of 64
+      // and exchange per-row maxima through shared memory (mbarrier xchg[quadrant]).
+      constexpr int kHalf = kBN / 2;
+      constexpr int kPPH = kPPT / 2;               // pages per column half
+      const int wq = warp & 3;
+      const int hf = (warp - 2) >> 2;
+      const int r = wq * 32 + lane;
       const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-      const uint32_t tS = tmem + kColS + lane_off, tP = tmem + kColP + lane_off, tO = tmem + kColO + lane_off;
+      const uint32_t tS = tmem + kColS + hf * kHalf + lane_off;
+      const uint32_t tP = tmem + kColP + hf * (kHalf / 2) + lane_off;
+      const uint32_t tO = tmem + kColO + hf * (kHD / 2) + lane_off;
       const float c = p.scale_log2;
       float m = -INFINITY, l = 0.f;
       bool ok = true;
+      // valid-slot counts of this half's pages of the next KV tile, loaded one tile ahead
+      int vnext[kPPH];
+#pragma unroll
+      for (int g = 0; g < kPPH; ++g) {
+        const int idx = tile0 * kPPT + hf * kPPH + g;
+        vnext[g] = idx < p.n_pages ? __ldg(&p.entries[idx].w) : 0;
+      }
       for (int j = 0; j < n_tiles; ++j) {
+        // invalid slots hold K = V = 0, so they score 0 and add exactly 2^-m to the row
+        // sum and nothing to O: count them and take them out of the sum below
+        int n_masked = 0;
+#pragma unroll
+        for (int g = 0; g < kPPH; ++g) n_masked += P - vnext[g];
+        if (j + 1 < n_tiles) {
+#pragma unroll
+          for (int g = 0; g < kPPH; ++g) {
+            const int idx = (tile0 + j + 1) * kPPT + hf * kPPH + g;
+            vnext[g] = idx < p.n_pages ? __ldg(&p.entries[idx].w) : 0;
+          }
+        }
         // tcgen05.ld/st are .sync.aligned: every branch around them is kept warp-uniform
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_full, j & 1, abort_flag, p.err))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t s[4][32];
+        uint32_t s[2][32];
         tmem_ld32(tS + 0, s[0]);
         tmem_ld32(tS + 32, s[1]);
-        tmem_ld32(tS + 64, s[2]);
-        tmem_ld32(tS + 96, s[3]);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free);
-        // mask the invalid tail slots of partial pages (and pages past the list end)
-        const int gt = tile0 + j;
-        int vcnt[kPPT];
-        bool need_mask = false;
+        float mxa = -INFINITY, mxb = -INFINITY, mxc = -INFINITY, mxd = -INFINITY;
 #pragma unroll
-        for (int g = 0; g < kPPT; ++g) {
-          const int idx = gt * kPPT + g;
-          vcnt[g] = idx < p.n_pages ? __ldg(&p.entries[idx].w) : 0;
-          need_mask |= vcnt[g] < P;
+        for (int cc = 0; cc < kHalf; cc += 8) {
+          mxa = max3(mxa, __uint_as_float(s[cc / 32][cc % 32 + 0]), __uint_as_float(s[cc / 32][cc % 32 + 1]));
+          mxb = max3(mxb, __uint_as_float(s[cc / 32][cc % 32 + 2]), __uint_as_float(s[cc / 32][cc % 32 + 3]));
+          mxc = max3(mxc, __uint_as_float(s[cc / 32][cc % 32 + 4]), __uint_as_float(s[cc / 32][cc % 32 + 5]));
+          mxd = max3(mxd, __uint_as_float(s[cc / 32][cc % 32 + 6]), __uint_as_float(s[cc / 32][cc % 32 + 7]));
         }
-        if (need_mask) {
-#pragma unroll
-          for (int cc = 0; cc < kBN; ++cc)
-            if ((cc % P) >= vcnt[cc / P]) s[cc / 32][cc % 32] = __float_as_uint(-INFINITY);
+        float mx = fmaxf(fmaxf(mxa, mxb), fmaxf(mxc, mxd));
+        // row max of the whole tile: swap halves with the partner warp
+        red[((j & 1) * 2 + hf) * kBM + r] = mx;
+        mbar_arrive(&xchg[wq]);
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&xchg[wq], j & 1, abort_flag, p.err))) {
+          ok = false;
+          break;
         }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int cc = 0; cc < kBN; cc += 2)
-          mx = max3(mx, __uint_as_float(s[cc / 32][cc % 32]), __uint_as_float(s[cc / 32][cc % 32 + 1]));
+        mx = fmaxf(mx, red[((j & 1) * 2 + (1 - hf)) * kBM + r]);
         const float mx_s = mx * c;
         float m_new = m;
         bool rescale = false;
@@ -326,40 +342,34 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           m_new = mx_s;
           rescale = true;
         }
-        // P = 2^(s*c - m): pairs scaled with one packed FMA; the first kBN - kPolyCols
-        // columns use the MUFU ex2, the last kPolyCols the FMA-pipe polynomial
-        const uint64_t c2 = pk2(c, c), nm2 = pk2(-m_new, -m_new);
+        // P = 2^(s*c - m) in scalar fp32: the first kHalf - kPolyCols columns on the MUFU
+        // ex2, the last kPolyCols with the FMA-pipe polynomial; each pair is summed into
+        // four independent accumulators and packed to bf16 right away.
+        const float nm = -m_new;
+        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+        uint32_t pk[kHalf / 2];
 #pragma unroll
-        for (int cc = 0; cc < kBN; cc += 2) {
-          float x0, x1;
-          up2(fma2(pk2(__uint_as_float(s[cc / 32][cc % 32]), __uint_as_float(s[cc / 32][cc % 32 + 1])), c2, nm2),
-              x0, x1);
-          if (cc >= kBN - kPolyCols) {
-            exp2_poly_pair(x0, x1);
+        for (int cc = 0; cc < kHalf; cc += 2) {
+          float x0 = fmaf(__uint_as_float(s[cc / 32][cc % 32]), c, nm);
+          float x1 = fmaf(__uint_as_float(s[cc / 32][cc % 32 + 1]), c, nm);
+          if (cc >= kHalf - kPolyCols) {
+            x0 = exp2_poly(x0);
+            x1 = exp2_poly(x1);
           } else {
             x0 = ex2(x0);
             x1 = ex2(x1);
           }
-          s[cc / 32][cc % 32] = __float_as_uint(x0);
-          s[cc / 32][cc % 32 + 1] = __float_as_uint(x1);
+          if ((cc / 2) & 1) {
+            acc2 += x0;
+            acc3 += x1;
+          } else {
+            acc0 += x0;
+            acc1 += x1;
+          }
+          pk[cc / 2] = pack_bf16(x0, x1);
         }
-        if (need_mask) {
-          // the polynomial maps -inf to 2^-125, not 0: clear masked columns explicitly
-#pragma unroll
-          for (int cc = kBN - kPolyCols; cc < kBN; ++cc)
-            if ((cc % P) >= vcnt[cc / P]) s[cc / 32][cc % 32] = 0u;
-        }
-        uint64_t acc0 = pk2(0.f, 0.f), acc1 = pk2(0.f, 0.f);
-#pragma unroll
-        for (int cc = 0; cc < kBN; cc += 4) {
-          acc0 = add2(acc0, pk2(__uint_as_float(s[cc / 32][cc % 32]), __uint_as_float(s[cc / 32][cc % 32 + 1])));
-          acc1 = add2(acc1,
-                      pk2(__uint_as_float(s[cc / 32][cc % 32 + 2]), __uint_as_float(s[cc / 32][cc % 32 + 3])));
-        }
-        float a0, a1, b0, b1;
-        up2(acc0, a0, a1);
-        up2(acc1, b0, b1);
-        const float rs = (a0 + a1) + (b0 + b1);
+        float rs = (acc0 + acc1) + (acc2 + acc3);
+        if (n_masked) rs -= static_cast<float>(n_masked) * ex2(nm);
         if (j > 0) {
           if (!__all_sync(0xffffffffu, mbar_wait_bounded(pv_done, (j - 1) & 1, abort_flag, p.err))) {
             ok = false;
@@ -368,12 +378,12 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           tc_fence_after();
         }
         if (__any_sync(0xffffffffu, rescale)) {
-          // O row *= 2^(m_old - m_new), 16 columns at a time to keep registers for P; the
-          // whole warp takes this branch, rows that keep their reference max scale by 1
+          // this warp's 32 O columns *= 2^(m_old - m_new); rows that keep their reference
+          // max scale by 1 (the branch is warp-uniform)
           const float corr = rescale ? ex2(m - m_new) : 1.0f;
           l *= corr;
 #pragma unroll
-          for (int q4 = 0; q4 < kHD / 16; ++q4) {
+          for (int q4 = 0; q4 < kHD / 32; ++q4) {
             uint32_t oc[16];
             tmem_ld16(tO + q4 * 16, oc);
             tmem_ld_wait();
@@ -384,32 +394,29 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
         }
         m = m_new;
         l += rs;
-        uint32_t pk0[32], pk1[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          pk0[i] = pack_bf16(__uint_as_float(s[(2 * i) / 32][(2 * i) % 32]),
-                             __uint_as_float(s[(2 * i + 1) / 32][(2 * i + 1) % 32]));
-          pk1[i] = pack_bf16(__uint_as_float(s[(64 + 2 * i) / 32][(64 + 2 * i) % 32]),
-                             __uint_as_float(s[(65 + 2 * i) / 32][(65 + 2 * i) % 32]));
-        }
-        tmem_st32(tP, pk0);
-        tmem_st32(tP + 32, pk1);
+        tmem_st32(tP, pk);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
       }
+      // row sum of the two halves, then the epilogue writes this warp's 32 columns
+      if (ok) {
+        red[((n_tiles & 1) * 2 + hf) * kBM + r] = l;
+        mbar_arrive(&xchg[wq]);
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&xchg[wq], n_tiles & 1, abort_flag, p.err));
+        if (ok) l += red[((n_tiles & 1) * 2 + (1 - hf)) * kBM + r];
+      }
       if (__all_sync(0xffffffffu, ok && mbar_wait_bounded(pv_done, (n_tiles - 1) & 1, abort_flag, p.err))) {
         tc_fence_after();
-        uint32_t o0[32], o1[32];
+        uint32_t o0[32];
         tmem_ld32(tO, o0);
-        tmem_ld32(tO + 32, o1);
         tmem_ld_wait();
         const float inv = 1.f / l;
         const int row = qt * kBM + r;
         if (p.splits == 1) {
           if (row < p.T) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<long long>(row) * p.H + h) * kHD);
+            uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<long long>(row) * p.H + h) * kHD + hf * 32);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               uint4 w;
@@ -419,28 +426,15 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
               w.w = pack_bf16(__uint_as_float(o0[8 * v + 6]) * inv, __uint_as_float(o0[8 * v + 7]) * inv);
               dst[v] = w;
             }
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 w;
-              w.x = pack_bf16(__uint_as_float(o1[8 * v + 0]) * inv, __uint_as_float(o1[8 * v + 1]) * inv);
-              w.y = pack_bf16(__uint_as_float(o1[8 * v + 2]) * inv, __uint_as_float(o1[8 * v + 3]) * inv);
-              w.z = pack_bf16(__uint_as_float(o1[8 * v + 4]) * inv, __uint_as_float(o1[8 * v + 5]) * inv);
-              w.w = pack_bf16(__uint_as_float(o1[8 * v + 6]) * inv, __uint_as_float(o1[8 * v + 7]) * inv);
-              dst[4 + v] = w;
-            }
           }
         } else {
           const long long pi = (static_cast<long long>(h) * p.splits + split) * p.q_tiles + qt;
-          float4* dst = reinterpret_cast<float4*>(p.part_o + (pi * kBM + r) * kHD);
+          float4* dst = reinterpret_cast<float4*>(p.part_o + (pi * kBM + r) * kHD + hf * 32);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
             dst[v] = make_float4(__uint_as_float(o0[4 * v + 0]) * inv, __uint_as_float(o0[4 * v + 1]) * inv,
                                  __uint_as_float(o0[4 * v + 2]) * inv, __uint_as_float(o0[4 * v + 3]) * inv);
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[8 + v] = make_float4(__uint_as_float(o1[4 * v + 0]) * inv, __uint_as_float(o1[4 * v + 1]) * inv,
-                                     __uint_as_float(o1[4 * v + 2]) * inv, __uint_as_float(o1[4 * v + 3]) * inv);
-          p.part_lse[pi * kBM + r] = m + __log2f(l);
+          if (hf == 0) p.part_lse[pi * kBM + r] = m + __log2f(l);
         }
       }
     }
@@ -579,6 +573,7 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   prm.tiles_per_split = tps;
   prm.total_tiles = total_tiles;
   prm.page_base = a.page_base;
+  prm.pool_rows = static_cast<int>(a.pool_rows);
   prm.scale_log2 = static_cast<float>(static_cast<double>(a.softmax_scale) * 1.4426950408889634);
   prm.out = static_cast<__nv_bfloat16*>(a.o);
   prm.part_o = a.part_o;

@@ -7,7 +7,7 @@
 #include <string>
 #include <vector>
 
-#include "../../include/kvc.h"
+#include "kvc.h"
 
 namespace kvc {
 
@@ -123,6 +123,7 @@ struct TcAttnArgs {
   const Entry* entries;
   int n_pages, T, H, P;
   long long page_base;              // first pool page of the layer (layer * pool_pages)
+  long long pool_rows;              // rows (pages x heads x P) of the pool tensor maps
   float softmax_scale;
   int splits;                       // 0: choose automatically
   const CUtensorMap* tmap_k;

@@ -101,6 +101,7 @@ extern "C" kvc_status kvc_attend_paged_noalloc(const void* q_dev, void* o_dev, c
   a.H = num_heads;
   a.P = page_size;
   a.page_base = 0;
+  a.pool_rows = static_cast<long long>(rows);
   a.softmax_scale = softmax_scale;
   a.splits = static_cast<int>(splits);
   a.tmap_k = &tk;
