@@ -3,33 +3,36 @@
 // Computes O[i, h] = sum_j softmax_j(scale * q_i . k_j) v_j for the T queries of the new
 // frame over every valid slot of the layer's page list ("How GCTStream ...",
 // Frame-by-Frame Causal Processing; "InfiniteVGGT" explainer, Causal Attention) without
-// materialising the score matrix, as a flash-attention pipeline built for Blackwell:
+// materialising the score matrix, as a flash-attention pipeline built for Blackwell. Each
+// CTA owns one 128-row query tile of one head and a range of 64-slot KV tiles (4 pages):
 //
-//   warp 0 (one lane)   TMA producer: the CTA's 128x64 query tile once, then per KV tile
-//                       the 128/P pages of K and of V, each page-head block one 2-D box
-//                       into a 128-byte-swizzled stage (ring of kStages stages).
-//   warp 1 (one lane)   MMA issuer: S = Q K^T (tcgen05.mma kind::f16, M=128, N=128,
-//                       4 K-steps of 16) into TMEM; O += P V with P read from TMEM
-//                       (M=128, N=64, 8 K-steps) and V as an MN-major operand.
-//   warps 2..9          softmax: two warps per TMEM lane quadrant, thread = query row =
-//                       TMEM lane, each warp of a pair owning 64 of the tile's 128
-//                       columns; S half-row to registers (tcgen05.ld), row max
-//                       exchanged with the partner warp through shared memory, online
-//                       max with lazy
-//                       rescaling (the running reference max only moves when the tile max
-//                       exceeds it by 2^8, which keeps the result exact after the final
-//                       normalisation), P = 2^(s - m) as bf16 back into TMEM (tcgen05.st),
-//                       the warp's 32 O columns rescaled in TMEM when the max moves.
+//   warp 0 (one lane)   TMA producer: the query tile once, then per KV tile the 4 pages of
+//                       K and of V, each page-head block one 2-D box, into a ring of
+//                       128-byte-swizzled stages. Pages past the end of the list are read
+//                       past the end of the pool, which TMA fills with zeros.
+//   warp 1 (one lane)   MMA issuer: S = Q K^T (tcgen05.mma kind::f16, M=128, N=64) into
+//                       TMEM, then O' += P [V | 1] (M=128, N=80, A = P read from TMEM,
+//                       B = the V tile as an MN-major operand followed by a constant block
+//                       of ones), so accumulator column 64 carries the row sum of P.
+//   warps 2..5          softmax, thread = query row = TMEM lane, 64 columns per tile:
+//                       x = s*c - m with packed f32x2 FMAs, x rounded to bf16 pairs, P =
+//                       2^x with one ex2.bf16x2 per pair (P comes out already in the bf16
+//                       form the MMA consumes), written back to TMEM (tcgen05.st).
+//
+// Online softmax with lazy rescaling: the reference max m of a row only moves when a
+// tile's exponent would exceed 2^8; the common case costs a bf16x2 max over the packed
+// exponents and no fp32 max at all. When a row's reference moves (the first tile, or a
+// new maximum), the exact fp32 tile max is taken and O' (including the row-sum column) is
+// rescaled in TMEM. The result is exact up to rounding after the final division by the
+// row sum.
 //
 // Partial pages need no per-column mask: slots past a page's valid count hold K = V = 0
-// (the append and compaction kernels write zeros there, and pages past the end of the
-// list are read out of bounds so TMA fills zeros), so each scores exactly 0, adds nothing
-// to O and exactly 2^-m to the row sum, which is subtracted once per tile.
+// (the append and compaction kernels write zeros there), so each scores exactly 0, adds
+// nothing to O and 2^-m to the row sum; that amount is tracked per row and taken out.
 //
-// TMEM (256 columns): S [0,128), P [128,192) (bf16 pairs), O [192,256). Two CTAs fit per
-// SM (TMEM 2 x 256 columns, shared memory 2 x ~85 KB, 96 registers per thread), which puts
-// four softmax warps on every SM sub-partition and lets one CTA's MMAs overlap the
-// other's softmax. The KV sequence can be split across CTAs; partial outputs carry the
+// P is double-buffered in TMEM so a tile's softmax never waits for the previous tile's
+// P.V product. TMEM (256 columns): S [0,64), P0 [64,96), P1 [96,128), O' [128,208). Two
+// CTAs fit per SM. The KV sequence can be split across CTAs; partial outputs carry the
 // log2-sum-exp and a combine kernel merges them. Every barrier wait is bounded: on
 // timeout the CTA records KVC_ERR_TIMEOUT in the error word, drains its own copies and
 // MMAs, frees TMEM and returns.
@@ -42,18 +45,18 @@
 namespace kvc {
 namespace tc {
 constexpr int kBM = 128;                      // query rows per CTA
-constexpr int kBN = 128;                      // KV slots per tile
+constexpr int kBN = 64;                       // KV slots per tile
 constexpr int kHD = 64;                       // head dim (one 128-byte swizzle row)
-constexpr int kStages = 2;
-constexpr int kTileBytes = kBN * kHD * 2;     // 16 KB
+constexpr int kON = kHD + 16;                 // O' columns: O plus the row-sum block
+constexpr int kStages = 4;
+constexpr int kTileBytes = kBN * kHD * 2;     // 8 KB (K or V tile)
 constexpr int kQBytes = kBM * kHD * 2;        // 16 KB
-constexpr int kThreads = 320;                 // producer, MMA, 8 softmax warps
+constexpr int kOnesBytes = kBN * kHD * 2;     // 8 KB block of bf16 ones
+constexpr int kThreads = 192;
 constexpr int kTmemCols = 256;
-constexpr int kColS = 0, kColP = 128, kColO = 192;
+constexpr int kColS = 0, kColP = 64, kColO = 128;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kPolyCols = 0;                  // of each warp's 64 columns, exponentiated on the FMA pipe
-                                              // (0: measured fastest; the MUFU is not the limit)                 // of each warp's 64 columns, exponentiated on the FMA pipe
-constexpr size_t kSmemBytes = 1024 + kQBytes + 2 * kStages * kTileBytes + 256 + 2 * 2 * kBM * 4;
+constexpr size_t kSmemBytes = 1024 + kQBytes + 2 * kStages * kTileBytes + kOnesBytes + 256;
 }  // namespace tc
 
 struct TcParams {
@@ -80,31 +83,43 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// 3-input max (sm_100a)
+// ---- packed arithmetic used by the softmax
+__device__ __forceinline__ uint64_t fma2_pair(uint32_t s0, uint32_t s1, uint64_t c2, uint64_t nm2) {
+  uint64_t x, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(s0), "r"(s1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(x), "l"(c2), "l"(nm2));
+  return r;
+}
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+// (lo, hi) fp32 pair -> bf16x2, round to nearest even
+__device__ __forceinline__ uint32_t bf16x2_of(uint64_t x) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t ex2_bf16x2(uint32_t x) {
+  uint32_t r;
+  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
+}
+__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
-
-// 2^x on the FMA pipe for x <= 8 (lazy rescaling bounds the exponent): x is split as
-// n + f with n = round(x) (adding and subtracting 1.5 * 2^23) and |f| <= 1/2; 2^f comes
-// from a degree-3 polynomial whose coefficients were fitted for this kernel (relative
-// minimax on [-1/2, 1/2], max relative error 7.6e-5, far below the 2^-9 rounding of P to
-// bf16); 2^n is applied by adding n to the exponent field. Inputs below -125 are clamped
-// so the result stays a normal number. Used for the last kPolyCols columns of a half.
-__device__ __forceinline__ float exp2_poly(float x) {
-  constexpr float kC0 = 0.9999281764030457f, kC1 = 0.6932609677314758f, kC2 = 0.2426096349954605f,
-                  kC3 = 0.055170949548482895f, kMagic = 12582912.0f;
-  x = fmaxf(x, -125.f);
-  const float t = x + kMagic;
-  const float n = t - kMagic;
-  const float f = x - n;
-  float q = fmaf(kC3, f, kC2);
-  q = fmaf(q, f, kC1);
-  q = fmaf(q, f, kC0);
-  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
-}
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
 // Wait without the abort shortcut, used only to drain a CTA's own in-flight work.
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, int* err) {
@@ -123,7 +138,8 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
   uint8_t* q_s = smem;
   uint8_t* k_s = smem + kQBytes;
   uint8_t* v_s = k_s + kStages * kTileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(v_s + kStages * kTileBytes);
+  uint8_t* ones_s = v_s + kStages * kTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ones_s + kOnesBytes);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = k_full + kStages;
@@ -131,12 +147,10 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
   uint64_t* s_full = kv_empty + kStages;
   uint64_t* s_free = s_full + 1;
   uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = s_full + 3;
-  uint64_t* mma_final = s_full + 4;
-  uint64_t* xchg = s_full + 5;                // [4] one per TMEM lane quadrant (softmax warp pair)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xchg + 4);
+  uint64_t* pv_done = s_full + 3;             // [2] one per P buffer
+  uint64_t* mma_final = s_full + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* red = reinterpret_cast<float*>(bars + 32);   // [2 parity][2 halves][128 rows] row values
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x % p.q_tiles;
@@ -155,14 +169,19 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 8);
-    mbar_init(p_full, 8);
-    for (int i = 0; i < 4; ++i) mbar_init(&xchg[i], 64);
-    mbar_init(pv_done, 1);
+    mbar_init(s_free, 4);
+    mbar_init(p_full, 4);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
     mbar_init(mma_final, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
+  // the constant ones block (every element 1.0, so the swizzle does not matter), made
+  // visible to the tensor core's operand reads
+  for (int i = threadIdx.x; i < kOnesBytes / 16; i += kThreads)
+    reinterpret_cast<uint4*>(ones_s)[i] = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -188,25 +207,22 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           const int st = j % kStages;
           if (j >= kStages && !mbar_wait_bounded(&kv_empty[st], ((j / kStages) - 1) & 1, abort_flag, p.err)) break;
           const int gt = tile0 + j;
-          uint8_t* kd = k_s + st * kTileBytes;
-          uint8_t* vd = v_s + st * kTileBytes;
-          mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+          int row[kPPT];
 #pragma unroll
           for (int g = 0; g < kPPT; ++g) {
             const int idx = gt * kPPT + g;
             // pages past the list end are read past the end of the pool: TMA fills zeros
-            const int row = idx < p.n_pages ? static_cast<int>(((p.page_base + __ldg(&p.entries[idx].x)) * p.H + h) * P)
-                                            : p.pool_rows;
-            tma_load_2d(kd + g * P * 128, &tmap_k, &k_full[st], 0, row);
+            row[g] = idx < p.n_pages ? static_cast<int>(((p.page_base + __ldg(&p.entries[idx].x)) * p.H + h) * P)
+                                     : p.pool_rows;
           }
+          mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+#pragma unroll
+          for (int g = 0; g < kPPT; ++g)
+            tma_load_2d(k_s + st * kTileBytes + g * P * 128, &tmap_k, &k_full[st], 0, row[g]);
           mbar_arrive_expect_tx(&v_full[st], kTileBytes);
 #pragma unroll
-          for (int g = 0; g < kPPT; ++g) {
-            const int idx = gt * kPPT + g;
-            const int row = idx < p.n_pages ? static_cast<int>(((p.page_base + __ldg(&p.entries[idx].x)) * p.H + h) * P)
-                                            : p.pool_rows;
-            tma_load_2d(vd + g * P * 128, &tmap_v, &v_full[st], 0, row);
-          }
+          for (int g = 0; g < kPPT; ++g)
+            tma_load_2d(v_s + st * kTileBytes + g * P * 128, &tmap_v, &v_full[st], 0, row[g]);
           last[st] = j;
         }
         // drain: every copy this CTA issued has landed before shared memory is released
@@ -223,9 +239,10 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
       if (lane == 0) {
         // ---------------------------------------------------------------- MMA issuer
         const uint32_t idesc_s = idesc_f16kind(1, kBM, kBN, 0, 0);
-        const uint32_t idesc_o = idesc_f16kind(1, kBM, kHD, 0, 1);
+        const uint32_t idesc_o = idesc_f16kind(1, kBM, kON, 0, 1);
         const uint32_t tS = tmem + kColS, tP = tmem + kColP, tO = tmem + kColO;
         const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
+        const uint32_t ones_addr = smem_u32(ones_s);
         bool ok = mbar_wait_bounded(q_full, 0, abort_flag, p.err) &&
                   mbar_wait_bounded(&k_full[0], 0, abort_flag, p.err);
         if (ok) {
@@ -255,11 +272,14 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           if (!mbar_wait_bounded(p_full, j & 1, abort_flag, p.err)) break;
           if (!mbar_wait_bounded(&v_full[st], ph, abort_flag, p.err)) break;
           tc_fence_after();
+          // B = [V | ones]: the V tile is MN atom 0, the ones block MN atom 1 (LBO apart)
           const uint32_t vb = v_addr + st * kTileBytes;
+          const uint32_t lbo = ones_addr - vb;
+          const uint32_t pa = tP + (j & 1) * (kBN / 2);
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_ts(tO, tP + kk * 8, sw128_desc(vb + kk * 2048, 8192, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(pv_done);
+            mma_ts(tO, pa + kk * 8, sw128_desc(vb + kk * 2048, lbo, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&pv_done[j & 1]);
           mma_commit(&kv_empty[st]);
         }
         // drain: all MMAs of this CTA complete before TMEM is released
@@ -268,38 +288,29 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
       }
     } else {
       // ------------------------------------------------------------------ softmax warps
-      // Eight warps. Warp w may only access TMEM lane quadrant w % 4 (its 32 query rows);
-      // the two warps sharing a quadrant split each 128-column S tile into halves of 64
-      // and exchange per-row maxima through shared memory (mbarrier xchg[quadrant]).
-      constexpr int kHalf = kBN / 2;
-      constexpr int kPPH = kPPT / 2;               // pages per column half
-      const int wq = warp & 3;
-      const int hf = (warp - 2) >> 2;
-      const int r = wq * 32 + lane;
+      const int wq = warp & 3;                      // TMEM lane quadrant this warp may access
+      const int r = wq * 32 + lane;                 // query row within the tile
       const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-      const uint32_t tS = tmem + kColS + hf * kHalf + lane_off;
-      const uint32_t tP = tmem + kColP + hf * (kHalf / 2) + lane_off;
-      const uint32_t tO = tmem + kColO + hf * (kHD / 2) + lane_off;
+      const uint32_t tS = tmem + kColS + lane_off, tP = tmem + kColP + lane_off, tO = tmem + kColO + lane_off;
       const float c = p.scale_log2;
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY;       // reference max (log2 domain) of the row
+      float masked = 0.f;        // row-sum share of zero-padded slots, rescaled like O'
       bool ok = true;
-      // valid-slot counts of this half's pages of the next KV tile, loaded one tile ahead
-      int vnext[kPPH];
+      // valid-slot counts of the next KV tile's pages, loaded one tile ahead
+      int vnext[kPPT];
 #pragma unroll
-      for (int g = 0; g < kPPH; ++g) {
-        const int idx = tile0 * kPPT + hf * kPPH + g;
+      for (int g = 0; g < kPPT; ++g) {
+        const int idx = tile0 * kPPT + g;
         vnext[g] = idx < p.n_pages ? __ldg(&p.entries[idx].w) : 0;
       }
       for (int j = 0; j < n_tiles; ++j) {
-        // invalid slots hold K = V = 0, so they score 0 and add exactly 2^-m to the row
-        // sum and nothing to O: count them and take them out of the sum below
         int n_masked = 0;
 #pragma unroll
-        for (int g = 0; g < kPPH; ++g) n_masked += P - vnext[g];
+        for (int g = 0; g < kPPT; ++g) n_masked += P - vnext[g];
         if (j + 1 < n_tiles) {
 #pragma unroll
-          for (int g = 0; g < kPPH; ++g) {
-            const int idx = (tile0 + j + 1) * kPPT + hf * kPPH + g;
+          for (int g = 0; g < kPPT; ++g) {
+            const int idx = (tile0 + j + 1) * kPPT + g;
             vnext[g] = idx < p.n_pages ? __ldg(&p.entries[idx].w) : 0;
           }
         }
@@ -316,107 +327,90 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free);
-        float mxa = -INFINITY, mxb = -INFINITY, mxc = -INFINITY, mxd = -INFINITY;
+        // exponents x = s*c - m as bf16 pairs, with their max
+        uint32_t xb[kBN / 2];
+        uint32_t mxb = 0xff80ff80u;               // bf16x2 (-inf, -inf)
+        {
+          const uint64_t c2 = pk2(c, c), nm2 = pk2(-m, -m);
 #pragma unroll
-        for (int cc = 0; cc < kHalf; cc += 8) {
-          mxa = max3(mxa, __uint_as_float(s[cc / 32][cc % 32 + 0]), __uint_as_float(s[cc / 32][cc % 32 + 1]));
-          mxb = max3(mxb, __uint_as_float(s[cc / 32][cc % 32 + 2]), __uint_as_float(s[cc / 32][cc % 32 + 3]));
-          mxc = max3(mxc, __uint_as_float(s[cc / 32][cc % 32 + 4]), __uint_as_float(s[cc / 32][cc % 32 + 5]));
-          mxd = max3(mxd, __uint_as_float(s[cc / 32][cc % 32 + 6]), __uint_as_float(s[cc / 32][cc % 32 + 7]));
+          for (int i = 0; i < kBN / 2; ++i) {
+            xb[i] = bf16x2_of(fma2_pair(s[(2 * i) / 32][(2 * i) % 32], s[(2 * i + 1) / 32][(2 * i + 1) % 32], c2, nm2));
+            mxb = max_bf16x2(mxb, xb[i]);
+          }
         }
-        float mx = fmaxf(fmaxf(mxa, mxb), fmaxf(mxc, mxd));
-        // row max of the whole tile: swap halves with the partner warp
-        red[((j & 1) * 2 + hf) * kBM + r] = mx;
-        mbar_arrive(&xchg[wq]);
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&xchg[wq], j & 1, abort_flag, p.err))) {
-          ok = false;
-          break;
-        }
-        mx = fmaxf(mx, red[((j & 1) * 2 + (1 - hf)) * kBM + r]);
-        const float mx_s = mx * c;
-        float m_new = m;
-        bool rescale = false;
-        if (j == 0) {
-          m_new = mx_s;
-        } else if (mx_s > m + kRescaleLog2) {
-          m_new = mx_s;
-          rescale = true;
-        }
-        // P = 2^(s*c - m) in scalar fp32: the first kHalf - kPolyCols columns on the MUFU
-        // ex2, the last kPolyCols with the FMA-pipe polynomial; each pair is summed into
-        // four independent accumulators and packed to bf16 right away.
-        const float nm = -m_new;
-        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-        uint32_t pk[kHalf / 2];
+        const bool move = (j == 0) || fmaxf(bf16lo(mxb), bf16hi(mxb)) > kRescaleLog2;
+        if (__any_sync(0xffffffffu, move)) {
+          // slow path (first tile or a new maximum): exact fp32 tile max for the rows that
+          // move their reference; rescale O' and the masked share by 2^(m_old - m_new)
+          float ta = -INFINITY, tb = -INFINITY;
 #pragma unroll
-        for (int cc = 0; cc < kHalf; cc += 2) {
-          float x0 = fmaf(__uint_as_float(s[cc / 32][cc % 32]), c, nm);
-          float x1 = fmaf(__uint_as_float(s[cc / 32][cc % 32 + 1]), c, nm);
-          if (cc >= kHalf - kPolyCols) {
-            x0 = exp2_poly(x0);
-            x1 = exp2_poly(x1);
-          } else {
-            x0 = ex2(x0);
-            x1 = ex2(x1);
+          for (int cc = 0; cc < kBN; cc += 4) {
+            ta = max3(ta, __uint_as_float(s[cc / 32][cc % 32]), __uint_as_float(s[cc / 32][cc % 32 + 1]));
+            tb = max3(tb, __uint_as_float(s[cc / 32][cc % 32 + 2]), __uint_as_float(s[cc / 32][cc % 32 + 3]));
           }
-          if ((cc / 2) & 1) {
-            acc2 += x0;
-            acc3 += x1;
-          } else {
-            acc0 += x0;
-            acc1 += x1;
+          const float m_new = move ? fmaxf(ta, tb) * c : m;
+          const bool resc = move && j > 0;
+          if (__any_sync(0xffffffffu, resc)) {
+            // O' row *= f; the previous tile's P.V must have landed
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait_bounded(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, p.err))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const float f = resc ? ex2(m - m_new) : 1.0f;
+            masked *= f;
+#pragma unroll
+            for (int q4 = 0; q4 < kON / 16; ++q4) {
+              uint32_t oc[16];
+              tmem_ld16(tO + q4 * 16, oc);
+              tmem_ld_wait();
+#pragma unroll
+              for (int d = 0; d < 16; ++d) oc[d] = __float_as_uint(__uint_as_float(oc[d]) * f);
+              tmem_st16(tO + q4 * 16, oc);
+            }
           }
-          pk[cc / 2] = pack_bf16(x0, x1);
+          m = m_new;
+          const uint64_t c2 = pk2(c, c), nm2 = pk2(-m, -m);
+#pragma unroll
+          for (int i = 0; i < kBN / 2; ++i)
+            xb[i] = bf16x2_of(fma2_pair(s[(2 * i) / 32][(2 * i) % 32], s[(2 * i + 1) / 32][(2 * i + 1) % 32], c2, nm2));
         }
-        float rs = (acc0 + acc1) + (acc2 + acc3);
-        if (n_masked) rs -= static_cast<float>(n_masked) * ex2(nm);
-        if (j > 0) {
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(pv_done, (j - 1) & 1, abort_flag, p.err))) {
+        // P = 2^x, two per instruction, already bf16
+#pragma unroll
+        for (int i = 0; i < kBN / 2; ++i) xb[i] = ex2_bf16x2(xb[i]);
+        if (n_masked) {
+          // each zero-padded slot scored 0 and contributed exactly 2^(bf16(-m)) to the sum
+          masked += static_cast<float>(n_masked) * bf16lo(ex2_bf16x2(bf16x2_of(pk2(-m, -m))));
+        }
+        // P buffer j & 1 was last read by the P.V product of tile j - 2
+        if (j >= 2) {
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, p.err))) {
             ok = false;
             break;
           }
           tc_fence_after();
         }
-        if (__any_sync(0xffffffffu, rescale)) {
-          // this warp's 32 O columns *= 2^(m_old - m_new); rows that keep their reference
-          // max scale by 1 (the branch is warp-uniform)
-          const float corr = rescale ? ex2(m - m_new) : 1.0f;
-          l *= corr;
-#pragma unroll
-          for (int q4 = 0; q4 < kHD / 32; ++q4) {
-            uint32_t oc[16];
-            tmem_ld16(tO + q4 * 16, oc);
-            tmem_ld_wait();
-#pragma unroll
-            for (int d = 0; d < 16; ++d) oc[d] = __float_as_uint(__uint_as_float(oc[d]) * corr);
-            tmem_st16(tO + q4 * 16, oc);
-          }
-        }
-        m = m_new;
-        l += rs;
-        tmem_st32(tP, pk);
+        tmem_st32(tP + (j & 1) * (kBN / 2), xb);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
       }
-      // row sum of the two halves, then the epilogue writes this warp's 32 columns
-      if (ok) {
-        red[((n_tiles & 1) * 2 + hf) * kBM + r] = l;
-        mbar_arrive(&xchg[wq]);
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&xchg[wq], n_tiles & 1, abort_flag, p.err));
-        if (ok) l += red[((n_tiles & 1) * 2 + (1 - hf)) * kBM + r];
-      }
-      if (__all_sync(0xffffffffu, ok && mbar_wait_bounded(pv_done, (n_tiles - 1) & 1, abort_flag, p.err))) {
+      const int jl = n_tiles - 1;
+      if (__all_sync(0xffffffffu, ok && mbar_wait_bounded(&pv_done[jl & 1], (jl >> 1) & 1, abort_flag, p.err))) {
         tc_fence_after();
-        uint32_t o0[32];
+        uint32_t o0[32], o1[32], ls[16];
         tmem_ld32(tO, o0);
+        tmem_ld32(tO + 32, o1);
+        tmem_ld16(tO + 64, ls);
         tmem_ld_wait();
+        const float l = __uint_as_float(ls[0]) - masked;
         const float inv = 1.f / l;
         const int row = qt * kBM + r;
         if (p.splits == 1) {
           if (row < p.T) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<long long>(row) * p.H + h) * kHD + hf * 32);
+            uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<long long>(row) * p.H + h) * kHD);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               uint4 w;
@@ -426,15 +420,28 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
               w.w = pack_bf16(__uint_as_float(o0[8 * v + 6]) * inv, __uint_as_float(o0[8 * v + 7]) * inv);
               dst[v] = w;
             }
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 w;
+              w.x = pack_bf16(__uint_as_float(o1[8 * v + 0]) * inv, __uint_as_float(o1[8 * v + 1]) * inv);
+              w.y = pack_bf16(__uint_as_float(o1[8 * v + 2]) * inv, __uint_as_float(o1[8 * v + 3]) * inv);
+              w.z = pack_bf16(__uint_as_float(o1[8 * v + 4]) * inv, __uint_as_float(o1[8 * v + 5]) * inv);
+              w.w = pack_bf16(__uint_as_float(o1[8 * v + 6]) * inv, __uint_as_float(o1[8 * v + 7]) * inv);
+              dst[4 + v] = w;
+            }
           }
         } else {
           const long long pi = (static_cast<long long>(h) * p.splits + split) * p.q_tiles + qt;
-          float4* dst = reinterpret_cast<float4*>(p.part_o + (pi * kBM + r) * kHD + hf * 32);
+          float4* dst = reinterpret_cast<float4*>(p.part_o + (pi * kBM + r) * kHD);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
             dst[v] = make_float4(__uint_as_float(o0[4 * v + 0]) * inv, __uint_as_float(o0[4 * v + 1]) * inv,
                                  __uint_as_float(o0[4 * v + 2]) * inv, __uint_as_float(o0[4 * v + 3]) * inv);
-          if (hf == 0) p.part_lse[pi * kBM + r] = m + __log2f(l);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[8 + v] = make_float4(__uint_as_float(o1[4 * v + 0]) * inv, __uint_as_float(o1[4 * v + 1]) * inv,
+                                     __uint_as_float(o1[4 * v + 2]) * inv, __uint_as_float(o1[4 * v + 3]) * inv);
+          p.part_lse[pi * kBM + r] = m + __log2f(l);
         }
       }
     }
