@@ -237,3 +237,28 @@ def test_rescale_in_some_rows_of_a_warp(kvc):
         torch.cuda.synchronize()
         compare_out(np64(o), ref, "bf16", f"frame {t}")
     kvc.kvc_destroy(h)
+
+
+def test_back_to_back_frames_without_host_sync(kvc):
+    """Frames issued back to back with no host synchronisation (as a streaming caller
+    does): no bounded wait may give up, and the last frame matches the oracle."""
+    wl = WORKLOADS["vggt_518x378"]
+    dev = torch.device("cuda")
+    h = kvc.kvc_create(kvc.config_from_workload(wl))
+    st = FrameStream(wl, seed=9, device=dev)
+    orc = StreamOracle(OracleConfig.from_workload(wl))
+    o = torch.empty((wl.tokens_per_frame, wl.num_heads, wl.head_dim), dtype=torch.bfloat16, device=dev)
+    frames = wl.scale_frames + wl.window_frames + 40
+    rows = sample_rows(wl.tokens_per_frame, 32, seed=3)
+    for t in range(frames):
+        q, k, v = st.frame(0, t)
+        kvc.kvc_append_frame(h, 0, t, k, v, True)
+        kvc.kvc_attend(h, 0, q, o)
+        orc.append(0, t, np64(k), np64(v), True)
+        if t < frames - 1:
+            orc.commit(0)
+        else:
+            ref = orc.attend(0, np64(q), rows=rows)
+    kvc.kvc_synchronize(h)                       # raises on a latched device error
+    compare_out(np64(o)[rows], ref, "bf16", "last frame")
+    kvc.kvc_destroy(h)

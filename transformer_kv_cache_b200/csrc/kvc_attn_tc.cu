@@ -15,13 +15,13 @@
 //                       B = the V tile as an MN-major operand followed by a constant block
 //                       of ones), so accumulator column 64 carries the row sum of P.
 //   warps 2..5          softmax, thread = query row = TMEM lane, 64 columns per tile:
-//                       x = s*c - m with packed f32x2 FMAs, x rounded to bf16 pairs, P =
-//                       2^x with one ex2.bf16x2 per pair (P comes out already in the bf16
-//                       form the MMA consumes), written back to TMEM (tcgen05.st).
+//                       x = s*c - m with packed f32x2 FMAs, P = 2^x on the MUFU, packed
+//                       to the bf16 pairs the MMA consumes and written back to TMEM
+//                       (tcgen05.st); no per-element sum (the MMA makes it).
 //
 // Online softmax with lazy rescaling: the reference max m of a row only moves when a
-// tile's exponent would exceed 2^8; the common case costs a bf16x2 max over the packed
-// exponents and no fp32 max at all. When a row's reference moves (the first tile, or a
+// tile's P would exceed 2^8; the common case costs a bf16x2 max over the packed P and no
+// fp32 max at all. When a row's reference moves (the first tile, or a
 // new maximum), the exact fp32 tile max is taken and O' (including the row-sum column) is
 // rescaled in TMEM. The result is exact up to rounding after the final division by the
 // row sum.
@@ -55,7 +55,7 @@ constexpr int kOnesBytes = kBN * kHD * 2;     // 8 KB block of bf16 ones
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 256;
 constexpr int kColS = 0, kColP = 64, kColO = 128;
-constexpr float kRescaleLog2 = 8.0f;
+constexpr float kPMax = 256.0f;               // a P above 2^8 moves the row's reference max
 constexpr size_t kSmemBytes = 1024 + kQBytes + 2 * kStages * kTileBytes + kOnesBytes + 256;
 }  // namespace tc
 
@@ -95,18 +95,8 @@ __device__ __forceinline__ uint64_t pk2(float a, float b) {
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
   return r;
 }
-// (lo, hi) fp32 pair -> bf16x2, round to nearest even
-__device__ __forceinline__ uint32_t bf16x2_of(uint64_t x) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-__device__ __forceinline__ uint32_t ex2_bf16x2(uint32_t x) {
-  uint32_t r;
-  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(r) : "r"(x));
-  return r;
+__device__ __forceinline__ void up2(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
 }
 __device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
   uint32_t r;
@@ -146,9 +136,9 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
   uint64_t* kv_empty = v_full + kStages;
   uint64_t* s_full = kv_empty + kStages;
   uint64_t* s_free = s_full + 1;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = s_full + 3;             // [2] one per P buffer
-  uint64_t* mma_final = s_full + 5;
+  uint64_t* p_full = s_full + 2;              // [2] one per P buffer
+  uint64_t* pv_done = s_full + 4;             // [2] one per P buffer
+  uint64_t* mma_final = s_full + 6;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -170,7 +160,8 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 4);
-    mbar_init(p_full, 4);
+    mbar_init(&p_full[0], 4);
+    mbar_init(&p_full[1], 4);
     mbar_init(&pv_done[0], 1);
     mbar_init(&pv_done[1], 1);
     mbar_init(mma_final, 1);
@@ -269,7 +260,9 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
                      kk > 0);
             mma_commit(s_full);
           }
-          if (!mbar_wait_bounded(p_full, j & 1, abort_flag, p.err)) break;
+          // one barrier per P buffer: the softmax may finish tile j + 1 before this wait,
+          // and phase j + 2 of a single barrier would alias phase j
+          if (!mbar_wait_bounded(&p_full[j & 1], (j >> 1) & 1, abort_flag, p.err)) break;
           if (!mbar_wait_bounded(&v_full[st], ph, abort_flag, p.err)) break;
           tc_fence_after();
           // B = [V | ones]: the V tile is MN atom 0, the ones block MN atom 1 (LBO apart)
@@ -327,18 +320,22 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free);
-        // exponents x = s*c - m as bf16 pairs, with their max
-        uint32_t xb[kBN / 2];
-        uint32_t mxb = 0xff80ff80u;               // bf16x2 (-inf, -inf)
+        // P = 2^(s*c - m): exponent pairs with one packed FMA, two MUFU ex2, one bf16 pack;
+        // a bf16x2 max over the packed P tells whether any exponent exceeded 2^8 (or the
+        // reference was unset), in which case the row's reference max moves (slow path)
+        uint32_t pb[kBN / 2];
+        uint32_t mxb = 0u;
         {
           const uint64_t c2 = pk2(c, c), nm2 = pk2(-m, -m);
 #pragma unroll
           for (int i = 0; i < kBN / 2; ++i) {
-            xb[i] = bf16x2_of(fma2_pair(s[(2 * i) / 32][(2 * i) % 32], s[(2 * i + 1) / 32][(2 * i + 1) % 32], c2, nm2));
-            mxb = max_bf16x2(mxb, xb[i]);
+            float x0, x1;
+            up2(fma2_pair(s[(2 * i) / 32][(2 * i) % 32], s[(2 * i + 1) / 32][(2 * i + 1) % 32], c2, nm2), x0, x1);
+            pb[i] = pack_bf16(ex2(x0), ex2(x1));
+            mxb = max_bf16x2(mxb, pb[i]);
           }
         }
-        const bool move = (j == 0) || fmaxf(bf16lo(mxb), bf16hi(mxb)) > kRescaleLog2;
+        const bool move = (j == 0) || fmaxf(bf16lo(mxb), bf16hi(mxb)) > kPMax;
         if (__any_sync(0xffffffffu, move)) {
           // slow path (first tile or a new maximum): exact fp32 tile max for the rows that
           // move their reference; rescale O' and the masked share by 2^(m_old - m_new)
@@ -373,15 +370,15 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           m = m_new;
           const uint64_t c2 = pk2(c, c), nm2 = pk2(-m, -m);
 #pragma unroll
-          for (int i = 0; i < kBN / 2; ++i)
-            xb[i] = bf16x2_of(fma2_pair(s[(2 * i) / 32][(2 * i) % 32], s[(2 * i + 1) / 32][(2 * i + 1) % 32], c2, nm2));
+          for (int i = 0; i < kBN / 2; ++i) {
+            float x0, x1;
+            up2(fma2_pair(s[(2 * i) / 32][(2 * i) % 32], s[(2 * i + 1) / 32][(2 * i + 1) % 32], c2, nm2), x0, x1);
+            pb[i] = pack_bf16(ex2(x0), ex2(x1));
+          }
         }
-        // P = 2^x, two per instruction, already bf16
-#pragma unroll
-        for (int i = 0; i < kBN / 2; ++i) xb[i] = ex2_bf16x2(xb[i]);
         if (n_masked) {
-          // each zero-padded slot scored 0 and contributed exactly 2^(bf16(-m)) to the sum
-          masked += static_cast<float>(n_masked) * bf16lo(ex2_bf16x2(bf16x2_of(pk2(-m, -m))));
+          // each zero-padded slot scored 0 and contributed exactly bf16(2^-m) to the sum
+          masked += static_cast<float>(n_masked) * bf16lo(pack_bf16(ex2(-m), 0.f));
         }
         // P buffer j & 1 was last read by the P.V product of tile j - 2
         if (j >= 2) {
@@ -391,11 +388,11 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           }
           tc_fence_after();
         }
-        tmem_st32(tP + (j & 1) * (kBN / 2), xb);
+        tmem_st32(tP + (j & 1) * (kBN / 2), pb);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(&p_full[j & 1]);
       }
       const int jl = n_tiles - 1;
       if (__all_sync(0xffffffffu, ok && mbar_wait_bounded(&pv_done[jl & 1], (jl >> 1) & 1, abort_flag, p.err))) {
