@@ -15,9 +15,11 @@
 //                       B = the V tile as an MN-major operand followed by a constant block
 //                       of ones), so accumulator column 64 carries the row sum of P.
 //   warps 2..5          softmax, thread = query row = TMEM lane, 64 columns per tile:
-//                       x = s*c - m with packed f32x2 FMAs, P = 2^x on the MUFU, packed
-//                       to the bf16 pairs the MMA consumes and written back to TMEM
-//                       (tcgen05.st); no per-element sum (the MMA makes it).
+//                       x = s*c - m with packed f32x2 FMAs, P = 2^x on the MUFU, its upper
+//                       halves taken as the bf16 pairs the MMA consumes (one byte permute
+//                       per pair) and written back to TMEM (tcgen05.st); no per-element sum
+//                       (the MMA makes it from the same bf16 P). The next tile's S is
+//                       loaded from TMEM while this tile's P store is in flight.
 //
 // Online softmax with lazy rescaling: the reference max m of a row only moves when a
 // tile's P would exceed 2^8; the common case costs a bf16x2 max over the packed P and no
@@ -110,6 +112,15 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 }
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// Upper halves of two fp32 values as a bf16 pair (truncation toward zero), one byte
+// permute; P is consumed by the MMA and summed by it from the same bf16 values, so the
+// truncation's common scale cancels in O / l.
+__device__ __forceinline__ uint32_t bf16x2_trunc(float lo, float hi) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(__float_as_uint(lo)), "r"(__float_as_uint(hi)));
+  return r;
+}
 
 // Wait without the abort shortcut, used only to drain a CTA's own in-flight work.
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, int* err) {
@@ -296,7 +307,20 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
         const int idx = tile0 * kPPT + g;
         vnext[g] = idx < p.n_pages ? __ldg(&p.entries[idx].w) : 0;
       }
-      for (int j = 0; j < n_tiles; ++j) {
+      // S of the current tile lives in registers; the next tile's S is loaded while this
+      // tile's P store is in flight
+      uint32_t s[2][32];
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_full, 0, abort_flag, p.err))) ok = false;
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(tS + 0, s[0]);
+        tmem_ld32(tS + 32, s[1]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+      }
+      for (int j = 0; ok && j < n_tiles; ++j) {
         int n_masked = 0;
 #pragma unroll
         for (int g = 0; g < kPPT; ++g) n_masked += P - vnext[g];
@@ -307,19 +331,6 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
             vnext[g] = idx < p.n_pages ? __ldg(&p.entries[idx].w) : 0;
           }
         }
-        // tcgen05.ld/st are .sync.aligned: every branch around them is kept warp-uniform
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_full, j & 1, abort_flag, p.err))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        uint32_t s[2][32];
-        tmem_ld32(tS + 0, s[0]);
-        tmem_ld32(tS + 32, s[1]);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);
         // P = 2^(s*c - m): exponent pairs with one packed FMA, two MUFU ex2, one bf16 pack;
         // a bf16x2 max over the packed P tells whether any exponent exceeded 2^8 (or the
         // reference was unset), in which case the row's reference max moves (slow path)
@@ -331,7 +342,7 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           for (int i = 0; i < kBN / 2; ++i) {
             float x0, x1;
             up2(fma2_pair(s[(2 * i) / 32][(2 * i) % 32], s[(2 * i + 1) / 32][(2 * i + 1) % 32], c2, nm2), x0, x1);
-            pb[i] = pack_bf16(ex2(x0), ex2(x1));
+            pb[i] = bf16x2_trunc(ex2(x0), ex2(x1));
             mxb = max_bf16x2(mxb, pb[i]);
           }
         }
@@ -373,12 +384,12 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           for (int i = 0; i < kBN / 2; ++i) {
             float x0, x1;
             up2(fma2_pair(s[(2 * i) / 32][(2 * i) % 32], s[(2 * i + 1) / 32][(2 * i + 1) % 32], c2, nm2), x0, x1);
-            pb[i] = pack_bf16(ex2(x0), ex2(x1));
+            pb[i] = bf16x2_trunc(ex2(x0), ex2(x1));
           }
         }
         if (n_masked) {
           // each zero-padded slot scored 0 and contributed exactly bf16(2^-m) to the sum
-          masked += static_cast<float>(n_masked) * bf16lo(pack_bf16(ex2(-m), 0.f));
+          masked += static_cast<float>(n_masked) * bf16lo(bf16x2_trunc(ex2(-m), 0.f));
         }
         // P buffer j & 1 was last read by the P.V product of tile j - 2
         if (j >= 2) {
@@ -389,10 +400,27 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           tc_fence_after();
         }
         tmem_st32(tP + (j & 1) * (kBN / 2), pb);
+        // tcgen05.ld/st are .sync.aligned: every branch around them is kept warp-uniform
+        const bool more = j + 1 < n_tiles;
+        if (more) {
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_full, (j + 1) & 1, abort_flag, p.err))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          tmem_ld32(tS + 0, s[0]);
+          tmem_ld32(tS + 32, s[1]);
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[j & 1]);
+        if (more) {
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free);
+        }
       }
       const int jl = n_tiles - 1;
       if (__all_sync(0xffffffffu, ok && mbar_wait_bounded(&pv_done[jl & 1], (jl >> 1) & 1, abort_flag, p.err))) {
