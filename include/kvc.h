@@ -153,6 +153,14 @@ KVC_API kvc_status kvc_reset(kvc_cache* c);
 KVC_API kvc_status kvc_append_frame(kvc_cache* c, int32_t layer, int32_t frame_idx,
                             const void* k_dev, const void* v_dev, int32_t is_keyframe);
 
+/* kvc_append_frame for every layer at once: k_devs[l], v_devs[l] (host arrays of
+ * num_layers device pointers) hold layer l's [T, H, D] K and V. One page-allocation
+ * launch and one append launch cover up to 64 layers, so the frame's whole K/V write is
+ * a single HBM-bound kernel. Same semantics, layout and errors as kvc_append_frame
+ * applied to each layer; nothing is appended unless every layer can take the frame. */
+KVC_API kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const void* const* k_devs,
+                                        const void* const* v_devs, int32_t is_keyframe);
+
 /* Frame attention of the pending frame's queries q_dev [T, H, D] over every
  * token of `layer` (committed + pending), writing o_dev [T, H, D]:
  * O[i,h] = sum_j softmax_j(softmax_scale * q_i . k_j) v_j, no mask

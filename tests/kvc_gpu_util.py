@@ -47,7 +47,7 @@ def compare_out(got: np.ndarray, ref: np.ndarray, io_dtype: str, what: str = "")
 
 
 def run_parity(kvc, wl, frames, *, check_frames=None, rows=None, seed=0, layers=None, kv_splits=0,
-               check_pages=False, record=None):
+               check_pages=False, record=None, batched_append=False):
     """Stream `frames` frames through the library and the oracle; compare page tables at
     every step and outputs on `check_frames` (all if None) for `rows` (all if None)."""
     dev = torch.device("cuda")
@@ -62,9 +62,13 @@ def run_parity(kvc, wl, frames, *, check_frames=None, rows=None, seed=0, layers=
         stats = []
         for t in range(frames):
             key = keyframe_schedule(t, wl.scale_frames, wl.keyframe_interval)
+            qkv = {l: st.frame(l, t) for l in layers}
+            if batched_append:
+                kvc.kvc_append_frame_all(h, t, [qkv[l][1] for l in layers], [qkv[l][2] for l in layers], key)
             for l in layers:
-                q, k, v = st.frame(l, t)
-                kvc.kvc_append_frame(h, l, t, k, v, key)
+                q, k, v = qkv[l]
+                if not batched_append:
+                    kvc.kvc_append_frame(h, l, t, k, v, key)
                 kvc.kvc_attend(h, l, q, out)
                 orc.append(l, t, np64(k), np64(v), key)
                 do_check = check_frames is None or t in check_frames

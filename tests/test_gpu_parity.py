@@ -46,6 +46,17 @@ def test_bf16_keyframes_two_layers(kvc):
     run_parity(kvc, wl, 16, check_pages=True)
 
 
+def test_batched_append_all_layers(kvc):
+    """kvc_append_frame_all (one allocation + one append launch for all layers) gives the
+    same page tables, pages and outputs as the oracle, bf16 with keyframes and FP8."""
+    wl = WORKLOADS["vggt_24layer_k4"].replace(num_layers=3, tokens_per_frame=200, num_heads=4,
+                                               window_frames=3, scale_frames=1)
+    run_parity(kvc, wl, 12, check_pages=True, batched_append=True)
+    wl8 = WORKLOADS["vggt_518x518_fp8"].replace(num_layers=2, tokens_per_frame=150, num_heads=4, window_frames=3,
+                                                scale_frames=1)
+    run_parity(kvc, wl8, 7, check_pages=True, batched_append=True)
+
+
 def test_fp8_small_codes_and_outputs(kvc):
     wl = WORKLOADS["vggt_518x518_fp8"].replace(tokens_per_frame=150, num_heads=4, window_frames=4, scale_frames=2)
     run_parity(kvc, wl, 9, check_pages=True)

@@ -27,7 +27,7 @@ STATUS = ["KVC_OK", "KVC_ERR_ARG", "KVC_ERR_OOM", "KVC_ERR_CUDA", "KVC_ERR_STATE
 EXPORTS = ["kvc_create", "kvc_destroy", "kvc_set_stream", "kvc_reset", "kvc_append_frame", "kvc_attend",
            "kvc_compress", "kvc_page_table", "kvc_token_meta", "kvc_last_merge", "kvc_export_pages",
            "kvc_step_host", "kvc_synchronize", "kvc_last_error", "kvc_status_string", "kvc_version",
-           "kvc_debug_fail_allocs", "kvc_debug_bounded_wait", "kvc_attend_paged_noalloc"]
+           "kvc_debug_fail_allocs", "kvc_debug_bounded_wait", "kvc_attend_paged_noalloc", "kvc_append_frame_all"]
 
 
 class kvc_config(ctypes.Structure):
@@ -71,6 +71,7 @@ def _load():
         "kvc_reset": ([vp], i32),
         "kvc_append_frame": ([vp, i32, i32, vp, vp, i32], i32),
         "kvc_attend": ([vp, i32, vp, vp], i32),
+        "kvc_append_frame_all": ([vp, i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32], i32),
         "kvc_compress": ([vp, i32, vp, i32p], i32),
         "kvc_page_table": ([vp, i32, i32p, i32, i32p, ctypes.POINTER(kvc_info)], i32),
         "kvc_token_meta": ([vp, i32, i64p, i32p, fp, i32, i32p], i32),
@@ -178,6 +179,14 @@ def kvc_reset(handle) -> None:
 
 def kvc_append_frame(handle, layer: int, frame_idx: int, k, v, is_keyframe: bool = True) -> None:
     _check(handle, _lib.kvc_append_frame(handle, layer, frame_idx, _ptr(k), _ptr(v), int(bool(is_keyframe))))
+
+
+def kvc_append_frame_all(handle, frame_idx: int, ks, vs, is_keyframe: bool = True) -> None:
+    """ks, vs: per-layer device tensors (or pointers), one per layer."""
+    n = len(ks)
+    ka = (ctypes.c_void_p * n)(*[_ptr(k) for k in ks])
+    va = (ctypes.c_void_p * n)(*[_ptr(v) for v in vs])
+    _check(handle, _lib.kvc_append_frame_all(handle, frame_idx, ka, va, int(bool(is_keyframe))))
 
 
 def kvc_attend(handle, layer: int, q, o) -> None:

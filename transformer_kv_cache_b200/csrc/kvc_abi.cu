@@ -338,6 +338,64 @@ kvc_status kvc_append_frame(kvc_cache* c, int32_t layer, int32_t frame_idx, cons
   return KVC_OK;
 }
 
+kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const void* const* k_devs,
+                                const void* const* v_devs, int32_t is_keyframe) {
+  if (!c) return KVC_ERR_ARG;
+  const kvc_config& g = c->cfg;
+  if (!k_devs || !v_devs || frame_idx < 0) return fail(c, KVC_ERR_ARG, "kvc_append_frame_all: bad argument");
+  const int n = c->ppf;
+  for (int l = 0; l < g.num_layers; ++l) {
+    if (!k_devs[l] || !v_devs[l] ||
+        ((reinterpret_cast<uintptr_t>(k_devs[l]) | reinterpret_cast<uintptr_t>(v_devs[l])) & 15))
+      return fail(c, KVC_ERR_ARG, "kvc_append_frame_all: K and V must be non-null and 16-byte aligned");
+    const LayerHost& L = c->L[l];
+    if (L.has_pending) return fail(c, KVC_ERR_STATE, "kvc_append_frame_all: a frame is already pending");
+    if (frame_idx <= L.last_frame) return fail(c, KVC_ERR_STATE, "kvc_append_frame_all: frame indices must increase");
+    if (L.n_entries + n > c->pool_pages) return fail(c, KVC_ERR_STATE, "kvc_append_frame_all: page pool full");
+  }
+  const int T = g.tokens_per_frame, P = g.page_size;
+  for (int l0 = 0; l0 < g.num_layers; l0 += kMaxBatchLayers) {
+    const int nl = std::min(kMaxBatchLayers, g.num_layers - l0);
+    LayerStarts st{};
+    AppendBatch in{};
+    st.first_layer = l0;
+    for (int b = 0; b < nl; ++b) {
+      st.start[b] = c->L[l0 + b].n_entries;
+      in.k[b] = k_devs[l0 + b];
+      in.v[b] = v_devs[l0 + b];
+    }
+    cudaError_t e = launch_mgr_alloc_layers(c->stream, c->entries, c->bitmap, c->bitmap_words, c->pool_pages, st, nl,
+                                            n, frame_idx, P, T - (n - 1) * P, c->d_err);
+    if (e != cudaSuccess) return cuda_fail(c, e, "page allocation (all layers)");
+    c->launches++;
+    if (g.kv_dtype == KVC_FP8_E4M3)
+      e = launch_append_fp8_layers(c->stream, in, st, nl, c->k_pool, c->v_pool, c->k_scale, c->v_scale, c->entries,
+                                   c->pool_pages, n, T, g.num_heads, g.head_dim, P);
+    else
+      e = launch_append_layers(c->stream, static_cast<int>(c->elem_kv), in, st, nl, c->k_pool, c->v_pool, c->entries,
+                               c->pool_pages, n, T, g.num_heads, g.head_dim, P);
+    if (e != cudaSuccess) return cuda_fail(c, e, "append (all layers)");
+    c->launches++;
+  }
+  for (int l = 0; l < g.num_layers; ++l) {
+    LayerHost& L = c->L[l];
+    if (g.budget_tokens > 0) {
+      kvc_status st = init_token_meta(c, l, L.n_entries, n, frame_idx);
+      if (st != KVC_OK) return st;
+    }
+    L.pending.frame = frame_idx;
+    L.pending.first_entry = L.n_entries;
+    L.pending.n_entries = n;
+    L.has_pending = true;
+    L.pending_key = is_keyframe != 0;
+    L.n_entries += n;
+    L.high_water = std::max<int64_t>(L.high_water, L.n_entries);
+    L.appended++;
+    L.last_frame = frame_idx;
+  }
+  return KVC_OK;
+}
+
 kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_dev) {
   if (!c) return KVC_ERR_ARG;
   if (!valid_layer(c, layer) || !q_dev || !o_dev) return fail(c, KVC_ERR_ARG, "kvc_attend: bad layer or pointer");

@@ -17,16 +17,21 @@
 
 namespace kvc {
 
-// One 16-byte chunk per thread-iteration; `vec` = elements per chunk.
-__global__ void append_kernel(const uint4* __restrict__ k_in, const uint4* __restrict__ v_in, uint4* k_pool,
-                              uint4* v_pool, const Entry* __restrict__ entries, int n_pages, int T, int H,
+// One 16-byte chunk per thread-iteration, over every (layer of the batch, tensor, page,
+// head, slot, chunk) in destination order.
+__global__ void append_kernel(AppendBatch in, LayerStarts starts, int n_layers, uint4* k_pool_all, uint4* v_pool_all,
+                              const Entry* __restrict__ entries_all, int pool_pages, int n_pages, int T, int H,
                               int chunks_per_row, int P) {
   const long long per_tensor = static_cast<long long>(n_pages) * H * P * chunks_per_row;
-  const long long total = 2 * per_tensor;
+  const long long per_layer = 2 * per_tensor;
+  const long long total = per_layer * n_layers;
+  const long long page_chunks = static_cast<long long>(H) * P * chunks_per_row;
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const bool is_v = idx >= per_tensor;
-    long long r = is_v ? idx - per_tensor : idx;
+    const int bl = static_cast<int>(idx / per_layer);
+    long long r = idx - static_cast<long long>(bl) * per_layer;
+    const bool is_v = r >= per_tensor;
+    if (is_v) r -= per_tensor;
     const int c = static_cast<int>(r % chunks_per_row);
     r /= chunks_per_row;
     const int slot = static_cast<int>(r % P);
@@ -34,12 +39,13 @@ __global__ void append_kernel(const uint4* __restrict__ k_in, const uint4* __res
     const int h = static_cast<int>(r % H);
     const int g = static_cast<int>(r / H);
     const int tok = g * P + slot;
-    const int phys = __ldg(&entries[g].x);
+    const long long layer = starts.first_layer + bl;
+    const int phys = __ldg(&entries_all[layer * pool_pages + starts.start[bl] + g].x);
     uint4 val = make_uint4(0, 0, 0, 0);
-    const uint4* src = is_v ? v_in : k_in;
+    const uint4* src = static_cast<const uint4*>(is_v ? in.v[bl] : in.k[bl]);
     if (tok < T) val = __ldg(&src[(static_cast<long long>(tok) * H + h) * chunks_per_row + c]);
-    uint4* dst = is_v ? v_pool : k_pool;
-    dst[((static_cast<long long>(phys) * H + h) * P + slot) * chunks_per_row + c] = val;
+    uint4* dst = (is_v ? v_pool_all : k_pool_all) + (layer * pool_pages + phys) * page_chunks;
+    dst[(static_cast<long long>(h) * P + slot) * chunks_per_row + c] = val;
   }
 }
 
@@ -50,27 +56,31 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   return r;
 }
 
-// One warp per (page, head, tensor). The block of valid tokens x D dims is reduced to its
-// absolute maximum; scale = fp32(amax / 448) with an IEEE-rounded division; each code is
-// the E4M3 rounding of the IEEE-rounded fp32 quotient x / scale; an all-zero block has
-// scale 0 and codes 0 ("XStreamVGGT" abstract: KV cache quantisation; OCP FP8 E4M3).
-// Requires D % 8 == 0 and P * D <= 32 * 64.
-__global__ void append_fp8_kernel(const __nv_bfloat16* __restrict__ k_in, const __nv_bfloat16* __restrict__ v_in,
-                                  uint8_t* k_pool, uint8_t* v_pool, float* k_scale, float* v_scale,
-                                  const Entry* __restrict__ entries, int n_pages, int T, int H, int D, int P) {
+// One warp per (layer of the batch, page, head, tensor). The block of valid tokens x D
+// dims is reduced to its absolute maximum; scale = fp32(amax / 448) with an IEEE-rounded
+// division; each code is the E4M3 rounding of the IEEE-rounded fp32 quotient x / scale; an
+// all-zero block has scale 0 and codes 0 ("XStreamVGGT" abstract: KV cache quantisation;
+// OCP FP8 E4M3). Requires D % 8 == 0 and P * D <= 32 * 64.
+__global__ void append_fp8_kernel(AppendBatch in, LayerStarts starts, int n_layers, uint8_t* k_pool_all,
+                                  uint8_t* v_pool_all, float* k_scale_all, float* v_scale_all,
+                                  const Entry* __restrict__ entries_all, int pool_pages, int n_pages, int T, int H,
+                                  int D, int P) {
   const int warps_per_block = blockDim.x / 32;
   const int gw = blockIdx.x * warps_per_block + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
-  const int n_items = n_pages * H * 2;
-  if (gw >= n_items) return;
-  const int tensor = gw % 2;
-  const int ph = gw / 2;
+  const int per_layer = n_pages * H * 2;
+  if (gw >= per_layer * n_layers) return;
+  const int bl = gw / per_layer;
+  const int item = gw % per_layer;
+  const int tensor = item % 2;
+  const int ph = item / 2;
   const int h = ph % H;
   const int g = ph / H;
-  const int phys = __ldg(&entries[g].x);
-  const __nv_bfloat16* src = tensor ? v_in : k_in;
-  uint8_t* dst = (tensor ? v_pool : k_pool) + (static_cast<long long>(phys) * H + h) * P * D;
-  float* sc = (tensor ? v_scale : k_scale) + static_cast<long long>(phys) * H + h;
+  const long long layer = starts.first_layer + bl;
+  const long long phys = layer * pool_pages + __ldg(&entries_all[layer * pool_pages + starts.start[bl] + g].x);
+  const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(tensor ? in.v[bl] : in.k[bl]);
+  uint8_t* dst = (tensor ? v_pool_all : k_pool_all) + (phys * H + h) * P * D;
+  float* sc = (tensor ? v_scale_all : k_scale_all) + phys * H + h;
   const int vec_per_row = D / 8;
   const int n_vec = P * vec_per_row;     // 8-element groups in the block
   // each lane handles groups lane, lane + 32, ... (at most 8 for P*D <= 2048)
@@ -121,29 +131,54 @@ __global__ void append_fp8_kernel(const __nv_bfloat16* __restrict__ k_in, const 
   }
 }
 
-cudaError_t launch_append(cudaStream_t s, int elem_bytes, const void* k, const void* v, void* k_pool,
-                          void* v_pool, const Entry* entries, int n_pages, int T, int H, int D, int P) {
+cudaError_t launch_append_layers(cudaStream_t s, int elem_bytes, const AppendBatch& in, const LayerStarts& starts,
+                                 int n_layers, void* k_pool_all, void* v_pool_all, const Entry* entries_all,
+                                 int pool_pages, int n_pages, int T, int H, int D, int P) {
   const int chunks_per_row = D * elem_bytes / 16;
-  const long long total = 2LL * n_pages * H * P * chunks_per_row;
+  const long long total = 2LL * n_layers * n_pages * H * P * chunks_per_row;
   const int threads = 256;
   long long blocks = (total + threads - 1) / threads;
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
-  append_kernel<<<static_cast<int>(blocks), threads, 0, s>>>(
-      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_pool),
-      static_cast<uint4*>(v_pool), entries, n_pages, T, H, chunks_per_row, P);
+  append_kernel<<<static_cast<int>(blocks), threads, 0, s>>>(in, starts, n_layers, static_cast<uint4*>(k_pool_all),
+                                                              static_cast<uint4*>(v_pool_all), entries_all, pool_pages,
+                                                              n_pages, T, H, chunks_per_row, P);
   return cudaGetLastError();
+}
+
+cudaError_t launch_append_fp8_layers(cudaStream_t s, const AppendBatch& in, const LayerStarts& starts, int n_layers,
+                                     uint8_t* k_pool_all, uint8_t* v_pool_all, float* k_scale_all,
+                                     float* v_scale_all, const Entry* entries_all, int pool_pages, int n_pages, int T,
+                                     int H, int D, int P) {
+  const int items = n_layers * n_pages * H * 2;
+  const int warps = 8;
+  append_fp8_kernel<<<(items + warps - 1) / warps, warps * 32, 0, s>>>(in, starts, n_layers, k_pool_all, v_pool_all,
+                                                                       k_scale_all, v_scale_all, entries_all,
+                                                                       pool_pages, n_pages, T, H, D, P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(cudaStream_t s, int elem_bytes, const void* k, const void* v, void* k_pool,
+                          void* v_pool, const Entry* entries, int n_pages, int T, int H, int D, int P) {
+  AppendBatch in{};
+  in.k[0] = k;
+  in.v[0] = v;
+  LayerStarts st{};
+  st.first_layer = 0;
+  st.start[0] = 0;
+  return launch_append_layers(s, elem_bytes, in, st, 1, k_pool, v_pool, entries, 0, n_pages, T, H, D, P);
 }
 
 cudaError_t launch_append_fp8(cudaStream_t s, const void* k, const void* v, uint8_t* k_pool, uint8_t* v_pool,
                               float* k_scale, float* v_scale, const Entry* entries, int n_pages, int T, int H,
                               int D, int P) {
-  const int items = n_pages * H * 2;
-  const int warps = 8;
-  append_fp8_kernel<<<(items + warps - 1) / warps, warps * 32, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), k_pool, v_pool, k_scale, v_scale,
-      entries, n_pages, T, H, D, P);
-  return cudaGetLastError();
+  AppendBatch in{};
+  in.k[0] = k;
+  in.v[0] = v;
+  LayerStarts st{};
+  st.first_layer = 0;
+  st.start[0] = 0;
+  return launch_append_fp8_layers(s, in, st, 1, k_pool, v_pool, k_scale, v_scale, entries, 0, n_pages, T, H, D, P);
 }
 
 }  // namespace kvc

@@ -96,9 +96,23 @@ struct kvc_cache : public kvc::Cache {};
 namespace kvc {
 
 // ------------------------------------------------------------------ launchers
+// Batched calls cover up to kMaxBatchLayers layers per launch (arrays passed by value).
+constexpr int kMaxBatchLayers = 64;
+struct LayerStarts {
+  int first_layer;
+  int start[kMaxBatchLayers];     // first page-table entry of the new frame, per layer of the batch
+};
+struct AppendBatch {
+  const void* k[kMaxBatchLayers];
+  const void* v[kMaxBatchLayers];
+};
+
 // Page-table manager (one CTA).
 cudaError_t launch_mgr_alloc(cudaStream_t s, Entry* entries, uint32_t* bitmap, int words, int pool_pages,
                              int start, int n_new, int owner, int valid_full, int valid_last, int* err);
+cudaError_t launch_mgr_alloc_layers(cudaStream_t s, Entry* entries_all, uint32_t* bitmap_all, int words,
+                                    int pool_pages, const LayerStarts& starts, int n_layers, int n_new, int owner,
+                                    int valid_full, int valid_last, int* err);
 cudaError_t launch_mgr_remove(cudaStream_t s, Entry* entries, uint32_t* bitmap, int n_entries, int a, int b,
                               int* err);
 cudaError_t launch_debug_wait(cudaStream_t s, int* flag, int* err, long long timeout_ns);
@@ -106,6 +120,15 @@ cudaError_t launch_debug_wait(cudaStream_t s, int* flag, int* err, long long tim
 // Append (same dtype in and out): K, V [T,H,D] -> pages of entries [0, n_pages).
 cudaError_t launch_append(cudaStream_t s, int elem_bytes, const void* k, const void* v, void* k_pool,
                           void* v_pool, const Entry* entries, int n_pages, int T, int H, int D, int P);
+// Batched append of one frame to layers [starts.first_layer, + n_layers): pools and
+// entries are the all-layer bases (pool_pages pages per layer).
+cudaError_t launch_append_layers(cudaStream_t s, int elem_bytes, const AppendBatch& in, const LayerStarts& starts,
+                                 int n_layers, void* k_pool_all, void* v_pool_all, const Entry* entries_all,
+                                 int pool_pages, int n_pages, int T, int H, int D, int P);
+cudaError_t launch_append_fp8_layers(cudaStream_t s, const AppendBatch& in, const LayerStarts& starts, int n_layers,
+                                     uint8_t* k_pool_all, uint8_t* v_pool_all, float* k_scale_all,
+                                     float* v_scale_all, const Entry* entries_all, int pool_pages, int n_pages, int T,
+                                     int H, int D, int P);
 // Append with FP8 E4M3 absmax quantisation per (page, head); bf16 input.
 cudaError_t launch_append_fp8(cudaStream_t s, const void* k, const void* v, uint8_t* k_pool, uint8_t* v_pool,
                               float* k_scale, float* v_scale, const Entry* entries, int n_pages, int T, int H,
