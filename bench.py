@@ -459,7 +459,9 @@ def run_workload(args):
                        "budget_tokens": wl.budget_tokens, "inputs": f"{distinct} seeded frames per layer, cycled",
                        "keyframes_timed": keys, "compressions_timed": fires},
             "clocks": clk.summary()}
-    app_bytes = 2 * 2 * T * H * D * 2 * L
+    # per layer: read K and V in bf16, write them as stored (bf16, or E4M3 codes + scales)
+    kv_elem = 1 if wl.kv_dtype == "fp8_e4m3" else 2
+    app_bytes = 2 * T * H * D * (2 + kv_elem) * L
     att_ms = statistics.mean(att)
     line["kernels"] = {
         "append_all_layers": {"bound": "hbm", "avg_ms": statistics.mean(app), "bytes_per_launch": app_bytes,

@@ -47,9 +47,10 @@ def compare_out(got: np.ndarray, ref: np.ndarray, io_dtype: str, what: str = "")
 
 
 def run_parity(kvc, wl, frames, *, check_frames=None, rows=None, seed=0, layers=None, kv_splits=0,
-               check_pages=False, record=None, batched_append=False):
+               check_pages=False, record=None, batched_append=False, transform=None):
     """Stream `frames` frames through the library and the oracle; compare page tables at
-    every step and outputs on `check_frames` (all if None) for `rows` (all if None)."""
+    every step and outputs on `check_frames` (all if None) for `rows` (all if None).
+    `transform(t, layer, q, k, v) -> (q, k, v)` edits a frame's inputs for both sides."""
     dev = torch.device("cuda")
     cfg = kvc.config_from_workload(wl, kv_splits=kv_splits)
     h = kvc.kvc_create(cfg)
@@ -63,6 +64,8 @@ def run_parity(kvc, wl, frames, *, check_frames=None, rows=None, seed=0, layers=
         for t in range(frames):
             key = keyframe_schedule(t, wl.scale_frames, wl.keyframe_interval)
             qkv = {l: st.frame(l, t) for l in layers}
+            if transform is not None:
+                qkv = {l: transform(t, l, *qkv[l]) for l in layers}
             if batched_append:
                 kvc.kvc_append_frame_all(h, t, [qkv[l][1] for l in layers], [qkv[l][2] for l in layers], key)
             for l in layers:

@@ -62,6 +62,49 @@ def test_fp8_small_codes_and_outputs(kvc):
     run_parity(kvc, wl, 9, check_pages=True)
 
 
+@pytest.mark.parametrize("T,H,splits", [
+    (300, 3, 1),     # one CTA per (q tile, head): every KV tile in one softmax pass
+    (300, 3, 3),     # three KV splits and the combine
+    (37, 2, 0),      # ragged q tile, partial last page of every frame
+])
+def test_fp8_tensor_core(kvc, T, H, splits):
+    """FP8 E4M3 storage on the tensor-core path (head dim 64, page size 16)."""
+    wl = WORKLOADS["vggt_518x518_fp8"].replace(tokens_per_frame=T, num_heads=H, window_frames=5, scale_frames=2,
+                                                num_special_tokens=min(5, T))
+    run_parity(kvc, wl, 10, kv_splits=splits, check_pages=True)
+
+
+def test_fp8_zero_blocks(kvc):
+    """All-zero K or V blocks quantise to scale 0 and codes 0; attention over them (the
+    first frame's K all zero, then a zero V frame, then both zero) matches the oracle."""
+    def zero(t, layer, q, k, v):
+        if t in (0, 3):
+            k = torch.zeros_like(k)
+        if t in (2, 3):
+            v = torch.zeros_like(v)
+        return q, k, v
+    wl = WORKLOADS["vggt_518x518_fp8"].replace(tokens_per_frame=150, num_heads=2, window_frames=4, scale_frames=1)
+    run_parity(kvc, wl, 7, check_pages=True, transform=zero)
+
+
+@pytest.mark.parametrize("D,P", [(32, 16), (64, 8)])
+def test_fp8_simt_shapes(kvc, D, P):
+    """FP8 storage with a head dim or page size the tensor-core kernel does not take."""
+    wl = WORKLOADS["vggt_518x518_fp8"].replace(tokens_per_frame=100, num_heads=2, head_dim=D, page_size=P,
+                                                window_frames=3, scale_frames=1, softmax_scale=D ** -0.5)
+    run_parity(kvc, wl, 6, check_pages=True)
+
+
+def test_fp8_full_size_steady_state_sampled(kvc):
+    """The 518x518 FP8 workload at full size past the window, sampled rows."""
+    wl = WORKLOADS["vggt_518x518_fp8"]
+    rows = sample_rows(wl.tokens_per_frame, 48, seed=2)
+    frames = wl.scale_frames + wl.window_frames + 2
+    check = {0, wl.scale_frames, wl.scale_frames + wl.window_frames, frames - 1}
+    stats = run_parity(kvc, wl, frames, check_frames=check, rows=rows)
+    assert len(stats) == len(check)
+
+
 def test_vggt_full_size_steady_state_sampled(kvc):
     """The 518x378 workload at full size past the window (eviction running), sampled rows."""
     wl = WORKLOADS["vggt_518x378"]

@@ -186,7 +186,7 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   c->page_bytes_kv = c->page_elems * c->elem_kv;
   const size_t L = g.num_layers;
   const size_t frame_bytes = static_cast<size_t>(T) * H * D * c->elem_io;
-  c->tc_path = g.io_dtype == KVC_BF16 && g.kv_dtype == KVC_BF16 && D == 64 && P == 16;
+  c->tc_path = g.io_dtype == KVC_BF16 && (g.kv_dtype == KVC_BF16 || g.kv_dtype == KVC_FP8_E4M3) && D == 64 && P == 16;
   const int q_tiles = (T + 127) / 128;
   c->part_rows = static_cast<size_t>(q_tiles) * H * 16;
 
@@ -251,8 +251,9 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
     c->tmap_k.resize(1);
     c->tmap_v.resize(1);
     const size_t rows = L * c->pool_pages * H * P;
-    if (!encode_pool_tmap(&c->tmap_k[0], c->k_pool, rows, D, P, 2, true) ||
-        !encode_pool_tmap(&c->tmap_v[0], c->v_pool, rows, D, P, 2, true)) {
+    const bool fp8 = g.kv_dtype == KVC_FP8_E4M3;
+    if (!encode_pool_tmap(&c->tmap_k[0], c->k_pool, rows, D, P, fp8 ? 1 : 2, !fp8) ||
+        !encode_pool_tmap(&c->tmap_v[0], c->v_pool, rows, D, P, fp8 ? 1 : 2, !fp8)) {
       free_all(c);
       delete c;
       return KVC_ERR_CUDA;
@@ -422,7 +423,9 @@ kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_de
     a.splits = g.kv_splits;
     a.tmap_k = &c->tmap_k[0];
     a.tmap_v = &c->tmap_v[0];
-    a.fp8 = false;
+    a.fp8 = g.kv_dtype == KVC_FP8_E4M3;
+    a.k_scale = c->k_scale;
+    a.v_scale = c->v_scale;
     a.part_o = c->part_o;
     a.part_lse = c->part_lse;
     a.part_rows = c->part_rows;

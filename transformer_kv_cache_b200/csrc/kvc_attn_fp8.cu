@@ -1,0 +1,506 @@
+// kvc_attn_fp8.cu -- frame attention over the paged FP8 E4M3 cache on sm_100a tensor cores.
+//
+// Same attention as kvc_attn_tc.cu ("How GCTStream ...", Frame-by-Frame Causal
+// Processing) over K/V stored as E4M3 codes with one absmax scale per (page, head)
+// ("XStreamVGGT" abstract: KV cache quantisation). The tensor cores multiply f16
+// operands (kind::f16 needs both operands of one type), so each KV tile is widened in
+// shared memory right after it lands:
+//
+//   warp 0              lane 0: TMA producer of the bf16 query tile (once) and, per 64-slot
+//                       KV tile, of the 4 page-head code blocks of K and of V (1 KB each)
+//                       into a three-stage staging ring. The whole warp converts: the query
+//                       tile bf16 -> f16 in place, then every code pair -> f16 pair with the
+//                       hardware E4M3 conversion (exact), written as a 128-byte-swizzled MMA
+//                       operand. K codes stay unscaled; each V pair is multiplied by the
+//                       page's V scale over the CTA's largest V scale of the head.
+//   warp 1 (one lane)   MMA issuer: S = Q K^T (M=128, N=64) and O' += P [V | 1] (M=128,
+//                       N=80), f16 inputs, fp32 accumulation in TMEM.
+//   warps 2..5          softmax: as in the bf16 kernel (one thread per row, 64 columns per
+//                       tile, lazy rescaling, row sum from the ones column), with P packed
+//                       as f16. The K scale of a page multiplies the logit factor of its 16
+//                       columns, so Q K^T runs on exact decoded codes.
+//
+// The epilogue multiplies by the V reference scale. Rounding V times s_page / s_ref to f16
+// is the only extra rounding of an operand (relative 2^-11). The query is held in f16,
+// which is exact for bf16 values of magnitude in [2^-14, 65504]. Every barrier wait is
+// bounded.
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include "kvc_attn_common.cuh"
+
+namespace kvc {
+namespace tc8 {
+constexpr int kBM = 128, kBN = 64, kHD = 64, kON = kHD + 16;
+constexpr int kStages = 3;
+constexpr int kCodeBytes = kBN * kHD;         // 4 KB of codes per K or V tile
+constexpr int kConvBytes = kBN * kHD * 2;     // 8 KB f16 tile
+constexpr int kQBytes = kBM * kHD * 2;        // 16 KB
+constexpr int kOnesBytes = kBN * kHD * 2;
+constexpr int kThreads = 192;
+constexpr int kConvThreads = 32;              // warp 0
+constexpr int kTmemCols = 256;
+constexpr int kColS = 0, kColP = 64, kColO = 128;
+constexpr float kPMax = 256.0f;
+constexpr size_t kSmemBytes =
+    1024 + kQBytes + 2 * kStages * kConvBytes + 2 * kStages * kCodeBytes + kOnesBytes + 512;
+}  // namespace tc8
+
+__device__ __forceinline__ uint32_t f16x2_of_e4m3x2(uint32_t code_pair) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(static_cast<uint16_t>(code_pair)));
+  return r;
+}
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t max_f16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float f16lo(uint32_t v) { return __half2float(__ushort_as_half(static_cast<uint16_t>(v))); }
+__device__ __forceinline__ float f16hi(uint32_t v) {
+  return __half2float(__ushort_as_half(static_cast<uint16_t>(v >> 16)));
+}
+__device__ __forceinline__ uint32_t f16x2_splat(float x) { return pack_f16(x, x); }
+
+template <int P>
+__global__ void __launch_bounds__(tc8::kThreads, 2)
+    attn_fp8_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                    const __grid_constant__ CUtensorMap tmap_v, const TcParams p) {
+  using namespace tc8;
+  constexpr int kPPT = kBN / P;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_s = smem;
+  uint8_t* ck_s = q_s + kQBytes;                       // converted K tiles [kStages]
+  uint8_t* cv_s = ck_s + kStages * kConvBytes;         // converted V tiles [kStages]
+  uint8_t* ones_s = cv_s + kStages * kConvBytes;
+  uint8_t* sk_s = ones_s + kOnesBytes;                 // K code staging [kStages]
+  uint8_t* sv_s = sk_s + kStages * kCodeBytes;         // V code staging [kStages]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sv_s + kStages * kCodeBytes);
+  uint64_t* q_full = bars;
+  uint64_t* q_ready = bars + 1;
+  uint64_t* c8_full = bars + 2;                        // [kStages] codes landed
+  uint64_t* kc_full = c8_full + kStages;               // [kStages] converted
+  uint64_t* kv_empty = kc_full + kStages;              // [kStages]
+  uint64_t* s_full = kv_empty + kStages;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_full = s_full + 2;                       // [2]
+  uint64_t* pv_done = s_full + 4;                      // [2]
+  uint64_t* mma_final = s_full + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* sref = reinterpret_cast<float*>(tmem_slot + 2);   // V reference scale
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x % p.q_tiles;
+  const int rest = blockIdx.x / p.q_tiles;
+  const int split = rest % p.splits;
+  const int h = rest / p.splits;
+  const int tile0 = split * p.tiles_per_split;
+  const int tile1 = min(tile0 + p.tiles_per_split, p.total_tiles);
+  const int n_tiles = tile1 - tile0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_ready, kConvThreads);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&c8_full[i], 1);
+      mbar_init(&kc_full[i], kConvThreads);
+      mbar_init(&kv_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
+    mbar_init(&p_full[0], 4);
+    mbar_init(&p_full[1], 4);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
+    mbar_init(mma_final, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  for (int i = threadIdx.x; i < kOnesBytes / 16; i += kThreads)
+    reinterpret_cast<uint4*>(ones_s)[i] = make_uint4(0x3c003c00u, 0x3c003c00u, 0x3c003c00u, 0x3c003c00u);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (n_tiles > 0) {
+    if (warp == 0) {
+      // ------------------------------------------------- TMA producer (lane 0) + converter
+      // V reference scale: the largest V scale of the head over this CTA's pages
+      float mv = 0.f;
+      for (int idx = tile0 * kPPT + lane; idx < min(tile1 * kPPT, p.n_pages); idx += 32)
+        mv = fmaxf(mv, __ldg(&p.v_scale[(p.page_base + __ldg(&p.entries[idx].x)) * p.H + h]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, o));
+      if (mv == 0.f) mv = 1.f;                          // all-zero pages: any reference works
+      const float iv = 1.f / mv;
+      if (lane == 0) *sref = mv;
+      // code blocks of tile t into code stage t % kStages (lane 0)
+      int last[kStages];
+#pragma unroll
+      for (int i = 0; i < kStages; ++i) last[i] = -1;
+      auto issue_codes = [&](int t) {
+        const int st = t % kStages;
+        mbar_arrive_expect_tx(&c8_full[st], 2 * kCodeBytes);
+#pragma unroll
+        for (int g = 0; g < kPPT; ++g) {
+          const int idx = (tile0 + t) * kPPT + g;
+          const int row = idx < p.n_pages ? static_cast<int>(((p.page_base + __ldg(&p.entries[idx].x)) * p.H + h) * P)
+                                          : p.pool_rows;
+          tma_load_2d(sk_s + st * kCodeBytes + g * P * kHD, &tmap_k, &c8_full[st], 0, row);
+          tma_load_2d(sv_s + st * kCodeBytes + g * P * kHD, &tmap_v, &c8_full[st], 0, row);
+        }
+        last[st] = t;
+      };
+      if (lane == 0) {
+        tma_prefetch_desc(&tmap_q);
+        tma_prefetch_desc(&tmap_k);
+        tma_prefetch_desc(&tmap_v);
+        mbar_arrive_expect_tx(q_full, kQBytes);
+        tma_load_3d(q_s, &tmap_q, q_full, 0, h, qt * kBM);
+        for (int t = 0; t < kStages && t < n_tiles; ++t) issue_codes(t);
+      }
+      __syncwarp();
+      // per-page V factors, loaded one tile ahead
+      float fv[kPPT];
+      auto load_fv = [&](int tile) {
+#pragma unroll
+        for (int g = 0; g < kPPT; ++g) {
+          const int idx = tile * kPPT + g;
+          fv[g] = idx < p.n_pages ? __ldg(&p.v_scale[(p.page_base + __ldg(&p.entries[idx].x)) * p.H + h]) * iv : 0.f;
+        }
+      };
+      load_fv(tile0);
+      bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(q_full, 0, abort_flag, p.err));
+      if (ok) {
+        // the query tile bf16 -> f16 in place (positions, hence the swizzle, unchanged)
+        uint32_t* q32 = reinterpret_cast<uint32_t*>(q_s);
+#pragma unroll 8
+        for (int i = lane; i < kQBytes / 4; i += 32) {
+          const uint32_t w = q32[i];
+          q32[i] = pack_f16(bf16lo(w), bf16hi(w));
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(q_ready);
+      }
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int st = j % kStages;
+        uint32_t rv[kPPT];
+#pragma unroll
+        for (int g = 0; g < kPPT; ++g) rv[g] = f16x2_splat(fv[g]);
+        if (j + 1 < n_tiles) load_fv(tile0 + j + 1);
+        // converted stage st is free once the MMAs of tile j - kStages have completed
+        if (j >= kStages &&
+            !__all_sync(0xffffffffu, mbar_wait_bounded(&kv_empty[st], ((j / kStages) - 1) & 1, abort_flag, p.err))) {
+          ok = false;
+          break;
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&c8_full[st], (j / kStages) & 1, abort_flag, p.err))) {
+          ok = false;
+          break;
+        }
+        const uint8_t* ksrc = sk_s + st * kCodeBytes;
+        const uint8_t* vsrc = sv_s + st * kCodeBytes;
+        uint8_t* kdst = ck_s + st * kConvBytes;
+        uint8_t* vdst = cv_s + st * kConvBytes;
+        // 64 rows x 8 chunks of 8 dims per tile and tensor; the code block of page g is
+        // rows [16g, 16g + 16) x 64 bytes, the f16 tile is 128-byte rows swizzled in 1 KB
+#pragma unroll 4
+        for (int q = lane; q < kBN * 8; q += 32) {
+          const int row = q >> 3, c = q & 7, g = row / P;
+          const uint2 kc = *reinterpret_cast<const uint2*>(ksrc + row * kHD + c * 8);
+          const uint2 vc = *reinterpret_cast<const uint2*>(vsrc + row * kHD + c * 8);
+          uint4 ko, vo;
+          ko.x = f16x2_of_e4m3x2(kc.x);
+          ko.y = f16x2_of_e4m3x2(kc.x >> 16);
+          ko.z = f16x2_of_e4m3x2(kc.y);
+          ko.w = f16x2_of_e4m3x2(kc.y >> 16);
+          vo.x = hmul2(f16x2_of_e4m3x2(vc.x), rv[g]);
+          vo.y = hmul2(f16x2_of_e4m3x2(vc.x >> 16), rv[g]);
+          vo.z = hmul2(f16x2_of_e4m3x2(vc.y), rv[g]);
+          vo.w = hmul2(f16x2_of_e4m3x2(vc.y >> 16), rv[g]);
+          const int off = row * 128 + ((c ^ (row & 7)) << 4);
+          *reinterpret_cast<uint4*>(kdst + off) = ko;
+          *reinterpret_cast<uint4*>(vdst + off) = vo;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(&kc_full[st]);
+        __syncwarp();
+        // code stage st has been read by the whole warp: refill it with tile j + kStages
+        if (lane == 0 && j + kStages < n_tiles) issue_codes(j + kStages);
+      }
+      if (lane == 0) {
+        mbar_wait_drain(q_full, 0, p.err);
+#pragma unroll
+        for (int i = 0; i < kStages; ++i)
+          if (last[i] >= 0) mbar_wait_drain(&c8_full[i], (last[i] / kStages) & 1, p.err);
+      }
+    } else if (warp == 1) {
+      if (lane == 0) {
+        // ---------------------------------------------------------------- MMA issuer
+        const uint32_t idesc_s = idesc_f16kind(0, kBM, kBN, 0, 0);
+        const uint32_t idesc_o = idesc_f16kind(0, kBM, kON, 0, 1);
+        const uint32_t tS = tmem + kColS, tP = tmem + kColP, tO = tmem + kColO;
+        const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(ck_s), v_addr = smem_u32(cv_s);
+        const uint32_t ones_addr = smem_u32(ones_s);
+        bool ok = mbar_wait_bounded(q_ready, 0, abort_flag, p.err) &&
+                  mbar_wait_bounded(&kc_full[0], 0, abort_flag, p.err);
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kHD / 16; ++kk)
+            mma_ss(tS, sw128_desc(q_addr + kk * 32, 16, 1024), sw128_desc(k_addr + kk * 32, 16, 1024), idesc_s,
+                   kk > 0);
+          mma_commit(s_full);
+        }
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const int st = j % kStages;
+          if (j + 1 < n_tiles) {
+            const int st1 = (j + 1) % kStages;
+            if (!mbar_wait_bounded(s_free, j & 1, abort_flag, p.err)) break;
+            if (!mbar_wait_bounded(&kc_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.err)) break;
+            tc_fence_after();
+            const uint32_t kb = k_addr + st1 * kConvBytes;
+#pragma unroll
+            for (int kk = 0; kk < kHD / 16; ++kk)
+              mma_ss(tS, sw128_desc(q_addr + kk * 32, 16, 1024), sw128_desc(kb + kk * 32, 16, 1024), idesc_s,
+                     kk > 0);
+            mma_commit(s_full);
+          }
+          if (!mbar_wait_bounded(&p_full[j & 1], (j >> 1) & 1, abort_flag, p.err)) break;
+          tc_fence_after();
+          const uint32_t vb = v_addr + st * kConvBytes;
+          const uint32_t lbo = ones_addr - vb;
+          const uint32_t pa = tP + (j & 1) * (kBN / 2);
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            mma_ts(tO, pa + kk * 8, sw128_desc(vb + kk * 2048, lbo, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&pv_done[j & 1]);
+          mma_commit(&kv_empty[st]);
+        }
+        mma_commit(mma_final);
+        mbar_wait_drain(mma_final, 0, p.err);
+      }
+    } else {
+      // ------------------------------------------------------------------ softmax warps
+      const int wq = warp & 3;
+      const int r = wq * 32 + lane;
+      const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+      const uint32_t tS = tmem + kColS + lane_off, tP = tmem + kColP + lane_off, tO = tmem + kColO + lane_off;
+      bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(q_ready, 0, abort_flag, p.err));
+      const float vref = ok ? *sref : 1.f;
+      float m = -INFINITY, masked = 0.f;
+      // per page of the next tile: the logit factor (log2 e x softmax scale x K scale) and
+      // the valid-slot count; pages past the list have factor 0 and no valid slots
+      float cgn[kPPT];
+      int vnext[kPPT];
+      auto load_tile = [&](int tile) {
+#pragma unroll
+        for (int g = 0; g < kPPT; ++g) {
+          const int idx = tile * kPPT + g;
+          cgn[g] = 0.f;
+          vnext[g] = 0;
+          if (idx < p.n_pages) {
+            const int4 e = __ldg(&p.entries[idx]);
+            cgn[g] = p.scale_log2 * __ldg(&p.k_scale[(p.page_base + e.x) * p.H + h]);
+            vnext[g] = e.w;
+          }
+        }
+      };
+      load_tile(tile0);
+      uint32_t s[2][32];
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(s_full, 0, abort_flag, p.err));
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(tS + 0, s[0]);
+        tmem_ld32(tS + 32, s[1]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+      }
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        int n_masked = 0;
+        float cg[kPPT];
+#pragma unroll
+        for (int g = 0; g < kPPT; ++g) {
+          n_masked += P - vnext[g];
+          cg[g] = cgn[g];
+        }
+        if (j + 1 < n_tiles) load_tile(tile0 + j + 1);
+        uint32_t pb[kBN / 2];
+        uint32_t mxb = 0u;
+        {
+          const uint64_t nm2 = pk2(-m, -m);
+#pragma unroll
+          for (int g = 0; g < kPPT; ++g) {
+            const uint64_t c2 = pk2(cg[g], cg[g]);
+#pragma unroll
+            for (int i = g * (P / 2); i < (g + 1) * (P / 2); ++i) {
+              float x0, x1;
+              up2(fma2_pair(s[(2 * i) / 32][(2 * i) % 32], s[(2 * i + 1) / 32][(2 * i + 1) % 32], c2, nm2), x0,
+                  x1);
+              pb[i] = pack_f16(ex2(x0), ex2(x1));
+              mxb = max_f16x2(mxb, pb[i]);
+            }
+          }
+        }
+        const bool move = (j == 0) || fmaxf(f16lo(mxb), f16hi(mxb)) > kPMax;
+        if (__any_sync(0xffffffffu, move)) {
+          // exact row maximum of the scaled logits: per page, the largest raw score times
+          // the page's (non-negative) factor
+          float mt = -INFINITY;
+#pragma unroll
+          for (int g = 0; g < kPPT; ++g) {
+            float ta = -INFINITY, tb = -INFINITY;
+#pragma unroll
+            for (int cc = g * P; cc < (g + 1) * P; cc += 4) {
+              ta = max3(ta, __uint_as_float(s[cc / 32][cc % 32]), __uint_as_float(s[cc / 32][cc % 32 + 1]));
+              tb = max3(tb, __uint_as_float(s[cc / 32][cc % 32 + 2]), __uint_as_float(s[cc / 32][cc % 32 + 3]));
+            }
+            mt = fmaxf(mt, fmaxf(ta, tb) * cg[g]);
+          }
+          const float m_new = move ? mt : m;
+          const bool resc = move && j > 0;
+          if (__any_sync(0xffffffffu, resc)) {
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait_bounded(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, p.err))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const float f = resc ? ex2(m - m_new) : 1.0f;
+            masked *= f;
+#pragma unroll
+            for (int q4 = 0; q4 < kON / 16; ++q4) {
+              uint32_t oc[16];
+              tmem_ld16(tO + q4 * 16, oc);
+              tmem_ld_wait();
+#pragma unroll
+              for (int d = 0; d < 16; ++d) oc[d] = __float_as_uint(__uint_as_float(oc[d]) * f);
+              tmem_st16(tO + q4 * 16, oc);
+            }
+          }
+          m = m_new;
+          const uint64_t nm2 = pk2(-m, -m);
+#pragma unroll
+          for (int g = 0; g < kPPT; ++g) {
+            const uint64_t c2 = pk2(cg[g], cg[g]);
+#pragma unroll
+            for (int i = g * (P / 2); i < (g + 1) * (P / 2); ++i) {
+              float x0, x1;
+              up2(fma2_pair(s[(2 * i) / 32][(2 * i) % 32], s[(2 * i + 1) / 32][(2 * i + 1) % 32], c2, nm2), x0,
+                  x1);
+              pb[i] = pack_f16(ex2(x0), ex2(x1));
+            }
+          }
+        }
+        // a masked slot holds zero codes: its score is 0 and its P entry is f16(2^-m)
+        if (n_masked) masked += static_cast<float>(n_masked) * f16lo(pack_f16(ex2(-m), 0.f));
+        if (j >= 2) {
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, p.err))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        tmem_st32(tP + (j & 1) * (kBN / 2), pb);
+        const bool more = j + 1 < n_tiles;
+        if (more) {
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_full, (j + 1) & 1, abort_flag, p.err))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          tmem_ld32(tS + 0, s[0]);
+          tmem_ld32(tS + 32, s[1]);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[j & 1]);
+        if (more) {
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free);
+        }
+      }
+      const int jl = n_tiles - 1;
+      if (__all_sync(0xffffffffu, ok && mbar_wait_bounded(&pv_done[jl & 1], (jl >> 1) & 1, abort_flag, p.err))) {
+        tc_fence_after();
+        uint32_t o0[32], o1[32], ls[16];
+        tmem_ld32(tO, o0);
+        tmem_ld32(tO + 32, o1);
+        tmem_ld16(tO + 64, ls);
+        tmem_ld_wait();
+        const float l = __uint_as_float(ls[0]) - masked;
+        const float inv = vref / l;
+        const int row = qt * kBM + r;
+        if (p.splits == 1) {
+          if (row < p.T) {
+            uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<long long>(row) * p.H + h) * kHD);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const uint32_t* src = v < 4 ? &o0[8 * v] : &o1[8 * (v - 4)];
+              uint4 w;
+              w.x = pack_bf16(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv);
+              w.y = pack_bf16(__uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv);
+              w.z = pack_bf16(__uint_as_float(src[4]) * inv, __uint_as_float(src[5]) * inv);
+              w.w = pack_bf16(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv);
+              dst[v] = w;
+            }
+          }
+        } else {
+          const long long pi = (static_cast<long long>(h) * p.splits + split) * p.q_tiles + qt;
+          float4* dst = reinterpret_cast<float4*>(p.part_o + (pi * kBM + r) * kHD);
+#pragma unroll
+          for (int v = 0; v < 16; ++v) {
+            const uint32_t* src = v < 8 ? &o0[4 * v] : &o1[4 * (v - 8)];
+            dst[v] = make_float4(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv,
+                                 __uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv);
+          }
+          p.part_lse[pi * kBM + r] = m + __log2f(l);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) {
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+cudaError_t launch_attn_fp8_kernel(cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                   const TcParams& prm, int grid) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fp8_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(tc8::kSmemBytes));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  attn_fp8_kernel<16><<<grid, tc8::kThreads, tc8::kSmemBytes, s>>>(tq, tk, tv, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace kvc

@@ -41,8 +41,7 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
-#include "kvc_internal.h"
-#include "sm100_ptx.cuh"
+#include "kvc_attn_common.cuh"
 
 namespace kvc {
 namespace tc {
@@ -60,73 +59,6 @@ constexpr int kColS = 0, kColP = 64, kColO = 128;
 constexpr float kPMax = 256.0f;               // a P above 2^8 moves the row's reference max
 constexpr size_t kSmemBytes = 1024 + kQBytes + 2 * kStages * kTileBytes + kOnesBytes + 256;
 }  // namespace tc
-
-struct TcParams {
-  const Entry* entries;
-  int n_pages, T, H;
-  int q_tiles, splits, tiles_per_split, total_tiles;
-  long long page_base;          // layer * pool_pages: first pool page of the layer
-  int pool_rows;                // rows of the pool tensor maps (a row index past the end reads zeros)
-  float scale_log2;
-  __nv_bfloat16* out;
-  float* part_o;
-  float* part_lse;
-  int* err;
-};
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// ---- packed arithmetic used by the softmax
-__device__ __forceinline__ uint64_t fma2_pair(uint32_t s0, uint32_t s1, uint64_t c2, uint64_t nm2) {
-  uint64_t x, r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(s0), "r"(s1));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(x), "l"(c2), "l"(nm2));
-  return r;
-}
-__device__ __forceinline__ uint64_t pk2(float a, float b) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void up2(uint64_t r, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
-}
-__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
-
-// Upper halves of two fp32 values as a bf16 pair (truncation toward zero), one byte
-// permute; P is consumed by the MMA and summed by it from the same bf16 values, so the
-// truncation's common scale cancels in O / l.
-__device__ __forceinline__ uint32_t bf16x2_trunc(float lo, float hi) {
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(__float_as_uint(lo)), "r"(__float_as_uint(hi)));
-  return r;
-}
-
-// Wait without the abort shortcut, used only to drain a CTA's own in-flight work.
-__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, int* err) {
-  volatile int never = 0;
-  mbar_wait_bounded(bar, parity, &never, err);
-}
 
 template <int P>
 __global__ void __launch_bounds__(tc::kThreads, 2)
@@ -571,9 +503,9 @@ int choose_splits(int units, int tiles, int slots) {
 
 cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used, int* launched) {
   if (launched) *launched = 0;
-  if (a.P != 16 || a.fp8) return cudaErrorInvalidValue;
+  if (a.P != 16) return cudaErrorInvalidValue;
   static bool attr_set = false;
-  if (!attr_set) {
+  if (!a.fp8 && !attr_set) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(tc::kSmemBytes));
     if (e != cudaSuccess) return e;
@@ -596,6 +528,8 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
     splits = (total_tiles + tps - 1) / tps;
   }
   TcParams prm;
+  prm.k_scale = a.k_scale;
+  prm.v_scale = a.v_scale;
   prm.entries = a.entries;
   prm.n_pages = a.n_pages;
   prm.T = a.T;
@@ -612,8 +546,13 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   prm.part_lse = a.part_lse;
   prm.err = a.err;
   const int grid = units * splits;
-  attn_tc_kernel<16><<<grid, tc::kThreads, tc::kSmemBytes, s>>>(tq, *a.tmap_k, *a.tmap_v, prm);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (a.fp8) {
+    e = launch_attn_fp8_kernel(s, tq, *a.tmap_k, *a.tmap_v, prm, grid);
+  } else {
+    attn_tc_kernel<16><<<grid, tc::kThreads, tc::kSmemBytes, s>>>(tq, *a.tmap_k, *a.tmap_v, prm);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
   if (launched) *launched = 1;
   if (splits > 1) {
