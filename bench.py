@@ -57,6 +57,9 @@ def parse():
     ap.add_argument("--kv-splits", type=int, default=0)
     ap.add_argument("--workload", default=WORKLOAD,
                     help="vggt_518x378 (default, the headline), vggt_24layer_k4, vggt_budget_16k, vggt_518x518_fp8")
+    ap.add_argument("--fill", type=int, default=0,
+                    help="frames streamed before warm-up for a non-default workload (0: enough to fill the window); "
+                         "smaller values give short cases for profiling")
     return ap.parse_args()
 
 
@@ -398,7 +401,9 @@ def run_workload(args):
     L, T, H, D, P = wl.num_layers, wl.tokens_per_frame, wl.num_heads, wl.head_dim, wl.page_size
     S, W, k = wl.scale_frames, wl.window_frames, wl.keyframe_interval
     budget = wl.budget_tokens > 0
-    if budget:
+    if args.fill > 0:
+        fill = args.fill
+    elif budget:
         fill = -(-wl.budget_tokens // T) + 3          # past the first compression of every layer
     else:
         fill = S + W * k                              # the window is full of keyframes
@@ -469,7 +474,7 @@ def run_workload(args):
                               "peak_gbs": float(peaks["hbm_gbs"])},
         "attention_all_layers": {"avg_ms": att_ms}}
     if not budget:
-        kv_tokens = (S + W + 1) * T
+        kv_tokens = info0["tokens"] + T               # the cache before the timed steps, plus the new frame
         flops = 4.0 * T * kv_tokens * H * D * L
         ach = flops / (att_ms * 1e-3) / 1e12
         line["roofline"] = {"bound": "tensor", "achieved": ach, "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",

@@ -32,7 +32,9 @@
 namespace kvc {
 namespace tc8 {
 constexpr int kBM = 128, kBN = 64, kHD = 64, kON = kHD + 16;
-constexpr int kStages = 3;
+constexpr int kCodeStages = 2;                // code staging ring (TMA destination)
+constexpr int kStages = 4;                    // converted f16 operand ring
+constexpr bool kEarlyPV = false;              // issue PV(j) while S(j+1) waits for its conversion
 constexpr int kCodeBytes = kBN * kHD;         // 4 KB of codes per K or V tile
 constexpr int kConvBytes = kBN * kHD * 2;     // 8 KB f16 tile
 constexpr int kQBytes = kBM * kHD * 2;        // 16 KB
@@ -43,7 +45,7 @@ constexpr int kTmemCols = 256;
 constexpr int kColS = 0, kColP = 64, kColO = 128;
 constexpr float kPMax = 256.0f;
 constexpr size_t kSmemBytes =
-    1024 + kQBytes + 2 * kStages * kConvBytes + 2 * kStages * kCodeBytes + kOnesBytes + 512;
+    1024 + kQBytes + 2 * kStages * kConvBytes + 2 * kCodeStages * kCodeBytes + kOnesBytes + 512;
 }  // namespace tc8
 
 __device__ __forceinline__ uint32_t f16x2_of_e4m3x2(uint32_t code_pair) {
@@ -71,6 +73,15 @@ __device__ __forceinline__ float f16hi(uint32_t v) {
 }
 __device__ __forceinline__ uint32_t f16x2_splat(float x) { return pack_f16(x, x); }
 
+// Page-table entry idx of the layer, or (-1, 0, 0, 0) past the end of the list.
+__device__ __forceinline__ int4 page_entry(const TcParams& p, int idx) {
+  return idx < p.n_pages ? __ldg(&p.entries[idx]) : make_int4(-1, 0, 0, 0);
+}
+// Scale of (physical page, head), 0 for the past-the-end sentinel.
+__device__ __forceinline__ float page_scale(const TcParams& p, const float* sc, int phys, int h) {
+  return phys >= 0 ? __ldg(&sc[(p.page_base + phys) * p.H + h]) : 0.f;
+}
+
 template <int P>
 __global__ void __launch_bounds__(tc8::kThreads, 2)
     attn_fp8_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -83,13 +94,13 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
   uint8_t* ck_s = q_s + kQBytes;                       // converted K tiles [kStages]
   uint8_t* cv_s = ck_s + kStages * kConvBytes;         // converted V tiles [kStages]
   uint8_t* ones_s = cv_s + kStages * kConvBytes;
-  uint8_t* sk_s = ones_s + kOnesBytes;                 // K code staging [kStages]
-  uint8_t* sv_s = sk_s + kStages * kCodeBytes;         // V code staging [kStages]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sv_s + kStages * kCodeBytes);
+  uint8_t* sk_s = ones_s + kOnesBytes;                 // K code staging [kCodeStages]
+  uint8_t* sv_s = sk_s + kCodeStages * kCodeBytes;     // V code staging [kCodeStages]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sv_s + kCodeStages * kCodeBytes);
   uint64_t* q_full = bars;
   uint64_t* q_ready = bars + 1;
-  uint64_t* c8_full = bars + 2;                        // [kStages] codes landed
-  uint64_t* kc_full = c8_full + kStages;               // [kStages] converted
+  uint64_t* c8_full = bars + 2;                        // [kCodeStages] codes landed
+  uint64_t* kc_full = c8_full + kCodeStages;           // [kStages] converted
   uint64_t* kv_empty = kc_full + kStages;              // [kStages]
   uint64_t* s_full = kv_empty + kStages;
   uint64_t* s_free = s_full + 1;
@@ -112,8 +123,8 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_ready, kConvThreads);
+    for (int i = 0; i < kCodeStages; ++i) mbar_init(&c8_full[i], 1);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&c8_full[i], 1);
       mbar_init(&kc_full[i], kConvThreads);
       mbar_init(&kv_empty[i], 1);
     }
@@ -141,52 +152,52 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
 
   if (n_tiles > 0) {
     if (warp == 0) {
-      // ------------------------------------------------- TMA producer (lane 0) + converter
+      // ------------------------------------------------------ TMA producer + converter
+      // Lanes 0..3 each track page g = lane of the tiles ahead (physical page, V scale), so
+      // no dependent global load sits on the conversion path.
+      const int gl = lane & 3;
       // V reference scale: the largest V scale of the head over this CTA's pages
       float mv = 0.f;
+#pragma unroll 4
       for (int idx = tile0 * kPPT + lane; idx < min(tile1 * kPPT, p.n_pages); idx += 32)
-        mv = fmaxf(mv, __ldg(&p.v_scale[(p.page_base + __ldg(&p.entries[idx].x)) * p.H + h]));
+        mv = fmaxf(mv, page_scale(p, p.v_scale, __ldg(&p.entries[idx].x), h));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, o));
       if (mv == 0.f) mv = 1.f;                          // all-zero pages: any reference works
       const float iv = 1.f / mv;
       if (lane == 0) *sref = mv;
-      // code blocks of tile t into code stage t % kStages (lane 0)
-      int last[kStages];
-#pragma unroll
-      for (int i = 0; i < kStages; ++i) last[i] = -1;
-      auto issue_codes = [&](int t) {
-        const int st = t % kStages;
-        mbar_arrive_expect_tx(&c8_full[st], 2 * kCodeBytes);
-#pragma unroll
-        for (int g = 0; g < kPPT; ++g) {
-          const int idx = (tile0 + t) * kPPT + g;
-          const int row = idx < p.n_pages ? static_cast<int>(((p.page_base + __ldg(&p.entries[idx].x)) * p.H + h) * P)
-                                          : p.pool_rows;
-          tma_load_2d(sk_s + st * kCodeBytes + g * P * kHD, &tmap_k, &c8_full[st], 0, row);
-          tma_load_2d(sv_s + st * kCodeBytes + g * P * kHD, &tmap_v, &c8_full[st], 0, row);
-        }
-        last[st] = t;
-      };
+      // Physical page g of tiles ahead and the V scale of the next tile. Every value loaded
+      // in iteration j is first used in iteration j + 1 (rotations happen at the loop top),
+      // so no copy waits on a load in flight.
+      const int pq0 = page_entry(p, tile0 * kPPT + gl).x;
+      int pq1 = page_entry(p, (tile0 + 1) * kPPT + gl).x;
+      int pq2 = page_entry(p, (tile0 + 2) * kPPT + gl).x;
+      int pq4n = page_entry(p, (tile0 + 3) * kPPT + gl).x;   // becomes pq3 at the loop top
+      float vsn = page_scale(p, p.v_scale, pq0, h);         // becomes the factor of tile j
+      // the code blocks of tile t (page gl's K and V from lanes 0..3) into stage t % kStages
+#define KVC_FP8_ISSUE(t, phys)                                                                    \
+  do {                                                                                            \
+    const int st_ = (t) % kCodeStages;                                                            \
+    if (lane == 0) mbar_arrive_expect_tx(&c8_full[st_], 2 * kCodeBytes);                          \
+    __syncwarp();                                                                                 \
+    if (lane < kPPT) {                                                                            \
+      const int row_ = (phys) >= 0 ? static_cast<int>(((p.page_base + (phys)) * p.H + h) * P) : p.pool_rows; \
+      tma_load_2d(sk_s + st_ * kCodeBytes + lane * P * kHD, &tmap_k, &c8_full[st_], 0, row_);     \
+      tma_load_2d(sv_s + st_ * kCodeBytes + lane * P * kHD, &tmap_v, &c8_full[st_], 0, row_);     \
+    }                                                                                             \
+  } while (0)
       if (lane == 0) {
         tma_prefetch_desc(&tmap_q);
         tma_prefetch_desc(&tmap_k);
         tma_prefetch_desc(&tmap_v);
         mbar_arrive_expect_tx(q_full, kQBytes);
         tma_load_3d(q_s, &tmap_q, q_full, 0, h, qt * kBM);
-        for (int t = 0; t < kStages && t < n_tiles; ++t) issue_codes(t);
       }
-      __syncwarp();
-      // per-page V factors, loaded one tile ahead
-      float fv[kPPT];
-      auto load_fv = [&](int tile) {
-#pragma unroll
-        for (int g = 0; g < kPPT; ++g) {
-          const int idx = tile * kPPT + g;
-          fv[g] = idx < p.n_pages ? __ldg(&p.v_scale[(p.page_base + __ldg(&p.entries[idx].x)) * p.H + h]) * iv : 0.f;
-        }
-      };
-      load_fv(tile0);
+      static_assert(kCodeStages == 2 || kCodeStages == 3, "code ring of 2 or 3 stages");
+      KVC_FP8_ISSUE(0, pq0);
+      if (n_tiles > 1) KVC_FP8_ISSUE(1, pq1);
+      if (kCodeStages == 3 && n_tiles > 2) KVC_FP8_ISSUE(2, pq2);
+      int issued = min(n_tiles, kCodeStages);
       bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(q_full, 0, abort_flag, p.err));
       if (ok) {
         // the query tile bf16 -> f16 in place (positions, hence the swizzle, unchanged)
@@ -199,57 +210,75 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive(q_ready);
       }
+      // per-lane constant parts of the conversion addresses: row (lane >> 3) + 4 i, chunk
+      // lane & 7 of 8 dims; in the swizzled f16 tile the chunk moves to chunk ^ (row & 7)
+      const int r0 = lane >> 3, c0 = lane & 7;
+      const int src_off = r0 * kHD + c0 * 8;
+      const int dst_even = r0 * 128 + ((c0 ^ r0) << 4);
+      const int dst_odd = r0 * 128 + ((c0 ^ r0 ^ 4) << 4);
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int st = j % kStages;
+        const float fvj = vsn * iv;                     // V factor of page g of tile j
+        const int pq3 = pq4n;                           // page g of tile j + 3
+        vsn = page_scale(p, p.v_scale, pq1, h);         // tile j + 1
+        pq4n = page_entry(p, (tile0 + j + 4) * kPPT + gl).x;
         uint32_t rv[kPPT];
 #pragma unroll
-        for (int g = 0; g < kPPT; ++g) rv[g] = f16x2_splat(fv[g]);
-        if (j + 1 < n_tiles) load_fv(tile0 + j + 1);
+        for (int g = 0; g < kPPT; ++g) rv[g] = f16x2_splat(__shfl_sync(0xffffffffu, fvj, g));
         // converted stage st is free once the MMAs of tile j - kStages have completed
         if (j >= kStages &&
             !__all_sync(0xffffffffu, mbar_wait_bounded(&kv_empty[st], ((j / kStages) - 1) & 1, abort_flag, p.err))) {
           ok = false;
           break;
         }
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&c8_full[st], (j / kStages) & 1, abort_flag, p.err))) {
+        const int cs = j % kCodeStages;
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&c8_full[cs], (j / kCodeStages) & 1, abort_flag, p.err))) {
           ok = false;
           break;
         }
-        const uint8_t* ksrc = sk_s + st * kCodeBytes;
-        const uint8_t* vsrc = sv_s + st * kCodeBytes;
+        const uint8_t* ksrc = sk_s + cs * kCodeBytes + src_off;
+        const uint8_t* vsrc = sv_s + cs * kCodeBytes + src_off;
         uint8_t* kdst = ck_s + st * kConvBytes;
         uint8_t* vdst = cv_s + st * kConvBytes;
-        // 64 rows x 8 chunks of 8 dims per tile and tensor; the code block of page g is
-        // rows [16g, 16g + 16) x 64 bytes, the f16 tile is 128-byte rows swizzled in 1 KB
-#pragma unroll 4
-        for (int q = lane; q < kBN * 8; q += 32) {
-          const int row = q >> 3, c = q & 7, g = row / P;
-          const uint2 kc = *reinterpret_cast<const uint2*>(ksrc + row * kHD + c * 8);
-          const uint2 vc = *reinterpret_cast<const uint2*>(vsrc + row * kHD + c * 8);
+#pragma unroll
+        for (int i = 0; i < kBN / 4; ++i) {            // row (lane >> 3) + 4 i, page i / 4
+          const uint2 kc = *reinterpret_cast<const uint2*>(ksrc + i * 4 * kHD);
+          const uint2 vc = *reinterpret_cast<const uint2*>(vsrc + i * 4 * kHD);
           uint4 ko, vo;
           ko.x = f16x2_of_e4m3x2(kc.x);
           ko.y = f16x2_of_e4m3x2(kc.x >> 16);
           ko.z = f16x2_of_e4m3x2(kc.y);
           ko.w = f16x2_of_e4m3x2(kc.y >> 16);
-          vo.x = hmul2(f16x2_of_e4m3x2(vc.x), rv[g]);
-          vo.y = hmul2(f16x2_of_e4m3x2(vc.x >> 16), rv[g]);
-          vo.z = hmul2(f16x2_of_e4m3x2(vc.y), rv[g]);
-          vo.w = hmul2(f16x2_of_e4m3x2(vc.y >> 16), rv[g]);
-          const int off = row * 128 + ((c ^ (row & 7)) << 4);
+          vo.x = hmul2(f16x2_of_e4m3x2(vc.x), rv[i >> 2]);
+          vo.y = hmul2(f16x2_of_e4m3x2(vc.x >> 16), rv[i >> 2]);
+          vo.z = hmul2(f16x2_of_e4m3x2(vc.y), rv[i >> 2]);
+          vo.w = hmul2(f16x2_of_e4m3x2(vc.y >> 16), rv[i >> 2]);
+          const int off = i * 512 + ((i & 1) ? dst_odd : dst_even);
           *reinterpret_cast<uint4*>(kdst + off) = ko;
           *reinterpret_cast<uint4*>(vdst + off) = vo;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive(&kc_full[st]);
         __syncwarp();
-        // code stage st has been read by the whole warp: refill it with tile j + kStages
-        if (lane == 0 && j + kStages < n_tiles) issue_codes(j + kStages);
+        // code stage cs has been read by the whole warp: refill it with tile j + kCodeStages
+        if (j + kCodeStages < n_tiles) {
+          KVC_FP8_ISSUE(j + kCodeStages, kCodeStages == 3 ? pq3 : pq2);
+          ++issued;
+        }
+        pq1 = pq2;
+        pq2 = pq3;
       }
+#undef KVC_FP8_ISSUE
+      // drain: the last code load issued into each stage (tile t = the largest issued t
+      // with t % kCodeStages == stage) has landed before the CTA exits
       if (lane == 0) {
         mbar_wait_drain(q_full, 0, p.err);
 #pragma unroll
-        for (int i = 0; i < kStages; ++i)
-          if (last[i] >= 0) mbar_wait_drain(&c8_full[i], (last[i] / kStages) & 1, p.err);
+        for (int i = 0; i < kCodeStages; ++i)
+          if (issued > i) {
+            const int t = i + kCodeStages * ((issued - 1 - i) / kCodeStages);
+            mbar_wait_drain(&c8_full[i], (t / kCodeStages) & 1, p.err);
+          }
       }
     } else if (warp == 1) {
       if (lane == 0) {
@@ -271,10 +300,47 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
         }
         for (int j = 0; ok && j < n_tiles; ++j) {
           const int st = j % kStages;
+          bool pv_issued = false;
+          // PV(j): O' += P(j) [V(j) | 1], then release P buffer j & 1 and operand stage st
+#define KVC_FP8_PV()                                                                                      \
+  do {                                                                                                    \
+    tc_fence_after();                                                                                     \
+    const uint32_t vb = v_addr + st * kConvBytes;                                                         \
+    const uint32_t lbo = ones_addr - vb;                                                                  \
+    const uint32_t pa = tP + (j & 1) * (kBN / 2);                                                         \
+    _Pragma("unroll") for (int kk = 0; kk < kBN / 16; ++kk)                                               \
+      mma_ts(tO, pa + kk * 8, sw128_desc(vb + kk * 2048, lbo, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u); \
+    mma_commit(&pv_done[j & 1]);                                                                          \
+    mma_commit(&kv_empty[st]);                                                                            \
+    pv_issued = true;                                                                                     \
+  } while (0)
           if (j + 1 < n_tiles) {
             const int st1 = (j + 1) % kStages;
             if (!mbar_wait_bounded(s_free, j & 1, abort_flag, p.err)) break;
-            if (!mbar_wait_bounded(&kc_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.err)) break;
+            if (kEarlyPV) {
+              // wait for the converted operands of tile j + 1; if P(j) is ready first, run
+              // PV(j) meanwhile (bounded like every wait)
+              const uint64_t t0 = globaltimer_ns();
+              bool got = false;
+              for (uint32_t i = 0;; ++i) {
+                if (!pv_issued && mbar_try_wait(&p_full[j & 1], (j >> 1) & 1)) KVC_FP8_PV();
+                if (mbar_try_wait(&kc_full[st1], ((j + 1) / kStages) & 1)) {
+                  got = true;
+                  break;
+                }
+                if ((i & 63u) == 63u) {
+                  if (*abort_flag) break;
+                  if (globaltimer_ns() - t0 > KVC_WAIT_LIMIT_NS) {
+                    *abort_flag = 1;
+                    latch_error(p.err, DERR_TIMEOUT);
+                    break;
+                  }
+                }
+              }
+              if (!got) break;
+            } else if (!mbar_wait_bounded(&kc_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.err)) {
+              break;
+            }
             tc_fence_after();
             const uint32_t kb = k_addr + st1 * kConvBytes;
 #pragma unroll
@@ -283,16 +349,11 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
                      kk > 0);
             mma_commit(s_full);
           }
-          if (!mbar_wait_bounded(&p_full[j & 1], (j >> 1) & 1, abort_flag, p.err)) break;
-          tc_fence_after();
-          const uint32_t vb = v_addr + st * kConvBytes;
-          const uint32_t lbo = ones_addr - vb;
-          const uint32_t pa = tP + (j & 1) * (kBN / 2);
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_ts(tO, pa + kk * 8, sw128_desc(vb + kk * 2048, lbo, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&pv_done[j & 1]);
-          mma_commit(&kv_empty[st]);
+          if (!pv_issued) {
+            if (!mbar_wait_bounded(&p_full[j & 1], (j >> 1) & 1, abort_flag, p.err)) break;
+            KVC_FP8_PV();
+          }
+#undef KVC_FP8_PV
         }
         mma_commit(mma_final);
         mbar_wait_drain(mma_final, 0, p.err);
@@ -306,24 +367,14 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
       bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(q_ready, 0, abort_flag, p.err));
       const float vref = ok ? *sref : 1.f;
       float m = -INFINITY, masked = 0.f;
-      // per page of the next tile: the logit factor (log2 e x softmax scale x K scale) and
-      // the valid-slot count; pages past the list have factor 0 and no valid slots
-      float cgn[kPPT];
-      int vnext[kPPT];
-      auto load_tile = [&](int tile) {
-#pragma unroll
-        for (int g = 0; g < kPPT; ++g) {
-          const int idx = tile * kPPT + g;
-          cgn[g] = 0.f;
-          vnext[g] = 0;
-          if (idx < p.n_pages) {
-            const int4 e = __ldg(&p.entries[idx]);
-            cgn[g] = p.scale_log2 * __ldg(&p.k_scale[(p.page_base + e.x) * p.H + h]);
-            vnext[g] = e.w;
-          }
-        }
-      };
-      load_tile(tile0);
+      // Lanes 0..3 hold page g = lane of the current tile (K scale, valid slots) and the
+      // entry of the next tile, loaded one tile ahead; every lane reads them by shuffle.
+      // Pages past the list have scale 0 and no valid slots.
+      const int gl = lane & 3;
+      int4 en = page_entry(p, tile0 * kPPT + gl);
+      float ksj = page_scale(p, p.k_scale, en.x, h);
+      int vj = en.w;
+      en = page_entry(p, (tile0 + 1) * kPPT + gl);
       uint32_t s[2][32];
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(s_full, 0, abort_flag, p.err));
       if (ok) {
@@ -337,13 +388,17 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
         int n_masked = 0;
-        float cg[kPPT];
+        float cg[kPPT];            // logit factor per page: log2(e) x softmax scale x K scale
 #pragma unroll
         for (int g = 0; g < kPPT; ++g) {
-          n_masked += P - vnext[g];
-          cg[g] = cgn[g];
+          n_masked += P - __shfl_sync(0xffffffffu, vj, g);
+          cg[g] = p.scale_log2 * __shfl_sync(0xffffffffu, ksj, g);
         }
-        if (j + 1 < n_tiles) load_tile(tile0 + j + 1);
+        if (j + 1 < n_tiles) {
+          ksj = page_scale(p, p.k_scale, en.x, h);
+          vj = en.w;
+          en = page_entry(p, (tile0 + j + 2) * kPPT + gl);
+        }
         uint32_t pb[kBN / 2];
         uint32_t mxb = 0u;
         {

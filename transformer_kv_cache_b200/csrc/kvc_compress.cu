@@ -30,8 +30,7 @@ namespace kvc {
 
 namespace {
 
-constexpr int kCosTile = 64;     // sources x targets per CTA in the cosine kernel
-constexpr int kCosK = 32;        // dims per shared-memory stage
+constexpr int kCosTile = 128;    // targets per tile of the merge-target screen
 
 struct Scratch {
   int64_t* ids;
@@ -46,12 +45,14 @@ struct Scratch {
   int32_t* counts;     // [0] N, [1] keep, [2] elig, [3] merge
   int32_t* target;     // index into elig, per merge source
   int32_t* order;      // merge sources sorted by (target, source)
-  float* ks;
-  float* ke;
-  double* ns;
+  __nv_bfloat16* ks;   // full keys of the merge sources [n_merge][H*D]
+  __nv_bfloat16* ke;   // full keys of the eligible targets [n_keep][H*D]
+  double* ns;          // fp64 key norms
   double* ne;
-  double* best_v;
-  int32_t* best_j;
+  float* inv_ns;       // fp32 inverse norms for the screen
+  float* inv_ne;
+  float* top_v;        // four best screened cosines per (source, target tile)
+  int32_t* top_j;
   float* s_raw;        // raw scores of the frame being scored [T]
   int64_t* last_src;   // [layers][merge cap]
   int64_t* last_dst;
@@ -97,12 +98,14 @@ size_t carve(const kvc_config& g, uint8_t* base, Scratch* s) {
   t.counts = reinterpret_cast<int32_t*>(take(16 * 4));
   t.target = reinterpret_cast<int32_t*>(take(c.n_merge * 4));
   t.order = reinterpret_cast<int32_t*>(take(c.n_merge * 4));
-  t.ks = reinterpret_cast<float*>(take(c.n_merge * c.hd * 4));
-  t.ke = reinterpret_cast<float*>(take(c.n_keep * c.hd * 4));
+  t.ks = reinterpret_cast<__nv_bfloat16*>(take(c.n_merge * c.hd * 2));
+  t.ke = reinterpret_cast<__nv_bfloat16*>(take(c.n_keep * c.hd * 2));
   t.ns = reinterpret_cast<double*>(take(c.n_merge * 8));
   t.ne = reinterpret_cast<double*>(take(c.n_keep * 8));
-  t.best_v = reinterpret_cast<double*>(take(c.n_merge * c.tiles * 8));
-  t.best_j = reinterpret_cast<int32_t*>(take(c.n_merge * c.tiles * 4));
+  t.inv_ns = reinterpret_cast<float*>(take(c.n_merge * 4));
+  t.inv_ne = reinterpret_cast<float*>(take(c.n_keep * 4));
+  t.top_v = reinterpret_cast<float*>(take(c.n_merge * c.tiles * 16));
+  t.top_j = reinterpret_cast<int32_t*>(take(c.n_merge * c.tiles * 16));
   t.s_raw = reinterpret_cast<float*>(take(static_cast<size_t>(g.tokens_per_frame) * 4));
   t.last_src = reinterpret_cast<int64_t*>(take(static_cast<size_t>(g.num_layers) * c.n_merge * 8));
   t.last_dst = reinterpret_cast<int64_t*>(take(static_cast<size_t>(g.num_layers) * c.n_merge * 8));
@@ -335,10 +338,12 @@ __global__ void __launch_bounds__(1024) tier_lists_kernel(Scratch sc, int N, int
 }
 
 // ------------------------------------------------------------------ merge targets
-// Full H*D keys of listed tokens as fp32 (bf16 values, exact) and their fp64 norms.
+// Full H*D keys of listed tokens (the stored bf16 values), their fp64 norms and fp32
+// inverse norms.
 __global__ void gather_keys_kernel(const int32_t* __restrict__ list, const int32_t* __restrict__ count, int cap,
                                    const int32_t* __restrict__ slot, const __nv_bfloat16* __restrict__ k_pool,
-                                   int H, int P, int D, float* __restrict__ out, double* __restrict__ norms) {
+                                   int H, int P, int D, __nv_bfloat16* __restrict__ out, double* __restrict__ norms,
+                                   float* __restrict__ inv_norms) {
   const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int n = min(*count, cap);
@@ -350,120 +355,17 @@ __global__ void gather_keys_kernel(const int32_t* __restrict__ list, const int32
   double acc = 0.0;
   for (int c = lane; c < HD; c += 32) {
     const int h = c / D, d = c % D;
-    const float x = __bfloat162float(k_pool[((phys * H + h) * P + s) * D + d]);
-    out[static_cast<long long>(w) * HD + c] = x;
-    acc = fma(static_cast<double>(x), static_cast<double>(x), acc);
+    const __nv_bfloat16 xb = k_pool[((phys * H + h) * P + s) * D + d];
+    out[static_cast<long long>(w) * HD + c] = xb;
+    const double x = static_cast<double>(__bfloat162float(xb));
+    acc = fma(x, x, acc);
   }
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (lane == 0) norms[w] = sqrt(acc);
-}
-
-// Cosine of every (source, eligible target) pair in fp64 (dot products accumulated in
-// ascending dimension order); each CTA reduces its 64x64 tile to the best target per
-// source (largest cosine, lowest target index on ties).
-__global__ void __launch_bounds__(256) cos_tile_kernel(const float* __restrict__ ks, const double* __restrict__ ns,
-                                                        const float* __restrict__ ke, const double* __restrict__ ne,
-                                                        const int32_t* __restrict__ counts, int cap_src, int cap_elig,
-                                                        int HD, double* __restrict__ best_v,
-                                                        int32_t* __restrict__ best_j, int tiles) {
-  __shared__ float a_sm[kCosK][kCosTile + 1];
-  __shared__ float b_sm[kCosK][kCosTile + 1];
-  __shared__ double red_v[kCosTile][16];
-  __shared__ int red_j[kCosTile][16];
-  const int n_src = min(counts[3], cap_src);
-  const int n_elig = min(counts[2], cap_elig);
-  const int s0 = blockIdx.y * kCosTile, e0 = blockIdx.x * kCosTile;
-  if (s0 >= n_src || e0 >= n_elig) return;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;   // 16 x 16 threads, 4 x 4 each
-  double acc[4][4];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
-  for (int k0 = 0; k0 < HD; k0 += kCosK) {
-    for (int idx = threadIdx.x; idx < kCosK * kCosTile; idx += blockDim.x) {
-      const int r = idx / kCosK, c = idx % kCosK;
-      const int si = s0 + r, ei = e0 + r;
-      a_sm[c][r] = si < n_src ? ks[static_cast<long long>(si) * HD + k0 + c] : 0.f;
-      b_sm[c][r] = ei < n_elig ? ke[static_cast<long long>(ei) * HD + k0 + c] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int c = 0; c < kCosK; ++c) {
-      double av[4], bv[4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a) av[a] = a_sm[c][ty * 4 + a];
-#pragma unroll
-      for (int b = 0; b < 4; ++b) bv[b] = b_sm[c][tx * 4 + b];
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fma(av[a], bv[b], acc[a][b]);
-    }
-    __syncthreads();
+  if (lane == 0) {
+    const double n = sqrt(acc);
+    norms[w] = n;
+    inv_norms[w] = static_cast<float>(1.0 / n);
   }
-  // per source row: best over this thread's 4 targets, then over the 16 threads of the row
-#pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int si = s0 + ty * 4 + a;
-    double bv = -INFINITY;
-    int bj = 0x7fffffff;
-    if (si < n_src) {
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int ei = e0 + tx * 4 + b;
-        if (ei < n_elig) {
-          const double cv = acc[a][b] / (ne[ei] * ns[si]);
-          if (cv > bv) {
-            bv = cv;
-            bj = ei;
-          }
-        }
-      }
-    }
-    red_v[ty * 4 + a][tx] = bv;
-    red_j[ty * 4 + a][tx] = bj;
-  }
-  __syncthreads();
-  if (threadIdx.x < kCosTile) {
-    const int r = threadIdx.x;
-    double bv = -INFINITY;
-    int bj = 0x7fffffff;
-    for (int t = 0; t < 16; ++t) {
-      const double v = red_v[r][t];
-      const int j = red_j[r][t];
-      if (v > bv || (v == bv && j < bj)) {
-        bv = v;
-        bj = j;
-      }
-    }
-    const int si = s0 + r;
-    if (si < n_src) {
-      best_v[static_cast<long long>(si) * tiles + blockIdx.x] = bv;
-      best_j[static_cast<long long>(si) * tiles + blockIdx.x] = bj;
-    }
-  }
-}
-
-__global__ void argmax_reduce_kernel(const double* __restrict__ best_v, const int32_t* __restrict__ best_j,
-                                     const int32_t* __restrict__ counts, int cap_src, int cap_elig, int tiles,
-                                     int32_t* __restrict__ target) {
-  const int si = blockIdx.x * blockDim.x + threadIdx.x;
-  const int n_src = min(counts[3], cap_src);
-  const int n_elig = min(counts[2], cap_elig);
-  if (si >= n_src) return;
-  const int nt = (n_elig + kCosTile - 1) / kCosTile;
-  double bv = -INFINITY;
-  int bj = 0;
-  for (int t = 0; t < nt; ++t) {
-    const double v = best_v[static_cast<long long>(si) * tiles + t];
-    const int j = best_j[static_cast<long long>(si) * tiles + t];
-    if (v > bv || (v == bv && j < bj)) {
-      bv = v;
-      bj = j;
-    }
-  }
-  target[si] = bj;
 }
 
 // Merge sources sorted by (target, source): rank by counting.
@@ -690,21 +592,18 @@ kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_
   int64_t* ldst = sc.last_dst + static_cast<size_t>(layer) * cp.n_merge;
   if (n_merge > 0) {
     gather_keys_kernel<<<(n_merge * 32 + 255) / 256, 256, 0, s>>>(sc.merge, sc.counts + 3, static_cast<int>(cp.n_merge),
-                                                                   sc.slot, kp, H, P, D, sc.ks, sc.ns);
+                                                                   sc.slot, kp, H, P, D, sc.ks, sc.ns, sc.inv_ns);
     ok();
     gather_keys_kernel<<<(n_keep_other * 32 + 255) / 256, 256, 0, s>>>(
-        sc.elig, sc.counts + 2, static_cast<int>(cp.n_keep), sc.slot, kp, H, P, D, sc.ke, sc.ne);
+        sc.elig, sc.counts + 2, static_cast<int>(cp.n_keep), sc.slot, kp, H, P, D, sc.ke, sc.ne, sc.inv_ne);
     ok();
-    dim3 grid((n_keep_other + kCosTile - 1) / kCosTile, (n_merge + kCosTile - 1) / kCosTile);
-    cos_tile_kernel<<<grid, 256, 0, s>>>(sc.ks, sc.ns, sc.ke, sc.ne, sc.counts, static_cast<int>(cp.n_merge),
-                                         static_cast<int>(cp.n_keep), HD, sc.best_v, sc.best_j,
-                                         static_cast<int>(cp.tiles));
-    ok();
-    argmax_reduce_kernel<<<(n_merge + 255) / 256, 256, 0, s>>>(sc.best_v, sc.best_j, sc.counts,
-                                                                static_cast<int>(cp.n_merge),
-                                                                static_cast<int>(cp.n_keep),
-                                                                static_cast<int>(cp.tiles), sc.target);
-    ok();
+    // merge targets: tensor-core screen, fp64 decision among the screened candidates
+    int launched = 0;
+    cudaError_t r = launch_merge_targets(s, sc.ks, sc.ke, sc.ns, sc.ne, sc.inv_ns, sc.inv_ne, n_merge, n_keep_other,
+                                         HD, sc.top_v, sc.top_j, static_cast<int>(cp.tiles), sc.target, c->d_err,
+                                         &launched);
+    if (r != cudaSuccess && e == cudaSuccess) e = r;
+    c->launches += launched;
     merge_order_kernel<<<(n_merge + 255) / 256, 256, 0, s>>>(sc.target, sc.counts, static_cast<int>(cp.n_merge),
                                                               sc.order);
     ok();

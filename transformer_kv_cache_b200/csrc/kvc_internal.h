@@ -1,6 +1,7 @@
 // kvc_internal.h -- host-side state of a kvc_cache and the launchers of every kernel.
 #pragma once
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -166,6 +167,13 @@ int choose_splits(int units, int tiles, int slots);
 
 // Tensor map for a pool: rows of D elements, box of P rows.
 bool encode_pool_tmap(CUtensorMap* map, void* base, size_t rows, int D, int P, int elem_bytes, bool swizzle128);
+
+// Merge targets (kvc_cos_tc.cu): for each of n_src source keys, the index of the eligible
+// target key of highest fp64 cosine (lowest index on ties), screened on the tensor cores.
+cudaError_t launch_merge_targets(cudaStream_t s, const __nv_bfloat16* ks, const __nv_bfloat16* ke,
+                                 const double* ns, const double* ne, const float* inv_ns, const float* inv_ne,
+                                 int n_src, int n_elig, int HD, float* top_v, int32_t* top_j, int tiles_n,
+                                 int32_t* target, int* err, int* launched);
 
 // Compression kernels.
 cudaError_t launch_score(cudaStream_t s, const float* residual, int T, int R, int layer_slot, int n_hist,
