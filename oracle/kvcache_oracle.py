@@ -396,7 +396,9 @@ class StreamOracle:
     def score(self, layer: int, t: int, residual: np.ndarray) -> np.ndarray:
         """Enhanced importance s_hat of frame t's tokens at ``layer``.
 
-        s_i: fp32 of sqrt(sum_c r_ic^2), the squares summed in fp64 in ascending c.
+        s_i: fp32 of sqrt(sum_c r_ic^2), the squares summed in fp64 per block of 32
+        consecutive channels (ascending c within the block), then the block sums in
+        ascending block order (the pages fix no summation order).
         R_i: rank of token i among the frame's T tokens, s descending, ties to the
         lower slot; history kept for the last n = min(W, number of layers scored
         this frame) layers and reset at each new frame. With N = T,
@@ -411,9 +413,13 @@ class StreamOracle:
         if t != self._rank_frame:
             self._rank_hist = {}
             self._rank_frame = t
+        R = r.shape[1]
         acc = np.zeros(T)
-        for c in range(r.shape[1]):
-            acc = acc + r[:, c] * r[:, c]
+        for b0 in range(0, R, 32):
+            blk = np.zeros(T)
+            for c in range(b0, min(b0 + 32, R)):
+                blk = blk + r[:, c] * r[:, c]
+            acc = acc + blk
         s = to_f32(np.sqrt(acc))
         order = sorted(range(T), key=lambda i: (-s[i], i))
         R = np.empty(T, np.int64)

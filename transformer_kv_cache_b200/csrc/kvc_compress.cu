@@ -38,13 +38,17 @@ struct Scratch {
   int32_t* slot;
   int32_t* cnt;
   uint8_t* prot;
-  int32_t* rank;
+  int32_t* page_off;   // first position of each page-table entry's tokens
   int32_t* keep;
   int32_t* elig;
   int32_t* merge;
-  int32_t* counts;     // [0] N, [1] keep, [2] elig, [3] merge
+  int32_t* counts;     // [0] N, [1] keep, [2] elig, [3] merge; [8..11] tier thresholds
   int32_t* target;     // index into elig, per merge source
   int32_t* order;      // merge sources sorted by (target, source)
+  int32_t* bucket;     // [n_keep + 1]: sources of target e are order[bucket[e] .. bucket[e+1])
+  int64_t* src_base;   // per entry of `order`: pool element offset of the source's (page, slot)
+  int32_t* src_cnt;    // per entry of `order`: the source's count
+  int32_t* cursor;     // [n_keep]
   __nv_bfloat16* ks;   // full keys of the merge sources [n_merge][H*D]
   __nv_bfloat16* ke;   // full keys of the eligible targets [n_keep][H*D]
   double* ns;          // fp64 key norms
@@ -91,13 +95,17 @@ size_t carve(const kvc_config& g, uint8_t* base, Scratch* s) {
   t.slot = reinterpret_cast<int32_t*>(take(c.n_max * 4));
   t.cnt = reinterpret_cast<int32_t*>(take(c.n_max * 4));
   t.prot = take(c.n_max);
-  t.rank = reinterpret_cast<int32_t*>(take(c.n_max * 4));
+  t.page_off = reinterpret_cast<int32_t*>(take(c.n_max * 4));
   t.keep = reinterpret_cast<int32_t*>(take(c.n_max * 4));
   t.elig = reinterpret_cast<int32_t*>(take(c.n_max * 4));
   t.merge = reinterpret_cast<int32_t*>(take(c.n_max * 4));
   t.counts = reinterpret_cast<int32_t*>(take(16 * 4));
   t.target = reinterpret_cast<int32_t*>(take(c.n_merge * 4));
   t.order = reinterpret_cast<int32_t*>(take(c.n_merge * 4));
+  t.bucket = reinterpret_cast<int32_t*>(take((c.n_keep + 1) * 4));
+  t.src_base = reinterpret_cast<int64_t*>(take(c.n_merge * 8));
+  t.src_cnt = reinterpret_cast<int32_t*>(take(c.n_merge * 4));
+  t.cursor = reinterpret_cast<int32_t*>(take(c.n_keep * 4));
   t.ks = reinterpret_cast<__nv_bfloat16*>(take(c.n_merge * c.hd * 2));
   t.ke = reinterpret_cast<__nv_bfloat16*>(take(c.n_keep * c.hd * 2));
   t.ns = reinterpret_cast<double*>(take(c.n_merge * 8));
@@ -116,6 +124,15 @@ size_t carve(const kvc_config& g, uint8_t* base, Scratch* s) {
 // fp64 -> bf16, round to nearest even, one rounding (written from the format's
 // definition: 8 significant bits, subnormal quantum 2^-133, overflow to infinity).
 __device__ __forceinline__ __nv_bfloat16 f64_to_bf16_rne(double x) {
+  // bf16 normal range (biased fp64 exponent 897..1150): round the 52 fraction bits to 7,
+  // to nearest even, on the bit pattern; a carry may raise the exponent (1151 = overflow)
+  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(x));
+  const int ex = static_cast<int>((b >> 52) & 0x7FF);
+  if (ex >= 897 && ex <= 1150) {
+    const unsigned long long r = (b + 0x0FFFFFFFFFFFull + ((b >> 45) & 1ull)) & ~0x1FFFFFFFFFFFull;
+    if (((r >> 52) & 0x7FF) > 1150) return __float2bfloat16_rn(x > 0 ? INFINITY : -INFINITY);
+    return __float2bfloat16_rn(static_cast<float>(__longlong_as_double(static_cast<long long>(r))));   // exact
+  }
   if (x == 0.0 || isnan(x) || isinf(x)) return __float2bfloat16_rn(static_cast<float>(x));
   int e = ilogb(x);                    // |x| in [2^e, 2^(e+1))
   int qe = e - 7;                      // quantum of 8 significant bits
@@ -126,30 +143,67 @@ __device__ __forceinline__ __nv_bfloat16 f64_to_bf16_rne(double x) {
 }
 
 // ------------------------------------------------------------------ scoring
-// s_i = fp32(sqrt(sum_c r_ic^2)); the squares (exact in fp64) are summed in ascending c.
+// s_i = fp32(sqrt(sum_c r_ic^2)); the squares (exact in fp64) are summed per block of 32
+// consecutive channels in ascending c, then the block sums in ascending block order. One
+// warp per token: lane b sums block b (its 32 channels are 8 float4 loads), lane 0 adds
+// the block sums in order; for more than 32 blocks the warp repeats per 32 blocks.
 __global__ void residual_norm_kernel(const float* __restrict__ r, int T, int R, float* __restrict__ s_out) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= T) return;
-  const float* row = r + static_cast<long long>(i) * R;
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= T) return;
+  const float* x = r + static_cast<long long>(row) * R;
+  const int nb = (R + 31) / 32;
   double acc = 0.0;
-  for (int c = 0; c < R; ++c) {
-    const double x = static_cast<double>(__ldg(&row[c]));
-    acc = __dadd_rn(acc, __dmul_rn(x, x));
+  for (int b0 = 0; b0 < nb; b0 += 32) {
+    const int b = b0 + lane;
+    double blk = 0.0;
+    if (b < nb) {
+      const int c0 = b * 32, n = min(32, R - c0);
+      if (n == 32 && (R & 3) == 0 && (reinterpret_cast<uintptr_t>(r) & 15) == 0) {
+        float v[32];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 f = __ldg(reinterpret_cast<const float4*>(x + c0) + q);
+          v[4 * q] = f.x;
+          v[4 * q + 1] = f.y;
+          v[4 * q + 2] = f.z;
+          v[4 * q + 3] = f.w;
+        }
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const double y = static_cast<double>(v[c]);
+          blk = __dadd_rn(blk, __dmul_rn(y, y));
+        }
+      } else {
+        for (int c = 0; c < n; ++c) {
+          const double y = static_cast<double>(__ldg(x + c0 + c));
+          blk = __dadd_rn(blk, __dmul_rn(y, y));
+        }
+      }
+    }
+    const int nin = min(32, nb - b0);
+    for (int q = 0; q < nin; ++q) {
+      const double pq = __shfl_sync(0xffffffffu, blk, q);
+      acc = __dadd_rn(acc, pq);
+    }
   }
-  s_out[i] = __double2float_rn(__dsqrt_rn(acc));
+  if (lane == 0) s_out[row] = __double2float_rn(__dsqrt_rn(acc));
 }
 
 // Ranks of the frame's T tokens (s descending, ties to the lower slot), stored in the
 // history slot of this layer; then, over the window layers in `mask`, the population
 // variance of the normalised ranks gives Cons and s_hat, written next to the tokens.
-__global__ void __launch_bounds__(1024) clces_kernel(const float* __restrict__ s, int T, int32_t* hist, int slot,
-                                                      uint32_t mask, int n_win, float lam,
-                                                      const Entry* __restrict__ frame_pages, int P,
-                                                      float* __restrict__ tok_shat_layer) {
+// One thread per token (every token reads all T scores from shared memory); a token's
+// Cons needs only its own ranks, so the CTAs are independent.
+__global__ void __launch_bounds__(128) clces_kernel(const float* __restrict__ s, int T, int32_t* hist, int slot,
+                                                     uint32_t mask, int n_win, float lam,
+                                                     const Entry* __restrict__ frame_pages, int P,
+                                                     float* __restrict__ tok_shat_layer) {
   extern __shared__ float s_sm[];
   for (int i = threadIdx.x; i < T; i += blockDim.x) s_sm[i] = s[i];
   __syncthreads();
-  for (int i = threadIdx.x; i < T; i += blockDim.x) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < T) {
     const float si = s_sm[i];
     int r = 0;
     for (int j = 0; j < T; ++j) {
@@ -158,10 +212,9 @@ __global__ void __launch_bounds__(1024) clces_kernel(const float* __restrict__ s
     }
     hist[slot * T + i] = r;
   }
-  __syncthreads();
   const double sqrt12 = __dsqrt_rn(12.0);
   const double lamd = static_cast<double>(lam);
-  for (int i = threadIdx.x; i < T; i += blockDim.x) {
+  if (i < T) {
     long long sr = 0, sr2 = 0;
     for (int k = 0; k < 32; ++k) {
       if (mask & (1u << k)) {
@@ -196,64 +249,75 @@ __global__ void meta_init_kernel(int64_t* tok_id, int32_t* tok_cnt, float* tok_s
   tok_shat[k] = 0.f;
 }
 
+// Exclusive scan of v over the CTA (blockDim.x a multiple of 32, at most 1024); *total
+// receives the CTA-wide sum. s_warp holds 32 ints.
+__device__ __forceinline__ int cta_exclusive_scan(int v, int* s_warp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nw ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  const int excl = (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
+  *total = s_warp[nw - 1];
+  __syncthreads();
+  return excl;
+}
+
 // ------------------------------------------------------------------ tiering
 // Flatten the cache into position order (page-table order, valid slots only; positions
-// ascend with token id) with the metadata each later step needs.
-__global__ void __launch_bounds__(1024) gather_meta_kernel(const Entry* __restrict__ entries, int n_entries, int P,
-                                                            const int64_t* __restrict__ tok_id,
-                                                            const int32_t* __restrict__ tok_cnt,
-                                                            const float* __restrict__ tok_shat, int T, int specials,
-                                                            int protect_first, Scratch sc) {
+// ascend with token id) with the metadata each later step needs: a one-CTA scan of the
+// entries' valid counts gives each entry's first position, then one thread per slot.
+__global__ void __launch_bounds__(1024) page_offsets_kernel(const Entry* __restrict__ entries, int n_entries,
+                                                             Scratch sc) {
   __shared__ int s_warp[32];
-  __shared__ int s_base;
-  if (threadIdx.x == 0) s_base = 0;
-  __syncthreads();
+  int base = 0;
   for (int chunk = 0; chunk < n_entries; chunk += blockDim.x) {
     const int e = chunk + threadIdx.x;
     const int v = e < n_entries ? entries[e].w : 0;
-    // block exclusive scan of v
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) s_warp[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-      int w = lane < static_cast<int>(blockDim.x >> 5) ? s_warp[lane] : 0;
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, w, o);
-        if (lane >= o) w += y;
-      }
-      s_warp[lane] = w;
-    }
-    __syncthreads();
-    const int pos0 = s_base + (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
-    const int total = s_warp[(blockDim.x >> 5) - 1];
-    if (e < n_entries) {
-      const int phys = entries[e].x;
-      for (int s = 0; s < v; ++s) {
-        const int pos = pos0 + s;
-        const long long k = static_cast<long long>(phys) * P + s;
-        const int64_t id = tok_id[k];
-        sc.ids[pos] = id;
-        sc.shat[pos] = tok_shat[k];
-        sc.cnt[pos] = tok_cnt[k];
-        sc.slot[pos] = static_cast<int32_t>(k);
-        const int64_t frame = id / T, tslot = id % T;
-        sc.prot[pos] = (tslot < specials) || (protect_first && frame == 0);
-      }
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) s_base += total;
-    __syncthreads();
+    int total;
+    const int excl = cta_exclusive_scan(v, s_warp, &total);
+    if (e < n_entries) sc.page_off[e] = base + excl;
+    base += total;
   }
-  if (threadIdx.x == 0) sc.counts[0] = s_base;
+  if (threadIdx.x == 0) sc.counts[0] = base;
 }
 
-// Order of the non-protected tokens by (s_hat descending, id ascending), as a rank found
-// by counting: positions ascend with id, so (key, position) is a strict total order.
+__global__ void gather_meta_kernel(const Entry* __restrict__ entries, int n_entries, int P,
+                                   const int64_t* __restrict__ tok_id, const int32_t* __restrict__ tok_cnt,
+                                   const float* __restrict__ tok_shat, int T, int specials, int protect_first,
+                                   Scratch sc) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n_entries * P) return;
+  const int e = idx / P, sl = idx % P;
+  const Entry en = entries[e];
+  if (sl >= en.w) return;
+  const int pos = sc.page_off[e] + sl;
+  const long long k = static_cast<long long>(en.x) * P + sl;
+  const int64_t id = tok_id[k];
+  sc.ids[pos] = id;
+  sc.shat[pos] = tok_shat[k];
+  sc.cnt[pos] = tok_cnt[k];
+  sc.slot[pos] = static_cast<int32_t>(k);
+  const int64_t frame = id / T, tslot = id % T;
+  sc.prot[pos] = (tslot < specials) || (protect_first && frame == 0);
+}
+
+// Order of the non-protected tokens by (s_hat descending, id ascending): positions ascend
+// with id, so (key, position) with the key below is a strict total order.
 __device__ __forceinline__ uint32_t desc_key(float f) {
   // maps larger floats to smaller unsigned keys (total order on finite values)
   uint32_t u = __float_as_uint(f);
@@ -261,80 +325,151 @@ __device__ __forceinline__ uint32_t desc_key(float f) {
   return ~u;
 }
 
-__global__ void tier_rank_kernel(Scratch sc, int N) {
-  extern __shared__ uint32_t keys_sm[];   // [chunk]
-  uint8_t* prot_sm = reinterpret_cast<uint8_t*>(keys_sm + 2048);
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  const bool mine = i < N && !sc.prot[i];
-  const uint32_t ki = i < N ? desc_key(sc.shat[i]) : 0u;
-  int r = 0;
-  for (int base = 0; base < N; base += 2048) {
-    const int n = min(2048, N - base);
+// The k-th smallest (key, position) pair of the non-protected tokens for k = k1 and
+// k = k2, by MSB-first radix selection on the 32-bit key (8 bits per pass); positions
+// break ties, so the pair is fixed by the key value v and how many tokens of key v (in
+// position order) come before it. Writes, per k: counts[8 + 2q] = v and counts[9 + 2q]
+// = that number (a token of key v is among the k smallest iff its index among the
+// non-protected tokens of key v is below it). k <= 0 selects nothing, k >= the number
+// of non-protected tokens selects everything.
+__global__ void __launch_bounds__(1024) tier_select_kernel(Scratch sc, int N, int k1, int k2) {
+  __shared__ int hist[2][256];
+  __shared__ uint32_t s_prefix[2];
+  __shared__ int s_krem[2];
+  __shared__ int s_np;
+  __shared__ int s_warp[32];
+  int np_local = 0;
+  for (int i = threadIdx.x; i < N; i += blockDim.x) np_local += !sc.prot[i];
+  int n_np;
+  cta_exclusive_scan(np_local, s_warp, &n_np);
+  if (threadIdx.x == 0) {
+    s_np = n_np;
+    s_prefix[0] = s_prefix[1] = 0u;
+    s_krem[0] = k1;
+    s_krem[1] = k2;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = threadIdx.x; b < 512; b += blockDim.x) hist[b >> 8][b & 255] = 0;
     __syncthreads();
-    for (int j = threadIdx.x; j < n; j += blockDim.x) {
-      keys_sm[j] = desc_key(sc.shat[base + j]);
-      prot_sm[j] = sc.prot[base + j];
-    }
-    __syncthreads();
-    if (mine) {
-      for (int j = 0; j < n; ++j) {
-        const uint32_t kj = keys_sm[j];
-        const int pj = base + j;
-        r += !prot_sm[j] && (kj < ki || (kj == ki && pj < i));
+    const uint32_t hi_mask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+    const uint32_t p0 = s_prefix[0], p1 = s_prefix[1];
+    for (int base = 0; base < N; base += blockDim.x) {
+      const int i = base + threadIdx.x;
+      bool np = false;
+      uint32_t key = 0;
+      if (i < N) {
+        np = !sc.prot[i];
+        key = desc_key(sc.shat[i]);
+      }
+      const int digit = (key >> shift) & 255;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const bool in = np && ((key & hi_mask) == ((q ? p1 : p0) & hi_mask));
+        const uint32_t act = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          // one shared atomic per distinct digit of the warp
+          const uint32_t peers = __match_any_sync(act, digit);
+          if (lane == __ffs(peers) - 1) atomicAdd(&hist[q][digit], __popc(peers));
+        }
       }
     }
+    __syncthreads();
+    if (warp < 2) {
+      const int q = warp;
+      const int kr = s_krem[q];
+      // lane owns digits [8 lane, 8 lane + 8)
+      int c8[8], sum = 0;
+#pragma unroll
+      for (int d = 0; d < 8; ++d) {
+        c8[d] = hist[q][lane * 8 + d];
+        sum += c8[d];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int before = incl - sum;
+      int found = -1, krem_new = 0;
+      if (kr >= 1 && before < kr && kr <= incl) {
+#pragma unroll
+        for (int d = 0; d < 8; ++d) {
+          if (found < 0 && kr <= before + c8[d]) {
+            found = lane * 8 + d;
+            krem_new = kr - before;
+          }
+          before += c8[d];
+        }
+      }
+      if (found >= 0) {
+        s_prefix[q] |= static_cast<uint32_t>(found) << shift;
+        s_krem[q] = krem_new;
+      }
+    }
+    __syncthreads();
   }
-  if (i < N) sc.rank[i] = mine ? r : -1;
+  if (threadIdx.x < 2) {
+    const int q = threadIdx.x;
+    const int k = q ? k2 : k1;
+    uint32_t v = s_prefix[q];
+    int need = s_krem[q];
+    if (k <= 0) {
+      v = 0u;                 // nothing is below key 0 and no index is below 0
+      need = 0;
+    } else if (k >= s_np) {
+      v = 0xFFFFFFFFu;        // everything: every key is <= v, every index below N
+      need = 0x7fffffff;
+    }
+    sc.counts[8 + 2 * q] = static_cast<int32_t>(v);
+    sc.counts[9 + 2 * q] = need;
+  }
 }
 
-// Tier lists in position order: keep (protected or rank < n_keep_other), eligible
-// targets (kept, not protected) and merge sources (next n_merge ranks).
-__global__ void __launch_bounds__(1024) tier_lists_kernel(Scratch sc, int N, int n_keep_other, int n_merge) {
-  __shared__ int s_warp[3][32];
-  __shared__ int s_base[3];
-  if (threadIdx.x < 3) s_base[threadIdx.x] = 0;
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+// Tier lists in position order: keep (protected, or among the n_keep_other smallest
+// (key, position) pairs), eligible targets (kept, not protected) and merge sources (the
+// next n_merge). Per chunk, two scans give each token its index among the non-protected
+// tokens of the threshold keys, three more place the tokens in the lists.
+__global__ void __launch_bounds__(1024) tier_lists_kernel(Scratch sc, int N) {
+  __shared__ int s_warp[32];
+  const uint32_t v1 = static_cast<uint32_t>(sc.counts[8]), v2 = static_cast<uint32_t>(sc.counts[10]);
+  const int need1 = sc.counts[9], need2 = sc.counts[11];
+  int eq_base[2] = {0, 0}, list_base[3] = {0, 0, 0};
+  int* lists[3] = {sc.keep, sc.elig, sc.merge};
   for (int chunk = 0; chunk < N; chunk += blockDim.x) {
     const int i = chunk + threadIdx.x;
-    int f[3] = {0, 0, 0};
+    bool p = true;
+    uint32_t key = 0;
     if (i < N) {
-      const bool p = sc.prot[i];
-      const int r = sc.rank[i];
-      f[0] = p || (r < n_keep_other);
-      f[1] = !p && r < n_keep_other;
-      f[2] = !p && r >= n_keep_other && r < n_keep_other + n_merge;
+      p = sc.prot[i];
+      key = desc_key(sc.shat[i]);
     }
-    int x[3];
+    const bool e1 = !p && key == v1, e2 = !p && key == v2;
+    int tot;
+    const int x1 = eq_base[0] + cta_exclusive_scan(e1, s_warp, &tot);
+    eq_base[0] += tot;
+    const int x2 = eq_base[1] + cta_exclusive_scan(e2, s_warp, &tot);
+    eq_base[1] += tot;
+    const bool lt1 = !p && (key < v1 || (e1 && x1 < need1));
+    const bool lt2 = !p && (key < v2 || (e2 && x2 < need2));
+    int f[3];
+    f[0] = i < N && (p || lt1);
+    f[1] = i < N && lt1;
+    f[2] = i < N && !lt1 && lt2;
+#pragma unroll
     for (int q = 0; q < 3; ++q) {
-      x[q] = f[q];
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x[q], o);
-        if (lane >= o) x[q] += y;
-      }
-      if (lane == 31) s_warp[q][warp] = x[q];
+      const int x = cta_exclusive_scan(f[q], s_warp, &tot);
+      if (f[q]) lists[q][list_base[q] + x] = i;
+      list_base[q] += tot;
     }
-    __syncthreads();
-    if (warp == 0) {
-      for (int q = 0; q < 3; ++q) {
-        int w = lane < nw ? s_warp[q][lane] : 0;
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, w, o);
-          if (lane >= o) w += y;
-        }
-        s_warp[q][lane] = w;
-      }
-    }
-    __syncthreads();
-    int* lists[3] = {sc.keep, sc.elig, sc.merge};
-    for (int q = 0; q < 3; ++q) {
-      if (f[q]) lists[q][s_base[q] + (warp > 0 ? s_warp[q][warp - 1] : 0) + x[q] - 1] = i;
-    }
-    __syncthreads();
-    if (threadIdx.x < 3) s_base[threadIdx.x] += s_warp[threadIdx.x][nw - 1];
-    __syncthreads();
   }
-  if (threadIdx.x < 3) sc.counts[1 + threadIdx.x] = s_base[threadIdx.x];
+  if (threadIdx.x == 0) {
+    sc.counts[1] = list_base[0];
+    sc.counts[2] = list_base[1];
+    sc.counts[3] = list_base[2];
+  }
 }
 
 // ------------------------------------------------------------------ merge targets
@@ -368,60 +503,83 @@ __global__ void gather_keys_kernel(const int32_t* __restrict__ list, const int32
   }
 }
 
-// Merge sources sorted by (target, source): rank by counting.
-__global__ void merge_order_kernel(const int32_t* __restrict__ target, const int32_t* __restrict__ counts, int cap,
-                                   int32_t* __restrict__ order) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  const int n = min(counts[3], cap);
-  if (i >= n) return;
-  const long long ki = (static_cast<long long>(target[i]) << 32) | i;
-  int r = 0;
-  for (int j = 0; j < n; ++j) r += ((static_cast<long long>(target[j]) << 32) | j) < ki;
-  order[r] = i;
+// Merge sources grouped by target, each group in ascending source index: counts per
+// target, their exclusive scan (the group offsets), a scatter, then a sort of every group
+// (groups are small). One CTA; every step is deterministic.
+__global__ void __launch_bounds__(1024) merge_group_kernel(Scratch sc, int n_src, int n_elig, int H, int P, int D) {
+  __shared__ int s_warp[32];
+  for (int e = threadIdx.x; e <= n_elig; e += blockDim.x) sc.bucket[e] = 0;
+  for (int e = threadIdx.x; e < n_elig; e += blockDim.x) sc.cursor[e] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_src; i += blockDim.x) atomicAdd(&sc.bucket[sc.target[i] + 1], 1);
+  __syncthreads();
+  int base = 0;
+  for (int chunk = 0; chunk < n_elig; chunk += blockDim.x) {
+    const int e = chunk + threadIdx.x;
+    const int v = e < n_elig ? sc.bucket[e + 1] : 0;
+    int total;
+    const int excl = cta_exclusive_scan(v, s_warp, &total);
+    if (e < n_elig) sc.bucket[e + 1] = base + excl + v;   // inclusive: end of group e
+    base += total;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_src; i += blockDim.x) {
+    const int e = sc.target[i];
+    sc.order[sc.bucket[e] + atomicAdd(&sc.cursor[e], 1)] = i;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n_elig; e += blockDim.x) {
+    const int b = sc.bucket[e], n = sc.bucket[e + 1] - b;
+    for (int x = 1; x < n; ++x) {                          // insertion sort of the group
+      const int v = sc.order[b + x];
+      int y = x - 1;
+      while (y >= 0 && sc.order[b + y] > v) {
+        sc.order[b + y + 1] = sc.order[b + y];
+        --y;
+      }
+      sc.order[b + y + 1] = v;
+    }
+  }
+  __syncthreads();
+  for (int q = threadIdx.x; q < n_src; q += blockDim.x) {
+    const int pos = sc.merge[sc.order[q]];
+    const long long k = sc.slot[pos];
+    sc.src_base[q] = ((k / P) * H * P + k % P) * D;
+    sc.src_cnt[q] = sc.cnt[pos];
+  }
 }
 
 // For every eligible target with at least one source: acc = c_j x_j, then acc += c_m x_m
 // for its sources in ascending id, all in fp64; x_j = bf16(acc / sum of counts), for
 // every dimension of K and V; the count becomes the sum. Sources are read before any
 // target is written because no token is both.
-__global__ void merge_apply_kernel(Scratch sc, int cap_src, int cap_elig, __nv_bfloat16* k_pool,
-                                   __nv_bfloat16* v_pool, int H, int P, int D) {
+__global__ void __launch_bounds__(256) merge_apply_kernel(Scratch sc, int cap_src, int cap_elig,
+                                                          __nv_bfloat16* k_pool, __nv_bfloat16* v_pool, int H, int P,
+                                                          int D) {
   const int e = blockIdx.x;
-  const int n_src = min(sc.counts[3], cap_src);
   const int n_elig = min(sc.counts[2], cap_elig);
   if (e >= n_elig) return;
-  // binary search the sorted (target, source) order for target e
-  int lo = 0, hi = n_src;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (sc.target[sc.order[mid]] < e) lo = mid + 1; else hi = mid;
-  }
-  const int begin = lo;
-  hi = n_src;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (sc.target[sc.order[mid]] <= e) lo = mid + 1; else hi = mid;
-  }
-  const int end = lo;
+  const int begin = sc.bucket[e], end = sc.bucket[e + 1];
   if (begin == end) return;
   const int jpos = sc.elig[e];
   const long long kj = sc.slot[jpos];
+  const long long bj = ((kj / P) * H * P + kj % P) * D;
   const int cj = sc.cnt[jpos];
   int tot = cj;
-  for (int q = begin; q < end; ++q) tot += sc.cnt[sc.merge[sc.order[q]]];
+  for (int q = begin; q < end; ++q) tot += sc.src_cnt[q];
+  const double dtot = static_cast<double>(tot);
   const int HD = H * D;
   for (int c = threadIdx.x; c < 2 * HD; c += blockDim.x) {
     __nv_bfloat16* pool = c < HD ? k_pool : v_pool;
     const int cc = c < HD ? c : c - HD;
-    const int h = cc / D, d = cc % D;
-    auto addr = [&](long long k) { return ((k / P * H + h) * P + k % P) * D + d; };
-    double acc = __dmul_rn(static_cast<double>(cj), static_cast<double>(__bfloat162float(pool[addr(kj)])));
+    const long long off = static_cast<long long>(cc / D) * P * D + cc % D;
+    double acc = __dmul_rn(static_cast<double>(cj), static_cast<double>(__bfloat162float(pool[bj + off])));
+#pragma unroll 4
     for (int q = begin; q < end; ++q) {
-      const int mpos = sc.merge[sc.order[q]];
-      const double xm = static_cast<double>(__bfloat162float(pool[addr(sc.slot[mpos])]));
-      acc = __dadd_rn(acc, __dmul_rn(static_cast<double>(sc.cnt[mpos]), xm));
+      const double xm = static_cast<double>(__bfloat162float(pool[sc.src_base[q] + off]));
+      acc = __dadd_rn(acc, __dmul_rn(static_cast<double>(sc.src_cnt[q]), xm));
     }
-    pool[addr(kj)] = f64_to_bf16_rne(__ddiv_rn(acc, static_cast<double>(tot)));
+    pool[bj + off] = f64_to_bf16_rne(__ddiv_rn(acc, dtot));
   }
   if (threadIdx.x == 0) sc.cnt[jpos] = tot;
 }
@@ -548,10 +706,10 @@ kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_
       mask |= 1u << (l % RW);
       ++n_win;
     }
-  residual_norm_kernel<<<(T + 127) / 128, 128, 0, s>>>(residual, T, g.residual_dim, sc.s_raw);
+  residual_norm_kernel<<<(T * 32 + 255) / 256, 256, 0, s>>>(residual, T, g.residual_dim, sc.s_raw);
   ok();
   const FrameRec& fr = L.frames.back();
-  clces_kernel<<<1, 1024, T * sizeof(float), s>>>(sc.s_raw, T, c->rank_hist, layer % RW, mask, n_win, g.lambda_,
+  clces_kernel<<<(T + 127) / 128, 128, T * sizeof(float), s>>>(sc.s_raw, T, c->rank_hist, layer % RW, mask, n_win, g.lambda_,
                                                   E + fr.first_entry, P, c->tok_shat + lay_slots);
   ok();
   c->hist_next_layer = layer + 1;
@@ -578,12 +736,15 @@ kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_
   __nv_bfloat16* kp = reinterpret_cast<__nv_bfloat16*>(c->k_pool) + static_cast<size_t>(layer) * c->pool_pages * c->page_elems;
   __nv_bfloat16* vp = reinterpret_cast<__nv_bfloat16*>(c->v_pool) + static_cast<size_t>(layer) * c->pool_pages * c->page_elems;
 
-  gather_meta_kernel<<<1, 1024, 0, s>>>(E, L.n_entries, P, c->tok_id + lay_slots, c->tok_cnt + lay_slots,
+  page_offsets_kernel<<<1, 1024, 0, s>>>(E, L.n_entries, sc);
+  ok();
+  gather_meta_kernel<<<(L.n_entries * P + 255) / 256, 256, 0, s>>>(E, L.n_entries, P, c->tok_id + lay_slots,
+                                                                     c->tok_cnt + lay_slots,
                                         c->tok_shat + lay_slots, T, g.num_special_tokens, g.protect_first_frame, sc);
   ok();
-  tier_rank_kernel<<<(N + 255) / 256, 256, 2048 * 5, s>>>(sc, N);
+  tier_select_kernel<<<1, 1024, 0, s>>>(sc, N, n_keep_other, n_keep_other + n_merge);
   ok();
-  tier_lists_kernel<<<1, 1024, 0, s>>>(sc, N, n_keep_other, n_merge);
+  tier_lists_kernel<<<1, 1024, 0, s>>>(sc, N);
   ok();
   check_counts_kernel<<<1, 1, 0, s>>>(sc.counts, N, n_keep, n_keep_other, n_merge, c->d_err);
   ok();
@@ -604,8 +765,7 @@ kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_
                                          &launched);
     if (r != cudaSuccess && e == cudaSuccess) e = r;
     c->launches += launched;
-    merge_order_kernel<<<(n_merge + 255) / 256, 256, 0, s>>>(sc.target, sc.counts, static_cast<int>(cp.n_merge),
-                                                              sc.order);
+    merge_group_kernel<<<1, 1024, 0, s>>>(sc, n_merge, n_keep_other, H, P, D);
     ok();
     merge_apply_kernel<<<n_keep_other, 256, 0, s>>>(sc, static_cast<int>(cp.n_merge), static_cast<int>(cp.n_keep),
                                                     kp, vp, H, P, D);

@@ -30,6 +30,7 @@ constexpr size_t kNoAllocLseFloats = kNoAllocTiles * 128;
 constexpr size_t kNoAllocScratchBytes = (kNoAllocPartFloats + kNoAllocLseFloats) * sizeof(float);
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocPartFloats + kNoAllocLseFloats];
+static_assert(sizeof(g_noalloc_scratch) == kNoAllocScratchBytes, "scratch size");
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
