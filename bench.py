@@ -233,6 +233,31 @@ def profile_traffic():
     return float(m.group(1)) if h.group(1) == cur else None
 
 
+# ------------------------------------------------------------------ ranks
+# N > 1: one process per GPU, each running its own independent stream (replicas, weak
+# scaling). The only collectives are the barriers around the timed region and the
+# max-over-ranks of the device times; none is on the data path.
+
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's synthetic stream: every rank streams different frames."""
+    return 1000 + rank
+
+
+def max_over_ranks(value_ms: float, world: int, device) -> float:
+    """The largest of the ranks' device times (all ranks must call it)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world: int, units_per_rank: int, max_ms: float) -> float:
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    return world * units_per_rank / (max_ms / 1e3)
+
+
 # ------------------------------------------------------------------ our CUDA path
 
 def run_ours(args):
@@ -265,7 +290,7 @@ def run_ours(args):
 
     log(f"rank {rank}/{world}: generating {n_frames} frames")
     with torch.cuda.stream(stream):
-        st = FrameStream(wl, seed=1000 + rank, device=dev)
+        st = FrameStream(wl, seed=rank_seed(rank), device=dev)
         frames = [st.frame(0, t) for t in range(n_frames)]
         torch.cuda.synchronize()
         log("frames ready; filling the cache")
@@ -301,10 +326,7 @@ def run_ours(args):
         launches = info1["kernel_launches"] - info0["kernel_launches"]
         assert info1["device_error"] == 0
 
-    t_max = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    elapsed_ms = float(t_max.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
 
     # end to end through the public API from pinned host buffers
     e2e = None
@@ -328,11 +350,9 @@ def run_ours(args):
             f1.record(stream)
             stream.synchronize()
             barrier()
-        e_ms = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e_ms = max_over_ranks(f0.elapsed_time(f1), world, dev)
         fb = T * H * D * 2
-        e2e = {"value": world * n_e2e / (float(e_ms.item()) / 1e3), "unit": UNIT, "h2d_bytes_per_step": 3 * fb,
+        e2e = {"value": job_rate(world, n_e2e, e_ms), "unit": UNIT, "h2d_bytes_per_step": 3 * fb,
                "d2h_bytes_per_step": fb, "steps": n_e2e, "api": "kvc_step_host"}
     kvc.kvc_destroy(h)
 
@@ -343,7 +363,7 @@ def run_ours(args):
         peak = float(peaks["bf16_tflops"])
         app_bytes = 2 * 2 * T * H * D * 2           # read K,V + write K,V (valid tokens)
         app_gbs = app_bytes / (append_ms * 1e-3) / 1e9
-        value = world * steps / (elapsed_ms / 1e3)
+        value = job_rate(world, steps, elapsed_ms)
         clocks = clk.summary()
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": warm,

@@ -1,0 +1,75 @@
+"""The multi-rank plumbing of bench.py on CPU: two gloo ranks on 127.0.0.1 run the same
+functions the N-GPU bench uses (independent per-rank streams, max over ranks, whole-job
+rate), and the reference arm's non-zero ranks exit without work."""
+import os
+import socket
+import sys
+from datetime import timedelta
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        import bench
+        from kvc_streams import WORKLOADS, FrameStream
+        m = bench.max_over_ranks(10.0 + 5.0 * rank, world, "cpu")
+        rate = bench.job_rate(world, 20, m)
+        st = FrameStream(WORKLOADS["tiny_f32"], seed=bench.rank_seed(rank))
+        k = st.frame(0, 0)[1]
+        ks = [torch.zeros_like(k) for _ in range(world)]
+        dist.all_gather(ks, k)
+        q.put((rank, m, rate, bool(torch.equal(ks[0], ks[1]))))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_max_time_and_independent_streams():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    for rank, m, rate, same in res:
+        assert m == 15.0                      # the slower rank's time, on every rank
+        assert rate == pytest.approx(2 * 20 / 0.015)
+        assert not same                       # replicas stream different frames
+
+
+def test_single_rank_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(7.5, 1, "cpu") == 7.5
+    assert bench.job_rate(1, 10, 100.0) == pytest.approx(100.0)
+
+
+def test_reference_arm_nonzero_rank_exits_without_work(monkeypatch, capsys):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    args = type("A", (), {"steps": 3, "warmup": 3, "gpus": 2})()
+    assert bench.run_reference(args) == 0
+    assert capsys.readouterr().out == ""
