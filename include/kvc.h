@@ -27,7 +27,8 @@
  *     memory).
  *   - Calls enqueue work on the cache's stream and return without waiting for
  *     the GPU, except kvc_page_table, kvc_token_meta, kvc_last_merge,
- *     kvc_export_pages, kvc_step_host and kvc_synchronize, which synchronise.
+ *     kvc_export_pages, kvc_step_host and kvc_synchronize, which synchronise
+ *     (the cache's stream and its internal copy streams).
  *   - Errors are status codes; kvc_last_error() gives a message. A status other
  *     than KVC_OK leaves the cache state unchanged unless stated otherwise.
  *     A device-side failure (a bounded wait that gave up, an exhausted page
@@ -222,6 +223,19 @@ KVC_API kvc_status kvc_export_pages(kvc_cache* c, int32_t layer, int32_t first_r
  * and wait for the copy. Pinned host memory gives full copy bandwidth. */
 KVC_API kvc_status kvc_step_host(kvc_cache* c, int32_t layer, int32_t frame_idx, int32_t is_keyframe,
                          const void* q_host, const void* k_host, const void* v_host, void* o_host);
+
+/* The same step without waiting: enqueues the upload of Q, K, V (on an internal copy
+ * stream), append + attend (on the cache's stream) and the download of O (on a second
+ * internal copy stream), then returns. Two consecutive steps use different staging
+ * buffers, so one step's copies overlap the neighbouring steps' compute; the streams are
+ * ordered by events. The host buffers must be pinned for the copies to overlap, must stay
+ * unchanged (q, k, v) and unread (o) until a synchronising call (kvc_synchronize, or any
+ * call documented to synchronise) returns. The pages define no host interface; this is
+ * the streaming form of kvc_step_host. Errors as for kvc_step_host; device-side errors
+ * appear at the next synchronising call. */
+KVC_API kvc_status kvc_step_host_async(kvc_cache* c, int32_t layer, int32_t frame_idx, int32_t is_keyframe,
+                                       const void* q_host, const void* k_host, const void* v_host,
+                                       void* o_host);
 
 /* Wait for all work of the cache and report any latched device error. */
 KVC_API kvc_status kvc_synchronize(kvc_cache* c);

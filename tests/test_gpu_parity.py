@@ -181,6 +181,39 @@ def test_host_buffer_step_matches_device_path(kvc):
     kvc.kvc_destroy(h2)
 
 
+def test_async_host_steps_match_device_path(kvc):
+    """kvc_step_host_async: nine frames (keyframe interval 2) enqueued back to back on a
+    user stream with no host sync in between, outputs downloaded into separate pinned
+    buffers; after one kvc_synchronize every output equals the device path's bit for bit."""
+    wl = WORKLOADS["vggt_24layer_k4"].replace(num_layers=1, tokens_per_frame=300, num_heads=4, window_frames=3,
+                                               scale_frames=1, keyframe_interval=2)
+    dev = torch.device("cuda")
+    user = torch.cuda.Stream(device=dev)
+    h1 = kvc.kvc_create(kvc.config_from_workload(wl))
+    h2 = kvc.kvc_create(kvc.config_from_workload(wl), user)
+    st = FrameStream(wl, seed=7, device=dev)
+    frames = [st.frame(0, t) for t in range(9)]
+    keys = [keyframe_schedule(t, wl.scale_frames, wl.keyframe_interval) for t in range(9)]
+    want = []
+    o = torch.empty((300, 4, 64), dtype=torch.bfloat16, device=dev)
+    for t, (q, k, v) in enumerate(frames):
+        kvc.kvc_append_frame(h1, 0, t, k, v, keys[t])
+        kvc.kvc_attend(h1, 0, q, o)
+        want.append(o.cpu())
+    host = [tuple(x.cpu().pin_memory() for x in f) for f in frames]
+    outs = [torch.full((300, 4, 64), float("nan"), dtype=torch.bfloat16).pin_memory() for _ in frames]
+    for t in range(9):
+        kvc.kvc_step_host_async(h2, 0, t, keys[t], *host[t], outs[t])
+    kvc.kvc_synchronize(h2)
+    for t in range(9):
+        assert torch.equal(outs[t], want[t]), f"frame {t}"
+    pt1, _ = kvc.kvc_page_table(h1, 0)
+    pt2, _ = kvc.kvc_page_table(h2, 0)
+    assert np.array_equal(pt1, pt2)
+    kvc.kvc_destroy(h1)
+    kvc.kvc_destroy(h2)
+
+
 def test_memory_constant_over_long_stream(kvc):
     wl = WORKLOADS["vggt_518x378"].replace(tokens_per_frame=200, num_heads=2, window_frames=3, scale_frames=1)
     dev = torch.device("cuda")

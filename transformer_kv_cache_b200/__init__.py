@@ -27,7 +27,8 @@ STATUS = ["KVC_OK", "KVC_ERR_ARG", "KVC_ERR_OOM", "KVC_ERR_CUDA", "KVC_ERR_STATE
 EXPORTS = ["kvc_create", "kvc_destroy", "kvc_set_stream", "kvc_reset", "kvc_append_frame", "kvc_attend",
            "kvc_compress", "kvc_page_table", "kvc_token_meta", "kvc_last_merge", "kvc_export_pages",
            "kvc_step_host", "kvc_synchronize", "kvc_last_error", "kvc_status_string", "kvc_version",
-           "kvc_debug_fail_allocs", "kvc_debug_bounded_wait", "kvc_attend_paged_noalloc", "kvc_append_frame_all"]
+           "kvc_debug_fail_allocs", "kvc_debug_bounded_wait", "kvc_attend_paged_noalloc", "kvc_append_frame_all",
+           "kvc_step_host_async"]
 
 
 class kvc_config(ctypes.Structure):
@@ -78,6 +79,7 @@ def _load():
         "kvc_last_merge": ([vp, i32, i64p, i64p, i32, i32p], i32),
         "kvc_export_pages": ([vp, i32, i32, i32, vp, vp, fp, fp], i32),
         "kvc_step_host": ([vp, i32, i32, i32, vp, vp, vp, vp], i32),
+        "kvc_step_host_async": ([vp, i32, i32, i32, vp, vp, vp, vp], i32),
         "kvc_synchronize": ([vp], i32),
         "kvc_last_error": ([vp], ctypes.c_char_p),
         "kvc_status_string": ([i32], ctypes.c_char_p),
@@ -249,6 +251,14 @@ def kvc_export_pages(handle, layer: int, first_row: int, n_rows: int, page_bytes
 def kvc_step_host(handle, layer: int, frame_idx: int, is_keyframe: bool, q_host, k_host, v_host, o_host) -> None:
     _check(handle, _lib.kvc_step_host(handle, layer, frame_idx, int(bool(is_keyframe)), _ptr(q_host),
                                       _ptr(k_host), _ptr(v_host), _ptr(o_host)))
+
+
+def kvc_step_host_async(handle, layer: int, frame_idx: int, is_keyframe: bool, q_host, k_host, v_host,
+                        o_host) -> None:
+    """Enqueue one host-buffer step and return; the buffers must stay alive (and o_host
+    unread) until kvc_synchronize."""
+    _check(handle, _lib.kvc_step_host_async(handle, layer, frame_idx, int(bool(is_keyframe)), _ptr(q_host),
+                                            _ptr(k_host), _ptr(v_host), _ptr(o_host)))
 
 
 def kvc_synchronize(handle) -> None:

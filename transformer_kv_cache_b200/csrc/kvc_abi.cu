@@ -36,11 +36,19 @@ cudaError_t dev_alloc_t(T** p, size_t bytes) {
 }
 
 void free_all(kvc_cache* c) {
-  void* ptrs[] = {c->k_pool,   c->v_pool,   c->k_scale,  c->v_scale, c->entries,  c->bitmap,
-                  c->d_err,    c->tok_id,   c->tok_cnt,  c->tok_shat, c->cmp_scratch, c->part_o,
-                  c->part_lse, c->stage_q,  c->stage_k,  c->stage_v, c->stage_o,  c->rank_hist};
+  void* ptrs[] = {c->k_pool,     c->v_pool,     c->k_scale,    c->v_scale,    c->entries,    c->bitmap,
+                  c->d_err,      c->tok_id,     c->tok_cnt,    c->tok_shat,   c->cmp_scratch, c->part_o,
+                  c->part_lse,   c->stage_q[0], c->stage_k[0], c->stage_v[0], c->stage_o[0], c->stage_q[1],
+                  c->stage_k[1], c->stage_v[1], c->stage_o[1], c->rank_hist};
   for (void* p : ptrs)
     if (p) cudaFree(p);
+  for (int i = 0; i < 2; ++i) {
+    if (c->ev_up[i]) cudaEventDestroy(c->ev_up[i]);
+    if (c->ev_done[i]) cudaEventDestroy(c->ev_done[i]);
+    if (c->ev_down[i]) cudaEventDestroy(c->ev_down[i]);
+  }
+  if (c->copy_up) cudaStreamDestroy(c->copy_up);
+  if (c->copy_down) cudaStreamDestroy(c->copy_down);
 }
 
 kvc_status fail(kvc_cache* c, kvc_status s, const char* msg) {
@@ -78,7 +86,9 @@ kvc_status check_device_error(kvc_cache* c) {
 }
 
 kvc_status sync_and_check(kvc_cache* c) {
-  cudaError_t e = cudaStreamSynchronize(c->stream);
+  cudaError_t e = cudaStreamSynchronize(c->copy_up);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(c->stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(c->copy_down);
   if (e != cudaSuccess) return cuda_fail(c, e, "cudaStreamSynchronize");
   return check_device_error(c);
 }
@@ -207,10 +217,19 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
     A(dev_alloc_t(&c->part_o, c->part_rows * 128 * 64 * sizeof(float)));
     A(dev_alloc_t(&c->part_lse, c->part_rows * 128 * sizeof(float)));
   }
-  A(dev_alloc_t(&c->stage_q, frame_bytes));
-  A(dev_alloc_t(&c->stage_k, frame_bytes));
-  A(dev_alloc_t(&c->stage_v, frame_bytes));
-  A(dev_alloc_t(&c->stage_o, frame_bytes));
+  for (int i = 0; i < 2; ++i) {
+    A(dev_alloc_t(&c->stage_q[i], frame_bytes));
+    A(dev_alloc_t(&c->stage_k[i], frame_bytes));
+    A(dev_alloc_t(&c->stage_v[i], frame_bytes));
+    A(dev_alloc_t(&c->stage_o[i], frame_bytes));
+  }
+  A(cudaStreamCreateWithFlags(&c->copy_up, cudaStreamNonBlocking));
+  A(cudaStreamCreateWithFlags(&c->copy_down, cudaStreamNonBlocking));
+  for (int i = 0; i < 2; ++i) {
+    A(cudaEventCreateWithFlags(&c->ev_up[i], cudaEventDisableTiming));
+    A(cudaEventCreateWithFlags(&c->ev_done[i], cudaEventDisableTiming));
+    A(cudaEventCreateWithFlags(&c->ev_down[i], cudaEventDisableTiming));
+  }
   if (g.budget_tokens > 0) {
     const size_t slots = L * c->pool_pages * P;
     A(dev_alloc_t(&c->tok_id, slots * sizeof(int64_t)));
@@ -266,7 +285,9 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
 
 kvc_status kvc_destroy(kvc_cache* c) {
   if (!c) return KVC_OK;
+  cudaStreamSynchronize(c->copy_up);
   cudaStreamSynchronize(c->stream);
+  cudaStreamSynchronize(c->copy_down);
   free_all(c);
   delete c;
   return KVC_OK;
@@ -589,25 +610,41 @@ kvc_status kvc_export_pages(kvc_cache* c, int32_t layer, int32_t first_row, int3
   return KVC_OK;
 }
 
-kvc_status kvc_step_host(kvc_cache* c, int32_t layer, int32_t frame_idx, int32_t is_keyframe, const void* q_host,
-                         const void* k_host, const void* v_host, void* o_host) {
+kvc_status kvc_step_host_async(kvc_cache* c, int32_t layer, int32_t frame_idx, int32_t is_keyframe,
+                               const void* q_host, const void* k_host, const void* v_host, void* o_host) {
   if (!c) return KVC_ERR_ARG;
   if (!q_host || !k_host || !v_host || !o_host) return fail(c, KVC_ERR_ARG, "kvc_step_host: NULL host buffer");
   const kvc_config& g = c->cfg;
   const size_t bytes = static_cast<size_t>(g.tokens_per_frame) * g.num_heads * g.head_dim * c->elem_io;
-  cudaError_t e = cudaMemcpyAsync(c->stage_q, q_host, bytes, cudaMemcpyHostToDevice, c->stream);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(c->stage_k, k_host, bytes, cudaMemcpyHostToDevice, c->stream);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(c->stage_v, v_host, bytes, cudaMemcpyHostToDevice, c->stream);
+  const int b = c->host_slot;
+  // upload once the step that last used this slot has consumed its inputs
+  cudaError_t e = cudaStreamWaitEvent(c->copy_up, c->ev_done[b], 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->stage_q[b], q_host, bytes, cudaMemcpyHostToDevice, c->copy_up);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->stage_k[b], k_host, bytes, cudaMemcpyHostToDevice, c->copy_up);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->stage_v[b], v_host, bytes, cudaMemcpyHostToDevice, c->copy_up);
+  if (e == cudaSuccess) e = cudaEventRecord(c->ev_up[b], c->copy_up);
+  // compute after the upload, and after this slot's previous output has left the device
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(c->stream, c->ev_up[b], 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(c->stream, c->ev_down[b], 0);
   if (e != cudaSuccess) return cuda_fail(c, e, "kvc_step_host upload");
-  kvc_status st = kvc_append_frame(c, layer, frame_idx, c->stage_k, c->stage_v, is_keyframe);
+  kvc_status st = kvc_append_frame(c, layer, frame_idx, c->stage_k[b], c->stage_v[b], is_keyframe);
   if (st != KVC_OK) return st;
-  st = kvc_attend(c, layer, c->stage_q, c->stage_o);
+  st = kvc_attend(c, layer, c->stage_q[b], c->stage_o[b]);
   if (st != KVC_OK) return st;
-  e = cudaMemcpyAsync(o_host, c->stage_o, bytes, cudaMemcpyDeviceToHost, c->stream);
+  e = cudaEventRecord(c->ev_done[b], c->stream);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(c->copy_down, c->ev_done[b], 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(o_host, c->stage_o[b], bytes, cudaMemcpyDeviceToHost, c->copy_down);
+  if (e == cudaSuccess) e = cudaEventRecord(c->ev_down[b], c->copy_down);
   if (e != cudaSuccess) return cuda_fail(c, e, "kvc_step_host download");
-  e = cudaStreamSynchronize(c->stream);
-  if (e != cudaSuccess) return cuda_fail(c, e, "kvc_step_host sync");
+  c->host_slot = b ^ 1;
   return KVC_OK;
+}
+
+kvc_status kvc_step_host(kvc_cache* c, int32_t layer, int32_t frame_idx, int32_t is_keyframe, const void* q_host,
+                         const void* k_host, const void* v_host, void* o_host) {
+  kvc_status st = kvc_step_host_async(c, layer, frame_idx, is_keyframe, q_host, k_host, v_host, o_host);
+  if (st != KVC_OK) return st;
+  return sync_and_check(c);
 }
 
 kvc_status kvc_synchronize(kvc_cache* c) {

@@ -71,11 +71,17 @@ struct Cache {
   float* part_o = nullptr;
   float* part_lse = nullptr;
   size_t part_rows = 0;             // capacity in 128-row partial tiles
-  // host-buffer step staging
-  uint8_t* stage_q = nullptr;
-  uint8_t* stage_k = nullptr;
-  uint8_t* stage_v = nullptr;
-  uint8_t* stage_o = nullptr;
+  // host-buffer steps: two staging slots so that one step's copies overlap another's
+  // compute; uploads and downloads run on their own streams, ordered by events
+  uint8_t* stage_q[2] = {nullptr, nullptr};
+  uint8_t* stage_k[2] = {nullptr, nullptr};
+  uint8_t* stage_v[2] = {nullptr, nullptr};
+  uint8_t* stage_o[2] = {nullptr, nullptr};
+  cudaStream_t copy_up = nullptr, copy_down = nullptr;
+  cudaEvent_t ev_up[2] = {nullptr, nullptr};      // slot's inputs uploaded
+  cudaEvent_t ev_done[2] = {nullptr, nullptr};    // slot's step computed
+  cudaEvent_t ev_down[2] = {nullptr, nullptr};    // slot's output downloaded
+  int host_slot = 0;
   // tensor maps of each layer's K and V pools (bf16 tensor-core path)
   std::vector<CUtensorMap> tmap_k, tmap_v;
   bool tc_path = false;
