@@ -4,21 +4,26 @@
 // Processing) over K/V stored as E4M3 codes with one absmax scale per (page, head)
 // ("XStreamVGGT" abstract: KV cache quantisation). The tensor cores multiply f16
 // operands (kind::f16 needs both operands of one type), so each KV tile is widened in
-// shared memory right after it lands:
+// shared memory right after it lands. One CTA per SM owns two 128-row query tiles of one
+// head, so every converted KV tile serves 256 query rows:
 //
-//   warp 0              lane 0: TMA producer of the bf16 query tile (once) and, per 64-slot
-//                       KV tile, of the 4 page-head code blocks of K and of V (1 KB each)
-//                       into a three-stage staging ring. The whole warp converts: the query
-//                       tile bf16 -> f16 in place, then every code pair -> f16 pair with the
-//                       hardware E4M3 conversion (exact), written as a 128-byte-swizzled MMA
-//                       operand. K codes stay unscaled; each V pair is multiplied by the
-//                       page's V scale over the CTA's largest V scale of the head.
-//   warp 1 (one lane)   MMA issuer: S = Q K^T (M=128, N=64) and O' += P [V | 1] (M=128,
-//                       N=80), f16 inputs, fp32 accumulation in TMEM.
-//   warps 2..5          softmax: as in the bf16 kernel (one thread per row, 64 columns per
-//                       tile, lazy rescaling, row sum from the ones column), with P packed
-//                       as f16. The K scale of a page multiplies the logit factor of its 16
-//                       columns, so Q K^T runs on exact decoded codes.
+//   warps 0, 10         converters, one half of each 64-slot KV tile (2 of its 4 pages)
+//                       each: lane 0 loads the half's K and V code blocks (1 KB per page
+//                       and tensor) by TMA into the warp's own three-stage ring; the warp
+//                       turns every code pair into an f16 pair with the hardware E4M3
+//                       conversion (exact) and writes it as a 128-byte-swizzled MMA operand.
+//                       K codes stay unscaled; each V pair is multiplied by the page's V
+//                       scale over the CTA's largest V scale of the head. Before the first
+//                       tile, each converter widens one query tile bf16 -> f16 in place
+//                       (warp 0 lane 0 loads both query tiles).
+//   warps 1, 11         MMA issuers, one lane each, one per query tile (so the two tiles'
+//                       pipelines do not wait on each other): per KV tile S = Q K^T (M=128,
+//                       N=64) and O' += P [V | 1] (M=128, N=80), f16 inputs, fp32
+//                       accumulation in TMEM (512 columns: 256 per query tile).
+//   warps 2..5, 6..9    softmax of query tile 0 and 1: as in the bf16 kernel (one thread
+//                       per row, 64 columns per tile, lazy rescaling, row sum from the ones
+//                       column), with P packed as f16. The K scale of a page multiplies the
+//                       logit factor of its 16 columns, so Q K^T runs on exact decoded codes.
 //
 // The epilogue multiplies by the V reference scale. Rounding V times s_page / s_ref to f16
 // is the only extra rounding of an operand (relative 2^-11). The query is held in f16,
@@ -32,20 +37,22 @@
 namespace kvc {
 namespace tc8 {
 constexpr int kBM = 128, kBN = 64, kHD = 64, kON = kHD + 16;
-constexpr int kCodeStages = 2;                // code staging ring (TMA destination)
+constexpr int kGroups = 2;                    // query tiles per CTA
+constexpr int kCodeStages = 3;                // code staging ring of each converter
 constexpr int kStages = 4;                    // converted f16 operand ring
-constexpr bool kEarlyPV = false;              // issue PV(j) while S(j+1) waits for its conversion
-constexpr int kCodeBytes = kBN * kHD;         // 4 KB of codes per K or V tile
+constexpr int kHalfCodeBytes = (kBN / 2) * kHD;   // 2 KB: a converter's half tile of one tensor
 constexpr int kConvBytes = kBN * kHD * 2;     // 8 KB f16 tile
-constexpr int kQBytes = kBM * kHD * 2;        // 16 KB
+constexpr int kQBytes = kBM * kHD * 2;        // 16 KB per query tile
 constexpr int kOnesBytes = kBN * kHD * 2;
-constexpr int kThreads = 192;
-constexpr int kConvThreads = 32;              // warp 0
-constexpr int kTmemCols = 256;
+constexpr int kThreads = 384;                 // 12 warps
+constexpr int kConvThreads = 64;              // warps 0 and 10
+constexpr int kTmemCols = 512;
+constexpr int kGroupCols = 256;               // TMEM columns per query tile
 constexpr int kColS = 0, kColP = 64, kColO = 128;
 constexpr float kPMax = 256.0f;
+constexpr size_t kCodesBytes = 2 * kCodeStages * 2 * kHalfCodeBytes;
 constexpr size_t kSmemBytes =
-    1024 + kQBytes + 2 * kStages * kConvBytes + 2 * kCodeStages * kCodeBytes + kOnesBytes + 512;
+    1024 + kGroups * kQBytes + 2 * kStages * kConvBytes + kOnesBytes + kCodesBytes + 512;
 }  // namespace tc8
 
 __device__ __forceinline__ uint32_t f16x2_of_e4m3x2(uint32_t code_pair) {
@@ -83,39 +90,42 @@ __device__ __forceinline__ float page_scale(const TcParams& p, const float* sc, 
 }
 
 template <int P>
-__global__ void __launch_bounds__(tc8::kThreads, 2)
+__global__ void __launch_bounds__(tc8::kThreads, 1)
     attn_fp8_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v, const TcParams p) {
   using namespace tc8;
-  constexpr int kPPT = kBN / P;
+  constexpr int kPPT = kBN / P;               // pages per KV tile
+  constexpr int kPPH = kPPT / 2;              // pages per converter half
+  static_assert(kPPT % 2 == 0, "a KV tile splits into two halves of whole pages");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_s = smem;
-  uint8_t* ck_s = q_s + kQBytes;                       // converted K tiles [kStages]
-  uint8_t* cv_s = ck_s + kStages * kConvBytes;         // converted V tiles [kStages]
+  uint8_t* q_s = smem;                                  // [kGroups] query tiles
+  uint8_t* ck_s = q_s + kGroups * kQBytes;              // converted K tiles [kStages]
+  uint8_t* cv_s = ck_s + kStages * kConvBytes;          // converted V tiles [kStages]
   uint8_t* ones_s = cv_s + kStages * kConvBytes;
-  uint8_t* sk_s = ones_s + kOnesBytes;                 // K code staging [kCodeStages]
-  uint8_t* sv_s = sk_s + kCodeStages * kCodeBytes;     // V code staging [kCodeStages]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sv_s + kCodeStages * kCodeBytes);
+  uint8_t* codes = ones_s + kOnesBytes;                 // [converter][kCodeStages][K, V][half tile]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(codes + kCodesBytes);
   uint64_t* q_full = bars;
   uint64_t* q_ready = bars + 1;
-  uint64_t* c8_full = bars + 2;                        // [kCodeStages] codes landed
-  uint64_t* kc_full = c8_full + kCodeStages;           // [kStages] converted
-  uint64_t* kv_empty = kc_full + kStages;              // [kStages]
-  uint64_t* s_full = kv_empty + kStages;
-  uint64_t* s_free = s_full + 1;
-  uint64_t* p_full = s_full + 2;                       // [2]
-  uint64_t* pv_done = s_full + 4;                      // [2]
-  uint64_t* mma_final = s_full + 6;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
+  uint64_t* c8_full = bars + 2;                         // [converter][kCodeStages]
+  uint64_t* kc_full = c8_full + 2 * kCodeStages;        // [kStages] both halves converted
+  uint64_t* kv_empty = kc_full + kStages;               // [kStages]
+  uint64_t* s_full = kv_empty + kStages;                // [kGroups]
+  uint64_t* s_free = s_full + kGroups;                  // [kGroups]
+  uint64_t* p_full = s_free + kGroups;                  // [kGroups][2]
+  uint64_t* pv_done = p_full + 2 * kGroups;             // [kGroups][2]
+  uint64_t* mma_final = pv_done + 2 * kGroups;          // [kGroups]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + kGroups);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* sref = reinterpret_cast<float*>(tmem_slot + 2);   // V reference scale
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x % p.q_tiles;
-  const int rest = blockIdx.x / p.q_tiles;
+  const int pairs = (p.q_tiles + 1) / 2;
+  const int qp = blockIdx.x % pairs;
+  const int rest = blockIdx.x / pairs;
   const int split = rest % p.splits;
   const int h = rest / p.splits;
+  const int ngroups = (2 * qp + 1 < p.q_tiles) ? 2 : 1;  // the last pair may hold one tile
   const int tile0 = split * p.tiles_per_split;
   const int tile1 = min(tile0 + p.tiles_per_split, p.total_tiles);
   const int n_tiles = tile1 - tile0;
@@ -123,18 +133,20 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_ready, kConvThreads);
-    for (int i = 0; i < kCodeStages; ++i) mbar_init(&c8_full[i], 1);
+    for (int i = 0; i < 2 * kCodeStages; ++i) mbar_init(&c8_full[i], 1);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&kc_full[i], kConvThreads);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&kv_empty[i], ngroups);                 // one commit per query tile's issuer
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 4);
-    mbar_init(&p_full[0], 4);
-    mbar_init(&p_full[1], 4);
-    mbar_init(&pv_done[0], 1);
-    mbar_init(&pv_done[1], 1);
-    mbar_init(mma_final, 1);
+    for (int g = 0; g < kGroups; ++g) {
+      mbar_init(&s_full[g], 1);
+      mbar_init(&s_free[g], 4);
+      mbar_init(&p_full[2 * g], 4);
+      mbar_init(&p_full[2 * g + 1], 4);
+      mbar_init(&pv_done[2 * g], 1);
+      mbar_init(&pv_done[2 * g + 1], 1);
+      mbar_init(&mma_final[g], 1);
+    }
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -151,12 +163,14 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
   const uint32_t tmem = *tmem_slot;
 
   if (n_tiles > 0) {
-    if (warp == 0) {
-      // ------------------------------------------------------ TMA producer + converter
-      // Lanes 0..3 each track page g = lane of the tiles ahead (physical page, V scale), so
-      // no dependent global load sits on the conversion path.
-      const int gl = lane & 3;
-      // V reference scale: the largest V scale of the head over this CTA's pages
+    if (warp == 0 || warp == 10) {
+      // ------------------------------------------------ converters (TMA in lane 0 each)
+      const int ci = warp == 0 ? 0 : 1;                 // half of every KV tile: pages 2ci, 2ci+1
+      const int gl = ci * kPPH + (lane & (kPPH - 1));   // page of the tile tracked by lanes 0..kPPH-1
+      uint64_t* c8f = c8_full + ci * kCodeStages;
+      uint8_t* my_codes = codes + ci * (kCodeStages * 2 * kHalfCodeBytes);
+      // V reference scale: the largest V scale of the head over this CTA's pages (both
+      // converters compute the same value)
       float mv = 0.f;
 #pragma unroll 4
       for (int idx = tile0 * kPPT + lane; idx < min(tile1 * kPPT, p.n_pages); idx += 32)
@@ -165,83 +179,85 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
       for (int o = 16; o > 0; o >>= 1) mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, o));
       if (mv == 0.f) mv = 1.f;                          // all-zero pages: any reference works
       const float iv = 1.f / mv;
-      if (lane == 0) *sref = mv;
-      // Physical page g of tiles ahead and the V scale of the next tile. Every value loaded
-      // in iteration j is first used in iteration j + 1 (rotations happen at the loop top),
-      // so no copy waits on a load in flight.
+      if (ci == 0 && lane == 0) *sref = mv;
+      // physical page gl of tiles ahead and its V scale; each value loaded in iteration j
+      // is first used in iteration j + 1
       const int pq0 = page_entry(p, tile0 * kPPT + gl).x;
       int pq1 = page_entry(p, (tile0 + 1) * kPPT + gl).x;
       int pq2 = page_entry(p, (tile0 + 2) * kPPT + gl).x;
-      int pq4n = page_entry(p, (tile0 + 3) * kPPT + gl).x;   // becomes pq3 at the loop top
-      float vsn = page_scale(p, p.v_scale, pq0, h);         // becomes the factor of tile j
-      // the code blocks of tile t (page gl's K and V from lanes 0..3) into stage t % kStages
-#define KVC_FP8_ISSUE(t, phys)                                                                    \
-  do {                                                                                            \
-    const int st_ = (t) % kCodeStages;                                                            \
-    if (lane == 0) mbar_arrive_expect_tx(&c8_full[st_], 2 * kCodeBytes);                          \
-    __syncwarp();                                                                                 \
-    if (lane < kPPT) {                                                                            \
+      int pq4n = page_entry(p, (tile0 + 3) * kPPT + gl).x;
+      float vsn = page_scale(p, p.v_scale, pq0, h);
+#define KVC_FP8_ISSUE(t, phys)                                                                      \
+  do {                                                                                              \
+    const int st_ = (t) % kCodeStages;                                                              \
+    uint8_t* kc_ = my_codes + st_ * 2 * kHalfCodeBytes;                                             \
+    if (lane == 0) mbar_arrive_expect_tx(&c8f[st_], 2 * kHalfCodeBytes);                            \
+    __syncwarp();                                                                                   \
+    if (lane < kPPH) {                                                                              \
       const int row_ = (phys) >= 0 ? static_cast<int>(((p.page_base + (phys)) * p.H + h) * P) : p.pool_rows; \
-      tma_load_2d(sk_s + st_ * kCodeBytes + lane * P * kHD, &tmap_k, &c8_full[st_], 0, row_);     \
-      tma_load_2d(sv_s + st_ * kCodeBytes + lane * P * kHD, &tmap_v, &c8_full[st_], 0, row_);     \
-    }                                                                                             \
+      tma_load_2d(kc_ + lane * P * kHD, &tmap_k, &c8f[st_], 0, row_);                               \
+      tma_load_2d(kc_ + kHalfCodeBytes + lane * P * kHD, &tmap_v, &c8f[st_], 0, row_);              \
+    }                                                                                               \
   } while (0)
-      if (lane == 0) {
+      if (ci == 0 && lane == 0) {
         tma_prefetch_desc(&tmap_q);
         tma_prefetch_desc(&tmap_k);
         tma_prefetch_desc(&tmap_v);
-        mbar_arrive_expect_tx(q_full, kQBytes);
-        tma_load_3d(q_s, &tmap_q, q_full, 0, h, qt * kBM);
+        mbar_arrive_expect_tx(q_full, ngroups * kQBytes);
+        for (int g = 0; g < ngroups; ++g) tma_load_3d(q_s + g * kQBytes, &tmap_q, q_full, 0, h, (2 * qp + g) * kBM);
       }
-      static_assert(kCodeStages == 2 || kCodeStages == 3, "code ring of 2 or 3 stages");
+      static_assert(kCodeStages == 3, "the issue distance below is three tiles");
       KVC_FP8_ISSUE(0, pq0);
       if (n_tiles > 1) KVC_FP8_ISSUE(1, pq1);
-      if (kCodeStages == 3 && n_tiles > 2) KVC_FP8_ISSUE(2, pq2);
+      if (n_tiles > 2) KVC_FP8_ISSUE(2, pq2);
       int issued = min(n_tiles, kCodeStages);
       bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(q_full, 0, abort_flag, p.err));
       if (ok) {
-        // the query tile bf16 -> f16 in place (positions, hence the swizzle, unchanged)
-        uint32_t* q32 = reinterpret_cast<uint32_t*>(q_s);
+        // query tile ci bf16 -> f16 in place (positions, hence the swizzle, unchanged)
+        if (ci < ngroups) {
+          uint32_t* q32 = reinterpret_cast<uint32_t*>(q_s + ci * kQBytes);
 #pragma unroll 8
-        for (int i = lane; i < kQBytes / 4; i += 32) {
-          const uint32_t w = q32[i];
-          q32[i] = pack_f16(bf16lo(w), bf16hi(w));
+          for (int i = lane; i < kQBytes / 4; i += 32) {
+            const uint32_t w = q32[i];
+            q32[i] = pack_f16(bf16lo(w), bf16hi(w));
+          }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive(q_ready);
       }
-      // per-lane constant parts of the conversion addresses: row (lane >> 3) + 4 i, chunk
-      // lane & 7 of 8 dims; in the swizzled f16 tile the chunk moves to chunk ^ (row & 7)
+      // this converter's rows of the tile: 32 ci + (lane >> 3) + 4 i, i < 8, chunk lane & 7
+      // of 8 dims; in the swizzled f16 tile the chunk moves to chunk ^ (row & 7)
       const int r0 = lane >> 3, c0 = lane & 7;
       const int src_off = r0 * kHD + c0 * 8;
-      const int dst_even = r0 * 128 + ((c0 ^ r0) << 4);
-      const int dst_odd = r0 * 128 + ((c0 ^ r0 ^ 4) << 4);
+      const int dst_base = ci * 32 * 128;
+      const int dst_even = dst_base + r0 * 128 + ((c0 ^ r0) << 4);
+      const int dst_odd = dst_base + r0 * 128 + ((c0 ^ r0 ^ 4) << 4);
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int st = j % kStages;
-        const float fvj = vsn * iv;                     // V factor of page g of tile j
-        const int pq3 = pq4n;                           // page g of tile j + 3
+        const int cs = j % kCodeStages;
+        const float fvj = vsn * iv;                     // V factor of page gl of tile j
+        const int pq3 = pq4n;                           // page gl of tile j + 3
         vsn = page_scale(p, p.v_scale, pq1, h);         // tile j + 1
         pq4n = page_entry(p, (tile0 + j + 4) * kPPT + gl).x;
-        uint32_t rv[kPPT];
+        uint32_t rv[kPPH];
 #pragma unroll
-        for (int g = 0; g < kPPT; ++g) rv[g] = f16x2_splat(__shfl_sync(0xffffffffu, fvj, g));
+        for (int g = 0; g < kPPH; ++g) rv[g] = f16x2_splat(__shfl_sync(0xffffffffu, fvj, g));
         // converted stage st is free once the MMAs of tile j - kStages have completed
         if (j >= kStages &&
             !__all_sync(0xffffffffu, mbar_wait_bounded(&kv_empty[st], ((j / kStages) - 1) & 1, abort_flag, p.err))) {
           ok = false;
           break;
         }
-        const int cs = j % kCodeStages;
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&c8_full[cs], (j / kCodeStages) & 1, abort_flag, p.err))) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&c8f[cs], (j / kCodeStages) & 1, abort_flag, p.err))) {
           ok = false;
           break;
         }
-        const uint8_t* ksrc = sk_s + cs * kCodeBytes + src_off;
-        const uint8_t* vsrc = sv_s + cs * kCodeBytes + src_off;
+        const uint8_t* ksrc = my_codes + cs * 2 * kHalfCodeBytes + src_off;
+        const uint8_t* vsrc = ksrc + kHalfCodeBytes;
         uint8_t* kdst = ck_s + st * kConvBytes;
         uint8_t* vdst = cv_s + st * kConvBytes;
 #pragma unroll
-        for (int i = 0; i < kBN / 4; ++i) {            // row (lane >> 3) + 4 i, page i / 4
+        for (int i = 0; i < kBN / 8; ++i) {             // local row (lane >> 3) + 4 i, page i / 4
           const uint2 kc = *reinterpret_cast<const uint2*>(ksrc + i * 4 * kHD);
           const uint2 vc = *reinterpret_cast<const uint2*>(vsrc + i * 4 * kHD);
           uint4 ko, vo;
@@ -260,110 +276,84 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive(&kc_full[st]);
         __syncwarp();
-        // code stage cs has been read by the whole warp: refill it with tile j + kCodeStages
+        // code stage cs has been read by the whole warp: refill it with tile j + 3
         if (j + kCodeStages < n_tiles) {
-          KVC_FP8_ISSUE(j + kCodeStages, kCodeStages == 3 ? pq3 : pq2);
+          KVC_FP8_ISSUE(j + kCodeStages, pq3);
           ++issued;
         }
         pq1 = pq2;
         pq2 = pq3;
       }
 #undef KVC_FP8_ISSUE
-      // drain: the last code load issued into each stage (tile t = the largest issued t
-      // with t % kCodeStages == stage) has landed before the CTA exits
+      // drain: the last code load issued into each stage has landed before the CTA exits
       if (lane == 0) {
-        mbar_wait_drain(q_full, 0, p.err);
+        if (ci == 0) mbar_wait_drain(q_full, 0, p.err);
 #pragma unroll
         for (int i = 0; i < kCodeStages; ++i)
           if (issued > i) {
             const int t = i + kCodeStages * ((issued - 1 - i) / kCodeStages);
-            mbar_wait_drain(&c8_full[i], (t / kCodeStages) & 1, p.err);
+            mbar_wait_drain(&c8f[i], (t / kCodeStages) & 1, p.err);
           }
       }
-    } else if (warp == 1) {
-      if (lane == 0) {
-        // ---------------------------------------------------------------- MMA issuer
+    } else if (warp == 1 || warp == 11) {
+      const int g = warp == 1 ? 0 : 1;
+      if (lane == 0 && g < ngroups) {
+        // -------------------------------------------------- MMA issuer of query tile g
         const uint32_t idesc_s = idesc_f16kind(0, kBM, kBN, 0, 0);
         const uint32_t idesc_o = idesc_f16kind(0, kBM, kON, 0, 1);
-        const uint32_t tS = tmem + kColS, tP = tmem + kColP, tO = tmem + kColO;
-        const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(ck_s), v_addr = smem_u32(cv_s);
+        const uint32_t qa = smem_u32(q_s) + g * kQBytes, k_addr = smem_u32(ck_s), v_addr = smem_u32(cv_s);
         const uint32_t ones_addr = smem_u32(ones_s);
+        const uint32_t tS = tmem + g * kGroupCols + kColS, tP = tmem + g * kGroupCols + kColP;
+        const uint32_t tO = tmem + g * kGroupCols + kColO;
         bool ok = mbar_wait_bounded(q_ready, 0, abort_flag, p.err) &&
                   mbar_wait_bounded(&kc_full[0], 0, abort_flag, p.err);
         if (ok) {
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kHD / 16; ++kk)
-            mma_ss(tS, sw128_desc(q_addr + kk * 32, 16, 1024), sw128_desc(k_addr + kk * 32, 16, 1024), idesc_s,
-                   kk > 0);
-          mma_commit(s_full);
+            mma_ss(tS, sw128_desc(qa + kk * 32, 16, 1024), sw128_desc(k_addr + kk * 32, 16, 1024), idesc_s, kk > 0);
+          mma_commit(&s_full[g]);
         }
         for (int j = 0; ok && j < n_tiles; ++j) {
           const int st = j % kStages;
-          bool pv_issued = false;
-          // PV(j): O' += P(j) [V(j) | 1], then release P buffer j & 1 and operand stage st
-#define KVC_FP8_PV()                                                                                      \
-  do {                                                                                                    \
-    tc_fence_after();                                                                                     \
-    const uint32_t vb = v_addr + st * kConvBytes;                                                         \
-    const uint32_t lbo = ones_addr - vb;                                                                  \
-    const uint32_t pa = tP + (j & 1) * (kBN / 2);                                                         \
-    _Pragma("unroll") for (int kk = 0; kk < kBN / 16; ++kk)                                               \
-      mma_ts(tO, pa + kk * 8, sw128_desc(vb + kk * 2048, lbo, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u); \
-    mma_commit(&pv_done[j & 1]);                                                                          \
-    mma_commit(&kv_empty[st]);                                                                            \
-    pv_issued = true;                                                                                     \
-  } while (0)
           if (j + 1 < n_tiles) {
             const int st1 = (j + 1) % kStages;
-            if (!mbar_wait_bounded(s_free, j & 1, abort_flag, p.err)) break;
-            if (kEarlyPV) {
-              // wait for the converted operands of tile j + 1; if P(j) is ready first, run
-              // PV(j) meanwhile (bounded like every wait)
-              const uint64_t t0 = globaltimer_ns();
-              bool got = false;
-              for (uint32_t i = 0;; ++i) {
-                if (!pv_issued && mbar_try_wait(&p_full[j & 1], (j >> 1) & 1)) KVC_FP8_PV();
-                if (mbar_try_wait(&kc_full[st1], ((j + 1) / kStages) & 1)) {
-                  got = true;
-                  break;
-                }
-                if ((i & 63u) == 63u) {
-                  if (*abort_flag) break;
-                  if (globaltimer_ns() - t0 > KVC_WAIT_LIMIT_NS) {
-                    *abort_flag = 1;
-                    latch_error(p.err, DERR_TIMEOUT);
-                    break;
-                  }
-                }
-              }
-              if (!got) break;
-            } else if (!mbar_wait_bounded(&kc_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.err)) {
-              break;
-            }
+            if (!mbar_wait_bounded(&kc_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.err)) break;
+            if (!mbar_wait_bounded(&s_free[g], j & 1, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t kb = k_addr + st1 * kConvBytes;
 #pragma unroll
             for (int kk = 0; kk < kHD / 16; ++kk)
-              mma_ss(tS, sw128_desc(q_addr + kk * 32, 16, 1024), sw128_desc(kb + kk * 32, 16, 1024), idesc_s,
-                     kk > 0);
-            mma_commit(s_full);
+              mma_ss(tS, sw128_desc(qa + kk * 32, 16, 1024), sw128_desc(kb + kk * 32, 16, 1024), idesc_s, kk > 0);
+            mma_commit(&s_full[g]);
           }
-          if (!pv_issued) {
-            if (!mbar_wait_bounded(&p_full[j & 1], (j >> 1) & 1, abort_flag, p.err)) break;
-            KVC_FP8_PV();
-          }
-#undef KVC_FP8_PV
+          if (!mbar_wait_bounded(&p_full[2 * g + (j & 1)], (j >> 1) & 1, abort_flag, p.err)) break;
+          tc_fence_after();
+          const uint32_t vb = v_addr + st * kConvBytes;
+          const uint32_t lbo = ones_addr - vb;
+          const uint32_t pa = tP + (j & 1) * (kBN / 2);
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            mma_ts(tO, pa + kk * 8, sw128_desc(vb + kk * 2048, lbo, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&pv_done[2 * g + (j & 1)]);
+          mma_commit(&kv_empty[st]);
         }
-        mma_commit(mma_final);
-        mbar_wait_drain(mma_final, 0, p.err);
+        mma_commit(&mma_final[g]);
+        mbar_wait_drain(&mma_final[g], 0, p.err);
       }
-    } else {
+    } else if (((warp - 2) >> 2) < ngroups) {
       // ------------------------------------------------------------------ softmax warps
+      const int g = (warp - 2) >> 2;                     // query tile of this warp
+      const int qt = 2 * qp + g;
       const int wq = warp & 3;
       const int r = wq * 32 + lane;
       const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-      const uint32_t tS = tmem + kColS + lane_off, tP = tmem + kColP + lane_off, tO = tmem + kColO + lane_off;
+      const uint32_t tbase = tmem + g * kGroupCols + lane_off;
+      const uint32_t tS = tbase + kColS, tP = tbase + kColP, tO = tbase + kColO;
+      uint64_t* my_s_full = &s_full[g];
+      uint64_t* my_s_free = &s_free[g];
+      uint64_t* my_p_full = &p_full[2 * g];
+      uint64_t* my_pv_done = &pv_done[2 * g];
       bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(q_ready, 0, abort_flag, p.err));
       const float vref = ok ? *sref : 1.f;
       float m = -INFINITY, masked = 0.f;
@@ -376,7 +366,7 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
       int vj = en.w;
       en = page_entry(p, (tile0 + 1) * kPPT + gl);
       uint32_t s[2][32];
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(s_full, 0, abort_flag, p.err));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(my_s_full, 0, abort_flag, p.err));
       if (ok) {
         tc_fence_after();
         tmem_ld32(tS + 0, s[0]);
@@ -384,15 +374,15 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);
+        if (lane == 0) mbar_arrive(my_s_free);
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
         int n_masked = 0;
         float cg[kPPT];            // logit factor per page: log2(e) x softmax scale x K scale
 #pragma unroll
-        for (int g = 0; g < kPPT; ++g) {
-          n_masked += P - __shfl_sync(0xffffffffu, vj, g);
-          cg[g] = p.scale_log2 * __shfl_sync(0xffffffffu, ksj, g);
+        for (int pg = 0; pg < kPPT; ++pg) {
+          n_masked += P - __shfl_sync(0xffffffffu, vj, pg);
+          cg[pg] = p.scale_log2 * __shfl_sync(0xffffffffu, ksj, pg);
         }
         if (j + 1 < n_tiles) {
           ksj = page_scale(p, p.k_scale, en.x, h);
@@ -404,10 +394,10 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
         {
           const uint64_t nm2 = pk2(-m, -m);
 #pragma unroll
-          for (int g = 0; g < kPPT; ++g) {
-            const uint64_t c2 = pk2(cg[g], cg[g]);
+          for (int pg = 0; pg < kPPT; ++pg) {
+            const uint64_t c2 = pk2(cg[pg], cg[pg]);
 #pragma unroll
-            for (int i = g * (P / 2); i < (g + 1) * (P / 2); ++i) {
+            for (int i = pg * (P / 2); i < (pg + 1) * (P / 2); ++i) {
               float x0, x1;
               up2(fma2_pair(s[(2 * i) / 32][(2 * i) % 32], s[(2 * i + 1) / 32][(2 * i + 1) % 32], c2, nm2), x0,
                   x1);
@@ -422,20 +412,20 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
           // the page's (non-negative) factor
           float mt = -INFINITY;
 #pragma unroll
-          for (int g = 0; g < kPPT; ++g) {
+          for (int pg = 0; pg < kPPT; ++pg) {
             float ta = -INFINITY, tb = -INFINITY;
 #pragma unroll
-            for (int cc = g * P; cc < (g + 1) * P; cc += 4) {
+            for (int cc = pg * P; cc < (pg + 1) * P; cc += 4) {
               ta = max3(ta, __uint_as_float(s[cc / 32][cc % 32]), __uint_as_float(s[cc / 32][cc % 32 + 1]));
               tb = max3(tb, __uint_as_float(s[cc / 32][cc % 32 + 2]), __uint_as_float(s[cc / 32][cc % 32 + 3]));
             }
-            mt = fmaxf(mt, fmaxf(ta, tb) * cg[g]);
+            mt = fmaxf(mt, fmaxf(ta, tb) * cg[pg]);
           }
           const float m_new = move ? mt : m;
           const bool resc = move && j > 0;
           if (__any_sync(0xffffffffu, resc)) {
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait_bounded(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, p.err))) {
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&my_pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag,
+                                                            p.err))) {
               ok = false;
               break;
             }
@@ -455,10 +445,10 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
           m = m_new;
           const uint64_t nm2 = pk2(-m, -m);
 #pragma unroll
-          for (int g = 0; g < kPPT; ++g) {
-            const uint64_t c2 = pk2(cg[g], cg[g]);
+          for (int pg = 0; pg < kPPT; ++pg) {
+            const uint64_t c2 = pk2(cg[pg], cg[pg]);
 #pragma unroll
-            for (int i = g * (P / 2); i < (g + 1) * (P / 2); ++i) {
+            for (int i = pg * (P / 2); i < (pg + 1) * (P / 2); ++i) {
               float x0, x1;
               up2(fma2_pair(s[(2 * i) / 32][(2 * i) % 32], s[(2 * i + 1) / 32][(2 * i + 1) % 32], c2, nm2), x0,
                   x1);
@@ -469,7 +459,8 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
         // a masked slot holds zero codes: its score is 0 and its P entry is f16(2^-m)
         if (n_masked) masked += static_cast<float>(n_masked) * f16lo(pack_f16(ex2(-m), 0.f));
         if (j >= 2) {
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, p.err))) {
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(&my_pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag,
+                                                          p.err))) {
             ok = false;
             break;
           }
@@ -478,7 +469,7 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
         tmem_st32(tP + (j & 1) * (kBN / 2), pb);
         const bool more = j + 1 < n_tiles;
         if (more) {
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_full, (j + 1) & 1, abort_flag, p.err))) {
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(my_s_full, (j + 1) & 1, abort_flag, p.err))) {
             ok = false;
             break;
           }
@@ -489,16 +480,16 @@ __global__ void __launch_bounds__(tc8::kThreads, 2)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[j & 1]);
+        if (lane == 0) mbar_arrive(&my_p_full[j & 1]);
         if (more) {
           tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(s_free);
+          if (lane == 0) mbar_arrive(my_s_free);
         }
       }
       const int jl = n_tiles - 1;
-      if (__all_sync(0xffffffffu, ok && mbar_wait_bounded(&pv_done[jl & 1], (jl >> 1) & 1, abort_flag, p.err))) {
+      if (__all_sync(0xffffffffu, ok && mbar_wait_bounded(&my_pv_done[jl & 1], (jl >> 1) & 1, abort_flag, p.err))) {
         tc_fence_after();
         uint32_t o0[32], o1[32], ls[16];
         tmem_ld32(tO, o0);

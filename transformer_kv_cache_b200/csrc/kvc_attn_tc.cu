@@ -515,14 +515,18 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   if (!encode_q_tmap(&tq, a.q, a.T, a.H)) return cudaErrorInvalidValue;
   const int q_tiles = (a.T + tc::kBM - 1) / tc::kBM;
   const int total_tiles = (a.n_pages * a.P + tc::kBN - 1) / tc::kBN;
-  const int units = q_tiles * a.H;
-  int splits = a.splits > 0 ? a.splits : choose_splits(units, total_tiles, 2 * a.sm_count);
+  // a CTA of the bf16 kernel takes one query tile (two CTAs per SM); a CTA of the FP8
+  // kernel takes two (one CTA per SM)
+  const int units = a.fp8 ? ((q_tiles + 1) / 2) * a.H : q_tiles * a.H;
+  const int slots = a.fp8 ? a.sm_count : 2 * a.sm_count;
+  const int part_units = q_tiles * a.H;       // 128-row partial tiles per split
+  int splits = a.splits > 0 ? a.splits : choose_splits(units, total_tiles, slots);
   if (splits > total_tiles) splits = total_tiles;
   int tps = (total_tiles + splits - 1) / splits;
   splits = (total_tiles + tps - 1) / tps;
-  if (splits > 1 && static_cast<size_t>(units) * splits > a.part_rows) {
+  if (splits > 1 && static_cast<size_t>(part_units) * splits > a.part_rows) {
     // not enough partial scratch: fall back to as many splits as fit
-    splits = static_cast<int>(a.part_rows / units);
+    splits = static_cast<int>(a.part_rows / part_units);
     if (splits < 1) splits = 1;
     tps = (total_tiles + splits - 1) / splits;
     splits = (total_tiles + tps - 1) / tps;
