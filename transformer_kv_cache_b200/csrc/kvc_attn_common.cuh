@@ -10,6 +10,7 @@
 namespace kvc {
 
 struct TcParams {
+  const __nv_bfloat16* q;       // [T][H][D] queries
   const float* k_scale;         // FP8 storage only: per (pool page, head) scales
   const float* v_scale;
   const Entry* entries;
@@ -70,6 +71,13 @@ __device__ __forceinline__ uint32_t bf16x2_trunc(float lo, float hi) {
   uint32_t r;
   asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(__float_as_uint(lo)), "r"(__float_as_uint(hi)));
   return r;
+}
+
+// True in exactly one lane of a converged warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}" : "=r"(pred));
+  return pred != 0;
 }
 
 // Wait without the abort shortcut, used only to drain a CTA's own in-flight work.

@@ -13,15 +13,15 @@
 //                       turns every code pair into an f16 pair with the hardware E4M3
 //                       conversion (exact) and writes it as a 128-byte-swizzled MMA operand.
 //                       K codes stay unscaled; each V pair is multiplied by the page's V
-//                       scale over the CTA's largest V scale of the head. Before the first
-//                       tile, each converter widens one query tile bf16 -> f16 in place
-//                       (warp 0 lane 0 loads both query tiles).
-//   warps 1, 11         MMA issuers, one lane each, one per query tile (so the two tiles'
-//                       pipelines do not wait on each other): per KV tile S = Q K^T (M=128,
-//                       N=64) and O' += P [V | 1] (M=128, N=80), f16 inputs, fp32
-//                       accumulation in TMEM (512 columns: 256 per query tile).
-//   warps 2..5, 6..9    softmax of query tile 0 and 1: as in the bf16 kernel (one thread
-//                       per row, 64 columns per tile, lazy rescaling, row sum from the ones
+//                       scale over the CTA's largest V scale of the head.
+//   warps 1, 11         MMA issuers, one per query tile (so the two tiles' pipelines do not
+//                       wait on each other; the warp waits, one elected lane issues): per
+//                       KV tile S = Q K^T (M=128, N=64, A = Q read from TMEM) and
+//                       O' += P [V | 1] (M=128, N=80), f16 inputs, fp32 accumulation in
+//                       TMEM (512 columns: 256 per query tile).
+//   warps 2..5, 6..9    softmax of query tile 0 and 1: each thread first widens its row of
+//                       Q bf16 -> f16 into TMEM; then as in the bf16 kernel (one thread per
+//                       row, 64 columns per tile, lazy rescaling, row sum from the ones
 //                       column), with P packed as f16. The K scale of a page multiplies the
 //                       logit factor of its 16 columns, so Q K^T runs on exact decoded codes.
 //
@@ -42,17 +42,16 @@ constexpr int kCodeStages = 3;                // code staging ring of each conve
 constexpr int kStages = 4;                    // converted f16 operand ring
 constexpr int kHalfCodeBytes = (kBN / 2) * kHD;   // 2 KB: a converter's half tile of one tensor
 constexpr int kConvBytes = kBN * kHD * 2;     // 8 KB f16 tile
-constexpr int kQBytes = kBM * kHD * 2;        // 16 KB per query tile
 constexpr int kOnesBytes = kBN * kHD * 2;
 constexpr int kThreads = 384;                 // 12 warps
 constexpr int kConvThreads = 64;              // warps 0 and 10
 constexpr int kTmemCols = 512;
 constexpr int kGroupCols = 256;               // TMEM columns per query tile
-constexpr int kColS = 0, kColP = 64, kColO = 128;
+constexpr int kColS = 0, kColP = 64, kColO = 128, kColQ = 208;   // per query tile
 constexpr float kPMax = 256.0f;
 constexpr size_t kCodesBytes = 2 * kCodeStages * 2 * kHalfCodeBytes;
 constexpr size_t kSmemBytes =
-    1024 + kGroups * kQBytes + 2 * kStages * kConvBytes + kOnesBytes + kCodesBytes + 512;
+    1024 + 2 * kStages * kConvBytes + kOnesBytes + kCodesBytes + 512;
 }  // namespace tc8
 
 __device__ __forceinline__ uint32_t f16x2_of_e4m3x2(uint32_t code_pair) {
@@ -99,15 +98,14 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
   static_assert(kPPT % 2 == 0, "a KV tile splits into two halves of whole pages");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_s = smem;                                  // [kGroups] query tiles
-  uint8_t* ck_s = q_s + kGroups * kQBytes;              // converted K tiles [kStages]
+  uint8_t* ck_s = smem;                                 // converted K tiles [kStages]
   uint8_t* cv_s = ck_s + kStages * kConvBytes;          // converted V tiles [kStages]
   uint8_t* ones_s = cv_s + kStages * kConvBytes;
   uint8_t* codes = ones_s + kOnesBytes;                 // [converter][kCodeStages][K, V][half tile]
   uint64_t* bars = reinterpret_cast<uint64_t*>(codes + kCodesBytes);
-  uint64_t* q_full = bars;
-  uint64_t* q_ready = bars + 1;
-  uint64_t* c8_full = bars + 2;                         // [converter][kCodeStages]
+  uint64_t* q_ready = bars;                             // [kGroups] Q of the tile stored in TMEM
+  uint64_t* ref_ready = bars + kGroups;                 // V reference scale written
+  uint64_t* c8_full = ref_ready + 1;                    // [converter][kCodeStages]
   uint64_t* kc_full = c8_full + 2 * kCodeStages;        // [kStages] both halves converted
   uint64_t* kv_empty = kc_full + kStages;               // [kStages]
   uint64_t* s_full = kv_empty + kStages;                // [kGroups]
@@ -131,8 +129,9 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
   const int n_tiles = tile1 - tile0;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_ready, kConvThreads);
+    mbar_init(&q_ready[0], 4);
+    mbar_init(&q_ready[1], 4);
+    mbar_init(ref_ready, 1);
     for (int i = 0; i < 2 * kCodeStages; ++i) mbar_init(&c8_full[i], 1);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&kc_full[i], kConvThreads);
@@ -179,7 +178,10 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
       for (int o = 16; o > 0; o >>= 1) mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, o));
       if (mv == 0.f) mv = 1.f;                          // all-zero pages: any reference works
       const float iv = 1.f / mv;
-      if (ci == 0 && lane == 0) *sref = mv;
+      if (ci == 0 && lane == 0) {
+        *sref = mv;
+        mbar_arrive(ref_ready);
+      }
       // physical page gl of tiles ahead and its V scale; each value loaded in iteration j
       // is first used in iteration j + 1
       const int pq0 = page_entry(p, tile0 * kPPT + gl).x;
@@ -199,32 +201,16 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
       tma_load_2d(kc_ + kHalfCodeBytes + lane * P * kHD, &tmap_v, &c8f[st_], 0, row_);              \
     }                                                                                               \
   } while (0)
-      if (ci == 0 && lane == 0) {
-        tma_prefetch_desc(&tmap_q);
+      if (lane == 0) {
         tma_prefetch_desc(&tmap_k);
         tma_prefetch_desc(&tmap_v);
-        mbar_arrive_expect_tx(q_full, ngroups * kQBytes);
-        for (int g = 0; g < ngroups; ++g) tma_load_3d(q_s + g * kQBytes, &tmap_q, q_full, 0, h, (2 * qp + g) * kBM);
       }
       static_assert(kCodeStages == 3, "the issue distance below is three tiles");
       KVC_FP8_ISSUE(0, pq0);
       if (n_tiles > 1) KVC_FP8_ISSUE(1, pq1);
       if (n_tiles > 2) KVC_FP8_ISSUE(2, pq2);
       int issued = min(n_tiles, kCodeStages);
-      bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(q_full, 0, abort_flag, p.err));
-      if (ok) {
-        // query tile ci bf16 -> f16 in place (positions, hence the swizzle, unchanged)
-        if (ci < ngroups) {
-          uint32_t* q32 = reinterpret_cast<uint32_t*>(q_s + ci * kQBytes);
-#pragma unroll 8
-          for (int i = lane; i < kQBytes / 4; i += 32) {
-            const uint32_t w = q32[i];
-            q32[i] = pack_f16(bf16lo(w), bf16hi(w));
-          }
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive(q_ready);
-      }
+      bool ok = true;
       // this converter's rows of the tile: 32 ci + (lane >> 3) + 4 i, i < 8, chunk lane & 7
       // of 8 dims; in the swizzled f16 tile the chunk moves to chunk ^ (row & 7)
       const int r0 = lane >> 3, c0 = lane & 7;
@@ -287,7 +273,6 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
 #undef KVC_FP8_ISSUE
       // drain: the last code load issued into each stage has landed before the CTA exits
       if (lane == 0) {
-        if (ci == 0) mbar_wait_drain(q_full, 0, p.err);
 #pragma unroll
         for (int i = 0; i < kCodeStages; ++i)
           if (issued > i) {
@@ -297,48 +282,62 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
       }
     } else if (warp == 1 || warp == 11) {
       const int g = warp == 1 ? 0 : 1;
-      if (lane == 0 && g < ngroups) {
-        // -------------------------------------------------- MMA issuer of query tile g
+      if (g < ngroups) {
+        // ---------------------------- MMA issuer of query tile g (one elected lane issues)
         const uint32_t idesc_s = idesc_f16kind(0, kBM, kBN, 0, 0);
         const uint32_t idesc_o = idesc_f16kind(0, kBM, kON, 0, 1);
-        const uint32_t qa = smem_u32(q_s) + g * kQBytes, k_addr = smem_u32(ck_s), v_addr = smem_u32(cv_s);
+        const uint32_t k_addr = smem_u32(ck_s), v_addr = smem_u32(cv_s);
         const uint32_t ones_addr = smem_u32(ones_s);
         const uint32_t tS = tmem + g * kGroupCols + kColS, tP = tmem + g * kGroupCols + kColP;
-        const uint32_t tO = tmem + g * kGroupCols + kColO;
-        bool ok = mbar_wait_bounded(q_ready, 0, abort_flag, p.err) &&
-                  mbar_wait_bounded(&kc_full[0], 0, abort_flag, p.err);
+        const uint32_t tO = tmem + g * kGroupCols + kColO, tQ = tmem + g * kGroupCols + kColQ;
+        const bool leader = elect_one();
+        bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&q_ready[g], 0, abort_flag, p.err) &&
+                                              mbar_wait_bounded(&kc_full[0], 0, abort_flag, p.err));
         if (ok) {
           tc_fence_after();
+          if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < kHD / 16; ++kk)
-            mma_ss(tS, sw128_desc(qa + kk * 32, 16, 1024), sw128_desc(k_addr + kk * 32, 16, 1024), idesc_s, kk > 0);
-          mma_commit(&s_full[g]);
+            for (int kk = 0; kk < kHD / 16; ++kk)
+              mma_ts(tS, tQ + kk * 8, sw128_desc(k_addr + kk * 32, 16, 1024), idesc_s, kk > 0);
+            mma_commit(&s_full[g]);
+          }
+          __syncwarp();
         }
         for (int j = 0; ok && j < n_tiles; ++j) {
           const int st = j % kStages;
           if (j + 1 < n_tiles) {
             const int st1 = (j + 1) % kStages;
-            if (!mbar_wait_bounded(&kc_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.err)) break;
-            if (!mbar_wait_bounded(&s_free[g], j & 1, abort_flag, p.err)) break;
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait_bounded(&kc_full[st1], ((j + 1) / kStages) & 1, abort_flag, p.err) &&
+                                mbar_wait_bounded(&s_free[g], j & 1, abort_flag, p.err)))
+              break;
             tc_fence_after();
             const uint32_t kb = k_addr + st1 * kConvBytes;
+            if (leader) {
 #pragma unroll
-            for (int kk = 0; kk < kHD / 16; ++kk)
-              mma_ss(tS, sw128_desc(qa + kk * 32, 16, 1024), sw128_desc(kb + kk * 32, 16, 1024), idesc_s, kk > 0);
-            mma_commit(&s_full[g]);
+              for (int kk = 0; kk < kHD / 16; ++kk)
+                mma_ts(tS, tQ + kk * 8, sw128_desc(kb + kk * 32, 16, 1024), idesc_s, kk > 0);
+              mma_commit(&s_full[g]);
+            }
+            __syncwarp();
           }
-          if (!mbar_wait_bounded(&p_full[2 * g + (j & 1)], (j >> 1) & 1, abort_flag, p.err)) break;
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(&p_full[2 * g + (j & 1)], (j >> 1) & 1, abort_flag, p.err)))
+            break;
           tc_fence_after();
           const uint32_t vb = v_addr + st * kConvBytes;
           const uint32_t lbo = ones_addr - vb;
           const uint32_t pa = tP + (j & 1) * (kBN / 2);
+          if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_ts(tO, pa + kk * 8, sw128_desc(vb + kk * 2048, lbo, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&pv_done[2 * g + (j & 1)]);
-          mma_commit(&kv_empty[st]);
+            for (int kk = 0; kk < kBN / 16; ++kk)
+              mma_ts(tO, pa + kk * 8, sw128_desc(vb + kk * 2048, lbo, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&pv_done[2 * g + (j & 1)]);
+            mma_commit(&kv_empty[st]);
+          }
+          __syncwarp();
         }
-        mma_commit(&mma_final[g]);
+        if (leader) mma_commit(&mma_final[g]);
+        __syncwarp();
         mbar_wait_drain(&mma_final[g], 0, p.err);
       }
     } else if (((warp - 2) >> 2) < ngroups) {
@@ -354,7 +353,31 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
       uint64_t* my_s_free = &s_free[g];
       uint64_t* my_p_full = &p_full[2 * g];
       uint64_t* my_pv_done = &pv_done[2 * g];
-      bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(q_ready, 0, abort_flag, p.err));
+      {
+        // this row of Q, bf16 -> f16 (exact in range), into TMEM: the A operand of S
+        uint32_t qv[32];
+        const int row = qt * kBM + r;
+        if (row < p.T) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.q + (static_cast<long long>(row) * p.H + h) * kHD);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint4 w = __ldg(src + v);
+            qv[4 * v] = pack_f16(bf16lo(w.x), bf16hi(w.x));
+            qv[4 * v + 1] = pack_f16(bf16lo(w.y), bf16hi(w.y));
+            qv[4 * v + 2] = pack_f16(bf16lo(w.z), bf16hi(w.z));
+            qv[4 * v + 3] = pack_f16(bf16lo(w.w), bf16hi(w.w));
+          }
+        } else {
+#pragma unroll
+          for (int v = 0; v < 32; ++v) qv[v] = 0u;
+        }
+        tmem_st32(tbase + kColQ, qv);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_ready[g]);
+      }
+      bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(ref_ready, 0, abort_flag, p.err));
       const float vref = ok ? *sref : 1.f;
       float m = -INFINITY, masked = 0.f;
       // Lanes 0..3 hold page g = lane of the current tile (K scale, valid slots) and the

@@ -6,15 +6,18 @@
 // materialising the score matrix, as a flash-attention pipeline built for Blackwell. Each
 // CTA owns one 128-row query tile of one head and a range of 64-slot KV tiles (4 pages):
 //
-//   warp 0 (one lane)   TMA producer: the query tile once, then per KV tile the 4 pages of
-//                       K and of V, each page-head block one 2-D box, into a ring of
-//                       128-byte-swizzled stages. Pages past the end of the list are read
-//                       past the end of the pool, which TMA fills with zeros.
-//   warp 1 (one lane)   MMA issuer: S = Q K^T (tcgen05.mma kind::f16, M=128, N=64) into
+//   warp 0 (one lane)   TMA producer: per KV tile the 4 pages of K and of V, each
+//                       page-head block one 2-D box, into a ring of 128-byte-swizzled
+//                       stages. Pages past the end of the list are read past the end of the
+//                       pool, which TMA fills with zeros.
+//   warp 1              MMA issuer (the warp waits, one elected lane issues): S = Q K^T
+//                       (tcgen05.mma kind::f16, M=128, N=64, A = Q read from TMEM) into
 //                       TMEM, then O' += P [V | 1] (M=128, N=80, A = P read from TMEM,
 //                       B = the V tile as an MN-major operand followed by a constant block
 //                       of ones), so accumulator column 64 carries the row sum of P.
-//   warps 2..5          softmax, thread = query row = TMEM lane, 64 columns per tile:
+//   warps 2..5          softmax, thread = query row = TMEM lane. First each thread stores
+//                       its row of Q into TMEM (so S reads only K from shared memory);
+//                       then per KV tile, 64 columns:
 //                       x = s*c - m with packed f32x2 FMAs, P = 2^x on the MUFU, its upper
 //                       halves taken as the bf16 pairs the MMA consumes (one byte permute
 //                       per pair) and written back to TMEM (tcgen05.st); no per-element sum
@@ -33,8 +36,8 @@
 // nothing to O and 2^-m to the row sum; that amount is tracked per row and taken out.
 //
 // P is double-buffered in TMEM so a tile's softmax never waits for the previous tile's
-// P.V product. TMEM (256 columns): S [0,64), P0 [64,96), P1 [96,128), O' [128,208). Two
-// CTAs fit per SM. The KV sequence can be split across CTAs; partial outputs carry the
+// P.V product. TMEM (256 columns): S [0,64), P0 [64,96), P1 [96,128), O' [128,208),
+// Q [208,240). Two CTAs fit per SM. The KV sequence can be split across CTAs; partial outputs carry the
 // log2-sum-exp and a combine kernel merges them. Every barrier wait is bounded: on
 // timeout the CTA records KVC_ERR_TIMEOUT in the error word, drains its own copies and
 // MMAs, frees TMEM and returns.
@@ -51,13 +54,12 @@ constexpr int kHD = 64;                       // head dim (one 128-byte swizzle 
 constexpr int kON = kHD + 16;                 // O' columns: O plus the row-sum block
 constexpr int kStages = 4;
 constexpr int kTileBytes = kBN * kHD * 2;     // 8 KB (K or V tile)
-constexpr int kQBytes = kBM * kHD * 2;        // 16 KB
 constexpr int kOnesBytes = kBN * kHD * 2;     // 8 KB block of bf16 ones
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 256;
-constexpr int kColS = 0, kColP = 64, kColO = 128;
+constexpr int kColS = 0, kColP = 64, kColO = 128, kColQ = 208;   // Q: 32 columns of bf16 pairs
 constexpr float kPMax = 256.0f;               // a P above 2^8 moves the row's reference max
-constexpr size_t kSmemBytes = 1024 + kQBytes + 2 * kStages * kTileBytes + kOnesBytes + 256;
+constexpr size_t kSmemBytes = 1024 + 2 * kStages * kTileBytes + kOnesBytes + 256;
 }  // namespace tc
 
 template <int P>
@@ -68,8 +70,7 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
   constexpr int kPPT = kBN / P;               // pages per KV tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_s = smem;
-  uint8_t* k_s = smem + kQBytes;
+  uint8_t* k_s = smem;
   uint8_t* v_s = k_s + kStages * kTileBytes;
   uint8_t* ones_s = v_s + kStages * kTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ones_s + kOnesBytes);
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
   const int n_tiles = tile1 - tile0;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    mbar_init(q_full, 4);                       // the four softmax warps stored Q in TMEM
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
@@ -129,11 +130,8 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
     if (warp == 0) {
       if (lane == 0) {
         // ---------------------------------------------------------------- TMA producer
-        tma_prefetch_desc(&tmap_q);
         tma_prefetch_desc(&tmap_k);
         tma_prefetch_desc(&tmap_v);
-        mbar_arrive_expect_tx(q_full, kQBytes);
-        tma_load_3d(q_s, &tmap_q, q_full, 0, h, qt * kBM);
         int last[kStages];
 #pragma unroll
         for (int i = 0; i < kStages; ++i) last[i] = -1;
@@ -160,7 +158,6 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           last[st] = j;
         }
         // drain: every copy this CTA issued has landed before shared memory is released
-        mbar_wait_drain(q_full, 0, p.err);
 #pragma unroll
         for (int i = 0; i < kStages; ++i) {
           if (last[i] >= 0) {
@@ -170,64 +167,95 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
         }
       }
     } else if (warp == 1) {
-      if (lane == 0) {
-        // ---------------------------------------------------------------- MMA issuer
-        const uint32_t idesc_s = idesc_f16kind(1, kBM, kBN, 0, 0);
-        const uint32_t idesc_o = idesc_f16kind(1, kBM, kON, 0, 1);
-        const uint32_t tS = tmem + kColS, tP = tmem + kColP, tO = tmem + kColO;
-        const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
-        const uint32_t ones_addr = smem_u32(ones_s);
-        bool ok = mbar_wait_bounded(q_full, 0, abort_flag, p.err) &&
-                  mbar_wait_bounded(&k_full[0], 0, abort_flag, p.err);
-        if (ok) {
-          tc_fence_after();
+      // ------------------------------------------------------------------ MMA issuer
+      // the whole warp runs the loop and waits; one elected lane issues the MMAs and
+      // commits (the warp stays converged)
+      const uint32_t idesc_s = idesc_f16kind(1, kBM, kBN, 0, 0);
+      const uint32_t idesc_o = idesc_f16kind(1, kBM, kON, 0, 1);
+      const uint32_t tS = tmem + kColS, tP = tmem + kColP, tO = tmem + kColO, tQ = tmem + kColQ;
+      const uint32_t k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
+      const uint32_t ones_addr = smem_u32(ones_s);
+      const bool leader = elect_one();
+      bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(q_full, 0, abort_flag, p.err) &&
+                                            mbar_wait_bounded(&k_full[0], 0, abort_flag, p.err));
+      if (ok) {
+        tc_fence_after();
+        if (leader) {
 #pragma unroll
           for (int kk = 0; kk < kHD / 16; ++kk)
-            mma_ss(tS, sw128_desc(q_addr + kk * 32, 16, 1024), sw128_desc(k_addr + kk * 32, 16, 1024), idesc_s,
-                   kk > 0);
+            mma_ts(tS, tQ + kk * 8, sw128_desc(k_addr + kk * 32, 16, 1024), idesc_s, kk > 0);
           mma_commit(s_full);
         }
-        for (int j = 0; ok && j < n_tiles; ++j) {
-          const int st = j % kStages;
-          const uint32_t ph = (j / kStages) & 1;
-          if (j + 1 < n_tiles) {
-            const int st1 = (j + 1) % kStages;
-            const uint32_t ph1 = ((j + 1) / kStages) & 1;
-            if (!mbar_wait_bounded(s_free, j & 1, abort_flag, p.err)) break;
-            if (!mbar_wait_bounded(&k_full[st1], ph1, abort_flag, p.err)) break;
-            tc_fence_after();
-            const uint32_t kb = k_addr + st1 * kTileBytes;
+        __syncwarp();
+      }
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int st = j % kStages;
+        const uint32_t ph = (j / kStages) & 1;
+        if (j + 1 < n_tiles) {
+          const int st1 = (j + 1) % kStages;
+          const uint32_t ph1 = ((j + 1) / kStages) & 1;
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_free, j & 1, abort_flag, p.err) &&
+                                           mbar_wait_bounded(&k_full[st1], ph1, abort_flag, p.err)))
+            break;
+          tc_fence_after();
+          const uint32_t kb = k_addr + st1 * kTileBytes;
+          if (leader) {
 #pragma unroll
             for (int kk = 0; kk < kHD / 16; ++kk)
-              mma_ss(tS, sw128_desc(q_addr + kk * 32, 16, 1024), sw128_desc(kb + kk * 32, 16, 1024), idesc_s,
-                     kk > 0);
+              mma_ts(tS, tQ + kk * 8, sw128_desc(kb + kk * 32, 16, 1024), idesc_s, kk > 0);
             mma_commit(s_full);
           }
-          // one barrier per P buffer: the softmax may finish tile j + 1 before this wait,
-          // and phase j + 2 of a single barrier would alias phase j
-          if (!mbar_wait_bounded(&p_full[j & 1], (j >> 1) & 1, abort_flag, p.err)) break;
-          if (!mbar_wait_bounded(&v_full[st], ph, abort_flag, p.err)) break;
-          tc_fence_after();
-          // B = [V | ones]: the V tile is MN atom 0, the ones block MN atom 1 (LBO apart)
-          const uint32_t vb = v_addr + st * kTileBytes;
-          const uint32_t lbo = ones_addr - vb;
-          const uint32_t pa = tP + (j & 1) * (kBN / 2);
+          __syncwarp();
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&p_full[j & 1], (j >> 1) & 1, abort_flag, p.err) &&
+                                         mbar_wait_bounded(&v_full[st], ph, abort_flag, p.err)))
+          break;
+        tc_fence_after();
+        const uint32_t vb = v_addr + st * kTileBytes;
+        const uint32_t lbo = ones_addr - vb;
+        const uint32_t pa = tP + (j & 1) * (kBN / 2);
+        if (leader) {
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
             mma_ts(tO, pa + kk * 8, sw128_desc(vb + kk * 2048, lbo, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&pv_done[j & 1]);
           mma_commit(&kv_empty[st]);
         }
-        // drain: all MMAs of this CTA complete before TMEM is released
-        mma_commit(mma_final);
-        mbar_wait_drain(mma_final, 0, p.err);
+        __syncwarp();
       }
+      if (leader) mma_commit(mma_final);
+      __syncwarp();
+      mbar_wait_drain(mma_final, 0, p.err);
     } else {
       // ------------------------------------------------------------------ softmax warps
       const int wq = warp & 3;                      // TMEM lane quadrant this warp may access
       const int r = wq * 32 + lane;                 // query row within the tile
       const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
       const uint32_t tS = tmem + kColS + lane_off, tP = tmem + kColP + lane_off, tO = tmem + kColO + lane_off;
+      {
+        // this row of Q into TMEM (the A operand of S = Q K^T): 64 bf16 = 32 packed columns
+        uint32_t qv[32];
+        const int row = qt * kBM + r;
+        if (row < p.T) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.q + (static_cast<long long>(row) * p.H + h) * kHD);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint4 w = __ldg(src + v);
+            qv[4 * v] = w.x;
+            qv[4 * v + 1] = w.y;
+            qv[4 * v + 2] = w.z;
+            qv[4 * v + 3] = w.w;
+          }
+        } else {
+#pragma unroll
+          for (int v = 0; v < 32; ++v) qv[v] = 0u;
+        }
+        tmem_st32(tmem + kColQ + lane_off, qv);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_full);
+      }
       const float c = p.scale_log2;
       float m = -INFINITY;       // reference max (log2 domain) of the row
       float masked = 0.f;        // row-sum share of zero-padded slots, rescaled like O'
@@ -532,6 +560,7 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
     splits = (total_tiles + tps - 1) / tps;
   }
   TcParams prm;
+  prm.q = static_cast<const __nv_bfloat16*>(a.q);
   prm.k_scale = a.k_scale;
   prm.v_scale = a.v_scale;
   prm.entries = a.entries;
