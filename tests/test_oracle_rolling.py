@@ -1,0 +1,153 @@
+"""CPU pins of the rolling diversity-pruned memory oracle ("InfiniteVGGT" explainer page):
+scipy's cosine distance and softmax, brute-force Top-K, the page's worked numbers and
+closed-form cases, and a planted mistake that the pins must catch."""
+import numpy as np
+import pytest
+from scipy.spatial.distance import cosine
+from scipy.special import softmax
+
+import oracle.rolling_oracle as ro
+from oracle import RollingOracle, diversity_scores, layer_budgets, top_k
+
+
+def _scores_by_scipy(Kc):
+    kh = [k / np.linalg.norm(k) for k in Kc]
+    mu = np.sum(kh, axis=0)
+    return np.array([-(1.0 - cosine(k, mu)) for k in Kc])
+
+
+def test_scores_are_negative_cosine_to_mean_key():
+    rng = np.random.default_rng(0)
+    Kc = rng.standard_normal((300, 64)) * np.exp(rng.standard_normal(300))[:, None]
+    np.testing.assert_allclose(diversity_scores(Kc), _scores_by_scipy(Kc), rtol=0, atol=1e-14)
+
+
+def test_unique_direction_scores_highest():
+    # n copies of one direction and one orthogonal key: the orthogonal key is the most
+    # diverse (score -1/sqrt(n^2+1) against -n/sqrt(n^2+1) for the copies)
+    n, D = 40, 16
+    Kc = np.zeros((n + 1, D))
+    Kc[:n, 0] = 2.0 ** np.arange(n) % 7 + 1.0       # different lengths, same direction
+    Kc[n, 3] = 5.0
+    sc = diversity_scores(Kc)
+    assert np.argmax(sc) == n
+    np.testing.assert_allclose(sc[n], -1.0 / np.sqrt(n * n + 1), rtol=1e-15)
+    np.testing.assert_allclose(sc[:n], -n / np.sqrt(n * n + 1), rtol=1e-15)
+
+
+def test_scores_invariant_to_positive_key_scaling():
+    rng = np.random.default_rng(1)
+    Kc = rng.standard_normal((50, 32))
+    K2 = Kc.copy()
+    K2[7] *= 8.0                                   # a power of two: the normalised key is identical
+    K2[19] *= 0.25
+    assert np.array_equal(diversity_scores(Kc), diversity_scores(K2))
+
+
+def test_zero_key_has_no_direction():
+    Kc = np.eye(4)
+    Kc[2] = 0.0
+    sc = diversity_scores(Kc)
+    assert sc[2] == 0.0 and np.all(np.isfinite(sc))
+
+
+def test_worked_example_1200_candidates_keep_512_drop_688():
+    rng = np.random.default_rng(2)
+    Kc = rng.standard_normal((1200, 64))
+    ids = np.arange(1200) * 3 + 11
+    sc = diversity_scores(Kc)
+    keep = top_k(sc, ids, 512)
+    assert len(keep) == 512 and 1200 - len(keep) == 688
+    # brute force: the kept set is exactly the 512 largest scores (no ties here)
+    want = set(np.argsort(-sc, kind="stable")[:512].tolist())
+    assert set(keep.tolist()) == want
+    assert np.all(np.diff(ids[keep]) > 0)           # stored in ascending id
+
+
+def test_ties_go_to_lower_ids():
+    Kc = np.ones((10, 8))
+    ids = np.arange(10)[::-1].copy()                # ids 9..0
+    keep = top_k(diversity_scores(Kc), ids, 4)
+    assert sorted(ids[keep].tolist()) == [0, 1, 2, 3]
+
+
+def test_budget_arithmetic_of_the_page():
+    # 512 tokens per head, 16 heads -> 8,192 per layer; 12 layers -> 98,304 (~98k)
+    b = layer_budgets([0.3] * 12, 1.0, 512)
+    assert b == [512] * 12
+    assert sum(x * 16 for x in b) == 98304
+    assert layer_budgets([0.1, 0.9, 0.5], 0.0, 512) == [512, 512, 512]
+
+
+def test_layer_budgets_follow_softmax_of_mean_diversity():
+    d = [-0.9, -0.5, -0.7, -0.2]
+    for tau in (0.05, 0.2, 1.0):
+        b = layer_budgets(d, tau, 512)
+        p = softmax(np.array(d) / tau)
+        np.testing.assert_array_equal(b, np.floor(4 * 512 * p).astype(int))
+        assert sum(b) <= 4 * 512
+        assert b[3] == max(b) and b[0] == min(b)   # more diverse layer, more memory
+
+
+def _stream(T=20, H=3, D=16, K=30, frames=7, seed=3):
+    rng = np.random.default_rng(seed)
+    orc = RollingOracle(2, H, D, T, K, 0.25)
+    seen = []
+    for t in range(frames):
+        q = rng.standard_normal((T, H, D))
+        k = rng.standard_normal((T, H, D))
+        v = rng.standard_normal((T, H, D))
+        seen.append((q, k, v))
+        orc.append(0, t, k, v)
+        out = orc.attend(0, q)
+        yield t, orc, (q, k, v), out
+
+
+def test_anchor_immutable_and_memory_bounded():
+    T, K = 20, 30
+    for t, orc, _, _ in _stream(T=T, K=K):
+        for h in range(3):
+            ids = orc.head_ids(0, h)
+            assert np.array_equal(ids[:T], np.arange(T))              # frame 0 kept whole
+            mut = orc.mut_ids[0][h]
+            assert len(mut) == min(K, T * t)                         # bounded at K
+            assert np.all(mut >= T) and np.all(np.diff(mut) > 0)
+
+
+def test_kept_set_is_top_k_of_candidates_each_frame():
+    # brute force on one head: candidates = previous kept + new frame, scored by scipy
+    T, H, D, K = 20, 3, 16, 30
+    prev = {h: (np.zeros(0, int), np.zeros((0, D))) for h in range(H)}
+    for t, orc, (q, k, v), _ in _stream(T=T, H=H, D=D, K=K):
+        if t == 0:
+            continue
+        for h in range(H):
+            ids = np.concatenate([prev[h][0], t * T + np.arange(T)])
+            Kc = np.concatenate([prev[h][1], k[:, h, :]])
+            sc = _scores_by_scipy(Kc)
+            order = sorted(range(len(ids)), key=lambda i: (-round(sc[i], 12), ids[i]))[:K]
+            assert set(ids[order].tolist()) == set(orc.mut_ids[0][h].tolist())
+            sel = sorted(order, key=lambda i: ids[i])
+            prev[h] = (ids[sel], Kc[sel])
+
+
+def test_attention_is_softmax_over_anchor_and_kept():
+    from scipy.special import softmax as sm
+    for t, orc, (q, k, v), out in _stream():
+        for h in range(3):
+            Kh = np.concatenate([orc.anchor_k[0][h], orc.mut_k[0][h]])
+            Vh = np.concatenate([orc.anchor_v[0][h], orc.mut_v[0][h]])
+            want = sm(q[:, h, :] @ Kh.T * 0.25, axis=1) @ Vh
+            np.testing.assert_allclose(out[:, h, :], want, rtol=0, atol=1e-12)
+
+
+def test_planted_sign_mistake_is_caught(monkeypatch):
+    # scoring by +cos (similarity) instead of -cos keeps the duplicates: the unique-key
+    # pin must fail
+    real = ro.diversity_scores
+    monkeypatch.setattr(ro, "diversity_scores", lambda Kc: -real(Kc))
+    n = 40
+    Kc = np.zeros((n + 1, 16))
+    Kc[:n, 0] = 1.0
+    Kc[n, 3] = 1.0
+    assert np.argmax(ro.diversity_scores(Kc)) != n
