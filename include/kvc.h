@@ -100,7 +100,9 @@ typedef struct {
   int32_t protect_first_frame;  /* 1: every token of frame 0 is always kept */
   int32_t max_frames;           /* cap on cached frames when W <= 0 and B == 0 */
   int32_t kv_splits;            /* KV splits per query tile in attention; 0 = automatic */
-  int32_t reserved[7];          /* must be zero */
+  int32_t diversity_budget;     /* K > 0: rolling diversity-pruned memory, K kept tokens per
+                                   head per layer besides the first frame (see kvc_attend) */
+  int32_t reserved[6];          /* must be zero */
 } kvc_config;
 
 /* Cache statistics ([GCT] Cache Monitoring: occupancy, memory use, eviction status). */
@@ -236,6 +238,34 @@ KVC_API kvc_status kvc_step_host(kvc_cache* c, int32_t layer, int32_t frame_idx,
 KVC_API kvc_status kvc_step_host_async(kvc_cache* c, int32_t layer, int32_t frame_idx, int32_t is_keyframe,
                                        const void* q_host, const void* k_host, const void* v_host,
                                        void* o_host);
+
+/* ---- Rolling diversity-pruned memory (diversity_budget = K > 0; [IVG] Building Blocks,
+ * Step-by-step recipe). Requires bf16 I/O and storage, head_dim 64, page_size 16, no
+ * window and no token budget. Every head keeps its own tokens: the first frame appended
+ * to a layer is its immutable anchor (all heads); each later frame joins the candidates,
+ * and kvc_attend first prunes each head to its Top-K candidates by diversity score
+ * (negative cosine of the L2-normalised key to the mean normalised candidate key; ties to
+ * the lower token id; fp64), then attends over anchor + kept. is_keyframe must be 1. */
+
+/* Per-layer budgets (tokens per head), each in [1, diversity_budget], from the next
+ * pruning on ([IVG] layer-wise adaptive budgets: the caller turns the layers' mean
+ * diversities into budgets, e.g. floor(L * k * softmax(mean / tau)) for an average k;
+ * diversity_budget is the largest budget a layer can take, as it sizes the pools).
+ * budgets: host array of num_layers values. Errors: KVC_ERR_ARG, KVC_ERR_STATE (not in
+ * this mode). */
+KVC_API kvc_status kvc_set_layer_budgets(kvc_cache* c, const int32_t* budgets, int32_t n);
+
+/* Mean diversity score of the layer's last pruning over all heads' candidates (fp64:
+ * per head the scores summed in ascending token id, then the heads in order, divided by
+ * H * candidates). Synchronises. Errors: KVC_ERR_STATE if the layer was never pruned. */
+KVC_API kvc_status kvc_layer_diversity(kvc_cache* c, int32_t layer, double* mean_out);
+
+/* Token ids (frame * T + slot) that head `head` of `layer` attends, in cache order
+ * (anchor, then the kept tokens in ascending id, then a pending frame). ids_out: host
+ * array of `capacity` entries; *n_out receives the count. Synchronises. Errors:
+ * KVC_ERR_ARG (capacity too small), KVC_ERR_STATE (not in this mode). */
+KVC_API kvc_status kvc_head_tokens(kvc_cache* c, int32_t layer, int32_t head, int64_t* ids_out, int32_t capacity,
+                                   int32_t* n_out);
 
 /* Wait for all work of the cache and report any latched device error. */
 KVC_API kvc_status kvc_synchronize(kvc_cache* c);

@@ -60,6 +60,7 @@ class Workload:
     rank_window: int = 5
     residual_dim: int = 1024
     protect_first_frame: int = 1
+    diversity_budget: int = 0
     description: str = ""
 
     def as_dict(self) -> Dict:
@@ -103,6 +104,13 @@ WORKLOADS: Dict[str, Workload] = {
         keyframe_interval=1, num_frames=10000, io_dtype="bf16", kv_dtype="fp8_e4m3",
         softmax_scale=0.125, temporal_keys=False, outlier_fraction=0.01,
         description="518x518 frames, 1374 tok/frame, W=128, S=8, FP8 E4M3 K/V, 10000 frames"),
+    "vggt_infinite_12l": Workload(
+        name="vggt_infinite_12l", num_layers=12, num_heads=16, head_dim=64, tokens_per_frame=1004,
+        num_special_tokens=5, page_size=16, window_frames=0, scale_frames=0,
+        keyframe_interval=1, num_frames=1000, io_dtype="bf16", kv_dtype="bf16",
+        softmax_scale=0.125, temporal_keys=True, diversity_budget=512,
+        description="rolling diversity-pruned memory: 12 layers, 512 kept tokens per head (8,192 per "
+                    "layer, ~98k total) besides the first frame, 518x378 frames, 1000 frames"),
 }
 
 

@@ -1,0 +1,105 @@
+"""GPU parity of the rolling diversity-pruned memory ("InfiniteVGGT" explainer page)
+through the C ABI: every head's kept token ids and every layer's mean diversity bit for
+bit, attention outputs within the bf16 tolerance, against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+from kvc_gpu_util import compare_out, np64, sample_rows
+from kvc_streams import WORKLOADS, FrameStream
+from oracle import RollingOracle, layer_budgets
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kvc():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    import transformer_kv_cache_b200 as m
+    return m
+
+
+def run_rolling(kvc, wl, frames, rows=None, budgets_at=None, check_ids=True, seed=11):
+    dev = torch.device("cuda")
+    L, H, D, T = wl.num_layers, wl.num_heads, wl.head_dim, wl.tokens_per_frame
+    h = kvc.kvc_create(kvc.config_from_workload(wl))
+    try:
+        st = FrameStream(wl, seed=seed, device=dev)
+        orc = RollingOracle(L, H, D, T, wl.diversity_budget, wl.softmax_scale)
+        o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+        for t in range(frames):
+            if budgets_at is not None and t in budgets_at:
+                kvc.kvc_set_layer_budgets(h, budgets_at[t])
+                orc.set_budgets(budgets_at[t])
+            for l in range(L):
+                q, k, v = st.frame(l, t)
+                kvc.kvc_append_frame(h, l, t, k, v, True)
+                kvc.kvc_attend(h, l, q, o)
+                orc.append(l, t, np64(k), np64(v))
+                ref = orc.attend(l, np64(q), rows=rows)
+                torch.cuda.synchronize()
+                got = np64(o) if rows is None else np64(o)[rows]
+                compare_out(got, ref, "bf16", f"frame {t} layer {l}")
+                if check_ids:
+                    for hh in range(H):
+                        ids = kvc.kvc_head_tokens(h, l, hh)
+                        assert np.array_equal(ids, orc.head_ids(l, hh)), f"kept ids differ: frame {t} layer {l} head {hh}"
+                if t >= 1:
+                    assert kvc.kvc_layer_diversity(h, l) == orc.layer_diversity(l)
+                _, info = kvc.kvc_page_table(h, l)
+                assert info["device_error"] == 0
+        return orc
+    finally:
+        kvc.kvc_destroy(h)
+
+
+@pytest.mark.parametrize("T,H,K,frames", [
+    (150, 4, 200, 7),    # candidates 350 -> 200 kept per head from the second pruning on
+    (150, 4, 100, 5),    # K not a multiple of the page size
+    (40, 2, 400, 6),     # K above the candidates for several frames: nothing pruned yet
+    (10, 2, 25, 6),      # T < P: every page partial
+])
+def test_rolling_memory_small(kvc, T, H, K, frames):
+    wl = WORKLOADS["vggt_infinite_12l"].replace(num_layers=2, tokens_per_frame=T, num_heads=H, diversity_budget=K,
+                                                num_special_tokens=min(5, T))
+    run_rolling(kvc, wl, frames)
+
+
+def test_layer_budgets_between_frames(kvc):
+    """Per-layer budgets set between frames (the softmax rule on the previous frame's
+    layer averages; the configured K is the largest budget a layer can take, since it
+    sizes the pools) take effect at the next pruning."""
+    wl = WORKLOADS["vggt_infinite_12l"].replace(num_layers=3, tokens_per_frame=120, num_heads=2,
+                                                diversity_budget=160)
+    b = layer_budgets([-0.2, -0.6, -0.4], 1.0, 120)     # an average of 120 per head
+    assert max(b) <= 160 and min(b) < 120 < max(b)       # the configured K caps every layer
+    run_rolling(kvc, wl, 6, budgets_at={3: b, 5: [160, 7, 33]})
+
+
+def test_rolling_memory_full_size_sampled(kvc):
+    """The page's shape on one layer: 1,004 tokens per frame, 16 heads, 512 kept per head
+    (1,516 candidates per head per frame), sampled query rows."""
+    wl = WORKLOADS["vggt_infinite_12l"].replace(num_layers=1)
+    run_rolling(kvc, wl, 4, rows=sample_rows(wl.tokens_per_frame, 48, seed=4))
+
+
+def test_rolling_memory_errors(kvc):
+    wl = WORKLOADS["vggt_infinite_12l"].replace(num_layers=2, tokens_per_frame=64, num_heads=2,
+                                                diversity_budget=64)
+    h = kvc.kvc_create(kvc.config_from_workload(wl))
+    try:
+        k = torch.zeros((64, 2, 64), dtype=torch.bfloat16, device="cuda")
+        with pytest.raises(kvc.KVCError):
+            kvc.kvc_append_frame(h, 0, 0, k, k, False)         # every frame is a candidate
+        with pytest.raises(kvc.KVCError):
+            kvc.kvc_set_layer_budgets(h, [64, 65])             # above the configured K
+        with pytest.raises(kvc.KVCError):
+            kvc.kvc_layer_diversity(h, 0)                       # never pruned
+        with pytest.raises(kvc.KVCError):
+            kvc.kvc_token_meta(h, 0)                            # not in this mode
+    finally:
+        kvc.kvc_destroy(h)
+    bad = wl.replace(kv_dtype="fp8_e4m3")
+    with pytest.raises(kvc.KVCError):
+        kvc.kvc_create(kvc.config_from_workload(bad))

@@ -28,7 +28,7 @@ EXPORTS = ["kvc_create", "kvc_destroy", "kvc_set_stream", "kvc_reset", "kvc_appe
            "kvc_compress", "kvc_page_table", "kvc_token_meta", "kvc_last_merge", "kvc_export_pages",
            "kvc_step_host", "kvc_synchronize", "kvc_last_error", "kvc_status_string", "kvc_version",
            "kvc_debug_fail_allocs", "kvc_debug_bounded_wait", "kvc_attend_paged_noalloc", "kvc_append_frame_all",
-           "kvc_step_host_async"]
+           "kvc_step_host_async", "kvc_set_layer_budgets", "kvc_layer_diversity", "kvc_head_tokens"]
 
 
 class kvc_config(ctypes.Structure):
@@ -39,7 +39,8 @@ class kvc_config(ctypes.Structure):
                 ("budget_tokens", ctypes.c_int32), ("keep_frac", ctypes.c_float), ("lambda_", ctypes.c_float),
                 ("rank_window", ctypes.c_int32), ("residual_dim", ctypes.c_int32),
                 ("protect_first_frame", ctypes.c_int32), ("max_frames", ctypes.c_int32),
-                ("kv_splits", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
+                ("kv_splits", ctypes.c_int32), ("diversity_budget", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 6)]
 
 
 class kvc_info(ctypes.Structure):
@@ -80,6 +81,9 @@ def _load():
         "kvc_export_pages": ([vp, i32, i32, i32, vp, vp, fp, fp], i32),
         "kvc_step_host": ([vp, i32, i32, i32, vp, vp, vp, vp], i32),
         "kvc_step_host_async": ([vp, i32, i32, i32, vp, vp, vp, vp], i32),
+        "kvc_set_layer_budgets": ([vp, vp, i32], i32),
+        "kvc_layer_diversity": ([vp, i32, vp], i32),
+        "kvc_head_tokens": ([vp, i32, i32, vp, i32, vp], i32),
         "kvc_synchronize": ([vp], i32),
         "kvc_last_error": ([vp], ctypes.c_char_p),
         "kvc_status_string": ([i32], ctypes.c_char_p),
@@ -128,7 +132,7 @@ def _check(handle, st: int):
 def make_config(num_layers, num_heads, head_dim, tokens_per_frame, num_special_tokens, page_size,
                 window_frames, scale_frames, io_dtype="bf16", kv_dtype="bf16", softmax_scale=0.125,
                 budget_tokens=0, keep_frac=0.6, lam=0.5, rank_window=5, residual_dim=1024,
-                protect_first_frame=1, max_frames=0, kv_splits=0) -> kvc_config:
+                protect_first_frame=1, max_frames=0, kv_splits=0, diversity_budget=0) -> kvc_config:
     c = kvc_config()
     c.num_layers, c.num_heads, c.head_dim = num_layers, num_heads, head_dim
     c.tokens_per_frame, c.num_special_tokens, c.page_size = tokens_per_frame, num_special_tokens, page_size
@@ -139,6 +143,7 @@ def make_config(num_layers, num_heads, head_dim, tokens_per_frame, num_special_t
     c.budget_tokens, c.keep_frac, c.lambda_ = budget_tokens, keep_frac, lam
     c.rank_window, c.residual_dim, c.protect_first_frame = rank_window, residual_dim, protect_first_frame
     c.max_frames, c.kv_splits = max_frames, kv_splits
+    c.diversity_budget = diversity_budget
     return c
 
 
@@ -148,7 +153,8 @@ def config_from_workload(wl, **over) -> kvc_config:
              page_size=wl.page_size, window_frames=wl.window_frames, scale_frames=wl.scale_frames,
              io_dtype=wl.io_dtype, kv_dtype=wl.kv_dtype, softmax_scale=wl.softmax_scale,
              budget_tokens=wl.budget_tokens, keep_frac=wl.keep_frac, lam=wl.lam, rank_window=wl.rank_window,
-             residual_dim=wl.residual_dim, protect_first_frame=wl.protect_first_frame)
+             residual_dim=wl.residual_dim, protect_first_frame=wl.protect_first_frame,
+             diversity_budget=getattr(wl, "diversity_budget", 0))
     d.update(over)
     return make_config(**d)
 
@@ -259,6 +265,24 @@ def kvc_step_host_async(handle, layer: int, frame_idx: int, is_keyframe: bool, q
     unread) until kvc_synchronize."""
     _check(handle, _lib.kvc_step_host_async(handle, layer, frame_idx, int(bool(is_keyframe)), _ptr(q_host),
                                             _ptr(k_host), _ptr(v_host), _ptr(o_host)))
+
+
+def kvc_set_layer_budgets(handle, budgets) -> None:
+    arr = (ctypes.c_int32 * len(budgets))(*[int(b) for b in budgets])
+    _check(handle, _lib.kvc_set_layer_budgets(handle, arr, len(budgets)))
+
+
+def kvc_layer_diversity(handle, layer: int) -> float:
+    out = ctypes.c_double()
+    _check(handle, _lib.kvc_layer_diversity(handle, layer, ctypes.byref(out)))
+    return float(out.value)
+
+
+def kvc_head_tokens(handle, layer: int, head: int, capacity: int = 1 << 20):
+    ids = np.zeros(capacity, np.int64)
+    n = ctypes.c_int32()
+    _check(handle, _lib.kvc_head_tokens(handle, layer, head, ids.ctypes.data, capacity, ctypes.byref(n)))
+    return ids[: n.value].copy()
 
 
 def kvc_synchronize(handle) -> None:

@@ -39,7 +39,7 @@ void free_all(kvc_cache* c) {
   void* ptrs[] = {c->k_pool,     c->v_pool,     c->k_scale,    c->v_scale,    c->entries,    c->bitmap,
                   c->d_err,      c->tok_id,     c->tok_cnt,    c->tok_shat,   c->cmp_scratch, c->part_o,
                   c->part_lse,   c->stage_q[0], c->stage_k[0], c->stage_v[0], c->stage_o[0], c->stage_q[1],
-                  c->stage_k[1], c->stage_v[1], c->stage_o[1], c->rank_hist};
+                  c->stage_k[1], c->stage_v[1], c->stage_o[1], c->rank_hist, c->div_sums};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   for (int i = 0; i < 2; ++i) {
@@ -65,7 +65,10 @@ kvc_status cuda_fail(kvc_cache* c, cudaError_t e, const char* where) {
 
 size_t dtype_bytes(int dt) { return dt == KVC_F32 ? 4 : (dt == KVC_BF16 ? 2 : 1); }
 
-Entry* layer_entries(kvc_cache* c, int layer) { return c->entries + static_cast<size_t>(layer) * c->pool_pages; }
+// A layer's page list (in per-head mode: head 0's).
+Entry* layer_entries(kvc_cache* c, int layer) {
+  return c->entries + static_cast<size_t>(layer) * (c->per_head ? c->cfg.num_heads : 1) * c->pool_pages;
+}
 uint32_t* layer_bitmap(kvc_cache* c, int layer) {
   return c->bitmap + static_cast<size_t>(layer) * c->bitmap_words;
 }
@@ -148,7 +151,7 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   if (!cfg || !out) return KVC_ERR_ARG;
   *out = nullptr;
   const kvc_config& g = *cfg;
-  for (int i = 0; i < 7; ++i)
+  for (int i = 0; i < 6; ++i)
     if (g.reserved[i] != 0) return KVC_ERR_ARG;
   const bool dims_ok = g.num_layers >= 1 && g.num_heads >= 1 && g.tokens_per_frame >= 1 && g.page_size >= 1 &&
                        g.num_special_tokens >= 0 && g.num_special_tokens <= g.tokens_per_frame &&
@@ -166,7 +169,19 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
         g.residual_dim < 1 || !(g.lambda_ >= 0.f) || g.budget_tokens > (1 << 24))
       return KVC_ERR_ARG;
   }
-  if (g.window_frames <= 0 && g.budget_tokens == 0 && g.max_frames < 1) return KVC_ERR_ARG;
+  if (g.diversity_budget < 0) return KVC_ERR_ARG;
+  if (g.diversity_budget > 0) {
+    // rolling diversity-pruned memory: bf16 tensor-core path, no window, no token budget;
+    // a head's candidates (kept pages + one frame) fit the pruning kernel's shared memory
+    const int ppf = (g.tokens_per_frame + g.page_size - 1) / g.page_size;
+    if (g.io_dtype != KVC_BF16 || g.kv_dtype != KVC_BF16 || g.head_dim != 64 || g.page_size != 16 ||
+        g.num_heads > kMaxBatchLayers ||
+        g.window_frames > 0 || g.budget_tokens > 0 ||
+        (g.diversity_budget + g.page_size - 1) / g.page_size + ppf > 340)
+      return KVC_ERR_ARG;
+  } else if (g.window_frames <= 0 && g.budget_tokens == 0 && g.max_frames < 1) {
+    return KVC_ERR_ARG;
+  }
   if (g.kv_splits < 0) return KVC_ERR_ARG;
 
   kvc_cache* c = new (std::nothrow) kvc_cache();
@@ -177,7 +192,13 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device);
   const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads, D = g.head_dim;
   c->ppf = (T + P - 1) / P;
-  if (g.window_frames > 0) {
+  c->per_head = g.diversity_budget > 0;
+  if (c->per_head) {
+    // per head: anchor frame, kept pages twice (old and new during a pruning), one frame
+    const int kp = (g.diversity_budget + P - 1) / P;
+    c->pool_pages = 2 * c->ppf + 2 * kp + 2;
+    c->layer_budget.assign(g.num_layers, g.diversity_budget);
+  } else if (g.window_frames > 0) {
     c->pool_pages = (g.scale_frames + g.window_frames + 1) * c->ppf;
   } else if (g.budget_tokens > 0) {
     const int B = g.budget_tokens;
@@ -192,9 +213,11 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
     delete c;
     return KVC_ERR_ARG;
   }
-  c->page_elems = static_cast<size_t>(H) * P * D;
+  // pages hold all heads ([page][head][slot][dim]), or one head per sub-layer
+  c->page_elems = static_cast<size_t>(c->per_head ? 1 : H) * P * D;
   c->page_bytes_kv = c->page_elems * c->elem_kv;
   const size_t L = g.num_layers;
+  const size_t NS = c->per_head ? L * H : L;   // page lists (sub-layers)
   const size_t frame_bytes = static_cast<size_t>(T) * H * D * c->elem_io;
   c->tc_path = g.io_dtype == KVC_BF16 && (g.kv_dtype == KVC_BF16 || g.kv_dtype == KVC_FP8_E4M3) && D == 64 && P == 16;
   const int q_tiles = (T + 127) / 128;
@@ -204,14 +227,18 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   auto A = [&](cudaError_t r) {
     if (e == cudaSuccess) e = r;
   };
-  A(dev_alloc_t(&c->k_pool, L * c->pool_pages * c->page_bytes_kv));
-  A(dev_alloc_t(&c->v_pool, L * c->pool_pages * c->page_bytes_kv));
+  A(dev_alloc_t(&c->k_pool, NS * c->pool_pages * c->page_bytes_kv));
+  A(dev_alloc_t(&c->v_pool, NS * c->pool_pages * c->page_bytes_kv));
   if (g.kv_dtype == KVC_FP8_E4M3) {
     A(dev_alloc_t(&c->k_scale, L * c->pool_pages * H * sizeof(float)));
     A(dev_alloc_t(&c->v_scale, L * c->pool_pages * H * sizeof(float)));
   }
-  A(dev_alloc_t(&c->entries, L * c->pool_pages * sizeof(Entry)));
-  A(dev_alloc_t(&c->bitmap, L * c->bitmap_words * sizeof(uint32_t)));
+  A(dev_alloc_t(&c->entries, NS * c->pool_pages * sizeof(Entry)));
+  A(dev_alloc_t(&c->bitmap, NS * c->bitmap_words * sizeof(uint32_t)));
+  if (c->per_head) {
+    A(dev_alloc_t(&c->tok_id, NS * c->pool_pages * P * sizeof(int64_t)));
+    A(dev_alloc_t(&c->div_sums, NS * sizeof(double)));
+  }
   A(dev_alloc_t(&c->d_err, 4 * sizeof(int)));
   if (c->tc_path) {
     A(dev_alloc_t(&c->part_o, c->part_rows * 128 * 64 * sizeof(float)));
@@ -246,14 +273,18 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
     return KVC_ERR_OOM;
   }
   // zero everything once so masked slots and unused pages never hold non-finite bytes
-  A(cudaMemsetAsync(c->k_pool, 0, L * c->pool_pages * c->page_bytes_kv, c->stream));
-  A(cudaMemsetAsync(c->v_pool, 0, L * c->pool_pages * c->page_bytes_kv, c->stream));
+  A(cudaMemsetAsync(c->k_pool, 0, NS * c->pool_pages * c->page_bytes_kv, c->stream));
+  A(cudaMemsetAsync(c->v_pool, 0, NS * c->pool_pages * c->page_bytes_kv, c->stream));
   if (c->k_scale) A(cudaMemsetAsync(c->k_scale, 0, L * c->pool_pages * H * sizeof(float), c->stream));
   if (c->v_scale) A(cudaMemsetAsync(c->v_scale, 0, L * c->pool_pages * H * sizeof(float), c->stream));
-  A(cudaMemsetAsync(c->entries, 0, L * c->pool_pages * sizeof(Entry), c->stream));
-  A(cudaMemsetAsync(c->bitmap, 0, L * c->bitmap_words * sizeof(uint32_t), c->stream));
+  A(cudaMemsetAsync(c->entries, 0, NS * c->pool_pages * sizeof(Entry), c->stream));
+  A(cudaMemsetAsync(c->bitmap, 0, NS * c->bitmap_words * sizeof(uint32_t), c->stream));
+  if (c->per_head) {
+    A(cudaMemsetAsync(c->tok_id, 0xff, NS * c->pool_pages * P * sizeof(int64_t), c->stream));
+    A(cudaMemsetAsync(c->div_sums, 0, NS * sizeof(double), c->stream));
+  }
   A(cudaMemsetAsync(c->d_err, 0, 4 * sizeof(int), c->stream));
-  if (c->tok_id) {
+  if (g.budget_tokens > 0) {
     const size_t slots = L * c->pool_pages * P;
     A(cudaMemsetAsync(c->tok_id, 0, slots * sizeof(int64_t), c->stream));
     A(cudaMemsetAsync(c->tok_cnt, 0, slots * sizeof(int32_t), c->stream));
@@ -302,14 +333,124 @@ kvc_status kvc_set_stream(kvc_cache* c, void* stream) {
 kvc_status kvc_reset(kvc_cache* c) {
   if (!c) return KVC_ERR_ARG;
   const size_t L = c->cfg.num_layers;
-  cudaError_t e = cudaMemsetAsync(c->entries, 0, L * c->pool_pages * sizeof(Entry), c->stream);
-  if (e == cudaSuccess) e = cudaMemsetAsync(c->bitmap, 0, L * c->bitmap_words * sizeof(uint32_t), c->stream);
+  const size_t NS = c->per_head ? L * c->cfg.num_heads : L;
+  cudaError_t e = cudaMemsetAsync(c->entries, 0, NS * c->pool_pages * sizeof(Entry), c->stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->bitmap, 0, NS * c->bitmap_words * sizeof(uint32_t), c->stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(c->d_err, 0, 4 * sizeof(int), c->stream);
   if (e != cudaSuccess) return cuda_fail(c, e, "kvc_reset");
   c->L.assign(c->cfg.num_layers, LayerHost());
   c->hist_frame = -1;
   c->hist_next_layer = 0;
   c->hist_layers.clear();
+  return KVC_OK;
+}
+
+// ---------------------------------------------------------- rolling diversity-pruned memory
+// Sub-layer (layer, head) = layer * H + head: its own page list, bitmap and pool region.
+// The first frame appended to a layer is the anchor; a later frame is pending until
+// kvc_attend prunes every head's candidates (kept pages + the frame's pages) to its
+// Top-K ("InfiniteVGGT" explainer, Step-by-step recipe: prune, then attend).
+kvc_status div_append(kvc_cache* c, int layer, int frame_idx, const void* k_dev, const void* v_dev) {
+  LayerHost& L = c->L[layer];
+  const kvc_config& g = c->cfg;
+  const int n = c->ppf, T = g.tokens_per_frame, P = g.page_size, H = g.num_heads;
+  if (L.n_entries + n > c->pool_pages) return fail(c, KVC_ERR_STATE, "kvc_append_frame: page pool full");
+  LayerStarts st{};
+  st.first_layer = layer * H;
+  for (int h = 0; h < H; ++h) st.start[h] = L.n_entries;
+  cudaError_t e = launch_mgr_alloc_layers(c->stream, c->entries, c->bitmap, c->bitmap_words, c->pool_pages, st, H, n,
+                                          frame_idx, P, T - (n - 1) * P, c->d_err);
+  if (e != cudaSuccess) return cuda_fail(c, e, "page allocation");
+  c->launches++;
+  const size_t sub0 = static_cast<size_t>(layer) * H * c->pool_pages;   // the layer's first pool page
+  uint8_t* kp = c->k_pool + sub0 * c->page_bytes_kv;
+  uint8_t* vp = c->v_pool + sub0 * c->page_bytes_kv;
+  e = launch_append_heads(c->stream, k_dev, v_dev, kp, vp, c->entries + sub0, c->tok_id + sub0 * P, c->pool_pages,
+                          L.n_entries, n, T, H, g.head_dim, P, frame_idx);
+  if (e != cudaSuccess) return cuda_fail(c, e, "append");
+  c->launches++;
+  if (!L.has_anchor) {
+    L.anchor_pages = n;
+    L.has_anchor = true;
+  } else {
+    L.pend_pages = n;
+  }
+  L.has_pending = true;
+  L.pending_key = true;
+  L.n_entries += n;
+  L.high_water = std::max<int64_t>(L.high_water, L.n_entries);
+  L.appended++;
+  L.last_frame = frame_idx;
+  return KVC_OK;
+}
+
+kvc_status div_attend(kvc_cache* c, int layer, const void* q_dev, void* o_dev) {
+  LayerHost& L = c->L[layer];
+  const kvc_config& g = c->cfg;
+  const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads;
+  const size_t sub0 = static_cast<size_t>(layer) * H * c->pool_pages;
+  cudaError_t e;
+  if (L.pend_pages > 0) {
+    const int64_t cand = L.mut_tokens + T;
+    const int keep = static_cast<int>(std::min<int64_t>(c->layer_budget[layer], cand));
+    const int n_new = (keep + P - 1) / P;
+    if (L.n_entries + n_new > c->pool_pages) return fail(c, KVC_ERR_STATE, "kvc_attend: page pool full");
+    LayerStarts st{};
+    st.first_layer = layer * H;
+    for (int h = 0; h < H; ++h) st.start[h] = L.n_entries;
+    e = launch_mgr_alloc_layers(c->stream, c->entries, c->bitmap, c->bitmap_words, c->pool_pages, st, H, n_new, -1, P,
+                                keep - (n_new - 1) * P, c->d_err);
+    if (e != cudaSuccess) return cuda_fail(c, e, "page allocation (kept tokens)");
+    c->launches++;
+    uint8_t* kp = c->k_pool + sub0 * c->page_bytes_kv;
+    uint8_t* vp = c->v_pool + sub0 * c->page_bytes_kv;
+    e = launch_diversity_prune(c->stream, c->entries + sub0, kp, vp, kp, vp, c->tok_id + sub0 * P, c->pool_pages, L.anchor_pages, L.mut_pages + L.pend_pages,
+                               L.n_entries, keep, H, g.head_dim, P, c->div_sums + static_cast<size_t>(layer) * H,
+                               c->d_err);
+    if (e != cudaSuccess) return cuda_fail(c, e, "diversity pruning");
+    c->launches++;
+    // release the previous kept pages and the frame's pages; the new kept pages follow
+    // the anchor
+    const int a = L.anchor_pages, b = L.anchor_pages + L.mut_pages + L.pend_pages;
+    e = launch_mgr_remove_layers(c->stream, c->entries, c->bitmap, c->bitmap_words, c->pool_pages, layer * H, H,
+                                 L.n_entries + n_new, a, b, c->d_err);
+    if (e != cudaSuccess) return cuda_fail(c, e, "page release");
+    c->launches++;
+    L.n_entries = L.anchor_pages + n_new;
+    L.mut_pages = n_new;
+    L.mut_tokens = keep;
+    L.pend_pages = 0;
+    L.cand_count = cand;
+    L.compressions++;
+  }
+  TcAttnArgs a{};
+  a.q = q_dev;
+  a.o = o_dev;
+  a.entries = c->entries + sub0;
+  a.n_pages = L.n_entries;
+  a.T = T;
+  a.H = H;
+  a.P = P;
+  a.page_base = static_cast<long long>(sub0);
+  a.pool_rows = static_cast<long long>(g.num_layers) * H * c->pool_pages * P;
+  a.softmax_scale = g.softmax_scale;
+  a.splits = g.kv_splits;
+  a.tmap_k = &c->tmap_k[0];
+  a.tmap_v = &c->tmap_v[0];
+  a.fp8 = false;
+  a.part_o = c->part_o;
+  a.part_lse = c->part_lse;
+  a.part_rows = c->part_rows;
+  a.sm_count = c->sm_count;
+  a.err = c->d_err;
+  a.head_pages = c->pool_pages;
+  int launched = 0;
+  e = launch_attn_tc(c->stream, a, nullptr, &launched);
+  c->launches += launched;
+  if (e != cudaSuccess) return cuda_fail(c, e, "attention launch");
+  L.has_pending = false;
+  L.committed++;
+  L.tokens = static_cast<int64_t>(T) + L.mut_tokens;
   return KVC_OK;
 }
 
@@ -323,6 +464,10 @@ kvc_status kvc_append_frame(kvc_cache* c, int32_t layer, int32_t frame_idx, cons
   LayerHost& L = c->L[layer];
   if (L.has_pending) return fail(c, KVC_ERR_STATE, "kvc_append_frame: a frame is already pending on this layer");
   if (frame_idx <= L.last_frame) return fail(c, KVC_ERR_STATE, "kvc_append_frame: frame indices must increase");
+  if (c->per_head) {
+    if (!is_keyframe) return fail(c, KVC_ERR_ARG, "kvc_append_frame: every frame is a candidate in this mode");
+    return div_append(c, layer, frame_idx, k_dev, v_dev);
+  }
   const kvc_config& g = c->cfg;
   const int n = c->ppf;
   int used = 0;
@@ -365,6 +510,17 @@ kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const void* con
   if (!c) return KVC_ERR_ARG;
   const kvc_config& g = c->cfg;
   if (!k_devs || !v_devs || frame_idx < 0) return fail(c, KVC_ERR_ARG, "kvc_append_frame_all: bad argument");
+  if (c->per_head) {
+    // one page list per head: the layers are appended one by one (checked first)
+    for (int l = 0; l < g.num_layers; ++l)
+      if (c->L[l].has_pending || frame_idx <= c->L[l].last_frame || !k_devs[l] || !v_devs[l])
+        return fail(c, KVC_ERR_STATE, "kvc_append_frame_all: a layer cannot take the frame");
+    for (int l = 0; l < g.num_layers; ++l) {
+      kvc_status st = kvc_append_frame(c, l, frame_idx, k_devs[l], v_devs[l], is_keyframe);
+      if (st != KVC_OK) return st;
+    }
+    return KVC_OK;
+  }
   const int n = c->ppf;
   for (int l = 0; l < g.num_layers; ++l) {
     if (!k_devs[l] || !v_devs[l] ||
@@ -425,6 +581,7 @@ kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_de
     return fail(c, KVC_ERR_ARG, "kvc_attend: Q and O must be 16-byte aligned");
   LayerHost& L = c->L[layer];
   if (!L.has_pending) return fail(c, KVC_ERR_STATE, "kvc_attend: no frame pending on this layer");
+  if (c->per_head) return div_attend(c, layer, q_dev, o_dev);
   const kvc_config& g = c->cfg;
   const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads, D = g.head_dim;
   Entry* E = layer_entries(c, layer);
@@ -542,6 +699,7 @@ kvc_status kvc_page_table(kvc_cache* c, int32_t layer, int32_t* rows_host, int32
 
 kvc_status kvc_token_meta(kvc_cache* c, int32_t layer, int64_t* ids_host, int32_t* counts_host, float* shat_host,
                           int32_t capacity, int32_t* n_out) {
+  if (c && c->per_head) return fail(c, KVC_ERR_STATE, "not available with per-head page lists");
   if (!c) return KVC_ERR_ARG;
   if (!valid_layer(c, layer)) return fail(c, KVC_ERR_ARG, "kvc_token_meta: bad layer");
   if (!c->tok_id) return fail(c, KVC_ERR_UNSUPPORTED, "kvc_token_meta: token metadata exists in budget mode only");
@@ -577,6 +735,7 @@ kvc_status kvc_token_meta(kvc_cache* c, int32_t layer, int64_t* ids_host, int32_
 
 kvc_status kvc_export_pages(kvc_cache* c, int32_t layer, int32_t first_row, int32_t n_rows, void* k_host,
                             void* v_host, float* k_scale_host, float* v_scale_host) {
+  if (c && c->per_head) return fail(c, KVC_ERR_STATE, "not available with per-head page lists");
   if (!c) return KVC_ERR_ARG;
   if (!valid_layer(c, layer)) return fail(c, KVC_ERR_ARG, "kvc_export_pages: bad layer");
   kvc_status st = sync_and_check(c);
@@ -645,6 +804,63 @@ kvc_status kvc_step_host(kvc_cache* c, int32_t layer, int32_t frame_idx, int32_t
   kvc_status st = kvc_step_host_async(c, layer, frame_idx, is_keyframe, q_host, k_host, v_host, o_host);
   if (st != KVC_OK) return st;
   return sync_and_check(c);
+}
+
+kvc_status kvc_set_layer_budgets(kvc_cache* c, const int32_t* budgets, int32_t n) {
+  if (!c) return KVC_ERR_ARG;
+  if (!c->per_head) return fail(c, KVC_ERR_STATE, "kvc_set_layer_budgets: not a diversity-pruned cache");
+  if (!budgets || n != c->cfg.num_layers) return fail(c, KVC_ERR_ARG, "kvc_set_layer_budgets: one budget per layer");
+  for (int l = 0; l < n; ++l)
+    if (budgets[l] < 1 || budgets[l] > c->cfg.diversity_budget)
+      return fail(c, KVC_ERR_ARG, "kvc_set_layer_budgets: budgets must lie in [1, diversity_budget]");
+  c->layer_budget.assign(budgets, budgets + n);
+  return KVC_OK;
+}
+
+kvc_status kvc_layer_diversity(kvc_cache* c, int32_t layer, double* mean_out) {
+  if (!c) return KVC_ERR_ARG;
+  if (!c->per_head) return fail(c, KVC_ERR_STATE, "kvc_layer_diversity: not a diversity-pruned cache");
+  if (!valid_layer(c, layer) || !mean_out) return fail(c, KVC_ERR_ARG, "kvc_layer_diversity: bad argument");
+  const LayerHost& L = c->L[layer];
+  if (L.cand_count == 0) return fail(c, KVC_ERR_STATE, "kvc_layer_diversity: the layer was never pruned");
+  kvc_status st = sync_and_check(c);
+  if (st != KVC_OK) return st;
+  const int H = c->cfg.num_heads;
+  std::vector<double> sums(H);
+  cudaError_t e = cudaMemcpy(sums.data(), c->div_sums + static_cast<size_t>(layer) * H, H * sizeof(double),
+                             cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(c, e, "kvc_layer_diversity copy");
+  double tot = 0.0;
+  for (int h = 0; h < H; ++h) tot += sums[h];       // heads in order
+  *mean_out = tot / static_cast<double>(static_cast<int64_t>(H) * L.cand_count);
+  return KVC_OK;
+}
+
+kvc_status kvc_head_tokens(kvc_cache* c, int32_t layer, int32_t head, int64_t* ids_out, int32_t capacity,
+                           int32_t* n_out) {
+  if (!c) return KVC_ERR_ARG;
+  if (!c->per_head) return fail(c, KVC_ERR_STATE, "kvc_head_tokens: not a diversity-pruned cache");
+  if (!valid_layer(c, layer) || head < 0 || head >= c->cfg.num_heads || !ids_out || !n_out)
+    return fail(c, KVC_ERR_ARG, "kvc_head_tokens: bad argument");
+  kvc_status st = sync_and_check(c);
+  if (st != KVC_OK) return st;
+  const int P = c->cfg.page_size;
+  const size_t sub = (static_cast<size_t>(layer) * c->cfg.num_heads + head) * c->pool_pages;
+  const int n = c->L[layer].n_entries;
+  std::vector<Entry> ent(n);
+  std::vector<int64_t> ids(static_cast<size_t>(c->pool_pages) * P);
+  cudaError_t e = n ? cudaMemcpy(ent.data(), c->entries + sub, n * sizeof(Entry), cudaMemcpyDeviceToHost) : cudaSuccess;
+  if (e == cudaSuccess)
+    e = cudaMemcpy(ids.data(), c->tok_id + sub * P, ids.size() * sizeof(int64_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(c, e, "kvc_head_tokens copy");
+  int m = 0;
+  for (int i = 0; i < n; ++i)
+    for (int s = 0; s < ent[i].w; ++s) {
+      if (m >= capacity) return fail(c, KVC_ERR_ARG, "kvc_head_tokens: capacity too small");
+      ids_out[m++] = ids[static_cast<size_t>(ent[i].x) * P + s];
+    }
+  *n_out = m;
+  return KVC_OK;
 }
 
 kvc_status kvc_synchronize(kvc_cache* c) {

@@ -23,6 +23,7 @@ struct TcParams {
   float* part_o;
   float* part_lse;
   int* err;
+  int head_pages;               // > 0: per-head page lists (see TcAttnArgs)
 };
 
 __device__ __forceinline__ float ex2(float x) {

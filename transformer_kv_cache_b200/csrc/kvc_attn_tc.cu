@@ -94,6 +94,10 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
   const int tile0 = split * p.tiles_per_split;
   const int tile1 = min(tile0 + p.tiles_per_split, p.total_tiles);
   const int n_tiles = tile1 - tile0;
+  // page list and pool rows of this head: shared pages [page][head][slot] or, with
+  // per-head page lists, single-head pages of head h's pool region
+  const long long hp = p.head_pages ? static_cast<long long>(h) * p.head_pages : 0;
+  const Entry* ent = p.entries + hp;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 4);                       // the four softmax warps stored Q in TMEM
@@ -144,8 +148,9 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           for (int g = 0; g < kPPT; ++g) {
             const int idx = gt * kPPT + g;
             // pages past the list end are read past the end of the pool: TMA fills zeros
-            row[g] = idx < p.n_pages ? static_cast<int>(((p.page_base + __ldg(&p.entries[idx].x)) * p.H + h) * P)
-                                     : p.pool_rows;
+            row[g] = idx >= p.n_pages ? p.pool_rows
+                     : p.head_pages    ? static_cast<int>((p.page_base + hp + __ldg(&ent[idx].x)) * P)
+                                       : static_cast<int>(((p.page_base + __ldg(&ent[idx].x)) * p.H + h) * P);
           }
           mbar_arrive_expect_tx(&k_full[st], kTileBytes);
 #pragma unroll
@@ -265,7 +270,7 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
 #pragma unroll
       for (int g = 0; g < kPPT; ++g) {
         const int idx = tile0 * kPPT + g;
-        vnext[g] = idx < p.n_pages ? __ldg(&p.entries[idx].w) : 0;
+        vnext[g] = idx < p.n_pages ? __ldg(&ent[idx].w) : 0;
       }
       // S of the current tile lives in registers; the next tile's S is loaded while this
       // tile's P store is in flight
@@ -288,7 +293,7 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
 #pragma unroll
           for (int g = 0; g < kPPT; ++g) {
             const int idx = (tile0 + j + 1) * kPPT + g;
-            vnext[g] = idx < p.n_pages ? __ldg(&p.entries[idx].w) : 0;
+            vnext[g] = idx < p.n_pages ? __ldg(&ent[idx].w) : 0;
           }
         }
         // P = 2^(s*c - m): exponent pairs with one packed FMA, two MUFU ex2, one bf16 pack;
@@ -531,7 +536,7 @@ int choose_splits(int units, int tiles, int slots) {
 
 cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used, int* launched) {
   if (launched) *launched = 0;
-  if (a.P != 16) return cudaErrorInvalidValue;
+  if (a.P != 16 || (a.fp8 && a.head_pages)) return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!a.fp8 && !attr_set) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -578,6 +583,7 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   prm.part_o = a.part_o;
   prm.part_lse = a.part_lse;
   prm.err = a.err;
+  prm.head_pages = a.head_pages;
   const int grid = units * splits;
   cudaError_t e;
   if (a.fp8) {

@@ -35,6 +35,13 @@ struct LayerHost {
   int64_t protected_tokens = 0;   // committed protected tokens (compression)
   int32_t last_merge_n = 0;
   int32_t scored_frame = -1;      // frame whose residual was last scored on this layer
+  // rolling diversity-pruned memory (one page list per head, all heads the same shape)
+  int32_t anchor_pages = 0;       // pages of the first frame (immutable)
+  int32_t mut_pages = 0;          // pages of the kept tokens (ascending id)
+  int32_t pend_pages = 0;         // pages of the frame appended and not yet pruned
+  int64_t mut_tokens = 0;
+  int64_t cand_count = 0;         // candidates of the last pruning (per head)
+  bool has_anchor = false;
 };
 
 // Device page-table entry: x = physical page, y = owner frame (-1: compaction block),
@@ -93,6 +100,11 @@ struct Cache {
   int32_t hist_next_layer = 0;
   std::vector<int> hist_layers;     // layers scored so far in the current frame
   int64_t launches = 0;             // kernels launched by this cache
+  // rolling diversity-pruned memory: sub-layer (layer, head) = index layer * H + head owns
+  // its own page list, bitmap and pool region of pool_pages single-head pages
+  bool per_head = false;
+  std::vector<int32_t> layer_budget;
+  double* div_sums = nullptr;       // [layers][H] fp64 score sums of the last pruning
 };
 
 }  // namespace kvc
@@ -166,6 +178,9 @@ struct TcAttnArgs {
   size_t part_rows;
   int sm_count;
   int* err;
+  int head_pages;                   // > 0: one page list per head, head h's pages at
+                                    // entries + h * head_pages, pool page index page_base +
+                                    // h * head_pages + phys (single-head pages)
 };
 // Returns the number of kernels launched through *launched.
 cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used, int* launched);
@@ -180,6 +195,19 @@ cudaError_t launch_merge_targets(cudaStream_t s, const __nv_bfloat16* ks, const 
                                  const double* ns, const double* ne, const float* inv_ns, const float* inv_ne,
                                  int n_src, int n_elig, int HD, float* top_v, int32_t* top_j, int tiles_n,
                                  int32_t* target, int* err, int* launched);
+
+// Rolling diversity-pruned memory (kvc_diversity.cu).
+cudaError_t launch_append_heads(cudaStream_t s, const void* k, const void* v, void* k_pool, void* v_pool,
+                                const Entry* entries_layer, int64_t* tok_id_layer, int pool_pages, int start,
+                                int n_pages, int T, int H, int D, int P, int frame);
+cudaError_t launch_diversity_prune(cudaStream_t s, Entry* entries_layer, const void* k_pool, const void* v_pool,
+                                   void* k_pool_w, void* v_pool_w, int64_t* tok_id_layer, int pool_pages,
+                                   int first_cand_entry, int n_cand_entries, int new_entry, int keep, int H, int D,
+                                   int P, double* sums_layer, int* err);
+cudaError_t launch_mgr_remove_layers(cudaStream_t s, Entry* entries_all, uint32_t* bitmap_all, int words,
+                                     int pool_pages, int first_layer, int n_layers, int n_entries, int a, int b,
+                                     int* err);
+size_t diversity_prune_smem(int n_cand);
 
 // Compression kernels.
 cudaError_t launch_score(cudaStream_t s, const float* residual, int T, int R, int layer_slot, int n_hist,
