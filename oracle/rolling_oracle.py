@@ -20,9 +20,11 @@ recipe, with its concrete mini-example):
 
 Readings taken where the page is silent (each is also listed in the design notes):
 the fp64 evaluation order below (squares summed over dims in ascending order for each
-norm; the normalised keys summed over candidates in ascending token id for the mean,
-whose direction equals that of the sum; dot products summed over dims in ascending
-order); a zero key has no direction and scores 0; ties are broken by the lower token
+norm; dot products summed over dims in ascending order; every sum over candidates -- the
+normalised keys for the mean, whose direction equals that of the sum, and the scores for
+a head's total -- taken in blocks of 32 consecutive candidates in ascending token id,
+ascending within a block, then the block sums in ascending block order); a zero key has
+no direction and scores 0; ties are broken by the lower token
 id; the kept tokens are stored in ascending id; pruning starts with the second frame;
 the budget of layer l is floor(L * K * softmax(mean diversity / tau)_l), computed from
 the previous frame's layer averages by the caller (the page gives neither the
@@ -40,11 +42,27 @@ from typing import List, Optional, Sequence
 import numpy as np
 
 
+CAND_BLOCK = 32          # candidates per block of every sum over candidates
+
+
+def blocked_sum(x: np.ndarray) -> np.ndarray:
+    """Sum over axis 0 in blocks of CAND_BLOCK rows: ascending within each block, then the
+    block sums ascending. Every addition is one IEEE fp64 operation."""
+    x = np.asarray(x, np.float64)
+    total = np.zeros(x.shape[1:])
+    for b0 in range(0, x.shape[0], CAND_BLOCK):
+        part = np.zeros(x.shape[1:])
+        for i in range(b0, min(b0 + CAND_BLOCK, x.shape[0])):
+            part = part + x[i]
+        total = total + part
+    return total
+
+
 def diversity_scores(Kc: np.ndarray) -> np.ndarray:
     """Scores of one (layer, head)'s candidates. Kc: [N, D] keys in ascending token id.
 
     k_hat_i = k_i / |k_i| (|k_i| = sqrt of the ascending-d fp64 sum of squares; a zero
-    key gives k_hat = 0); mu = sum_i k_hat_i in ascending i; score_i = -(k_hat_i . mu) /
+    key gives k_hat = 0); mu = the blocked sum of the k_hat_i; score_i = -(k_hat_i . mu) /
     |mu| (dot and |mu| summed over ascending d). Every step is one IEEE fp64 operation.
     """
     Kc = np.asarray(Kc, np.float64)
@@ -56,9 +74,7 @@ def diversity_scores(Kc: np.ndarray) -> np.ndarray:
     khat = np.zeros_like(Kc)
     nz = norms > 0
     khat[nz] = Kc[nz] / norms[nz, None]
-    mu = np.zeros(D)
-    for i in range(N):                          # sequential over candidates, ascending id
-        mu = mu + khat[i]
+    mu = blocked_sum(khat) if N else np.zeros(D)
     m2 = 0.0
     for d in range(D):
         m2 = m2 + mu[d] * mu[d]
@@ -140,10 +156,7 @@ class RollingOracle:
             Kc = np.concatenate([self.mut_k[layer][h], K[:, h, :]])
             Vc = np.concatenate([self.mut_v[layer][h], V[:, h, :]])
             sc = diversity_scores(Kc)
-            s = 0.0
-            for x in sc:                          # ascending id
-                s = s + float(x)
-            sums.append(s)
+            sums.append(float(blocked_sum(sc[:, None])[0]))
             keep = top_k(sc, ids, self.budgets[layer])
             self.mut_ids[layer][h] = ids[keep]
             self.mut_k[layer][h] = Kc[keep]

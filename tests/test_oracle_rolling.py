@@ -151,3 +151,42 @@ def test_planted_sign_mistake_is_caught(monkeypatch):
     Kc[:n, 0] = 1.0
     Kc[n, 3] = 1.0
     assert np.argmax(ro.diversity_scores(Kc)) != n
+
+
+def test_blocked_sum_order_hand_derived():
+    # 2^53 then 63 ones. Sequential: every +1 is a tie at 2^53 that rounds to even, so the
+    # ones vanish (2^53). Blocked: block 0 (2^53 and 31 ones) gives 2^53, block 1 (32 ones)
+    # gives 32 exactly, and 2^53 + 32 is representable.
+    x = np.array([2.0 ** 53] + [1.0] * 63)
+    assert ro.blocked_sum(x[:, None])[0] == 2.0 ** 53 + 32.0
+    seq = 0.0
+    for v in x:
+        seq += v
+    assert seq == 2.0 ** 53                      # the orders really differ here
+
+
+def test_blocked_sum_close_to_exact_sum():
+    import math
+    rng = np.random.default_rng(9)
+    for n in (1, 31, 32, 33, 1516):
+        x = rng.standard_normal((n, 3))
+        got = ro.blocked_sum(x)
+        for d in range(3):
+            exact = math.fsum(x[:, d])
+            assert abs(got[d] - exact) <= n * 2.0 ** -52 * np.sum(np.abs(x[:, d]))
+
+
+def test_layer_diversity_is_mean_of_scores():
+    rng = np.random.default_rng(10)
+    L, H, D, T, K = 1, 3, 16, 40, 50
+    orc = RollingOracle(L, H, D, T, K, 0.25)
+    for t in range(3):
+        K_ = rng.standard_normal((T, H, D))
+        orc.append(0, t, K_, K_)
+        if t == 0:
+            continue
+        cands = [(orc.mut_k[0][h], K_[:, h, :]) for h in range(H)]
+        orc.prune(0)
+        ref = [_scores_by_scipy(np.concatenate(c)) for c in cands]
+        mean = np.mean(np.concatenate(ref))
+        assert abs(orc.layer_diversity(0) - mean) < 1e-13
