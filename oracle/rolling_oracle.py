@@ -20,6 +20,7 @@ recipe, with its concrete mini-example):
 
 Readings taken where the page is silent (each is also listed in the design notes):
 the fp64 evaluation order below (squares summed over dims in ascending order for each
+norm; a key is normalised by multiplying it with the correctly rounded reciprocal of its
 norm; dot products summed over dims in ascending order; every sum over candidates -- the
 normalised keys for the mean, whose direction equals that of the sum, and the scores for
 a head's total -- taken in blocks of 32 consecutive candidates in ascending token id,
@@ -58,22 +59,32 @@ def blocked_sum(x: np.ndarray) -> np.ndarray:
     return total
 
 
-def diversity_scores(Kc: np.ndarray) -> np.ndarray:
-    """Scores of one (layer, head)'s candidates. Kc: [N, D] keys in ascending token id.
-
-    k_hat_i = k_i / |k_i| (|k_i| = sqrt of the ascending-d fp64 sum of squares; a zero
-    key gives k_hat = 0); mu = the blocked sum of the k_hat_i; score_i = -(k_hat_i . mu) /
-    |mu| (dot and |mu| summed over ascending d). Every step is one IEEE fp64 operation.
-    """
+def normalised_keys(Kc: np.ndarray) -> np.ndarray:
+    """k_hat_i = k_i * RN(1 / |k_i|), |k_i| = sqrt of the squares summed over ascending d;
+    a zero key gives k_hat = 0."""
     Kc = np.asarray(Kc, np.float64)
     N, D = Kc.shape
     sq = np.zeros(N)
     for d in range(D):                          # sequential over d for every candidate
         sq = sq + Kc[:, d] * Kc[:, d]
     norms = np.sqrt(sq)
-    khat = np.zeros_like(Kc)
+    rcp = np.zeros(N)
     nz = norms > 0
-    khat[nz] = Kc[nz] / norms[nz, None]
+    rcp[nz] = 1.0 / norms[nz]
+    return Kc * rcp[:, None]
+
+
+def diversity_scores(Kc: np.ndarray) -> np.ndarray:
+    """Scores of one (layer, head)'s candidates. Kc: [N, D] keys in ascending token id.
+
+    k_hat_i = k_i * (1 / |k_i|) (|k_i| = sqrt of the ascending-d fp64 sum of squares, its
+    reciprocal rounded once; a zero key gives k_hat = 0); mu = the blocked sum of the
+    k_hat_i; score_i = -(k_hat_i . mu) / |mu| (dot and |mu| summed over ascending d).
+    Every step is one IEEE fp64 operation.
+    """
+    Kc = np.asarray(Kc, np.float64)
+    N, D = Kc.shape
+    khat = normalised_keys(Kc)
     mu = blocked_sum(khat) if N else np.zeros(D)
     m2 = 0.0
     for d in range(D):

@@ -190,3 +190,13 @@ def test_layer_diversity_is_mean_of_scores():
         ref = [_scores_by_scipy(np.concatenate(c)) for c in cands]
         mean = np.mean(np.concatenate(ref))
         assert abs(orc.layer_diversity(0) - mean) < 1e-13
+
+
+def test_normalisation_by_rounded_reciprocal_hand_derived():
+    # |(3, 4)| = 5; RN(1/5) = 3602879701896397 / 2^54. Times 3 the exact product is
+    # 10808639105689191 / 2^54 = 5404319552844595.5 / 2^53, a tie that rounds to the even
+    # 5404319552844596 / 2^53: one ulp above RN(3/5). Times 4 it is exact: RN(4/5).
+    kh = ro.normalised_keys(np.array([[3.0, 4.0]]))
+    assert kh[0, 0] == 5404319552844596 / 2.0 ** 53 and kh[0, 0] != 3.0 / 5.0
+    assert kh[0, 1] == 7205759403792794 / 2.0 ** 53 == 4.0 / 5.0
+    assert np.array_equal(ro.normalised_keys(np.zeros((1, 4))), np.zeros((1, 4)))
