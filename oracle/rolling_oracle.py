@@ -19,9 +19,10 @@ recipe, with its concrete mini-example):
   tokens.
 
 Readings taken where the page is silent (each is also listed in the design notes):
-the fp64 evaluation order below (squares summed over dims in ascending order for each
-norm; a key is normalised by multiplying it with the correctly rounded reciprocal of its
-norm; dot products summed over dims in ascending order; every sum over candidates -- the
+the fp64 evaluation order below (every sum over the dims -- the squares of a norm, the
+terms of a dot product -- taken in blocks of 8 consecutive dims, ascending within a block,
+then the block sums in ascending order; a key is normalised by multiplying it with the
+correctly rounded reciprocal of its norm; every sum over candidates -- the
 normalised keys for the mean, whose direction equals that of the sum, and the scores for
 a head's total -- taken in blocks of 32 consecutive candidates in ascending token id,
 ascending within a block, then the block sums in ascending block order); a zero key has
@@ -44,6 +45,21 @@ import numpy as np
 
 
 CAND_BLOCK = 32          # candidates per block of every sum over candidates
+DIM_BLOCK = 8            # dims per block of every sum over the dims
+
+
+def dim_sum(terms: np.ndarray) -> np.ndarray:
+    """Sum over the last axis in blocks of DIM_BLOCK entries: ascending within each block,
+    then the block sums ascending. Every addition is one IEEE fp64 operation."""
+    terms = np.asarray(terms, np.float64)
+    D = terms.shape[-1]
+    total = np.zeros(terms.shape[:-1])
+    for d0 in range(0, D, DIM_BLOCK):
+        part = np.zeros(terms.shape[:-1])
+        for d in range(d0, min(d0 + DIM_BLOCK, D)):
+            part = part + terms[..., d]
+        total = total + part
+    return total
 
 
 def blocked_sum(x: np.ndarray) -> np.ndarray:
@@ -60,14 +76,11 @@ def blocked_sum(x: np.ndarray) -> np.ndarray:
 
 
 def normalised_keys(Kc: np.ndarray) -> np.ndarray:
-    """k_hat_i = k_i * RN(1 / |k_i|), |k_i| = sqrt of the squares summed over ascending d;
-    a zero key gives k_hat = 0."""
+    """k_hat_i = k_i * RN(1 / |k_i|), |k_i| = sqrt of the dim_sum of the squares; a zero
+    key gives k_hat = 0."""
     Kc = np.asarray(Kc, np.float64)
-    N, D = Kc.shape
-    sq = np.zeros(N)
-    for d in range(D):                          # sequential over d for every candidate
-        sq = sq + Kc[:, d] * Kc[:, d]
-    norms = np.sqrt(sq)
+    N = Kc.shape[0]
+    norms = np.sqrt(dim_sum(Kc * Kc))
     rcp = np.zeros(N)
     nz = norms > 0
     rcp[nz] = 1.0 / norms[nz]
@@ -77,24 +90,19 @@ def normalised_keys(Kc: np.ndarray) -> np.ndarray:
 def diversity_scores(Kc: np.ndarray) -> np.ndarray:
     """Scores of one (layer, head)'s candidates. Kc: [N, D] keys in ascending token id.
 
-    k_hat_i = k_i * (1 / |k_i|) (|k_i| = sqrt of the ascending-d fp64 sum of squares, its
+    k_hat_i = k_i * (1 / |k_i|) (|k_i| = sqrt of the dim_sum of the squares, its
     reciprocal rounded once; a zero key gives k_hat = 0); mu = the blocked sum of the
-    k_hat_i; score_i = -(k_hat_i . mu) / |mu| (dot and |mu| summed over ascending d).
+    k_hat_i; score_i = -(k_hat_i . mu) / |mu| (dot and |mu|^2 as dim_sums of the products).
     Every step is one IEEE fp64 operation.
     """
     Kc = np.asarray(Kc, np.float64)
     N, D = Kc.shape
     khat = normalised_keys(Kc)
     mu = blocked_sum(khat) if N else np.zeros(D)
-    m2 = 0.0
-    for d in range(D):
-        m2 = m2 + mu[d] * mu[d]
-    mnorm = math.sqrt(m2)
+    mnorm = math.sqrt(float(dim_sum(mu * mu)))
     if mnorm == 0.0:
         return np.zeros(N)
-    dot = np.zeros(N)
-    for d in range(D):
-        dot = dot + khat[:, d] * mu[d]
+    dot = dim_sum(khat * mu[None, :])
     return -(dot / mnorm)
 
 

@@ -200,3 +200,11 @@ def test_normalisation_by_rounded_reciprocal_hand_derived():
     assert kh[0, 0] == 5404319552844596 / 2.0 ** 53 and kh[0, 0] != 3.0 / 5.0
     assert kh[0, 1] == 7205759403792794 / 2.0 ** 53 == 4.0 / 5.0
     assert np.array_equal(ro.normalised_keys(np.zeros((1, 4))), np.zeros((1, 4)))
+
+
+def test_dim_sum_order_hand_derived():
+    # 16 dims: 2^53, then 15 ones. Block 0 (2^53 and 7 ones): every +1 is a tie at 2^53
+    # that rounds to even, 2^53. Block 1 (8 ones): 8 exactly. Total 2^53 + 8, representable.
+    x = np.array([[2.0 ** 53] + [1.0] * 15])
+    assert ro.dim_sum(x)[0] == 2.0 ** 53 + 8.0
+    np.testing.assert_array_equal(ro.dim_sum(np.arange(64.0)[None, :]), [2016.0])   # exact integers
