@@ -56,7 +56,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kv-splits", type=int, default=0)
     ap.add_argument("--workload", default=WORKLOAD,
-                    help="vggt_518x378 (default, the headline), vggt_24layer_k4, vggt_budget_16k, vggt_518x518_fp8")
+                    help="vggt_518x378 (default, the headline), vggt_24layer_k4, vggt_budget_16k, vggt_518x518_fp8, "
+                         "vggt_infinite_12l")
     ap.add_argument("--fill", type=int, default=0,
                     help="frames streamed before warm-up for a non-default workload (0: enough to fill the window); "
                          "smaller values give short cases for profiling")
@@ -410,8 +411,9 @@ def run_ours(args):
 def run_workload(args):
     """One JSON line for a non-default workload: a step is one frame through every layer
     (batched append of all layers, attention per layer, and scoring/compression per layer in
-    budget mode). Inputs cycle through a few seeded frames per layer (data values do not
-    change the work) so that all K steps' inputs are resident in HBM."""
+    budget mode, or pruning per layer with the rolling memory). All K steps' inputs are
+    resident in HBM: a few seeded frames per layer cycle, except with the rolling memory,
+    whose pruning depends on the key values and so gets a distinct frame every step."""
     import torch
     import transformer_kv_cache_b200 as kvc
     from kvc_streams import WORKLOADS, FrameStream, keyframe_schedule
@@ -425,14 +427,20 @@ def run_workload(args):
     L, T, H, D, P = wl.num_layers, wl.tokens_per_frame, wl.num_heads, wl.head_dim, wl.page_size
     S, W, k = wl.scale_frames, wl.window_frames, wl.keyframe_interval
     budget = wl.budget_tokens > 0
+    rolling = wl.diversity_budget > 0
     if args.fill > 0:
         fill = args.fill
+    elif rolling:
+        fill = 3                                      # anchor, then two prunings: the kept sets are full
     elif budget:
         fill = -(-wl.budget_tokens // T) + 3          # past the first compression of every layer
     else:
         fill = S + W * k                              # the window is full of keyframes
-    distinct = 4
     warm, steps = args.warmup, args.steps
+    # the rolling memory's pruning depends on the key values: every frame distinct, as in a
+    # video (a repeated frame would duplicate every key of the kept set); elsewhere data
+    # values do not change the work and a few frames cycle
+    distinct = fill + warm + steps if rolling else 4
     log(f"{wl.name}: {L} layers, fill {fill} frames, {distinct} distinct input frames per layer")
     with torch.cuda.stream(stream):
         st = FrameStream(wl, seed=2000, device=dev)
@@ -442,15 +450,25 @@ def run_workload(args):
         h = kvc.kvc_create(kvc.config_from_workload(wl, kv_splits=args.kv_splits), stream)
 
         def step(t, ev=None):
-            key = keyframe_schedule(t, S, k)
+            key = True if rolling else keyframe_schedule(t, S, k)
             i = t % distinct
             if ev: ev[0].record(stream)
             kvc.kvc_append_frame_all(h, t, [pool[l][i][1] for l in range(L)], [pool[l][i][2] for l in range(L)], key)
             if ev: ev[1].record(stream)
+            fired = 0
+            if rolling:                               # prune every layer, then attend every layer
+                if t > 0:
+                    for l in range(L):
+                        kvc.kvc_prune(h, l)
+                    fired = L
+                if ev: ev[2].record(stream)
+                for l in range(L):
+                    kvc.kvc_attend(h, l, pool[l][i][0], out)
+                if ev: ev[3].record(stream)
+                return key, fired
             for l in range(L):
                 kvc.kvc_attend(h, l, pool[l][i][0], out)
             if ev: ev[2].record(stream)
-            fired = 0
             if budget:
                 for l in range(L):
                     fired += kvc.kvc_compress(h, l, res[l][i])
@@ -479,13 +497,17 @@ def run_workload(args):
     app = [evs[i][0].elapsed_time(evs[i][1]) for i in range(steps)]
     att = [evs[i][1].elapsed_time(evs[i][2]) for i in range(steps)]
     cmp_ = [evs[i][2].elapsed_time(evs[i][3]) for i in range(steps)]
+    if rolling:                                       # the prune comes before the attention
+        att, cmp_ = cmp_, att
     ms = statistics.mean(tot)
     line = {"metric": METRIC, "value": 1e3 / ms, "unit": UNIT, "n_gpus": 1, "steps": steps, "warmup": warm,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp8_e4m3 storage, bf16 I/O" if wl.kv_dtype == "fp8_e4m3" else "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "layers": L, "tokens_per_frame": T, "heads": H, "head_dim": D,
                        "page_size": P, "window_frames": W, "scale_frames": S, "keyframe_interval": k,
-                       "budget_tokens": wl.budget_tokens, "inputs": f"{distinct} seeded frames per layer, cycled",
+                       "budget_tokens": wl.budget_tokens, "diversity_budget": wl.diversity_budget,
+                       "inputs": (f"{distinct} distinct seeded frames per layer" if rolling else
+                                  f"{distinct} seeded frames per layer, cycled"),
                        "keyframes_timed": keys, "compressions_timed": fires},
             "clocks": clk.summary()}
     # per layer: read K and V in bf16, write them as stored (bf16, or E4M3 codes + scales)
@@ -497,8 +519,11 @@ def run_workload(args):
                               "achieved_gbs": app_bytes / (statistics.mean(app) * 1e-3) / 1e9,
                               "peak_gbs": float(peaks["hbm_gbs"])},
         "attention_all_layers": {"avg_ms": att_ms}}
+    if rolling:
+        kv_tokens = T + min(wl.diversity_budget, 2 * T)   # per head: the anchor and the kept tokens
     if not budget:
-        kv_tokens = info0["tokens"] + T               # the cache before the timed steps, plus the new frame
+        if not rolling:
+            kv_tokens = info0["tokens"] + T           # the cache before the timed steps, plus the new frame
         flops = 4.0 * T * kv_tokens * H * D * L
         ach = flops / (att_ms * 1e-3) / 1e12
         line["roofline"] = {"bound": "tensor", "achieved": ach, "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
@@ -507,6 +532,15 @@ def run_workload(args):
     if budget:
         line["kernels"]["score_and_compress_all_layers"] = {"avg_ms": statistics.mean(cmp_),
                                                             "max_ms": max(cmp_)}
+    if rolling:
+        # per layer and head: read the candidates' keys, move the kept tokens' K and V
+        n_cand = min(wl.diversity_budget, 2 * T) + T
+        prune_bytes = H * L * (n_cand * D * 2 + 4 * min(wl.diversity_budget, n_cand) * D * 2)
+        pm = statistics.mean(cmp_)
+        line["kernels"]["prune_all_layers"] = {"bound": "hbm", "avg_ms": pm, "max_ms": max(cmp_),
+                                               "bytes_per_step": prune_bytes,
+                                               "achieved_gbs": prune_bytes / (pm * 1e-3) / 1e9,
+                                               "candidates_per_head": n_cand}
     line["kernels"]["append_all_layers"]["frac"] = (line["kernels"]["append_all_layers"]["achieved_gbs"] /
                                                     float(peaks["hbm_gbs"]))
     print(json.dumps(line), flush=True)

@@ -241,7 +241,9 @@ KVC_API kvc_status kvc_step_host_async(kvc_cache* c, int32_t layer, int32_t fram
 
 /* ---- Rolling diversity-pruned memory (diversity_budget = K > 0; [IVG] Building Blocks,
  * Step-by-step recipe). Requires bf16 I/O and storage, head_dim 64, page_size 16, no
- * window and no token budget. Every head keeps its own tokens: the first frame appended
+ * window, no token budget, and at most 2,048 candidate slots per head:
+ * (ceil(K / 16) + ceil(T / 16)) * 16 <= 2048 (T = tokens_per_frame; kvc_create returns
+ * KVC_ERR_ARG otherwise). Every head keeps its own tokens: the first frame appended
  * to a layer is its immutable anchor (all heads); each later frame joins the candidates,
  * and kvc_attend first prunes each head to its Top-K candidates by diversity score
  * (negative cosine of the L2-normalised key to the mean normalised candidate key; ties to
@@ -254,6 +256,13 @@ KVC_API kvc_status kvc_step_host_async(kvc_cache* c, int32_t layer, int32_t fram
  * budgets: host array of num_layers values. Errors: KVC_ERR_ARG, KVC_ERR_STATE (not in
  * this mode). */
 KVC_API kvc_status kvc_set_layer_budgets(kvc_cache* c, const int32_t* budgets, int32_t n);
+
+/* The pruning step alone ([IVG] Step-by-step recipe: prune, then attend): scores every
+ * head's candidates (kept tokens + the pending frame) and keeps each head's Top-K; the
+ * pending frame stays pending for kvc_attend, which then only attends. Enqueued on the
+ * cache's stream. Errors: KVC_ERR_ARG (bad layer), KVC_ERR_STATE (not in this mode, or
+ * no frame pending); calling it twice prunes once. */
+KVC_API kvc_status kvc_prune(kvc_cache* c, int32_t layer);
 
 /* Mean diversity score of the layer's last pruning over all heads' candidates (fp64:
  * per head the scores summed in ascending token id, then the heads in order, divided by

@@ -20,7 +20,7 @@ def kvc():
     return m
 
 
-def run_rolling(kvc, wl, frames, rows=None, budgets_at=None, check_ids=True, seed=11):
+def run_rolling(kvc, wl, frames, rows=None, budgets_at=None, check_ids=True, seed=11, prune_first=False):
     dev = torch.device("cuda")
     L, H, D, T = wl.num_layers, wl.num_heads, wl.head_dim, wl.tokens_per_frame
     h = kvc.kvc_create(kvc.config_from_workload(wl))
@@ -35,6 +35,9 @@ def run_rolling(kvc, wl, frames, rows=None, budgets_at=None, check_ids=True, see
             for l in range(L):
                 q, k, v = st.frame(l, t)
                 kvc.kvc_append_frame(h, l, t, k, v, True)
+                if prune_first and t > 0:
+                    kvc.kvc_prune(h, l)                 # the pruning step on its own; twice prunes once
+                    kvc.kvc_prune(h, l)
                 kvc.kvc_attend(h, l, q, o)
                 orc.append(l, t, np64(k), np64(v))
                 ref = orc.attend(l, np64(q), rows=rows)
@@ -54,16 +57,16 @@ def run_rolling(kvc, wl, frames, rows=None, budgets_at=None, check_ids=True, see
         kvc.kvc_destroy(h)
 
 
-@pytest.mark.parametrize("T,H,K,frames", [
-    (150, 4, 200, 7),    # candidates 350 -> 200 kept per head from the second pruning on
-    (150, 4, 100, 5),    # K not a multiple of the page size
-    (40, 2, 400, 6),     # K above the candidates for several frames: nothing pruned yet
-    (10, 2, 25, 6),      # T < P: every page partial
+@pytest.mark.parametrize("T,H,K,frames,prune_first", [
+    (150, 4, 200, 7, False),    # candidates 350 -> 200 kept per head from the second pruning on
+    (150, 4, 100, 5, True),     # K not a multiple of the page size; kvc_prune before kvc_attend
+    (40, 2, 400, 6, False),     # K above the candidates for several frames: nothing pruned yet
+    (10, 2, 25, 6, True),       # T < P: every page partial
 ])
-def test_rolling_memory_small(kvc, T, H, K, frames):
+def test_rolling_memory_small(kvc, T, H, K, frames, prune_first):
     wl = WORKLOADS["vggt_infinite_12l"].replace(num_layers=2, tokens_per_frame=T, num_heads=H, diversity_budget=K,
                                                 num_special_tokens=min(5, T))
-    run_rolling(kvc, wl, frames)
+    run_rolling(kvc, wl, frames, prune_first=prune_first)
 
 
 def test_layer_budgets_between_frames(kvc):
@@ -84,6 +87,13 @@ def test_rolling_memory_full_size_sampled(kvc):
     run_rolling(kvc, wl, 4, rows=sample_rows(wl.tokens_per_frame, 48, seed=4))
 
 
+def test_rolling_memory_largest_candidate_set(kvc):
+    """K = 1,040 with 1,004-token frames: 65 + 63 pages, the 2,048 candidate slots a head
+    can hold (256 per CTA of the pruning cluster), sampled query rows."""
+    wl = WORKLOADS["vggt_infinite_12l"].replace(num_layers=1, num_heads=4, diversity_budget=1040)
+    run_rolling(kvc, wl, 4, rows=sample_rows(wl.tokens_per_frame, 32, seed=5))
+
+
 def test_rolling_memory_errors(kvc):
     wl = WORKLOADS["vggt_infinite_12l"].replace(num_layers=2, tokens_per_frame=64, num_heads=2,
                                                 diversity_budget=64)
@@ -98,8 +108,22 @@ def test_rolling_memory_errors(kvc):
             kvc.kvc_layer_diversity(h, 0)                       # never pruned
         with pytest.raises(kvc.KVCError):
             kvc.kvc_token_meta(h, 0)                            # not in this mode
+        with pytest.raises(kvc.KVCError):
+            kvc.kvc_prune(h, 0)                                 # no frame pending
+        with pytest.raises(kvc.KVCError):
+            kvc.kvc_prune(h, 2)                                 # no such layer
     finally:
         kvc.kvc_destroy(h)
-    bad = wl.replace(kv_dtype="fp8_e4m3")
-    with pytest.raises(kvc.KVCError):
-        kvc.kvc_create(kvc.config_from_workload(bad))
+    plain = WORKLOADS["vggt_518x378"].replace(num_layers=1)
+    h = kvc.kvc_create(kvc.config_from_workload(plain))
+    try:
+        with pytest.raises(kvc.KVCError):
+            kvc.kvc_prune(h, 0)                                 # not a diversity-pruned cache
+    finally:
+        kvc.kvc_destroy(h)
+    for bad in (wl.replace(kv_dtype="fp8_e4m3"),
+                WORKLOADS["vggt_infinite_12l"].replace(diversity_budget=1040 + 16)):   # 2,064 candidate slots
+        with pytest.raises(kvc.KVCError):
+            kvc.kvc_create(kvc.config_from_workload(bad))
+    ok = WORKLOADS["vggt_infinite_12l"].replace(num_layers=1, diversity_budget=1040)  # 2,048: the largest
+    kvc.kvc_destroy(kvc.kvc_create(kvc.config_from_workload(ok)))

@@ -28,7 +28,8 @@ EXPORTS = ["kvc_create", "kvc_destroy", "kvc_set_stream", "kvc_reset", "kvc_appe
            "kvc_compress", "kvc_page_table", "kvc_token_meta", "kvc_last_merge", "kvc_export_pages",
            "kvc_step_host", "kvc_synchronize", "kvc_last_error", "kvc_status_string", "kvc_version",
            "kvc_debug_fail_allocs", "kvc_debug_bounded_wait", "kvc_attend_paged_noalloc", "kvc_append_frame_all",
-           "kvc_step_host_async", "kvc_set_layer_budgets", "kvc_layer_diversity", "kvc_head_tokens"]
+           "kvc_step_host_async", "kvc_set_layer_budgets", "kvc_prune", "kvc_layer_diversity",
+           "kvc_head_tokens"]
 
 
 class kvc_config(ctypes.Structure):
@@ -82,6 +83,7 @@ def _load():
         "kvc_step_host": ([vp, i32, i32, i32, vp, vp, vp, vp], i32),
         "kvc_step_host_async": ([vp, i32, i32, i32, vp, vp, vp, vp], i32),
         "kvc_set_layer_budgets": ([vp, vp, i32], i32),
+        "kvc_prune": ([vp, i32], i32),
         "kvc_layer_diversity": ([vp, i32, vp], i32),
         "kvc_head_tokens": ([vp, i32, i32, vp, i32, vp], i32),
         "kvc_synchronize": ([vp], i32),
@@ -270,6 +272,11 @@ def kvc_step_host_async(handle, layer: int, frame_idx: int, is_keyframe: bool, q
 def kvc_set_layer_budgets(handle, budgets) -> None:
     arr = (ctypes.c_int32 * len(budgets))(*[int(b) for b in budgets])
     _check(handle, _lib.kvc_set_layer_budgets(handle, arr, len(budgets)))
+
+
+def kvc_prune(handle, layer: int) -> None:
+    """Prune every head of `layer` to its Top-K candidates (the step before kvc_attend)."""
+    _check(handle, _lib.kvc_prune(handle, layer))
 
 
 def kvc_layer_diversity(handle, layer: int) -> float:

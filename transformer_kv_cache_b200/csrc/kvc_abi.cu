@@ -177,7 +177,7 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
     if (g.io_dtype != KVC_BF16 || g.kv_dtype != KVC_BF16 || g.head_dim != 64 || g.page_size != 16 ||
         g.num_heads > kMaxBatchLayers ||
         g.window_frames > 0 || g.budget_tokens > 0 ||
-        (g.diversity_budget + g.page_size - 1) / g.page_size + ppf > 340)
+        ((g.diversity_budget + g.page_size - 1) / g.page_size + ppf) * g.page_size > diversity_prune_max_candidates())
       return KVC_ERR_ARG;
   } else if (g.window_frames <= 0 && g.budget_tokens == 0 && g.max_frames < 1) {
     return KVC_ERR_ARG;
@@ -194,9 +194,10 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   c->ppf = (T + P - 1) / P;
   c->per_head = g.diversity_budget > 0;
   if (c->per_head) {
-    // per head: anchor frame, kept pages twice (old and new during a pruning), one frame
+    // per head: the anchor frame, the kept pages and one pending frame (pruning compacts
+    // the kept tokens in place)
     const int kp = (g.diversity_budget + P - 1) / P;
-    c->pool_pages = 2 * c->ppf + 2 * kp + 2;
+    c->pool_pages = 2 * c->ppf + kp + 1;
     c->layer_budget.assign(g.num_layers, g.diversity_budget);
   } else if (g.window_frames > 0) {
     c->pool_pages = (g.scale_frames + g.window_frames + 1) * c->ppf;
@@ -384,45 +385,43 @@ kvc_status div_append(kvc_cache* c, int layer, int frame_idx, const void* k_dev,
   return KVC_OK;
 }
 
+// Scores every head's candidates and keeps its Top-K (no-op without a pending frame).
+kvc_status div_prune(kvc_cache* c, int layer) {
+  LayerHost& L = c->L[layer];
+  const kvc_config& g = c->cfg;
+  const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads;
+  if (L.pend_pages == 0) return KVC_OK;
+  const size_t sub0 = static_cast<size_t>(layer) * H * c->pool_pages;
+  const int64_t cand = L.mut_tokens + T;
+  const int keep = static_cast<int>(std::min<int64_t>(c->layer_budget[layer], cand));
+  const int n_new = (keep + P - 1) / P;
+  // the kept tokens are compacted in place into the first n_new candidate pages; the
+  // other candidate pages are freed by the kernel
+  cudaError_t e = launch_diversity_prune(c->stream, c->entries + sub0, c->k_pool + sub0 * c->page_bytes_kv,
+                                         c->v_pool + sub0 * c->page_bytes_kv,
+                                         c->bitmap + static_cast<size_t>(layer) * H * c->bitmap_words,
+                                         c->bitmap_words, c->tok_id + sub0 * P, c->pool_pages, L.anchor_pages,
+                                         L.mut_pages + L.pend_pages, keep, H, g.head_dim, P,
+                                         c->div_sums + static_cast<size_t>(layer) * H, c->d_err);
+  if (e != cudaSuccess) return cuda_fail(c, e, "diversity pruning");
+  c->launches++;
+  L.n_entries = L.anchor_pages + n_new;
+  L.mut_pages = n_new;
+  L.mut_tokens = keep;
+  L.pend_pages = 0;
+  L.cand_count = cand;
+  L.compressions++;
+  return KVC_OK;
+}
+
 kvc_status div_attend(kvc_cache* c, int layer, const void* q_dev, void* o_dev) {
+  kvc_status st = div_prune(c, layer);
+  if (st != KVC_OK) return st;
   LayerHost& L = c->L[layer];
   const kvc_config& g = c->cfg;
   const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads;
   const size_t sub0 = static_cast<size_t>(layer) * H * c->pool_pages;
   cudaError_t e;
-  if (L.pend_pages > 0) {
-    const int64_t cand = L.mut_tokens + T;
-    const int keep = static_cast<int>(std::min<int64_t>(c->layer_budget[layer], cand));
-    const int n_new = (keep + P - 1) / P;
-    if (L.n_entries + n_new > c->pool_pages) return fail(c, KVC_ERR_STATE, "kvc_attend: page pool full");
-    LayerStarts st{};
-    st.first_layer = layer * H;
-    for (int h = 0; h < H; ++h) st.start[h] = L.n_entries;
-    e = launch_mgr_alloc_layers(c->stream, c->entries, c->bitmap, c->bitmap_words, c->pool_pages, st, H, n_new, -1, P,
-                                keep - (n_new - 1) * P, c->d_err);
-    if (e != cudaSuccess) return cuda_fail(c, e, "page allocation (kept tokens)");
-    c->launches++;
-    uint8_t* kp = c->k_pool + sub0 * c->page_bytes_kv;
-    uint8_t* vp = c->v_pool + sub0 * c->page_bytes_kv;
-    e = launch_diversity_prune(c->stream, c->entries + sub0, kp, vp, kp, vp, c->tok_id + sub0 * P, c->pool_pages, L.anchor_pages, L.mut_pages + L.pend_pages,
-                               L.n_entries, keep, H, g.head_dim, P, c->div_sums + static_cast<size_t>(layer) * H,
-                               c->d_err);
-    if (e != cudaSuccess) return cuda_fail(c, e, "diversity pruning");
-    c->launches++;
-    // release the previous kept pages and the frame's pages; the new kept pages follow
-    // the anchor
-    const int a = L.anchor_pages, b = L.anchor_pages + L.mut_pages + L.pend_pages;
-    e = launch_mgr_remove_layers(c->stream, c->entries, c->bitmap, c->bitmap_words, c->pool_pages, layer * H, H,
-                                 L.n_entries + n_new, a, b, c->d_err);
-    if (e != cudaSuccess) return cuda_fail(c, e, "page release");
-    c->launches++;
-    L.n_entries = L.anchor_pages + n_new;
-    L.mut_pages = n_new;
-    L.mut_tokens = keep;
-    L.pend_pages = 0;
-    L.cand_count = cand;
-    L.compressions++;
-  }
   TcAttnArgs a{};
   a.q = q_dev;
   a.o = o_dev;
@@ -815,6 +814,14 @@ kvc_status kvc_set_layer_budgets(kvc_cache* c, const int32_t* budgets, int32_t n
       return fail(c, KVC_ERR_ARG, "kvc_set_layer_budgets: budgets must lie in [1, diversity_budget]");
   c->layer_budget.assign(budgets, budgets + n);
   return KVC_OK;
+}
+
+kvc_status kvc_prune(kvc_cache* c, int32_t layer) {
+  if (!c) return KVC_ERR_ARG;
+  if (!c->per_head) return fail(c, KVC_ERR_STATE, "kvc_prune: not a diversity-pruned cache");
+  if (!valid_layer(c, layer)) return fail(c, KVC_ERR_ARG, "kvc_prune: bad layer");
+  if (!c->L[layer].has_pending) return fail(c, KVC_ERR_STATE, "kvc_prune: no frame pending on this layer");
+  return div_prune(c, layer);
 }
 
 kvc_status kvc_layer_diversity(kvc_cache* c, int32_t layer, double* mean_out) {

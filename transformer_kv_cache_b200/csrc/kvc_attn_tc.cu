@@ -62,7 +62,7 @@ constexpr float kPMax = 256.0f;               // a P above 2^8 moves the row's r
 constexpr size_t kSmemBytes = 1024 + 2 * kStages * kTileBytes + kOnesBytes + 256;
 }  // namespace tc
 
-template <int P>
+template <int P, bool kPerHead>
 __global__ void __launch_bounds__(tc::kThreads, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const TcParams p) {
@@ -96,8 +96,8 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
   const int n_tiles = tile1 - tile0;
   // page list and pool rows of this head: shared pages [page][head][slot] or, with
   // per-head page lists, single-head pages of head h's pool region
-  const long long hp = p.head_pages ? static_cast<long long>(h) * p.head_pages : 0;
-  const Entry* ent = p.entries + hp;
+  const long long hp = kPerHead ? static_cast<long long>(h) * p.head_pages : 0;
+  const Entry* ent = kPerHead ? p.entries + hp : p.entries;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 4);                       // the four softmax warps stored Q in TMEM
@@ -148,9 +148,11 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           for (int g = 0; g < kPPT; ++g) {
             const int idx = gt * kPPT + g;
             // pages past the list end are read past the end of the pool: TMA fills zeros
-            row[g] = idx >= p.n_pages ? p.pool_rows
-                     : p.head_pages    ? static_cast<int>((p.page_base + hp + __ldg(&ent[idx].x)) * P)
-                                       : static_cast<int>(((p.page_base + __ldg(&ent[idx].x)) * p.H + h) * P);
+            if (kPerHead)
+              row[g] = idx < p.n_pages ? static_cast<int>((p.page_base + hp + __ldg(&ent[idx].x)) * P) : p.pool_rows;
+            else
+              row[g] = idx < p.n_pages ? static_cast<int>(((p.page_base + __ldg(&ent[idx].x)) * p.H + h) * P)
+                                       : p.pool_rows;
           }
           mbar_arrive_expect_tx(&k_full[st], kTileBytes);
 #pragma unroll
@@ -514,24 +516,27 @@ static bool encode_q_tmap(CUtensorMap* map, const void* q, int T, int H) {
   return r == CUDA_SUCCESS;
 }
 
-// Pick the number of KV splits: fewest waves x tiles-per-CTA over two resident CTAs per SM.
+// Pick the number of KV splits. Cost of a split count, in units of one KV tile of one
+// CTA: waves x (fixed cost of a CTA, about 2.5 tiles: TMEM and barrier set-up, the query
+// tile, the pipeline's fill and drain, the epilogue + tiles per CTA), plus the combine
+// pass that a split needs (about 1 + 0.5 per split). Among counts within 1% of the best
+// cost the fewest splits win (less partial traffic for the same time).
 int choose_splits(int units, int tiles, int slots) {
-  int best = 1;
-  double best_cost = 1e30;
   const int max_s = tiles < 64 ? tiles : 64;
+  double cost[65];
+  double best_cost = 1e30;
   for (int s = 1; s <= max_s; ++s) {
+    cost[s] = 1e30;
     const int tps = (tiles + s - 1) / s;
-    const int s_eff = (tiles + tps - 1) / tps;
-    const long long ctas = static_cast<long long>(units) * s_eff;
+    if ((tiles + tps - 1) / tps != s) continue;        // the same as a smaller split count
+    const long long ctas = static_cast<long long>(units) * s;
     const long long waves = (ctas + slots - 1) / slots;
-    // combine traffic grows with the split count: charge it lightly
-    const double cost = static_cast<double>(waves) * tps * (1.0 + 0.004 * s_eff);
-    if (cost < best_cost - 1e-9) {
-      best_cost = cost;
-      best = s_eff;
-    }
+    cost[s] = static_cast<double>(waves) * (2.5 + tps) + (s > 1 ? 1.0 + 0.5 * s : 0.0);
+    if (cost[s] < best_cost) best_cost = cost[s];
   }
-  return best;
+  for (int s = 1; s <= max_s; ++s)
+    if (cost[s] <= best_cost * 1.01) return s;
+  return 1;
 }
 
 cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used, int* launched) {
@@ -539,8 +544,11 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   if (a.P != 16 || (a.fp8 && a.head_pages)) return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!a.fp8 && !attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(tc::kSmemBytes));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_tc_kernel<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(tc::kSmemBytes));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -589,7 +597,10 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   if (a.fp8) {
     e = launch_attn_fp8_kernel(s, tq, *a.tmap_k, *a.tmap_v, prm, grid);
   } else {
-    attn_tc_kernel<16><<<grid, tc::kThreads, tc::kSmemBytes, s>>>(tq, *a.tmap_k, *a.tmap_v, prm);
+    if (a.head_pages)
+      attn_tc_kernel<16, true><<<grid, tc::kThreads, tc::kSmemBytes, s>>>(tq, *a.tmap_k, *a.tmap_v, prm);
+    else
+      attn_tc_kernel<16, false><<<grid, tc::kThreads, tc::kSmemBytes, s>>>(tq, *a.tmap_k, *a.tmap_v, prm);
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return e;

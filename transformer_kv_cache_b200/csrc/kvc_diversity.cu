@@ -9,12 +9,17 @@
 // kernels serve the sub-layers exactly as they serve layers.
 //
 // Scores follow the definition in fp64 with a fixed evaluation order, so the kept sets
-// match an fp64 reference bit for bit: |k| = sqrt of the squares summed over ascending
-// dims; k_hat = k / |k| (0 for a zero key); mu = sum of k_hat over the candidates in
-// ascending token id (the direction of the mean); score = -(k_hat . mu) / |mu| with both
-// sums over ascending dims; each step one IEEE operation (explicitly rounded intrinsics,
-// no contraction).
+// match an fp64 reference bit for bit: every sum over the 64 dims (the squares of |k|,
+// the dot k_hat . mu, the squares of |mu|) is taken in 8 blocks of 8 consecutive dims,
+// ascending within a block, then the block sums ascending; k_hat = k * RN(1 / |k|) (0 for
+// a zero key); mu = the sum of k_hat over the candidates (the direction of the mean) and a
+// head's score total are both taken in blocks of 32 consecutive candidates in ascending
+// token id, ascending within a block, then the block sums ascending; score =
+// -(k_hat . mu) / |mu|; each step one IEEE operation (explicitly rounded intrinsics, no
+// contraction).
 #include <cuda_bf16.h>
+
+#include <climits>
 
 #include "kvc_internal.h"
 #include "sm100_ptx.cuh"
@@ -22,7 +27,6 @@
 namespace kvc {
 namespace {
 
-constexpr int kDivThreads = 512;
 constexpr int kDivD = 64;
 
 // One 16-byte chunk per thread-iteration over (head, page, slot, chunk) of one frame, for
@@ -53,183 +57,459 @@ __global__ void append_heads_kernel(const uint4* __restrict__ k, const uint4* __
   }
 }
 
-// One CTA per head of the layer. Candidates: the slots of page-list entries
-// [first, first + n_entries) of the head (the kept pages, then the new frame's pages),
-// in ascending token id. Keeps the `keep` best by (score descending, id ascending),
-// writes them in ascending id into the head's pages at entries [new_entry, ...), zeroes
-// the tail slots of the last new page, and stores the head's score sum (ascending id).
-__global__ void __launch_bounds__(kDivThreads) diversity_prune_kernel(
-    const Entry* __restrict__ entries_layer, const __nv_bfloat16* __restrict__ k_pool,
-    const __nv_bfloat16* __restrict__ v_pool, __nv_bfloat16* k_pool_w, __nv_bfloat16* v_pool_w, int64_t* tok_id_layer,
-    int pool_pages, int first, int n_entries, int new_entry, int keep, int P, double* sums_layer, int* err) {
+// ------------------------------------------------------------------ pruning
+// One cluster of kPruneCluster CTAs per head. The head's candidates are the valid slots
+// of its page-list entries [first, first + n_entries) (the kept pages, then the new
+// frame's pages), in ascending token id; CTA r of the cluster owns candidates
+// [r * B, r * B + B) (B a multiple of the 32-candidate block, so every block of a sum
+// over candidates lies in one CTA) and stages their K and V rows in shared memory first.
+// Each CTA publishes its blocks' partial sums of the normalised keys, then its scores, in
+// its own shared memory; after a cluster barrier the others read them (distributed shared
+// memory), and every CTA selects the Top-K itself. The kept candidates are written in
+// place, in ascending id, over the slots of the first ceil(kept / P) candidate entries
+// (every CTA's reads of the pool precede the first barrier); the pages of the remaining
+// candidate entries go back to the head's free bitmap.
+constexpr int kPruneCluster = 8;
+constexpr int kPruneThreads = 512;
+constexpr int kCandBlock = 32;          // candidates per block of every sum over candidates
+constexpr int kDimBlock = 8;            // dims per block of every sum over the dims
+constexpr int kPruneMaxB = 256;         // candidates per CTA (2,048 per head)
+constexpr int kKRowStride = kDivD + 8;  // bf16 per staged key row: 144 bytes spread the banks
+constexpr int kBins = 2048;             // selection histogram over [-1, 1]
+
+struct PruneLayout {
+  uint32_t sc_all, bsum_own, bsum_all, ssum_own, ssum_all, krow, vrow, rcp, score, id, slot, pos, page, hist, sbin,
+      bucket, kflag, total;
+};
+
+__host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
+
+__host__ __device__ inline PruneLayout prune_layout(int n_max, int B, int n_entries) {
+  PruneLayout l;
+  const size_t nblk = static_cast<size_t>((n_max + kCandBlock - 1) / kCandBlock);
+  const size_t b = static_cast<size_t>(B), bb = b / kCandBlock, n = static_cast<size_t>(n_max);
+  size_t o = 0;
+  auto take = [&o](size_t bytes) {
+    const uint32_t r = static_cast<uint32_t>(o);
+    o += align16(bytes);
+    return r;
+  };
+  l.sc_all = take((n + 1) * 8);           // one spare: pairs are read 16 bytes at a time
+  l.bsum_own = take(bb * kDivD * 8);
+  // the block sums of all CTAs are dead once mu is known: the selection reuses their space
+  const size_t sel_bytes = align16(kBins * 4) + align16(n * 2) + align16(n * 4) + align16(n);
+  const size_t bsum_bytes = nblk * kDivD * 8;
+  l.bsum_all = take(bsum_bytes > sel_bytes ? bsum_bytes : sel_bytes);
+  l.hist = l.bsum_all;
+  l.sbin = l.hist + static_cast<uint32_t>(align16(kBins * 4));
+  l.bucket = l.sbin + static_cast<uint32_t>(align16(n * 2));
+  l.kflag = l.bucket + static_cast<uint32_t>(align16(n * 4));
+  l.ssum_own = take(bb * 8);
+  l.ssum_all = take(nblk * 8);
+  l.krow = take(b * kKRowStride * 2);
+  l.vrow = take(b * kDivD * 2);
+  l.rcp = take(b * 8);
+  l.score = take(b * 8);
+  l.id = take(b * 8);
+  l.slot = take(b * 4);
+  l.pos = take(b * 4);
+  l.page = take(static_cast<size_t>(n_entries) * 4);
+  l.total = static_cast<uint32_t>(o);
+  return l;
+}
+
+__device__ __forceinline__ double bf16_lo(uint32_t w) { return static_cast<double>(__uint_as_float(w << 16)); }
+__device__ __forceinline__ double bf16_hi(uint32_t w) { return static_cast<double>(__uint_as_float(w & 0xffff0000u)); }
+
+// One 8-dim block of a sum over the dims, from 8 bf16 values (ascending):
+// part = sum of x * x, or of (x * r) * m[d]
+__device__ __forceinline__ double block_sq(const uint4 u) {
+  const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+  double part = 0.0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const double a = bf16_lo(wv[j]), b = bf16_hi(wv[j]);
+    part = __dadd_rn(part, __dmul_rn(a, a));
+    part = __dadd_rn(part, __dmul_rn(b, b));
+  }
+  return part;
+}
+// m is read from shared memory at every use (volatile): the mean's 64 components kept in
+// registers across the candidate loop would not fit beside the rest of the kernel.
+__device__ __forceinline__ double block_dot(const uint4 u, double r, const volatile double* m) {
+  const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+  double part = 0.0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    part = __dadd_rn(part, __dmul_rn(__dmul_rn(bf16_lo(wv[j]), r), m[2 * j]));
+    part = __dadd_rn(part, __dmul_rn(__dmul_rn(bf16_hi(wv[j]), r), m[2 * j + 1]));
+  }
+  return part;
+}
+
+// Monotone histogram bin of a score in [-1, 1] (clamped): a higher bin means a higher score.
+__device__ __forceinline__ int score_bin(double s) {
+  const double t = (s + 1.0) * (kBins / 2);
+  return t >= kBins - 1 ? kBins - 1 : (t > 0.0 ? static_cast<int>(t) : 0);
+}
+
+__device__ __forceinline__ int warp_incl_scan(int v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
+  }
+  return v;
+}
+
+// Exclusive prefix sum of one value per thread over the CTA; every thread calls it.
+__device__ int cta_scan_excl(int x, int* s_warp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int v = warp_incl_scan(x);
+  if (lane == 31) s_warp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = warp_incl_scan(lane < nw ? s_warp[lane] : 0);
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  const int r = v - x + (warp > 0 ? s_warp[warp - 1] : 0);
+  *total = s_warp[nw - 1];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __cluster_dims__(kPruneCluster, 1, 1) __launch_bounds__(kPruneThreads, 2) diversity_prune_kernel(
+    Entry* entries_layer, __nv_bfloat16* k_pool, __nv_bfloat16* v_pool, uint32_t* bitmap_layer, int words,
+    int64_t* tok_id_layer, int pool_pages, int first, int n_entries, int keep, int P, int B, double* sums_layer,
+    int* err) {
   extern __shared__ __align__(16) uint8_t sm[];
-  const int h = blockIdx.x;
-  const long long sub = static_cast<long long>(h) * pool_pages;
-  const Entry* E = entries_layer + sub;
-  __shared__ int s_off[1025];
+  __shared__ int s_warp[32];
   __shared__ double s_mu[kDivD];
   __shared__ double s_mnorm;
-  __shared__ int s_n;
-  __shared__ int s_warp[32];
-  // candidate slots (offset of each entry's first candidate: one thread, <= 1024 entries)
-  if (threadIdx.x == 0) {
-    int o = 0;
-    for (int e = 0; e < n_entries; ++e) {
-      s_off[e] = o;
-      o += E[first + e].w;
-    }
-    s_off[n_entries] = o;
-    s_n = o;
+  __shared__ int s_sel, s_above, s_cnt, s_bcnt;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int h = blockIdx.x / kPruneCluster;
+  const int tid = threadIdx.x;
+  const long long sub = static_cast<long long>(h) * pool_pages;
+  Entry* E = entries_layer + sub;
+  const PruneLayout lay = prune_layout(n_entries * P, B, n_entries);
+  double* sc_all = reinterpret_cast<double*>(sm + lay.sc_all);          // [N] every candidate's score
+  double* bsum_own = reinterpret_cast<double*>(sm + lay.bsum_own);      // [B/32][D] published
+  double* bsum_all = reinterpret_cast<double*>(sm + lay.bsum_all);      // [blocks][D]
+  double* ssum_own = reinterpret_cast<double*>(sm + lay.ssum_own);      // [B/32] published
+  double* ssum_all = reinterpret_cast<double*>(sm + lay.ssum_all);      // [blocks] (CTA 0)
+  __nv_bfloat16* krow = reinterpret_cast<__nv_bfloat16*>(sm + lay.krow);  // [B][kKRowStride]
+  uint4* vrow = reinterpret_cast<uint4*>(sm + lay.vrow);                // [B][8]
+  double* rcp = reinterpret_cast<double*>(sm + lay.rcp);                // [B] RN(1 / |k|), 0 for |k| = 0
+  double* score = reinterpret_cast<double*>(sm + lay.score);            // [B] published
+  int64_t* ids = reinterpret_cast<int64_t*>(sm + lay.id);               // [B] token ids
+  int* slot = reinterpret_cast<int*>(sm + lay.slot);                    // [B] pool slot within the head
+  int* pos = reinterpret_cast<int*>(sm + lay.pos);                      // [B] kept position, or -1
+  int* page = reinterpret_cast<int*>(sm + lay.page);                    // [n_entries] physical pages
+  int* s_hist = reinterpret_cast<int*>(sm + lay.hist);                  // [kBins] (after mu)
+  uint16_t* sbin = reinterpret_cast<uint16_t*>(sm + lay.sbin);          // [N] histogram bin
+  int* bucket = reinterpret_cast<int*>(sm + lay.bucket);                // [N] the threshold bin's members
+  uint8_t* kflag = sm + lay.kflag;                                      // [N] kept
+  const int bpc = B / kCandBlock;                                       // blocks per CTA
+
+  // candidate offsets of the entries (one entry per thread) and the own candidates' slots
+  int w = 0, x = 0;
+  if (tid < n_entries) {
+    const Entry en = E[first + tid];
+    w = en.w;
+    x = en.x;
+    page[tid] = x;
   }
-  __syncthreads();
-  const int N = s_n;
-  int32_t* c_slot = reinterpret_cast<int32_t*>(sm);                      // [N] pool slot within the head
-  double* c_norm = reinterpret_cast<double*>(sm + ((static_cast<size_t>(N) * 4 + 15) & ~size_t(15)));
-  double* c_score = c_norm + N;
-  int64_t* c_id = reinterpret_cast<int64_t*>(c_score + N);
-  int32_t* c_keep = reinterpret_cast<int32_t*>(c_id + N);
-  for (int e = threadIdx.x; e < n_entries; e += blockDim.x) {
-    const Entry en = E[first + e];
-    for (int s = 0; s < en.w; ++s) {
-      const int i = s_off[e] + s;
-      c_slot[i] = en.x * P + s;
-      c_id[i] = tok_id_layer[(sub + en.x) * P + s];
-    }
+  int N;
+  const int o = cta_scan_excl(w, s_warp, &N);
+  const int c0 = rank * B;
+  const int nl = max(0, min(N, c0 + B) - c0);
+  for (int s = 0; s < w; ++s) {
+    const int i = o + s - c0;
+    if (i >= 0 && i < nl) slot[i] = x * P + s;
   }
+  if (rank == 0 && tid == 0 && N < keep) latch_error(err, DERR_BOUNDS);
   __syncthreads();
-  auto krow = [&](int i) { return k_pool + (sub * P + c_slot[i]) * kDivD; };
-  // norms: squares summed over ascending dims
-  for (int i = threadIdx.x; i < N; i += blockDim.x) {
-    const __nv_bfloat16* kr = krow(i);
+  // own K and V rows and token ids into shared memory: every read of the pool happens here
+  for (int it = tid; it < nl * 16; it += blockDim.x) {
+    const int li = it >> 4, q = it & 15;
+    const long long src = sub * P + slot[li];
+    if (q < 8) cp_async16(krow + li * kKRowStride + q * 8, k_pool + src * kDivD + q * 8);
+    else cp_async16(vrow + li * 8 + q - 8, v_pool + src * kDivD + (q - 8) * 8);
+    if (q == 0) cp_async8(ids + li, tok_id_layer + src);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  // |k| (a sum over the dims in 8-dim blocks) and its reciprocal
+#pragma unroll 1
+  for (int li = tid; li < nl; li += blockDim.x) {
+    const uint4* kr = reinterpret_cast<const uint4*>(krow + li * kKRowStride);
     double acc = 0.0;
-    for (int d = 0; d < kDivD; ++d) {
-      const double x = static_cast<double>(__bfloat162float(kr[d]));
-      acc = __dadd_rn(acc, __dmul_rn(x, x));
+#pragma unroll
+    for (int hq = 0; hq < kDivD / kDimBlock; hq += 4) {   // four blocks in flight, added in order
+      double part[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) part[q] = block_sq(kr[hq + q]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc = __dadd_rn(acc, part[q]);
     }
-    c_norm[i] = __dsqrt_rn(acc);
+    const double n = __dsqrt_rn(acc);
+    rcp[li] = n > 0.0 ? __ddiv_rn(1.0, n) : 0.0;
   }
   __syncthreads();
-  // mu_d: normalised keys summed over ascending candidates (one thread per dim)
-  if (threadIdx.x < kDivD) {
-    const int d = threadIdx.x;
-    double mu = 0.0;
-    for (int i = 0; i < N; ++i) {
-      const double n = c_norm[i];
-      const double kh = n > 0.0 ? __ddiv_rn(static_cast<double>(__bfloat162float(krow(i)[d])), n) : 0.0;
-      mu = __dadd_rn(mu, kh);
+  // own blocks' sums of k_hat = k * rcp, ascending within the block
+  const int nb_own = (nl + kCandBlock - 1) / kCandBlock;
+  for (int it = tid; it < nb_own * kDivD; it += blockDim.x) {
+    const int j = it / kDivD, d = it % kDivD;
+    const int i0 = j * kCandBlock, n = min(nl - i0, kCandBlock);
+    const __nv_bfloat16* kc = krow + i0 * kKRowStride + d;
+    double sum = 0.0;
+#pragma unroll 8
+    for (int t = 0; t < kCandBlock; ++t)
+      if (t < n)
+        sum = __dadd_rn(sum, __dmul_rn(static_cast<double>(__bfloat162float(kc[t * kKRowStride])), rcp[i0 + t]));
+    bsum_own[j * kDivD + d] = sum;
+  }
+  __syncwarp();
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  // every block's partial sums, read from the CTA that owns it (all loads in flight first)
+  const int nblk = (N + kCandBlock - 1) / kCandBlock;
+  {
+    constexpr int kMaxIt = kPruneCluster * kPruneMaxB / kCandBlock * (kDivD / 2) / kPruneThreads;
+    uint64_t u[kMaxIt][2];
+#pragma unroll
+    for (int k = 0; k < kMaxIt; ++k) {
+      const int it = tid + k * kPruneThreads;
+      if (it < nblk * (kDivD / 2)) {
+        const int b = it / (kDivD / 2), d2 = it % (kDivD / 2);
+        ld_cluster_v2u64(cluster_map(smem_u32(bsum_own + (b % bpc) * kDivD + 2 * d2), b / bpc), u[k][0], u[k][1]);
+      }
     }
-    s_mu[d] = mu;
+#pragma unroll
+    for (int k = 0; k < kMaxIt; ++k) {
+      const int it = tid + k * kPruneThreads;
+      if (it < nblk * (kDivD / 2)) {
+        bsum_all[2 * it] = __longlong_as_double(static_cast<long long>(u[k][0]));
+        bsum_all[2 * it + 1] = __longlong_as_double(static_cast<long long>(u[k][1]));
+      }
+    }
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    double m2 = 0.0;
-    for (int d = 0; d < kDivD; ++d) m2 = __dadd_rn(m2, __dmul_rn(s_mu[d], s_mu[d]));
-    s_mnorm = __dsqrt_rn(m2);
+  // mu: the block sums in ascending block order; |mu|^2 a sum over the dims in 8-dim blocks
+  if (tid < kDivD) {
+    double m = 0.0;
+    for (int b = 0; b < nblk; ++b) m = __dadd_rn(m, bsum_all[b * kDivD + tid]);
+    s_mu[tid] = m;
+  }
+  __syncthreads();
+  if (tid < kDivD / kDimBlock) {
+    double part = 0.0;
+#pragma unroll
+    for (int d = 0; d < kDimBlock; ++d) {
+      const double m = s_mu[tid * kDimBlock + d];
+      part = __dadd_rn(part, __dmul_rn(m, m));
+    }
+    double acc = __shfl_sync(0xffu, part, 0, 8);
+    acc = __dadd_rn(0.0, acc);
+#pragma unroll
+    for (int q = 1; q < kDivD / kDimBlock; ++q) acc = __dadd_rn(acc, __shfl_sync(0xffu, part, q, 8));
+    if (tid == 0) s_mnorm = __dsqrt_rn(acc);
   }
   __syncthreads();
   const double mnorm = s_mnorm;
-  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+  // scores -(k_hat . mu) / |mu| (the dot a sum over the dims in 8-dim blocks)
+#pragma unroll 1
+  for (int li = tid; li < nl; li += blockDim.x) {
     double sc = 0.0;
-    const double n = c_norm[i];
     if (mnorm > 0.0) {
-      const __nv_bfloat16* kr = krow(i);
+      const uint4* kr = reinterpret_cast<const uint4*>(krow + li * kKRowStride);
+      const double r = rcp[li];
       double dot = 0.0;
-      for (int d = 0; d < kDivD; ++d) {
-        const double kh = n > 0.0 ? __ddiv_rn(static_cast<double>(__bfloat162float(kr[d])), n) : 0.0;
-        dot = __dadd_rn(dot, __dmul_rn(kh, s_mu[d]));
+#pragma unroll
+      for (int hq = 0; hq < kDivD / kDimBlock; hq += 4) {
+        double part[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) part[q] = block_dot(kr[hq + q], r, s_mu + (hq + q) * kDimBlock);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dot = __dadd_rn(dot, part[q]);
       }
       sc = -__ddiv_rn(dot, mnorm);
     }
-    c_score[i] = sc;
+    score[li] = sc;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    double s = 0.0;
-    for (int i = 0; i < N; ++i) s = __dadd_rn(s, c_score[i]);
-    sums_layer[h] = s;
+  for (int j = tid; j < nb_own; j += blockDim.x) {
+    const int i1 = min(nl, (j + 1) * kCandBlock);
+    double sum = 0.0;
+    for (int li = j * kCandBlock; li < i1; ++li) sum = __dadd_rn(sum, score[li]);
+    ssum_own[j] = sum;
   }
-  // rank by counting: (score descending, id ascending) is a strict total order
-  for (int i = threadIdx.x; i < N; i += blockDim.x) {
-    const double si = c_score[i];
-    const int64_t ii = c_id[i];
-    int r = 0;
-    for (int j = 0; j < N; ++j) {
-      const double sj = c_score[j];
-      r += (sj > si) || (sj == si && c_id[j] < ii);
-    }
-    c_keep[i] = r < keep;
-  }
-  __syncthreads();
-  // compaction: kept candidates in ascending id (= candidate order) into the new pages
-  int base = 0;
-  for (int chunk = 0; chunk < N; chunk += blockDim.x) {
-    const int i = chunk + threadIdx.x;
-    const int f = i < N ? c_keep[i] : 0;
-    int x = f;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  __syncwarp();
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  // every candidate's score (pairs of 16 bytes; B is even, so a pair never spans two CTAs);
+  // CTA 0 also the score block sums
+  {
+    constexpr int kMaxIt = kPruneCluster * kPruneMaxB / 2 / kPruneThreads;
+    uint64_t u[kMaxIt][2];
+    const int npair = (N + 1) / 2;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) s_warp[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-      int w = lane < nw ? s_warp[lane] : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, w, o);
-        if (lane >= o) w += y;
+    for (int k = 0; k < kMaxIt; ++k) {
+      const int it = tid + k * kPruneThreads;
+      if (it < npair) {
+        const int i = 2 * it;
+        ld_cluster_v2u64(cluster_map(smem_u32(score + i % B), i / B), u[k][0], u[k][1]);
       }
-      s_warp[lane] = w;
+    }
+    double sb = 0.0;
+    if (rank == 0 && tid < nblk)
+      sb = __longlong_as_double(
+          static_cast<long long>(ld_cluster_u64(cluster_map(smem_u32(ssum_own + tid % bpc), tid / bpc))));
+#pragma unroll
+    for (int k = 0; k < kMaxIt; ++k) {
+      const int it = tid + k * kPruneThreads;
+      if (it < npair) {
+        sc_all[2 * it] = __longlong_as_double(static_cast<long long>(u[k][0]));
+        sc_all[2 * it + 1] = __longlong_as_double(static_cast<long long>(u[k][1]));
+      }
+    }
+    if (rank == 0 && tid < nblk) ssum_all[tid] = sb;
+  }
+  __syncthreads();
+  __syncwarp();
+  cluster_arrive_release();   // this CTA reads no other CTA's shared memory any more
+
+  // Top-K by (score descending, id ascending): a histogram of monotone score bins finds the
+  // bin that holds the kk-th best; candidates in higher bins are kept, and the members of
+  // that bin are ranked exactly among themselves (ties to the lower id).
+  const int kk = keep < N ? keep : N;
+  if (kk >= N) {
+    for (int i = tid; i < N; i += blockDim.x) kflag[i] = 1;
+  } else {
+    for (int b = tid; b < kBins; b += blockDim.x) s_hist[b] = 0;
+    if (tid == 0) s_bcnt = 0;
+    __syncthreads();
+    for (int i = tid; i < N; i += blockDim.x) {
+      const int b = score_bin(sc_all[i]);
+      sbin[i] = static_cast<uint16_t>(b);
+      atomicAdd(&s_hist[b], 1);
     }
     __syncthreads();
-    const int pos = base + (warp > 0 ? s_warp[warp - 1] : 0) + x - f;
-    const int total = s_warp[nw - 1];
-    if (f) {
-      if (pos >= keep) latch_error(err, DERR_BOUNDS);
-      else {
-        const int phys = E[new_entry + pos / P].x;
-        const long long dst = (sub + phys) * P + pos % P;
-        const long long src = sub * P + c_slot[i];
-        const uint4* ks = reinterpret_cast<const uint4*>(k_pool + src * kDivD);
-        const uint4* vs = reinterpret_cast<const uint4*>(v_pool + src * kDivD);
-        uint4* kd = reinterpret_cast<uint4*>(k_pool_w + dst * kDivD);
-        uint4* vd = reinterpret_cast<uint4*>(v_pool_w + dst * kDivD);
+    // thread t holds bins 2047 - 4t down to 2044 - 4t
+    constexpr int kPer = kBins / kPruneThreads;
+    int c[kPer], lsum = 0;
 #pragma unroll
-        for (int q = 0; q < kDivD / 8; ++q) {
-          kd[q] = ks[q];
-          vd[q] = vs[q];
+    for (int k = 0; k < kPer; ++k) {
+      c[k] = s_hist[kBins - 1 - kPer * tid - k];
+      lsum += c[k];
+    }
+    int tot;
+    int acc = cta_scan_excl(lsum, s_warp, &tot);
+    if (acc < kk && kk <= acc + lsum) {
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        if (acc < kk && kk <= acc + c[k]) {
+          s_sel = kBins - 1 - kPer * tid - k;
+          s_above = acc;
+          s_cnt = c[k];
         }
-        tok_id_layer[dst] = c_id[i];
+        acc += c[k];
       }
     }
-    base += total;
+    __syncthreads();
+    const int sel = s_sel, rem = kk - s_above, cnt = s_cnt;
+    for (int i = tid; i < N; i += blockDim.x) {
+      const int b = sbin[i];
+      kflag[i] = b > sel;
+      if (b == sel) bucket[atomicAdd(&s_bcnt, 1)] = i;
+    }
+    __syncthreads();
+    if (tid == 0 && s_bcnt != cnt) latch_error(err, DERR_BOUNDS);
+    for (int m = tid; m < cnt; m += blockDim.x) {
+      const int a = bucket[m];
+      const double sa = sc_all[a];
+      int r = 0;
+      for (int m2 = 0; m2 < cnt; ++m2) {
+        const int b = bucket[m2];
+        const double sbv = sc_all[b];
+        r += (sbv > sa) || (sbv == sa && b < a);
+      }
+      kflag[a] = r < rem;
+    }
     __syncthreads();
   }
-  // the last new page's slots past the kept count: zero K and V, no token
-  const int n_new = (keep + P - 1) / P;
-  const int tail0 = keep, tail1 = n_new * P;
-  for (int t = tail0 + static_cast<int>(threadIdx.x); t < tail1; t += blockDim.x) {
-    const int phys = E[new_entry + t / P].x;
-    const long long dst = (sub + phys) * P + t % P;
-    uint4* kd = reinterpret_cast<uint4*>(k_pool_w + dst * kDivD);
-    uint4* vd = reinterpret_cast<uint4*>(v_pool_w + dst * kDivD);
-#pragma unroll
-    for (int q = 0; q < kDivD / 8; ++q) {
-      kd[q] = make_uint4(0, 0, 0, 0);
-      vd[q] = make_uint4(0, 0, 0, 0);
+  // positions: kept candidates numbered in ascending id (contiguous chunks per thread)
+  {
+    const int ch = (N + blockDim.x - 1) / blockDim.x;
+    const int i0 = min(N, tid * ch), i1 = min(N, i0 + ch);
+    int n_kept = 0;
+    for (int i = i0; i < i1; ++i) n_kept += kflag[i];
+    int tot;
+    int p = cta_scan_excl(n_kept, s_warp, &tot);
+    if (tid == 0 && tot != kk) latch_error(err, DERR_BOUNDS);
+    for (int i = i0; i < i1; ++i) {
+      const bool kept = kflag[i];
+      if (i >= c0 && i < c0 + nl) pos[i - c0] = kept ? p : -1;
+      p += kept;
     }
-    tok_id_layer[dst] = -1;
   }
+  __syncthreads();
+  // kept position p goes to slot p % P of candidate entry first + p / P
+  uint4* kd = reinterpret_cast<uint4*>(k_pool);
+  uint4* vd = reinterpret_cast<uint4*>(v_pool);
+  for (int it = tid; it < nl * 16; it += blockDim.x) {
+    const int li = it >> 4, q = it & 15;
+    const int p = pos[li];
+    if (p < 0) continue;
+    if (p >= kk) {
+      latch_error(err, DERR_BOUNDS);
+      continue;
+    }
+    const long long dst = (sub + page[p / P]) * P + p % P;
+    if (q < 8) kd[dst * 8 + q] = reinterpret_cast<const uint4*>(krow + li * kKRowStride)[q];
+    else vd[dst * 8 + q - 8] = vrow[li * 8 + q - 8];
+    if (q == 0) tok_id_layer[dst] = ids[li];
+  }
+  const int n_new = (kk + P - 1) / P;
+  if (rank == kPruneCluster - 1) {
+    // the last kept page's slots past the kept count: zero K and V, no token
+    for (int it = tid; it < (n_new * P - kk) * 16; it += blockDim.x) {
+      const int t = kk + (it >> 4), q = it & 15;
+      const long long dst = (sub + page[t / P]) * P + t % P;
+      if (q < 8) kd[dst * 8 + q] = make_uint4(0, 0, 0, 0);
+      else vd[dst * 8 + q - 8] = make_uint4(0, 0, 0, 0);
+      if (q == 0) tok_id_layer[dst] = -1;
+    }
+  }
+  if (rank == 0) {
+    // the kept pages' entries (owner -1: compaction), the other candidate pages freed
+    uint32_t* bitmap = bitmap_layer + static_cast<long long>(h) * words;
+    for (int e = tid; e < n_entries; e += blockDim.x) {
+      int* en = reinterpret_cast<int*>(E + first + e);
+      if (e < n_new) {
+        en[1] = -1;
+        en[2] = e;
+        en[3] = min(P, kk - e * P);
+      } else {
+        const uint32_t bit = 1u << (page[e] & 31);
+        const uint32_t old = atomicAnd(&bitmap[page[e] >> 5], ~bit);
+        if (!(old & bit)) latch_error(err, DERR_BOUNDS);
+      }
+    }
+    if (tid == 0) {
+      double t = 0.0;
+      for (int b = 0; b < nblk; ++b) t = __dadd_rn(t, ssum_all[b]);
+      sums_layer[h] = t;
+    }
+  }
+  __syncwarp();
+  cluster_wait_acquire();     // no CTA leaves while another may still read its shared memory
 }
 
 }  // namespace
-
-size_t diversity_prune_smem(int n_cand) {
-  const size_t a = (static_cast<size_t>(n_cand) * 4 + 15) & ~size_t(15);
-  return a + static_cast<size_t>(n_cand) * (8 + 8 + 8 + 4);
-}
 
 cudaError_t launch_append_heads(cudaStream_t s, const void* k, const void* v, void* k_pool, void* v_pool,
                                 const Entry* entries_layer, int64_t* tok_id_layer, int pool_pages, int start,
@@ -246,14 +526,19 @@ cudaError_t launch_append_heads(cudaStream_t s, const void* k, const void* v, vo
   return cudaGetLastError();
 }
 
-cudaError_t launch_diversity_prune(cudaStream_t s, Entry* entries_layer, const void* k_pool, const void* v_pool,
-                                   void* k_pool_w, void* v_pool_w, int64_t* tok_id_layer, int pool_pages,
-                                   int first_cand_entry, int n_cand_entries, int new_entry, int keep, int H, int D,
-                                   int P, double* sums_layer, int* err) {
-  if (D != kDivD || n_cand_entries > 1024) return cudaErrorInvalidValue;
+int diversity_prune_max_candidates() { return kPruneCluster * kPruneMaxB; }
+
+cudaError_t launch_diversity_prune(cudaStream_t s, Entry* entries_layer, void* k_pool, void* v_pool,
+                                   uint32_t* bitmap_layer, int words, int64_t* tok_id_layer, int pool_pages,
+                                   int first_cand_entry, int n_cand_entries, int keep, int H, int D, int P,
+                                   double* sums_layer, int* err) {
   const int n_max = n_cand_entries * P;
-  const size_t smem = diversity_prune_smem(n_max);
-  // dynamic plus static shared memory above 48 KB needs the opt-in limit raised
+  if (D != kDivD || n_cand_entries < 1 || n_cand_entries > kPruneThreads || keep < 1 ||
+      n_max > kPruneCluster * kPruneMaxB)
+    return cudaErrorInvalidValue;
+  int B = (n_max + kPruneCluster - 1) / kPruneCluster;
+  B = (B + kCandBlock - 1) / kCandBlock * kCandBlock;
+  const size_t smem = prune_layout(n_max, B, n_cand_entries).total;
   static size_t attr = 0;
   if (smem > attr) {
     cudaError_t e = cudaFuncSetAttribute(diversity_prune_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -261,10 +546,9 @@ cudaError_t launch_diversity_prune(cudaStream_t s, Entry* entries_layer, const v
     if (e != cudaSuccess) return e;
     attr = smem;
   }
-  diversity_prune_kernel<<<H, kDivThreads, smem, s>>>(
-      entries_layer, static_cast<const __nv_bfloat16*>(k_pool), static_cast<const __nv_bfloat16*>(v_pool),
-      static_cast<__nv_bfloat16*>(k_pool_w), static_cast<__nv_bfloat16*>(v_pool_w), tok_id_layer, pool_pages,
-      first_cand_entry, n_cand_entries, new_entry, keep, P, sums_layer, err);
+  diversity_prune_kernel<<<H * kPruneCluster, kPruneThreads, smem, s>>>(
+      entries_layer, static_cast<__nv_bfloat16*>(k_pool), static_cast<__nv_bfloat16*>(v_pool), bitmap_layer, words,
+      tok_id_layer, pool_pages, first_cand_entry, n_cand_entries, keep, P, B, sums_layer, err);
   return cudaGetLastError();
 }
 

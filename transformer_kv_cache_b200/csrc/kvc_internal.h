@@ -200,14 +200,11 @@ cudaError_t launch_merge_targets(cudaStream_t s, const __nv_bfloat16* ks, const 
 cudaError_t launch_append_heads(cudaStream_t s, const void* k, const void* v, void* k_pool, void* v_pool,
                                 const Entry* entries_layer, int64_t* tok_id_layer, int pool_pages, int start,
                                 int n_pages, int T, int H, int D, int P, int frame);
-cudaError_t launch_diversity_prune(cudaStream_t s, Entry* entries_layer, const void* k_pool, const void* v_pool,
-                                   void* k_pool_w, void* v_pool_w, int64_t* tok_id_layer, int pool_pages,
-                                   int first_cand_entry, int n_cand_entries, int new_entry, int keep, int H, int D,
-                                   int P, double* sums_layer, int* err);
-cudaError_t launch_mgr_remove_layers(cudaStream_t s, Entry* entries_all, uint32_t* bitmap_all, int words,
-                                     int pool_pages, int first_layer, int n_layers, int n_entries, int a, int b,
-                                     int* err);
-size_t diversity_prune_smem(int n_cand);
+int diversity_prune_max_candidates();
+cudaError_t launch_diversity_prune(cudaStream_t s, Entry* entries_layer, void* k_pool, void* v_pool,
+                                   uint32_t* bitmap_layer, int words, int64_t* tok_id_layer, int pool_pages,
+                                   int first_cand_entry, int n_cand_entries, int keep, int H, int D, int P,
+                                   double* sums_layer, int* err);
 
 // Compression kernels.
 cudaError_t launch_score(cudaStream_t s, const float* residual, int T, int R, int layer_slot, int n_hist,

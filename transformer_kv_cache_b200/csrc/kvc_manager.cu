@@ -92,11 +92,9 @@ __global__ void __launch_bounds__(kMgrThreads) mgr_alloc_kernel(Entry* entries_a
 // Release the pages of entries [a, b) and close the gap: entries [b, n) move to [a, ...).
 // The move runs in chunks of the block size with a barrier between the reads and the
 // writes of each chunk; destinations are always below every not-yet-read source, so the
-// in-place move is safe. Block i works on the page list and bitmap `i` strides on.
+// in-place move is safe.
 __global__ void __launch_bounds__(kMgrThreads) mgr_remove_kernel(Entry* entries, uint32_t* bitmap, int n, int a,
-                                                                  int b, int* err, int entry_stride, int words) {
-  entries += static_cast<size_t>(blockIdx.x) * entry_stride;
-  bitmap += static_cast<size_t>(blockIdx.x) * words;
+                                                                  int b, int* err) {
   for (int i = a + threadIdx.x; i < b; i += kMgrThreads) {
     const int page = entries[i].x;
     const uint32_t bit = 1u << (page & 31);
@@ -149,16 +147,7 @@ cudaError_t launch_mgr_alloc_layers(cudaStream_t s, Entry* entries_all, uint32_t
 
 cudaError_t launch_mgr_remove(cudaStream_t s, Entry* entries, uint32_t* bitmap, int n_entries, int a, int b,
                               int* err) {
-  mgr_remove_kernel<<<1, kMgrThreads, 0, s>>>(entries, bitmap, n_entries, a, b, err, 0, 0);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_mgr_remove_layers(cudaStream_t s, Entry* entries_all, uint32_t* bitmap_all, int words,
-                                     int pool_pages, int first_layer, int n_layers, int n_entries, int a, int b,
-                                     int* err) {
-  mgr_remove_kernel<<<n_layers, kMgrThreads, 0, s>>>(entries_all + static_cast<size_t>(first_layer) * pool_pages,
-                                                     bitmap_all + static_cast<size_t>(first_layer) * words, n_entries,
-                                                     a, b, err, pool_pages, words);
+  mgr_remove_kernel<<<1, kMgrThreads, 0, s>>>(entries, bitmap, n_entries, a, b, err);
   return cudaGetLastError();
 }
 

@@ -1,6 +1,7 @@
 // sm100_ptx.cuh -- thin inline-PTX wrappers for the sm_100a features the kernels use:
 // mbarriers with bounded waits, TMA tile loads (no multicast), tcgen05 MMA with TMEM
-// accumulators, TMEM loads/stores, and the shared-memory matrix descriptors.
+// accumulators, TMEM loads/stores, the shared-memory matrix descriptors, and the
+// thread-block-cluster barrier with stores into a peer CTA's shared memory.
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -201,6 +202,54 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
 __host__ __device__ constexpr uint32_t idesc_f16kind(uint32_t fmt, int M, int N, uint32_t a_mn, uint32_t b_mn) {
   return (1u << 4) | (fmt << 7) | (fmt << 10) | (a_mn << 15) | (b_mn << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ asynchronous copies
+// Global -> shared copies that bypass the registers; completion by commit + wait.
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* dst_smem, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ thread-block clusters
+// Every thread of every CTA of the cluster executes the arrive and the wait (.aligned):
+// a hardware barrier, nothing spins in software.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_u64(uint32_t caddr, uint64_t v) {
+  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(caddr), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_cluster_u64(uint32_t caddr) {
+  uint64_t v;
+  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(caddr) : "memory");
+  return v;
+}
+// 16-byte load; caddr must be 16-byte aligned.
+__device__ __forceinline__ void ld_cluster_v2u64(uint32_t caddr, uint64_t& a, uint64_t& b) {
+  asm volatile("ld.shared::cluster.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(caddr) : "memory");
 }
 
 }  // namespace kvc
