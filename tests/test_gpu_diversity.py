@@ -20,7 +20,8 @@ def kvc():
     return m
 
 
-def run_rolling(kvc, wl, frames, rows=None, budgets_at=None, check_ids=True, seed=11, prune_first=False):
+def run_rolling(kvc, wl, frames, rows=None, budgets_at=None, check_ids=True, seed=11, prune_first=False,
+                append_all=False):
     dev = torch.device("cuda")
     L, H, D, T = wl.num_layers, wl.num_heads, wl.head_dim, wl.tokens_per_frame
     h = kvc.kvc_create(kvc.config_from_workload(wl))
@@ -32,9 +33,13 @@ def run_rolling(kvc, wl, frames, rows=None, budgets_at=None, check_ids=True, see
             if budgets_at is not None and t in budgets_at:
                 kvc.kvc_set_layer_budgets(h, budgets_at[t])
                 orc.set_budgets(budgets_at[t])
+            qkv = [st.frame(l, t) for l in range(L)]
+            if append_all:                              # every layer's frame in one call
+                kvc.kvc_append_frame_all(h, t, [x[1] for x in qkv], [x[2] for x in qkv], True)
             for l in range(L):
-                q, k, v = st.frame(l, t)
-                kvc.kvc_append_frame(h, l, t, k, v, True)
+                q, k, v = qkv[l]
+                if not append_all:
+                    kvc.kvc_append_frame(h, l, t, k, v, True)
                 if prune_first and t > 0:
                     kvc.kvc_prune(h, l)                 # the pruning step on its own; twice prunes once
                     kvc.kvc_prune(h, l)
@@ -67,6 +72,14 @@ def test_rolling_memory_small(kvc, T, H, K, frames, prune_first):
     wl = WORKLOADS["vggt_infinite_12l"].replace(num_layers=2, tokens_per_frame=T, num_heads=H, diversity_budget=K,
                                                 num_special_tokens=min(5, T))
     run_rolling(kvc, wl, frames, prune_first=prune_first)
+
+
+def test_rolling_memory_append_all_layers(kvc):
+    """kvc_append_frame_all: one allocation and one append launch for every head of every
+    layer."""
+    wl = WORKLOADS["vggt_infinite_12l"].replace(num_layers=3, tokens_per_frame=150, num_heads=4,
+                                                diversity_budget=200)
+    run_rolling(kvc, wl, 6, append_all=True)
 
 
 def test_layer_budgets_between_frames(kvc):

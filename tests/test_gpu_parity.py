@@ -33,6 +33,7 @@ def test_tiny_f32_full_stream(kvc):
     (37, 2, 3, 1, 8, 0),        # one ragged q tile, 3 pages/frame, last page 5 valid
     (5, 2, 2, 0, 6, 0),         # T < P: every page partial
     (256, 2, 2, 1, 6, 3),       # T a multiple of the page size and of the q tile
+    (300, 4, 20, 2, 24, 16),    # 16 split CTAs per query tile merged by the last to finish
 ])
 def test_bf16_tensor_core_small(kvc, T, H, W, S, frames, splits):
     wl = WORKLOADS["vggt_518x378"].replace(tokens_per_frame=T, num_heads=H, window_frames=W, scale_frames=S,

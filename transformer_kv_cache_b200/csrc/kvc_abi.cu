@@ -35,11 +35,16 @@ cudaError_t dev_alloc_t(T** p, size_t bytes) {
   return e;
 }
 
+// Split counters of the attention kernel: one per (head, 128-row query tile).
+size_t split_cnt_count(const kvc_config& g) {
+  return static_cast<size_t>(g.num_heads) * ((g.tokens_per_frame + 127) / 128);
+}
+
 void free_all(kvc_cache* c) {
   void* ptrs[] = {c->k_pool,     c->v_pool,     c->k_scale,    c->v_scale,    c->entries,    c->bitmap,
                   c->d_err,      c->tok_id,     c->tok_cnt,    c->tok_shat,   c->cmp_scratch, c->part_o,
                   c->part_lse,   c->stage_q[0], c->stage_k[0], c->stage_v[0], c->stage_o[0], c->stage_q[1],
-                  c->stage_k[1], c->stage_v[1], c->stage_o[1], c->rank_hist, c->div_sums};
+                  c->stage_k[1], c->stage_v[1], c->stage_o[1], c->rank_hist, c->div_sums, c->split_cnt};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   for (int i = 0; i < 2; ++i) {
@@ -244,6 +249,7 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   if (c->tc_path) {
     A(dev_alloc_t(&c->part_o, c->part_rows * 128 * 64 * sizeof(float)));
     A(dev_alloc_t(&c->part_lse, c->part_rows * 128 * sizeof(float)));
+    A(dev_alloc_t(&c->split_cnt, split_cnt_count(g) * sizeof(int)));
   }
   for (int i = 0; i < 2; ++i) {
     A(dev_alloc_t(&c->stage_q[i], frame_bytes));
@@ -285,6 +291,7 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
     A(cudaMemsetAsync(c->div_sums, 0, NS * sizeof(double), c->stream));
   }
   A(cudaMemsetAsync(c->d_err, 0, 4 * sizeof(int), c->stream));
+  if (c->split_cnt) A(cudaMemsetAsync(c->split_cnt, 0, split_cnt_count(g) * sizeof(int), c->stream));
   if (g.budget_tokens > 0) {
     const size_t slots = L * c->pool_pages * P;
     A(cudaMemsetAsync(c->tok_id, 0, slots * sizeof(int64_t), c->stream));
@@ -338,6 +345,8 @@ kvc_status kvc_reset(kvc_cache* c) {
   cudaError_t e = cudaMemsetAsync(c->entries, 0, NS * c->pool_pages * sizeof(Entry), c->stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(c->bitmap, 0, NS * c->bitmap_words * sizeof(uint32_t), c->stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(c->d_err, 0, 4 * sizeof(int), c->stream);
+  if (e == cudaSuccess && c->split_cnt)   // a launch that gave up may have left a count behind
+    e = cudaMemsetAsync(c->split_cnt, 0, split_cnt_count(c->cfg) * sizeof(int), c->stream);
   if (e != cudaSuccess) return cuda_fail(c, e, "kvc_reset");
   c->L.assign(c->cfg.num_layers, LayerHost());
   c->hist_frame = -1;
@@ -351,37 +360,45 @@ kvc_status kvc_reset(kvc_cache* c) {
 // The first frame appended to a layer is the anchor; a later frame is pending until
 // kvc_attend prunes every head's candidates (kept pages + the frame's pages) to its
 // Top-K ("InfiniteVGGT" explainer, Step-by-step recipe: prune, then attend).
-kvc_status div_append(kvc_cache* c, int layer, int frame_idx, const void* k_dev, const void* v_dev) {
-  LayerHost& L = c->L[layer];
+// One frame into layers [l0, l0 + nl) (nl <= kMaxBatchLayers): one allocation launch for
+// every head of every layer, one append launch.
+kvc_status div_append_layers(kvc_cache* c, int l0, int nl, int frame_idx, const void* const* k_devs,
+                             const void* const* v_devs) {
   const kvc_config& g = c->cfg;
   const int n = c->ppf, T = g.tokens_per_frame, P = g.page_size, H = g.num_heads;
-  if (L.n_entries + n > c->pool_pages) return fail(c, KVC_ERR_STATE, "kvc_append_frame: page pool full");
+  for (int b = 0; b < nl; ++b)
+    if (c->L[l0 + b].n_entries + n > c->pool_pages) return fail(c, KVC_ERR_STATE, "kvc_append_frame: page pool full");
   LayerStarts st{};
-  st.first_layer = layer * H;
-  for (int h = 0; h < H; ++h) st.start[h] = L.n_entries;
-  cudaError_t e = launch_mgr_alloc_layers(c->stream, c->entries, c->bitmap, c->bitmap_words, c->pool_pages, st, H, n,
-                                          frame_idx, P, T - (n - 1) * P, c->d_err);
+  AppendBatch in{};
+  st.first_layer = l0 * H;
+  for (int b = 0; b < nl; ++b) {
+    st.start[b] = c->L[l0 + b].n_entries;
+    in.k[b] = k_devs[b];
+    in.v[b] = v_devs[b];
+  }
+  cudaError_t e = launch_mgr_alloc_layers(c->stream, c->entries, c->bitmap, c->bitmap_words, c->pool_pages, st,
+                                          nl * H, n, frame_idx, P, T - (n - 1) * P, c->d_err, H);
   if (e != cudaSuccess) return cuda_fail(c, e, "page allocation");
   c->launches++;
-  const size_t sub0 = static_cast<size_t>(layer) * H * c->pool_pages;   // the layer's first pool page
-  uint8_t* kp = c->k_pool + sub0 * c->page_bytes_kv;
-  uint8_t* vp = c->v_pool + sub0 * c->page_bytes_kv;
-  e = launch_append_heads(c->stream, k_dev, v_dev, kp, vp, c->entries + sub0, c->tok_id + sub0 * P, c->pool_pages,
-                          L.n_entries, n, T, H, g.head_dim, P, frame_idx);
+  e = launch_append_heads(c->stream, in, l0, st, nl, c->k_pool, c->v_pool, c->entries, c->tok_id, c->pool_pages, n, T,
+                          H, g.head_dim, P, frame_idx);
   if (e != cudaSuccess) return cuda_fail(c, e, "append");
   c->launches++;
-  if (!L.has_anchor) {
-    L.anchor_pages = n;
-    L.has_anchor = true;
-  } else {
-    L.pend_pages = n;
+  for (int b = 0; b < nl; ++b) {
+    LayerHost& L = c->L[l0 + b];
+    if (!L.has_anchor) {
+      L.anchor_pages = n;
+      L.has_anchor = true;
+    } else {
+      L.pend_pages = n;
+    }
+    L.has_pending = true;
+    L.pending_key = true;
+    L.n_entries += n;
+    L.high_water = std::max<int64_t>(L.high_water, L.n_entries);
+    L.appended++;
+    L.last_frame = frame_idx;
   }
-  L.has_pending = true;
-  L.pending_key = true;
-  L.n_entries += n;
-  L.high_water = std::max<int64_t>(L.high_water, L.n_entries);
-  L.appended++;
-  L.last_frame = frame_idx;
   return KVC_OK;
 }
 
@@ -440,6 +457,7 @@ kvc_status div_attend(kvc_cache* c, int layer, const void* q_dev, void* o_dev) {
   a.part_o = c->part_o;
   a.part_lse = c->part_lse;
   a.part_rows = c->part_rows;
+  a.split_cnt = c->split_cnt;
   a.sm_count = c->sm_count;
   a.err = c->d_err;
   a.head_pages = c->pool_pages;
@@ -465,7 +483,7 @@ kvc_status kvc_append_frame(kvc_cache* c, int32_t layer, int32_t frame_idx, cons
   if (frame_idx <= L.last_frame) return fail(c, KVC_ERR_STATE, "kvc_append_frame: frame indices must increase");
   if (c->per_head) {
     if (!is_keyframe) return fail(c, KVC_ERR_ARG, "kvc_append_frame: every frame is a candidate in this mode");
-    return div_append(c, layer, frame_idx, k_dev, v_dev);
+    return div_append_layers(c, layer, 1, frame_idx, &k_dev, &v_dev);
   }
   const kvc_config& g = c->cfg;
   const int n = c->ppf;
@@ -510,12 +528,20 @@ kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const void* con
   const kvc_config& g = c->cfg;
   if (!k_devs || !v_devs || frame_idx < 0) return fail(c, KVC_ERR_ARG, "kvc_append_frame_all: bad argument");
   if (c->per_head) {
-    // one page list per head: the layers are appended one by one (checked first)
-    for (int l = 0; l < g.num_layers; ++l)
-      if (c->L[l].has_pending || frame_idx <= c->L[l].last_frame || !k_devs[l] || !v_devs[l])
-        return fail(c, KVC_ERR_STATE, "kvc_append_frame_all: a layer cannot take the frame");
+    // one page list per head (all layers checked first)
+    if (!is_keyframe) return fail(c, KVC_ERR_ARG, "kvc_append_frame_all: every frame is a candidate in this mode");
     for (int l = 0; l < g.num_layers; ++l) {
-      kvc_status st = kvc_append_frame(c, l, frame_idx, k_devs[l], v_devs[l], is_keyframe);
+      if (!k_devs[l] || !v_devs[l] ||
+          ((reinterpret_cast<uintptr_t>(k_devs[l]) | reinterpret_cast<uintptr_t>(v_devs[l])) & 15))
+        return fail(c, KVC_ERR_ARG, "kvc_append_frame_all: K and V must be non-null and 16-byte aligned");
+      if (c->L[l].has_pending || frame_idx <= c->L[l].last_frame)
+        return fail(c, KVC_ERR_STATE, "kvc_append_frame_all: a layer cannot take the frame");
+      if (c->L[l].n_entries + c->ppf > c->pool_pages)
+        return fail(c, KVC_ERR_STATE, "kvc_append_frame_all: page pool full");
+    }
+    for (int l0 = 0; l0 < g.num_layers; l0 += kMaxBatchLayers) {
+      const int nl = std::min(kMaxBatchLayers, g.num_layers - l0);
+      kvc_status st = div_append_layers(c, l0, nl, frame_idx, k_devs + l0, v_devs + l0);
       if (st != KVC_OK) return st;
     }
     return KVC_OK;
@@ -606,6 +632,7 @@ kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_de
     a.part_o = c->part_o;
     a.part_lse = c->part_lse;
     a.part_rows = c->part_rows;
+    a.split_cnt = c->split_cnt;
     a.sm_count = c->sm_count;
     a.err = c->d_err;
     int launched = 0;

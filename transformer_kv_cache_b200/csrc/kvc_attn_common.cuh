@@ -24,6 +24,7 @@ struct TcParams {
   float* part_lse;
   int* err;
   int head_pages;               // > 0: per-head page lists (see TcAttnArgs)
+  int* split_cnt;               // [H][q_tiles] zeroed counters: the last split CTA merges (bf16 kernel)
 };
 
 __device__ __forceinline__ float ex2(float x) {

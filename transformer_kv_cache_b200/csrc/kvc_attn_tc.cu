@@ -38,7 +38,8 @@
 // P is double-buffered in TMEM so a tile's softmax never waits for the previous tile's
 // P.V product. TMEM (256 columns): S [0,64), P0 [64,96), P1 [96,128), O' [128,208),
 // Q [208,240). Two CTAs fit per SM. The KV sequence can be split across CTAs; partial outputs carry the
-// log2-sum-exp and a combine kernel merges them. Every barrier wait is bounded: on
+// log2-sum-exp, and the split CTA of a query tile that finishes last merges them (a
+// separate combine kernel does it where no split counters are given). Every barrier wait is bounded: on
 // timeout the CTA records KVC_ERR_TIMEOUT in the error word, drains its own copies and
 // MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -61,6 +62,109 @@ constexpr int kColS = 0, kColP = 64, kColO = 128, kColQ = 208;   // Q: 32 column
 constexpr float kPMax = 256.0f;               // a P above 2^8 moves the row's reference max
 constexpr size_t kSmemBytes = 1024 + 2 * kStages * kTileBytes + kOnesBytes + 256;
 }  // namespace tc
+
+// Barrier over the softmax warps only (named barrier 1; barrier 0 is __syncthreads).
+__device__ __forceinline__ void softmax_warps_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Merge one query row's split partials: O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M)
+// (M the largest lse), splits in ascending order. Partials were written by other CTAs of
+// this launch and are read through L2: half rows (32 dims) of up to four splits at a time
+// are copied (cp.async, every row's copies in flight together) into `stage`, the CTA's
+// K/V stage buffers, dead once the last P.V product has completed; with two splits both
+// halves come in one round. Each thread reads only its own row, whose eight 16-byte
+// chunks per half sit XOR-swizzled by the row so that neighbouring rows use other banks.
+__device__ __forceinline__ void merge_split_row(const TcParams& p, uint8_t* stage, int h, int qt, int r, int row) {
+  constexpr int kHalf = tc::kHD / 2;                  // dims per pass
+  constexpr int kSlot = tc::kBM * kHalf * 4;          // 16 KB: one split's half rows
+  constexpr int kSlots = 4;                           // the 64 KB of K/V stages
+  constexpr int kKeep = 8;                            // lse values kept in registers
+  const long long pi0 = static_cast<long long>(h) * p.splits * p.q_tiles + qt;
+  auto lse_at = [&](int s) { return __ldcg(p.part_lse + (pi0 + static_cast<long long>(s) * p.q_tiles) * tc::kBM + r); };
+  auto part_at = [&](int s, int half) {
+    return p.part_o + ((pi0 + static_cast<long long>(s) * p.q_tiles) * tc::kBM + r) * tc::kHD + half * kHalf;
+  };
+  // copy a half row into slot j / read chunk c of slot j
+  auto stage_in = [&](int j, const float* src) {
+    uint8_t* dst = stage + j * kSlot + r * kHalf * 4;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) cp_async16(dst + ((c ^ (r & 7)) << 4), src + 4 * c);
+  };
+  auto accumulate = [&](float (&a)[kHalf], int j, float w) {
+    const uint8_t* rowp = stage + j * kSlot + r * kHalf * 4;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float4 f = *reinterpret_cast<const float4*>(rowp + ((c ^ (r & 7)) << 4));
+      a[4 * c + 0] = fmaf(w, f.x, a[4 * c + 0]);
+      a[4 * c + 1] = fmaf(w, f.y, a[4 * c + 1]);
+      a[4 * c + 2] = fmaf(w, f.z, a[4 * c + 2]);
+      a[4 * c + 3] = fmaf(w, f.w, a[4 * c + 3]);
+    }
+  };
+  uint4* out = reinterpret_cast<uint4*>(p.out + (static_cast<long long>(row) * p.H + h) * tc::kHD);
+  auto store_half = [&](const float (&a)[kHalf], int half, float inv) {
+#pragma unroll
+    for (int v = 0; v < kHalf / 8; ++v) {
+      uint4 q;
+      q.x = pack_bf16(a[8 * v + 0] * inv, a[8 * v + 1] * inv);
+      q.y = pack_bf16(a[8 * v + 2] * inv, a[8 * v + 3] * inv);
+      q.z = pack_bf16(a[8 * v + 4] * inv, a[8 * v + 5] * inv);
+      q.w = pack_bf16(a[8 * v + 6] * inv, a[8 * v + 7] * inv);
+      out[half * (kHalf / 8) + v] = q;
+    }
+  };
+  const bool one_round = p.splits <= kSlots / 2;
+  if (one_round)                                      // both halves of every split, issued first
+    for (int s = 0; s < p.splits; ++s) {
+      stage_in(2 * s, part_at(s, 0));
+      stage_in(2 * s + 1, part_at(s, 1));
+    }
+  float lr[kKeep];
+  float M = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < kKeep; ++k) {
+    lr[k] = k < p.splits ? lse_at(k) : -INFINITY;
+    M = fmaxf(M, lr[k]);
+  }
+  for (int s = kKeep; s < p.splits; ++s) M = fmaxf(M, lse_at(s));
+  float ws = 0.f;
+#pragma unroll
+  for (int k = 0; k < kKeep; ++k)
+    if (k < p.splits) ws += exp2f(lr[k] - M);
+  for (int s = kKeep; s < p.splits; ++s) ws += exp2f(lse_at(s) - M);
+  const float inv = 1.f / ws;
+  auto weight = [&](int s) {
+    float l = 0.f;
+#pragma unroll
+    for (int k = 0; k < kKeep; ++k)
+      if (k == s) l = lr[k];
+    return exp2f((s < kKeep ? l : lse_at(s)) - M);
+  };
+  if (one_round) {
+    cp_async_wait_all();
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+      float a[kHalf];
+#pragma unroll
+      for (int k = 0; k < kHalf; ++k) a[k] = 0.f;
+      for (int s = 0; s < p.splits; ++s) accumulate(a, 2 * s + half, weight(s));
+      store_half(a, half, inv);
+    }
+    return;
+  }
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    float a[kHalf];
+#pragma unroll
+    for (int k = 0; k < kHalf; ++k) a[k] = 0.f;
+    for (int s0 = 0; s0 < p.splits; s0 += kSlots) {
+      const int ns = min(kSlots, p.splits - s0);
+      for (int j = 0; j < ns; ++j) stage_in(j, part_at(s0 + j, half));
+      cp_async_wait_all();
+      for (int j = 0; j < ns; ++j) accumulate(a, j, weight(s0 + j));
+    }
+    store_half(a, half, inv);
+  }
+}
 
 template <int P, bool kPerHead>
 __global__ void __launch_bounds__(tc::kThreads, 2)
@@ -436,6 +540,21 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
           p.part_lse[pi * kBM + r] = m + __log2f(l);
         }
       }
+      if (p.splits > 1 && p.split_cnt) {
+        // the split CTA that finishes a (query tile, head) last merges every split's
+        // partial (threadfence-then-count: each partial is visible before its count)
+        __shared__ int s_last;
+        __threadfence();
+        softmax_warps_sync();
+        if (warp == 2 && lane == 0) s_last = atomicAdd(&p.split_cnt[h * p.q_tiles + qt], 1) == p.splits - 1;
+        softmax_warps_sync();
+        if (s_last) {
+          __threadfence();
+          const int row = qt * kBM + r;
+          if (row < p.T) merge_split_row(p, k_s, h, qt, r, row);
+          if (warp == 2 && lane == 0) p.split_cnt[h * p.q_tiles + qt] = 0;   // ready for the next launch
+        }
+      }
     }
   }
   tc_fence_before();
@@ -516,12 +635,15 @@ static bool encode_q_tmap(CUtensorMap* map, const void* q, int T, int H) {
   return r == CUDA_SUCCESS;
 }
 
-// Pick the number of KV splits. Cost of a split count, in units of one KV tile of one
-// CTA: waves x (fixed cost of a CTA, about 2.5 tiles: TMEM and barrier set-up, the query
-// tile, the pipeline's fill and drain, the epilogue + tiles per CTA), plus the combine
-// pass that a split needs (about 1 + 0.5 per split). Among counts within 1% of the best
-// cost the fewest splits win (less partial traffic for the same time).
-int choose_splits(int units, int tiles, int slots) {
+// Pick the number of KV splits. Cost of a split count, in units of one KV tile of a CTA
+// that shares its SM: waves x (fixed cost of a CTA + tiles per CTA), where a CTA alone on
+// its SM (at most one per SM in the whole launch) runs a tile in about 0.84 of the time,
+// plus a cost per split (the partials written and merged). Fixed cost and split cost:
+// 8 and 2 tiles for the bf16 kernel, whose last split CTA merges (measured on 24-, 272- and
+// 1,146-tile caches); 4 and 0.25 (+ 0.5 for the combine launch) for the FP8 kernel, one CTA
+// per SM. Among counts within 1% of the best cost the fewest splits win.
+int choose_splits(int units, int tiles, int slots, bool fp8) {
+  const double cta_cost = fp8 ? 4.0 : 8.0;
   const int max_s = tiles < 64 ? tiles : 64;
   double cost[65];
   double best_cost = 1e30;
@@ -531,7 +653,9 @@ int choose_splits(int units, int tiles, int slots) {
     if ((tiles + tps - 1) / tps != s) continue;        // the same as a smaller split count
     const long long ctas = static_cast<long long>(units) * s;
     const long long waves = (ctas + slots - 1) / slots;
-    cost[s] = static_cast<double>(waves) * (2.5 + tps) + (s > 1 ? 1.0 + 0.5 * s : 0.0);
+    const double per_tile = !fp8 && 2 * ctas <= slots ? 0.84 : 1.0;
+    const double split_cost = s == 1 ? 0.0 : fp8 ? 0.5 + 0.25 * s : 2.0 * s;
+    cost[s] = static_cast<double>(waves) * (cta_cost + tps) * per_tile + split_cost;
     if (cost[s] < best_cost) best_cost = cost[s];
   }
   for (int s = 1; s <= max_s; ++s)
@@ -561,7 +685,7 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   const int units = a.fp8 ? ((q_tiles + 1) / 2) * a.H : q_tiles * a.H;
   const int slots = a.fp8 ? a.sm_count : 2 * a.sm_count;
   const int part_units = q_tiles * a.H;       // 128-row partial tiles per split
-  int splits = a.splits > 0 ? a.splits : choose_splits(units, total_tiles, slots);
+  int splits = a.splits > 0 ? a.splits : choose_splits(units, total_tiles, slots, a.fp8);
   if (splits > total_tiles) splits = total_tiles;
   int tps = (total_tiles + splits - 1) / splits;
   splits = (total_tiles + tps - 1) / tps;
@@ -592,6 +716,9 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   prm.part_lse = a.part_lse;
   prm.err = a.err;
   prm.head_pages = a.head_pages;
+  // the last split CTA merges when a merge is one copy round per half row (up to four
+  // splits); with more, a separate combine launch is faster (measured at 9 splits)
+  prm.split_cnt = a.fp8 || splits > 4 ? nullptr : a.split_cnt;
   const int grid = units * splits;
   cudaError_t e;
   if (a.fp8) {
@@ -605,7 +732,7 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   }
   if (e != cudaSuccess) return e;
   if (launched) *launched = 1;
-  if (splits > 1) {
+  if (splits > 1 && !prm.split_cnt) {
     const long long warps = static_cast<long long>(a.T) * a.H;
     const int threads = 256;
     combine_kernel<<<static_cast<int>((warps * 32 + threads - 1) / threads), threads, 0, s>>>(

@@ -29,31 +29,45 @@ namespace {
 
 constexpr int kDivD = 64;
 
-// One 16-byte chunk per thread-iteration over (head, page, slot, chunk) of one frame, for
-// K and for V; also the token ids of the frame's slots (-1 past T).
-__global__ void append_heads_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, uint4* k_pool,
-                                    uint4* v_pool, const Entry* __restrict__ entries_layer, int64_t* tok_id_layer,
-                                    int pool_pages, int start, int n_pages, int T, int H, int P, int chunks,
-                                    long long frame_base) {
-  const long long per_tensor = static_cast<long long>(H) * n_pages * P * chunks;
-  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < 2 * per_tensor;
+// One frame into the per-head pages of a batch of layers: one thread per (layer, slot,
+// head) row of 64 dims, heads fastest (the source rows of a slot are contiguous). A slot
+// past T gets zeros and token id -1. The page-table entries [start, start + n_pages) of
+// every head were just written by the allocator.
+__global__ void __launch_bounds__(256) append_heads_kernel(AppendBatch in, int first_layer, LayerStarts starts,
+                                                           int n_layers, uint4* k_pool, uint4* v_pool,
+                                                           const Entry* __restrict__ entries_all,
+                                                           int64_t* tok_id_all, int pool_pages, int n_pages, int T,
+                                                           int H, int P, long long frame_base) {
+  const int slots = n_pages * P;
+  const long long total = static_cast<long long>(n_layers) * slots * H;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const bool is_v = idx >= per_tensor;
-    long long r = is_v ? idx - per_tensor : idx;
-    const int c = static_cast<int>(r % chunks);
-    r /= chunks;
-    const int slot = static_cast<int>(r % P);
-    r /= P;
-    const int g = static_cast<int>(r % n_pages);
-    const int h = static_cast<int>(r / n_pages);
-    const long long sub = static_cast<long long>(h) * pool_pages;
-    const int phys = __ldg(&entries_layer[sub + start + g].x);
-    const int tok = g * P + slot;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (tok < T) val = __ldg(&(is_v ? v : k)[(static_cast<long long>(tok) * H + h) * chunks + c]);
-    const long long dst = ((sub + phys) * P + slot) * chunks + c;
-    (is_v ? v_pool : k_pool)[dst] = val;
-    if (!is_v && c == 0) tok_id_layer[(sub + phys) * P + slot] = tok < T ? frame_base + tok : -1;
+    const int h = static_cast<int>(idx % H);
+    const long long rt = idx / H;
+    const int t = static_cast<int>(rt % slots);
+    const int b = static_cast<int>(rt / slots);
+    const long long sub = (static_cast<long long>(first_layer + b) * H + h) * pool_pages;
+    const int phys = __ldg(&entries_all[sub + starts.start[b] + t / P].x);
+    const long long dst = ((sub + phys) * P + t % P) * (kDivD / 8);
+    uint4 kv[2][kDivD / 8];
+    if (t < T) {
+      const uint4* ks = static_cast<const uint4*>(in.k[b]) + (static_cast<long long>(t) * H + h) * (kDivD / 8);
+      const uint4* vs = static_cast<const uint4*>(in.v[b]) + (static_cast<long long>(t) * H + h) * (kDivD / 8);
+#pragma unroll
+      for (int q = 0; q < kDivD / 8; ++q) {
+        kv[0][q] = __ldg(ks + q);
+        kv[1][q] = __ldg(vs + q);
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < kDivD / 8; ++q) kv[0][q] = kv[1][q] = make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int q = 0; q < kDivD / 8; ++q) {
+      k_pool[dst + q] = kv[0][q];
+      v_pool[dst + q] = kv[1][q];
+    }
+    tok_id_all[(sub + phys) * P + t % P] = t < T ? frame_base + t : -1;
   }
 }
 
@@ -511,18 +525,18 @@ __global__ void __cluster_dims__(kPruneCluster, 1, 1) __launch_bounds__(kPruneTh
 
 }  // namespace
 
-cudaError_t launch_append_heads(cudaStream_t s, const void* k, const void* v, void* k_pool, void* v_pool,
-                                const Entry* entries_layer, int64_t* tok_id_layer, int pool_pages, int start,
-                                int n_pages, int T, int H, int D, int P, int frame) {
-  const int chunks = D * 2 / 16;
-  const long long total = 2LL * H * n_pages * P * chunks;
+cudaError_t launch_append_heads(cudaStream_t s, const AppendBatch& in, int first_layer, const LayerStarts& starts,
+                                int n_layers, void* k_pool, void* v_pool, const Entry* entries_all,
+                                int64_t* tok_id_all, int pool_pages, int n_pages, int T, int H, int D, int P,
+                                int frame) {
+  if (D != kDivD) return cudaErrorInvalidValue;
+  const long long total = static_cast<long long>(n_layers) * n_pages * P * H;
   const int threads = 256;
   long long blocks = (total + threads - 1) / threads;
-  if (blocks > 148 * 8) blocks = 148 * 8;
+  if (blocks > 148 * 16) blocks = 148 * 16;
   append_heads_kernel<<<static_cast<int>(blocks), threads, 0, s>>>(
-      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_pool),
-      static_cast<uint4*>(v_pool), entries_layer, tok_id_layer, pool_pages, start, n_pages, T, H, P, chunks,
-      static_cast<long long>(frame) * T);
+      in, first_layer, starts, n_layers, static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), entries_all,
+      tok_id_all, pool_pages, n_pages, T, H, P, static_cast<long long>(frame) * T);
   return cudaGetLastError();
 }
 

@@ -77,6 +77,7 @@ struct Cache {
   // attention split scratch (partial O and log-sum-exp)
   float* part_o = nullptr;
   float* part_lse = nullptr;
+  int* split_cnt = nullptr;         // [H][q_tiles] attention split counters (zero between launches)
   size_t part_rows = 0;             // capacity in 128-row partial tiles
   // host-buffer steps: two staging slots so that one step's copies overlap another's
   // compute; uploads and downloads run on their own streams, ordered by events
@@ -130,8 +131,8 @@ struct AppendBatch {
 cudaError_t launch_mgr_alloc(cudaStream_t s, Entry* entries, uint32_t* bitmap, int words, int pool_pages,
                              int start, int n_new, int owner, int valid_full, int valid_last, int* err);
 cudaError_t launch_mgr_alloc_layers(cudaStream_t s, Entry* entries_all, uint32_t* bitmap_all, int words,
-                                    int pool_pages, const LayerStarts& starts, int n_layers, int n_new, int owner,
-                                    int valid_full, int valid_last, int* err);
+                                    int pool_pages, const LayerStarts& starts, int n_lists, int n_new, int owner,
+                                    int valid_full, int valid_last, int* err, int group = 1);
 cudaError_t launch_mgr_remove(cudaStream_t s, Entry* entries, uint32_t* bitmap, int n_entries, int a, int b,
                               int* err);
 cudaError_t launch_debug_wait(cudaStream_t s, int* flag, int* err, long long timeout_ns);
@@ -181,10 +182,12 @@ struct TcAttnArgs {
   int head_pages;                   // > 0: one page list per head, head h's pages at
                                     // entries + h * head_pages, pool page index page_base +
                                     // h * head_pages + phys (single-head pages)
+  int* split_cnt = nullptr;         // [H][q_tiles] zeroed counters (bf16 kernel): the last
+                                    // split CTA of a query tile merges, no combine launch
 };
 // Returns the number of kernels launched through *launched.
 cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used, int* launched);
-int choose_splits(int units, int tiles, int slots);
+int choose_splits(int units, int tiles, int slots, bool fp8);
 
 // Tensor map for a pool: rows of D elements, box of P rows.
 bool encode_pool_tmap(CUtensorMap* map, void* base, size_t rows, int D, int P, int elem_bytes, bool swizzle128);
@@ -197,9 +200,10 @@ cudaError_t launch_merge_targets(cudaStream_t s, const __nv_bfloat16* ks, const 
                                  int32_t* target, int* err, int* launched);
 
 // Rolling diversity-pruned memory (kvc_diversity.cu).
-cudaError_t launch_append_heads(cudaStream_t s, const void* k, const void* v, void* k_pool, void* v_pool,
-                                const Entry* entries_layer, int64_t* tok_id_layer, int pool_pages, int start,
-                                int n_pages, int T, int H, int D, int P, int frame);
+cudaError_t launch_append_heads(cudaStream_t s, const AppendBatch& in, int first_layer, const LayerStarts& starts,
+                                int n_layers, void* k_pool, void* v_pool, const Entry* entries_all,
+                                int64_t* tok_id_all, int pool_pages, int n_pages, int T, int H, int D, int P,
+                                int frame);
 int diversity_prune_max_candidates();
 cudaError_t launch_diversity_prune(cudaStream_t s, Entry* entries_layer, void* k_pool, void* v_pool,
                                    uint32_t* bitmap_layer, int words, int64_t* tok_id_layer, int pool_pages,

@@ -44,16 +44,18 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
 // Allocate the n_new lowest free pages of a pool and write page-table entries
 // [start, start + n_new): (phys, owner, index, valid), valid = valid_full except the
 // last page, which gets valid_last. Pages are marked used in the bitmap.
-// One CTA per layer of a batch: layer (first_layer + blockIdx.x) of the pools starting at
-// `entries` / `bitmap` (strides pool_pages entries and `words` bitmap words per layer).
+// One CTA per page list of a batch: list (first_layer + blockIdx.x) of the pools starting
+// at `entries` / `bitmap` (strides pool_pages entries and `words` bitmap words per list);
+// `group` consecutive lists share one start (the heads of a layer with per-head lists).
 __global__ void __launch_bounds__(kMgrThreads) mgr_alloc_kernel(Entry* entries_all, uint32_t* bitmap_all, int words,
-                                                                 int pool_pages, LayerStarts starts, int n_new,
-                                                                 int owner, int valid_full, int valid_last, int* err) {
+                                                                 int pool_pages, LayerStarts starts, int group,
+                                                                 int n_new, int owner, int valid_full, int valid_last,
+                                                                 int* err) {
   __shared__ int s_warp[32];
   const int layer = starts.first_layer + blockIdx.x;
   Entry* entries = entries_all + static_cast<size_t>(layer) * pool_pages;
   uint32_t* bitmap = bitmap_all + static_cast<size_t>(layer) * words;
-  const int start = starts.start[blockIdx.x];
+  const int start = starts.start[blockIdx.x / group];
   int found = 0;
   for (int chunk = 0; chunk < words && found < n_new; chunk += kMgrThreads) {
     const int w = chunk + threadIdx.x;
@@ -132,16 +134,16 @@ cudaError_t launch_mgr_alloc(cudaStream_t s, Entry* entries, uint32_t* bitmap, i
   LayerStarts st{};
   st.first_layer = 0;
   st.start[0] = start;
-  mgr_alloc_kernel<<<1, kMgrThreads, 0, s>>>(entries, bitmap, words, pool_pages, st, n_new, owner, valid_full,
+  mgr_alloc_kernel<<<1, kMgrThreads, 0, s>>>(entries, bitmap, words, pool_pages, st, 1, n_new, owner, valid_full,
                                              valid_last, err);
   return cudaGetLastError();
 }
 
 cudaError_t launch_mgr_alloc_layers(cudaStream_t s, Entry* entries_all, uint32_t* bitmap_all, int words,
-                                    int pool_pages, const LayerStarts& starts, int n_layers, int n_new, int owner,
-                                    int valid_full, int valid_last, int* err) {
-  mgr_alloc_kernel<<<n_layers, kMgrThreads, 0, s>>>(entries_all, bitmap_all, words, pool_pages, starts, n_new, owner,
-                                                    valid_full, valid_last, err);
+                                    int pool_pages, const LayerStarts& starts, int n_lists, int n_new, int owner,
+                                    int valid_full, int valid_last, int* err, int group) {
+  mgr_alloc_kernel<<<n_lists, kMgrThreads, 0, s>>>(entries_all, bitmap_all, words, pool_pages, starts, group, n_new,
+                                                   owner, valid_full, valid_last, err);
   return cudaGetLastError();
 }
 
