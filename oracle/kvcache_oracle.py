@@ -23,6 +23,11 @@ What it follows (the web pages are cited by title and section):
 * Keyframe skip-append -- GCTStream page, Selective Frame Caching with Skip Append
   and Frame-by-Frame Causal Processing: a non-keyframe attends, then its K/V are
   discarded.
+* Joint scale-frame phase -- GCTStream page, Scale-Frame Phase and the FAQ on the two
+  phases: the first frames are processed together with bidirectional attention and
+  share cache entries; the causal frame-by-frame phase follows.
+* Cross-frame special tokens -- GCTStream page, Special Token Persistence: special
+  tokens (camera / register) stay cached when their frame's other K/V are evicted.
 * Reset -- GCTStream page, Cache Initialization and Cleanup.
 * Cross-layer consistency scoring (CLCES) -- StreamCacheVGGT page, sections
   2.1.1 to 2.1.4: raw score = L2 norm of the FFN residual, ranks 0..N-1 over a
@@ -43,7 +48,14 @@ notes): the order append -> attend -> commit/evict; lowest-free page allocation;
 population variance; the fp64 evaluation order of the score; ties broken by the
 lower token id; protected tokens never absorb merges; merges applied
 simultaneously from pre-merge values in ascending source id and rounded once to
-bf16; the FP8 scale fp32(amax / 448) and codes RNE-satfinite of fp32(x / scale).
+bf16; the FP8 scale fp32(amax / 448) and codes RNE-satfinite of fp32(x / scale);
+the joint phase appends its n <= S frames first, then all n*T queries attend over
+all of them (no mask), then the n frames are committed; a frame's special tokens
+are its first num_special_tokens tokens, and when a committed frame is evicted its
+first ceil(ns / P) pages stay where they are in the page table, trimmed to those
+tokens (other slots zero, page valid counts ns, P, ...), for at most
+special_frames evicted frames, the oldest dropped first beyond that; a
+non-keyframe is discarded whole.
 
 Nothing here is pinned only to itself: tests/test_oracle_*.py check it against
 brute force over explicitly concatenated frames, closed forms, library routines
@@ -165,6 +177,7 @@ class OracleConfig:
     rank_window: int = 5
     residual_dim: int = 1024
     protect_first_frame: int = 1
+    special_frames: int = 0       # evicted frames whose special tokens stay (0: off)
 
     @staticmethod
     def from_workload(wl) -> "OracleConfig":
@@ -174,7 +187,8 @@ class OracleConfig:
             page_size=wl.page_size, window_frames=wl.window_frames, scale_frames=wl.scale_frames,
             kv_dtype=wl.kv_dtype, softmax_scale=wl.softmax_scale, budget_tokens=wl.budget_tokens,
             keep_frac=wl.keep_frac, lam=wl.lam, rank_window=wl.rank_window,
-            residual_dim=wl.residual_dim, protect_first_frame=wl.protect_first_frame)
+            residual_dim=wl.residual_dim, protect_first_frame=wl.protect_first_frame,
+            special_frames=getattr(wl, "special_frames", 0))
 
 
 class _Page:
@@ -200,6 +214,7 @@ class _LayerState:
         # page table entries in cache order: [phys, owner, page_in_owner, valid]
         self.entries: List[List[int]] = []
         self.committed: List[int] = []        # committed frame ids in commit order
+        self.retained: List[int] = []         # evicted frames whose special tokens stay
         self.pending: Optional[int] = None    # frame id appended but not yet committed
         self.pending_key: bool = False
         self.high_water = 0
@@ -341,13 +356,85 @@ class StreamOracle:
                 evict = [f for f in L.committed if f not in keep]
                 if evict:
                     ev = set(evict)
+                    L.committed = [f for f in L.committed if f not in ev]
+                    if cfg.special_frames > 0:
+                        for f in evict:
+                            self._retain_special(L, f)
+                        ev = set(evict) - set(L.retained)
                     self._free(L, [e[0] for e in L.entries if e[1] in ev])
                     L.entries = [e for e in L.entries if e[1] not in ev]
-                    L.committed = [f for f in L.committed if f not in ev]
         else:
             self._free(L, [e[0] for e in L.entries if e[1] == t])
             L.entries = [e for e in L.entries if e[1] != t]
         L.pending = None
+
+    def _retain_special(self, L: _LayerState, f: int):
+        """Evicted frame f keeps its first ceil(ns / P) pages, trimmed to its special
+        tokens (slots past them zeroed); its other pages are freed. Beyond special_frames
+        retained frames the oldest is dropped whole."""
+        cfg, P = self.cfg, self.P
+        ns = min(cfg.num_special_tokens, self.T)
+        keep_pages = -(-ns // P)
+        drop = []
+        for e in L.entries:
+            if e[1] != f:
+                continue
+            if e[2] < keep_pages:
+                n = min(P, ns - e[2] * P)
+                pg = L.pages[e[0]]
+                pg.k[:, n:] = 0.0
+                pg.v[:, n:] = 0.0
+                if pg.k_codes is not None:
+                    pg.k_codes[:, n:] = 0
+                    pg.v_codes[:, n:] = 0
+                pg.ids[n:] = -1
+                pg.counts[n:] = 0
+                pg.valid = n
+                e[3] = n
+            else:
+                drop.append(e[0])
+        self._free(L, drop)
+        L.entries = [e for e in L.entries if not (e[1] == f and e[2] >= keep_pages)]
+        L.retained.append(f)
+        while len(L.retained) > cfg.special_frames:
+            old = L.retained.pop(0)
+            self._free(L, [e[0] for e in L.entries if e[1] == old])
+            L.entries = [e for e in L.entries if e[1] != old]
+
+    # ---------------------------------------------------------------- joint scale-frame phase
+    def scale_phase(self, layer: int, n: int, Q: np.ndarray, K: np.ndarray, V: np.ndarray,
+                    rows: Optional[Sequence[int]] = None) -> np.ndarray:
+        """The first n frames together: Q, K, V are [n*T, H, D] (frame-major). Frames
+        0..n-1 are appended and committed, then all n*T queries attend over all of them
+        with no mask. Returns fp64 [len(rows), H, D]."""
+        L = self.layers[layer]
+        if L.entries or L.committed or L.pending is not None:
+            raise RuntimeError("the joint phase starts an empty layer")
+        if not 1 <= n <= max(1, self.cfg.scale_frames):
+            raise ValueError("the joint phase takes 1..scale_frames frames")
+        T = self.T
+        K = np.asarray(K, np.float64)
+        V = np.asarray(V, np.float64)
+        for f in range(n):
+            self.append(layer, f, K[f * T:(f + 1) * T], V[f * T:(f + 1) * T], True)
+            self.commit(layer)
+        return self.attend_cache(layer, Q, rows)
+
+    def attend_cache(self, layer: int, Q: np.ndarray, rows: Optional[Sequence[int]] = None) -> np.ndarray:
+        """Attention of any number of queries over every cached token, nothing changed."""
+        Q = np.asarray(Q, np.float64)
+        if rows is not None:
+            Q = Q[np.asarray(rows)]
+        Kc, Vc, _ = self.gather(layer)
+        H = self.cfg.num_heads
+        out = np.empty((Q.shape[0], H, self.cfg.head_dim))
+        for h in range(H):
+            z = self.scale * (Q[:, h, :] @ Kc[:, h, :].T)
+            z = z - z.max(axis=1, keepdims=True)
+            p = np.exp(z)
+            p /= p.sum(axis=1, keepdims=True)
+            out[:, h, :] = p @ Vc[:, h, :]
+        return out
 
     # ---------------------------------------------------------------- reset
     def reset(self):
