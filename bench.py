@@ -57,7 +57,7 @@ def parse():
     ap.add_argument("--kv-splits", type=int, default=0)
     ap.add_argument("--workload", default=WORKLOAD,
                     help="vggt_518x378 (default, the headline), vggt_24layer_k4, vggt_budget_16k, vggt_518x518_fp8, "
-                         "vggt_infinite_12l")
+                         "vggt_infinite_12l, vggt_518x378_joint, vggt_518x378_special")
     ap.add_argument("--fill", type=int, default=0,
                     help="frames streamed before warm-up for a non-default workload (0: enough to fill the window); "
                          "smaller values give short cases for profiling")
@@ -434,6 +434,8 @@ def run_workload(args):
         fill = 3                                      # anchor, then two prunings: the kept sets are full
     elif budget:
         fill = -(-wl.budget_tokens // T) + 3          # past the first compression of every layer
+    elif wl.special_frames > 0:                       # the window is full and 128 frames have
+        fill = S + W * k + min(wl.special_frames, 128)   # left it, keeping their special tokens
     else:
         fill = S + W * k                              # the window is full of keyframes
     warm, steps = args.warmup, args.steps
@@ -506,6 +508,7 @@ def run_workload(args):
             "config": {"workload": wl.name, "layers": L, "tokens_per_frame": T, "heads": H, "head_dim": D,
                        "page_size": P, "window_frames": W, "scale_frames": S, "keyframe_interval": k,
                        "budget_tokens": wl.budget_tokens, "diversity_budget": wl.diversity_budget,
+                       "special_frames": wl.special_frames, "kv_tokens_attended": info0["tokens"] + T,
                        "inputs": (f"{distinct} distinct seeded frames per layer" if rolling else
                                   f"{distinct} seeded frames per layer, cycled"),
                        "keyframes_timed": keys, "compressions_timed": fires},
@@ -547,6 +550,70 @@ def run_workload(args):
     return 0
 
 
+def run_joint(args):
+    """The joint scale-frame phase: a step is kvc_reset (a new stream) followed by
+    kvc_scale_phase of the stream's first joint_frames frames on every layer; the metric
+    counts those frames. Inputs are resident in HBM."""
+    import torch
+    import transformer_kv_cache_b200 as kvc
+    from kvc_streams import WORKLOADS, FrameStream
+
+    wl = WORKLOADS[args.workload]
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device=dev)
+    peaks, peak_kind = load_peaks()
+    L, T, H, D, n = wl.num_layers, wl.tokens_per_frame, wl.num_heads, wl.head_dim, wl.joint_frames
+    warm, steps = args.warmup, args.steps
+    with torch.cuda.stream(stream):
+        st = FrameStream(wl, seed=2000, device=dev)
+        qkv = []
+        for l in range(L):
+            fr = [st.frame(l, t) for t in range(n)]
+            qkv.append(tuple(torch.cat([x[i] for x in fr]) for i in range(3)))
+        out = torch.empty((n * T, H, D), dtype=torch.bfloat16, device=dev)
+        h = kvc.kvc_create(kvc.config_from_workload(wl, kv_splits=args.kv_splits), stream)
+
+        def step(ev=None):
+            if ev: ev[0].record(stream)
+            kvc.kvc_reset(h)
+            if ev: ev[1].record(stream)
+            for l in range(L):
+                kvc.kvc_scale_phase(h, l, n, qkv[l][0], qkv[l][1], qkv[l][2], out)
+            if ev: ev[2].record(stream)
+
+        for _ in range(warm):
+            step()
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        with ClockSampler(local) as clk:
+            for i in range(steps):
+                step(evs[i])
+            stream.synchronize()
+        _, info = kvc.kvc_page_table(h, 0)
+        assert info["device_error"] == 0
+        kvc.kvc_destroy(h)
+    tot = statistics.mean(evs[i][0].elapsed_time(evs[i][2]) for i in range(steps))
+    ph = statistics.mean(evs[i][1].elapsed_time(evs[i][2]) for i in range(steps))
+    flops = 4.0 * (n * T) ** 2 * H * D * L
+    ach = flops / (ph * 1e-3) / 1e12
+    line = {"metric": METRIC, "value": n * 1e3 / tot, "unit": UNIT, "n_gpus": 1, "steps": steps, "warmup": warm,
+            "ms_per_step": tot, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "layers": L, "tokens_per_frame": T, "heads": H, "head_dim": D,
+                       "joint_frames": n, "queries": n * T, "keys": n * T,
+                       "step": "kvc_reset, then the joint phase of every layer"},
+            "clocks": clk.summary(),
+            "kernels": {"reset_ms": tot - ph, "joint_phase_ms": ph},
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
+                         "frac": ach / float(peaks["bf16_tflops"]), "traffic": None,
+                         "kernel": "attention of the joint phase (append of the frames included)",
+                         "flops_per_launch": flops / L, "peak_source": peak_kind}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if os.environ.get("KVC_BENCH_WATCHDOG"):
@@ -555,6 +622,9 @@ def main():
     if args.impl == "reference":
         return run_reference(args)
     if args.workload != WORKLOAD:
+        from kvc_streams import WORKLOADS
+        if WORKLOADS[args.workload].joint_frames > 0:
+            return run_joint(args)
         return run_workload(args)
     return run_ours(args)
 

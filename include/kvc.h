@@ -102,7 +102,9 @@ typedef struct {
   int32_t kv_splits;            /* KV splits per query tile in attention; 0 = automatic */
   int32_t diversity_budget;     /* K > 0: rolling diversity-pruned memory, K kept tokens per
                                    head per layer besides the first frame (see kvc_attend) */
-  int32_t reserved[6];          /* must be zero */
+  int32_t special_frames;       /* > 0 (window mode only): cross-frame special tokens, see
+                                   kvc_attend; the evicted frames whose special tokens stay */
+  int32_t reserved[5];          /* must be zero */
 } kvc_config;
 
 /* Cache statistics ([GCT] Cache Monitoring: occupancy, memory use, eviction status). */
@@ -170,9 +172,25 @@ KVC_API kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const v
  * ([GCT] Frame-by-Frame Causal Processing; [IVG] Causal Attention). Then the
  * pending frame is committed (keyframe; frames outside the first S and last W
  * committed are evicted and their pages freed) or released (non-keyframe).
+ * With special_frames > 0 an evicted frame keeps its special tokens ([GCT] Special
+ * Token Persistence): its first ceil(num_special_tokens / P) pages stay in the page
+ * table, trimmed to those tokens (other slots zeroed), and later frames attend to them;
+ * beyond special_frames such frames the oldest one's pages are freed. A non-keyframe
+ * keeps nothing.
  * bf16 with D = 64 runs on tcgen05 tensor cores (fp32 accumulation); fp32 I/O
  * runs fp32 FMA arithmetic. Errors: KVC_ERR_STATE if nothing is pending. */
 KVC_API kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_dev);
+
+/* The joint scale-frame phase ([GCT] Scale-Frame Phase): the first n_frames frames of a
+ * stream, processed together with bidirectional attention. q_dev, k_dev, v_dev and o_dev
+ * are [n_frames * T, H, D] (frame-major, io dtype). Frames 0 .. n_frames-1 are appended
+ * and committed (as kvc_append_frame with is_keyframe = 1), then all n_frames * T
+ * queries attend over all of their tokens with no mask; the causal frame-by-frame phase
+ * continues with frame n_frames. 1 <= n_frames <= max(1, scale_frames). Errors:
+ * KVC_ERR_ARG (pointers, alignment, frame count), KVC_ERR_STATE (the layer is not empty,
+ * a token budget or per-head page lists). */
+KVC_API kvc_status kvc_scale_phase(kvc_cache* c, int32_t layer, int32_t n_frames, const void* q_dev,
+                                   const void* k_dev, const void* v_dev, void* o_dev);
 
 /* Importance scoring and, when the committed cache of `layer` holds more than
  * B tokens, keep/merge/drop compression ([SCV] 2.1.1-2.1.4, 2). Must follow

@@ -61,6 +61,8 @@ class Workload:
     residual_dim: int = 1024
     protect_first_frame: int = 1
     diversity_budget: int = 0
+    special_frames: int = 0      # evicted frames whose special tokens stay cached (0: off)
+    joint_frames: int = 0        # > 0: the stream opens with a joint phase of this many frames
     description: str = ""
 
     def as_dict(self) -> Dict:
@@ -104,6 +106,19 @@ WORKLOADS: Dict[str, Workload] = {
         keyframe_interval=1, num_frames=10000, io_dtype="bf16", kv_dtype="fp8_e4m3",
         softmax_scale=0.125, temporal_keys=False, outlier_fraction=0.01,
         description="518x518 frames, 1374 tok/frame, W=128, S=8, FP8 E4M3 K/V, 10000 frames"),
+    "vggt_518x378_joint": Workload(
+        name="vggt_518x378_joint", num_layers=1, num_heads=16, head_dim=64, tokens_per_frame=1004,
+        num_special_tokens=5, page_size=16, window_frames=64, scale_frames=8,
+        keyframe_interval=1, num_frames=8, io_dtype="bf16", kv_dtype="bf16",
+        softmax_scale=0.125, temporal_keys=True, joint_frames=8,
+        description="joint scale-frame phase: the first 8 frames of a 518x378 stream together, "
+                    "8,032 queries over 8,032 keys per head"),
+    "vggt_518x378_special": Workload(
+        name="vggt_518x378_special", num_layers=1, num_heads=16, head_dim=64, tokens_per_frame=1004,
+        num_special_tokens=5, page_size=16, window_frames=64, scale_frames=8,
+        keyframe_interval=1, num_frames=10000, io_dtype="bf16", kv_dtype="bf16",
+        softmax_scale=0.125, temporal_keys=True, special_frames=4096,
+        description="518x378 stream keeping the 5 special tokens of up to 4,096 evicted frames"),
     "vggt_infinite_12l": Workload(
         name="vggt_infinite_12l", num_layers=12, num_heads=16, head_dim=64, tokens_per_frame=1004,
         num_special_tokens=5, page_size=16, window_frames=0, scale_frames=0,

@@ -47,10 +47,12 @@ def compare_out(got: np.ndarray, ref: np.ndarray, io_dtype: str, what: str = "")
 
 
 def run_parity(kvc, wl, frames, *, check_frames=None, rows=None, seed=0, layers=None, kv_splits=0,
-               check_pages=False, record=None, batched_append=False, transform=None):
+               check_pages=False, record=None, batched_append=False, transform=None, joint=0, joint_rows=None):
     """Stream `frames` frames through the library and the oracle; compare page tables at
     every step and outputs on `check_frames` (all if None) for `rows` (all if None).
-    `transform(t, layer, q, k, v) -> (q, k, v)` edits a frame's inputs for both sides."""
+    `transform(t, layer, q, k, v) -> (q, k, v)` edits a frame's inputs for both sides.
+    `joint` = n > 0 runs frames 0..n-1 as the joint scale-frame phase first (its output
+    compared on `joint_rows`, all if None), then the stream continues causally."""
     dev = torch.device("cuda")
     cfg = kvc.config_from_workload(wl, kv_splits=kv_splits)
     h = kvc.kvc_create(cfg)
@@ -61,7 +63,20 @@ def run_parity(kvc, wl, frames, *, check_frames=None, rows=None, seed=0, layers=
         T, H, D = wl.tokens_per_frame, wl.num_heads, wl.head_dim
         out = torch.empty((T, H, D), dtype=q_dtype(wl), device=dev)
         stats = []
-        for t in range(frames):
+        if joint:
+            oj = torch.empty((joint * T, H, D), dtype=q_dtype(wl), device=dev)
+            for l in layers:
+                fr = [st.frame(l, t) for t in range(joint)]
+                Q, K, V = (torch.cat([x[i] for x in fr]) for i in range(3))
+                kvc.kvc_scale_phase(h, l, joint, Q, K, V, oj)
+                ref = orc.scale_phase(l, joint, np64(Q), np64(K), np64(V), rows=joint_rows)
+                torch.cuda.synchronize()
+                got = np64(oj) if joint_rows is None else np64(oj)[joint_rows]
+                stats.append((-1, l) + compare_out(got, ref, wl.io_dtype, f"joint phase layer {l}"))
+                pt, info = kvc.kvc_page_table(h, l)
+                assert np.array_equal(pt, orc.page_table(l)), f"page table differs after the joint phase, layer {l}"
+                assert info["device_error"] == 0
+        for t in range(joint, frames):
             key = keyframe_schedule(t, wl.scale_frames, wl.keyframe_interval)
             qkv = {l: st.frame(l, t) for l in layers}
             if transform is not None:

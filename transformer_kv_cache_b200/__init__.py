@@ -29,7 +29,7 @@ EXPORTS = ["kvc_create", "kvc_destroy", "kvc_set_stream", "kvc_reset", "kvc_appe
            "kvc_step_host", "kvc_synchronize", "kvc_last_error", "kvc_status_string", "kvc_version",
            "kvc_debug_fail_allocs", "kvc_debug_bounded_wait", "kvc_attend_paged_noalloc", "kvc_append_frame_all",
            "kvc_step_host_async", "kvc_set_layer_budgets", "kvc_prune", "kvc_layer_diversity",
-           "kvc_head_tokens"]
+           "kvc_head_tokens", "kvc_scale_phase"]
 
 
 class kvc_config(ctypes.Structure):
@@ -41,7 +41,7 @@ class kvc_config(ctypes.Structure):
                 ("rank_window", ctypes.c_int32), ("residual_dim", ctypes.c_int32),
                 ("protect_first_frame", ctypes.c_int32), ("max_frames", ctypes.c_int32),
                 ("kv_splits", ctypes.c_int32), ("diversity_budget", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 6)]
+                ("special_frames", ctypes.c_int32), ("reserved", ctypes.c_int32 * 5)]
 
 
 class kvc_info(ctypes.Structure):
@@ -84,6 +84,7 @@ def _load():
         "kvc_step_host_async": ([vp, i32, i32, i32, vp, vp, vp, vp], i32),
         "kvc_set_layer_budgets": ([vp, vp, i32], i32),
         "kvc_prune": ([vp, i32], i32),
+        "kvc_scale_phase": ([vp, i32, i32, vp, vp, vp, vp], i32),
         "kvc_layer_diversity": ([vp, i32, vp], i32),
         "kvc_head_tokens": ([vp, i32, i32, vp, i32, vp], i32),
         "kvc_synchronize": ([vp], i32),
@@ -134,7 +135,8 @@ def _check(handle, st: int):
 def make_config(num_layers, num_heads, head_dim, tokens_per_frame, num_special_tokens, page_size,
                 window_frames, scale_frames, io_dtype="bf16", kv_dtype="bf16", softmax_scale=0.125,
                 budget_tokens=0, keep_frac=0.6, lam=0.5, rank_window=5, residual_dim=1024,
-                protect_first_frame=1, max_frames=0, kv_splits=0, diversity_budget=0) -> kvc_config:
+                protect_first_frame=1, max_frames=0, kv_splits=0, diversity_budget=0,
+                special_frames=0) -> kvc_config:
     c = kvc_config()
     c.num_layers, c.num_heads, c.head_dim = num_layers, num_heads, head_dim
     c.tokens_per_frame, c.num_special_tokens, c.page_size = tokens_per_frame, num_special_tokens, page_size
@@ -146,6 +148,7 @@ def make_config(num_layers, num_heads, head_dim, tokens_per_frame, num_special_t
     c.rank_window, c.residual_dim, c.protect_first_frame = rank_window, residual_dim, protect_first_frame
     c.max_frames, c.kv_splits = max_frames, kv_splits
     c.diversity_budget = diversity_budget
+    c.special_frames = special_frames
     return c
 
 
@@ -156,7 +159,8 @@ def config_from_workload(wl, **over) -> kvc_config:
              io_dtype=wl.io_dtype, kv_dtype=wl.kv_dtype, softmax_scale=wl.softmax_scale,
              budget_tokens=wl.budget_tokens, keep_frac=wl.keep_frac, lam=wl.lam, rank_window=wl.rank_window,
              residual_dim=wl.residual_dim, protect_first_frame=wl.protect_first_frame,
-             diversity_budget=getattr(wl, "diversity_budget", 0))
+             diversity_budget=getattr(wl, "diversity_budget", 0),
+             special_frames=getattr(wl, "special_frames", 0))
     d.update(over)
     return make_config(**d)
 
@@ -272,6 +276,12 @@ def kvc_step_host_async(handle, layer: int, frame_idx: int, is_keyframe: bool, q
 def kvc_set_layer_budgets(handle, budgets) -> None:
     arr = (ctypes.c_int32 * len(budgets))(*[int(b) for b in budgets])
     _check(handle, _lib.kvc_set_layer_budgets(handle, arr, len(budgets)))
+
+
+def kvc_scale_phase(handle, layer: int, n_frames: int, q, k, v, o) -> None:
+    """The joint scale-frame phase: frames 0..n_frames-1 ([n_frames*T, H, D] tensors)
+    appended, committed, and attended bidirectionally."""
+    _check(handle, _lib.kvc_scale_phase(handle, layer, n_frames, _ptr(q), _ptr(k), _ptr(v), _ptr(o)))
 
 
 def kvc_prune(handle, layer: int) -> None:

@@ -36,8 +36,11 @@ cudaError_t dev_alloc_t(T** p, size_t bytes) {
 }
 
 // Split counters of the attention kernel: one per (head, 128-row query tile).
+// Split counters of the attention kernel: one per (head, 128-row query tile), for the
+// largest query count (a frame, or the joint phase's S frames).
 size_t split_cnt_count(const kvc_config& g) {
-  return static_cast<size_t>(g.num_heads) * ((g.tokens_per_frame + 127) / 128);
+  const long long rows = static_cast<long long>(g.tokens_per_frame) * std::max(1, g.scale_frames);
+  return static_cast<size_t>(g.num_heads) * static_cast<size_t>((rows + 127) / 128);
 }
 
 void free_all(kvc_cache* c) {
@@ -114,6 +117,48 @@ kvc_status remove_entries(kvc_cache* c, int layer, int a, int b) {
   L.n_entries -= n;
   for (FrameRec& f : L.frames)
     if (f.first_entry >= b) f.first_entry -= n;
+  for (FrameRec& f : L.retained)
+    if (f.first_entry >= b) f.first_entry -= n;
+  return KVC_OK;
+}
+
+// Pages of a frame that hold its special tokens (the first num_special_tokens tokens).
+int special_pages(const kvc_config& g) {
+  return g.special_frames > 0 ? (std::min(g.num_special_tokens, g.tokens_per_frame) + g.page_size - 1) / g.page_size
+                              : 0;
+}
+
+// Evict a committed frame ([GCT] Sliding Window Eviction). With special-token persistence
+// ([GCT] Special Token Persistence) its first special_pages() pages stay where they are,
+// trimmed to the special tokens; beyond special_frames retained frames the oldest goes.
+kvc_status evict_frame(kvc_cache* c, int layer, const FrameRec& f) {
+  const kvc_config& g = c->cfg;
+  LayerHost& L = c->L[layer];
+  const int sp = special_pages(g);
+  if (sp == 0) {
+    L.tokens -= g.tokens_per_frame;
+    return remove_entries(c, layer, f.first_entry, f.first_entry + f.n_entries);
+  }
+  const int ns = std::min(g.num_special_tokens, g.tokens_per_frame);
+  cudaError_t e = launch_trim_pages(c->stream, layer_pool(c, c->k_pool, layer), layer_pool(c, c->v_pool, layer),
+                                    layer_entries(c, layer), f.first_entry, sp, ns, g.num_heads, g.page_size,
+                                    static_cast<int>(g.head_dim * c->elem_kv));
+  if (e != cudaSuccess) return cuda_fail(c, e, "special-token trim");
+  c->launches++;
+  if (f.n_entries > sp) {
+    kvc_status st = remove_entries(c, layer, f.first_entry + sp, f.first_entry + f.n_entries);
+    if (st != KVC_OK) return st;
+  }
+  FrameRec r = f;
+  r.n_entries = sp;
+  L.retained.push_back(r);
+  L.tokens -= g.tokens_per_frame - ns;
+  if (static_cast<int>(L.retained.size()) > g.special_frames) {
+    const FrameRec old = L.retained.front();
+    L.retained.erase(L.retained.begin());
+    L.tokens -= ns;
+    return remove_entries(c, layer, old.first_entry, old.first_entry + old.n_entries);
+  }
   return KVC_OK;
 }
 
@@ -156,8 +201,11 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   if (!cfg || !out) return KVC_ERR_ARG;
   *out = nullptr;
   const kvc_config& g = *cfg;
-  for (int i = 0; i < 6; ++i)
+  for (int i = 0; i < 5; ++i)
     if (g.reserved[i] != 0) return KVC_ERR_ARG;
+  if (g.special_frames < 0 || g.special_frames > (1 << 20) ||
+      (g.special_frames > 0 && (g.window_frames <= 0 || g.budget_tokens > 0 || g.diversity_budget > 0)))
+    return KVC_ERR_ARG;
   const bool dims_ok = g.num_layers >= 1 && g.num_heads >= 1 && g.tokens_per_frame >= 1 && g.page_size >= 1 &&
                        g.num_special_tokens >= 0 && g.num_special_tokens <= g.tokens_per_frame &&
                        g.scale_frames >= 0 && g.budget_tokens >= 0 &&
@@ -205,7 +253,7 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
     c->pool_pages = 2 * c->ppf + kp + 1;
     c->layer_budget.assign(g.num_layers, g.diversity_budget);
   } else if (g.window_frames > 0) {
-    c->pool_pages = (g.scale_frames + g.window_frames + 1) * c->ppf;
+    c->pool_pages = (g.scale_frames + g.window_frames + 1) * c->ppf + g.special_frames * special_pages(g);
   } else if (g.budget_tokens > 0) {
     const int B = g.budget_tokens;
     c->pool_pages = 2 * ((B + P - 1) / P) + ((B + T - 1) / T + 2) * c->ppf;
@@ -599,16 +647,11 @@ kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const void* con
   return KVC_OK;
 }
 
-kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_dev) {
-  if (!c) return KVC_ERR_ARG;
-  if (!valid_layer(c, layer) || !q_dev || !o_dev) return fail(c, KVC_ERR_ARG, "kvc_attend: bad layer or pointer");
-  if ((reinterpret_cast<uintptr_t>(q_dev) | reinterpret_cast<uintptr_t>(o_dev)) & 15)
-    return fail(c, KVC_ERR_ARG, "kvc_attend: Q and O must be 16-byte aligned");
-  LayerHost& L = c->L[layer];
-  if (!L.has_pending) return fail(c, KVC_ERR_STATE, "kvc_attend: no frame pending on this layer");
-  if (c->per_head) return div_attend(c, layer, q_dev, o_dev);
+// Attention of Tq query rows over every page of the layer's list (shared pages).
+kvc_status attend_layer(kvc_cache* c, int layer, const void* q_dev, void* o_dev, int Tq) {
   const kvc_config& g = c->cfg;
-  const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads, D = g.head_dim;
+  const int P = g.page_size, H = g.num_heads, D = g.head_dim;
+  const LayerHost& L = c->L[layer];
   Entry* E = layer_entries(c, layer);
   cudaError_t e;
   if (c->tc_path) {
@@ -617,7 +660,7 @@ kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_de
     a.o = o_dev;
     a.entries = E;
     a.n_pages = L.n_entries;
-    a.T = T;
+    a.T = Tq;
     a.H = H;
     a.P = P;
     a.page_base = static_cast<long long>(layer) * c->pool_pages;
@@ -641,10 +684,25 @@ kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_de
   } else {
     e = launch_attn_simt(c->stream, g.io_dtype, g.kv_dtype, q_dev, o_dev, layer_pool(c, c->k_pool, layer),
                          layer_pool(c, c->v_pool, layer), layer_scale(c, c->k_scale, layer),
-                         layer_scale(c, c->v_scale, layer), E, L.n_entries, T, H, D, P, g.softmax_scale);
+                         layer_scale(c, c->v_scale, layer), E, L.n_entries, Tq, H, D, P, g.softmax_scale);
     if (e == cudaSuccess) c->launches++;
   }
   if (e != cudaSuccess) return cuda_fail(c, e, "attention launch");
+  return KVC_OK;
+}
+
+kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_dev) {
+  if (!c) return KVC_ERR_ARG;
+  if (!valid_layer(c, layer) || !q_dev || !o_dev) return fail(c, KVC_ERR_ARG, "kvc_attend: bad layer or pointer");
+  if ((reinterpret_cast<uintptr_t>(q_dev) | reinterpret_cast<uintptr_t>(o_dev)) & 15)
+    return fail(c, KVC_ERR_ARG, "kvc_attend: Q and O must be 16-byte aligned");
+  LayerHost& L = c->L[layer];
+  if (!L.has_pending) return fail(c, KVC_ERR_STATE, "kvc_attend: no frame pending on this layer");
+  if (c->per_head) return div_attend(c, layer, q_dev, o_dev);
+  const kvc_config& g = c->cfg;
+  const int T = g.tokens_per_frame;
+  kvc_status ast = attend_layer(c, layer, q_dev, o_dev, T);
+  if (ast != KVC_OK) return ast;
   // commit / evict, or release the skipped frame
   if (L.pending_key) {
     L.frames.push_back(L.pending);
@@ -659,9 +717,8 @@ kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_de
       while (L.frames.size() > S + W) {
         const FrameRec f = L.frames[S];
         L.frames.erase(L.frames.begin() + S);
-        kvc_status st = remove_entries(c, layer, f.first_entry, f.first_entry + f.n_entries);
+        kvc_status st = evict_frame(c, layer, f);
         if (st != KVC_OK) return st;
-        L.tokens -= T;
         L.evicted++;
       }
     }
@@ -672,6 +729,35 @@ kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_de
   }
   L.has_pending = false;
   return KVC_OK;
+}
+
+kvc_status kvc_scale_phase(kvc_cache* c, int32_t layer, int32_t n_frames, const void* q_dev, const void* k_dev,
+                           const void* v_dev, void* o_dev) {
+  if (!c) return KVC_ERR_ARG;
+  const kvc_config& g = c->cfg;
+  if (!valid_layer(c, layer) || !q_dev || !k_dev || !v_dev || !o_dev || n_frames < 1 ||
+      n_frames > std::max(1, g.scale_frames))
+    return fail(c, KVC_ERR_ARG, "kvc_scale_phase: bad layer, pointer or frame count (1..scale_frames)");
+  if ((reinterpret_cast<uintptr_t>(q_dev) | reinterpret_cast<uintptr_t>(k_dev) | reinterpret_cast<uintptr_t>(v_dev) |
+       reinterpret_cast<uintptr_t>(o_dev)) & 15)
+    return fail(c, KVC_ERR_ARG, "kvc_scale_phase: Q, K, V and O must be 16-byte aligned");
+  if (c->per_head || g.budget_tokens > 0)
+    return fail(c, KVC_ERR_STATE, "kvc_scale_phase: not with a token budget or per-head page lists");
+  LayerHost& L = c->L[layer];
+  if (L.n_entries != 0 || L.has_pending || L.last_frame >= 0)
+    return fail(c, KVC_ERR_STATE, "kvc_scale_phase: the joint phase starts an empty layer");
+  // frames 0 .. n-1 appended and committed, then all n*T queries over all of them
+  const size_t frame_bytes = static_cast<size_t>(g.tokens_per_frame) * g.num_heads * g.head_dim * c->elem_io;
+  for (int f = 0; f < n_frames; ++f) {
+    kvc_status st = kvc_append_frame(c, layer, f, static_cast<const uint8_t*>(k_dev) + f * frame_bytes,
+                                     static_cast<const uint8_t*>(v_dev) + f * frame_bytes, 1);
+    if (st != KVC_OK) return st;
+    L.frames.push_back(L.pending);
+    L.tokens += g.tokens_per_frame;
+    L.committed++;
+    L.has_pending = false;
+  }
+  return attend_layer(c, layer, q_dev, o_dev, n_frames * g.tokens_per_frame);
 }
 
 kvc_status kvc_compress(kvc_cache* c, int32_t layer, const float* residual_dev, int32_t* fired_out) {

@@ -24,6 +24,7 @@ struct LayerHost {
   int32_t block_entries = 0;      // leading entries written by compaction (owner -1)
   int64_t block_tokens = 0;
   std::vector<FrameRec> frames;   // committed frames after the block, in cache order
+  std::vector<FrameRec> retained; // evicted frames whose special-token pages stay, oldest first
   bool has_pending = false;
   bool pending_key = false;
   FrameRec pending;
@@ -135,6 +136,10 @@ cudaError_t launch_mgr_alloc_layers(cudaStream_t s, Entry* entries_all, uint32_t
                                     int valid_full, int valid_last, int* err, int group = 1);
 cudaError_t launch_mgr_remove(cudaStream_t s, Entry* entries, uint32_t* bitmap, int n_entries, int a, int b,
                               int* err);
+// Trim entries [first, first + n_pages) to the first `keep` tokens: zero the other slots of
+// every head (K and V) and set the entries' valid counts.
+cudaError_t launch_trim_pages(cudaStream_t s, uint8_t* k_pool_layer, uint8_t* v_pool_layer, Entry* entries, int first,
+                              int n_pages, int keep, int H, int P, int row_bytes);
 cudaError_t launch_debug_wait(cudaStream_t s, int* flag, int* err, long long timeout_ns);
 
 // Append (same dtype in and out): K, V [T,H,D] -> pages of entries [0, n_pages).

@@ -153,6 +153,45 @@ cudaError_t launch_mgr_remove(cudaStream_t s, Entry* entries, uint32_t* bitmap, 
   return cudaGetLastError();
 }
 
+// One 16-byte chunk per thread over (page, head, slot past the kept tokens, chunk) for K
+// and V; the first thread of each page writes its valid count.
+__global__ void trim_pages_kernel(uint8_t* k_pool, uint8_t* v_pool, Entry* entries, int first, int n_pages, int keep,
+                                  int H, int P, int chunks) {
+  const long long per_tensor = static_cast<long long>(n_pages) * H * P * chunks;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < 2 * per_tensor;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const bool is_v = idx >= per_tensor;
+    long long r = is_v ? idx - per_tensor : idx;
+    const int ch = static_cast<int>(r % chunks);
+    r /= chunks;
+    const int slot = static_cast<int>(r % P);
+    r /= P;
+    const int h = static_cast<int>(r % H);
+    const int j = static_cast<int>(r / H);
+    const int kept = min(P, keep - j * P);
+    const int page = entries[first + j].x;
+    if (slot >= kept) {
+      uint4* dst = reinterpret_cast<uint4*>((is_v ? v_pool : k_pool) +
+                                            ((static_cast<long long>(page) * H + h) * P + slot) * chunks * 16);
+      dst[ch] = make_uint4(0, 0, 0, 0);
+    }
+    if (!is_v && h == 0 && slot == 0 && ch == 0) entries[first + j].w = kept;
+  }
+}
+
+cudaError_t launch_trim_pages(cudaStream_t s, uint8_t* k_pool_layer, uint8_t* v_pool_layer, Entry* entries, int first,
+                              int n_pages, int keep, int H, int P, int row_bytes) {
+  if (row_bytes % 16 != 0 || n_pages < 1 || keep < 1 || keep > n_pages * P) return cudaErrorInvalidValue;
+  const int chunks = row_bytes / 16;
+  const long long total = 2LL * n_pages * H * P * chunks;
+  const int threads = 256;
+  long long blocks = (total + threads - 1) / threads;
+  if (blocks > 1184) blocks = 1184;
+  trim_pages_kernel<<<static_cast<int>(blocks), threads, 0, s>>>(k_pool_layer, v_pool_layer, entries, first, n_pages,
+                                                                 keep, H, P, chunks);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_debug_wait(cudaStream_t s, int* flag, int* err, long long timeout_ns) {
   debug_wait_kernel<<<1, 32, 0, s>>>(flag, err, timeout_ns);
   return cudaGetLastError();
