@@ -63,6 +63,7 @@ class Workload:
     diversity_budget: int = 0
     special_frames: int = 0      # evicted frames whose special tokens stay cached (0: off)
     joint_frames: int = 0        # > 0: the stream opens with a joint phase of this many frames
+    fp8_dim_adaptive: int = 0    # FP8 storage: K scales per channel, V scales per token
     description: str = ""
 
     def as_dict(self) -> Dict:

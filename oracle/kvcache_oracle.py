@@ -41,7 +41,10 @@ What it follows (the web pages are cited by title and section):
   register tokens) follow the budgeted-compression workload's statement.
 * FP8 KV quantisation -- XStreamVGGT abstract (KV cache quantisation); the
   format is OCP FP8 E4M3 (bias 7, max finite 448, no infinities), one absmax
-  scale per (page, head), separately for K and V.
+  scale per (page, head), separately for K and V. Its "dimension-adaptive" variant
+  (the abstract's wording; KIVI, which it cites, quantises keys per channel and
+  values per token) takes one absmax scale per (page, head, channel) for K and one
+  per (page, head, token) for V.
 
 Readings taken where the pages are silent (each is also listed in the design
 notes): the order append -> attend -> commit/evict; lowest-free page allocation;
@@ -155,6 +158,34 @@ def fp8_quantise_block(x: np.ndarray):
     return codes, scale, e4m3_decode(codes) * scale
 
 
+def fp8_quantise_channels(x: np.ndarray):
+    """Dimension-adaptive FP8 of a K block [n, D] of valid tokens: each channel (column)
+    quantised as its own block by fp8_quantise_block. Returns (codes [n, D], scales [D],
+    dequantised fp64 [n, D])."""
+    x = np.asarray(x, dtype=np.float64)
+    n, D = x.shape
+    codes = np.zeros((n, D), np.uint8)
+    scales = np.zeros(D)
+    deq = np.zeros((n, D))
+    for d in range(D):
+        codes[:, d], scales[d], deq[:, d] = fp8_quantise_block(x[:, d])
+    return codes, scales, deq
+
+
+def fp8_quantise_tokens(x: np.ndarray):
+    """Dimension-adaptive FP8 of a V block [n, D] of valid tokens: each token (row)
+    quantised as its own block by fp8_quantise_block. Returns (codes [n, D], scales [n],
+    dequantised fp64 [n, D])."""
+    x = np.asarray(x, dtype=np.float64)
+    n, D = x.shape
+    codes = np.zeros((n, D), np.uint8)
+    scales = np.zeros(n)
+    deq = np.zeros((n, D))
+    for i in range(n):
+        codes[i], scales[i], deq[i] = fp8_quantise_block(x[i])
+    return codes, scales, deq
+
+
 # --------------------------------------------------------------------------------------
 # Cache configuration and state
 # --------------------------------------------------------------------------------------
@@ -178,6 +209,7 @@ class OracleConfig:
     residual_dim: int = 1024
     protect_first_frame: int = 1
     special_frames: int = 0       # evicted frames whose special tokens stay (0: off)
+    fp8_dim_adaptive: int = 0     # FP8: K scales per channel, V scales per token
 
     @staticmethod
     def from_workload(wl) -> "OracleConfig":
@@ -188,7 +220,8 @@ class OracleConfig:
             kv_dtype=wl.kv_dtype, softmax_scale=wl.softmax_scale, budget_tokens=wl.budget_tokens,
             keep_frac=wl.keep_frac, lam=wl.lam, rank_window=wl.rank_window,
             residual_dim=wl.residual_dim, protect_first_frame=wl.protect_first_frame,
-            special_frames=getattr(wl, "special_frames", 0))
+            special_frames=getattr(wl, "special_frames", 0),
+            fp8_dim_adaptive=getattr(wl, "fp8_dim_adaptive", 0))
 
 
 class _Page:
@@ -199,8 +232,10 @@ class _Page:
         self.v = np.zeros((H, P, D))
         self.k_codes = None                   # FP8 only: uint8 [H, P, D]
         self.v_codes = None
-        self.k_scale = None                   # FP8 only: float64 [H]
-        self.v_scale = None
+        self.k_scale = None                   # FP8 only: float64 [H] (the largest of the
+        self.v_scale = None                   # channel / token scales when dimension-adaptive)
+        self.k_chan_scale = None              # dimension-adaptive FP8: [H, D]
+        self.v_tok_scale = None               # dimension-adaptive FP8: [H, P]
         self.ids = np.full(P, -1, np.int64)   # global token id = frame * T + slot
         self.counts = np.zeros(P, np.int64)   # merge counts (1 for an original token)
         self.shat = np.zeros(P, np.float64)   # enhanced score, fp32 value
@@ -286,7 +321,18 @@ class StreamOracle:
                 pg.v_codes = np.zeros((H, P, cfg.head_dim), np.uint8)
                 pg.k_scale = np.zeros(H)
                 pg.v_scale = np.zeros(H)
+                if cfg.fp8_dim_adaptive:
+                    pg.k_chan_scale = np.zeros((H, cfg.head_dim))
+                    pg.v_tok_scale = np.zeros((H, P))
                 for h in range(H):
+                    if cfg.fp8_dim_adaptive:
+                        c, s, dq = fp8_quantise_channels(kb[h])
+                        pg.k_codes[h, :n], pg.k_chan_scale[h], pg.k[h, :n] = c, s, dq
+                        pg.k_scale[h] = s.max()
+                        c, s, dq = fp8_quantise_tokens(vb[h])
+                        pg.v_codes[h, :n], pg.v_tok_scale[h, :n], pg.v[h, :n] = c, s, dq
+                        pg.v_scale[h] = s.max()
+                        continue
                     c, s, dq = fp8_quantise_block(kb[h])
                     pg.k_codes[h, :n], pg.k_scale[h], pg.k[h, :n] = c, s, dq
                     c, s, dq = fp8_quantise_block(vb[h])
@@ -478,6 +524,12 @@ class StreamOracle:
         ks = np.stack([L.pages[e[0]].k_scale for e in L.entries])
         vs = np.stack([L.pages[e[0]].v_scale for e in L.entries])
         return kc, vc, ks, vs
+
+    def fp8_da_scales(self, layer: int):
+        """Dimension-adaptive FP8 scales in page-table order: K [n, H, D], V [n, H, P]."""
+        L = self.layers[layer]
+        return (np.stack([L.pages[e[0]].k_chan_scale for e in L.entries]),
+                np.stack([L.pages[e[0]].v_tok_scale for e in L.entries]))
 
     # ---------------------------------------------------------------- CLCES scoring
     def score(self, layer: int, t: int, residual: np.ndarray) -> np.ndarray:

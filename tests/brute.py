@@ -47,6 +47,24 @@ def stored(K: np.ndarray, kv_dtype: str, P: int) -> np.ndarray:
     return out
 
 
+def stored_dim_adaptive(X: np.ndarray, P: int, per: str) -> np.ndarray:
+    """Values the cache stores for one frame's K (per="channel": a scale per page, head and
+    channel) or V (per="token": a scale per page, head and token) with dimension-adaptive
+    FP8, through torch's float8 cast."""
+    T, H, D = X.shape
+    out = np.zeros_like(X)
+    for g in range(0, T, P):
+        for h in range(H):
+            blk = X[g:g + P, h]
+            if per == "channel":
+                for d in range(D):
+                    out[g:g + P, h, d] = fp8_dequant_torch(blk[:, d])
+            else:
+                for i in range(blk.shape[0]):
+                    out[g + i, h] = fp8_dequant_torch(blk[i])
+    return out
+
+
 def attention(Q, K, V, scale):
     """Full softmax attention per head, fp64, scipy softmax."""
     N, H, D = K.shape

@@ -24,8 +24,12 @@ def _run_and_check(wl, frames, seed=0, check_rows=None):
         q, kk, vv = _np(q), _np(kk), _np(vv)
         key = keyframe_schedule(t, S, k)
         orc.append(0, t, kk, vv, key)
-        hist_k[t] = brute.stored(kk, wl.kv_dtype, wl.page_size)
-        hist_v[t] = brute.stored(vv, wl.kv_dtype, wl.page_size)
+        if getattr(wl, "fp8_dim_adaptive", 0):
+            hist_k[t] = brute.stored_dim_adaptive(kk, wl.page_size, "channel")
+            hist_v[t] = brute.stored_dim_adaptive(vv, wl.page_size, "token")
+        else:
+            hist_k[t] = brute.stored(kk, wl.kv_dtype, wl.page_size)
+            hist_v[t] = brute.stored(vv, wl.kv_dtype, wl.page_size)
         rows = check_rows
         got = orc.attend(0, q, rows=rows)
         fr = brute.retained_frames(t, S, W, k)
@@ -76,6 +80,13 @@ def test_fp8_small_matches_brute_force():
     wl = WORKLOADS["vggt_518x518_fp8"].replace(tokens_per_frame=37, num_heads=2, head_dim=16,
                                                 window_frames=3, scale_frames=2, page_size=8)
     _run_and_check(wl, 9, seed=5)
+
+
+def test_fp8_dimension_adaptive_small_matches_brute_force():
+    wl = WORKLOADS["vggt_518x518_fp8"].replace(tokens_per_frame=37, num_heads=2, head_dim=16,
+                                                window_frames=3, scale_frames=2, page_size=8,
+                                                fp8_dim_adaptive=1)
+    _run_and_check(wl, 9, seed=6)
 
 
 def test_bf16_temporal_small_matches_brute_force():

@@ -94,3 +94,49 @@ def test_fp8_block_error_bound():
     # subnormal floor of half of 2^-9 * scale
     bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * scale) * (1 + 1e-6)
     assert np.all(np.abs(deq - x) <= bound)
+
+
+# ---- dimension-adaptive FP8 ("XStreamVGGT" abstract; K per channel, V per token)
+
+def test_dimension_adaptive_reduces_to_per_block_quantisation():
+    from oracle import fp8_quantise_block, fp8_quantise_channels, fp8_quantise_tokens
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((16, 64)) * np.exp(rng.standard_normal(64))[None, :]
+    x[:, 3] *= 1000.0                               # an outlier channel
+    ck, sk, dk = fp8_quantise_channels(x)
+    cv, sv, dv = fp8_quantise_tokens(x)
+    for d in range(64):
+        c, s_, q = fp8_quantise_block(x[:, d])
+        assert np.array_equal(ck[:, d], c) and sk[d] == s_ and np.array_equal(dk[:, d], q)
+    for i in range(16):
+        c, s_, q = fp8_quantise_block(x[i])
+        assert np.array_equal(cv[i], c) and sv[i] == s_ and np.array_equal(dv[i], q)
+
+
+def test_dimension_adaptive_matches_torch_float8_per_channel_and_token():
+    import brute
+    from oracle import fp8_quantise_channels, fp8_quantise_tokens
+    from oracle import bf16_round
+    rng = np.random.default_rng(22)
+    x = bf16_round(rng.standard_normal((16, 32)) * np.exp(2 * rng.standard_normal(32))[None, :])   # cache inputs
+    _, _, dk = fp8_quantise_channels(x)
+    _, _, dv = fp8_quantise_tokens(x)
+    for d in range(32):
+        np.testing.assert_array_equal(dk[:, d], brute.fp8_dequant_torch(x[:, d]))
+    for i in range(16):
+        np.testing.assert_array_equal(dv[i], brute.fp8_dequant_torch(x[i]))
+
+
+def test_outlier_channel_costs_other_channels_nothing():
+    """Per-block scales let one outlier channel flush its block's small values; per-channel
+    scales keep every other channel at E4M3's relative precision (2^-4)."""
+    from oracle import fp8_quantise_block, fp8_quantise_channels
+    from oracle import bf16_round
+    rng = np.random.default_rng(23)
+    x = bf16_round(rng.uniform(0.5, 1.0, (16, 8)))
+    x[:, 0] = 2.0 ** 20                             # the page's amax lives in channel 0
+    _, _, blk = fp8_quantise_block(x)
+    _, _, ch = fp8_quantise_channels(x)
+    rel_ch = np.abs(ch[:, 1:] - x[:, 1:]) / x[:, 1:]
+    assert rel_ch.max() <= 2.0 ** -4
+    assert (blk[:, 1:] == 0).all()                  # x / (2^20 / 448) < 2^-10: below E4M3's subnormals
