@@ -104,7 +104,9 @@ typedef struct {
                                    head per layer besides the first frame (see kvc_attend) */
   int32_t special_frames;       /* > 0 (window mode only): cross-frame special tokens, see
                                    kvc_attend; the evicted frames whose special tokens stay */
-  int32_t reserved[5];          /* must be zero */
+  int32_t fp8_dim_adaptive;     /* 1 with kv_dtype FP8 (D = 64, P = 16): dimension-adaptive
+                                   scales, see kvc_append_frame; 0: one scale per (page, head) */
+  int32_t reserved[4];          /* must be zero */
 } kvc_config;
 
 /* Cache statistics ([GCT] Cache Monitoring: occupancy, memory use, eviction status). */
@@ -151,6 +153,10 @@ KVC_API kvc_status kvc_reset(kvc_cache* c);
  * the last page are zero. With kv_dtype FP8 each (page, head) block of K and V
  * is quantised with its own absmax scale: scale = fp32(amax / 448), code =
  * E4M3 round-to-nearest-even saturating of fp32(x / scale) ([XSV] abstract).
+ * With fp8_dim_adaptive ([XSV] abstract: dimension-adaptive KV quantisation, read as
+ * KIVI's keys per channel and values per token) the same rule applies to each channel of
+ * K (a scale per (page, head, channel)) and each token of V (a scale per (page, head,
+ * slot)); the per-(page, head) scale arrays then hold the largest of a block's scales.
  * The frame is *pending* until kvc_attend: `is_keyframe` = 0 makes attention
  * release it afterwards ([GCT] Selective Frame Caching with Skip Append).
  * Frame indices must increase per layer. Errors: KVC_ERR_STATE if a frame is
@@ -237,6 +243,13 @@ KVC_API kvc_status kvc_last_merge(kvc_cache* c, int32_t layer, int64_t* src_host
  * head) scales [n_rows][H] fp32 (scale pointers may be NULL otherwise). */
 KVC_API kvc_status kvc_export_pages(kvc_cache* c, int32_t layer, int32_t first_row, int32_t n_rows,
                             void* k_host, void* v_host, float* k_scale_host, float* v_scale_host);
+
+/* Dimension-adaptive FP8 scales of page-table rows [first_row, first_row + n_rows) of
+ * `layer`: k_chan_host [n_rows][H][D] (K, per channel) and v_tok_host [n_rows][H][P] (V,
+ * per slot; 0 for slots without a token). Host buffers owned by the caller. Synchronises.
+ * Errors: KVC_ERR_STATE (not dimension-adaptive FP8), KVC_ERR_ARG (range, pointers). */
+KVC_API kvc_status kvc_export_fp8_group_scales(kvc_cache* c, int32_t layer, int32_t first_row, int32_t n_rows,
+                                               float* k_chan_host, float* v_tok_host);
 
 /* One whole frame step of `layer` from HOST buffers: copy q, k, v [T, H, D]
  * host -> device, append, attend (+ commit/evict), copy O device -> host,

@@ -120,6 +120,12 @@ WORKLOADS: Dict[str, Workload] = {
         keyframe_interval=1, num_frames=10000, io_dtype="bf16", kv_dtype="bf16",
         softmax_scale=0.125, temporal_keys=True, special_frames=4096,
         description="518x378 stream keeping the 5 special tokens of up to 4,096 evicted frames"),
+    "vggt_518x518_fp8da": Workload(
+        name="vggt_518x518_fp8da", num_layers=1, num_heads=16, head_dim=64, tokens_per_frame=1374,
+        num_special_tokens=5, page_size=16, window_frames=128, scale_frames=8,
+        keyframe_interval=1, num_frames=10000, io_dtype="bf16", kv_dtype="fp8_e4m3",
+        softmax_scale=0.125, temporal_keys=False, outlier_fraction=0.01, fp8_dim_adaptive=1,
+        description="518x518 frames, W=128, dimension-adaptive FP8 storage (K per channel, V per token)"),
     "vggt_infinite_12l": Workload(
         name="vggt_infinite_12l", num_layers=12, num_heads=16, head_dim=64, tokens_per_frame=1004,
         num_special_tokens=5, page_size=16, window_frames=0, scale_frames=0,

@@ -131,6 +131,11 @@ def check_page_bytes(kvc, h, layer, wl, orc):
         assert np.array_equal(vb.reshape(n, H, P, D), vc), "FP8 V codes differ"
         assert np.array_equal(ks.astype(np.float64), kso), "FP8 K scales differ"
         assert np.array_equal(vs.astype(np.float64), vso), "FP8 V scales differ"
+        if getattr(wl, "fp8_dim_adaptive", 0):
+            kc_g, vt_g = kvc.kvc_export_fp8_group_scales(h, layer, 0, n, H, D, P)
+            kc_o, vt_o = orc.fp8_da_scales(layer)
+            assert np.array_equal(kc_g.astype(np.float64), kc_o), "FP8 K channel scales differ"
+            assert np.array_equal(vt_g.astype(np.float64), vt_o), "FP8 V token scales differ"
     else:
         dt = torch.float32 if elem == 4 else torch.bfloat16
         L = orc.layers[layer]

@@ -29,7 +29,7 @@ EXPORTS = ["kvc_create", "kvc_destroy", "kvc_set_stream", "kvc_reset", "kvc_appe
            "kvc_step_host", "kvc_synchronize", "kvc_last_error", "kvc_status_string", "kvc_version",
            "kvc_debug_fail_allocs", "kvc_debug_bounded_wait", "kvc_attend_paged_noalloc", "kvc_append_frame_all",
            "kvc_step_host_async", "kvc_set_layer_budgets", "kvc_prune", "kvc_layer_diversity",
-           "kvc_head_tokens", "kvc_scale_phase"]
+           "kvc_head_tokens", "kvc_scale_phase", "kvc_export_fp8_group_scales"]
 
 
 class kvc_config(ctypes.Structure):
@@ -41,7 +41,8 @@ class kvc_config(ctypes.Structure):
                 ("rank_window", ctypes.c_int32), ("residual_dim", ctypes.c_int32),
                 ("protect_first_frame", ctypes.c_int32), ("max_frames", ctypes.c_int32),
                 ("kv_splits", ctypes.c_int32), ("diversity_budget", ctypes.c_int32),
-                ("special_frames", ctypes.c_int32), ("reserved", ctypes.c_int32 * 5)]
+                ("special_frames", ctypes.c_int32), ("fp8_dim_adaptive", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 4)]
 
 
 class kvc_info(ctypes.Structure):
@@ -85,6 +86,7 @@ def _load():
         "kvc_set_layer_budgets": ([vp, vp, i32], i32),
         "kvc_prune": ([vp, i32], i32),
         "kvc_scale_phase": ([vp, i32, i32, vp, vp, vp, vp], i32),
+        "kvc_export_fp8_group_scales": ([vp, i32, i32, i32, vp, vp], i32),
         "kvc_layer_diversity": ([vp, i32, vp], i32),
         "kvc_head_tokens": ([vp, i32, i32, vp, i32, vp], i32),
         "kvc_synchronize": ([vp], i32),
@@ -136,7 +138,7 @@ def make_config(num_layers, num_heads, head_dim, tokens_per_frame, num_special_t
                 window_frames, scale_frames, io_dtype="bf16", kv_dtype="bf16", softmax_scale=0.125,
                 budget_tokens=0, keep_frac=0.6, lam=0.5, rank_window=5, residual_dim=1024,
                 protect_first_frame=1, max_frames=0, kv_splits=0, diversity_budget=0,
-                special_frames=0) -> kvc_config:
+                special_frames=0, fp8_dim_adaptive=0) -> kvc_config:
     c = kvc_config()
     c.num_layers, c.num_heads, c.head_dim = num_layers, num_heads, head_dim
     c.tokens_per_frame, c.num_special_tokens, c.page_size = tokens_per_frame, num_special_tokens, page_size
@@ -149,6 +151,7 @@ def make_config(num_layers, num_heads, head_dim, tokens_per_frame, num_special_t
     c.max_frames, c.kv_splits = max_frames, kv_splits
     c.diversity_budget = diversity_budget
     c.special_frames = special_frames
+    c.fp8_dim_adaptive = fp8_dim_adaptive
     return c
 
 
@@ -160,7 +163,8 @@ def config_from_workload(wl, **over) -> kvc_config:
              budget_tokens=wl.budget_tokens, keep_frac=wl.keep_frac, lam=wl.lam, rank_window=wl.rank_window,
              residual_dim=wl.residual_dim, protect_first_frame=wl.protect_first_frame,
              diversity_budget=getattr(wl, "diversity_budget", 0),
-             special_frames=getattr(wl, "special_frames", 0))
+             special_frames=getattr(wl, "special_frames", 0),
+             fp8_dim_adaptive=getattr(wl, "fp8_dim_adaptive", 0))
     d.update(over)
     return make_config(**d)
 
@@ -282,6 +286,15 @@ def kvc_scale_phase(handle, layer: int, n_frames: int, q, k, v, o) -> None:
     """The joint scale-frame phase: frames 0..n_frames-1 ([n_frames*T, H, D] tensors)
     appended, committed, and attended bidirectionally."""
     _check(handle, _lib.kvc_scale_phase(handle, layer, n_frames, _ptr(q), _ptr(k), _ptr(v), _ptr(o)))
+
+
+def kvc_export_fp8_group_scales(handle, layer: int, first_row: int, n_rows: int, H: int, D: int, P: int):
+    """Dimension-adaptive FP8 scales of page-table rows: K [n, H, D], V [n, H, P] (float32)."""
+    kc = np.zeros((n_rows, H, D), np.float32)
+    vt = np.zeros((n_rows, H, P), np.float32)
+    _check(handle, _lib.kvc_export_fp8_group_scales(handle, layer, first_row, n_rows,
+                                                    kc.ctypes.data, vt.ctypes.data))
+    return kc, vt
 
 
 def kvc_prune(handle, layer: int) -> None:

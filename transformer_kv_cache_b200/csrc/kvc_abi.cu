@@ -47,7 +47,8 @@ void free_all(kvc_cache* c) {
   void* ptrs[] = {c->k_pool,     c->v_pool,     c->k_scale,    c->v_scale,    c->entries,    c->bitmap,
                   c->d_err,      c->tok_id,     c->tok_cnt,    c->tok_shat,   c->cmp_scratch, c->part_o,
                   c->part_lse,   c->stage_q[0], c->stage_k[0], c->stage_v[0], c->stage_o[0], c->stage_q[1],
-                  c->stage_k[1], c->stage_v[1], c->stage_o[1], c->rank_hist, c->div_sums, c->split_cnt};
+                  c->stage_k[1], c->stage_v[1], c->stage_o[1], c->rank_hist, c->div_sums, c->split_cnt,
+                  c->k_chan,     c->v_tok};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   for (int i = 0; i < 2; ++i) {
@@ -82,6 +83,10 @@ uint32_t* layer_bitmap(kvc_cache* c, int layer) {
 }
 uint8_t* layer_pool(kvc_cache* c, uint8_t* pool, int layer) {
   return pool + static_cast<size_t>(layer) * c->pool_pages * c->page_bytes_kv;
+}
+// Dimension-adaptive FP8 group scales of a layer (per = D for K channels, P for V tokens).
+float* layer_group_scales(kvc_cache* c, float* sc, int layer, int per) {
+  return sc ? sc + static_cast<size_t>(layer) * c->pool_pages * c->cfg.num_heads * per : nullptr;
 }
 float* layer_scale(kvc_cache* c, float* sc, int layer) {
   return sc ? sc + static_cast<size_t>(layer) * c->pool_pages * c->cfg.num_heads : nullptr;
@@ -201,8 +206,11 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   if (!cfg || !out) return KVC_ERR_ARG;
   *out = nullptr;
   const kvc_config& g = *cfg;
-  for (int i = 0; i < 5; ++i)
+  for (int i = 0; i < 4; ++i)
     if (g.reserved[i] != 0) return KVC_ERR_ARG;
+  if (g.fp8_dim_adaptive != 0 &&
+      (g.fp8_dim_adaptive != 1 || g.kv_dtype != KVC_FP8_E4M3 || g.head_dim != 64 || g.page_size != 16))
+    return KVC_ERR_ARG;
   if (g.special_frames < 0 || g.special_frames > (1 << 20) ||
       (g.special_frames > 0 && (g.window_frames <= 0 || g.budget_tokens > 0 || g.diversity_budget > 0)))
     return KVC_ERR_ARG;
@@ -285,6 +293,10 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   A(dev_alloc_t(&c->v_pool, NS * c->pool_pages * c->page_bytes_kv));
   if (g.kv_dtype == KVC_FP8_E4M3) {
     A(dev_alloc_t(&c->k_scale, L * c->pool_pages * H * sizeof(float)));
+    if (g.fp8_dim_adaptive) {
+      A(dev_alloc_t(&c->k_chan, L * c->pool_pages * H * D * sizeof(float)));
+      A(dev_alloc_t(&c->v_tok, L * c->pool_pages * H * P * sizeof(float)));
+    }
     A(dev_alloc_t(&c->v_scale, L * c->pool_pages * H * sizeof(float)));
   }
   A(dev_alloc_t(&c->entries, NS * c->pool_pages * sizeof(Entry)));
@@ -332,6 +344,8 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   A(cudaMemsetAsync(c->v_pool, 0, NS * c->pool_pages * c->page_bytes_kv, c->stream));
   if (c->k_scale) A(cudaMemsetAsync(c->k_scale, 0, L * c->pool_pages * H * sizeof(float), c->stream));
   if (c->v_scale) A(cudaMemsetAsync(c->v_scale, 0, L * c->pool_pages * H * sizeof(float), c->stream));
+  if (c->k_chan) A(cudaMemsetAsync(c->k_chan, 0, L * c->pool_pages * H * D * sizeof(float), c->stream));
+  if (c->v_tok) A(cudaMemsetAsync(c->v_tok, 0, L * c->pool_pages * H * P * sizeof(float), c->stream));
   A(cudaMemsetAsync(c->entries, 0, NS * c->pool_pages * sizeof(Entry), c->stream));
   A(cudaMemsetAsync(c->bitmap, 0, NS * c->bitmap_words * sizeof(uint32_t), c->stream));
   if (c->per_head) {
@@ -547,7 +561,8 @@ kvc_status kvc_append_frame(kvc_cache* c, int32_t layer, int32_t frame_idx, cons
   if (g.kv_dtype == KVC_FP8_E4M3) {
     e = launch_append_fp8(c->stream, k_dev, v_dev, layer_pool(c, c->k_pool, layer), layer_pool(c, c->v_pool, layer),
                           layer_scale(c, c->k_scale, layer), layer_scale(c, c->v_scale, layer), E + L.n_entries, n, T,
-                          g.num_heads, g.head_dim, P);
+                          g.num_heads, g.head_dim, P, layer_group_scales(c, c->k_chan, layer, g.head_dim),
+                          layer_group_scales(c, c->v_tok, layer, P));
   } else {
     e = launch_append(c->stream, static_cast<int>(c->elem_kv), k_dev, v_dev, layer_pool(c, c->k_pool, layer),
                       layer_pool(c, c->v_pool, layer), E + L.n_entries, n, T, g.num_heads, g.head_dim, P);
@@ -621,7 +636,7 @@ kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const void* con
     c->launches++;
     if (g.kv_dtype == KVC_FP8_E4M3)
       e = launch_append_fp8_layers(c->stream, in, st, nl, c->k_pool, c->v_pool, c->k_scale, c->v_scale, c->entries,
-                                   c->pool_pages, n, T, g.num_heads, g.head_dim, P);
+                                   c->pool_pages, n, T, g.num_heads, g.head_dim, P, c->k_chan, c->v_tok);
     else
       e = launch_append_layers(c->stream, static_cast<int>(c->elem_kv), in, st, nl, c->k_pool, c->v_pool, c->entries,
                                c->pool_pages, n, T, g.num_heads, g.head_dim, P);
@@ -672,6 +687,8 @@ kvc_status attend_layer(kvc_cache* c, int layer, const void* q_dev, void* o_dev,
     a.fp8 = g.kv_dtype == KVC_FP8_E4M3;
     a.k_scale = c->k_scale;
     a.v_scale = c->v_scale;
+    a.k_chan = c->k_chan;
+    a.v_tok = c->v_tok;
     a.part_o = c->part_o;
     a.part_lse = c->part_lse;
     a.part_rows = c->part_rows;
@@ -878,6 +895,35 @@ kvc_status kvc_export_pages(kvc_cache* c, int32_t layer, int32_t first_row, int3
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(c, e, "kvc_export_pages");
+  return KVC_OK;
+}
+
+kvc_status kvc_export_fp8_group_scales(kvc_cache* c, int32_t layer, int32_t first_row, int32_t n_rows,
+                                       float* k_chan_host, float* v_tok_host) {
+  if (!c) return KVC_ERR_ARG;
+  if (!c->k_chan) return fail(c, KVC_ERR_STATE, "kvc_export_fp8_group_scales: not dimension-adaptive FP8");
+  if (!valid_layer(c, layer) || !k_chan_host || !v_tok_host)
+    return fail(c, KVC_ERR_ARG, "kvc_export_fp8_group_scales: bad argument");
+  kvc_status st = sync_and_check(c);
+  if (st != KVC_OK) return st;
+  LayerHost& L = c->L[layer];
+  if (first_row < 0 || n_rows < 0 || first_row + n_rows > L.n_entries)
+    return fail(c, KVC_ERR_ARG, "kvc_export_fp8_group_scales: row range outside the page table");
+  std::vector<Entry> ent(n_rows);
+  if (n_rows > 0 && cudaMemcpy(ent.data(), layer_entries(c, layer) + first_row, n_rows * sizeof(Entry),
+                               cudaMemcpyDeviceToHost) != cudaSuccess)
+    return fail(c, KVC_ERR_CUDA, "kvc_export_fp8_group_scales copy");
+  const size_t H = c->cfg.num_heads, D = c->cfg.head_dim, P = c->cfg.page_size;
+  const float* kc = layer_group_scales(c, c->k_chan, layer, static_cast<int>(D));
+  const float* vt = layer_group_scales(c, c->v_tok, layer, static_cast<int>(P));
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < n_rows && e == cudaSuccess; ++i) {
+    const size_t phys = ent[i].x;
+    e = cudaMemcpy(k_chan_host + i * H * D, kc + phys * H * D, H * D * sizeof(float), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(v_tok_host + i * H * P, vt + phys * H * P, H * P * sizeof(float), cudaMemcpyDeviceToHost);
+  }
+  if (e != cudaSuccess) return cuda_fail(c, e, "kvc_export_fp8_group_scales");
   return KVC_OK;
 }
 

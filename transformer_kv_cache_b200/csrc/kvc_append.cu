@@ -61,10 +61,15 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
 // division; each code is the E4M3 rounding of the IEEE-rounded fp32 quotient x / scale; an
 // all-zero block has scale 0 and codes 0 ("XStreamVGGT" abstract: KV cache quantisation;
 // OCP FP8 E4M3). Requires D % 8 == 0 and P * D <= 32 * 64.
+// Dimension-adaptive (k_chan_all != nullptr; D = 64, P = 16): the same quantisation per
+// channel of K (a scale per (page, head, channel), into k_chan_all) and per token of V (a
+// scale per (page, head, slot), into v_tok_all); the page's scale is the largest of them.
+// A lane then holds the 8-dim chunk lane % 8 of slots lane / 8 + 4k, k < 4: a channel's
+// maximum reduces over the four lanes of its chunk, a token's over the eight of its slot.
 __global__ void append_fp8_kernel(AppendBatch in, LayerStarts starts, int n_layers, uint8_t* k_pool_all,
-                                  uint8_t* v_pool_all, float* k_scale_all, float* v_scale_all,
-                                  const Entry* __restrict__ entries_all, int pool_pages, int n_pages, int T, int H,
-                                  int D, int P) {
+                                  uint8_t* v_pool_all, float* k_scale_all, float* v_scale_all, float* k_chan_all,
+                                  float* v_tok_all, const Entry* __restrict__ entries_all, int pool_pages,
+                                  int n_pages, int T, int H, int D, int P) {
   const int warps_per_block = blockDim.x / 32;
   const int gw = blockIdx.x * warps_per_block + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
@@ -110,6 +115,58 @@ __global__ void append_fp8_kernel(AppendBatch in, LayerStarts starts, int n_laye
       nmine = k + 1;
     }
   }
+  if (k_chan_all) {
+    // dimension-adaptive: D = 64, P = 16, four groups per lane
+    float gs[8];                                  // K: per dim of the chunk; V: per group k
+    if (tensor == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float m = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) m = fmaxf(m, fabsf(x[k][e]));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        gs[e] = m > 0.f ? __fdiv_rn(m, 448.0f) : 0.f;
+      }
+      if (lane < 8) {
+        float4* cs = reinterpret_cast<float4*>(k_chan_all + (phys * H + h) * D + 8 * lane);
+        cs[0] = make_float4(gs[0], gs[1], gs[2], gs[3]);
+        cs[1] = make_float4(gs[4], gs[5], gs[6], gs[7]);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float m = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(x[k][e]));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        gs[k] = m > 0.f ? __fdiv_rn(m, 448.0f) : 0.f;
+        if ((lane & 7) == 0) v_tok_all[(phys * H + h) * P + (lane >> 3) + 4 * k] = gs[k];
+      }
+    }
+    float pm = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (tensor == 0 || e < 4) pm = fmaxf(pm, gs[e]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, o));
+    if (lane == 0) *sc = pm;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float s0 = tensor == 0 ? gs[2 * e] : gs[k], s1 = tensor == 0 ? gs[2 * e + 1] : gs[k];
+        const float a = s0 > 0.f ? __fdiv_rn(x[k][2 * e], s0) : 0.f;
+        const float b = s1 > 0.f ? __fdiv_rn(x[k][2 * e + 1], s1) : 0.f;
+        w[e] = e4m3x2(a, b);
+      }
+      reinterpret_cast<uint2*>(dst)[lane + 32 * k] = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+    }
+    return;
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 0.f;
@@ -149,12 +206,13 @@ cudaError_t launch_append_layers(cudaStream_t s, int elem_bytes, const AppendBat
 cudaError_t launch_append_fp8_layers(cudaStream_t s, const AppendBatch& in, const LayerStarts& starts, int n_layers,
                                      uint8_t* k_pool_all, uint8_t* v_pool_all, float* k_scale_all,
                                      float* v_scale_all, const Entry* entries_all, int pool_pages, int n_pages, int T,
-                                     int H, int D, int P) {
+                                     int H, int D, int P, float* k_chan_all, float* v_tok_all) {
+  if (k_chan_all && (D != 64 || P != 16 || !v_tok_all)) return cudaErrorInvalidValue;
   const int items = n_layers * n_pages * H * 2;
   const int warps = 8;
-  append_fp8_kernel<<<(items + warps - 1) / warps, warps * 32, 0, s>>>(in, starts, n_layers, k_pool_all, v_pool_all,
-                                                                       k_scale_all, v_scale_all, entries_all,
-                                                                       pool_pages, n_pages, T, H, D, P);
+  append_fp8_kernel<<<(items + warps - 1) / warps, warps * 32, 0, s>>>(
+      in, starts, n_layers, k_pool_all, v_pool_all, k_scale_all, v_scale_all, k_chan_all, v_tok_all, entries_all,
+      pool_pages, n_pages, T, H, D, P);
   return cudaGetLastError();
 }
 
@@ -171,14 +229,15 @@ cudaError_t launch_append(cudaStream_t s, int elem_bytes, const void* k, const v
 
 cudaError_t launch_append_fp8(cudaStream_t s, const void* k, const void* v, uint8_t* k_pool, uint8_t* v_pool,
                               float* k_scale, float* v_scale, const Entry* entries, int n_pages, int T, int H,
-                              int D, int P) {
+                              int D, int P, float* k_chan, float* v_tok) {
   AppendBatch in{};
   in.k[0] = k;
   in.v[0] = v;
   LayerStarts st{};
   st.first_layer = 0;
   st.start[0] = 0;
-  return launch_append_fp8_layers(s, in, st, 1, k_pool, v_pool, k_scale, v_scale, entries, 0, n_pages, T, H, D, P);
+  return launch_append_fp8_layers(s, in, st, 1, k_pool, v_pool, k_scale, v_scale, entries, 0, n_pages, T, H, D, P,
+                                  k_chan, v_tok);
 }
 
 }  // namespace kvc

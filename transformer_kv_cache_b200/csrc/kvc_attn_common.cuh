@@ -25,6 +25,8 @@ struct TcParams {
   int* err;
   int head_pages;               // > 0: per-head page lists (see TcAttnArgs)
   int* split_cnt;               // [H][q_tiles] zeroed counters: the last split CTA merges (bf16 kernel)
+  const float* k_chan;          // dimension-adaptive FP8: [pool page][head][64] K channel scales
+  const float* v_tok;           // dimension-adaptive FP8: [pool page][head][16] V token scales
 };
 
 __device__ __forceinline__ float ex2(float x) {

@@ -88,7 +88,38 @@ __device__ __forceinline__ float page_scale(const TcParams& p, const float* sc, 
   return phys >= 0 ? __ldg(&sc[(p.page_base + phys) * p.H + h]) : 0.f;
 }
 
-template <int P>
+// Dimension-adaptive scales a converter lane needs for one tile: for each of its half's two
+// pages, the K scales of its 8-dim chunk and the page's K scale, and the V scales of its
+// rows r0 + 4i (slot r0 + 4 (i mod 4) of page i / 4). Zero for the past-the-end page.
+struct DaScales {
+  float kc[2][8];
+  float ks[2];
+  float vt[8];
+};
+__device__ __forceinline__ void load_da_scales(const TcParams& p, int phys_lane, int h, int r0, int c0, DaScales& d) {
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    const int phys = __shfl_sync(0xffffffffu, phys_lane, g);
+    if (phys >= 0) {
+      const long long base = (p.page_base + phys) * p.H + h;
+      const float4 a = __ldg(reinterpret_cast<const float4*>(p.k_chan + base * 64 + 8 * c0));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(p.k_chan + base * 64 + 8 * c0) + 1);
+      d.kc[g][0] = a.x; d.kc[g][1] = a.y; d.kc[g][2] = a.z; d.kc[g][3] = a.w;
+      d.kc[g][4] = b.x; d.kc[g][5] = b.y; d.kc[g][6] = b.z; d.kc[g][7] = b.w;
+      d.ks[g] = __ldg(&p.k_scale[base]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d.vt[4 * g + i] = __ldg(&p.v_tok[base * 16 + r0 + 4 * i]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) d.kc[g][e] = 0.f;
+      d.ks[g] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d.vt[4 * g + i] = 0.f;
+    }
+  }
+}
+
+template <int P, bool kDA>
 __global__ void __launch_bounds__(tc8::kThreads, 1)
     attn_fp8_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v, const TcParams p) {
@@ -189,6 +220,8 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
       int pq2 = page_entry(p, (tile0 + 2) * kPPT + gl).x;
       int pq4n = page_entry(p, (tile0 + 3) * kPPT + gl).x;
       float vsn = page_scale(p, p.v_scale, pq0, h);
+      DaScales dan;                                     // dimension-adaptive scales of the next tile
+      if (kDA) load_da_scales(p, pq0, h, lane >> 3, lane & 7, dan);
 #define KVC_FP8_ISSUE(t, phys)                                                                      \
   do {                                                                                              \
     const int st_ = (t) % kCodeStages;                                                              \
@@ -228,6 +261,20 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
         uint32_t rv[kPPH];
 #pragma unroll
         for (int g = 0; g < kPPH; ++g) rv[g] = f16x2_splat(__shfl_sync(0xffffffffu, fvj, g));
+        // dimension-adaptive factors of tile j: K chunk scale over the page's K scale (the
+        // page's logit factor carries the rest), V token scale over the V reference
+        uint32_t kf[2][4], rvr[8];
+        if (kDA) {
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            const float inv = dan.ks[g] > 0.f ? 1.f / dan.ks[g] : 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) kf[g][e] = pack_f16(dan.kc[g][2 * e] * inv, dan.kc[g][2 * e + 1] * inv);
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) rvr[i] = f16x2_splat(dan.vt[i] * iv);
+          load_da_scales(p, pq1, h, lane >> 3, lane & 7, dan);   // tile j + 1
+        }
         // converted stage st is free once the MMAs of tile j - kStages have completed
         if (j >= kStages &&
             !__all_sync(0xffffffffu, mbar_wait_bounded(&kv_empty[st], ((j / kStages) - 1) & 1, abort_flag, p.err))) {
@@ -251,10 +298,17 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
           ko.y = f16x2_of_e4m3x2(kc.x >> 16);
           ko.z = f16x2_of_e4m3x2(kc.y);
           ko.w = f16x2_of_e4m3x2(kc.y >> 16);
-          vo.x = hmul2(f16x2_of_e4m3x2(vc.x), rv[i >> 2]);
-          vo.y = hmul2(f16x2_of_e4m3x2(vc.x >> 16), rv[i >> 2]);
-          vo.z = hmul2(f16x2_of_e4m3x2(vc.y), rv[i >> 2]);
-          vo.w = hmul2(f16x2_of_e4m3x2(vc.y >> 16), rv[i >> 2]);
+          if (kDA) {
+            ko.x = hmul2(ko.x, kf[i >> 2][0]);
+            ko.y = hmul2(ko.y, kf[i >> 2][1]);
+            ko.z = hmul2(ko.z, kf[i >> 2][2]);
+            ko.w = hmul2(ko.w, kf[i >> 2][3]);
+          }
+          const uint32_t vr = kDA ? rvr[i] : rv[i >> 2];
+          vo.x = hmul2(f16x2_of_e4m3x2(vc.x), vr);
+          vo.y = hmul2(f16x2_of_e4m3x2(vc.x >> 16), vr);
+          vo.z = hmul2(f16x2_of_e4m3x2(vc.y), vr);
+          vo.w = hmul2(f16x2_of_e4m3x2(vc.y >> 16), vr);
           const int off = i * 512 + ((i & 1) ? dst_odd : dst_even);
           *reinterpret_cast<uint4*>(kdst + off) = ko;
           *reinterpret_cast<uint4*>(vdst + off) = vo;
@@ -563,12 +617,18 @@ cudaError_t launch_attn_fp8_kernel(cudaStream_t s, const CUtensorMap& tq, const 
                                    const TcParams& prm, int grid) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fp8_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_fp8_kernel<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(tc8::kSmemBytes));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_fp8_kernel<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(tc8::kSmemBytes));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  attn_fp8_kernel<16><<<grid, tc8::kThreads, tc8::kSmemBytes, s>>>(tq, tk, tv, prm);
+  if (prm.k_chan)
+    attn_fp8_kernel<16, true><<<grid, tc8::kThreads, tc8::kSmemBytes, s>>>(tq, tk, tv, prm);
+  else
+    attn_fp8_kernel<16, false><<<grid, tc8::kThreads, tc8::kSmemBytes, s>>>(tq, tk, tv, prm);
   return cudaGetLastError();
 }
 

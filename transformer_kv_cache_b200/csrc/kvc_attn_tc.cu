@@ -716,6 +716,8 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   prm.part_lse = a.part_lse;
   prm.err = a.err;
   prm.head_pages = a.head_pages;
+  prm.k_chan = a.fp8 ? a.k_chan : nullptr;
+  prm.v_tok = a.fp8 ? a.v_tok : nullptr;
   // the last split CTA merges when a merge is one copy round per half row (up to four
   // splits); with more, a separate combine launch is faster (measured at 9 splits)
   prm.split_cnt = a.fp8 || splits > 4 ? nullptr : a.split_cnt;

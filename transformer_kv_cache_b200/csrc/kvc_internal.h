@@ -76,6 +76,8 @@ struct Cache {
   void* cmp_scratch = nullptr;
   size_t cmp_scratch_bytes = 0;
   // attention split scratch (partial O and log-sum-exp)
+  float* k_chan = nullptr;          // dimension-adaptive FP8: [layer][page][head][D] K channel scales
+  float* v_tok = nullptr;           // dimension-adaptive FP8: [layer][page][head][P] V token scales
   float* part_o = nullptr;
   float* part_lse = nullptr;
   int* split_cnt = nullptr;         // [H][q_tiles] attention split counters (zero between launches)
@@ -153,11 +155,11 @@ cudaError_t launch_append_layers(cudaStream_t s, int elem_bytes, const AppendBat
 cudaError_t launch_append_fp8_layers(cudaStream_t s, const AppendBatch& in, const LayerStarts& starts, int n_layers,
                                      uint8_t* k_pool_all, uint8_t* v_pool_all, float* k_scale_all,
                                      float* v_scale_all, const Entry* entries_all, int pool_pages, int n_pages, int T,
-                                     int H, int D, int P);
+                                     int H, int D, int P, float* k_chan_all = nullptr, float* v_tok_all = nullptr);
 // Append with FP8 E4M3 absmax quantisation per (page, head); bf16 input.
 cudaError_t launch_append_fp8(cudaStream_t s, const void* k, const void* v, uint8_t* k_pool, uint8_t* v_pool,
                               float* k_scale, float* v_scale, const Entry* entries, int n_pages, int T, int H,
-                              int D, int P);
+                              int D, int P, float* k_chan = nullptr, float* v_tok = nullptr);
 
 // SIMT attention (fp32 arithmetic) over pages [0, n_pages) of a layer.
 cudaError_t launch_attn_simt(cudaStream_t s, int io_dtype, int kv_dtype, const void* q, void* o,
@@ -187,6 +189,8 @@ struct TcAttnArgs {
   int head_pages;                   // > 0: one page list per head, head h's pages at
                                     // entries + h * head_pages, pool page index page_base +
                                     // h * head_pages + phys (single-head pages)
+  const float* k_chan = nullptr;    // dimension-adaptive FP8 scales (FP8 kernel), or null
+  const float* v_tok = nullptr;
   int* split_cnt = nullptr;         // [H][q_tiles] zeroed counters (bf16 kernel): the last
                                     // split CTA of a query tile merges, no combine launch
 };
