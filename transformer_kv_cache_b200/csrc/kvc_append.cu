@@ -22,6 +22,8 @@ namespace kvc {
 __global__ void append_kernel(AppendBatch in, LayerStarts starts, int n_layers, uint4* k_pool_all, uint4* v_pool_all,
                               const Entry* __restrict__ entries_all, int pool_pages, int n_pages, int T, int H,
                               int chunks_per_row, int P) {
+  griddep_wait();
+  griddep_launch_dependents();
   const long long per_tensor = static_cast<long long>(n_pages) * H * P * chunks_per_row;
   const long long per_layer = 2 * per_tensor;
   const long long total = per_layer * n_layers;
@@ -70,6 +72,8 @@ __global__ void append_fp8_kernel(AppendBatch in, LayerStarts starts, int n_laye
                                   uint8_t* v_pool_all, float* k_scale_all, float* v_scale_all, float* k_chan_all,
                                   float* v_tok_all, const Entry* __restrict__ entries_all, int pool_pages,
                                   int n_pages, int T, int H, int D, int P) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int warps_per_block = blockDim.x / 32;
   const int gw = blockIdx.x * warps_per_block + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
@@ -197,10 +201,9 @@ cudaError_t launch_append_layers(cudaStream_t s, int elem_bytes, const AppendBat
   long long blocks = (total + threads - 1) / threads;
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
-  append_kernel<<<static_cast<int>(blocks), threads, 0, s>>>(in, starts, n_layers, static_cast<uint4*>(k_pool_all),
-                                                              static_cast<uint4*>(v_pool_all), entries_all, pool_pages,
-                                                              n_pages, T, H, chunks_per_row, P);
-  return cudaGetLastError();
+  return launch_pdl(append_kernel, dim3(static_cast<int>(blocks)), dim3(threads), 0, s, in, starts, n_layers,
+                    static_cast<uint4*>(k_pool_all), static_cast<uint4*>(v_pool_all), entries_all, pool_pages, n_pages,
+                    T, H, chunks_per_row, P);
 }
 
 cudaError_t launch_append_fp8_layers(cudaStream_t s, const AppendBatch& in, const LayerStarts& starts, int n_layers,
@@ -210,10 +213,9 @@ cudaError_t launch_append_fp8_layers(cudaStream_t s, const AppendBatch& in, cons
   if (k_chan_all && (D != 64 || P != 16 || !v_tok_all)) return cudaErrorInvalidValue;
   const int items = n_layers * n_pages * H * 2;
   const int warps = 8;
-  append_fp8_kernel<<<(items + warps - 1) / warps, warps * 32, 0, s>>>(
-      in, starts, n_layers, k_pool_all, v_pool_all, k_scale_all, v_scale_all, k_chan_all, v_tok_all, entries_all,
-      pool_pages, n_pages, T, H, D, P);
-  return cudaGetLastError();
+  return launch_pdl(append_fp8_kernel, dim3((items + warps - 1) / warps), dim3(warps * 32), 0, s, in, starts,
+                    n_layers, k_pool_all, v_pool_all, k_scale_all, v_scale_all, k_chan_all, v_tok_all, entries_all,
+                    pool_pages, n_pages, T, H, D, P);
 }
 
 cudaError_t launch_append(cudaStream_t s, int elem_bytes, const void* k, const void* v, void* k_pool,

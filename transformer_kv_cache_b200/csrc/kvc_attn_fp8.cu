@@ -123,6 +123,8 @@ template <int P, bool kDA>
 __global__ void __launch_bounds__(tc8::kThreads, 1)
     attn_fp8_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v, const TcParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   using namespace tc8;
   constexpr int kPPT = kBN / P;               // pages per KV tile
   constexpr int kPPH = kPPT / 2;              // pages per converter half
@@ -626,10 +628,8 @@ cudaError_t launch_attn_fp8_kernel(cudaStream_t s, const CUtensorMap& tq, const 
     attr_set = true;
   }
   if (prm.k_chan)
-    attn_fp8_kernel<16, true><<<grid, tc8::kThreads, tc8::kSmemBytes, s>>>(tq, tk, tv, prm);
-  else
-    attn_fp8_kernel<16, false><<<grid, tc8::kThreads, tc8::kSmemBytes, s>>>(tq, tk, tv, prm);
-  return cudaGetLastError();
+    return launch_pdl(attn_fp8_kernel<16, true>, dim3(grid), dim3(tc8::kThreads), tc8::kSmemBytes, s, tq, tk, tv, prm);
+  return launch_pdl(attn_fp8_kernel<16, false>, dim3(grid), dim3(tc8::kThreads), tc8::kSmemBytes, s, tq, tk, tv, prm);
 }
 
 }  // namespace kvc

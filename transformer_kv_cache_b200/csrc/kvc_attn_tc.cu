@@ -170,6 +170,8 @@ template <int P, bool kPerHead>
 __global__ void __launch_bounds__(tc::kThreads, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const TcParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   using namespace tc;
   constexpr int kPPT = kBN / P;               // pages per KV tile
   extern __shared__ uint8_t smem_raw[];
@@ -570,6 +572,8 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
 // (row, head); lane covers two of the 64 dims.
 __global__ void combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                                __nv_bfloat16* __restrict__ out, int T, int H, int q_tiles, int splits) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= T * H) return;
@@ -727,19 +731,19 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
     e = launch_attn_fp8_kernel(s, tq, *a.tmap_k, *a.tmap_v, prm, grid);
   } else {
     if (a.head_pages)
-      attn_tc_kernel<16, true><<<grid, tc::kThreads, tc::kSmemBytes, s>>>(tq, *a.tmap_k, *a.tmap_v, prm);
+      e = launch_pdl(attn_tc_kernel<16, true>, dim3(grid), dim3(tc::kThreads), tc::kSmemBytes, s, tq, *a.tmap_k,
+                     *a.tmap_v, prm);
     else
-      attn_tc_kernel<16, false><<<grid, tc::kThreads, tc::kSmemBytes, s>>>(tq, *a.tmap_k, *a.tmap_v, prm);
-    e = cudaGetLastError();
+      e = launch_pdl(attn_tc_kernel<16, false>, dim3(grid), dim3(tc::kThreads), tc::kSmemBytes, s, tq, *a.tmap_k,
+                     *a.tmap_v, prm);
   }
   if (e != cudaSuccess) return e;
   if (launched) *launched = 1;
   if (splits > 1 && !prm.split_cnt) {
     const long long warps = static_cast<long long>(a.T) * a.H;
     const int threads = 256;
-    combine_kernel<<<static_cast<int>((warps * 32 + threads - 1) / threads), threads, 0, s>>>(
-        a.part_o, a.part_lse, static_cast<__nv_bfloat16*>(a.o), a.T, a.H, q_tiles, splits);
-    e = cudaGetLastError();
+    e = launch_pdl(combine_kernel, dim3(static_cast<int>((warps * 32 + threads - 1) / threads)), dim3(threads), 0, s,
+                   a.part_o, a.part_lse, static_cast<__nv_bfloat16*>(a.o), a.T, a.H, q_tiles, splits);
     if (launched) *launched = 2;
   }
   if (splits_used) *splits_used = splits;

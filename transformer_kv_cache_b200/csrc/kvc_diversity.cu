@@ -38,6 +38,8 @@ __global__ void __launch_bounds__(256) append_heads_kernel(AppendBatch in, int f
                                                            const Entry* __restrict__ entries_all,
                                                            int64_t* tok_id_all, int pool_pages, int n_pages, int T,
                                                            int H, int P, long long frame_base) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int slots = n_pages * P;
   const long long total = static_cast<long long>(n_layers) * slots * H;
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
@@ -198,6 +200,8 @@ __global__ void __cluster_dims__(kPruneCluster, 1, 1) __launch_bounds__(kPruneTh
     Entry* entries_layer, __nv_bfloat16* k_pool, __nv_bfloat16* v_pool, uint32_t* bitmap_layer, int words,
     int64_t* tok_id_layer, int pool_pages, int first, int n_entries, int keep, int P, int B, double* sums_layer,
     int* err) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ int s_warp[32];
   __shared__ double s_mu[kDivD];
@@ -534,10 +538,9 @@ cudaError_t launch_append_heads(cudaStream_t s, const AppendBatch& in, int first
   const int threads = 256;
   long long blocks = (total + threads - 1) / threads;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  append_heads_kernel<<<static_cast<int>(blocks), threads, 0, s>>>(
-      in, first_layer, starts, n_layers, static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), entries_all,
-      tok_id_all, pool_pages, n_pages, T, H, P, static_cast<long long>(frame) * T);
-  return cudaGetLastError();
+  return launch_pdl(append_heads_kernel, dim3(static_cast<int>(blocks)), dim3(threads), 0, s,
+                    in, first_layer, starts, n_layers, static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool),
+                    entries_all, tok_id_all, pool_pages, n_pages, T, H, P, static_cast<long long>(frame) * T);
 }
 
 int diversity_prune_max_candidates() { return kPruneCluster * kPruneMaxB; }
@@ -560,10 +563,10 @@ cudaError_t launch_diversity_prune(cudaStream_t s, Entry* entries_layer, void* k
     if (e != cudaSuccess) return e;
     attr = smem;
   }
-  diversity_prune_kernel<<<H * kPruneCluster, kPruneThreads, smem, s>>>(
-      entries_layer, static_cast<__nv_bfloat16*>(k_pool), static_cast<__nv_bfloat16*>(v_pool), bitmap_layer, words,
-      tok_id_layer, pool_pages, first_cand_entry, n_cand_entries, keep, P, B, sums_layer, err);
-  return cudaGetLastError();
+  return launch_pdl(diversity_prune_kernel, dim3(H * kPruneCluster), dim3(kPruneThreads), smem, s,
+                    entries_layer, static_cast<__nv_bfloat16*>(k_pool), static_cast<__nv_bfloat16*>(v_pool),
+                    bitmap_layer, words, tok_id_layer, pool_pages, first_cand_entry, n_cand_entries, keep, P, B,
+                    sums_layer, err);
 }
 
 }  // namespace kvc

@@ -12,6 +12,24 @@
 
 namespace kvc {
 
+// Launch with programmatic stream serialization: the kernel may start launching while the
+// previous kernel of the stream finishes. Every kernel launched this way calls
+// griddep_wait() (sm100_ptx.cuh) before it touches global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // A committed frame's pages are a contiguous run of entries in the layer's page list.
 struct FrameRec {
   int32_t frame = -1;

@@ -51,6 +51,8 @@ __global__ void __launch_bounds__(kMgrThreads) mgr_alloc_kernel(Entry* entries_a
                                                                  int pool_pages, LayerStarts starts, int group,
                                                                  int n_new, int owner, int valid_full, int valid_last,
                                                                  int* err) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ int s_warp[32];
   const int layer = starts.first_layer + blockIdx.x;
   Entry* entries = entries_all + static_cast<size_t>(layer) * pool_pages;
@@ -97,6 +99,8 @@ __global__ void __launch_bounds__(kMgrThreads) mgr_alloc_kernel(Entry* entries_a
 // in-place move is safe.
 __global__ void __launch_bounds__(kMgrThreads) mgr_remove_kernel(Entry* entries, uint32_t* bitmap, int n, int a,
                                                                   int b, int* err) {
+  griddep_wait();
+  griddep_launch_dependents();
   for (int i = a + threadIdx.x; i < b; i += kMgrThreads) {
     const int page = entries[i].x;
     const uint32_t bit = 1u << (page & 31);
@@ -134,29 +138,30 @@ cudaError_t launch_mgr_alloc(cudaStream_t s, Entry* entries, uint32_t* bitmap, i
   LayerStarts st{};
   st.first_layer = 0;
   st.start[0] = start;
-  mgr_alloc_kernel<<<1, kMgrThreads, 0, s>>>(entries, bitmap, words, pool_pages, st, 1, n_new, owner, valid_full,
-                                             valid_last, err);
-  return cudaGetLastError();
+  return launch_pdl(mgr_alloc_kernel, dim3(1), dim3(kMgrThreads), 0, s,
+                    entries, bitmap, words, pool_pages, st, 1, n_new, owner, valid_full, valid_last, err);
 }
 
 cudaError_t launch_mgr_alloc_layers(cudaStream_t s, Entry* entries_all, uint32_t* bitmap_all, int words,
                                     int pool_pages, const LayerStarts& starts, int n_lists, int n_new, int owner,
                                     int valid_full, int valid_last, int* err, int group) {
-  mgr_alloc_kernel<<<n_lists, kMgrThreads, 0, s>>>(entries_all, bitmap_all, words, pool_pages, starts, group, n_new,
-                                                   owner, valid_full, valid_last, err);
-  return cudaGetLastError();
+  return launch_pdl(mgr_alloc_kernel, dim3(n_lists), dim3(kMgrThreads), 0, s,
+                    entries_all, bitmap_all, words, pool_pages, starts, group, n_new, owner, valid_full, valid_last,
+                    err);
 }
 
 cudaError_t launch_mgr_remove(cudaStream_t s, Entry* entries, uint32_t* bitmap, int n_entries, int a, int b,
                               int* err) {
-  mgr_remove_kernel<<<1, kMgrThreads, 0, s>>>(entries, bitmap, n_entries, a, b, err);
-  return cudaGetLastError();
+  return launch_pdl(mgr_remove_kernel, dim3(1), dim3(kMgrThreads), 0, s,
+                    entries, bitmap, n_entries, a, b, err);
 }
 
 // One 16-byte chunk per thread over (page, head, slot past the kept tokens, chunk) for K
 // and V; the first thread of each page writes its valid count.
 __global__ void trim_pages_kernel(uint8_t* k_pool, uint8_t* v_pool, Entry* entries, int first, int n_pages, int keep,
                                   int H, int P, int chunks) {
+  griddep_wait();
+  griddep_launch_dependents();
   const long long per_tensor = static_cast<long long>(n_pages) * H * P * chunks;
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < 2 * per_tensor;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -187,9 +192,8 @@ cudaError_t launch_trim_pages(cudaStream_t s, uint8_t* k_pool_layer, uint8_t* v_
   const int threads = 256;
   long long blocks = (total + threads - 1) / threads;
   if (blocks > 1184) blocks = 1184;
-  trim_pages_kernel<<<static_cast<int>(blocks), threads, 0, s>>>(k_pool_layer, v_pool_layer, entries, first, n_pages,
-                                                                 keep, H, P, chunks);
-  return cudaGetLastError();
+  return launch_pdl(trim_pages_kernel, dim3(static_cast<int>(blocks)), dim3(threads), 0, s,
+                    k_pool_layer, v_pool_layer, entries, first, n_pages, keep, H, P, chunks);
 }
 
 cudaError_t launch_debug_wait(cudaStream_t s, int* flag, int* err, long long timeout_ns) {

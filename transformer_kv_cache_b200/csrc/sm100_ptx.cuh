@@ -204,6 +204,17 @@ __host__ __device__ constexpr uint32_t idesc_f16kind(uint32_t fmt, int M, int N,
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start before the previous
+// kernel of the stream has finished. griddep_wait() returns once that kernel has
+// completed and its memory is visible; every such kernel calls it before touching global
+// memory. griddep_launch_dependents() lets the next kernel start launching (its CTAs then
+// wait in their own griddep_wait()). Both are no-ops for a normal launch.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ asynchronous copies
 // Global -> shared copies that bypass the registers; completion by commit + wait.
 __device__ __forceinline__ void cp_async16(void* dst_smem, const void* src) {
