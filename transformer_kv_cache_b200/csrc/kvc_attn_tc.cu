@@ -569,7 +569,9 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
 }
 
 // Merge split partials: O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M). One warp per
-// (row, head); lane covers two of the 64 dims.
+// (row, head): lane s (and s + 32) loads split s's log-sum-exp, so the maximum and the
+// weights take one round of loads and warp shuffles; then each lane accumulates two of
+// the 64 dims over the splits, four partial rows in flight at a time (up to 64 splits).
 __global__ void combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                                __nv_bfloat16* __restrict__ out, int T, int H, int q_tiles, int splits) {
   griddep_wait();
@@ -579,19 +581,25 @@ __global__ void combine_kernel(const float* __restrict__ part_o, const float* __
   if (gw >= T * H) return;
   const int t = gw / H, h = gw % H;
   const int qt = t / tc::kBM, r = t % tc::kBM;
-  float M = -INFINITY;
+  const long long pi0 = static_cast<long long>(h) * splits * q_tiles + qt;
+  auto row_of = [&](int s) { return (pi0 + static_cast<long long>(s) * q_tiles) * tc::kBM + r; };
+  const float l0 = lane < splits ? __ldg(&part_lse[row_of(lane)]) : -INFINITY;
+  const float l1 = lane + 32 < splits ? __ldg(&part_lse[row_of(lane + 32)]) : -INFINITY;
+  float M = fmaxf(l0, l1);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float w0 = lane < splits ? exp2f(l0 - M) : 0.f;
+  const float w1 = lane + 32 < splits ? exp2f(l1 - M) : 0.f;
+  float ws = w0 + w1;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll 4
   for (int s = 0; s < splits; ++s) {
-    const long long pi = (static_cast<long long>(h) * splits + s) * q_tiles + qt;
-    M = fmaxf(M, part_lse[pi * tc::kBM + r]);
-  }
-  float a0 = 0.f, a1 = 0.f, ws = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const long long pi = (static_cast<long long>(h) * splits + s) * q_tiles + qt;
-    const float w = exp2f(part_lse[pi * tc::kBM + r] - M);
-    const float2 o = reinterpret_cast<const float2*>(part_o + (pi * tc::kBM + r) * tc::kHD)[lane];
+    const float w = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
+    const float2 o = __ldg(reinterpret_cast<const float2*>(part_o + row_of(s) * tc::kHD) + lane);
     a0 = fmaf(w, o.x, a0);
     a1 = fmaf(w, o.y, a1);
-    ws += w;
   }
   const float inv = 1.f / ws;
   reinterpret_cast<__nv_bfloat162*>(out + (static_cast<long long>(t) * H + h) * tc::kHD)[lane] =
@@ -691,6 +699,7 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   const int part_units = q_tiles * a.H;       // 128-row partial tiles per split
   int splits = a.splits > 0 ? a.splits : choose_splits(units, total_tiles, slots, a.fp8);
   if (splits > total_tiles) splits = total_tiles;
+  if (splits > 64) splits = 64;                  // the combine takes up to 64 partials per row
   int tps = (total_tiles + splits - 1) / splits;
   splits = (total_tiles + tps - 1) / tps;
   if (splits > 1 && static_cast<size_t>(part_units) * splits > a.part_rows) {
