@@ -565,7 +565,7 @@ kvc_status kvc_append_frame(kvc_cache* c, int32_t layer, int32_t frame_idx, cons
                           layer_group_scales(c, c->v_tok, layer, P));
   } else {
     e = launch_append(c->stream, static_cast<int>(c->elem_kv), k_dev, v_dev, layer_pool(c, c->k_pool, layer),
-                      layer_pool(c, c->v_pool, layer), E + L.n_entries, n, T, g.num_heads, g.head_dim, P);
+                      layer_pool(c, c->v_pool, layer), E + L.n_entries, n, T, g.num_heads, g.head_dim, P, c->d_err);
   }
   if (e != cudaSuccess) return cuda_fail(c, e, "append");
   c->launches++;
@@ -639,7 +639,7 @@ kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const void* con
                                    c->pool_pages, n, T, g.num_heads, g.head_dim, P, c->k_chan, c->v_tok);
     else
       e = launch_append_layers(c->stream, static_cast<int>(c->elem_kv), in, st, nl, c->k_pool, c->v_pool, c->entries,
-                               c->pool_pages, n, T, g.num_heads, g.head_dim, P);
+                               c->pool_pages, n, T, g.num_heads, g.head_dim, P, c->d_err);
     if (e != cudaSuccess) return cuda_fail(c, e, "append (all layers)");
     c->launches++;
   }

@@ -17,25 +17,27 @@
 
 namespace kvc {
 
-// One 16-byte chunk per thread-iteration, over every (layer of the batch, tensor, page,
-// head, slot, chunk) in destination order.
+constexpr int kBulkAppendMaxSmem = 96 * 1024;   // two pages staged per CTA
+
+// One thread per destination row of one tensor: (layer of the batch, tensor, page, head,
+// slot), slots fastest, so a warp writes 32 consecutive rows of a (page, head) block. The
+// thread decodes its indices and reads the page entry once, then moves the row 8 chunks
+// of 16 bytes at a time, all 8 loads issued before their stores. Slots past T get zeros.
 __global__ void append_kernel(AppendBatch in, LayerStarts starts, int n_layers, uint4* k_pool_all, uint4* v_pool_all,
                               const Entry* __restrict__ entries_all, int pool_pages, int n_pages, int T, int H,
                               int chunks_per_row, int P) {
   griddep_wait();
   griddep_launch_dependents();
-  const long long per_tensor = static_cast<long long>(n_pages) * H * P * chunks_per_row;
-  const long long per_layer = 2 * per_tensor;
-  const long long total = per_layer * n_layers;
+  constexpr int kGroup = 8;
+  const long long rows_per_tensor = static_cast<long long>(n_pages) * H * P;
+  const long long total = 2 * rows_per_tensor * n_layers;
   const long long page_chunks = static_cast<long long>(H) * P * chunks_per_row;
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int bl = static_cast<int>(idx / per_layer);
-    long long r = idx - static_cast<long long>(bl) * per_layer;
-    const bool is_v = r >= per_tensor;
-    if (is_v) r -= per_tensor;
-    const int c = static_cast<int>(r % chunks_per_row);
-    r /= chunks_per_row;
+    const int bl = static_cast<int>(idx / (2 * rows_per_tensor));
+    long long r = idx - static_cast<long long>(bl) * 2 * rows_per_tensor;
+    const bool is_v = r >= rows_per_tensor;
+    if (is_v) r -= rows_per_tensor;
     const int slot = static_cast<int>(r % P);
     r /= P;
     const int h = static_cast<int>(r % H);
@@ -43,11 +45,70 @@ __global__ void append_kernel(AppendBatch in, LayerStarts starts, int n_layers, 
     const int tok = g * P + slot;
     const long long layer = starts.first_layer + bl;
     const int phys = __ldg(&entries_all[layer * pool_pages + starts.start[bl] + g].x);
-    uint4 val = make_uint4(0, 0, 0, 0);
-    const uint4* src = static_cast<const uint4*>(is_v ? in.v[bl] : in.k[bl]);
-    if (tok < T) val = __ldg(&src[(static_cast<long long>(tok) * H + h) * chunks_per_row + c]);
-    uint4* dst = (is_v ? v_pool_all : k_pool_all) + (layer * pool_pages + phys) * page_chunks;
-    dst[(static_cast<long long>(h) * P + slot) * chunks_per_row + c] = val;
+    const uint4* src = static_cast<const uint4*>(is_v ? in.v[bl] : in.k[bl]) +
+                       (static_cast<long long>(tok) * H + h) * chunks_per_row;
+    uint4* dst = (is_v ? v_pool_all : k_pool_all) + (layer * pool_pages + phys) * page_chunks +
+                 (static_cast<long long>(h) * P + slot) * chunks_per_row;
+    for (int c0 = 0; c0 < chunks_per_row; c0 += kGroup) {
+      uint4 val[kGroup];
+#pragma unroll
+      for (int c = 0; c < kGroup; ++c)
+        if (c0 + c < chunks_per_row) val[c] = tok < T ? __ldg(src + c0 + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int c = 0; c < kGroup; ++c)
+        if (c0 + c < chunks_per_row) dst[c0 + c] = val[c];
+    }
+  }
+}
+
+// One CTA per (layer of the batch, tensor, page). A page's P tokens x H heads x D dims
+// are contiguous in the source ([T][H][D]) and in the pool ([head][slot][dim]), so the
+// CTA brings them in with one bulk copy, transposes 16-byte chunks in shared memory
+// (tokens past T become zeros) and writes the page out with one bulk copy: every HBM
+// byte moves in large contiguous transfers. The load wait is bounded (error word).
+__global__ void __launch_bounds__(256) append_bulk_kernel(AppendBatch in, LayerStarts starts, int n_layers,
+                                                          uint8_t* k_pool_all, uint8_t* v_pool_all,
+                                                          const Entry* __restrict__ entries_all, int pool_pages,
+                                                          int n_pages, int T, int H, int row_bytes, int P, int* err) {
+  griddep_wait();
+  griddep_launch_dependents();
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const int page_bytes = P * H * row_bytes;
+  uint4* src_s = reinterpret_cast<uint4*>(sm);                 // [slot][head][chunk]
+  uint4* dst_s = reinterpret_cast<uint4*>(sm + page_bytes);    // [head][slot][chunk]
+  const int g = blockIdx.x % n_pages;
+  const int tensor = (blockIdx.x / n_pages) & 1;
+  const int bl = blockIdx.x / (2 * n_pages);
+  const int ntok = min(P, T - g * P);
+  const long long layer = starts.first_layer + bl;
+  const uint8_t* src = static_cast<const uint8_t*>(tensor ? in.v[bl] : in.k[bl]) + static_cast<long long>(g) * page_bytes;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(ntok * H * row_bytes));
+    bulk_load(src_s, src, static_cast<uint32_t>(ntok * H * row_bytes), &bar);
+  }
+  const int phys = __ldg(&entries_all[layer * pool_pages + starts.start[bl] + g].x);
+  uint8_t* dst = (tensor ? v_pool_all : k_pool_all) + (layer * pool_pages + phys) * static_cast<long long>(page_bytes);
+  if (!mbar_wait_bounded(&bar, 0, &abort_flag, err)) return;
+  const int chunks = row_bytes / 16;
+  for (int i = threadIdx.x; i < page_bytes / 16; i += blockDim.x) {
+    const int q = i % chunks;
+    const int r = i / chunks;
+    const int slot = r % P, h = r / P;
+    dst_s[i] = slot < ntok ? src_s[(slot * H + h) * chunks + q] : make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_shared();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    bulk_store(dst, dst_s, static_cast<uint32_t>(page_bytes));
+    bulk_store_wait_all();
   }
 }
 
@@ -194,9 +255,25 @@ __global__ void append_fp8_kernel(AppendBatch in, LayerStarts starts, int n_laye
 
 cudaError_t launch_append_layers(cudaStream_t s, int elem_bytes, const AppendBatch& in, const LayerStarts& starts,
                                  int n_layers, void* k_pool_all, void* v_pool_all, const Entry* entries_all,
-                                 int pool_pages, int n_pages, int T, int H, int D, int P) {
+                                 int pool_pages, int n_pages, int T, int H, int D, int P, int* err) {
   const int chunks_per_row = D * elem_bytes / 16;
-  const long long total = 2LL * n_layers * n_pages * H * P * chunks_per_row;
+  if (chunks_per_row < 1) return cudaErrorInvalidValue;
+  const int page_bytes = P * H * D * elem_bytes;
+  if (2 * page_bytes <= kBulkAppendMaxSmem) {
+    // bulk copies through shared memory: the K/V tensors and pools are 16-byte aligned and
+    // every transfer is a whole number of 16-byte rows
+    static int attr = 0;
+    if (2 * page_bytes > attr) {
+      cudaError_t e = cudaFuncSetAttribute(append_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           2 * page_bytes);
+      if (e != cudaSuccess) return e;
+      attr = 2 * page_bytes;
+    }
+    return launch_pdl(append_bulk_kernel, dim3(2 * n_layers * n_pages), dim3(256), static_cast<size_t>(2 * page_bytes),
+                      s, in, starts, n_layers, static_cast<uint8_t*>(k_pool_all), static_cast<uint8_t*>(v_pool_all),
+                      entries_all, pool_pages, n_pages, T, H, D * elem_bytes, P, err);
+  }
+  const long long total = 2LL * n_layers * n_pages * H * P;
   const int threads = 256;
   long long blocks = (total + threads - 1) / threads;
   if (blocks > 148 * 16) blocks = 148 * 16;
@@ -219,14 +296,14 @@ cudaError_t launch_append_fp8_layers(cudaStream_t s, const AppendBatch& in, cons
 }
 
 cudaError_t launch_append(cudaStream_t s, int elem_bytes, const void* k, const void* v, void* k_pool,
-                          void* v_pool, const Entry* entries, int n_pages, int T, int H, int D, int P) {
+                          void* v_pool, const Entry* entries, int n_pages, int T, int H, int D, int P, int* err) {
   AppendBatch in{};
   in.k[0] = k;
   in.v[0] = v;
   LayerStarts st{};
   st.first_layer = 0;
   st.start[0] = 0;
-  return launch_append_layers(s, elem_bytes, in, st, 1, k_pool, v_pool, entries, 0, n_pages, T, H, D, P);
+  return launch_append_layers(s, elem_bytes, in, st, 1, k_pool, v_pool, entries, 0, n_pages, T, H, D, P, err);
 }
 
 cudaError_t launch_append_fp8(cudaStream_t s, const void* k, const void* v, uint8_t* k_pool, uint8_t* v_pool,

@@ -164,12 +164,13 @@ cudaError_t launch_debug_wait(cudaStream_t s, int* flag, int* err, long long tim
 
 // Append (same dtype in and out): K, V [T,H,D] -> pages of entries [0, n_pages).
 cudaError_t launch_append(cudaStream_t s, int elem_bytes, const void* k, const void* v, void* k_pool,
-                          void* v_pool, const Entry* entries, int n_pages, int T, int H, int D, int P);
+                          void* v_pool, const Entry* entries, int n_pages, int T, int H, int D, int P,
+                          int* err = nullptr);
 // Batched append of one frame to layers [starts.first_layer, + n_layers): pools and
 // entries are the all-layer bases (pool_pages pages per layer).
 cudaError_t launch_append_layers(cudaStream_t s, int elem_bytes, const AppendBatch& in, const LayerStarts& starts,
                                  int n_layers, void* k_pool_all, void* v_pool_all, const Entry* entries_all,
-                                 int pool_pages, int n_pages, int T, int H, int D, int P);
+                                 int pool_pages, int n_pages, int T, int H, int D, int P, int* err = nullptr);
 cudaError_t launch_append_fp8_layers(cudaStream_t s, const AppendBatch& in, const LayerStarts& starts, int n_layers,
                                      uint8_t* k_pool_all, uint8_t* v_pool_all, float* k_scale_all,
                                      float* v_scale_all, const Entry* entries_all, int pool_pages, int n_pages, int T,
