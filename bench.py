@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kv-splits", type=int, default=0)
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="replicas (default): one independent stream per rank; heads: one stream, "
+                         "heads sharded over the ranks, O all-gathered")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="vggt_518x378 (default, the headline), vggt_24layer_k4, vggt_budget_16k, vggt_518x518_fp8, "
                          "vggt_infinite_12l, vggt_518x378_joint, vggt_518x378_special")
@@ -257,6 +260,28 @@ def max_over_ranks(value_ms: float, world: int, device) -> float:
 def job_rate(world: int, units_per_rank: int, max_ms: float) -> float:
     """Whole-job throughput: all ranks' units over the slowest rank's time."""
     return world * units_per_rank / (max_ms / 1e3)
+
+
+def head_range(rank: int, world: int, H: int):
+    """Heads [h0, h1) of a rank when one stream's step is sharded by head (attention and
+    cache are independent per head, so each rank holds its heads' pages)."""
+    if H % world:
+        raise ValueError(f"{world} ranks do not divide {H} heads")
+    n = H // world
+    return rank * n, (rank + 1) * n
+
+
+def gather_heads(o_local, world: int):
+    """Every rank's O slice [T, H/N, D] gathered into the full [T, H, D] on every rank,
+    heads in rank order: the one exchange of a head-sharded step (NCCL on GPUs, any
+    torch.distributed backend)."""
+    import torch
+    import torch.distributed as dist
+    if world == 1:
+        return o_local
+    parts = [torch.empty_like(o_local) for _ in range(world)]
+    dist.all_gather(parts, o_local.contiguous())
+    return torch.cat(parts, dim=1)
 
 
 # ------------------------------------------------------------------ our CUDA path
@@ -614,6 +639,70 @@ def run_joint(args):
     return 0
 
 
+def run_sharded(args):
+    """One 518x378 stream with its step sharded by head over the ranks: each rank appends
+    and attends its H/N heads, then O is all-gathered. Total work per step is fixed
+    (strong scaling); the value is the stream's frames/s."""
+    import torch
+    import torch.distributed as dist
+    import transformer_kv_cache_b200 as kvc
+    from kvc_streams import WORKLOADS, FrameStream, keyframe_schedule
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    wl = WORKLOADS[WORKLOAD]
+    T, H, D, S, W = wl.tokens_per_frame, wl.num_heads, wl.head_dim, wl.scale_frames, wl.window_frames
+    h0, h1 = head_range(rank, world, H)
+    stream = torch.cuda.Stream(device=dev)
+    distinct = 4
+    with torch.cuda.stream(stream):
+        st = FrameStream(wl, seed=rank_seed(0), device=dev)            # one stream, the same on every rank
+        frames = [tuple(x[:, h0:h1].contiguous() for x in st.frame(0, t)) for t in range(distinct)]
+        out = torch.empty((T, h1 - h0, D), dtype=torch.bfloat16, device=dev)
+        h = kvc.kvc_create(kvc.config_from_workload(wl.replace(num_heads=h1 - h0), kv_splits=args.kv_splits), stream)
+
+        def step(t):
+            q, k, v = frames[t % distinct]
+            key = keyframe_schedule(t, S, wl.keyframe_interval)
+            kvc.kvc_append_frame(h, 0, t, k, v, key)
+            kvc.kvc_attend(h, 0, q, out)
+            return gather_heads(out, world)
+
+        fill = S + W
+        for t in range(fill + args.warmup):
+            step(t)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            full = step(fill + args.warmup + i)
+        e1.record(stream)
+        stream.synchronize()
+        _, info = kvc.kvc_page_table(h, 0)
+        assert info["device_error"] == 0 and full.shape == (T, H, D)
+        kvc.kvc_destroy(h)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    if rank == 0:
+        line = {"metric": METRIC, "value": 1e3 / ms, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": wl.name, "tokens_per_frame": T, "heads": H, "heads_per_rank": h1 - h0,
+                           "head_dim": D, "window_frames": W, "scale_frames": S, "parallelism": f"heads{world}",
+                           "exchange": "all-gather of O per step (NCCL)"}}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if os.environ.get("KVC_BENCH_WATCHDOG"):
@@ -621,6 +710,8 @@ def main():
         faulthandler.dump_traceback_later(float(os.environ["KVC_BENCH_WATCHDOG"]), exit=False)
     if args.impl == "reference":
         return run_reference(args)
+    if args.shard == "heads":
+        return run_sharded(args)
     if args.workload != WORKLOAD:
         from kvc_streams import WORKLOADS
         if WORKLOADS[args.workload].joint_frames > 0:

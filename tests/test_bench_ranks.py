@@ -73,3 +73,55 @@ def test_reference_arm_nonzero_rank_exits_without_work(monkeypatch, capsys):
     args = type("A", (), {"steps": 3, "warmup": 3, "gpus": 2})()
     assert bench.run_reference(args) == 0
     assert capsys.readouterr().out == ""
+
+
+def _sharded_worker(rank, world, port, results):
+    """Each rank computes its heads of one stream with the fp64 oracle (heads are
+    independent), then bench.gather_heads assembles the full output."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        import bench
+        from kvc_streams import WORKLOADS, FrameStream, keyframe_schedule
+        from oracle import OracleConfig, StreamOracle
+        wl = WORKLOADS["tiny_f32"].replace(num_heads=4)
+        h0, h1 = bench.head_range(rank, world, wl.num_heads)
+        st = FrameStream(wl, seed=bench.rank_seed(0))
+        mine = StreamOracle(OracleConfig.from_workload(wl.replace(num_heads=h1 - h0)))
+        full = StreamOracle(OracleConfig.from_workload(wl))
+        worst = 0.0
+        for t in range(8):
+            key = keyframe_schedule(t, wl.scale_frames, wl.keyframe_interval)
+            qf, kf, vf = (x.to(torch.float64).numpy() for x in st.frame(0, t))
+            mine.append(0, t, kf[:, h0:h1], vf[:, h0:h1], key)
+            o_local = torch.from_numpy(mine.attend(0, qf[:, h0:h1]))
+            o_all = bench.gather_heads(o_local, world)
+            full.append(0, t, kf, vf, key)
+            ref = full.attend(0, qf)
+            worst = max(worst, float(np.abs(o_all.numpy() - ref).max()))
+        results.put((rank, (h0, h1), worst))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_sharded_step_reassembles_the_full_output():
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_sharded_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == [(0, 2), (2, 4)]
+    assert all(r[2] <= 1e-12 for r in res)          # heads are independent: the same answer
+    import bench
+    with pytest.raises(ValueError):
+        bench.head_range(0, 3, 4)
