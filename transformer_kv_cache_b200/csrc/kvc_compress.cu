@@ -552,7 +552,8 @@ __global__ void __launch_bounds__(1024) merge_group_kernel(Scratch sc, int n_src
 // For every eligible target with at least one source: acc = c_j x_j, then acc += c_m x_m
 // for its sources in ascending id, all in fp64; x_j = bf16(acc / sum of counts), for
 // every dimension of K and V; the count becomes the sum. Sources are read before any
-// target is written because no token is both.
+// target is written because no token is both. A thread takes 8 consecutive dims of one
+// head row (16-byte loads of the target and of each source, 8 accumulators).
 __global__ void __launch_bounds__(256) merge_apply_kernel(Scratch sc, int cap_src, int cap_elig,
                                                           __nv_bfloat16* k_pool, __nv_bfloat16* v_pool, int H, int P,
                                                           int D) {
@@ -568,18 +569,31 @@ __global__ void __launch_bounds__(256) merge_apply_kernel(Scratch sc, int cap_sr
   int tot = cj;
   for (int q = begin; q < end; ++q) tot += sc.src_cnt[q];
   const double dtot = static_cast<double>(tot);
-  const int HD = H * D;
-  for (int c = threadIdx.x; c < 2 * HD; c += blockDim.x) {
-    __nv_bfloat16* pool = c < HD ? k_pool : v_pool;
-    const int cc = c < HD ? c : c - HD;
+  const int chunks = H * D / 8;                     // 8-dim chunks of one tensor's row
+  for (int ch = threadIdx.x; ch < 2 * chunks; ch += blockDim.x) {
+    const bool is_v = ch >= chunks;
+    __nv_bfloat16* pool = is_v ? v_pool : k_pool;
+    const int cc = (is_v ? ch - chunks : ch) * 8;
     const long long off = static_cast<long long>(cc / D) * P * D + cc % D;
-    double acc = __dmul_rn(static_cast<double>(cj), static_cast<double>(__bfloat162float(pool[bj + off])));
-#pragma unroll 4
+    const uint4 tj = *reinterpret_cast<const uint4*>(pool + bj + off);
+    const __nv_bfloat16* tv = reinterpret_cast<const __nv_bfloat16*>(&tj);
+    double acc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      acc[k] = __dmul_rn(static_cast<double>(cj), static_cast<double>(__bfloat162float(tv[k])));
     for (int q = begin; q < end; ++q) {
-      const double xm = static_cast<double>(__bfloat162float(pool[sc.src_base[q] + off]));
-      acc = __dadd_rn(acc, __dmul_rn(static_cast<double>(sc.src_cnt[q]), xm));
+      const uint4 xm = *reinterpret_cast<const uint4*>(pool + sc.src_base[q] + off);
+      const __nv_bfloat16* xv = reinterpret_cast<const __nv_bfloat16*>(&xm);
+      const double cm = static_cast<double>(sc.src_cnt[q]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        acc[k] = __dadd_rn(acc[k], __dmul_rn(cm, static_cast<double>(__bfloat162float(xv[k]))));
     }
-    pool[bj + off] = f64_to_bf16_rne(__ddiv_rn(acc, dtot));
+    uint4 o;
+    __nv_bfloat16* ov = reinterpret_cast<__nv_bfloat16*>(&o);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) ov[k] = f64_to_bf16_rne(__ddiv_rn(acc[k], dtot));
+    *reinterpret_cast<uint4*>(pool + bj + off) = o;
   }
   if (threadIdx.x == 0) sc.cnt[jpos] = tot;
 }
