@@ -430,45 +430,65 @@ __global__ void __launch_bounds__(1024) tier_select_kernel(Scratch sc, int N, in
 
 // Tier lists in position order: keep (protected, or among the n_keep_other smallest
 // (key, position) pairs), eligible targets (kept, not protected) and merge sources (the
-// next n_merge). Per chunk, two scans give each token its index among the non-protected
-// tokens of the threshold keys, three more place the tokens in the lists.
+// next n_merge). Each thread walks a contiguous range of positions three times: counts of
+// the threshold keys (two scans give each token its index among the non-protected tokens
+// of those keys), counts per list (three scans give the list offsets), then the writes.
 __global__ void __launch_bounds__(1024) tier_lists_kernel(Scratch sc, int N) {
   __shared__ int s_warp[32];
   const uint32_t v1 = static_cast<uint32_t>(sc.counts[8]), v2 = static_cast<uint32_t>(sc.counts[10]);
   const int need1 = sc.counts[9], need2 = sc.counts[11];
-  int eq_base[2] = {0, 0}, list_base[3] = {0, 0, 0};
-  int* lists[3] = {sc.keep, sc.elig, sc.merge};
-  for (int chunk = 0; chunk < N; chunk += blockDim.x) {
-    const int i = chunk + threadIdx.x;
-    bool p = true;
-    uint32_t key = 0;
-    if (i < N) {
-      p = sc.prot[i];
-      key = desc_key(sc.shat[i]);
-    }
+  const int ch = (N + blockDim.x - 1) / blockDim.x;
+  const int i0 = min(N, static_cast<int>(threadIdx.x) * ch), i1 = min(N, i0 + ch);
+  int c1 = 0, c2 = 0;
+  for (int i = i0; i < i1; ++i) {
+    const bool p = sc.prot[i];
+    const uint32_t key = desc_key(sc.shat[i]);
+    c1 += !p && key == v1;
+    c2 += !p && key == v2;
+  }
+  int tot;
+  const int b1 = cta_exclusive_scan(c1, s_warp, &tot);
+  const int b2 = cta_exclusive_scan(c2, s_warp, &tot);
+  // flags of position i given the running indices among the threshold keys
+  auto flags = [&](int i, int& r1, int& r2, int (&f)[3]) {
+    const bool p = sc.prot[i];
+    const uint32_t key = desc_key(sc.shat[i]);
     const bool e1 = !p && key == v1, e2 = !p && key == v2;
-    int tot;
-    const int x1 = eq_base[0] + cta_exclusive_scan(e1, s_warp, &tot);
-    eq_base[0] += tot;
-    const int x2 = eq_base[1] + cta_exclusive_scan(e2, s_warp, &tot);
-    eq_base[1] += tot;
-    const bool lt1 = !p && (key < v1 || (e1 && x1 < need1));
-    const bool lt2 = !p && (key < v2 || (e2 && x2 < need2));
-    int f[3];
-    f[0] = i < N && (p || lt1);
-    f[1] = i < N && lt1;
-    f[2] = i < N && !lt1 && lt2;
+    const bool lt1 = !p && (key < v1 || (e1 && r1 < need1));
+    const bool lt2 = !p && (key < v2 || (e2 && r2 < need2));
+    r1 += e1;
+    r2 += e2;
+    f[0] = p || lt1;
+    f[1] = lt1;
+    f[2] = !lt1 && lt2;
+  };
+  int n[3] = {0, 0, 0};
+  {
+    int r1 = b1, r2 = b2, f[3];
+    for (int i = i0; i < i1; ++i) {
+      flags(i, r1, r2, f);
+      n[0] += f[0];
+      n[1] += f[1];
+      n[2] += f[2];
+    }
+  }
+  int off[3], total[3];
 #pragma unroll
-    for (int q = 0; q < 3; ++q) {
-      const int x = cta_exclusive_scan(f[q], s_warp, &tot);
-      if (f[q]) lists[q][list_base[q] + x] = i;
-      list_base[q] += tot;
+  for (int q = 0; q < 3; ++q) off[q] = cta_exclusive_scan(n[q], s_warp, &total[q]);
+  int* lists[3] = {sc.keep, sc.elig, sc.merge};
+  {
+    int r1 = b1, r2 = b2, f[3];
+    for (int i = i0; i < i1; ++i) {
+      flags(i, r1, r2, f);
+#pragma unroll
+      for (int q = 0; q < 3; ++q)
+        if (f[q]) lists[q][off[q]++] = i;
     }
   }
   if (threadIdx.x == 0) {
-    sc.counts[1] = list_base[0];
-    sc.counts[2] = list_base[1];
-    sc.counts[3] = list_base[2];
+    sc.counts[1] = total[0];
+    sc.counts[2] = total[1];
+    sc.counts[3] = total[2];
   }
 }
 
@@ -513,14 +533,18 @@ __global__ void __launch_bounds__(1024) merge_group_kernel(Scratch sc, int n_src
   __syncthreads();
   for (int i = threadIdx.x; i < n_src; i += blockDim.x) atomicAdd(&sc.bucket[sc.target[i] + 1], 1);
   __syncthreads();
-  int base = 0;
-  for (int chunk = 0; chunk < n_elig; chunk += blockDim.x) {
-    const int e = chunk + threadIdx.x;
-    const int v = e < n_elig ? sc.bucket[e + 1] : 0;
+  {
+    // group ends: an inclusive scan of the counts, contiguous ranges per thread
+    const int ch = (n_elig + blockDim.x - 1) / blockDim.x;
+    const int e0 = min(n_elig, static_cast<int>(threadIdx.x) * ch), e1 = min(n_elig, e0 + ch);
+    int local = 0;
+    for (int e = e0; e < e1; ++e) local += sc.bucket[e + 1];
     int total;
-    const int excl = cta_exclusive_scan(v, s_warp, &total);
-    if (e < n_elig) sc.bucket[e + 1] = base + excl + v;   // inclusive: end of group e
-    base += total;
+    int run = cta_exclusive_scan(local, s_warp, &total);
+    for (int e = e0; e < e1; ++e) {
+      run += sc.bucket[e + 1];
+      sc.bucket[e + 1] = run;                                // inclusive: end of group e
+    }
   }
   __syncthreads();
   for (int i = threadIdx.x; i < n_src; i += blockDim.x) {
