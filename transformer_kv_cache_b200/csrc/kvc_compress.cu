@@ -193,8 +193,10 @@ __global__ void residual_norm_kernel(const float* __restrict__ r, int T, int R, 
 // Ranks of the frame's T tokens (s descending, ties to the lower slot), stored in the
 // history slot of this layer; then, over the window layers in `mask`, the population
 // variance of the normalised ranks gives Cons and s_hat, written next to the tokens.
-// One thread per token (every token reads all T scores from shared memory); a token's
-// Cons needs only its own ranks, so the CTAs are independent.
+// Eight lanes per token (every token's lanes read all T scores from shared memory, each
+// counting every eighth, then a shuffle sum); a token's Cons needs only its own ranks, so
+// the CTAs are independent. kClcesTokens tokens per 128-thread CTA.
+constexpr int kClcesTokens = 16;
 __global__ void __launch_bounds__(128) clces_kernel(const float* __restrict__ s, int T, int32_t* hist, int slot,
                                                      uint32_t mask, int n_win, float lam,
                                                      const Entry* __restrict__ frame_pages, int P,
@@ -202,19 +204,24 @@ __global__ void __launch_bounds__(128) clces_kernel(const float* __restrict__ s,
   extern __shared__ float s_sm[];
   for (int i = threadIdx.x; i < T; i += blockDim.x) s_sm[i] = s[i];
   __syncthreads();
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int sub = threadIdx.x & 7;
+  const int i = blockIdx.x * kClcesTokens + static_cast<int>(threadIdx.x >> 3);
+  int r = 0;
   if (i < T) {
     const float si = s_sm[i];
-    int r = 0;
-    for (int j = 0; j < T; ++j) {
+    for (int j = sub; j < T; j += 8) {
       const float sj = s_sm[j];
       r += (sj > si) || (sj == si && j < i);
     }
-    hist[slot * T + i] = r;
   }
+  r += __shfl_xor_sync(0xffffffffu, r, 1);
+  r += __shfl_xor_sync(0xffffffffu, r, 2);
+  r += __shfl_xor_sync(0xffffffffu, r, 4);
+  if (i >= T || sub != 0) return;
+  hist[slot * T + i] = r;
   const double sqrt12 = __dsqrt_rn(12.0);
   const double lamd = static_cast<double>(lam);
-  if (i < T) {
+  {
     long long sr = 0, sr2 = 0;
     for (int k = 0; k < 32; ++k) {
       if (mask & (1u << k)) {
@@ -747,7 +754,7 @@ kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_
   residual_norm_kernel<<<(T * 32 + 255) / 256, 256, 0, s>>>(residual, T, g.residual_dim, sc.s_raw);
   ok();
   const FrameRec& fr = L.frames.back();
-  clces_kernel<<<(T + 127) / 128, 128, T * sizeof(float), s>>>(sc.s_raw, T, c->rank_hist, layer % RW, mask, n_win, g.lambda_,
+  clces_kernel<<<(T + kClcesTokens - 1) / kClcesTokens, 128, T * sizeof(float), s>>>(sc.s_raw, T, c->rank_hist, layer % RW, mask, n_win, g.lambda_,
                                                   E + fr.first_entry, P, c->tok_shat + lay_slots);
   ok();
   c->hist_next_layer = layer + 1;
