@@ -160,3 +160,41 @@ def test_reset_clears_everything_and_replays_identically():
         assert orc.page_table(0).shape[0] == 0 and orc.pages_in_use(0) == 0
     for a, b in zip(*outs):
         np.testing.assert_array_equal(a, b)
+
+
+# ------------------------------------------------------------------ planted mistakes
+# Dimension-adaptive FP8 misread in the oracle (on the CPU); the brute-force pin over
+# torch's float8 cast must fail on each.
+
+def _da_small():
+    return WORKLOADS["vggt_518x518_fp8"].replace(tokens_per_frame=37, num_heads=2, head_dim=16,
+                                                  window_frames=3, scale_frames=2, page_size=8,
+                                                  fp8_dim_adaptive=1)
+
+
+def test_planted_swapped_dimension_adaptive_axes_are_caught(monkeypatch):
+    """K grouped per token and V per channel (KIVI's split the wrong way round)."""
+    import oracle.kvcache_oracle as ko
+    ch, tok = ko.fp8_quantise_channels, ko.fp8_quantise_tokens
+    monkeypatch.setattr(ko, "fp8_quantise_channels", tok)
+    monkeypatch.setattr(ko, "fp8_quantise_tokens", ch)
+    # full pages with P = D, so that the swapped scale arrays still fit their slots and
+    # only the values tell the two apart
+    wl = _da_small().replace(tokens_per_frame=32, page_size=16)
+    with pytest.raises(AssertionError):
+        _run_and_check(wl, 5, seed=6)
+
+
+def test_planted_per_page_scales_in_dimension_adaptive_mode_are_caught(monkeypatch):
+    """One scale per (page, head) although the mode asks for per-channel / per-token ones."""
+    import oracle.kvcache_oracle as ko
+
+    def per_block(axis):
+        def q(x):
+            codes, scale, deq = ko.fp8_quantise_block(x)
+            return codes, np.full(np.shape(x)[axis], scale), deq
+        return q
+    monkeypatch.setattr(ko, "fp8_quantise_channels", per_block(1))
+    monkeypatch.setattr(ko, "fp8_quantise_tokens", per_block(0))
+    with pytest.raises(AssertionError):
+        _run_and_check(_da_small(), 5, seed=6)

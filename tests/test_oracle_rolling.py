@@ -114,7 +114,7 @@ def test_anchor_immutable_and_memory_bounded():
             assert np.all(mut >= T) and np.all(np.diff(mut) > 0)
 
 
-def test_kept_set_is_top_k_of_candidates_each_frame():
+def _kept_set_check():
     # brute force on one head: candidates = previous kept + new frame, scored by scipy
     T, H, D, K = 20, 3, 16, 30
     prev = {h: (np.zeros(0, int), np.zeros((0, D))) for h in range(H)}
@@ -129,6 +129,17 @@ def test_kept_set_is_top_k_of_candidates_each_frame():
             assert set(ids[order].tolist()) == set(orc.mut_ids[0][h].tolist())
             sel = sorted(order, key=lambda i: ids[i])
             prev[h] = (ids[sel], Kc[sel])
+
+
+def test_kept_set_is_top_k_of_candidates_each_frame():
+    _kept_set_check()
+
+
+def _ties_check():
+    Kc = np.ones((10, 8))
+    ids = np.arange(10)[::-1].copy()                # ids 9..0
+    keep = ro.top_k(ro.diversity_scores(Kc), ids, 4)
+    assert sorted(ids[keep].tolist()) == [0, 1, 2, 3]
 
 
 def test_attention_is_softmax_over_anchor_and_kept():
@@ -208,3 +219,47 @@ def test_dim_sum_order_hand_derived():
     x = np.array([[2.0 ** 53] + [1.0] * 15])
     assert ro.dim_sum(x)[0] == 2.0 ** 53 + 8.0
     np.testing.assert_array_equal(ro.dim_sum(np.arange(64.0)[None, :]), [2016.0])   # exact integers
+
+
+# ------------------------------------------------------------------ planted mistakes
+# Plausible misreadings planted in the oracle (on the CPU), each run through a pin above.
+
+def test_planted_similarity_instead_of_diversity_is_caught(monkeypatch):
+    """Keeping the candidates most similar to the mean (+cos) instead of the most diverse."""
+    real = ro.diversity_scores
+    monkeypatch.setattr(ro, "diversity_scores", lambda Kc: -real(Kc))
+    with pytest.raises(AssertionError):
+        _kept_set_check()
+
+
+def test_planted_unnormalised_keys_are_caught(monkeypatch):
+    """The mean taken over raw keys (long keys dominate) instead of unit keys."""
+    monkeypatch.setattr(ro, "normalised_keys", lambda Kc: np.asarray(Kc, np.float64))
+    with pytest.raises(AssertionError):
+        _kept_set_check()
+
+
+def test_planted_new_frame_only_candidates_are_caught(monkeypatch):
+    """Pruning that forgets the kept set and ranks only the new frame's tokens."""
+    orig = RollingOracle.prune
+
+    def forgetful(self, layer):
+        for h in range(len(self.mut_ids[layer])):
+            D = self.mut_k[layer][h].shape[1]
+            self.mut_ids[layer][h] = np.zeros(0, np.int64)
+            self.mut_k[layer][h] = np.zeros((0, D))
+            self.mut_v[layer][h] = np.zeros((0, D))
+        return orig(self, layer)
+    monkeypatch.setattr(RollingOracle, "prune", forgetful)
+    with pytest.raises(AssertionError):
+        _kept_set_check()
+
+
+def test_planted_ties_to_higher_ids_are_caught(monkeypatch):
+    """Equal scores resolved towards the higher token id."""
+    def top_k_high(scores, ids, k):
+        order = sorted(range(len(ids)), key=lambda i: (-scores[i], -ids[i]))[:k]
+        return np.array(sorted(order, key=lambda i: ids[i]), dtype=np.int64)
+    monkeypatch.setattr(ro, "top_k", top_k_high)
+    with pytest.raises(AssertionError):
+        _ties_check()

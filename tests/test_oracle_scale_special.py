@@ -19,7 +19,7 @@ def _frames(n, T, H, D, seed):
     return [tuple(rng.standard_normal((T, H, D)) for _ in range(3)) for _ in range(n)]
 
 
-def test_joint_phase_is_bidirectional_attention_over_all_scale_frames():
+def _joint_phase_check():
     cfg = _cfg(T=37, S=4, W=3, special=0)
     fr = _frames(4, cfg.tokens_per_frame, cfg.num_heads, cfg.head_dim, 1)
     Q = np.concatenate([f[0] for f in fr])
@@ -38,6 +38,10 @@ def test_joint_phase_is_bidirectional_attention_over_all_scale_frames():
     nxt = orc.attend(0, q4)
     ref4 = brute.attention(q4, np.concatenate([K, k4]), np.concatenate([V, v4]), cfg.softmax_scale)
     np.testing.assert_allclose(nxt, ref4, rtol=0, atol=1e-12)
+
+
+def test_joint_phase_is_bidirectional_attention_over_all_scale_frames():
+    _joint_phase_check()
 
 
 def test_joint_phase_needs_an_empty_layer_and_at_most_S_frames():
@@ -68,12 +72,14 @@ def _expected_tokens(t, S, W, cap, T, ns):
     return ids + [t * T + i for i in range(T)]
 
 
-@pytest.mark.parametrize("T,P,ns,cap,S,W", [
+SPECIAL_CASES = [
     (37, 16, 5, 3, 1, 2),     # one special page per evicted frame, FIFO after 3
     (40, 16, 18, 2, 2, 3),    # specials span two pages (16 + 2)
     (10, 16, 5, 50, 0, 1),    # T < P, no scale frame, cap never reached
-])
-def test_special_tokens_outlive_their_frames(T, P, ns, cap, S, W):
+]
+
+
+def _special_tokens_check(T, P, ns, cap, S, W):
     cfg = _cfg(T=T, P=P, ns=ns, special=cap, S=S, W=W)
     H, D = cfg.num_heads, cfg.head_dim
     fr = _frames(14, T, H, D, 3)
@@ -95,6 +101,11 @@ def test_special_tokens_outlive_their_frames(T, P, ns, cap, S, W):
     n_ret = min(cap, 14 - S - W)
     assert len(L.retained) == n_ret
     assert sum(L.free_used) == (S + W) * -(-T // P) + n_ret * -(-ns // P)
+
+
+@pytest.mark.parametrize("T,P,ns,cap,S,W", SPECIAL_CASES)
+def test_special_tokens_outlive_their_frames(T, P, ns, cap, S, W):
+    _special_tokens_check(T, P, ns, cap, S, W)
 
 
 def test_trimmed_pages_hold_zeros_past_the_special_tokens():
@@ -120,3 +131,65 @@ def test_non_keyframes_leave_no_special_tokens():
     assert all(f % 2 == 0 for f in orc.layers[0].retained)
     _, _, ids = orc.gather(0)
     assert all((i // 37) % 2 == 0 for i in ids.tolist())
+
+
+# ------------------------------------------------------------------ planted mistakes
+# Each plants one plausible misreading in the oracle (on the CPU); the pins above must
+# fail on it.
+
+def test_planted_causal_joint_phase_is_caught(monkeypatch):
+    """The joint phase read as frame-by-frame causal steps over the scale frames."""
+    def causal(self, layer, n, Q, K, V, rows=None):
+        T = self.T
+        outs = []
+        for f in range(n):
+            self.append(layer, f, K[f * T:(f + 1) * T], V[f * T:(f + 1) * T], True)
+            outs.append(self.attend(layer, Q[f * T:(f + 1) * T]))
+        return np.concatenate(outs)
+    monkeypatch.setattr(StreamOracle, "scale_phase", causal)
+    with pytest.raises(AssertionError):
+        _joint_phase_check()
+
+
+def test_planted_dropped_special_tokens_are_caught(monkeypatch):
+    """Eviction that forgets the special tokens (plain sliding window)."""
+    monkeypatch.setattr(StreamOracle, "_retain_special", lambda self, L, f: None)
+    with pytest.raises(AssertionError):
+        _special_tokens_check(*SPECIAL_CASES[0])
+
+
+def test_planted_newest_first_special_cap_is_caught(monkeypatch):
+    """At the special_frames cap, the newest retained frame dropped instead of the oldest."""
+    orig = StreamOracle._retain_special
+
+    def newest_first(self, L, f):
+        cap = self.cfg.special_frames
+        self.cfg.special_frames = 1 << 30
+        try:
+            orig(self, L, f)
+        finally:
+            self.cfg.special_frames = cap
+        while len(L.retained) > cap:
+            new = L.retained.pop()
+            self._free(L, [e[0] for e in L.entries if e[1] == new])
+            L.entries = [e for e in L.entries if e[1] != new]
+    monkeypatch.setattr(StreamOracle, "_retain_special", newest_first)
+    with pytest.raises(AssertionError):
+        _special_tokens_check(*SPECIAL_CASES[0])
+
+
+def test_planted_untrimmed_special_page_is_caught(monkeypatch):
+    """The special page kept whole: the non-special tokens sharing it survive eviction."""
+    def untrimmed(self, L, f):
+        keep_pages = -(-min(self.cfg.num_special_tokens, self.T) // self.P)
+        drop = [e[0] for e in L.entries if e[1] == f and e[2] >= keep_pages]
+        self._free(L, drop)
+        L.entries = [e for e in L.entries if not (e[1] == f and e[2] >= keep_pages)]
+        L.retained.append(f)
+        while len(L.retained) > self.cfg.special_frames:
+            old = L.retained.pop(0)
+            self._free(L, [e[0] for e in L.entries if e[1] == old])
+            L.entries = [e for e in L.entries if e[1] != old]
+    monkeypatch.setattr(StreamOracle, "_retain_special", untrimmed)
+    with pytest.raises(AssertionError):
+        _special_tokens_check(*SPECIAL_CASES[0])
