@@ -43,7 +43,7 @@ def _drive(wl, frames, seed=0, on_event=None):
     return orc, events
 
 
-def test_compression_properties():
+def _compression_check():
     wl = _small_wl()
     n_keep = math.floor(float(np.float32(wl.keep_frac)) * wl.budget_tokens)
     n_merge = wl.budget_tokens - n_keep
@@ -104,6 +104,8 @@ def test_compression_properties():
                 stack = np.stack([before[pos[m]].reshape(-1) for m in members])
                 mean = np.average(stack, axis=0, weights=w)
                 got = after[list(ida).index(j)].reshape(-1)
+                # the cache stores bf16: the merged value is rounded once to a bf16 number
+                assert np.array_equal(torch.tensor(got).to(torch.bfloat16).to(torch.float64).numpy(), got)
                 ulp = np.abs(bf16_round(mean) - bf16_round(mean * (1 + 2 ** -8)))
                 assert np.all(np.abs(got - bf16_round(mean)) <= ulp + 1e-300)
         # compaction packs P per page in ascending id, into the lowest free pages
@@ -113,6 +115,10 @@ def test_compression_properties():
 
     orc, events = _drive(wl, 9, on_event=check)
     assert events >= 4 and len(seen) == events
+
+
+def test_compression_properties():
+    _compression_check()
 
 
 def test_full_protected_keep_tier_drops_merge_tier():
@@ -135,3 +141,13 @@ def test_no_compression_below_budget():
     assert events == 0
     ids, cnt, sh = orc.token_meta(0)
     assert ids.size == 5 * wl.tokens_per_frame and np.all(cnt == 1)
+
+
+# ------------------------------------------------------------------ planted mistakes
+
+def test_planted_unrounded_merge_is_caught(monkeypatch):
+    """The merged mean stored in fp64 without its single rounding to bf16."""
+    import oracle.kvcache_oracle as ko
+    monkeypatch.setattr(ko, "bf16_round", lambda x: np.asarray(x, np.float64))
+    with pytest.raises(AssertionError):
+        _compression_check()
