@@ -64,3 +64,60 @@ def test_host_only_calls_and_config_validation():
     bad = kvc.make_config(1, 2, 64, 10, 1, 8, 2, 0, budget_tokens=100)   # window and budget together
     with pytest.raises(kvc.KVCError):
         kvc.kvc_create(bad, stream=0)
+
+
+# Each rule of kvc_create's argument check, one at a time: the unmodified workload config
+# passes the check (without a GPU it then fails at its first device allocation, never with
+# KVC_ERR_ARG; with one it is created and destroyed), and the one change makes it
+# KVC_ERR_ARG before any CUDA call.
+CONFIG_RULES = [
+    ("vggt_518x378", dict(head_dim=48), "head dim outside 16/32/64/128"),
+    ("vggt_518x378", dict(num_special_tokens=1005), "more special tokens than a frame holds"),
+    ("vggt_518x378", dict(io_dtype="f32"), "bf16 storage under fp32 inputs"),
+    ("vggt_518x378", dict(softmax_scale=float("nan")), "softmax scale not finite"),
+    ("vggt_518x378", dict(softmax_scale=0.0), "softmax scale not positive"),
+    ("vggt_518x378", dict(kv_splits=-1), "negative KV split count"),
+    ("vggt_518x378", dict(budget_tokens=16384), "window and token budget together"),
+    ("vggt_518x378", dict(window_frames=0, max_frames=0), "no window, budget or frame cap"),
+    ("vggt_518x378", dict(fp8_dim_adaptive=1), "dimension-adaptive scales on bf16 storage"),
+    ("vggt_518x378_special", dict(special_frames=-1), "negative special-frame cap"),
+    ("vggt_518x378_special", dict(window_frames=0, max_frames=100), "special tokens without a window"),
+    ("vggt_518x518_fp8", dict(io_dtype="f32"), "FP8 storage under fp32 inputs"),
+    ("vggt_518x518_fp8", dict(page_size=64), "FP8 page-head block over 2 KB"),
+    ("vggt_518x518_fp8da", dict(fp8_dim_adaptive=2), "unknown quantisation mode"),
+    ("vggt_518x518_fp8da", dict(page_size=8), "dimension-adaptive FP8 off the 16 x 64 block"),
+    ("vggt_budget_16k", dict(kv_dtype="fp8_e4m3"), "token budget on FP8 storage"),
+    ("vggt_budget_16k", dict(keep_frac=0.0), "empty keep tier"),
+    ("vggt_budget_16k", dict(rank_window=0), "empty rank window"),
+    ("vggt_budget_16k", dict(lam=-0.5), "negative consistency weight"),
+    ("vggt_infinite_12l", dict(page_size=8), "rolling memory off the 16-slot page"),
+    ("vggt_infinite_12l", dict(diversity_budget=1100), "more candidates than the pruning cluster holds"),
+    ("vggt_infinite_12l", dict(diversity_budget=-1), "negative diversity budget"),
+    ("vggt_infinite_12l", dict(window_frames=64), "rolling memory with a window"),
+]
+
+
+@pytest.mark.parametrize("workload,change,why", CONFIG_RULES, ids=[r[2] for r in CONFIG_RULES])
+def test_config_rule_rejected_before_any_cuda_call(workload, change, why):
+    import transformer_kv_cache_b200 as kvc
+    from kvc_streams import WORKLOADS
+    wl = WORKLOADS[workload]
+    try:
+        h = kvc.kvc_create(kvc.config_from_workload(wl), stream=0)
+    except kvc.KVCError as e:
+        assert e.status_name != "KVC_ERR_ARG", f"base config of {workload} fails the argument check"
+    else:
+        kvc.kvc_destroy(h)                      # a device is present and the base was created
+    with pytest.raises(kvc.KVCError) as e:
+        kvc.kvc_create(kvc.config_from_workload(wl, **change), stream=0)
+    assert e.value.status_name == "KVC_ERR_ARG", why
+
+
+def test_reserved_config_words_must_be_zero():
+    import transformer_kv_cache_b200 as kvc
+    from kvc_streams import WORKLOADS
+    cfg = kvc.config_from_workload(WORKLOADS["vggt_518x378"])
+    cfg.reserved[2] = 7
+    with pytest.raises(kvc.KVCError) as e:
+        kvc.kvc_create(cfg, stream=0)
+    assert e.value.status_name == "KVC_ERR_ARG"
