@@ -121,3 +121,38 @@ def test_reserved_config_words_must_be_zero():
     with pytest.raises(kvc.KVCError) as e:
         kvc.kvc_create(cfg, stream=0)
     assert e.value.status_name == "KVC_ERR_ARG"
+
+
+def test_null_handle_is_rejected_by_every_entry_point():
+    """Host-only: every call that takes a cache handle returns KVC_ERR_ARG for NULL (no
+    dereference, no CUDA call); kvc_destroy(NULL) is a no-op; the allocation-free entry
+    point rejects NULL device pointers."""
+    import transformer_kv_cache_b200 as kvc
+    lib = kvc._lib
+    no_handle = {"kvc_create", "kvc_status_string", "kvc_version", "kvc_debug_fail_allocs",
+                 "kvc_attend_paged_noalloc", "kvc_destroy", "kvc_last_error"}
+
+    def zero_args(fn):
+        out = []
+        for t in fn.argtypes:
+            if t in (ctypes.c_float, ctypes.c_double):
+                out.append(0.0)
+            elif t in (ctypes.c_int32, ctypes.c_int64, ctypes.c_int):
+                out.append(0)
+            else:
+                out.append(None)                    # handle and every pointer
+        return out
+
+    checked = 0
+    for name in kvc.EXPORTS:
+        if name in no_handle:
+            continue
+        fn = getattr(lib, name)
+        assert fn.argtypes, f"{name} has no declared signature in the binding"
+        assert fn(*zero_args(fn)) == 1, name       # KVC_ERR_ARG
+        checked += 1
+    assert checked >= 20
+    assert lib.kvc_destroy(None) == 0
+    assert ctypes.string_at(lib.kvc_last_error(None)) == b"null cache"
+    fn = lib.kvc_attend_paged_noalloc
+    assert fn(*zero_args(fn)) == 1
