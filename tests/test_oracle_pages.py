@@ -94,3 +94,16 @@ def test_planted_oracle_mistakes_are_caught(monkeypatch, mistake):
         monkeypatch.setattr(StreamOracle, "append", bad)
     with pytest.raises(AssertionError):
         _brute_frame_check(wl)
+
+
+def test_harness_keyframe_schedule_is_the_oracles_rule():
+    """The streams hand both sides the same is_keyframe decision (the library takes it as an
+    argument); it must be the oracle's reading of the keyframe rule, and match a hand-listed
+    case: S = 2, k = 3 keeps frames 0, 1, 2, 5, 8, 11."""
+    from kvc_streams import keyframe_schedule
+    from oracle import is_keyframe
+    for S in range(0, 5):
+        for k in range(1, 6):
+            for t in range(40):
+                assert keyframe_schedule(t, S, k) == is_keyframe(t, S, k), (t, S, k)
+    assert [t for t in range(12) if is_keyframe(t, 2, 3)] == [0, 1, 2, 5, 8, 11]
