@@ -211,7 +211,8 @@ struct TcAttnArgs {
   const float* k_chan = nullptr;    // dimension-adaptive FP8 scales (FP8 kernel), or null
   const float* v_tok = nullptr;
   int* split_cnt = nullptr;         // [H][q_tiles] zeroed counters (bf16 kernel): the last
-                                    // split CTA of a query tile merges, no combine launch
+                                    // split CTA of a query tile merges, no combine launch;
+                                    // the launcher uses them for up to 4 splits only
 };
 // Returns the number of kernels launched through *launched.
 cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used, int* launched);
