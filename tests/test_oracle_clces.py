@@ -5,6 +5,7 @@ import statistics
 from fractions import Fraction
 
 import numpy as np
+import pytest
 
 from oracle import OracleConfig, StreamOracle, to_f32
 
@@ -30,6 +31,19 @@ def test_constant_rank_gives_cons_one_and_fifty_percent_bonus():
         sh = orc.score(l, 0, _residual_with_norms(norms))
         # ranks never move -> sigma = 0 -> Cons = 1 -> s_hat = fp32(s * 1.5)
         np.testing.assert_array_equal(sh, to_f32(to_f32(norms) * 1.5))
+
+
+def test_raw_score_is_rounded_to_fp32_before_the_bonus():
+    # norms that fp32 does not hold, in the same order at every layer: Cons = 1 and
+    # s_hat = fp32(fp32(s) * 1.5), which differs from rounding s * 1.5 once for some of them
+    T = 16
+    norms = 1.0 + np.sort(np.random.default_rng(11).uniform(0, 1, T))
+    want = to_f32(to_f32(norms) * 1.5)
+    assert np.any(want != to_f32(norms * 1.5))      # the two readings differ on this input
+    orc = _orc(T)
+    for l in range(3):
+        sh = orc.score(l, 0, _residual_with_norms(norms))
+    np.testing.assert_array_equal(sh, want)
 
 
 def test_lambda_zero_returns_raw_score():
@@ -111,3 +125,45 @@ def test_raw_score_is_fp32_of_exact_norm():
     sh = orc.score(0, 0, r.astype(np.float64))
     exact = np.array([math.sqrt(math.fsum(float(v) * float(v) for v in row)) for row in r])
     np.testing.assert_array_equal(sh, to_f32(exact))
+
+
+# ------------------------------------------------------------------ planted mistakes
+
+def test_planted_unrounded_raw_score_is_caught(monkeypatch):
+    """s kept in fp64 instead of rounded once to fp32 (StreamCacheVGGT page, 2.1.1)."""
+    import oracle.kvcache_oracle as ko
+    monkeypatch.setattr(ko, "to_f32", lambda x: np.asarray(x, np.float64))
+    with pytest.raises(AssertionError):
+        test_raw_score_is_rounded_to_fp32_before_the_bonus()
+
+
+def test_planted_sample_variance_is_caught(monkeypatch):
+    """sigma from the sample variance (divide by n - 1) instead of the population one: the
+    exact-rational pin must fail. Planted through the oracle's square root of D, scaled by
+    n / (n - 1) inside the same expression."""
+    import oracle.kvcache_oracle as ko
+    real_sqrt = math.sqrt
+    state = {}
+
+    class M:
+        def __getattr__(self, name):
+            return getattr(math, name)
+
+        @staticmethod
+        def sqrt(x):
+            n = state.get("n")
+            if n is not None and n > 1 and x != 12.0:
+                return real_sqrt(x * n / (n - 1))
+            return real_sqrt(x)
+
+    orig_score = ko.StreamOracle.score
+
+    def score(self, layer, t, residual):
+        # the window length the oracle will use for this call
+        hist = self._rank_hist if t == self._rank_frame else {}
+        state["n"] = 1 + sum(1 for l in range(layer - self.cfg.rank_window + 1, layer) if l in hist)
+        return orig_score(self, layer, t, residual)
+    monkeypatch.setattr(ko, "math", M())
+    monkeypatch.setattr(ko.StreamOracle, "score", score)
+    with pytest.raises(AssertionError):
+        test_sigma_matches_library_population_variance()

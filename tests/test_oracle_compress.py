@@ -151,3 +151,18 @@ def test_planted_unrounded_merge_is_caught(monkeypatch):
     monkeypatch.setattr(ko, "bf16_round", lambda x: np.asarray(x, np.float64))
     with pytest.raises(AssertionError):
         _compression_check()
+
+
+def test_planted_least_similar_target_is_caught(monkeypatch):
+    """Merge targets taken by the smallest cosine instead of the largest (the oracle's
+    numpy is swapped for a view whose argmax is argmin; the pins use the real numpy)."""
+    import oracle.kvcache_oracle as ko
+
+    class NP:
+        def __getattr__(self, name):
+            return getattr(np, name)
+
+        argmax = staticmethod(np.argmin)
+    monkeypatch.setattr(ko, "np", NP())
+    with pytest.raises(AssertionError):
+        _compression_check()
