@@ -193,3 +193,19 @@ def test_planted_untrimmed_special_page_is_caught(monkeypatch):
     monkeypatch.setattr(StreamOracle, "_retain_special", untrimmed)
     with pytest.raises(AssertionError):
         _special_tokens_check(*SPECIAL_CASES[0])
+
+
+def test_joint_phase_over_fp8_pages_matches_brute_force():
+    """FP8 storage: every frame's pages quantised per (page, head) through torch's float8
+    cast, then bidirectional attention over all of them."""
+    import torch
+    cfg = _cfg(T=37, P=8, S=3, W=2, special=0, kv="fp8_e4m3")
+    T, H, D = cfg.tokens_per_frame, cfg.num_heads, cfg.head_dim
+    bf = lambda x: torch.tensor(x).to(torch.bfloat16).to(torch.float64).numpy()
+    fr = [tuple(bf(x) for x in f) for f in _frames(3, T, H, D, 9)]
+    Q = np.concatenate([f[0] for f in fr])
+    got = StreamOracle(cfg).scale_phase(0, 3, Q, np.concatenate([f[1] for f in fr]),
+                                        np.concatenate([f[2] for f in fr]))
+    Ks = np.concatenate([brute.stored(f[1], "fp8_e4m3", cfg.page_size) for f in fr])
+    Vs = np.concatenate([brute.stored(f[2], "fp8_e4m3", cfg.page_size) for f in fr])
+    np.testing.assert_allclose(got, brute.attention(Q, Ks, Vs, cfg.softmax_scale), rtol=1e-10, atol=1e-12)
