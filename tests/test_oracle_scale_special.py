@@ -209,3 +209,26 @@ def test_joint_phase_over_fp8_pages_matches_brute_force():
     Ks = np.concatenate([brute.stored(f[1], "fp8_e4m3", cfg.page_size) for f in fr])
     Vs = np.concatenate([brute.stored(f[2], "fp8_e4m3", cfg.page_size) for f in fr])
     np.testing.assert_allclose(got, brute.attention(Q, Ks, Vs, cfg.softmax_scale), rtol=1e-10, atol=1e-12)
+
+
+def test_fp8_special_tokens_keep_their_stored_values_after_eviction():
+    """Trimming keeps the page's codes and scale for the special tokens: their stored values
+    after eviction are the ones the frame's quantisation gave them (no requantisation over
+    the survivors), and equal torch's float8 cast of the whole page."""
+    import torch
+    cfg = _cfg(T=37, P=16, ns=5, special=4, S=0, W=1, kv="fp8_e4m3")
+    orc = StreamOracle(cfg)
+    bf = lambda x: torch.tensor(x).to(torch.bfloat16).to(torch.float64).numpy()   # the library's inputs
+    fr = [tuple(bf(x) for x in f) for f in _frames(4, 37, 2, 16, 12)]
+    for t, (q, k, v) in enumerate(fr):
+        orc.append(0, t, k, v, True)
+        orc.attend(0, q)
+    L = orc.layers[0]
+    assert L.retained
+    for pid, owner, idx, n in L.entries:
+        if owner in L.retained:
+            pg = L.pages[pid]
+            want_k = brute.stored(fr[owner][1], "fp8_e4m3", cfg.page_size)[:5]
+            want_v = brute.stored(fr[owner][2], "fp8_e4m3", cfg.page_size)[:5]
+            np.testing.assert_array_equal(pg.k[:, :5], np.transpose(want_k, (1, 0, 2)))
+            np.testing.assert_array_equal(pg.v[:, :5], np.transpose(want_v, (1, 0, 2)))
