@@ -69,7 +69,8 @@ def test_tiny_f32_matches_brute_force():
     assert orc.high_water(0) == (S + W + 1) * ppf
 
 
-@pytest.mark.parametrize("T,P,S,W,k", [(13, 4, 2, 3, 1), (9, 8, 1, 2, 3), (16, 16, 0, 2, 2), (7, 2, 3, 1, 1)])
+@pytest.mark.parametrize("T,P,S,W,k", [(13, 4, 2, 3, 1), (9, 8, 1, 2, 3), (16, 16, 0, 2, 2), (7, 2, 3, 1, 1),
+                                       (13, 4, 2, 0, 2)])    # W = 0: no window, every keyframe stays
 def test_random_small_configs_match_brute_force(T, P, S, W, k):
     wl = WORKLOADS["tiny_f32"].replace(tokens_per_frame=T, page_size=P, scale_frames=S,
                                         window_frames=W, keyframe_interval=k, num_heads=3, head_dim=8)

@@ -232,3 +232,20 @@ def test_fp8_special_tokens_keep_their_stored_values_after_eviction():
             want_v = brute.stored(fr[owner][2], "fp8_e4m3", cfg.page_size)[:5]
             np.testing.assert_array_equal(pg.k[:, :5], np.transpose(want_k, (1, 0, 2)))
             np.testing.assert_array_equal(pg.v[:, :5], np.transpose(want_v, (1, 0, 2)))
+
+
+def test_no_special_tokens_is_the_plain_window():
+    """num_special_tokens = 0 with a special-frame cap: nothing survives an eviction, and the
+    stream equals the plain sliding window bit for bit."""
+    fr = _frames(9, 37, 2, 16, 13)
+    outs = {}
+    for special in (3, 0):
+        orc = StreamOracle(_cfg(T=37, ns=0, special=special, S=1, W=2))
+        outs[special] = []
+        for t, (q, k, v) in enumerate(fr):
+            orc.append(0, t, k, v, True)
+            outs[special].append(orc.attend(0, q))
+        L = orc.layers[0]
+        assert all(e[1] not in L.retained for e in L.entries)   # no page kept for an evicted frame
+    for a, b in zip(outs[3], outs[0]):
+        np.testing.assert_array_equal(a, b)
