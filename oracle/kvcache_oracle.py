@@ -35,10 +35,11 @@ What it follows (the web pages are cited by title and section):
   uniform reference 1/12, Cons = max(0, 1 - sigma*sqrt(12)), enhanced score
   s_hat = s * (1 + lambda * Cons), rank history reset at each new frame.
 * Keep / merge / drop tiers -- StreamCacheVGGT page, section 2 (core tokens kept,
-  medium tokens merged into the core, lowest dropped); the page is cut off before
-  section 2.2, so tier sizes, the merge rule (count-weighted mean into the kept
-  token with highest key cosine) and the protected set (frame 0 and the camera /
-  register tokens) follow the budgeted-compression workload's statement.
+  medium tokens merged into the core, lowest dropped); the page breaks off right after
+  the heading of section 2.2 (hybrid compression, from dropping to merging), so tier
+  sizes, the merge rule (count-weighted mean into the kept token with highest key
+  cosine) and the protected set (frame 0 and the camera / register tokens) follow the
+  budgeted-compression workload's statement.
 * FP8 KV quantisation -- XStreamVGGT abstract (KV cache quantisation); the
   format is OCP FP8 E4M3 (bias 7, max finite 448, no infinities), one absmax
   scale per (page, head), separately for K and V. Its "dimension-adaptive" variant
