@@ -18,6 +18,7 @@ bounded sample of the same workload, extrapolated to a whole frame).
 from __future__ import annotations
 
 import argparse
+import contextlib
 import hashlib
 import json
 import math
@@ -141,11 +142,21 @@ def run_reference(args):
     # (append, gather, commit of one head) plus ~6 ms per sampled query row
     budget_per_step = 150.0 / max(1, steps + warm)
     rows = int(max(1, min(16, (budget_per_step - 0.15) / 0.006)))
-    per_frame, r, wall = oracle_sample(wl, steps + warm, rows)
+    # torchrun sets OMP_NUM_THREADS=1 in every rank; here rank 0 is the only one at work,
+    # so the oracle gets the host's cores as it does in a plain single-process run
+    ctx = contextlib.nullcontext()
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        try:
+            from threadpoolctl import threadpool_limits
+            ctx = threadpool_limits(limits=len(os.sched_getaffinity(0)))
+        except Exception:
+            pass
+    with ctx:
+        per_frame, r, wall = oracle_sample(wl, steps + warm, rows)
+        cores = blas_threads()
     timed = per_frame[warm:] if len(per_frame) > warm else per_frame
     mean_s = statistics.mean(timed)
     value = 1.0 / mean_s
-    cores = blas_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": len(timed), "warmup": warm, "ms_per_step": mean_s * 1e3, "higher_is_better": True,
