@@ -156,3 +156,34 @@ def test_null_handle_is_rejected_by_every_entry_point():
     assert ctypes.string_at(lib.kvc_last_error(None)) == b"null cache"
     fn = lib.kvc_attend_paged_noalloc
     assert fn(*zero_args(fn)) == 1
+
+
+def test_plain_c_program_links_and_calls_the_library():
+    """A C99 program compiled against include/kvc.h and linked with libkvc.so: the host-only
+    calls work without Python (version, status strings, argument rejection, NULL handles)."""
+    import transformer_kv_cache_b200 as kvc
+    prog = r'''
+#include <stdio.h>
+#include <string.h>
+#include "kvc.h"
+int main(void) {
+  kvc_config cfg;
+  kvc_cache* c = (kvc_cache*)1;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.num_layers = 1; cfg.num_heads = 16; cfg.head_dim = 48;   /* head dim 48 is rejected */
+  cfg.tokens_per_frame = 1004; cfg.page_size = 16; cfg.window_frames = 64;
+  cfg.io_dtype = KVC_BF16; cfg.kv_dtype = KVC_BF16; cfg.softmax_scale = 0.125f;
+  kvc_status st = kvc_create(&cfg, NULL, &c);
+  printf("%d %d %s %d %d %s\n", (int)kvc_version(), (int)st, kvc_status_string(st), c == NULL,
+         (int)kvc_attend(NULL, 0, NULL, NULL), kvc_last_error(NULL));
+  return 0;
+}'''
+    lib_dir = os.path.dirname(kvc.LIB_PATH)
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "use_kvc.c")
+        open(c, "w").write(prog)
+        exe = os.path.join(d, "use_kvc")
+        subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), c, "-o", exe,
+                        "-L", lib_dir, "-lkvc", "-Wl,-rpath," + lib_dir], check=True)
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()
+    assert out == ["1", "1", "KVC_ERR_ARG", "1", "1", "null", "cache"]
