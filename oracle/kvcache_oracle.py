@@ -49,7 +49,7 @@ What it follows (the web pages are cited by title and section):
 
 Readings taken where the pages are silent (each is also listed in the design
 notes): the order append -> attend -> commit/evict; lowest-free page allocation;
-population variance; the fp64 evaluation order of the score; ties broken by the
+population variance; the raw score as the fp32 rounding of the exactly summed fp64 norm; ties broken by the
 lower token id; protected tokens never absorb merges; merges applied
 simultaneously from pre-merge values in ascending source id and rounded once to
 bf16; the FP8 scale fp32(amax / 448) and codes RNE-satfinite of fp32(x / scale);
@@ -533,12 +533,12 @@ class StreamOracle:
                 np.stack([L.pages[e[0]].v_tok_scale for e in L.entries]))
 
     # ---------------------------------------------------------------- CLCES scoring
-    def score(self, layer: int, t: int, residual: np.ndarray) -> np.ndarray:
+    def score(self, layer: int, t: int, residual: np.ndarray, s_choice: Optional[Dict[int, float]] = None) -> np.ndarray:
         """Enhanced importance s_hat of frame t's tokens at ``layer``.
 
-        s_i: fp32 of sqrt(sum_c r_ic^2), the squares summed in fp64 per block of 32
-        consecutive channels (ascending c within the block), then the block sums in
-        ascending block order (the pages fix no summation order).
+        s_i: fp32 of sqrt(sum_c r_ic^2), the sum of the fp64 squares taken exactly and
+        rounded once (math.fsum; the pages fix no summation order, and any order the GPU
+        takes is allowed for in the tests by its error bound).
         R_i: rank of token i among the frame's T tokens, s descending, ties to the
         lower slot; history kept for the last n = min(W, number of layers scored
         this frame) layers and reset at each new frame. With N = T,
@@ -546,6 +546,10 @@ class StreamOracle:
         Cons_i = max(0, 1 - sigma_i sqrt(12)), s_hat_i = fp32(s_i (1 + lambda Cons_i)),
         each step one fp64 operation in this order. The scores are stored with the
         frame's tokens in the cache.
+
+        s_choice (tests only) maps token slots to the other fp32 neighbour of the exact
+        norm, for tokens whose rounding to fp32 another correct evaluation order may
+        decide the other way; any other value is refused.
         """
         cfg = self.cfg
         r = np.asarray(residual, np.float64)
@@ -553,14 +557,14 @@ class StreamOracle:
         if t != self._rank_frame:
             self._rank_hist = {}
             self._rank_frame = t
-        R = r.shape[1]
-        acc = np.zeros(T)
-        for b0 in range(0, R, 32):
-            blk = np.zeros(T)
-            for c in range(b0, min(b0 + 32, R)):
-                blk = blk + r[:, c] * r[:, c]
-            acc = acc + blk
+        acc = np.array([math.fsum(row * row) for row in r])
         s = to_f32(np.sqrt(acc))
+        for i, v in (s_choice or {}).items():
+            f = np.float32(s[i])
+            if float(v) not in (float(f), float(np.nextafter(f, np.float32(np.inf))),
+                                float(np.nextafter(f, np.float32(-np.inf)))):
+                raise ValueError(f"token {i}: {v} is not an fp32 neighbour of the norm")
+            s[i] = float(v)
         order = sorted(range(T), key=lambda i: (-s[i], i))
         R = np.empty(T, np.int64)
         R[np.array(order)] = np.arange(T)
@@ -600,10 +604,19 @@ class StreamOracle:
             prot |= frame == 0
         return prot
 
-    def compress(self, layer: int):
+    # Two fp64 evaluations of one cosine of 1,024-dim keys (the dot product and the norms,
+    # summed in any order) differ by at most about 2 * 1,028 * 2^-53 = 2.3e-13; targets
+    # whose cosines are within COS_TIE of the best are ties that the order may decide.
+    COS_TIE = 1e-12
+
+    def compress(self, layer: int, target_choice: Optional[Dict[int, int]] = None):
         """Keep / merge / drop the committed cache of ``layer`` when it holds more than B
         tokens. Returns None when nothing happens, else a dict with the kept ids,
-        the (source id, target id) merge pairs and the dropped ids."""
+        the (source id, target id) merge pairs and the dropped ids.
+
+        target_choice (tests only) maps merge-source ids to another side's target id; it is
+        followed where that target's cosine ties the best within COS_TIE, and refused
+        (ValueError) otherwise."""
         cfg, P = self.cfg, self.P
         L = self.layers[layer]
         if L.pending is not None:
@@ -640,8 +653,16 @@ class StreamOracle:
             Mn = np.sqrt((M * M).sum(axis=1))
             cos = (M @ E.T) / (En[None, :] * Mn[:, None])
             best = np.argmax(cos, axis=1)
+            epos = {int(ids[j]): e for e, j in enumerate(eligible)}
             for r, m in enumerate(merged):
-                targets[m] = eligible[int(best[r])]
+                b = int(best[r])
+                if target_choice is not None and int(ids[m]) in target_choice:
+                    alt = epos.get(int(target_choice[int(ids[m])]))
+                    if alt is None or cos[r, alt] < cos[r, b] - self.COS_TIE:
+                        raise ValueError(f"merge source {int(ids[m])}: target "
+                                         f"{target_choice[int(ids[m])]} neither the best nor tied with it")
+                    b = alt
+                targets[m] = eligible[b]
         else:
             dropped = sorted(dropped + merged)
             merged = []

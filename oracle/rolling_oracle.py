@@ -18,19 +18,16 @@ recipe, with its concrete mini-example):
 * Attention of the current frame runs after the pruning, over the anchor and the kept
   tokens.
 
-Readings taken where the page is silent (each is also listed in the design notes):
-the fp64 evaluation order below (every sum over the dims -- the squares of a norm, the
-terms of a dot product -- taken in blocks of 8 consecutive dims, ascending within a block,
-then the block sums in ascending order; a key is normalised by multiplying it with the
-correctly rounded reciprocal of its norm; every sum over candidates -- the
-normalised keys for the mean, whose direction equals that of the sum, and the scores for
-a head's total -- taken in blocks of 32 consecutive candidates in ascending token id,
-ascending within a block, then the block sums in ascending block order); a zero key has
-no direction and scores 0; ties are broken by the lower token
-id; the kept tokens are stored in ascending id; pruning starts with the second frame;
-the budget of layer l is floor(L * K * softmax(mean diversity / tau)_l), computed from
-the previous frame's layer averages by the caller (the page gives neither the
-temperature nor when budgets are recomputed).
+Readings taken where the page is silent (each is also listed in the design notes): a
+candidate's score is the plain definition, -cos(k_i, mu) = -(k_i . mu) / (|k_i| |mu|) with
+mu the mean of the normalised candidate keys k_i / |k_i|, evaluated in fp64 by numpy in
+whatever order its routines take (the page fixes no order; the GPU tests allow for the
+rounding of any order by a bound derived from the sums' lengths); a zero key has no
+direction and scores 0, and so does every candidate when mu = 0; ties are broken by the
+lower token id; the kept tokens are stored in ascending id; pruning starts with the second
+frame; the budget of layer l is floor(L * K * softmax(mean diversity / tau)_l), the mean
+diversity being the mean score over all heads' candidates of the layer's last pruning (the
+page gives neither the temperature nor when budgets are recomputed).
 
 Nothing here is pinned only to itself: tests/test_oracle_rolling.py checks it against
 scipy's cosine distance and softmax, brute-force Top-K, the page's worked numbers and
@@ -44,66 +41,35 @@ from typing import List, Optional, Sequence
 import numpy as np
 
 
-CAND_BLOCK = 32          # candidates per block of every sum over candidates
-DIM_BLOCK = 8            # dims per block of every sum over the dims
-
-
-def dim_sum(terms: np.ndarray) -> np.ndarray:
-    """Sum over the last axis in blocks of DIM_BLOCK entries: ascending within each block,
-    then the block sums ascending. Every addition is one IEEE fp64 operation."""
-    terms = np.asarray(terms, np.float64)
-    D = terms.shape[-1]
-    total = np.zeros(terms.shape[:-1])
-    for d0 in range(0, D, DIM_BLOCK):
-        part = np.zeros(terms.shape[:-1])
-        for d in range(d0, min(d0 + DIM_BLOCK, D)):
-            part = part + terms[..., d]
-        total = total + part
-    return total
-
-
-def blocked_sum(x: np.ndarray) -> np.ndarray:
-    """Sum over axis 0 in blocks of CAND_BLOCK rows: ascending within each block, then the
-    block sums ascending. Every addition is one IEEE fp64 operation."""
-    x = np.asarray(x, np.float64)
-    total = np.zeros(x.shape[1:])
-    for b0 in range(0, x.shape[0], CAND_BLOCK):
-        part = np.zeros(x.shape[1:])
-        for i in range(b0, min(b0 + CAND_BLOCK, x.shape[0])):
-            part = part + x[i]
-        total = total + part
-    return total
-
-
 def normalised_keys(Kc: np.ndarray) -> np.ndarray:
-    """k_hat_i = k_i * RN(1 / |k_i|), |k_i| = sqrt of the dim_sum of the squares; a zero
-    key gives k_hat = 0."""
+    """k_hat_i = k_i / |k_i|; a zero key has no direction and gives k_hat = 0."""
     Kc = np.asarray(Kc, np.float64)
-    N = Kc.shape[0]
-    norms = np.sqrt(dim_sum(Kc * Kc))
-    rcp = np.zeros(N)
+    norms = np.linalg.norm(Kc, axis=1)
+    out = np.zeros_like(Kc)
     nz = norms > 0
-    rcp[nz] = 1.0 / norms[nz]
-    return Kc * rcp[:, None]
+    out[nz] = Kc[nz] / norms[nz, None]
+    return out
 
 
 def diversity_scores(Kc: np.ndarray) -> np.ndarray:
     """Scores of one (layer, head)'s candidates. Kc: [N, D] keys in ascending token id.
 
-    k_hat_i = k_i * (1 / |k_i|) (|k_i| = sqrt of the dim_sum of the squares, its
-    reciprocal rounded once; a zero key gives k_hat = 0); mu = the blocked sum of the
-    k_hat_i; score_i = -(k_hat_i . mu) / |mu| (dot and |mu|^2 as dim_sums of the products).
-    Every step is one IEEE fp64 operation.
+    mu = the mean of the normalised candidate keys; score_i = -cos(k_i, mu)
+    = -(k_i . mu) / (|k_i| |mu|). A zero key scores 0; every score is 0 when mu = 0.
     """
     Kc = np.asarray(Kc, np.float64)
     N, D = Kc.shape
-    khat = normalised_keys(Kc)
-    mu = blocked_sum(khat) if N else np.zeros(D)
-    mnorm = math.sqrt(float(dim_sum(mu * mu)))
+    if N == 0:
+        return np.zeros(0)
+    mu = normalised_keys(Kc).mean(axis=0)
+    mnorm = float(np.linalg.norm(mu))
     if mnorm == 0.0:
         return np.zeros(N)
-    dot = dim_sum(khat * mu[None, :])
-    return -(dot / mnorm)
+    knorm = np.linalg.norm(Kc, axis=1)
+    out = np.zeros(N)
+    nz = knorm > 0
+    out[nz] = -((Kc[nz] @ mu) / (knorm[nz] * mnorm))
+    return out
 
 
 def top_k(scores: np.ndarray, ids: np.ndarray, k: int) -> np.ndarray:
@@ -145,8 +111,8 @@ class RollingOracle:
         self.mut_k = [[np.zeros((0, D)) for _ in range(H)] for _ in range(L)]
         self.mut_v = [[np.zeros((0, D)) for _ in range(H)] for _ in range(L)]
         self.pending = [None] * L                 # (ids, K [T,H,D], V) of the frame appended last
-        self.score_sum = [None] * L               # per head: fp64 sum of the last scores
-        self.cand_count = [0] * L
+        self.last_scores = [None] * L             # per head: scores of the last pruning's candidates
+        self.last_cands = [None] * L              # per head: (ids, K, V) of those candidates
 
     def set_budgets(self, budgets: Sequence[int]):
         self.budgets = [int(b) for b in budgets]
@@ -169,28 +135,36 @@ class RollingOracle:
         if pend is None:
             return
         ids_new, K, V = pend
-        sums = []
+        scores, cands = [], []
         for h in range(self.H):
             ids = np.concatenate([self.mut_ids[layer][h], ids_new])
             Kc = np.concatenate([self.mut_k[layer][h], K[:, h, :]])
             Vc = np.concatenate([self.mut_v[layer][h], V[:, h, :]])
             sc = diversity_scores(Kc)
-            sums.append(float(blocked_sum(sc[:, None])[0]))
+            scores.append(sc)
+            cands.append((ids, Kc, Vc))
             keep = top_k(sc, ids, self.budgets[layer])
             self.mut_ids[layer][h] = ids[keep]
             self.mut_k[layer][h] = Kc[keep]
             self.mut_v[layer][h] = Vc[keep]
-            self.cand_count[layer] = len(ids)
-        self.score_sum[layer] = sums
+        self.last_scores[layer] = scores
+        self.last_cands[layer] = cands
         self.pending[layer] = None
+
+    def set_kept(self, layer: int, h: int, kept_ids: Sequence[int]):
+        """Make head h keep `kept_ids` out of its last pruning's candidates instead of its
+        own Top-K. Tests use this where the Top-K is not unique within the rounding of the
+        scores: the other side's choice among the tied candidates is then followed."""
+        ids, Kc, Vc = self.last_cands[layer][h]
+        pos = {int(x): i for i, x in enumerate(ids)}
+        sel = sorted(pos[int(x)] for x in kept_ids)
+        self.mut_ids[layer][h] = ids[sel]
+        self.mut_k[layer][h] = Kc[sel]
+        self.mut_v[layer][h] = Vc[sel]
 
     def layer_diversity(self, layer: int) -> float:
         """Mean score over all heads' candidates of the layer's last pruning."""
-        sums = self.score_sum[layer]
-        tot = 0.0
-        for s in sums:                            # heads ascending
-            tot = tot + s
-        return tot / float(self.H * self.cand_count[layer])
+        return float(np.mean(np.concatenate(self.last_scores[layer])))
 
     def head_ids(self, layer: int, h: int) -> np.ndarray:
         """Token ids attended by head h (anchor, then the kept tokens), ascending."""

@@ -7,6 +7,7 @@ from fractions import Fraction
 import numpy as np
 import pytest
 
+from kvc_streams import WORKLOADS
 from oracle import OracleConfig, StreamOracle, to_f32
 
 
@@ -167,3 +168,19 @@ def test_planted_sample_variance_is_caught(monkeypatch):
     monkeypatch.setattr(ko.StreamOracle, "score", score)
     with pytest.raises(AssertionError):
         test_sigma_matches_library_population_variance()
+
+
+def test_s_choice_takes_only_an_fp32_neighbour_of_the_norm():
+    # the oracle follows another side's fp32 rounding of a norm only where it is the
+    # adjacent fp32 value; two steps away is refused
+    wl = WORKLOADS["vggt_budget_16k"].replace(tokens_per_frame=16, num_heads=2, residual_dim=32, num_layers=1)
+    r = np.random.default_rng(4).standard_normal((16, 32)).astype(np.float32).astype(np.float64)
+    exact = math.sqrt(math.fsum(float(v) * float(v) for v in r[3]))
+    f = np.float32(exact)
+    up1 = float(np.nextafter(f, np.float32(np.inf)))
+    up2 = float(np.nextafter(np.float32(up1), np.float32(np.inf)))
+    orc = StreamOracle(OracleConfig.from_workload(wl))
+    sh = orc.score(0, 0, r, s_choice={3: up1})
+    assert sh[3] == float(np.float32(up1 * 1.5))       # one layer: Cons = 1
+    with pytest.raises(ValueError):
+        StreamOracle(OracleConfig.from_workload(wl)).score(0, 0, r, s_choice={3: up2})

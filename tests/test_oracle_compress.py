@@ -166,3 +166,56 @@ def test_planted_least_similar_target_is_caught(monkeypatch):
     monkeypatch.setattr(ko, "np", NP())
     with pytest.raises(AssertionError):
         _compression_check()
+
+
+# ------------------------------------------------------------------ validated alternatives
+# A test may make the oracle follow the GPU where two correct fp64 evaluations can differ;
+# the oracle accepts only what the definitions allow.
+
+def _one_event(target_choice=None, dup=False):
+    """A budget stream up to its first compression; with `dup`, frame 2's keys and
+    residuals are copies of frame 1's, so the twins have equal scores and a source's
+    cosines to the two copies of a target are equal."""
+    wl = _small_wl(num_layers=1)
+    st = FrameStream(wl, seed=3)
+    orc = StreamOracle(OracleConfig.from_workload(wl))
+    keep = {}
+    for t in range(12):
+        q, k, v = (_np(x) for x in st.frame(0, t))
+        r = _np(st.residual(0, t))
+        if dup and t in (1, 2):
+            k = keep.setdefault("k", k)
+            r = keep.setdefault("r", r)
+        orc.append(0, t, k, v, True)
+        orc.attend(0, q)
+        orc.score(0, t, r)
+        res = orc.compress(0, target_choice=target_choice)
+        if res is not None:
+            return orc, res
+    raise AssertionError("no compression event")
+
+
+def test_target_choice_refuses_a_target_that_is_not_tied():
+    _, res = _one_event()
+    src, dst = res["merge_src"], res["merge_dst"]
+    others = [int(i) for i in res["kept_ids"] if int(i) not in set(dst.tolist()) and int(i) // 8 != 0 and int(i) % 8]
+    assert others
+    with pytest.raises(ValueError):
+        _one_event(target_choice={int(src[0]): others[0]})
+
+
+def test_target_choice_follows_an_exact_tie():
+    # identical keys in frames 1 and 2: a source's cosine to the two copies of a target is
+    # the same number, so either copy is a correct target
+    _, res = _one_event(dup=True)
+    tie = None
+    for s_id, d_id in zip(res["merge_src"], res["merge_dst"]):
+        twin = int(d_id) + 8 if int(d_id) // 8 == 1 else int(d_id) - 8 if int(d_id) // 8 == 2 else None
+        if twin is not None and twin in set(res["kept_ids"].tolist()) and twin % 8:
+            tie = (int(s_id), twin)
+            break
+    if tie is None:
+        pytest.skip("no merge into a duplicated key on this seed")
+    _, res2 = _one_event(target_choice={tie[0]: tie[1]}, dup=True)
+    got = dict(zip(res2["merge_src"].tolist(), res2["merge_dst"].tolist()))
+    assert got[tie[0]] == tie[1]

@@ -164,29 +164,6 @@ def test_planted_sign_mistake_is_caught(monkeypatch):
     assert np.argmax(ro.diversity_scores(Kc)) != n
 
 
-def test_blocked_sum_order_hand_derived():
-    # 2^53 then 63 ones. Sequential: every +1 is a tie at 2^53 that rounds to even, so the
-    # ones vanish (2^53). Blocked: block 0 (2^53 and 31 ones) gives 2^53, block 1 (32 ones)
-    # gives 32 exactly, and 2^53 + 32 is representable.
-    x = np.array([2.0 ** 53] + [1.0] * 63)
-    assert ro.blocked_sum(x[:, None])[0] == 2.0 ** 53 + 32.0
-    seq = 0.0
-    for v in x:
-        seq += v
-    assert seq == 2.0 ** 53                      # the orders really differ here
-
-
-def test_blocked_sum_close_to_exact_sum():
-    import math
-    rng = np.random.default_rng(9)
-    for n in (1, 31, 32, 33, 1516):
-        x = rng.standard_normal((n, 3))
-        got = ro.blocked_sum(x)
-        for d in range(3):
-            exact = math.fsum(x[:, d])
-            assert abs(got[d] - exact) <= n * 2.0 ** -52 * np.sum(np.abs(x[:, d]))
-
-
 def test_layer_diversity_is_mean_of_scores():
     rng = np.random.default_rng(10)
     L, H, D, T, K = 1, 3, 16, 40, 50
@@ -203,22 +180,23 @@ def test_layer_diversity_is_mean_of_scores():
         assert abs(orc.layer_diversity(0) - mean) < 1e-13
 
 
-def test_normalisation_by_rounded_reciprocal_hand_derived():
-    # |(3, 4)| = 5; RN(1/5) = 3602879701896397 / 2^54. Times 3 the exact product is
-    # 10808639105689191 / 2^54 = 5404319552844595.5 / 2^53, a tie that rounds to the even
-    # 5404319552844596 / 2^53: one ulp above RN(3/5). Times 4 it is exact: RN(4/5).
-    kh = ro.normalised_keys(np.array([[3.0, 4.0]]))
-    assert kh[0, 0] == 5404319552844596 / 2.0 ** 53 and kh[0, 0] != 3.0 / 5.0
-    assert kh[0, 1] == 7205759403792794 / 2.0 ** 53 == 4.0 / 5.0
-    assert np.array_equal(ro.normalised_keys(np.zeros((1, 4))), np.zeros((1, 4)))
+def test_normalisation_is_division_by_the_norm():
+    # |(3, 4)| = 5 exactly, so the unit key is (3/5, 4/5), each one IEEE division; a zero
+    # key stays zero
+    kh = ro.normalised_keys(np.array([[3.0, 4.0], [0.0, 0.0]]))
+    assert kh[0, 0] == 3.0 / 5.0 and kh[0, 1] == 4.0 / 5.0
+    assert np.array_equal(kh[1], [0.0, 0.0])
 
 
-def test_dim_sum_order_hand_derived():
-    # 16 dims: 2^53, then 15 ones. Block 0 (2^53 and 7 ones): every +1 is a tie at 2^53
-    # that rounds to even, 2^53. Block 1 (8 ones): 8 exactly. Total 2^53 + 8, representable.
-    x = np.array([[2.0 ** 53] + [1.0] * 15])
-    assert ro.dim_sum(x)[0] == 2.0 ** 53 + 8.0
-    np.testing.assert_array_equal(ro.dim_sum(np.arange(64.0)[None, :]), [2016.0])   # exact integers
+def test_mean_and_sum_give_the_same_scores():
+    # the cosine to the mean of the unit keys equals the cosine to their sum (same
+    # direction): the scores against an explicit sum-based evaluation
+    rng = np.random.default_rng(12)
+    Kc = rng.standard_normal((77, 64))
+    kh = Kc / np.linalg.norm(Kc, axis=1, keepdims=True)
+    mu = kh.sum(axis=0)
+    want = -(Kc @ mu) / (np.linalg.norm(Kc, axis=1) * np.linalg.norm(mu))
+    np.testing.assert_allclose(diversity_scores(Kc), want, rtol=0, atol=1e-14)
 
 
 # ------------------------------------------------------------------ planted mistakes
