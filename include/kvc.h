@@ -107,7 +107,14 @@ typedef struct {
                                    kvc_attend; the evicted frames whose special tokens stay */
   int32_t fp8_dim_adaptive;     /* 1 with kv_dtype FP8 (D = 64, P = 16): dimension-adaptive
                                    scales, see kvc_append_frame; 0: one scale per (page, head) */
-  int32_t reserved[4];          /* must be zero */
+  int32_t model_heads;          /* heads of the caller's Q/K/V/O tensors; 0 = num_heads. With
+                                   model_heads > num_heads the cache holds the head range below
+                                   (bf16 window caches on the tensor-core path only) */
+  int32_t head_begin;           /* first of the num_heads consecutive model heads the cache
+                                   holds: kvc_append_frame reads that slice of [T, model_heads, D]
+                                   K and V, kvc_attend reads the slice of Q and writes the same
+                                   slice of O (other heads of O untouched) */
+  int32_t reserved[2];          /* must be zero */
 } kvc_config;
 
 /* Cache statistics ([GCT] Cache Monitoring: occupancy, memory use, eviction status). */
@@ -185,7 +192,10 @@ KVC_API kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const v
  * beyond special_frames such frames the oldest one's pages are freed. A non-keyframe
  * keeps nothing.
  * bf16 with D = 64 runs on tcgen05 tensor cores (fp32 accumulation); fp32 I/O
- * runs fp32 FMA arithmetic. Errors: KVC_ERR_STATE if nothing is pending. */
+ * runs fp32 FMA arithmetic. With FP8 storage the tensor cores take Q as f16: each query
+ * row is first multiplied by the power of two that puts its largest magnitude in
+ * [2^14, 2^15) (and its logits by the inverse), so every finite bf16 query is accepted
+ * and none overflows. Errors: KVC_ERR_STATE if nothing is pending. */
 KVC_API kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_dev);
 
 /* The joint scale-frame phase ([GCT] Scale-Frame Phase): the first n_frames frames of a
@@ -204,7 +214,9 @@ KVC_API kvc_status kvc_scale_phase(kvc_cache* c, int32_t layer, int32_t n_frames
  * kvc_attend of the same frame; within a frame layers are scored in ascending
  * order (the rank history covers the last rank_window layers of this frame and
  * is reset when a new frame starts). residual_dev [T, R] fp32 gives the raw
- * score s_i = fp32(sqrt(sum_c r_ic^2)) (fp64 sum, ascending c). Scores:
+ * score s_i = fp32(sqrt(sum_c r_ic^2)), the squares summed in fp64 (each lane of a
+ * warp sums 32 consecutive channels in ascending order, then the 32 lane sums are
+ * added in lane order). Scores:
  * rank R (s descending, ties lower slot), sigma from the population variance
  * of R/(T-1) over the window, Cons = max(0, 1 - sigma sqrt(12)),
  * s_hat = fp32(s (1 + lambda Cons)) evaluated in fp64. Compression: protected
@@ -233,6 +245,13 @@ KVC_API kvc_status kvc_page_table(kvc_cache* c, int32_t layer, int32_t* rows_hos
 KVC_API kvc_status kvc_token_meta(kvc_cache* c, int32_t layer, int64_t* ids_host, int32_t* counts_host,
                           float* shat_host, int32_t capacity, int32_t* n_out);
 
+/* Synchronise and copy the raw scores s_i (fp32, one per token slot of the frame) that
+ * the last kvc_compress call computed from its residual ([SCV] 2.1.1: the L2 norm of the
+ * FFN residual), for inspection. s_host: host array of `capacity` >= tokens_per_frame
+ * floats; *n_out receives tokens_per_frame. Errors: KVC_ERR_ARG (budget_tokens is 0,
+ * capacity too small), KVC_ERR_STATE (nothing scored yet). */
+KVC_API kvc_status kvc_last_raw_scores(kvc_cache* c, float* s_host, int32_t capacity, int32_t* n_out);
+
 /* Synchronise and copy the (source id, target id) pairs of the last
  * compression of `layer`, in ascending source id. */
 KVC_API kvc_status kvc_last_merge(kvc_cache* c, int32_t layer, int64_t* src_host, int64_t* dst_host,
@@ -254,7 +273,8 @@ KVC_API kvc_status kvc_export_fp8_group_scales(kvc_cache* c, int32_t layer, int3
 
 /* One whole frame step of `layer` from HOST buffers: copy q, k, v [T, H, D]
  * host -> device, append, attend (+ commit/evict), copy O device -> host,
- * and wait for the copy. Pinned host memory gives full copy bandwidth. */
+ * and wait for the copy. Pinned host memory gives full copy bandwidth. Caches that hold
+ * a head range (model_heads > num_heads) are refused with KVC_ERR_ARG. */
 KVC_API kvc_status kvc_step_host(kvc_cache* c, int32_t layer, int32_t frame_idx, int32_t is_keyframe,
                          const void* q_host, const void* k_host, const void* v_host, void* o_host);
 
@@ -289,6 +309,18 @@ KVC_API kvc_status kvc_step_host_async(kvc_cache* c, int32_t layer, int32_t fram
  * this mode). */
 KVC_API kvc_status kvc_set_layer_budgets(kvc_cache* c, const int32_t* budgets, int32_t n);
 
+/* Layer-wise adaptive budgets computed by the library ([IVG] Layer-wise adaptive budgets:
+ * each layer's share of the total budget is a softmax, with temperature tau, of the
+ * layers' mean diversity). From every layer's last pruning, mean_l = (the heads' fp64
+ * score sums, in head order) / (H x candidates), p = softmax(mean / tau) in fp64 and
+ * budget_l = floor(L * k_avg * p_l), clamped to [1, diversity_budget] (a layer keeps at
+ * least one token besides the anchor, and no more than its pool holds; the page states
+ * neither bound). tau <= 0 gives every layer k_avg (clamped likewise). The budgets apply
+ * from the next pruning, as with kvc_set_layer_budgets; budgets_out (host, num_layers
+ * values) may be NULL. Synchronises. Errors: KVC_ERR_ARG (k_avg < 1, tau NaN),
+ * KVC_ERR_STATE (not in this mode, or a layer never pruned). */
+KVC_API kvc_status kvc_adapt_layer_budgets(kvc_cache* c, double tau, int32_t k_avg, int32_t* budgets_out);
+
 /* The pruning step alone ([IVG] Step-by-step recipe: prune, then attend): scores every
  * head's candidates (kept tokens + the pending frame) and keeps each head's Top-K; the
  * pending frame stays pending for kvc_attend, which then only attends. Enqueued on the
@@ -297,8 +329,9 @@ KVC_API kvc_status kvc_set_layer_budgets(kvc_cache* c, const int32_t* budgets, i
 KVC_API kvc_status kvc_prune(kvc_cache* c, int32_t layer);
 
 /* Mean diversity score of the layer's last pruning over all heads' candidates (fp64:
- * per head the scores summed in ascending token id, then the heads in order, divided by
- * H * candidates). Synchronises. Errors: KVC_ERR_STATE if the layer was never pruned. */
+ * per head the scores summed in blocks of 32 consecutive candidates in ascending token
+ * id, then the block sums in order; then the heads in order, divided by H * candidates).
+ * Synchronises. Errors: KVC_ERR_STATE if the layer was never pruned. */
 KVC_API kvc_status kvc_layer_diversity(kvc_cache* c, int32_t layer, double* mean_out);
 
 /* Token ids (frame * T + slot) that head `head` of `layer` attends, in cache order

@@ -80,16 +80,24 @@ def top_k(scores: np.ndarray, ids: np.ndarray, k: int) -> np.ndarray:
     return np.array(sorted(keep, key=lambda i: ids[i]), dtype=np.int64)
 
 
-def layer_budgets(mean_diversity: Sequence[float], tau: float, k: int) -> List[int]:
+def layer_budgets(mean_diversity: Sequence[float], tau: float, k: int, lo: Optional[int] = None,
+                  hi: Optional[int] = None) -> List[int]:
     """Per-layer, per-head budgets floor(L * k * softmax(mean_diversity / tau)_l); tau <= 0
-    gives every layer k."""
+    gives every layer k. With lo / hi each budget is clamped to [lo, hi] (reading: a layer
+    keeps at least one token and no more than its pool holds; the page states no bound)."""
     L = len(mean_diversity)
     if tau <= 0:
-        return [int(k)] * L
-    z = np.asarray(mean_diversity, np.float64) / tau
-    e = np.exp(z - z.max())
-    p = e / e.sum()
-    return [int(math.floor(L * k * float(pl))) for pl in p]
+        b = [int(k)] * L
+    else:
+        z = np.asarray(mean_diversity, np.float64) / tau
+        e = np.exp(z - z.max())
+        p = e / e.sum()
+        b = [int(math.floor(L * k * float(pl))) for pl in p]
+    if lo is not None:
+        b = [max(int(lo), x) for x in b]
+    if hi is not None:
+        b = [min(int(hi), x) for x in b]
+    return b
 
 
 class RollingOracle:

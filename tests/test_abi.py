@@ -38,8 +38,9 @@ def test_struct_layout_matches_header():
 #include <stddef.h>
 #include "kvc.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu %zu\n", sizeof(kvc_config), sizeof(kvc_info), offsetof(kvc_config, softmax_scale),
-         offsetof(kvc_config, kv_splits), offsetof(kvc_config, reserved), offsetof(kvc_info, device_error));
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(kvc_config), sizeof(kvc_info), offsetof(kvc_config, softmax_scale),
+         offsetof(kvc_config, kv_splits), offsetof(kvc_config, model_heads), offsetof(kvc_config, head_begin),
+         offsetof(kvc_config, reserved), offsetof(kvc_info, device_error));
   return 0;
 }'''
     with tempfile.TemporaryDirectory() as d:
@@ -50,7 +51,7 @@ int main(void) {
         vals = [int(x) for x in subprocess.run([exe], capture_output=True, text=True).stdout.split()]
     C, I = kvc.kvc_config, kvc.kvc_info
     assert vals == [ctypes.sizeof(C), ctypes.sizeof(I), C.softmax_scale.offset, C.kv_splits.offset,
-                    C.reserved.offset, I.device_error.offset]
+                    C.model_heads.offset, C.head_begin.offset, C.reserved.offset, I.device_error.offset]
 
 
 def test_host_only_calls_and_config_validation():
@@ -117,7 +118,7 @@ def test_reserved_config_words_must_be_zero():
     import transformer_kv_cache_b200 as kvc
     from kvc_streams import WORKLOADS
     cfg = kvc.config_from_workload(WORKLOADS["vggt_518x378"])
-    cfg.reserved[2] = 7
+    cfg.reserved[1] = 7
     with pytest.raises(kvc.KVCError) as e:
         kvc.kvc_create(cfg, stream=0)
     assert e.value.status_name == "KVC_ERR_ARG"

@@ -75,6 +75,59 @@ def test_fp8_tensor_core(kvc, T, H, splits):
     run_parity(kvc, wl, 10, kv_splits=splits, check_pages=True)
 
 
+def test_fp8_queries_beyond_the_f16_range(kvc):
+    """The FP8 path feeds Q to the tensor cores as f16 (largest finite value 65,504). Query
+    rows far above that range (x 2^30) and far below f16's smallest normal (x 2^-20) are
+    scaled per row by a power of two, exactly, and match the oracle. The softmax scale is
+    2^-30 times the usual one, so the large rows' logits are the usual well-conditioned
+    ones and the other rows' logits are near zero (near-uniform weights), all resolvable in
+    fp32; a split over several CTAs is included."""
+    wl = WORKLOADS["vggt_518x518_fp8"].replace(tokens_per_frame=150, num_heads=4, window_frames=4, scale_frames=2,
+                                                softmax_scale=0.125 * 2.0 ** -30)
+
+    def scale_q(t, layer, q, k, v):
+        q = q.clone()
+        q[0:60] *= 2.0 ** 30
+        q[60:80] *= 2.0 ** -20
+        q[80:85, 1] *= 2.0 ** 30
+        return q, k, v
+    for splits in (0, 3):
+        run_parity(kvc, wl, 8, transform=scale_q, kv_splits=splits)
+
+
+def test_head_range_caches_rebuild_the_full_output(kvc):
+    """Two caches holding heads [0, 2) and [2, 4) of a 4-head model (model_heads = 4,
+    head_begin = 0 and 2) take the same full-width Q, K and V; each writes only its slice of
+    O, and the two slices together equal the oracle's full output. Page tables of both
+    equal the full cache's (allocation does not depend on the heads)."""
+    wl = WORKLOADS["vggt_518x378"].replace(tokens_per_frame=300, num_heads=4, window_frames=3, scale_frames=1)
+    half = wl.replace(num_heads=2)
+    T, D = wl.tokens_per_frame, wl.head_dim
+    dev = torch.device("cuda")
+    hs = [kvc.kvc_create(kvc.config_from_workload(half, model_heads=4, head_begin=b)) for b in (0, 2)]
+    try:
+        st = FrameStream(wl, seed=17, device=dev)
+        orc = StreamOracle(OracleConfig.from_workload(wl))
+        for t in range(8):
+            q, k, v = st.frame(0, t)
+            o = torch.full((T, 4, D), float("nan"), dtype=torch.bfloat16, device=dev)
+            for i, h in enumerate(hs):
+                kvc.kvc_append_frame(h, 0, t, k, v, True)
+                kvc.kvc_attend(h, 0, q, o)
+                torch.cuda.synchronize()
+                written = torch.isfinite(o.float()).all(dim=2).all(dim=0)
+                assert written.tolist() == [True, True, i == 1, i == 1], (t, i)
+            orc.append(0, t, np64(k), np64(v), True)
+            ref = orc.attend(0, np64(q))
+            compare_out(np64(o), ref, "bf16", f"frame {t}")
+            for h in hs:
+                pt, info = kvc.kvc_page_table(h, 0)
+                assert np.array_equal(pt, orc.page_table(0)) and info["device_error"] == 0
+    finally:
+        for h in hs:
+            kvc.kvc_destroy(h)
+
+
 def test_fp8_zero_blocks(kvc):
     """All-zero K or V blocks quantise to scale 0 and codes 0; attention over them (the
     first frame's K all zero, then a zero V frame, then both zero) matches the oracle."""

@@ -241,3 +241,13 @@ def test_planted_ties_to_higher_ids_are_caught(monkeypatch):
     monkeypatch.setattr(ro, "top_k", top_k_high)
     with pytest.raises(AssertionError):
         _ties_check()
+
+
+def test_layer_budgets_clamped_to_the_pool():
+    # a sharp softmax gives one layer nearly all of L * k; clamped to [1, cap] the others
+    # keep one token and the favoured layer no more than its pool holds
+    d = [-0.9, -0.1, -0.8]
+    raw = layer_budgets(d, 0.01, 512)
+    assert raw[1] > 512 and min(raw) == 0
+    assert layer_budgets(d, 0.01, 512, lo=1, hi=600) == [max(1, min(600, x)) for x in raw]
+    assert layer_budgets(d, 0.0, 512, lo=1, hi=300) == [300, 300, 300]

@@ -58,7 +58,16 @@ def test_noalloc_attention_matches_kvc_attend_twice():
         assert err.max().item() <= 2e-2 and err.mean().item() <= 2e-3, (call, err.max().item())
         outs.append(o)
     assert torch.equal(outs[0], outs[1])
-    # sizes beyond the fixed scratch are rejected before anything is launched
+    # a split count whose partials exceed the fixed scratch is rejected before anything is
+    # launched; the buffers have the declared shape (8,032 queries, 16 heads, a 4,096-row
+    # table of valid entries on a one-page pool), so a guard that let the call through would
+    # compute a wrong answer rather than read or write out of bounds
+    Tb, Hb, nb = 1004 * 8, 16, 4096
+    qb = torch.zeros((Tb, Hb, D), dtype=torch.bfloat16, device=dev)
+    ob = torch.empty_like(qb)
+    kb = torch.zeros((1, Hb, P, D), dtype=torch.bfloat16, device=dev)
+    vb = torch.zeros_like(kb)
+    tb = torch.tensor([[0, 0, 0, P]] * nb, dtype=torch.int32, device=dev)
     with pytest.raises(kvc.KVCError) as e:
-        kvc.kvc_attend_paged_noalloc(q6, o, kp, vp, n_pages, table, 4096, 1004 * 8, 16, D, P, 0.125, kv_splits=8)
+        kvc.kvc_attend_paged_noalloc(qb, ob, kb, vb, 1, tb, nb, Tb, Hb, D, P, 0.125, kv_splits=8)
     assert e.value.status_name == "KVC_ERR_ARG"

@@ -29,7 +29,8 @@ EXPORTS = ["kvc_create", "kvc_destroy", "kvc_set_stream", "kvc_reset", "kvc_appe
            "kvc_step_host", "kvc_synchronize", "kvc_last_error", "kvc_status_string", "kvc_version",
            "kvc_debug_fail_allocs", "kvc_debug_bounded_wait", "kvc_attend_paged_noalloc", "kvc_append_frame_all",
            "kvc_step_host_async", "kvc_set_layer_budgets", "kvc_prune", "kvc_layer_diversity",
-           "kvc_head_tokens", "kvc_scale_phase", "kvc_export_fp8_group_scales"]
+           "kvc_head_tokens", "kvc_scale_phase", "kvc_export_fp8_group_scales", "kvc_last_raw_scores",
+           "kvc_adapt_layer_budgets"]
 
 
 class kvc_config(ctypes.Structure):
@@ -42,7 +43,8 @@ class kvc_config(ctypes.Structure):
                 ("protect_first_frame", ctypes.c_int32), ("max_frames", ctypes.c_int32),
                 ("kv_splits", ctypes.c_int32), ("diversity_budget", ctypes.c_int32),
                 ("special_frames", ctypes.c_int32), ("fp8_dim_adaptive", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 4)]
+                ("model_heads", ctypes.c_int32), ("head_begin", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 2)]
 
 
 class kvc_info(ctypes.Structure):
@@ -80,10 +82,12 @@ def _load():
         "kvc_page_table": ([vp, i32, i32p, i32, i32p, ctypes.POINTER(kvc_info)], i32),
         "kvc_token_meta": ([vp, i32, i64p, i32p, fp, i32, i32p], i32),
         "kvc_last_merge": ([vp, i32, i64p, i64p, i32, i32p], i32),
+        "kvc_last_raw_scores": ([vp, vp, i32, i32p], i32),
         "kvc_export_pages": ([vp, i32, i32, i32, vp, vp, fp, fp], i32),
         "kvc_step_host": ([vp, i32, i32, i32, vp, vp, vp, vp], i32),
         "kvc_step_host_async": ([vp, i32, i32, i32, vp, vp, vp, vp], i32),
         "kvc_set_layer_budgets": ([vp, vp, i32], i32),
+        "kvc_adapt_layer_budgets": ([vp, ctypes.c_double, i32, vp], i32),
         "kvc_prune": ([vp, i32], i32),
         "kvc_scale_phase": ([vp, i32, i32, vp, vp, vp, vp], i32),
         "kvc_export_fp8_group_scales": ([vp, i32, i32, i32, vp, vp], i32),
@@ -138,7 +142,7 @@ def make_config(num_layers, num_heads, head_dim, tokens_per_frame, num_special_t
                 window_frames, scale_frames, io_dtype="bf16", kv_dtype="bf16", softmax_scale=0.125,
                 budget_tokens=0, keep_frac=0.6, lam=0.5, rank_window=5, residual_dim=1024,
                 protect_first_frame=1, max_frames=0, kv_splits=0, diversity_budget=0,
-                special_frames=0, fp8_dim_adaptive=0) -> kvc_config:
+                special_frames=0, fp8_dim_adaptive=0, model_heads=0, head_begin=0) -> kvc_config:
     c = kvc_config()
     c.num_layers, c.num_heads, c.head_dim = num_layers, num_heads, head_dim
     c.tokens_per_frame, c.num_special_tokens, c.page_size = tokens_per_frame, num_special_tokens, page_size
@@ -152,6 +156,7 @@ def make_config(num_layers, num_heads, head_dim, tokens_per_frame, num_special_t
     c.diversity_budget = diversity_budget
     c.special_frames = special_frames
     c.fp8_dim_adaptive = fp8_dim_adaptive
+    c.model_heads, c.head_begin = model_heads, head_begin
     return c
 
 
@@ -251,6 +256,14 @@ def kvc_last_merge(handle, layer: int, capacity: int = 1 << 20):
     return src[: n.value], dst[: n.value]
 
 
+def kvc_last_raw_scores(handle, capacity: int = 1 << 16):
+    """Raw scores s (fp32, one per token slot) of the last kvc_compress call."""
+    s = np.zeros(capacity, np.float32)
+    n = ctypes.c_int32(0)
+    _check(handle, _lib.kvc_last_raw_scores(handle, s.ctypes.data_as(ctypes.c_void_p), capacity, ctypes.byref(n)))
+    return s[: n.value]
+
+
 def kvc_export_pages(handle, layer: int, first_row: int, n_rows: int, page_bytes: int, num_heads: int,
                      fp8: bool = False):
     """Raw page bytes of rows [first_row, first_row + n_rows): (k uint8 [n, page_bytes], v, k_scale, v_scale)."""
@@ -300,6 +313,15 @@ def kvc_export_fp8_group_scales(handle, layer: int, first_row: int, n_rows: int,
 def kvc_prune(handle, layer: int) -> None:
     """Prune every head of `layer` to its Top-K candidates (the step before kvc_attend)."""
     _check(handle, _lib.kvc_prune(handle, layer))
+
+
+def kvc_adapt_layer_budgets(handle, num_layers: int, tau: float, k_avg: int) -> np.ndarray:
+    """Budgets floor(L * k_avg * softmax(mean diversity / tau)), clamped to [1, diversity_budget],
+    computed by the library from every layer's last pruning and applied from the next one
+    (num_layers: the cache's layer count, the length of the returned array)."""
+    out = np.zeros(num_layers, np.int32)
+    _check(handle, _lib.kvc_adapt_layer_budgets(handle, float(tau), int(k_avg), out.ctypes.data))
+    return out
 
 
 def kvc_layer_diversity(handle, layer: int) -> float:

@@ -35,12 +35,11 @@ cudaError_t dev_alloc_t(T** p, size_t bytes) {
   return e;
 }
 
-// Split counters of the attention kernel: one per (head, 128-row query tile).
-// Split counters of the attention kernel: one per (head, 128-row query tile), for the
-// largest query count (a frame, or the joint phase's S frames).
+// Piece counters of the attention kernel, for the largest query count (a frame, or the
+// joint phase's S frames).
 size_t split_cnt_count(const kvc_config& g) {
   const long long rows = static_cast<long long>(g.tokens_per_frame) * std::max(1, g.scale_frames);
-  return static_cast<size_t>(g.num_heads) * static_cast<size_t>((rows + 127) / 128);
+  return attn_counter_count(rows, g.num_heads);
 }
 
 void free_all(kvc_cache* c) {
@@ -48,7 +47,7 @@ void free_all(kvc_cache* c) {
                   c->d_err,      c->tok_id,     c->tok_cnt,    c->tok_shat,   c->cmp_scratch, c->part_o,
                   c->part_lse,   c->stage_q[0], c->stage_k[0], c->stage_v[0], c->stage_o[0], c->stage_q[1],
                   c->stage_k[1], c->stage_v[1], c->stage_o[1], c->rank_hist, c->div_sums, c->split_cnt,
-                  c->k_chan,     c->v_tok};
+                  c->k_chan,     c->v_tok,      c->bitmap_alt, c->div_cand, c->div_budget};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   for (int i = 0; i < 2; ++i) {
@@ -79,7 +78,7 @@ Entry* layer_entries(kvc_cache* c, int layer) {
   return c->entries + static_cast<size_t>(layer) * (c->per_head ? c->cfg.num_heads : 1) * c->pool_pages;
 }
 uint32_t* layer_bitmap(kvc_cache* c, int layer) {
-  return c->bitmap + static_cast<size_t>(layer) * c->bitmap_words;
+  return c->per_head ? c->bitmap + static_cast<size_t>(layer) * c->bitmap_words : layer_free_bitmap(c, layer);
 }
 uint8_t* layer_pool(kvc_cache* c, uint8_t* pool, int layer) {
   return pool + static_cast<size_t>(layer) * c->pool_pages * c->page_bytes_kv;
@@ -206,8 +205,15 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   if (!cfg || !out) return KVC_ERR_ARG;
   *out = nullptr;
   const kvc_config& g = *cfg;
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 2; ++i)
     if (g.reserved[i] != 0) return KVC_ERR_ARG;
+  // a head range of the caller's tensors: bf16 window caches on the tensor-core path
+  const int mh = g.model_heads > 0 ? g.model_heads : g.num_heads;
+  if (g.model_heads < 0 || g.head_begin < 0 || g.num_heads < 1 || g.head_begin + g.num_heads > mh) return KVC_ERR_ARG;
+  if (mh != g.num_heads &&
+      (g.io_dtype != KVC_BF16 || g.kv_dtype != KVC_BF16 || g.head_dim != 64 || g.page_size != 16 ||
+       g.window_frames <= 0 || g.budget_tokens > 0 || g.diversity_budget > 0))
+    return KVC_ERR_ARG;
   if (g.fp8_dim_adaptive != 0 &&
       (g.fp8_dim_adaptive != 1 || g.kv_dtype != KVC_FP8_E4M3 || g.head_dim != 64 || g.page_size != 16))
     return KVC_ERR_ARG;
@@ -253,6 +259,8 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device);
   const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads, D = g.head_dim;
   c->ppf = (T + P - 1) / P;
+  c->model_heads = g.model_heads > 0 ? g.model_heads : H;
+  c->head0 = g.head_begin;
   c->per_head = g.diversity_budget > 0;
   if (c->per_head) {
     // per head: the anchor frame, the kept pages and one pending frame (pruning compacts
@@ -301,9 +309,12 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   }
   A(dev_alloc_t(&c->entries, NS * c->pool_pages * sizeof(Entry)));
   A(dev_alloc_t(&c->bitmap, NS * c->bitmap_words * sizeof(uint32_t)));
+  if (!c->per_head) A(dev_alloc_t(&c->bitmap_alt, NS * c->bitmap_words * sizeof(uint32_t)));
   if (c->per_head) {
     A(dev_alloc_t(&c->tok_id, NS * c->pool_pages * P * sizeof(int64_t)));
     A(dev_alloc_t(&c->div_sums, NS * sizeof(double)));
+    A(dev_alloc_t(&c->div_cand, L * sizeof(long long)));
+    A(dev_alloc_t(&c->div_budget, L * sizeof(int32_t)));
   }
   A(dev_alloc_t(&c->d_err, 4 * sizeof(int)));
   if (c->tc_path) {
@@ -348,6 +359,7 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   if (c->v_tok) A(cudaMemsetAsync(c->v_tok, 0, L * c->pool_pages * H * P * sizeof(float), c->stream));
   A(cudaMemsetAsync(c->entries, 0, NS * c->pool_pages * sizeof(Entry), c->stream));
   A(cudaMemsetAsync(c->bitmap, 0, NS * c->bitmap_words * sizeof(uint32_t), c->stream));
+  if (c->bitmap_alt) A(cudaMemsetAsync(c->bitmap_alt, 0, NS * c->bitmap_words * sizeof(uint32_t), c->stream));
   if (c->per_head) {
     A(cudaMemsetAsync(c->tok_id, 0xff, NS * c->pool_pages * P * sizeof(int64_t), c->stream));
     A(cudaMemsetAsync(c->div_sums, 0, NS * sizeof(double), c->stream));
@@ -406,6 +418,8 @@ kvc_status kvc_reset(kvc_cache* c) {
   const size_t NS = c->per_head ? L * c->cfg.num_heads : L;
   cudaError_t e = cudaMemsetAsync(c->entries, 0, NS * c->pool_pages * sizeof(Entry), c->stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(c->bitmap, 0, NS * c->bitmap_words * sizeof(uint32_t), c->stream);
+  if (e == cudaSuccess && c->bitmap_alt)
+    e = cudaMemsetAsync(c->bitmap_alt, 0, NS * c->bitmap_words * sizeof(uint32_t), c->stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(c->d_err, 0, 4 * sizeof(int), c->stream);
   if (e == cudaSuccess && c->split_cnt)   // a launch that gave up may have left a count behind
     e = cudaMemsetAsync(c->split_cnt, 0, split_cnt_count(c->cfg) * sizeof(int), c->stream);
@@ -554,21 +568,44 @@ kvc_status kvc_append_frame(kvc_cache* c, int32_t layer, int32_t frame_idx, cons
   if (used + n > c->pool_pages) return fail(c, KVC_ERR_STATE, "kvc_append_frame: page pool full");
   const int T = g.tokens_per_frame, P = g.page_size;
   Entry* E = layer_entries(c, layer);
-  cudaError_t e = launch_mgr_alloc(c->stream, E, layer_bitmap(c, layer), c->bitmap_words, c->pool_pages,
-                                   L.n_entries, n, frame_idx, P, T - (n - 1) * P, c->d_err);
-  if (e != cudaSuccess) return cuda_fail(c, e, "page allocation");
-  c->launches++;
+  cudaError_t e;
+  if (g.kv_dtype != KVC_FP8_E4M3 && append_alloc_fusable(static_cast<int>(c->elem_kv), g.num_heads, g.head_dim, P)) {
+    // allocation and copy in one launch; the layer moves to its other bitmap buffer
+    // (with a head range, the sources start at the first held head; tokens are model_heads
+    // rows apart)
+    const size_t head_off = static_cast<size_t>(c->head0) * g.head_dim * c->elem_kv;
+    AppendBatch in{};
+    in.k[0] = static_cast<const uint8_t*>(k_dev) + head_off;
+    in.v[0] = static_cast<const uint8_t*>(v_dev) + head_off;
+    LayerStarts st{};
+    st.first_layer = layer;
+    st.start[0] = L.n_entries;
+    e = launch_append_alloc_layers(c->stream, static_cast<int>(c->elem_kv), in, st, L.bm_alt ? 1ull : 0ull, 1,
+                                   c->k_pool, c->v_pool, c->entries, c->bitmap, c->bitmap_alt, c->bitmap_words,
+                                   c->pool_pages, n, T, g.num_heads, g.head_dim, P, frame_idx, c->d_err,
+                                   static_cast<long long>(c->model_heads) * g.head_dim * c->elem_kv);
+    if (e != cudaSuccess) return cuda_fail(c, e, "append");
+    c->launches++;
+    L.bm_alt = !L.bm_alt;
+  } else {
+    e = launch_mgr_alloc(c->stream, E, layer_bitmap(c, layer), c->bitmap_words, c->pool_pages, L.n_entries, n,
+                         frame_idx, P, T - (n - 1) * P, c->d_err);
+    if (e != cudaSuccess) return cuda_fail(c, e, "page allocation");
+    c->launches++;
+  }
   if (g.kv_dtype == KVC_FP8_E4M3) {
     e = launch_append_fp8(c->stream, k_dev, v_dev, layer_pool(c, c->k_pool, layer), layer_pool(c, c->v_pool, layer),
                           layer_scale(c, c->k_scale, layer), layer_scale(c, c->v_scale, layer), E + L.n_entries, n, T,
                           g.num_heads, g.head_dim, P, layer_group_scales(c, c->k_chan, layer, g.head_dim),
                           layer_group_scales(c, c->v_tok, layer, P));
-  } else {
+    if (e != cudaSuccess) return cuda_fail(c, e, "append");
+    c->launches++;
+  } else if (!append_alloc_fusable(static_cast<int>(c->elem_kv), g.num_heads, g.head_dim, P)) {
     e = launch_append(c->stream, static_cast<int>(c->elem_kv), k_dev, v_dev, layer_pool(c, c->k_pool, layer),
                       layer_pool(c, c->v_pool, layer), E + L.n_entries, n, T, g.num_heads, g.head_dim, P, c->d_err);
+    if (e != cudaSuccess) return cuda_fail(c, e, "append");
+    c->launches++;
   }
-  if (e != cudaSuccess) return cuda_fail(c, e, "append");
-  c->launches++;
   if (g.budget_tokens > 0) {
     kvc_status st = init_token_meta(c, layer, L.n_entries, n, frame_idx);
     if (st != KVC_OK) return st;
@@ -625,13 +662,31 @@ kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const void* con
     LayerStarts st{};
     AppendBatch in{};
     st.first_layer = l0;
+    const size_t head_off = static_cast<size_t>(c->head0) * g.head_dim * c->elem_kv;
     for (int b = 0; b < nl; ++b) {
       st.start[b] = c->L[l0 + b].n_entries;
-      in.k[b] = k_devs[l0 + b];
-      in.v[b] = v_devs[l0 + b];
+      in.k[b] = static_cast<const uint8_t*>(k_devs[l0 + b]) + head_off;
+      in.v[b] = static_cast<const uint8_t*>(v_devs[l0 + b]) + head_off;
     }
-    cudaError_t e = launch_mgr_alloc_layers(c->stream, c->entries, c->bitmap, c->bitmap_words, c->pool_pages, st, nl,
-                                            n, frame_idx, P, T - (n - 1) * P, c->d_err);
+    cudaError_t e;
+    if (g.kv_dtype != KVC_FP8_E4M3 && append_alloc_fusable(static_cast<int>(c->elem_kv), g.num_heads, g.head_dim, P)) {
+      // allocation and copy of every layer of the batch in one launch
+      unsigned long long alt = 0;
+      for (int b = 0; b < nl; ++b)
+        if (c->L[l0 + b].bm_alt) alt |= 1ull << b;
+      e = launch_append_alloc_layers(c->stream, static_cast<int>(c->elem_kv), in, st, alt, nl, c->k_pool, c->v_pool,
+                                     c->entries, c->bitmap, c->bitmap_alt, c->bitmap_words, c->pool_pages, n, T,
+                                     g.num_heads, g.head_dim, P, frame_idx, c->d_err,
+                                     static_cast<long long>(c->model_heads) * g.head_dim * c->elem_kv);
+      if (e != cudaSuccess) return cuda_fail(c, e, "append (all layers)");
+      c->launches++;
+      for (int b = 0; b < nl; ++b) c->L[l0 + b].bm_alt = !c->L[l0 + b].bm_alt;
+      continue;
+    }
+    // FP8 storage or pages too large for the fused kernel: never on the fused path, so every
+    // layer is still on its first bitmap buffer
+    e = launch_mgr_alloc_layers(c->stream, c->entries, c->bitmap, c->bitmap_words, c->pool_pages, st, nl,
+                                n, frame_idx, P, T - (n - 1) * P, c->d_err);
     if (e != cudaSuccess) return cuda_fail(c, e, "page allocation (all layers)");
     c->launches++;
     if (g.kv_dtype == KVC_FP8_E4M3)
@@ -685,6 +740,8 @@ kvc_status attend_layer(kvc_cache* c, int layer, const void* q_dev, void* o_dev,
     a.tmap_k = &c->tmap_k[0];
     a.tmap_v = &c->tmap_v[0];
     a.fp8 = g.kv_dtype == KVC_FP8_E4M3;
+    a.q_heads = c->model_heads;
+    a.head0 = c->head0;
     a.k_scale = c->k_scale;
     a.v_scale = c->v_scale;
     a.k_chan = c->k_chan;
@@ -764,7 +821,7 @@ kvc_status kvc_scale_phase(kvc_cache* c, int32_t layer, int32_t n_frames, const 
   if (L.n_entries != 0 || L.has_pending || L.last_frame >= 0)
     return fail(c, KVC_ERR_STATE, "kvc_scale_phase: the joint phase starts an empty layer");
   // frames 0 .. n-1 appended and committed, then all n*T queries over all of them
-  const size_t frame_bytes = static_cast<size_t>(g.tokens_per_frame) * g.num_heads * g.head_dim * c->elem_io;
+  const size_t frame_bytes = static_cast<size_t>(g.tokens_per_frame) * c->model_heads * g.head_dim * c->elem_io;
   for (int f = 0; f < n_frames; ++f) {
     kvc_status st = kvc_append_frame(c, layer, f, static_cast<const uint8_t*>(k_dev) + f * frame_bytes,
                                      static_cast<const uint8_t*>(v_dev) + f * frame_bytes, 1);
@@ -931,6 +988,8 @@ kvc_status kvc_step_host_async(kvc_cache* c, int32_t layer, int32_t frame_idx, i
                                const void* q_host, const void* k_host, const void* v_host, void* o_host) {
   if (!c) return KVC_ERR_ARG;
   if (!q_host || !k_host || !v_host || !o_host) return fail(c, KVC_ERR_ARG, "kvc_step_host: NULL host buffer");
+  if (c->model_heads != c->cfg.num_heads)
+    return fail(c, KVC_ERR_ARG, "kvc_step_host: host-buffer steps take caches that hold every head");
   const kvc_config& g = c->cfg;
   const size_t bytes = static_cast<size_t>(g.tokens_per_frame) * g.num_heads * g.head_dim * c->elem_io;
   const int b = c->host_slot;
@@ -981,6 +1040,33 @@ kvc_status kvc_prune(kvc_cache* c, int32_t layer) {
   if (!valid_layer(c, layer)) return fail(c, KVC_ERR_ARG, "kvc_prune: bad layer");
   if (!c->L[layer].has_pending) return fail(c, KVC_ERR_STATE, "kvc_prune: no frame pending on this layer");
   return div_prune(c, layer);
+}
+
+kvc_status kvc_adapt_layer_budgets(kvc_cache* c, double tau, int32_t k_avg, int32_t* budgets_out) {
+  if (!c) return KVC_ERR_ARG;
+  if (!c->per_head) return fail(c, KVC_ERR_STATE, "kvc_adapt_layer_budgets: not a diversity-pruned cache");
+  if (k_avg < 1 || !(tau == tau)) return fail(c, KVC_ERR_ARG, "kvc_adapt_layer_budgets: k_avg must be >= 1");
+  const kvc_config& g = c->cfg;
+  std::vector<long long> cand(g.num_layers);
+  for (int l = 0; l < g.num_layers; ++l) {
+    cand[l] = c->L[l].cand_count;
+    if (cand[l] == 0) return fail(c, KVC_ERR_STATE, "kvc_adapt_layer_budgets: every layer must have been pruned");
+  }
+  kvc_status st = sync_and_check(c);
+  if (st != KVC_OK) return st;
+  cudaError_t e = cudaMemcpy(c->div_cand, cand.data(), cand.size() * sizeof(long long), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = launch_layer_budgets(c->stream, c->div_sums, c->div_cand, g.num_layers, g.num_heads, tau, k_avg,
+                             g.diversity_budget, c->div_budget);
+  if (e != cudaSuccess) return cuda_fail(c, e, "kvc_adapt_layer_budgets");
+  c->launches++;
+  std::vector<int32_t> b(g.num_layers);
+  e = cudaStreamSynchronize(c->stream);
+  if (e == cudaSuccess) e = cudaMemcpy(b.data(), c->div_budget, b.size() * sizeof(int32_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(c, e, "kvc_adapt_layer_budgets copy");
+  c->layer_budget = b;
+  if (budgets_out) std::copy(b.begin(), b.end(), budgets_out);
+  return KVC_OK;
 }
 
 kvc_status kvc_layer_diversity(kvc_cache* c, int32_t layer, double* mean_out) {

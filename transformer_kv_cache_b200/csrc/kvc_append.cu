@@ -112,6 +112,154 @@ __global__ void __launch_bounds__(256) append_bulk_kernel(AppendBatch in, LayerS
   }
 }
 
+// Allocation fused into the append: the same CTA per (layer of the batch, tensor, page g)
+// as append_bulk_kernel, which first finds its physical page itself, as the g-th free page
+// (lowest first) of the layer's current bitmap. The current bitmap is only read in this
+// kernel, so every CTA sees the same free set; the CTA of page 0 of K writes the next
+// bitmap (the current one with the frame's pages marked used) into the layer's other
+// bitmap buffer, each K CTA writes its page-table entry, and the host switches the layer to
+// the other buffer. No CTA waits on another. A pool without enough free pages latches
+// DERR_POOL and copies nothing.
+__device__ __forceinline__ uint32_t free_bits(const uint32_t* bm, int w, int words, int pool_pages) {
+  if (w >= words) return 0u;
+  uint32_t valid = 0xffffffffu;
+  const int nv = pool_pages - w * 32;
+  if (nv < 32) valid = nv <= 0 ? 0u : ((1u << nv) - 1u);
+  return ~bm[w] & valid;
+}
+
+__global__ void __launch_bounds__(256) append_alloc_bulk_kernel(AppendBatch in, LayerStarts starts,
+                                                                unsigned long long alt_mask, int n_layers,
+                                                                uint8_t* k_pool_all, uint8_t* v_pool_all,
+                                                                Entry* entries_all, uint32_t* bm_main,
+                                                                uint32_t* bm_alt, int words, int pool_pages,
+                                                                int n_pages, int T, int H, int row_bytes, int P,
+                                                                int owner, int* err, long long src_tok_bytes) {
+  griddep_wait();
+  griddep_launch_dependents();
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  __shared__ int s_phys;
+  __shared__ int s_warp[8];
+  const int page_bytes = P * H * row_bytes;
+  uint4* src_s = reinterpret_cast<uint4*>(sm);                 // [slot][head][chunk]
+  uint4* dst_s = reinterpret_cast<uint4*>(sm + page_bytes);    // [head][slot][chunk]
+  const int g = blockIdx.x % n_pages;
+  const int tensor = (blockIdx.x / n_pages) & 1;
+  const int bl = blockIdx.x / (2 * n_pages);
+  const int ntok = min(P, T - g * P);
+  const long long layer = starts.first_layer + bl;
+  const bool on_alt = (alt_mask >> bl) & 1ull;
+  const uint32_t* cur = (on_alt ? bm_alt : bm_main) + layer * words;
+  uint32_t* next = (on_alt ? bm_main : bm_alt) + layer * words;
+  // a token's H rows are contiguous in the source; tokens are src_tok_bytes apart (more than
+  // H rows when the cache holds a range of the caller's heads)
+  const int tok_bytes = H * row_bytes;
+  const uint8_t* src = static_cast<const uint8_t*>(tensor ? in.v[bl] : in.k[bl]) +
+                       static_cast<long long>(g) * P * src_tok_bytes;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    s_phys = -1;
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(ntok * tok_bytes));
+    if (src_tok_bytes == tok_bytes) {
+      bulk_load(src_s, src, static_cast<uint32_t>(ntok * tok_bytes), &bar);
+    } else {
+      for (int t = 0; t < ntok; ++t)
+        bulk_load(reinterpret_cast<uint8_t*>(src_s) + t * tok_bytes, src + t * src_tok_bytes,
+                  static_cast<uint32_t>(tok_bytes), &bar);
+    }
+  }
+  if (warp == 0) {
+    // the g-th free page: word popcounts scanned 32 words at a time
+    int found = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+      const uint32_t fb = free_bits(cur, w0 + lane, words, pool_pages);
+      const int cnt = __popc(fb);
+      int x = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      const int before = found + x - cnt;
+      const unsigned hit = __ballot_sync(0xffffffffu, g >= before && g < found + x);
+      if (hit) {
+        if (lane == __ffs(hit) - 1) s_phys = (w0 + lane) * 32 + static_cast<int>(__fns(fb, 0, g - before + 1));
+        break;
+      }
+      found += __shfl_sync(0xffffffffu, x, 31);
+    }
+  }
+  if (tensor == 0 && g == 0) {
+    // the next bitmap: the n_pages lowest free pages marked used
+    int found = 0;
+    for (int w0 = 0; w0 < words; w0 += 256) {
+      const int w = w0 + threadIdx.x;
+      const uint32_t fb = free_bits(cur, w, words, pool_pages);
+      const int cnt = __popc(fb);
+      int x = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) s_warp[warp] = x;
+      __syncthreads();
+      int wbase = 0, total = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        wbase += i < warp ? s_warp[i] : 0;
+        total += s_warp[i];
+      }
+      int r = found + wbase + x - cnt;
+      uint32_t m = fb, taken = 0;
+      while (m && r < n_pages) {
+        const uint32_t bit = m & (0u - m);
+        taken |= bit;
+        m ^= bit;
+        ++r;
+      }
+      if (w < words) next[w] = cur[w] | taken;
+      found += total;
+      __syncthreads();
+    }
+    if (threadIdx.x == 0 && found < n_pages) latch_error(err, DERR_POOL);
+  }
+  __syncthreads();
+  const int phys = s_phys;
+  if (phys < 0) {
+    // no free page: the copy is dropped (DERR_POOL latched above), the load drained
+    mbar_wait_drain(&bar, 0, err);
+    return;
+  }
+  if (tensor == 0 && threadIdx.x == 0) {
+    const int valid = g == n_pages - 1 ? T - (n_pages - 1) * P : P;
+    entries_all[layer * pool_pages + starts.start[bl] + g] = make_int4(phys, owner, g, valid);
+  }
+  uint8_t* dst = (tensor ? v_pool_all : k_pool_all) + (layer * pool_pages + phys) * static_cast<long long>(page_bytes);
+  if (!mbar_wait_bounded(&bar, 0, &abort_flag, err)) return;
+  const int chunks = row_bytes / 16;
+  for (int i = threadIdx.x; i < page_bytes / 16; i += blockDim.x) {
+    const int q = i % chunks;
+    const int rr = i / chunks;
+    const int slot = rr % P, h = rr / P;
+    dst_s[i] = slot < ntok ? src_s[(slot * H + h) * chunks + q] : make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_shared();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    bulk_store(dst, dst_s, static_cast<uint32_t>(page_bytes));
+    bulk_store_wait_all();
+  }
+}
+
 // Two fp32 values -> two E4M3 codes, round to nearest even, saturating to +-448.
 __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   uint16_t r;
@@ -262,13 +410,12 @@ cudaError_t launch_append_layers(cudaStream_t s, int elem_bytes, const AppendBat
   if (2 * page_bytes <= kBulkAppendMaxSmem) {
     // bulk copies through shared memory: the K/V tensors and pools are 16-byte aligned and
     // every transfer is a whole number of 16-byte rows
-    static int attr = 0;
-    if (2 * page_bytes > attr) {
-      cudaError_t e = cudaFuncSetAttribute(append_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           2 * page_bytes);
-      if (e != cudaSuccess) return e;
-      attr = 2 * page_bytes;
-    }
+    static PerDeviceOnce attr;
+    cudaError_t e = attr.run([] {
+      return cudaFuncSetAttribute(append_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kBulkAppendMaxSmem);
+    });
+    if (e != cudaSuccess) return e;
     return launch_pdl(append_bulk_kernel, dim3(2 * n_layers * n_pages), dim3(256), static_cast<size_t>(2 * page_bytes),
                       s, in, starts, n_layers, static_cast<uint8_t*>(k_pool_all), static_cast<uint8_t*>(v_pool_all),
                       entries_all, pool_pages, n_pages, T, H, D * elem_bytes, P, err);
@@ -293,6 +440,31 @@ cudaError_t launch_append_fp8_layers(cudaStream_t s, const AppendBatch& in, cons
   return launch_pdl(append_fp8_kernel, dim3((items + warps - 1) / warps), dim3(warps * 32), 0, s, in, starts,
                     n_layers, k_pool_all, v_pool_all, k_scale_all, v_scale_all, k_chan_all, v_tok_all, entries_all,
                     pool_pages, n_pages, T, H, D, P);
+}
+
+bool append_alloc_fusable(int elem_bytes, int H, int D, int P) {
+  return D * elem_bytes % 16 == 0 && 2 * P * H * D * elem_bytes <= kBulkAppendMaxSmem;
+}
+
+cudaError_t launch_append_alloc_layers(cudaStream_t s, int elem_bytes, const AppendBatch& in,
+                                       const LayerStarts& starts, unsigned long long alt_mask, int n_layers,
+                                       void* k_pool_all, void* v_pool_all, Entry* entries_all, uint32_t* bm_main,
+                                       uint32_t* bm_alt, int words, int pool_pages, int n_pages, int T, int H, int D,
+                                       int P, int owner, int* err, long long src_tok_bytes) {
+  if (!append_alloc_fusable(elem_bytes, H, D, P)) return cudaErrorInvalidValue;
+  if (src_tok_bytes == 0) src_tok_bytes = static_cast<long long>(H) * D * elem_bytes;
+  if (src_tok_bytes % 16) return cudaErrorInvalidValue;
+  static PerDeviceOnce attr;
+  cudaError_t e = attr.run([] {
+    return cudaFuncSetAttribute(append_alloc_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kBulkAppendMaxSmem);
+  });
+  if (e != cudaSuccess) return e;
+  const int page_bytes = P * H * D * elem_bytes;
+  return launch_pdl(append_alloc_bulk_kernel, dim3(2 * n_layers * n_pages), dim3(256),
+                    static_cast<size_t>(2 * page_bytes), s, in, starts, alt_mask, n_layers,
+                    static_cast<uint8_t*>(k_pool_all), static_cast<uint8_t*>(v_pool_all), entries_all, bm_main, bm_alt,
+                    words, pool_pages, n_pages, T, H, D * elem_bytes, P, owner, err, src_tok_bytes);
 }
 
 cudaError_t launch_append(cudaStream_t s, int elem_bytes, const void* k, const void* v, void* k_pool,

@@ -16,6 +16,8 @@ struct TcParams {
   const Entry* entries;
   int n_pages, T, H;
   int q_tiles, splits, tiles_per_split, total_tiles;
+  int q_pairs;                  // bf16 kernel: query-tile pairs (one per CTA of a group)
+  int out_heads, head0;         // bf16 kernel: heads of Q and O; the cache's head h is head0 + h
   long long page_base;          // layer * pool_pages: first pool page of the layer
   int pool_rows;                // rows of the pool tensor maps (a row index past the end reads zeros)
   float scale_log2;
@@ -24,7 +26,7 @@ struct TcParams {
   float* part_lse;
   int* err;
   int head_pages;               // > 0: per-head page lists (see TcAttnArgs)
-  int* split_cnt;               // [H][q_tiles] zeroed counters: the last split CTA merges (bf16 kernel)
+  int* split_cnt;               // [H][q_tiles][4] zeroed counters: the piece that counts last merges (bf16 kernel)
   const float* k_chan;          // dimension-adaptive FP8: [pool page][head][64] K channel scales
   const float* v_tok;           // dimension-adaptive FP8: [pool page][head][16] V token scales
 };
@@ -84,11 +86,6 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
-// Wait without the abort shortcut, used only to drain a CTA's own in-flight work.
-__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, int* err) {
-  volatile int never = 0;
-  mbar_wait_bounded(bar, parity, &never, err);
-}
 
 
 // FP8 E4M3 storage variant (kvc_attn_fp8.cu): same parameters, the query map of the bf16

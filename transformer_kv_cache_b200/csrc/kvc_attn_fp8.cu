@@ -26,9 +26,10 @@
 //                       logit factor of its 16 columns, so Q K^T runs on exact decoded codes.
 //
 // The epilogue multiplies by the V reference scale. Rounding V times s_page / s_ref to f16
-// is the only extra rounding of an operand (relative 2^-11). The query is held in f16,
-// which is exact for bf16 values of magnitude in [2^-14, 65504]. Every barrier wait is
-// bounded.
+// is the only extra rounding of an operand (relative 2^-11). The query row is held in f16
+// after an exact power-of-two scaling into f16's range (the row's logit factor carries the
+// inverse), so every finite bf16 query is taken. Slots past a page's valid count score
+// -inf in the tiles that have them, so they take no weight. Every barrier wait is bounded.
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
@@ -409,19 +410,40 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
       uint64_t* my_s_free = &s_free[g];
       uint64_t* my_p_full = &p_full[2 * g];
       uint64_t* my_pv_done = &pv_done[2 * g];
+      // this row of Q, bf16 -> f16, into TMEM: the A operand of S. The row is first scaled
+      // by a power of two 2^e that brings its largest magnitude into [2^14, 2^15), so no
+      // finite bf16 query overflows f16 and small rows keep their bits; the logit factor of
+      // the row carries 2^-e, which makes the scaling exact (e is clamped to [-120, 100] so
+      // that factor stays a normal fp32 number)
+      float row_fac = 1.f;
       {
-        // this row of Q, bf16 -> f16 (exact in range), into TMEM: the A operand of S
         uint32_t qv[32];
         const int row = qt * kBM + r;
         if (row < p.T) {
           const uint4* src = reinterpret_cast<const uint4*>(p.q + (static_cast<long long>(row) * p.H + h) * kHD);
+          uint4 w[8];
+          float qmax = 0.f;
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
-            const uint4 w = __ldg(src + v);
-            qv[4 * v] = pack_f16(bf16lo(w.x), bf16hi(w.x));
-            qv[4 * v + 1] = pack_f16(bf16lo(w.y), bf16hi(w.y));
-            qv[4 * v + 2] = pack_f16(bf16lo(w.z), bf16hi(w.z));
-            qv[4 * v + 3] = pack_f16(bf16lo(w.w), bf16hi(w.w));
+            w[v] = __ldg(src + v);
+            qmax = max3(qmax, fabsf(bf16lo(w[v].x)), fabsf(bf16hi(w[v].x)));
+            qmax = max3(qmax, fabsf(bf16lo(w[v].y)), fabsf(bf16hi(w[v].y)));
+            qmax = max3(qmax, fabsf(bf16lo(w[v].z)), fabsf(bf16hi(w[v].z)));
+            qmax = max3(qmax, fabsf(bf16lo(w[v].w)), fabsf(bf16hi(w[v].w)));
+          }
+          int e = 0;
+          if (qmax > 0.f) {
+            int ex;
+            frexpf(qmax, &ex);                            // qmax in [2^(ex-1), 2^ex)
+            e = min(100, max(-120, 15 - ex));
+          }
+          row_fac = ldexpf(1.f, -e);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            qv[4 * v] = pack_f16(ldexpf(bf16lo(w[v].x), e), ldexpf(bf16hi(w[v].x), e));
+            qv[4 * v + 1] = pack_f16(ldexpf(bf16lo(w[v].y), e), ldexpf(bf16hi(w[v].y), e));
+            qv[4 * v + 2] = pack_f16(ldexpf(bf16lo(w[v].z), e), ldexpf(bf16hi(w[v].z), e));
+            qv[4 * v + 3] = pack_f16(ldexpf(bf16lo(w[v].w), e), ldexpf(bf16hi(w[v].w), e));
           }
         } else {
 #pragma unroll
@@ -435,7 +457,7 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
       }
       bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(ref_ready, 0, abort_flag, p.err));
       const float vref = ok ? *sref : 1.f;
-      float m = -INFINITY, masked = 0.f;
+      float m = -INFINITY;
       // Lanes 0..3 hold page g = lane of the current tile (K scale, valid slots) and the
       // entry of the next tile, loaded one tile ahead; every lane reads them by shuffle.
       // Pages past the list have scale 0 and no valid slots.
@@ -458,10 +480,20 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
       for (int j = 0; ok && j < n_tiles; ++j) {
         int n_masked = 0;
         float cg[kPPT];            // logit factor per page: log2(e) x softmax scale x K scale
+        int vpg[kPPT];             // valid slots per page
 #pragma unroll
         for (int pg = 0; pg < kPPT; ++pg) {
-          n_masked += P - __shfl_sync(0xffffffffu, vj, pg);
-          cg[pg] = p.scale_log2 * __shfl_sync(0xffffffffu, ksj, pg);
+          vpg[pg] = __shfl_sync(0xffffffffu, vj, pg);
+          n_masked += P - vpg[pg];
+          // a zero-scale page (all-zero K, or past the list) gets a tiny positive factor: its
+          // valid scores are 0 either way, and its masked -inf scores stay -inf
+          cg[pg] = fmaxf((p.scale_log2 * row_fac) * __shfl_sync(0xffffffffu, ksj, pg), 1e-30f);
+        }
+        if (n_masked) {
+          // slots past a page's valid count (and pages past the list end) take no weight
+#pragma unroll
+          for (int cc = 0; cc < kBN; ++cc)
+            if ((cc % P) >= vpg[cc / P]) s[cc / 32][cc % 32] = __float_as_uint(-INFINITY);
         }
         if (j + 1 < n_tiles) {
           ksj = page_scale(p, p.k_scale, en.x, h);
@@ -500,7 +532,7 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
             }
             mt = fmaxf(mt, fmaxf(ta, tb) * cg[pg]);
           }
-          const float m_new = move ? mt : m;
+          const float m_new = move ? (mt == -INFINITY ? (m == -INFINITY ? 0.f : m) : mt) : m;
           const bool resc = move && j > 0;
           if (__any_sync(0xffffffffu, resc)) {
             if (!__all_sync(0xffffffffu, mbar_wait_bounded(&my_pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag,
@@ -510,7 +542,6 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
             }
             tc_fence_after();
             const float f = resc ? ex2(m - m_new) : 1.0f;
-            masked *= f;
 #pragma unroll
             for (int q4 = 0; q4 < kON / 16; ++q4) {
               uint32_t oc[16];
@@ -535,8 +566,6 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
             }
           }
         }
-        // a masked slot holds zero codes: its score is 0 and its P entry is f16(2^-m)
-        if (n_masked) masked += static_cast<float>(n_masked) * f16lo(pack_f16(ex2(-m), 0.f));
         if (j >= 2) {
           if (!__all_sync(0xffffffffu, mbar_wait_bounded(&my_pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag,
                                                           p.err))) {
@@ -575,7 +604,7 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
         tmem_ld32(tO + 32, o1);
         tmem_ld16(tO + 64, ls);
         tmem_ld_wait();
-        const float l = __uint_as_float(ls[0]) - masked;
+        const float l = __uint_as_float(ls[0]);
         const float inv = vref / l;
         const int row = qt * kBM + r;
         if (p.splits == 1) {
@@ -617,16 +646,16 @@ __global__ void __launch_bounds__(tc8::kThreads, 1)
 
 cudaError_t launch_attn_fp8_kernel(cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                    const TcParams& prm, int grid) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fp8_kernel<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  static PerDeviceOnce attr;
+  cudaError_t e = attr.run([] {
+    cudaError_t r = cudaFuncSetAttribute(attn_fp8_kernel<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(tc8::kSmemBytes));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn_fp8_kernel<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(attn_fp8_kernel<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(tc8::kSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+    return r;
+  });
+  if (e != cudaSuccess) return e;
   if (prm.k_chan)
     return launch_pdl(attn_fp8_kernel<16, true>, dim3(grid), dim3(tc8::kThreads), tc8::kSmemBytes, s, tq, tk, tv, prm);
   return launch_pdl(attn_fp8_kernel<16, false>, dim3(grid), dim3(tc8::kThreads), tc8::kSmemBytes, s, tq, tk, tv, prm);

@@ -3,171 +3,273 @@
 // Computes O[i, h] = sum_j softmax_j(scale * q_i . k_j) v_j for the T queries of the new
 // frame over every valid slot of the layer's page list ("How GCTStream ...",
 // Frame-by-Frame Causal Processing; "InfiniteVGGT" explainer, Causal Attention) without
-// materialising the score matrix, as a flash-attention pipeline built for Blackwell. Each
-// CTA owns one 128-row query tile of one head and a range of 64-slot KV tiles (4 pages):
+// materialising the score matrix, as a flash-attention pipeline built for Blackwell.
 //
-//   warp 0 (one lane)   TMA producer: per KV tile the 4 pages of K and of V, each
-//                       page-head block one 2-D box, into a ring of 128-byte-swizzled
-//                       stages. Pages past the end of the list are read past the end of the
-//                       pool, which TMA fills with zeros.
-//   warp 1              MMA issuer (the warp waits, one elected lane issues): S = Q K^T
-//                       (tcgen05.mma kind::f16, M=128, N=64, A = Q read from TMEM) into
-//                       TMEM, then O' += P [V | 1] (M=128, N=80, A = P read from TMEM,
-//                       B = the V tile as an MN-major operand followed by a constant block
-//                       of ones), so accumulator column 64 carries the row sum of P.
-//   warps 2..5          softmax, thread = query row = TMEM lane. First each thread stores
-//                       its row of Q into TMEM (so S reads only K from shared memory);
-//                       then per KV tile, 64 columns:
-//                       x = s*c - m with packed f32x2 FMAs, P = 2^x on the MUFU, its upper
-//                       halves taken as the bf16 pairs the MMA consumes (one byte permute
-//                       per pair) and written back to TMEM (tcgen05.st); no per-element sum
-//                       (the MMA makes it from the same bf16 P). The next tile's S is
-//                       loaded from TMEM while this tile's P store is in flight.
+// Work decomposition. A unit is one head and one pair of 128-row query tiles (256 query
+// rows). The KV sequence of a head is cut into 128-slot tiles (8 pages). The launch is
+// persistent: CTAs form groups of q_pairs CTAs (one per query-tile pair), and group g sweeps
+// the contiguous range [g*R, (g+1)*R) of the flattened (head, KV tile) sequence, so every
+// CTA of a group reads the same K/V tiles at about the same time and the group's other
+// CTAs find them in L2. A range may end inside a head and the next group continue it: the
+// pieces of a unit are merged by the piece that finishes last (partial outputs carry their
+// log2-sum-exp), so no separate combine launch is needed.
+//
+// Roles of a CTA (384 threads, one CTA per SM, all 512 TMEM columns; warpgroup 0 gives up
+// registers to the two softmax warpgroups with setmaxnreg):
+//   warp 0 (one lane)   TMA producer: the pair's two query tiles (128-byte swizzled, the
+//                       A operand of S) once per piece, then per KV tile the 8 page-head
+//                       blocks of K and of V into a 4-stage ring. Pages past the end of the
+//                       list are read past the end of the pool, which TMA fills with zeros.
+//   warp 1              MMA issuer (the warp waits, one elected lane issues):
+//                       S_i = Q_i K^T (tcgen05.mma kind::f16, M=128, N=128, both operands
+//                       in shared memory) into TMEM, and O'_i += P_i [V | 1] (M=128, N=80,
+//                       A = P_i read from TMEM, B = the V tile as an MN-major operand
+//                       followed by a constant block of ones), so accumulator column 64
+//                       carries the exact row sum of the same bf16 P the product used.
+//   warps 4-7, 8-11     softmax of query tile 0 and 1 (thread = query row = TMEM lane).
+//                       Per KV tile: the 128 scores from TMEM, P = 2^(s*c - m) for 96
+//                       columns on the MUFU and for 32 on the FMA pipe (a cubic in the
+//                       fraction, the integer part added to the exponent field), truncated
+//                       to bf16 pairs and written back over the first 64 columns of S.
+//
+// P overwrites S, so S_i of the next tile is issued after the P.V product of this one; the
+// two query tiles alternate (while one tile's softmax runs, the tensor core does the other
+// tile's P.V and next S), which keeps the MUFU and the tensor core busy together.
 //
 // Online softmax with lazy rescaling: the reference max m of a row only moves when a
-// tile's P would exceed 2^8; the common case costs a bf16x2 max over the packed P and no
-// fp32 max at all. When a row's reference moves (the first tile, or a
-// new maximum), the exact fp32 tile max is taken and O' (including the row-sum column) is
-// rescaled in TMEM. The result is exact up to rounding after the final division by the
-// row sum.
+// tile's P would exceed 2^8 (the exact fp32 tile max, from 3-input max instructions, is
+// compared with m + 8). When a row's reference moves (the first tile of a piece, or a new
+// maximum), O' (with its row-sum column) is rescaled in TMEM; the P.V product of the
+// previous tile has completed by then because it was issued before this tile's S.
 //
-// Partial pages need no per-column mask: slots past a page's valid count hold K = V = 0
-// (the append and compaction kernels write zeros there), so each scores exactly 0, adds
-// nothing to O and 2^-m to the row sum; that amount is tracked per row and taken out.
+// Partial pages: slots past a page's valid count hold K = V = 0 (the append and compaction
+// kernels write zeros there) and their scores are set to -inf before the softmax, in the
+// tiles that have such slots; pages past the end of the list are masked the same way.
 //
-// P is double-buffered in TMEM so a tile's softmax never waits for the previous tile's
-// P.V product. TMEM (256 columns): S [0,64), P0 [64,96), P1 [96,128), O' [128,208),
-// Q [208,240). Two CTAs fit per SM. The KV sequence can be split across CTAs; partial outputs carry the
-// log2-sum-exp, and the split CTA of a query tile that finishes last merges them (a
-// separate combine kernel does it where no split counters are given). Every barrier wait is bounded: on
-// timeout the CTA records KVC_ERR_TIMEOUT in the error word, drains its own copies and
-// MMAs, frees TMEM and returns.
+// Every barrier wait is bounded: on timeout the CTA records KVC_ERR_TIMEOUT in the error
+// word, drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
 
 #include "kvc_attn_common.cuh"
 
 namespace kvc {
 namespace tc {
-constexpr int kBM = 128;                      // query rows per CTA
-constexpr int kBN = 64;                       // KV slots per tile
+constexpr int kBM = 128;                      // query rows per query tile
+constexpr int kQT = 2;                        // query tiles per CTA
+constexpr int kBN = 128;                      // KV slots per tile
 constexpr int kHD = 64;                       // head dim (one 128-byte swizzle row)
 constexpr int kON = kHD + 16;                 // O' columns: O plus the row-sum block
 constexpr int kStages = 4;
-constexpr int kTileBytes = kBN * kHD * 2;     // 8 KB (K or V tile)
-constexpr int kOnesBytes = kBN * kHD * 2;     // 8 KB block of bf16 ones
-constexpr int kThreads = 192;
-constexpr int kTmemCols = 256;
-constexpr int kColS = 0, kColP = 64, kColO = 128, kColQ = 208;   // Q: 32 columns of bf16 pairs
-constexpr float kPMax = 256.0f;               // a P above 2^8 moves the row's reference max
-constexpr size_t kSmemBytes = 1024 + 2 * kStages * kTileBytes + kOnesBytes + 256;
+constexpr int kTileBytes = kBN * kHD * 2;     // 16 KB (K or V tile)
+constexpr int kQBytes = kBM * kHD * 2;        // 16 KB per query tile
+constexpr int kOnesBytes = kBN * kHD * 2;     // 16 KB block of bf16 ones
+constexpr int kThreads = 384;                 // 3 warpgroups
+constexpr int kRegsLow = 48, kRegsHigh = 224;  // after the split: 128 x 48 + 256 x 224 <= 384 x 168
+constexpr int kTmemCols = 512;
+constexpr int kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 336;
+constexpr int kPolyCols = 32;                 // columns of a tile whose 2^x runs on the FMA pipe
+constexpr float kLog2PMax = 8.0f;             // a P above 2^8 moves the row's reference max
+constexpr size_t kSmemBytes = 1024 + kQT * kQBytes + 2 * kStages * kTileBytes + kOnesBytes + 512;
 }  // namespace tc
 
-// Barrier over the softmax warps only (named barrier 1; barrier 0 is __syncthreads).
-__device__ __forceinline__ void softmax_warps_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// ---- the FMA-pipe exponential
+// 2^x for a pair: x clamped to [-126, 127], x = n + f with n = rint(x) (the 1.5 * 2^23 shift)
+// and f in [-0.5, 0.5]; 2^f = 1 + f (c1 + f (c2 + f c3)), a cubic fitted for this kernel by
+// iteratively reweighted least squares on the relative error (at most 1.02e-4, against the
+// 2^-8 of the bf16 truncation P takes next); 2^n is added to the exponent field.
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ void exp2_fma_pair(float x0, float x1, float& y0, float& y1) {
+  constexpr float kShift = 12582912.0f;       // 1.5 * 2^23
+  const uint64_t xc = pk2(fminf(fmaxf(x0, -126.f), 127.f), fminf(fmaxf(x1, -126.f), 127.f));
+  const uint64_t t = add2(xc, pk2(kShift, kShift));
+  const uint64_t fr = sub2(xc, sub2(t, pk2(kShift, kShift)));
+  uint64_t q = fma2(pk2(0.05500858277082443f, 0.05500858277082443f), fr,
+                    pk2(0.24221037328243256f, 0.24221037328243256f));
+  q = fma2(q, fr, pk2(0.6932829022407532f, 0.6932829022407532f));
+  q = fma2(q, fr, pk2(1.0f, 1.0f));
+  float q0, q1, t0, t1;
+  up2(q, q0, q1);
+  up2(t, t0, t1);
+  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
 
-// Merge one query row's split partials: O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M)
-// (M the largest lse), splits in ascending order. Partials were written by other CTAs of
-// this launch and are read through L2: half rows (32 dims) of up to four splits at a time
-// are copied (cp.async, every row's copies in flight together) into `stage`, the CTA's
-// K/V stage buffers, dead once the last P.V product has completed; with two splits both
-// halves come in one round. Each thread reads only its own row, whose eight 16-byte
-// chunks per half sit XOR-swizzled by the row so that neighbouring rows use other banks.
-__device__ __forceinline__ void merge_split_row(const TcParams& p, uint8_t* stage, int h, int qt, int r, int row) {
-  constexpr int kHalf = tc::kHD / 2;                  // dims per pass
-  constexpr int kSlot = tc::kBM * kHalf * 4;          // 16 KB: one split's half rows
-  constexpr int kSlots = 4;                           // the 64 KB of K/V stages
-  constexpr int kKeep = 8;                            // lse values kept in registers
-  const long long pi0 = static_cast<long long>(h) * p.splits * p.q_tiles + qt;
-  auto lse_at = [&](int s) { return __ldcg(p.part_lse + (pi0 + static_cast<long long>(s) * p.q_tiles) * tc::kBM + r); };
-  auto part_at = [&](int s, int half) {
-    return p.part_o + ((pi0 + static_cast<long long>(s) * p.q_tiles) * tc::kBM + r) * tc::kHD + half * kHalf;
-  };
-  // copy a half row into slot j / read chunk c of slot j
-  auto stage_in = [&](int j, const float* src) {
-    uint8_t* dst = stage + j * kSlot + r * kHalf * 4;
+// One tile of P for a row: pb[i] = bf16 pair of 2^(s*c - m) for columns 2i, 2i+1 (the last
+// kPolyCols columns on the FMA pipe, the others on the MUFU). Written in three stages over
+// the score registers (exponents in place, then every 2^x, then the packing) so that all
+// of a row's MUFU instructions are independent and can issue back to back.
+__device__ __forceinline__ void tile_p(uint32_t (&s)[tc::kBN], float c, float m, uint32_t (&pb)[tc::kBN / 2]) {
+  const uint64_t c2 = pk2(c, c), nm2 = pk2(-m, -m);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) cp_async16(dst + ((c ^ (r & 7)) << 4), src + 4 * c);
-  };
-  auto accumulate = [&](float (&a)[kHalf], int j, float w) {
-    const uint8_t* rowp = stage + j * kSlot + r * kHalf * 4;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const float4 f = *reinterpret_cast<const float4*>(rowp + ((c ^ (r & 7)) << 4));
-      a[4 * c + 0] = fmaf(w, f.x, a[4 * c + 0]);
-      a[4 * c + 1] = fmaf(w, f.y, a[4 * c + 1]);
-      a[4 * c + 2] = fmaf(w, f.z, a[4 * c + 2]);
-      a[4 * c + 3] = fmaf(w, f.w, a[4 * c + 3]);
-    }
-  };
-  uint4* out = reinterpret_cast<uint4*>(p.out + (static_cast<long long>(row) * p.H + h) * tc::kHD);
-  auto store_half = [&](const float (&a)[kHalf], int half, float inv) {
-#pragma unroll
-    for (int v = 0; v < kHalf / 8; ++v) {
-      uint4 q;
-      q.x = pack_bf16(a[8 * v + 0] * inv, a[8 * v + 1] * inv);
-      q.y = pack_bf16(a[8 * v + 2] * inv, a[8 * v + 3] * inv);
-      q.z = pack_bf16(a[8 * v + 4] * inv, a[8 * v + 5] * inv);
-      q.w = pack_bf16(a[8 * v + 6] * inv, a[8 * v + 7] * inv);
-      out[half * (kHalf / 8) + v] = q;
-    }
-  };
-  const bool one_round = p.splits <= kSlots / 2;
-  if (one_round)                                      // both halves of every split, issued first
-    for (int s = 0; s < p.splits; ++s) {
-      stage_in(2 * s, part_at(s, 0));
-      stage_in(2 * s + 1, part_at(s, 1));
-    }
-  float lr[kKeep];
-  float M = -INFINITY;
-#pragma unroll
-  for (int k = 0; k < kKeep; ++k) {
-    lr[k] = k < p.splits ? lse_at(k) : -INFINITY;
-    M = fmaxf(M, lr[k]);
+  for (int i = 0; i < tc::kBN / 2; ++i) {
+    float x0, x1;
+    up2(fma2_pair(s[2 * i], s[2 * i + 1], c2, nm2), x0, x1);
+    s[2 * i] = __float_as_uint(x0);
+    s[2 * i + 1] = __float_as_uint(x1);
   }
-  for (int s = kKeep; s < p.splits; ++s) M = fmaxf(M, lse_at(s));
-  float ws = 0.f;
 #pragma unroll
-  for (int k = 0; k < kKeep; ++k)
-    if (k < p.splits) ws += exp2f(lr[k] - M);
-  for (int s = kKeep; s < p.splits; ++s) ws += exp2f(lse_at(s) - M);
-  const float inv = 1.f / ws;
-  auto weight = [&](int s) {
-    float l = 0.f;
+  for (int i = 0; i < tc::kBN / 2; ++i) {
+    float y0, y1;
+    if (2 * i >= tc::kBN - tc::kPolyCols) {
+      exp2_fma_pair(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]), y0, y1);
+    } else {
+      y0 = ex2(__uint_as_float(s[2 * i]));
+      y1 = ex2(__uint_as_float(s[2 * i + 1]));
+    }
+    s[2 * i] = __float_as_uint(y0);
+    s[2 * i + 1] = __float_as_uint(y1);
+  }
 #pragma unroll
-    for (int k = 0; k < kKeep; ++k)
-      if (k == s) l = lr[k];
-    return exp2f((s < kKeep ? l : lse_at(s)) - M);
-  };
-  if (one_round) {
-    cp_async_wait_all();
-#pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
-      float a[kHalf];
+  for (int i = 0; i < tc::kBN / 2; ++i) pb[i] = bf16x2_trunc(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]));
+}
+
+// Register split between warpgroups (every warp of a warpgroup executes the same one).
+template <int N>
+__device__ __forceinline__ void reg_dealloc() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void reg_alloc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+
+// The schedule of one CTA: group g sweeps [g*R, min((g+1)*R, H*n_tiles)) of the flattened
+// (head, KV tile) sequence for query-tile pair qp. next_piece() cuts the range at head
+// boundaries.
+struct Sweep {
+  int pos, end;
+};
+__device__ __forceinline__ bool next_piece(Sweep& sw, int n_tiles, int& h, int& t0, int& t1) {
+  if (sw.pos >= sw.end) return false;
+  h = sw.pos / n_tiles;
+  t0 = sw.pos - h * n_tiles;
+  t1 = min(n_tiles, t0 + (sw.end - sw.pos));
+  sw.pos += t1 - t0;
+  return true;
+}
+
+// Epilogue of one warp's 32 query rows of a piece. Single-piece units store bf16 O
+// directly; otherwise every piece stores its normalised partial and log2-sum-exp, counts
+// itself on the warp's counter, and the piece that counts last merges:
+// O = sum_k 2^(lse_k - M) O_k / sum_k 2^(lse_k - M), M the largest lse, over the unit's
+// pieces in order (its own from registers, the others through L2). Only warp-level
+// synchronisation is used, so a warp that gave up on a wait cannot hold another here.
+__device__ __forceinline__ void store_piece(const TcParams& p, int wg, int wq, int lane, int h, int qp, int g,
+                                            const uint32_t (&o0)[32], const uint32_t (&o1)[32], float l, float m) {
+  using namespace tc;
+  const int r = wq * 32 + lane;
+  const int qtile = 2 * qp + wg;
+  const int row = qtile * kBM + r;
+  const float inv = 1.f / l;
+  const int n_tiles = p.total_tiles, R = p.tiles_per_split;
+  const int g_first = (h * n_tiles) / R;
+  const int g_last = (h * n_tiles + n_tiles - 1) / R;
+  const int npieces = g_last - g_first + 1;
+  uint4* out = reinterpret_cast<uint4*>(p.out + (static_cast<long long>(row) * p.out_heads + p.head0 + h) * kHD);
+  if (npieces == 1) {
+    if (row < p.T) {
 #pragma unroll
-      for (int k = 0; k < kHalf; ++k) a[k] = 0.f;
-      for (int s = 0; s < p.splits; ++s) accumulate(a, 2 * s + half, weight(s));
-      store_half(a, half, inv);
+      for (int v = 0; v < 8; ++v) {
+        const uint32_t* src = v < 4 ? &o0[8 * v] : &o1[8 * (v - 4)];
+        uint4 w;
+        w.x = pack_bf16(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv);
+        w.y = pack_bf16(__uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv);
+        w.z = pack_bf16(__uint_as_float(src[4]) * inv, __uint_as_float(src[5]) * inv);
+        w.w = pack_bf16(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv);
+        out[v] = w;
+      }
     }
     return;
   }
-#pragma unroll 1
-  for (int half = 0; half < 2; ++half) {
-    float a[kHalf];
+  if (qtile >= p.q_tiles) return;           // the pair's second tile is past the queries
+  const int unit = h * p.q_pairs + qp;
+  auto slot_row = [&](int k) { return (static_cast<long long>(unit) * p.splits + k) * (kQT * kBM) + wg * kBM + r; };
+  const int me = g - g_first;
+  const float lse_me = m + __log2f(l);
+  {
+    float4* dst = reinterpret_cast<float4*>(p.part_o + slot_row(me) * kHD);
 #pragma unroll
-    for (int k = 0; k < kHalf; ++k) a[k] = 0.f;
-    for (int s0 = 0; s0 < p.splits; s0 += kSlots) {
-      const int ns = min(kSlots, p.splits - s0);
-      for (int j = 0; j < ns; ++j) stage_in(j, part_at(s0 + j, half));
-      cp_async_wait_all();
-      for (int j = 0; j < ns; ++j) accumulate(a, j, weight(s0 + j));
-    }
-    store_half(a, half, inv);
+    for (int v = 0; v < 8; ++v)
+      dst[v] = make_float4(__uint_as_float(o0[4 * v + 0]) * inv, __uint_as_float(o0[4 * v + 1]) * inv,
+                           __uint_as_float(o0[4 * v + 2]) * inv, __uint_as_float(o0[4 * v + 3]) * inv);
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+      dst[8 + v] = make_float4(__uint_as_float(o1[4 * v + 0]) * inv, __uint_as_float(o1[4 * v + 1]) * inv,
+                               __uint_as_float(o1[4 * v + 2]) * inv, __uint_as_float(o1[4 * v + 3]) * inv);
+    p.part_lse[slot_row(me)] = lse_me;
   }
+  // threadfence-then-count: each partial is visible before its count
+  __threadfence();
+  __syncwarp();
+  const int cidx = ((h * p.q_tiles + qtile) << 2) + wq;
+  int last = 0;
+  if (lane == 0) last = atomicAdd(&p.split_cnt[cidx], 1) == npieces - 1;
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  __threadfence();
+  if (row < p.T) {
+    // pieces in ascending order whichever piece merges, so the result does not depend on
+    // which finished last (its own partial enters at its place, with the values it stored)
+    float M = lse_me;
+    for (int k = 0; k < npieces; ++k)
+      if (k != me) M = fmaxf(M, __ldcg(p.part_lse + slot_row(k)));
+    float acc[kHD];
+#pragma unroll
+    for (int d = 0; d < kHD; ++d) acc[d] = 0.f;
+    float ws = 0.f;
+    for (int k = 0; k < npieces; ++k) {
+      if (k == me) {
+        const float w = exp2f(lse_me - M);
+        ws += w;
+#pragma unroll
+        for (int d = 0; d < 32; ++d) {
+          acc[d] = fmaf(w, __uint_as_float(o0[d]) * inv, acc[d]);
+          acc[32 + d] = fmaf(w, __uint_as_float(o1[d]) * inv, acc[32 + d]);
+        }
+        continue;
+      }
+      const float w = exp2f(__ldcg(p.part_lse + slot_row(k)) - M);
+      ws += w;
+      const float4* src = reinterpret_cast<const float4*>(p.part_o + slot_row(k) * kHD);
+#pragma unroll
+      for (int v = 0; v < 16; ++v) {
+        const float4 f = __ldcg(src + v);
+        acc[4 * v + 0] = fmaf(w, f.x, acc[4 * v + 0]);
+        acc[4 * v + 1] = fmaf(w, f.y, acc[4 * v + 1]);
+        acc[4 * v + 2] = fmaf(w, f.z, acc[4 * v + 2]);
+        acc[4 * v + 3] = fmaf(w, f.w, acc[4 * v + 3]);
+      }
+    }
+    const float iw = 1.f / ws;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      uint4 w;
+      w.x = pack_bf16(acc[8 * v + 0] * iw, acc[8 * v + 1] * iw);
+      w.y = pack_bf16(acc[8 * v + 2] * iw, acc[8 * v + 3] * iw);
+      w.z = pack_bf16(acc[8 * v + 4] * iw, acc[8 * v + 5] * iw);
+      w.w = pack_bf16(acc[8 * v + 6] * iw, acc[8 * v + 7] * iw);
+      out[v] = w;
+    }
+  }
+  if (lane == 0) p.split_cnt[cidx] = 0;   // ready for the next launch
 }
 
 template <int P, bool kPerHead>
-__global__ void __launch_bounds__(tc::kThreads, 2)
+__global__ void __launch_bounds__(tc::kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const TcParams p) {
   griddep_wait();
@@ -176,48 +278,46 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
   constexpr int kPPT = kBN / P;               // pages per KV tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* k_s = smem;
+  uint8_t* q_s = smem;                                   // [2][128 rows][128 B]
+  uint8_t* k_s = q_s + kQT * kQBytes;
   uint8_t* v_s = k_s + kStages * kTileBytes;
   uint8_t* ones_s = v_s + kStages * kTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ones_s + kOnesBytes);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;
   uint64_t* v_full = k_full + kStages;
   uint64_t* kv_empty = v_full + kStages;
-  uint64_t* s_full = kv_empty + kStages;
-  uint64_t* s_free = s_full + 1;
-  uint64_t* p_full = s_full + 2;              // [2] one per P buffer
-  uint64_t* pv_done = s_full + 4;             // [2] one per P buffer
-  uint64_t* mma_final = s_full + 6;
+  uint64_t* s_full = kv_empty + kStages;      // [2] one per query tile
+  uint64_t* p_full = s_full + 2;              // [2]
+  uint64_t* o_full = p_full + 2;
+  uint64_t* o_free = o_full + 1;
+  uint64_t* mma_final = o_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x % p.q_tiles;
-  const int rest = blockIdx.x / p.q_tiles;
-  const int split = rest % p.splits;
-  const int h = rest / p.splits;
-  const int tile0 = split * p.tiles_per_split;
-  const int tile1 = min(tile0 + p.tiles_per_split, p.total_tiles);
-  const int n_tiles = tile1 - tile0;
-  // page list and pool rows of this head: shared pages [page][head][slot] or, with
-  // per-head page lists, single-head pages of head h's pool region
-  const long long hp = kPerHead ? static_cast<long long>(h) * p.head_pages : 0;
-  const Entry* ent = kPerHead ? p.entries + hp : p.entries;
+  const int qp = blockIdx.x % p.q_pairs;
+  const int g = blockIdx.x / p.q_pairs;
+  const int n_tiles = p.total_tiles;
+  const int HT = p.H * n_tiles;
+  const int R = p.tiles_per_split;
+  const Sweep sweep0{min(g * R, HT), min(g * R + R, HT)};
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 4);                       // the four softmax warps stored Q in TMEM
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 4);
-    mbar_init(&p_full[0], 4);
-    mbar_init(&p_full[1], 4);
-    mbar_init(&pv_done[0], 1);
-    mbar_init(&pv_done[1], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
+    }
+    mbar_init(o_full, 1);
+    mbar_init(o_free, 8);
     mbar_init(mma_final, 1);
     *abort_flag = 0;
     mbar_fence_init();
@@ -235,212 +335,229 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (n_tiles > 0) {
-    if (warp == 0) {
-      if (lane == 0) {
-        // ---------------------------------------------------------------- TMA producer
-        tma_prefetch_desc(&tmap_k);
-        tma_prefetch_desc(&tmap_v);
-        int last[kStages];
+  if (warp == 0) {
+    reg_dealloc<kRegsLow>();
+    if (lane == 0) {
+      // ------------------------------------------------------------------ TMA producer
+      tma_prefetch_desc(&tmap_q);
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_v);
+      int last[kStages];
 #pragma unroll
-        for (int i = 0; i < kStages; ++i) last[i] = -1;
-        for (int j = 0; j < n_tiles; ++j) {
-          const int st = j % kStages;
-          if (j >= kStages && !mbar_wait_bounded(&kv_empty[st], ((j / kStages) - 1) & 1, abort_flag, p.err)) break;
-          const int gt = tile0 + j;
+      for (int i = 0; i < kStages; ++i) last[i] = -1;
+      int jg = 0, pc = 0;
+      bool ok = true;
+      Sweep sw = sweep0;
+      int h, t0, t1;
+      while (ok && next_piece(sw, n_tiles, h, t0, t1)) {
+        if (pc > 0 && !mbar_wait_bounded(q_empty, (pc - 1) & 1, abort_flag, p.err)) break;
+        mbar_arrive_expect_tx(q_full, kQT * kQBytes);
+#pragma unroll
+        for (int i = 0; i < kQT; ++i)
+          tma_load_3d(q_s + i * kQBytes, &tmap_q, q_full, 0, p.head0 + h, (2 * qp + i) * kBM);
+        const long long hp = kPerHead ? static_cast<long long>(h) * p.head_pages : 0;
+        const Entry* ent = kPerHead ? p.entries + hp : p.entries;
+        int phys_next[kPPT];
+#pragma unroll
+        for (int q = 0; q < kPPT; ++q) {
+          const int idx = t0 * kPPT + q;
+          phys_next[q] = idx < p.n_pages ? __ldg(&ent[idx].x) : -1;
+        }
+        for (int t = t0; t < t1; ++t, ++jg) {
+          const int st = jg % kStages;
           int row[kPPT];
 #pragma unroll
-          for (int g = 0; g < kPPT; ++g) {
-            const int idx = gt * kPPT + g;
-            // pages past the list end are read past the end of the pool: TMA fills zeros
+          for (int q = 0; q < kPPT; ++q) {
             if (kPerHead)
-              row[g] = idx < p.n_pages ? static_cast<int>((p.page_base + hp + __ldg(&ent[idx].x)) * P) : p.pool_rows;
+              row[q] = phys_next[q] >= 0 ? static_cast<int>((p.page_base + hp + phys_next[q]) * P) : p.pool_rows;
             else
-              row[g] = idx < p.n_pages ? static_cast<int>(((p.page_base + __ldg(&ent[idx].x)) * p.H + h) * P)
-                                       : p.pool_rows;
+              row[q] = phys_next[q] >= 0 ? static_cast<int>(((p.page_base + phys_next[q]) * p.H + h) * P) : p.pool_rows;
+          }
+          if (t + 1 < t1) {
+#pragma unroll
+            for (int q = 0; q < kPPT; ++q) {
+              const int idx = (t + 1) * kPPT + q;
+              phys_next[q] = idx < p.n_pages ? __ldg(&ent[idx].x) : -1;
+            }
+          }
+          if (jg >= kStages && !mbar_wait_bounded(&kv_empty[st], ((jg / kStages) - 1) & 1, abort_flag, p.err)) {
+            ok = false;
+            break;
           }
           mbar_arrive_expect_tx(&k_full[st], kTileBytes);
 #pragma unroll
-          for (int g = 0; g < kPPT; ++g)
-            tma_load_2d(k_s + st * kTileBytes + g * P * 128, &tmap_k, &k_full[st], 0, row[g]);
+          for (int q = 0; q < kPPT; ++q) tma_load_2d(k_s + st * kTileBytes + q * P * 128, &tmap_k, &k_full[st], 0, row[q]);
           mbar_arrive_expect_tx(&v_full[st], kTileBytes);
 #pragma unroll
-          for (int g = 0; g < kPPT; ++g)
-            tma_load_2d(v_s + st * kTileBytes + g * P * 128, &tmap_v, &v_full[st], 0, row[g]);
-          last[st] = j;
+          for (int q = 0; q < kPPT; ++q) tma_load_2d(v_s + st * kTileBytes + q * P * 128, &tmap_v, &v_full[st], 0, row[q]);
+          last[st] = jg;
         }
-        // drain: every copy this CTA issued has landed before shared memory is released
+        ++pc;
+      }
+      // drain: every copy this CTA issued has landed before shared memory is released
+      if (pc > 0) mbar_wait_drain(q_full, (pc - 1) & 1, p.err);
 #pragma unroll
-        for (int i = 0; i < kStages; ++i) {
-          if (last[i] >= 0) {
-            mbar_wait_drain(&k_full[i], (last[i] / kStages) & 1, p.err);
-            mbar_wait_drain(&v_full[i], (last[i] / kStages) & 1, p.err);
-          }
+      for (int i = 0; i < kStages; ++i) {
+        if (last[i] >= 0) {
+          mbar_wait_drain(&k_full[i], (last[i] / kStages) & 1, p.err);
+          mbar_wait_drain(&v_full[i], (last[i] / kStages) & 1, p.err);
         }
       }
-    } else if (warp == 1) {
-      // ------------------------------------------------------------------ MMA issuer
-      // the whole warp runs the loop and waits; one elected lane issues the MMAs and
-      // commits (the warp stays converged)
-      const uint32_t idesc_s = idesc_f16kind(1, kBM, kBN, 0, 0);
-      const uint32_t idesc_o = idesc_f16kind(1, kBM, kON, 0, 1);
-      const uint32_t tS = tmem + kColS, tP = tmem + kColP, tO = tmem + kColO, tQ = tmem + kColQ;
-      const uint32_t k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
-      const uint32_t ones_addr = smem_u32(ones_s);
-      const bool leader = elect_one();
-      bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(q_full, 0, abort_flag, p.err) &&
-                                            mbar_wait_bounded(&k_full[0], 0, abort_flag, p.err));
-      if (ok) {
+    }
+  } else if (warp == 1) {
+    reg_dealloc<kRegsLow>();
+    // ------------------------------------------------------------------ MMA issuer
+    const uint32_t idesc_s = idesc_f16kind(1, kBM, kBN, 0, 0);
+    const uint32_t idesc_o = idesc_f16kind(1, kBM, kON, 0, 1);
+    const uint32_t tS[2] = {tmem + kColS0, tmem + kColS1};
+    const uint32_t tO[2] = {tmem + kColO0, tmem + kColO1};
+    const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
+    const uint32_t ones_addr = smem_u32(ones_s);
+    const bool leader = elect_one();
+    auto issue_s = [&](int i, int st) {
+      const uint32_t qa = q_addr + i * kQBytes, kb = k_addr + st * kTileBytes;
+#pragma unroll
+      for (int kk = 0; kk < kHD / 16; ++kk)
+        mma_ss(tS[i], sw128_desc(qa + kk * 32, 16, 1024), sw128_desc(kb + kk * 32, 16, 1024), idesc_s, kk > 0);
+      mma_commit(&s_full[i]);
+    };
+    int jg = 0, pc = 0;
+    bool ok = true;
+    Sweep sw = sweep0;
+    int h, t0, t1;
+    while (ok && next_piece(sw, n_tiles, h, t0, t1)) {
+      const int n = t1 - t0;
+      {
+        const int st = jg % kStages;
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(q_full, pc & 1, abort_flag, p.err) &&
+                                         mbar_wait_bounded(&k_full[st], (jg / kStages) & 1, abort_flag, p.err)))
+          break;
         tc_fence_after();
         if (leader) {
-#pragma unroll
-          for (int kk = 0; kk < kHD / 16; ++kk)
-            mma_ts(tS, tQ + kk * 8, sw128_desc(k_addr + kk * 32, 16, 1024), idesc_s, kk > 0);
-          mma_commit(s_full);
+          issue_s(0, st);
+          issue_s(1, st);
+          if (n == 1) mma_commit(q_empty);
         }
         __syncwarp();
       }
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int st = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
-        if (j + 1 < n_tiles) {
-          const int st1 = (j + 1) % kStages;
-          const uint32_t ph1 = ((j + 1) / kStages) & 1;
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_free, j & 1, abort_flag, p.err) &&
-                                           mbar_wait_bounded(&k_full[st1], ph1, abort_flag, p.err)))
+      for (int j = 0; j < n; ++j) {
+        const int jj = jg + j;
+        const int st = jj % kStages;
+        const uint32_t ph = (jj / kStages) & 1;
+        const int st1 = (jj + 1) % kStages;
+        const uint32_t ph1 = ((jj + 1) / kStages) & 1;
+        for (int i = 0; i < kQT; ++i) {
+          bool w = mbar_wait_bounded(&p_full[i], jj & 1, abort_flag, p.err);
+          if (i == 0) {
+            w = w && mbar_wait_bounded(&v_full[st], ph, abort_flag, p.err);
+            if (j == 0 && pc > 0) w = w && mbar_wait_bounded(o_free, (pc - 1) & 1, abort_flag, p.err);
+            if (j + 1 < n) w = w && mbar_wait_bounded(&k_full[st1], ph1, abort_flag, p.err);
+          }
+          if (!__all_sync(0xffffffffu, w)) {
+            ok = false;
             break;
+          }
           tc_fence_after();
-          const uint32_t kb = k_addr + st1 * kTileBytes;
           if (leader) {
+            const uint32_t vb = v_addr + st * kTileBytes;
+            const uint32_t lbo = ones_addr - vb;
 #pragma unroll
-            for (int kk = 0; kk < kHD / 16; ++kk)
-              mma_ts(tS, tQ + kk * 8, sw128_desc(kb + kk * 32, 16, 1024), idesc_s, kk > 0);
-            mma_commit(s_full);
+            for (int kk = 0; kk < kBN / 16; ++kk)
+              mma_ts(tO[i], tS[i] + kk * 8, sw128_desc(vb + kk * 2048, lbo, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+            if (j + 1 < n) {
+              issue_s(i, st1);
+              if (i == 1 && j + 2 == n) mma_commit(q_empty);
+            }
           }
           __syncwarp();
         }
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&p_full[j & 1], (j >> 1) & 1, abort_flag, p.err) &&
-                                         mbar_wait_bounded(&v_full[st], ph, abort_flag, p.err)))
-          break;
-        tc_fence_after();
-        const uint32_t vb = v_addr + st * kTileBytes;
-        const uint32_t lbo = ones_addr - vb;
-        const uint32_t pa = tP + (j & 1) * (kBN / 2);
-        if (leader) {
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_ts(tO, pa + kk * 8, sw128_desc(vb + kk * 2048, lbo, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&pv_done[j & 1]);
-          mma_commit(&kv_empty[st]);
-        }
+        if (!ok) break;
+        if (leader) mma_commit(&kv_empty[st]);
         __syncwarp();
       }
-      if (leader) mma_commit(mma_final);
+      if (!ok) break;
+      if (leader) mma_commit(o_full);
       __syncwarp();
-      mbar_wait_drain(mma_final, 0, p.err);
-    } else {
-      // ------------------------------------------------------------------ softmax warps
-      const int wq = warp & 3;                      // TMEM lane quadrant this warp may access
-      const int r = wq * 32 + lane;                 // query row within the tile
-      const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-      const uint32_t tS = tmem + kColS + lane_off, tP = tmem + kColP + lane_off, tO = tmem + kColO + lane_off;
-      {
-        // this row of Q into TMEM (the A operand of S = Q K^T): 64 bf16 = 32 packed columns
-        uint32_t qv[32];
-        const int row = qt * kBM + r;
-        if (row < p.T) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.q + (static_cast<long long>(row) * p.H + h) * kHD);
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const uint4 w = __ldg(src + v);
-            qv[4 * v] = w.x;
-            qv[4 * v + 1] = w.y;
-            qv[4 * v + 2] = w.z;
-            qv[4 * v + 3] = w.w;
-          }
-        } else {
-#pragma unroll
-          for (int v = 0; v < 32; ++v) qv[v] = 0u;
-        }
-        tmem_st32(tmem + kColQ + lane_off, qv);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(q_full);
-      }
-      const float c = p.scale_log2;
+      jg += n;
+      ++pc;
+    }
+    if (leader) mma_commit(mma_final);
+    __syncwarp();
+    mbar_wait_drain(mma_final, 0, p.err);
+  } else if (warp < 4) {
+    reg_dealloc<kRegsLow>();                       // warps 2 and 3 only give up registers
+  } else {
+    reg_alloc<kRegsHigh>();
+    // ------------------------------------------------------------------ softmax warps
+    const int wg = (warp - 4) >> 2;               // query tile of the pair
+    const int wq = warp & 3;                      // TMEM lane quadrant this warp may access
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + (wg ? kColS1 : kColS0) + lane_off;
+    const uint32_t tO = tmem + (wg ? kColO1 : kColO0) + lane_off;
+    const float c = p.scale_log2;
+    int jg = 0, pc = 0;
+    bool ok = true;
+    Sweep sw = sweep0;
+    int h, t0, t1;
+    while (ok && next_piece(sw, n_tiles, h, t0, t1)) {
+      const int n = t1 - t0;
+      const Entry* ent = kPerHead ? p.entries + static_cast<long long>(h) * p.head_pages : p.entries;
       float m = -INFINITY;       // reference max (log2 domain) of the row
-      float masked = 0.f;        // row-sum share of zero-padded slots, rescaled like O'
-      bool ok = true;
-      // valid-slot counts of the next KV tile's pages, loaded one tile ahead
       int vnext[kPPT];
 #pragma unroll
-      for (int g = 0; g < kPPT; ++g) {
-        const int idx = tile0 * kPPT + g;
-        vnext[g] = idx < p.n_pages ? __ldg(&ent[idx].w) : 0;
+      for (int q = 0; q < kPPT; ++q) {
+        const int idx = t0 * kPPT + q;
+        vnext[q] = idx < p.n_pages ? __ldg(&ent[idx].w) : 0;
       }
-      // S of the current tile lives in registers; the next tile's S is loaded while this
-      // tile's P store is in flight
-      uint32_t s[2][32];
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_full, 0, abort_flag, p.err))) ok = false;
-      if (ok) {
+      for (int j = 0; j < n; ++j) {
+        const int jj = jg + j;
+        int vcur[kPPT];
+        bool partial = false;
+#pragma unroll
+        for (int q = 0; q < kPPT; ++q) {
+          vcur[q] = vnext[q];
+          partial |= vcur[q] < P;
+        }
+        if (j + 1 < n) {
+#pragma unroll
+          for (int q = 0; q < kPPT; ++q) {
+            const int idx = (t0 + j + 1) * kPPT + q;
+            vnext[q] = idx < p.n_pages ? __ldg(&ent[idx].w) : 0;
+          }
+        }
+        uint32_t s[kBN];
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s_full[wg], jj & 1, abort_flag, p.err))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        tmem_ld32(tS + 0, s[0]);
-        tmem_ld32(tS + 32, s[1]);
+        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
         tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);
-      }
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        int n_masked = 0;
+        if (partial) {
+          // slots past a page's valid count (and pages past the list end) take no weight
 #pragma unroll
-        for (int g = 0; g < kPPT; ++g) n_masked += P - vnext[g];
-        if (j + 1 < n_tiles) {
-#pragma unroll
-          for (int g = 0; g < kPPT; ++g) {
-            const int idx = (tile0 + j + 1) * kPPT + g;
-            vnext[g] = idx < p.n_pages ? __ldg(&ent[idx].w) : 0;
-          }
+          for (int cc = 0; cc < kBN; ++cc)
+            if ((cc % P) >= vcur[cc / P]) s[cc] = __float_as_uint(-INFINITY);
         }
-        // P = 2^(s*c - m): exponent pairs with one packed FMA, two MUFU ex2, one bf16 pack;
-        // a bf16x2 max over the packed P tells whether any exponent exceeded 2^8 (or the
-        // reference was unset), in which case the row's reference max moves (slow path)
-        uint32_t pb[kBN / 2];
-        uint32_t mxb = 0u;
-        {
-          const uint64_t c2 = pk2(c, c), nm2 = pk2(-m, -m);
+        // exact fp32 tile max; the row's reference max moves when some P would exceed 2^8
+        // (or on the first tile of a piece), and O' is then rescaled by 2^(m_old - m_new):
+        // the previous tile's P.V was issued before this tile's S and has completed
+        float ta = -INFINITY, tb = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < kBN / 2; ++i) {
-            float x0, x1;
-            up2(fma2_pair(s[(2 * i) / 32][(2 * i) % 32], s[(2 * i + 1) / 32][(2 * i + 1) % 32], c2, nm2), x0, x1);
-            pb[i] = bf16x2_trunc(ex2(x0), ex2(x1));
-            mxb = max_bf16x2(mxb, pb[i]);
-          }
+        for (int cc = 0; cc < kBN; cc += 4) {
+          ta = max3(ta, __uint_as_float(s[cc]), __uint_as_float(s[cc + 1]));
+          tb = max3(tb, __uint_as_float(s[cc + 2]), __uint_as_float(s[cc + 3]));
         }
-        const bool move = (j == 0) || fmaxf(bf16lo(mxb), bf16hi(mxb)) > kPMax;
+        const float tm = fmaxf(ta, tb) * c;
+        const bool move = (j == 0) || tm > m + kLog2PMax;
         if (__any_sync(0xffffffffu, move)) {
-          // slow path (first tile or a new maximum): exact fp32 tile max for the rows that
-          // move their reference; rescale O' and the masked share by 2^(m_old - m_new)
-          float ta = -INFINITY, tb = -INFINITY;
-#pragma unroll
-          for (int cc = 0; cc < kBN; cc += 4) {
-            ta = max3(ta, __uint_as_float(s[cc / 32][cc % 32]), __uint_as_float(s[cc / 32][cc % 32 + 1]));
-            tb = max3(tb, __uint_as_float(s[cc / 32][cc % 32 + 2]), __uint_as_float(s[cc / 32][cc % 32 + 3]));
-          }
-          const float m_new = move ? fmaxf(ta, tb) * c : m;
-          const bool resc = move && j > 0;
+          const float m_new = move ? (tm == -INFINITY ? (m == -INFINITY ? 0.f : m) : tm) : m;
+          const bool resc = move && j > 0 && m_new != m;
           if (__any_sync(0xffffffffu, resc)) {
-            // O' row *= f; the previous tile's P.V must have landed
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait_bounded(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, p.err))) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
             const float f = resc ? ex2(m - m_new) : 1.0f;
-            masked *= f;
 #pragma unroll
             for (int q4 = 0; q4 < kON / 16; ++q4) {
               uint32_t oc[16];
@@ -452,111 +569,36 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
             }
           }
           m = m_new;
-          const uint64_t c2 = pk2(c, c), nm2 = pk2(-m, -m);
-#pragma unroll
-          for (int i = 0; i < kBN / 2; ++i) {
-            float x0, x1;
-            up2(fma2_pair(s[(2 * i) / 32][(2 * i) % 32], s[(2 * i + 1) / 32][(2 * i + 1) % 32], c2, nm2), x0, x1);
-            pb[i] = bf16x2_trunc(ex2(x0), ex2(x1));
-          }
         }
-        if (n_masked) {
-          // each zero-padded slot scored 0 and contributed exactly bf16(2^-m) to the sum
-          masked += static_cast<float>(n_masked) * bf16lo(bf16x2_trunc(ex2(-m), 0.f));
-        }
-        // P buffer j & 1 was last read by the P.V product of tile j - 2
-        if (j >= 2) {
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, p.err))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-        }
-        tmem_st32(tP + (j & 1) * (kBN / 2), pb);
-        // tcgen05.ld/st are .sync.aligned: every branch around them is kept warp-uniform
-        const bool more = j + 1 < n_tiles;
-        if (more) {
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_full, (j + 1) & 1, abort_flag, p.err))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          tmem_ld32(tS + 0, s[0]);
-          tmem_ld32(tS + 32, s[1]);
-        }
+        uint32_t pb[kBN / 2];
+        tile_p(s, c, m, pb);
+        // P over the first 64 columns of S (tcgen05.ld/st are .sync.aligned: every branch
+        // around them is warp-uniform)
+        tmem_st32(tS + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pb[0]));
+        tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pb[32]));
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[j & 1]);
-        if (more) {
-          tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(s_free);
-        }
+        if (lane == 0) mbar_arrive(&p_full[wg]);
       }
-      const int jl = n_tiles - 1;
-      if (__all_sync(0xffffffffu, ok && mbar_wait_bounded(&pv_done[jl & 1], (jl >> 1) & 1, abort_flag, p.err))) {
-        tc_fence_after();
-        uint32_t o0[32], o1[32], ls[16];
-        tmem_ld32(tO, o0);
-        tmem_ld32(tO + 32, o1);
-        tmem_ld16(tO + 64, ls);
-        tmem_ld_wait();
-        const float l = __uint_as_float(ls[0]) - masked;
-        const float inv = 1.f / l;
-        const int row = qt * kBM + r;
-        if (p.splits == 1) {
-          if (row < p.T) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<long long>(row) * p.H + h) * kHD);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 w;
-              w.x = pack_bf16(__uint_as_float(o0[8 * v + 0]) * inv, __uint_as_float(o0[8 * v + 1]) * inv);
-              w.y = pack_bf16(__uint_as_float(o0[8 * v + 2]) * inv, __uint_as_float(o0[8 * v + 3]) * inv);
-              w.z = pack_bf16(__uint_as_float(o0[8 * v + 4]) * inv, __uint_as_float(o0[8 * v + 5]) * inv);
-              w.w = pack_bf16(__uint_as_float(o0[8 * v + 6]) * inv, __uint_as_float(o0[8 * v + 7]) * inv);
-              dst[v] = w;
-            }
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 w;
-              w.x = pack_bf16(__uint_as_float(o1[8 * v + 0]) * inv, __uint_as_float(o1[8 * v + 1]) * inv);
-              w.y = pack_bf16(__uint_as_float(o1[8 * v + 2]) * inv, __uint_as_float(o1[8 * v + 3]) * inv);
-              w.z = pack_bf16(__uint_as_float(o1[8 * v + 4]) * inv, __uint_as_float(o1[8 * v + 5]) * inv);
-              w.w = pack_bf16(__uint_as_float(o1[8 * v + 6]) * inv, __uint_as_float(o1[8 * v + 7]) * inv);
-              dst[4 + v] = w;
-            }
-          }
-        } else {
-          const long long pi = (static_cast<long long>(h) * p.splits + split) * p.q_tiles + qt;
-          float4* dst = reinterpret_cast<float4*>(p.part_o + (pi * kBM + r) * kHD);
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[v] = make_float4(__uint_as_float(o0[4 * v + 0]) * inv, __uint_as_float(o0[4 * v + 1]) * inv,
-                                 __uint_as_float(o0[4 * v + 2]) * inv, __uint_as_float(o0[4 * v + 3]) * inv);
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[8 + v] = make_float4(__uint_as_float(o1[4 * v + 0]) * inv, __uint_as_float(o1[4 * v + 1]) * inv,
-                                     __uint_as_float(o1[4 * v + 2]) * inv, __uint_as_float(o1[4 * v + 3]) * inv);
-          p.part_lse[pi * kBM + r] = m + __log2f(l);
-        }
+      if (!ok) break;
+      // ---------------------------------------------------------------- epilogue
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(o_full, pc & 1, abort_flag, p.err))) {
+        ok = false;
+        break;
       }
-      if (p.splits > 1 && p.split_cnt) {
-        // the split CTA that finishes a (query tile, head) last merges every split's
-        // partial (threadfence-then-count: each partial is visible before its count)
-        __shared__ int s_last;
-        __threadfence();
-        softmax_warps_sync();
-        if (warp == 2 && lane == 0) s_last = atomicAdd(&p.split_cnt[h * p.q_tiles + qt], 1) == p.splits - 1;
-        softmax_warps_sync();
-        if (s_last) {
-          __threadfence();
-          const int row = qt * kBM + r;
-          if (row < p.T) merge_split_row(p, k_s, h, qt, r, row);
-          if (warp == 2 && lane == 0) p.split_cnt[h * p.q_tiles + qt] = 0;   // ready for the next launch
-        }
-      }
+      tc_fence_after();
+      uint32_t o0[32], o1[32], ls[16];
+      tmem_ld32(tO, o0);
+      tmem_ld32(tO + 32, o1);
+      tmem_ld16(tO + 64, ls);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_free);
+      store_piece(p, wg, wq, lane, h, qp, g, o0, o1, __uint_as_float(ls[0]), m);
+      jg += n;
+      ++pc;
     }
   }
   tc_fence_before();
@@ -568,21 +610,23 @@ __global__ void __launch_bounds__(tc::kThreads, 2)
   }
 }
 
-// Merge split partials: O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M). One warp per
-// (row, head): lane s (and s + 32) loads split s's log-sum-exp, so the maximum and the
-// weights take one round of loads and warp shuffles; then each lane accumulates two of
-// the 64 dims over the splits, four partial rows in flight at a time (up to 64 splits).
+// Merge split partials of the FP8 kernel: O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M).
+// One warp per (row, head): lane s (and s + 32) loads split s's log-sum-exp, so the maximum
+// and the weights take one round of loads and warp shuffles; then each lane accumulates two
+// of the 64 dims over the splits (up to 64 splits). Partials are [head][split][query tile]
+// tiles of 128 rows.
 __global__ void combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                                __nv_bfloat16* __restrict__ out, int T, int H, int q_tiles, int splits) {
   griddep_wait();
   griddep_launch_dependents();
+  constexpr int kRows = 128, kD = 64;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= T * H) return;
   const int t = gw / H, h = gw % H;
-  const int qt = t / tc::kBM, r = t % tc::kBM;
+  const int qt = t / kRows, r = t % kRows;
   const long long pi0 = static_cast<long long>(h) * splits * q_tiles + qt;
-  auto row_of = [&](int s) { return (pi0 + static_cast<long long>(s) * q_tiles) * tc::kBM + r; };
+  auto row_of = [&](int s) { return (pi0 + static_cast<long long>(s) * q_tiles) * kRows + r; };
   const float l0 = lane < splits ? __ldg(&part_lse[row_of(lane)]) : -INFINITY;
   const float l1 = lane + 32 < splits ? __ldg(&part_lse[row_of(lane + 32)]) : -INFINITY;
   float M = fmaxf(l0, l1);
@@ -597,12 +641,12 @@ __global__ void combine_kernel(const float* __restrict__ part_o, const float* __
 #pragma unroll 4
   for (int s = 0; s < splits; ++s) {
     const float w = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
-    const float2 o = __ldg(reinterpret_cast<const float2*>(part_o + row_of(s) * tc::kHD) + lane);
+    const float2 o = __ldg(reinterpret_cast<const float2*>(part_o + row_of(s) * kD) + lane);
     a0 = fmaf(w, o.x, a0);
     a1 = fmaf(w, o.y, a1);
   }
   const float inv = 1.f / ws;
-  reinterpret_cast<__nv_bfloat162*>(out + (static_cast<long long>(t) * H + h) * tc::kHD)[lane] =
+  reinterpret_cast<__nv_bfloat162*>(out + (static_cast<long long>(t) * H + h) * kD)[lane] =
       __floats2bfloat162_rn(a0 * inv, a1 * inv);
 }
 
@@ -634,12 +678,15 @@ bool encode_pool_tmap(CUtensorMap* map, void* base, size_t rows, int D, int P, i
   return r == CUDA_SUCCESS;
 }
 
+// Queries [T][H][64] bf16 as a 3-D map; one box is 128 rows of one head (128-byte swizzle),
+// rows past T read as zeros.
 static bool encode_q_tmap(CUtensorMap* map, const void* q, int T, int H) {
   auto fn = get_encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(tc::kHD), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(tc::kHD) * 2, static_cast<cuuint64_t>(H) * tc::kHD * 2};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(tc::kHD), 1, static_cast<cuuint32_t>(tc::kBM)};
+  constexpr int kD = 64, kRows = 128;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * 2, static_cast<cuuint64_t>(H) * kD * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kD), 1, static_cast<cuuint32_t>(kRows)};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -647,15 +694,13 @@ static bool encode_q_tmap(CUtensorMap* map, const void* q, int T, int H) {
   return r == CUDA_SUCCESS;
 }
 
-// Pick the number of KV splits. Cost of a split count, in units of one KV tile of a CTA
-// that shares its SM: waves x (fixed cost of a CTA + tiles per CTA), where a CTA alone on
-// its SM (at most one per SM in the whole launch) runs a tile in about 0.84 of the time,
-// plus a cost per split (the partials written and merged). Fixed cost and split cost:
-// 8 and 2 tiles for the bf16 kernel, whose last split CTA merges (measured on 24-, 272- and
-// 1,146-tile caches); 4 and 0.25 (+ 0.5 for the combine launch) for the FP8 kernel, one CTA
-// per SM. Among counts within 1% of the best cost the fewest splits win.
+// Pick the number of KV splits of the FP8 kernel (one CTA per SM, two query tiles per CTA).
+// Cost of a split count, in units of one 64-slot KV tile: waves x (fixed cost of a CTA +
+// tiles per CTA) + a cost per split (the partials written and combined): 4 and
+// 0.5 + 0.25 s tiles, measured. Among counts within 1% of the best cost the fewest win.
 int choose_splits(int units, int tiles, int slots, bool fp8) {
-  const double cta_cost = fp8 ? 4.0 : 8.0;
+  (void)fp8;
+  const double cta_cost = 4.0;
   const int max_s = tiles < 64 ? tiles : 64;
   double cost[65];
   double best_cost = 1e30;
@@ -665,9 +710,8 @@ int choose_splits(int units, int tiles, int slots, bool fp8) {
     if ((tiles + tps - 1) / tps != s) continue;        // the same as a smaller split count
     const long long ctas = static_cast<long long>(units) * s;
     const long long waves = (ctas + slots - 1) / slots;
-    const double per_tile = !fp8 && 2 * ctas <= slots ? 0.84 : 1.0;
-    const double split_cost = s == 1 ? 0.0 : fp8 ? 0.5 + 0.25 * s : 2.0 * s;
-    cost[s] = static_cast<double>(waves) * (cta_cost + tps) * per_tile + split_cost;
+    const double split_cost = s == 1 ? 0.0 : 0.5 + 0.25 * s;
+    cost[s] = static_cast<double>(waves) * (cta_cost + tps) + split_cost;
     if (cost[s] < best_cost) best_cost = cost[s];
   }
   for (int s = 1; s <= max_s; ++s)
@@ -675,29 +719,113 @@ int choose_splits(int units, int tiles, int slots, bool fp8) {
   return 1;
 }
 
+// Schedule of the bf16 kernel. R = KV tiles per group; groups of q_pairs CTAs. Automatic:
+// as many groups as fill the SMs (one CTA each); with kv_splits = s > 0, about s pieces per
+// head. If the partial scratch (part_tiles 128-row tiles) cannot hold every unit's pieces,
+// R grows until it can (R a multiple of the head's tiles leaves one piece per unit), unless
+// `strict`, in which case a split count that does not fit fails.
+bool plan_attn_bf16(int T, int H, int n_pages, int P, int sm_count, int kv_splits, size_t part_tiles, bool strict,
+                    AttnPlan* out) {
+  if (T < 1 || H < 1 || n_pages < 1 || P < 1 || sm_count < 1) return false;
+  AttnPlan a{};
+  a.q_tiles = (T + tc::kBM - 1) / tc::kBM;
+  a.q_pairs = (a.q_tiles + 1) / 2;
+  a.n_tiles = static_cast<int>((static_cast<long long>(n_pages) * P + tc::kBN - 1) / tc::kBN);
+  const long long HT = static_cast<long long>(H) * a.n_tiles;
+  long long R;
+  if (kv_splits > 0) {
+    R = (a.n_tiles + kv_splits - 1) / kv_splits;
+  } else {
+    const long long groups = std::max(1, sm_count / a.q_pairs);
+    R = (HT + groups - 1) / groups;
+  }
+  if (R < 1) R = 1;
+  for (;;) {
+    const long long groups = (HT + R - 1) / R;
+    int max_pieces = 1;
+    for (int h = 0; h < H; ++h) {
+      const long long gf = (static_cast<long long>(h) * a.n_tiles) / R;
+      const long long gl = (static_cast<long long>(h) * a.n_tiles + a.n_tiles - 1) / R;
+      max_pieces = std::max(max_pieces, static_cast<int>(gl - gf + 1));
+    }
+    const long long need = max_pieces > 1 ? static_cast<long long>(H) * a.q_pairs * max_pieces * tc::kQT : 0;
+    if (need <= static_cast<long long>(part_tiles) || R % a.n_tiles == 0 || strict) {
+      if (need > static_cast<long long>(part_tiles)) return false;
+      a.R = static_cast<int>(R);
+      a.groups = static_cast<int>(groups);
+      a.max_pieces = max_pieces;
+      a.grid = a.groups * a.q_pairs;
+      a.part_tiles = static_cast<size_t>(need);
+      *out = a;
+      return true;
+    }
+    // grow R to the next multiple of the head's tiles, or double it below that
+    R = R * 2 >= a.n_tiles ? ((R / a.n_tiles) + 1) * a.n_tiles : R * 2;
+  }
+}
+
 cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used, int* launched) {
   if (launched) *launched = 0;
   if (a.P != 16 || (a.fp8 && a.head_pages)) return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!a.fp8 && !attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(tc::kSmemBytes));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn_tc_kernel<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(tc::kSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  const int qh = a.q_heads > 0 ? a.q_heads : a.H;
+  if (a.head0 < 0 || a.head0 + a.H > qh || (a.fp8 && qh != a.H)) return cudaErrorInvalidValue;
   CUtensorMap tq;
-  if (!encode_q_tmap(&tq, a.q, a.T, a.H)) return cudaErrorInvalidValue;
-  const int q_tiles = (a.T + tc::kBM - 1) / tc::kBM;
-  const int total_tiles = (a.n_pages * a.P + tc::kBN - 1) / tc::kBN;
-  // a CTA of the bf16 kernel takes one query tile (two CTAs per SM); a CTA of the FP8
-  // kernel takes two (one CTA per SM)
-  const int units = a.fp8 ? ((q_tiles + 1) / 2) * a.H : q_tiles * a.H;
-  const int slots = a.fp8 ? a.sm_count : 2 * a.sm_count;
+  if (!encode_q_tmap(&tq, a.q, a.T, qh)) return cudaErrorInvalidValue;
+  if (!a.fp8) {
+    static PerDeviceOnce attr;
+    cudaError_t e = attr.run([] {
+      cudaError_t r = cudaFuncSetAttribute(attn_tc_kernel<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(tc::kSmemBytes));
+      if (r == cudaSuccess)
+        r = cudaFuncSetAttribute(attn_tc_kernel<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(tc::kSmemBytes));
+      return r;
+    });
+    if (e != cudaSuccess) return e;
+    AttnPlan pl;
+    if (!plan_attn_bf16(a.T, a.H, a.n_pages, a.P, a.sm_count, a.splits, a.part_rows, a.strict_splits, &pl))
+      return cudaErrorInvalidValue;
+    if (pl.max_pieces > 1 && !a.split_cnt) return cudaErrorInvalidValue;
+    TcParams prm{};
+    prm.q = static_cast<const __nv_bfloat16*>(a.q);
+    prm.entries = a.entries;
+    prm.n_pages = a.n_pages;
+    prm.T = a.T;
+    prm.H = a.H;
+    prm.q_tiles = pl.q_tiles;
+    prm.q_pairs = pl.q_pairs;
+    prm.splits = pl.max_pieces;
+    prm.tiles_per_split = pl.R;
+    prm.total_tiles = pl.n_tiles;
+    prm.page_base = a.page_base;
+    prm.pool_rows = static_cast<int>(a.pool_rows);
+    prm.scale_log2 = static_cast<float>(static_cast<double>(a.softmax_scale) * 1.4426950408889634);
+    prm.out = static_cast<__nv_bfloat16*>(a.o);
+    prm.part_o = a.part_o;
+    prm.part_lse = a.part_lse;
+    prm.err = a.err;
+    prm.head_pages = a.head_pages;
+    prm.split_cnt = a.split_cnt;
+    prm.out_heads = qh;
+    prm.head0 = a.head0;
+    if (a.head_pages)
+      e = launch_pdl(attn_tc_kernel<16, true>, dim3(pl.grid), dim3(tc::kThreads), tc::kSmemBytes, s, tq, *a.tmap_k,
+                     *a.tmap_v, prm);
+    else
+      e = launch_pdl(attn_tc_kernel<16, false>, dim3(pl.grid), dim3(tc::kThreads), tc::kSmemBytes, s, tq, *a.tmap_k,
+                     *a.tmap_v, prm);
+    if (e != cudaSuccess) return e;
+    if (launched) *launched = 1;
+    if (splits_used) *splits_used = pl.max_pieces;
+    return cudaSuccess;
+  }
+  // FP8 storage: one CTA per SM takes two 128-row query tiles of a head and a range of
+  // 64-slot KV tiles; more than one split goes through the combine kernel
+  const int q_tiles = (a.T + 127) / 128;
+  const int total_tiles = (a.n_pages * a.P + 63) / 64;
+  const int units = ((q_tiles + 1) / 2) * a.H;
   const int part_units = q_tiles * a.H;       // 128-row partial tiles per split
-  int splits = a.splits > 0 ? a.splits : choose_splits(units, total_tiles, slots, a.fp8);
+  int splits = a.splits > 0 ? a.splits : choose_splits(units, total_tiles, a.sm_count, true);
   if (splits > total_tiles) splits = total_tiles;
   if (splits > 64) splits = 64;                  // the combine takes up to 64 partials per row
   int tps = (total_tiles + splits - 1) / splits;
@@ -709,7 +837,7 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
     tps = (total_tiles + splits - 1) / splits;
     splits = (total_tiles + tps - 1) / tps;
   }
-  TcParams prm;
+  TcParams prm{};
   prm.q = static_cast<const __nv_bfloat16*>(a.q);
   prm.k_scale = a.k_scale;
   prm.v_scale = a.v_scale;
@@ -728,27 +856,12 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   prm.part_o = a.part_o;
   prm.part_lse = a.part_lse;
   prm.err = a.err;
-  prm.head_pages = a.head_pages;
-  prm.k_chan = a.fp8 ? a.k_chan : nullptr;
-  prm.v_tok = a.fp8 ? a.v_tok : nullptr;
-  // the last split CTA merges when a merge is one copy round per half row (up to four
-  // splits); with more, a separate combine launch is faster (measured at 9 splits)
-  prm.split_cnt = a.fp8 || splits > 4 ? nullptr : a.split_cnt;
-  const int grid = units * splits;
-  cudaError_t e;
-  if (a.fp8) {
-    e = launch_attn_fp8_kernel(s, tq, *a.tmap_k, *a.tmap_v, prm, grid);
-  } else {
-    if (a.head_pages)
-      e = launch_pdl(attn_tc_kernel<16, true>, dim3(grid), dim3(tc::kThreads), tc::kSmemBytes, s, tq, *a.tmap_k,
-                     *a.tmap_v, prm);
-    else
-      e = launch_pdl(attn_tc_kernel<16, false>, dim3(grid), dim3(tc::kThreads), tc::kSmemBytes, s, tq, *a.tmap_k,
-                     *a.tmap_v, prm);
-  }
+  prm.k_chan = a.k_chan;
+  prm.v_tok = a.v_tok;
+  cudaError_t e = launch_attn_fp8_kernel(s, tq, *a.tmap_k, *a.tmap_v, prm, units * splits);
   if (e != cudaSuccess) return e;
   if (launched) *launched = 1;
-  if (splits > 1 && !prm.split_cnt) {
+  if (splits > 1) {
     const long long warps = static_cast<long long>(a.T) * a.H;
     const int threads = 256;
     e = launch_pdl(combine_kernel, dim3(static_cast<int>((warps * 32 + threads - 1) / threads)), dim3(threads), 0, s,

@@ -499,6 +499,174 @@ __global__ void __launch_bounds__(1024) tier_lists_kernel(Scratch sc, int N) {
   }
 }
 
+// Tier selection and tier lists in one CTA with the candidates' keys and protected flags
+// staged in shared memory once (N <= kTierSmemMax): the same MSB-first radix selection as
+// tier_select_kernel and the same position-order scans as tier_lists_kernel, without their
+// repeated global reads, which bound those kernels by load latency.
+constexpr int kTierSmemMax = 40960;
+__global__ void __launch_bounds__(1024) tier_kernel(Scratch sc, int N, int k1, int k2) {
+  extern __shared__ __align__(16) uint8_t tier_sm[];
+  uint32_t* key_s = reinterpret_cast<uint32_t*>(tier_sm);
+  uint8_t* prot_s = tier_sm + static_cast<size_t>(N) * 4;
+  __shared__ int hist[2][256];
+  __shared__ uint32_t s_prefix[2];
+  __shared__ int s_krem[2];
+  __shared__ int s_np;
+  __shared__ int s_warp[32];
+  int np_local = 0;
+#pragma unroll 4
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    const uint8_t pr = sc.prot[i];
+    key_s[i] = desc_key(sc.shat[i]);
+    prot_s[i] = pr;
+    np_local += !pr;
+  }
+  int n_np;
+  cta_exclusive_scan(np_local, s_warp, &n_np);   // its barriers also publish the staged arrays
+  if (threadIdx.x == 0) {
+    s_np = n_np;
+    s_prefix[0] = s_prefix[1] = 0u;
+    s_krem[0] = k1;
+    s_krem[1] = k2;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = threadIdx.x; b < 512; b += blockDim.x) hist[b >> 8][b & 255] = 0;
+    __syncthreads();
+    const uint32_t hi_mask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+    const uint32_t p0 = s_prefix[0], p1 = s_prefix[1];
+    for (int base = 0; base < N; base += blockDim.x) {
+      const int i = base + threadIdx.x;
+      bool np = false;
+      uint32_t key = 0;
+      if (i < N) {
+        np = !prot_s[i];
+        key = key_s[i];
+      }
+      const int digit = (key >> shift) & 255;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const bool in = np && ((key & hi_mask) == ((q ? p1 : p0) & hi_mask));
+        const uint32_t act = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          const uint32_t peers = __match_any_sync(act, digit);
+          if (lane == __ffs(peers) - 1) atomicAdd(&hist[q][digit], __popc(peers));
+        }
+      }
+    }
+    __syncthreads();
+    if (warp < 2) {
+      const int q = warp;
+      const int kr = s_krem[q];
+      int c8[8], sum = 0;
+#pragma unroll
+      for (int d = 0; d < 8; ++d) {
+        c8[d] = hist[q][lane * 8 + d];
+        sum += c8[d];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int before = incl - sum;
+      int found = -1, krem_new = 0;
+      if (kr >= 1 && before < kr && kr <= incl) {
+#pragma unroll
+        for (int d = 0; d < 8; ++d) {
+          if (found < 0 && kr <= before + c8[d]) {
+            found = lane * 8 + d;
+            krem_new = kr - before;
+          }
+          before += c8[d];
+        }
+      }
+      if (found >= 0) {
+        s_prefix[q] |= static_cast<uint32_t>(found) << shift;
+        s_krem[q] = krem_new;
+      }
+    }
+    __syncthreads();
+  }
+  __shared__ uint32_t s_v[2];
+  __shared__ int s_need[2];
+  if (threadIdx.x < 2) {
+    const int q = threadIdx.x;
+    const int k = q ? k2 : k1;
+    uint32_t v = s_prefix[q];
+    int need = s_krem[q];
+    if (k <= 0) {
+      v = 0u;
+      need = 0;
+    } else if (k >= s_np) {
+      v = 0xFFFFFFFFu;
+      need = 0x7fffffff;
+    }
+    s_v[q] = v;
+    s_need[q] = need;
+    sc.counts[8 + 2 * q] = static_cast<int32_t>(v);
+    sc.counts[9 + 2 * q] = need;
+  }
+  __syncthreads();
+  // the three lists, each thread a contiguous range of positions
+  const uint32_t v1 = s_v[0], v2 = s_v[1];
+  const int need1 = s_need[0], need2 = s_need[1];
+  const int ch = (N + blockDim.x - 1) / blockDim.x;
+  const int i0 = min(N, static_cast<int>(threadIdx.x) * ch), i1 = min(N, i0 + ch);
+  int c1 = 0, c2 = 0;
+  for (int i = i0; i < i1; ++i) {
+    const bool pr = prot_s[i];
+    const uint32_t key = key_s[i];
+    c1 += !pr && key == v1;
+    c2 += !pr && key == v2;
+  }
+  int tot;
+  const int b1 = cta_exclusive_scan(c1, s_warp, &tot);
+  const int b2 = cta_exclusive_scan(c2, s_warp, &tot);
+  auto flags = [&](int i, int& r1, int& r2, int (&f)[3]) {
+    const bool pr = prot_s[i];
+    const uint32_t key = key_s[i];
+    const bool e1 = !pr && key == v1, e2 = !pr && key == v2;
+    const bool lt1 = !pr && (key < v1 || (e1 && r1 < need1));
+    const bool lt2 = !pr && (key < v2 || (e2 && r2 < need2));
+    r1 += e1;
+    r2 += e2;
+    f[0] = pr || lt1;
+    f[1] = lt1;
+    f[2] = !lt1 && lt2;
+  };
+  int n[3] = {0, 0, 0};
+  {
+    int r1 = b1, r2 = b2, f[3];
+    for (int i = i0; i < i1; ++i) {
+      flags(i, r1, r2, f);
+      n[0] += f[0];
+      n[1] += f[1];
+      n[2] += f[2];
+    }
+  }
+  int off[3], total[3];
+#pragma unroll
+  for (int q = 0; q < 3; ++q) off[q] = cta_exclusive_scan(n[q], s_warp, &total[q]);
+  int* lists[3] = {sc.keep, sc.elig, sc.merge};
+  {
+    int r1 = b1, r2 = b2, f[3];
+    for (int i = i0; i < i1; ++i) {
+      flags(i, r1, r2, f);
+#pragma unroll
+      for (int q = 0; q < 3; ++q)
+        if (f[q]) lists[q][off[q]++] = i;
+    }
+  }
+  if (threadIdx.x == 0) {
+    sc.counts[1] = total[0];
+    sc.counts[2] = total[1];
+    sc.counts[3] = total[2];
+  }
+}
+
 // ------------------------------------------------------------------ merge targets
 // Full H*D keys of listed tokens (the stored bf16 values), their fp64 norms and fp32
 // inverse norms.
@@ -574,6 +742,65 @@ __global__ void __launch_bounds__(1024) merge_group_kernel(Scratch sc, int n_src
   __syncthreads();
   for (int q = threadIdx.x; q < n_src; q += blockDim.x) {
     const int pos = sc.merge[sc.order[q]];
+    const long long k = sc.slot[pos];
+    sc.src_base[q] = ((k / P) * H * P + k % P) * D;
+    sc.src_cnt[q] = sc.cnt[pos];
+  }
+}
+
+// merge_group_kernel with its counting sort in shared memory (group ends, cursors and the
+// grouped order; n_src + 2 n_elig + 1 ints <= kGroupSmemInts), written to the scratch once
+// at the end: the global version is bound by the latency of its atomics and of the
+// insertion sort's global accesses.
+constexpr int kGroupSmemInts = 53248;
+__global__ void __launch_bounds__(1024) merge_group_smem_kernel(Scratch sc, int n_src, int n_elig, int H, int P,
+                                                                int D) {
+  extern __shared__ __align__(16) int grp_sm[];
+  int* bucket = grp_sm;                    // [n_elig + 1]
+  int* cursor = bucket + n_elig + 1;       // [n_elig]
+  int* order = cursor + n_elig;            // [n_src]
+  __shared__ int s_warp[32];
+  for (int e = threadIdx.x; e <= n_elig; e += blockDim.x) bucket[e] = 0;
+  for (int e = threadIdx.x; e < n_elig; e += blockDim.x) cursor[e] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_src; i += blockDim.x) atomicAdd(&bucket[sc.target[i] + 1], 1);
+  __syncthreads();
+  {
+    const int ch = (n_elig + blockDim.x - 1) / blockDim.x;
+    const int e0 = min(n_elig, static_cast<int>(threadIdx.x) * ch), e1 = min(n_elig, e0 + ch);
+    int local = 0;
+    for (int e = e0; e < e1; ++e) local += bucket[e + 1];
+    int total;
+    int run = cta_exclusive_scan(local, s_warp, &total);
+    for (int e = e0; e < e1; ++e) {
+      run += bucket[e + 1];
+      bucket[e + 1] = run;                                   // inclusive: end of group e
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_src; i += blockDim.x) {
+    const int e = sc.target[i];
+    order[bucket[e] + atomicAdd(&cursor[e], 1)] = i;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n_elig; e += blockDim.x) {
+    const int b = bucket[e], n = bucket[e + 1] - b;
+    for (int x = 1; x < n; ++x) {                          // insertion sort of the group
+      const int v = order[b + x];
+      int y = x - 1;
+      while (y >= 0 && order[b + y] > v) {
+        order[b + y + 1] = order[b + y];
+        --y;
+      }
+      order[b + y + 1] = v;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e <= n_elig; e += blockDim.x) sc.bucket[e] = bucket[e];
+  for (int q = threadIdx.x; q < n_src; q += blockDim.x) {
+    const int o = order[q];
+    sc.order[q] = o;
+    const int pos = sc.merge[o];
     const long long k = sc.slot[pos];
     sc.src_base[q] = ((k / P) * H * P + k % P) * D;
     sc.src_cnt[q] = sc.cnt[pos];
@@ -787,10 +1014,20 @@ kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_
                                                                      c->tok_cnt + lay_slots,
                                         c->tok_shat + lay_slots, T, g.num_special_tokens, g.protect_first_frame, sc);
   ok();
-  tier_select_kernel<<<1, 1024, 0, s>>>(sc, N, n_keep_other, n_keep_other + n_merge);
-  ok();
-  tier_lists_kernel<<<1, 1024, 0, s>>>(sc, N);
-  ok();
+  if (N <= kTierSmemMax) {
+    static PerDeviceOnce attr;
+    cudaError_t ea = attr.run([] {
+      return cudaFuncSetAttribute(tier_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTierSmemMax * 5);
+    });
+    if (ea != cudaSuccess && e == cudaSuccess) e = ea;
+    tier_kernel<<<1, 1024, static_cast<size_t>(N) * 5, s>>>(sc, N, n_keep_other, n_keep_other + n_merge);
+    ok();
+  } else {
+    tier_select_kernel<<<1, 1024, 0, s>>>(sc, N, n_keep_other, n_keep_other + n_merge);
+    ok();
+    tier_lists_kernel<<<1, 1024, 0, s>>>(sc, N);
+    ok();
+  }
   check_counts_kernel<<<1, 1, 0, s>>>(sc.counts, N, n_keep, n_keep_other, n_merge, c->d_err);
   ok();
   const int HD = H * D;
@@ -810,7 +1047,18 @@ kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_
                                          &launched);
     if (r != cudaSuccess && e == cudaSuccess) e = r;
     c->launches += launched;
-    merge_group_kernel<<<1, 1024, 0, s>>>(sc, n_merge, n_keep_other, H, P, D);
+    if (n_merge + 2 * n_keep_other + 1 <= kGroupSmemInts) {
+      static PerDeviceOnce attr;
+      cudaError_t ea = attr.run([] {
+        return cudaFuncSetAttribute(merge_group_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kGroupSmemInts * 4);
+      });
+      if (ea != cudaSuccess && e == cudaSuccess) e = ea;
+      merge_group_smem_kernel<<<1, 1024, static_cast<size_t>(n_merge + 2 * n_keep_other + 1) * 4, s>>>(
+          sc, n_merge, n_keep_other, H, P, D);
+    } else {
+      merge_group_kernel<<<1, 1024, 0, s>>>(sc, n_merge, n_keep_other, H, P, D);
+    }
     ok();
     merge_apply_kernel<<<n_keep_other, 256, 0, s>>>(sc, static_cast<int>(cp.n_merge), static_cast<int>(cp.n_keep),
                                                     kp, vp, H, P, D);
@@ -825,7 +1073,7 @@ kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_
     c->last_error = "kvc_compress: page pool too small for compaction";
     return KVC_ERR_STATE;
   }
-  e = e != cudaSuccess ? e : launch_mgr_alloc(s, E, c->bitmap + static_cast<size_t>(layer) * c->bitmap_words,
+  e = e != cudaSuccess ? e : launch_mgr_alloc(s, E, layer_free_bitmap(c, layer),
                                               c->bitmap_words, c->pool_pages, n_old, n_new, -1, P,
                                               n_keep - (n_new - 1) * P, c->d_err);
   c->launches++;
@@ -833,7 +1081,7 @@ kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_
                                                               c->tok_id + lay_slots, c->tok_cnt + lay_slots,
                                                               c->tok_shat + lay_slots, H, P, D);
   ok();
-  e = e != cudaSuccess ? e : launch_mgr_remove(s, E, c->bitmap + static_cast<size_t>(layer) * c->bitmap_words,
+  e = e != cudaSuccess ? e : launch_mgr_remove(s, E, layer_free_bitmap(c, layer),
                                                n_old + n_new, 0, n_old, c->d_err);
   c->launches++;
   if (e != cudaSuccess) {
@@ -881,5 +1129,29 @@ extern "C" kvc_status kvc_last_merge(kvc_cache* c, int32_t layer, int64_t* src_h
     if (dst_host) cudaMemcpy(dst_host, sc.last_dst + static_cast<size_t>(layer) * cp.n_merge, m * 8, cudaMemcpyDeviceToHost);
   }
   if (n_out) *n_out = n;
+  return KVC_OK;
+}
+
+extern "C" kvc_status kvc_last_raw_scores(kvc_cache* c, float* s_host, int32_t capacity, int32_t* n_out) {
+  if (!c) return KVC_ERR_ARG;
+  if (n_out) *n_out = 0;
+  const int T = c->cfg.tokens_per_frame;
+  if (c->cfg.budget_tokens <= 0 || !s_host || capacity < T) {
+    c->last_error = "kvc_last_raw_scores: budget_tokens is 0, or no host array of tokens_per_frame floats";
+    return KVC_ERR_ARG;
+  }
+  if (c->hist_layers.empty() && c->hist_frame < 0) {
+    c->last_error = "kvc_last_raw_scores: nothing scored yet";
+    return KVC_ERR_STATE;
+  }
+  kvc::Scratch sc;
+  kvc::carve(c->cfg, static_cast<uint8_t*>(c->cmp_scratch), &sc);
+  cudaError_t e = cudaStreamSynchronize(c->stream);
+  if (e == cudaSuccess) e = cudaMemcpy(s_host, sc.s_raw, static_cast<size_t>(T) * sizeof(float), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) {
+    c->last_error = cudaGetErrorString(e);
+    return KVC_ERR_CUDA;
+  }
+  if (n_out) *n_out = T;
   return KVC_OK;
 }

@@ -297,13 +297,12 @@ cudaError_t launch_merge_targets(cudaStream_t s, const __nv_bfloat16* ks, const 
   *launched = 0;
   if (n_src <= 0 || n_elig <= 0) return cudaSuccess;
   if (HD % 8 != 0 || (n_elig + cs::kBN - 1) / cs::kBN > tiles_n) return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(cos_screen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(cs::kSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce attr;
+  cudaError_t ea = attr.run([] {
+    return cudaFuncSetAttribute(cos_screen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(cs::kSmemBytes));
+  });
+  if (ea != cudaSuccess) return ea;
   CUtensorMap ts, te;
   if (!encode_keys_tmap(&ts, ks, n_src, HD) || !encode_keys_tmap(&te, ke, n_elig, HD)) return cudaErrorInvalidValue;
   dim3 grid((n_elig + cs::kBN - 1) / cs::kBN, (n_src + cs::kBM - 1) / cs::kBM);

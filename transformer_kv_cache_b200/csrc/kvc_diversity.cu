@@ -8,15 +8,15 @@
 // attention kernel reads head h's pages through its own page list. The page manager's
 // kernels serve the sub-layers exactly as they serve layers.
 //
-// Scores follow the definition in fp64 with a fixed evaluation order, so the kept sets
-// match an fp64 reference bit for bit: every sum over the 64 dims (the squares of |k|,
-// the dot k_hat . mu, the squares of |mu|) is taken in 8 blocks of 8 consecutive dims,
-// ascending within a block, then the block sums ascending; k_hat = k * RN(1 / |k|) (0 for
-// a zero key); mu = the sum of k_hat over the candidates (the direction of the mean) and a
-// head's score total are both taken in blocks of 32 consecutive candidates in ascending
-// token id, ascending within a block, then the block sums ascending; score =
-// -(k_hat . mu) / |mu|; each step one IEEE operation (explicitly rounded intrinsics, no
-// contraction).
+// Scores follow the definition in fp64, each step one IEEE operation (explicitly rounded
+// intrinsics, no contraction), in the order a parallel evaluation takes: every sum over the
+// 64 dims (the squares of |k|, the dot k_hat . mu, the squares of |mu|) in 8 blocks of 8
+// consecutive dims, then the block sums; k_hat = k * RN(1 / |k|) (0 for a zero key);
+// mu = the sum of k_hat over the candidates (the direction of the mean) and a head's score
+// total in blocks of 32 consecutive candidates in ascending token id, then the block sums;
+// score = -(k_hat . mu) / |mu|. Any other correct fp64 order differs from this one only
+// within the rounding bound of these sums, so kept sets agree with an fp64 reference except
+// among candidates whose scores tie within that bound.
 #include <cuda_bf16.h>
 
 #include <climits>
@@ -556,17 +556,58 @@ cudaError_t launch_diversity_prune(cudaStream_t s, Entry* entries_layer, void* k
   int B = (n_max + kPruneCluster - 1) / kPruneCluster;
   B = (B + kCandBlock - 1) / kCandBlock * kCandBlock;
   const size_t smem = prune_layout(n_max, B, n_cand_entries).total;
-  static size_t attr = 0;
-  if (smem > attr) {
-    cudaError_t e = cudaFuncSetAttribute(diversity_prune_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attr = smem;
-  }
+  // opt in once per device for the largest layout any call can need
+  static PerDeviceOnce attr;
+  cudaError_t e = attr.run([] {
+    const size_t most = prune_layout(kPruneCluster * kPruneMaxB, kPruneMaxB, kPruneThreads).total;
+    return cudaFuncSetAttribute(diversity_prune_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(most));
+  });
+  if (e != cudaSuccess) return e;
   return launch_pdl(diversity_prune_kernel, dim3(H * kPruneCluster), dim3(kPruneThreads), smem, s,
                     entries_layer, static_cast<__nv_bfloat16*>(k_pool), static_cast<__nv_bfloat16*>(v_pool),
                     bitmap_layer, words, tok_id_layer, pool_pages, first_cand_entry, n_cand_entries, keep, P, B,
                     sums_layer, err);
+}
+
+// Layer-wise adaptive budgets ("InfiniteVGGT" explainer, Layer-wise adaptive budgets): from
+// each layer's mean diversity of its last pruning (the heads' fp64 score sums in head order
+// over H x candidates), p = softmax(mean / tau) over the layers in fp64 and
+// budget_l = floor(L * k * p_l), clamped to [1, cap] (a layer keeps at least one token and
+// at most what its pool holds); tau <= 0 gives every layer k. One warp.
+__global__ void layer_budget_kernel(const double* __restrict__ sums, const long long* __restrict__ cand, int L,
+                                    int H, double tau, int k, int cap, int32_t* __restrict__ out) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x;
+  auto mean_of = [&](int l) {
+    double tot = 0.0;
+    for (int h = 0; h < H; ++h) tot = __dadd_rn(tot, sums[static_cast<long long>(l) * H + h]);
+    return __ddiv_rn(tot, static_cast<double>(static_cast<long long>(H) * cand[l]));
+  };
+  if (tau <= 0.0) {
+    for (int l = lane; l < L; l += 32) out[l] = min(max(k, 1), cap);
+    return;
+  }
+  double zmax = -INFINITY;
+  for (int l = lane; l < L; l += 32) zmax = fmax(zmax, __ddiv_rn(mean_of(l), tau));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) zmax = fmax(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
+  // the denominator: the layers' exponentials summed in layer order by lane 0
+  double den = 0.0;
+  if (lane == 0)
+    for (int l = 0; l < L; ++l) den = __dadd_rn(den, exp(__ddiv_rn(mean_of(l), tau) - zmax));
+  den = __shfl_sync(0xffffffffu, den, 0);
+  for (int l = lane; l < L; l += 32) {
+    const double p = __ddiv_rn(exp(__ddiv_rn(mean_of(l), tau) - zmax), den);
+    const double b = floor(__dmul_rn(static_cast<double>(L) * static_cast<double>(k), p));
+    out[l] = static_cast<int32_t>(fmin(fmax(b, 1.0), static_cast<double>(cap)));
+  }
+}
+
+cudaError_t launch_layer_budgets(cudaStream_t s, const double* sums, const long long* cand, int L, int H, double tau,
+                                 int k, int cap, int32_t* out) {
+  return launch_pdl(layer_budget_kernel, dim3(1), dim3(32), 0, s, sums, cand, L, H, tau, k, cap, out);
 }
 
 }  // namespace kvc

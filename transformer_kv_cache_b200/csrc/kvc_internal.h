@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -61,6 +62,7 @@ struct LayerHost {
   int64_t mut_tokens = 0;
   int64_t cand_count = 0;         // candidates of the last pruning (per head)
   bool has_anchor = false;
+  bool bm_alt = false;            // the layer's current free bitmap is Cache::bitmap_alt
 };
 
 // Device page-table entry: x = physical page, y = owner frame (-1: compaction block),
@@ -73,6 +75,8 @@ struct Cache {
   int device = 0;
   int sm_count = 148;
   int ppf = 0;                      // pages per frame
+  int model_heads = 0;              // heads of the caller's tensors (the cache holds a range of them)
+  int head0 = 0;                    // first model head the cache holds
   int pool_pages = 0;               // pages per layer
   int bitmap_words = 0;
   size_t elem_io = 4, elem_kv = 4;  // bytes
@@ -85,6 +89,7 @@ struct Cache {
   float* v_scale = nullptr;
   Entry* entries = nullptr;         // [layers][pool_pages]
   uint32_t* bitmap = nullptr;       // [layers][bitmap_words]
+  uint32_t* bitmap_alt = nullptr;   // [layers][bitmap_words]: the other buffer of the fused append
   int* d_err = nullptr;             // [0] error word, [1] a flag nobody sets
   // compression metadata, budget mode only: [layers][pool_pages][P]
   int64_t* tok_id = nullptr;
@@ -98,7 +103,7 @@ struct Cache {
   float* v_tok = nullptr;           // dimension-adaptive FP8: [layer][page][head][P] V token scales
   float* part_o = nullptr;
   float* part_lse = nullptr;
-  int* split_cnt = nullptr;         // [H][q_tiles] attention split counters (zero between launches)
+  int* split_cnt = nullptr;         // [H][q_tiles][4] attention piece counters (zero between launches)
   size_t part_rows = 0;             // capacity in 128-row partial tiles
   // host-buffer steps: two staging slots so that one step's copies overlap another's
   // compute; uploads and downloads run on their own streams, ordered by events
@@ -127,12 +132,22 @@ struct Cache {
   bool per_head = false;
   std::vector<int32_t> layer_budget;
   double* div_sums = nullptr;       // [layers][H] fp64 score sums of the last pruning
+  long long* div_cand = nullptr;    // [layers] candidates of the last pruning (for the budgets)
+  int32_t* div_budget = nullptr;    // [layers] budgets computed on the device
 };
 
 }  // namespace kvc
 
 // The opaque handle of the C ABI is the host-side cache state.
 struct kvc_cache : public kvc::Cache {};
+
+namespace kvc {
+// The current free-page bitmap of a layer (shared pages): the fused append writes the next
+// bitmap into the layer's other buffer and switches to it.
+inline uint32_t* layer_free_bitmap(Cache* c, int layer) {
+  return (c->L[layer].bm_alt ? c->bitmap_alt : c->bitmap) + static_cast<size_t>(layer) * c->bitmap_words;
+}
+}  // namespace kvc
 
 namespace kvc {
 
@@ -171,6 +186,20 @@ cudaError_t launch_append(cudaStream_t s, int elem_bytes, const void* k, const v
 cudaError_t launch_append_layers(cudaStream_t s, int elem_bytes, const AppendBatch& in, const LayerStarts& starts,
                                  int n_layers, void* k_pool_all, void* v_pool_all, const Entry* entries_all,
                                  int pool_pages, int n_pages, int T, int H, int D, int P, int* err = nullptr);
+// Allocation and append of one frame in one launch (kvc_append.cu): for layers
+// [starts.first_layer, + n_layers), the n_pages lowest free pages of each layer's current
+// bitmap (bm_alt when the layer's bit of alt_mask is set, else bm_main; `words` words per
+// layer) are written as entries [start, start + n_pages) with the given owner, the next
+// bitmap goes to the layer's other buffer, and the frame's K/V are copied in. The caller
+// then switches each layer to its other bitmap buffer.
+bool append_alloc_fusable(int elem_bytes, int H, int D, int P);
+// src_tok_bytes: bytes between consecutive tokens of the sources (0: H * D * elem_bytes,
+// the cache holds every head); the source pointers then point at the first held head.
+cudaError_t launch_append_alloc_layers(cudaStream_t s, int elem_bytes, const AppendBatch& in,
+                                       const LayerStarts& starts, unsigned long long alt_mask, int n_layers,
+                                       void* k_pool_all, void* v_pool_all, Entry* entries_all, uint32_t* bm_main,
+                                       uint32_t* bm_alt, int words, int pool_pages, int n_pages, int T, int H, int D,
+                                       int P, int owner, int* err, long long src_tok_bytes = 0);
 cudaError_t launch_append_fp8_layers(cudaStream_t s, const AppendBatch& in, const LayerStarts& starts, int n_layers,
                                      uint8_t* k_pool_all, uint8_t* v_pool_all, float* k_scale_all,
                                      float* v_scale_all, const Entry* entries_all, int pool_pages, int n_pages, int T,
@@ -210,13 +239,51 @@ struct TcAttnArgs {
                                     // h * head_pages + phys (single-head pages)
   const float* k_chan = nullptr;    // dimension-adaptive FP8 scales (FP8 kernel), or null
   const float* v_tok = nullptr;
-  int* split_cnt = nullptr;         // [H][q_tiles] zeroed counters (bf16 kernel): the last
-                                    // split CTA of a query tile merges, no combine launch;
-                                    // the launcher uses them for up to 4 splits only
+  int q_heads = 0;                  // heads of the Q and O tensors (0: H); the kernel reads and
+  int head0 = 0;                    // writes heads [head0, head0 + H) of them (bf16 kernel)
+  int* split_cnt = nullptr;         // [H][q_tiles][4] zeroed counters (bf16 kernel): the
+                                    // piece of a unit that finishes last merges, no combine
+                                    // launch
+  bool strict_splits = false;       // bf16: fail (cudaErrorInvalidValue) rather than use fewer
+                                    // pieces when the requested split count's partials do not fit
 };
 // Returns the number of kernels launched through *launched.
 cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used, int* launched);
 int choose_splits(int units, int tiles, int slots, bool fp8);
+
+// Schedule of the bf16 tensor-core attention (kvc_attn_tc.cu): units are (head, pair of
+// 128-row query tiles); groups of q_pairs CTAs sweep R consecutive (head, 128-slot KV tile)
+// steps each; a unit's pieces (at most max_pieces) are merged in the kernel through
+// part_tiles 128-row partial tiles and [H][q_tiles][4] counters.
+struct AttnPlan {
+  int q_tiles, q_pairs, n_tiles, R, groups, grid, max_pieces;
+  size_t part_tiles;
+};
+bool plan_attn_bf16(int T, int H, int n_pages, int P, int sm_count, int kv_splits, size_t part_tiles, bool strict,
+                    AttnPlan* out);
+// Split counters the bf16 kernel needs for T query rows and H heads.
+inline size_t attn_counter_count(long long T, int H) { return static_cast<size_t>(H) * ((T + 127) / 128) * 4; }
+
+// Runs a set-up step (a kernel attribute, which applies per device) once for each device
+// it is called on, with that device current; thread-safe; a failed step is retried on the
+// next call.
+constexpr int kMaxAttrDevices = 64;
+struct PerDeviceOnce {
+  std::mutex mu;
+  bool done[kMaxAttrDevices] = {};
+  template <typename F>
+  cudaError_t run(F&& fn) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxAttrDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[dev]) return cudaSuccess;
+    e = fn();
+    if (e == cudaSuccess) done[dev] = true;
+    return e;
+  }
+};
 
 // Tensor map for a pool: rows of D elements, box of P rows.
 bool encode_pool_tmap(CUtensorMap* map, void* base, size_t rows, int D, int P, int elem_bytes, bool swizzle128);
@@ -238,6 +305,11 @@ cudaError_t launch_diversity_prune(cudaStream_t s, Entry* entries_layer, void* k
                                    uint32_t* bitmap_layer, int words, int64_t* tok_id_layer, int pool_pages,
                                    int first_cand_entry, int n_cand_entries, int keep, int H, int D, int P,
                                    double* sums_layer, int* err);
+
+// Layer-wise adaptive budgets of the rolling memory: budget_l = clamp(floor(L * k *
+// softmax(mean_l / tau)), 1, cap) from the layers' per-head score sums and candidate counts.
+cudaError_t launch_layer_budgets(cudaStream_t s, const double* sums, const long long* cand, int L, int H, double tau,
+                                 int k, int cap, int32_t* out);
 
 // Compression kernels.
 cudaError_t launch_score(cudaStream_t s, const float* residual, int T, int R, int layer_slot, int n_hist,

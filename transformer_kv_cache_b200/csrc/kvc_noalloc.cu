@@ -1,21 +1,24 @@
 // kvc_noalloc.cu -- paged frame attention for callers that cannot allocate device memory.
 //
-// kvc_attend needs split-KV scratch (partial outputs and log-sum-exps), which a cache
-// allocates once in kvc_create. Some callers cannot call cudaMalloc at all: code that runs
-// inside a CUDA-graph capture it does not own, allocator-less embedded runtimes, or
-// plug-ins whose host process forbids device allocations after start-up. For them,
-// kvc_attend_paged_noalloc runs the same tensor-core attention kernel over caller-owned
-// pools and page table, keeping its scratch in one fixed file-scope device array.
+// kvc_attend needs scratch for the KV pieces it merges (partial outputs, log-sum-exps and
+// piece counters), which a cache allocates once in kvc_create. Some callers cannot call
+// cudaMalloc at all: code that runs inside a CUDA-graph capture it does not own,
+// allocator-less embedded runtimes, or plug-ins whose host process forbids device
+// allocations after start-up. For them, kvc_attend_paged_noalloc runs the same tensor-core
+// attention kernel over caller-owned pools and page table, keeping its scratch in one fixed
+// file-scope device array.
 //
 // The array is part of the loaded module: every GPU that loads libkvc holds
 // kNoAllocScratchBytes of it until the process exits. Its device address is looked up
 // once per device (cudaGetSymbolAddress, with that device current) on the first call made
 // on that device; make that first call before any stream capture. All calls share the
-// array and it keeps the last call's contents; nothing in it needs to start at zero (every
-// partial a call reads was written by the same call). Calls whose kernels overlap on the
-// GPU (different streams, or different host threads) race on the array: serialise them.
+// array and it keeps the last call's contents: each call clears the piece counters (they
+// must start at zero) with cudaMemsetAsync on its stream; the partials need no clearing
+// (every partial a call reads was written by the same call). Calls whose kernels overlap on
+// the GPU (different streams, or different host threads) race on the array: serialise them.
 #include <cuda_bf16.h>
 
+#include <climits>
 #include <mutex>
 
 #include "kvc_internal.h"
@@ -23,13 +26,16 @@
 namespace kvc {
 namespace {
 
-// Partial tiles of 128 query rows x 64 dims (fp32) plus one log-sum-exp per row.
-constexpr size_t kNoAllocTiles = 480;
+// Partial tiles of 128 query rows x 64 dims (fp32) plus one log-sum-exp per row, and the
+// piece counters ([heads][128-row query tiles][4] ints).
+constexpr size_t kNoAllocTiles = 544;
+constexpr size_t kNoAllocCounters = 16384;
 constexpr size_t kNoAllocPartFloats = kNoAllocTiles * 128 * 64;
 constexpr size_t kNoAllocLseFloats = kNoAllocTiles * 128;
-constexpr size_t kNoAllocScratchBytes = (kNoAllocPartFloats + kNoAllocLseFloats) * sizeof(float);
+constexpr size_t kNoAllocFloats = kNoAllocPartFloats + kNoAllocLseFloats + kNoAllocCounters;
+constexpr size_t kNoAllocScratchBytes = kNoAllocFloats * sizeof(float);
 
-static __device__ __align__(256) float g_noalloc_scratch[kNoAllocPartFloats + kNoAllocLseFloats];
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocFloats];
 static_assert(sizeof(g_noalloc_scratch) == kNoAllocScratchBytes, "scratch size");
 
 constexpr int kMaxDevices = 64;
@@ -78,20 +84,26 @@ extern "C" kvc_status kvc_attend_paged_noalloc(const void* q_dev, void* o_dev, c
        reinterpret_cast<uintptr_t>(k_pool_dev) | reinterpret_cast<uintptr_t>(v_pool_dev) |
        reinterpret_cast<uintptr_t>(page_table_dev)) & 15)
     return KVC_ERR_ARG;
-  const long long q_tiles = (tokens + 127) / 128;
-  const long long units = q_tiles * num_heads;
-  const long long total_tiles = (static_cast<long long>(n_pages) * page_size + 127) / 128;
-  const long long splits = kv_splits < total_tiles ? kv_splits : total_tiles;
-  // the scratch holds one 128-row partial per (query tile, head, split)
-  if (splits > 1 && units * splits > static_cast<long long>(kNoAllocTiles)) return KVC_ERR_ARG;
-  if (pool_pages * num_heads * page_size > (1LL << 31)) return KVC_ERR_ARG;
+  // pool rows (pages x heads x slots) index the tensor maps as int: reject pools past that
+  // without forming an overflowing product
+  if (pool_pages > INT_MAX / (static_cast<long long>(num_heads) * page_size)) return KVC_ERR_ARG;
+  if (attn_counter_count(tokens, num_heads) > kNoAllocCounters) return KVC_ERR_ARG;
   float* scratch = nullptr;
   int sms = 0;
   if (scratch_for_current_device(&scratch, &sms) != cudaSuccess) return KVC_ERR_CUDA;
+  // the requested split count as the kernel runs it; one whose partials exceed the array
+  // is rejected
+  AttnPlan plan;
+  if (!plan_attn_bf16(tokens, num_heads, n_pages, page_size, sms, kv_splits, kNoAllocTiles, true, &plan))
+    return KVC_ERR_ARG;
   CUtensorMap tk, tv;
   const size_t rows = static_cast<size_t>(pool_pages) * num_heads * page_size;
   if (!encode_pool_tmap(&tk, const_cast<void*>(k_pool_dev), rows, head_dim, page_size, 2, true) ||
       !encode_pool_tmap(&tv, const_cast<void*>(v_pool_dev), rows, head_dim, page_size, 2, true))
+    return KVC_ERR_CUDA;
+  int* counters = reinterpret_cast<int*>(scratch + kNoAllocPartFloats + kNoAllocLseFloats);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(counters, 0, attn_counter_count(tokens, num_heads) * sizeof(int), s) != cudaSuccess)
     return KVC_ERR_CUDA;
   TcAttnArgs a{};
   a.q = q_dev;
@@ -104,15 +116,17 @@ extern "C" kvc_status kvc_attend_paged_noalloc(const void* q_dev, void* o_dev, c
   a.page_base = 0;
   a.pool_rows = static_cast<long long>(rows);
   a.softmax_scale = softmax_scale;
-  a.splits = static_cast<int>(splits);
+  a.splits = kv_splits;
   a.tmap_k = &tk;
   a.tmap_v = &tv;
   a.fp8 = false;
   a.part_o = scratch;
   a.part_lse = scratch + kNoAllocPartFloats;
   a.part_rows = kNoAllocTiles;
+  a.split_cnt = counters;
+  a.strict_splits = true;
   a.sm_count = sms;
   a.err = nullptr;   // no error word: a wait that gives up ends the kernel without a report
-  cudaError_t e = launch_attn_tc(static_cast<cudaStream_t>(stream), a, nullptr, nullptr);
+  cudaError_t e = launch_attn_tc(s, a, nullptr, nullptr);
   return e == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
 }

@@ -77,6 +77,12 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Wait without the abort shortcut, used only to drain a CTA's own in-flight work.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, int* err) {
+  volatile int never = 0;
+  mbar_wait_bounded(bar, parity, &never, err);
+}
+
 // ------------------------------------------------------------------ TMA (tile mode, no multicast)
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
