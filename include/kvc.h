@@ -195,7 +195,11 @@ KVC_API kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const v
  * runs fp32 FMA arithmetic. With FP8 storage the tensor cores take Q as f16: each query
  * row is first multiplied by the power of two that puts its largest magnitude in
  * [2^14, 2^15) (and its logits by the inverse), so every finite bf16 query is accepted
- * and none overflows. Errors: KVC_ERR_STATE if nothing is pending. */
+ * and none overflows. On every path the logits are formed and exponentiated in fp32:
+ * while |softmax_scale * q . k| stays far below 2^20 the softmax keeps its full
+ * resolution; logits of 2^24 and beyond (where fp32 cannot tell logits one unit apart)
+ * are outside the supported range and may give non-finite outputs.
+ * Errors: KVC_ERR_STATE if nothing is pending. */
 KVC_API kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_dev);
 
 /* The joint scale-frame phase ([GCT] Scale-Frame Phase): the first n_frames frames of a

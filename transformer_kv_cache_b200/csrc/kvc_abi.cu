@@ -822,6 +822,43 @@ kvc_status kvc_scale_phase(kvc_cache* c, int32_t layer, int32_t n_frames, const 
     return fail(c, KVC_ERR_STATE, "kvc_scale_phase: the joint phase starts an empty layer");
   // frames 0 .. n-1 appended and committed, then all n*T queries over all of them
   const size_t frame_bytes = static_cast<size_t>(g.tokens_per_frame) * c->model_heads * g.head_dim * c->elem_io;
+  const int n = c->ppf;
+  if (L.n_entries + n_frames * n > c->pool_pages)
+    return fail(c, KVC_ERR_STATE, "kvc_scale_phase: page pool full");
+  if (g.kv_dtype != KVC_FP8_E4M3 &&
+      append_alloc_fusable(static_cast<int>(c->elem_kv), g.num_heads, g.head_dim, g.page_size)) {
+    // the n frames' allocation and copy in one launch (page g of frame f is the
+    // (f * pages_per_frame + g)-th free page, as n appends in order would take it)
+    const size_t head_off = static_cast<size_t>(c->head0) * g.head_dim * c->elem_kv;
+    AppendBatch in{};
+    in.k[0] = static_cast<const uint8_t*>(k_dev) + head_off;
+    in.v[0] = static_cast<const uint8_t*>(v_dev) + head_off;
+    LayerStarts st{};
+    st.first_layer = layer;
+    st.start[0] = L.n_entries;
+    cudaError_t e = launch_append_alloc_layers(
+        c->stream, static_cast<int>(c->elem_kv), in, st, L.bm_alt ? 1ull : 0ull, 1, c->k_pool, c->v_pool,
+        c->entries, c->bitmap, c->bitmap_alt, c->bitmap_words, c->pool_pages, n, g.tokens_per_frame, g.num_heads,
+        g.head_dim, g.page_size, 0, c->d_err, static_cast<long long>(c->model_heads) * g.head_dim * c->elem_kv,
+        n_frames);
+    if (e != cudaSuccess) return cuda_fail(c, e, "append (joint phase)");
+    c->launches++;
+    L.bm_alt = !L.bm_alt;
+    for (int f = 0; f < n_frames; ++f) {
+      FrameRec r;
+      r.frame = f;
+      r.first_entry = L.n_entries;
+      r.n_entries = n;
+      L.frames.push_back(r);
+      L.n_entries += n;
+      L.tokens += g.tokens_per_frame;
+      L.appended++;
+      L.committed++;
+    }
+    L.high_water = std::max<int64_t>(L.high_water, L.n_entries);
+    L.last_frame = n_frames - 1;
+    return attend_layer(c, layer, q_dev, o_dev, n_frames * g.tokens_per_frame);
+  }
   for (int f = 0; f < n_frames; ++f) {
     kvc_status st = kvc_append_frame(c, layer, f, static_cast<const uint8_t*>(k_dev) + f * frame_bytes,
                                      static_cast<const uint8_t*>(v_dev) + f * frame_bytes, 1);

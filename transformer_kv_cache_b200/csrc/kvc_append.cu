@@ -119,7 +119,9 @@ __global__ void __launch_bounds__(256) append_bulk_kernel(AppendBatch in, LayerS
 // bitmap (the current one with the frame's pages marked used) into the layer's other
 // bitmap buffer, each K CTA writes its page-table entry, and the host switches the layer to
 // the other buffer. No CTA waits on another. A pool without enough free pages latches
-// DERR_POOL and copies nothing.
+// DERR_POOL; the CTAs whose page is missing copy nothing. Several frames of one layer (the
+// joint scale-frame phase) take consecutive ranks: page g of frame f is the
+// (f * n_pages + g)-th free page, so the result equals n single-frame appends in order.
 __device__ __forceinline__ uint32_t free_bits(const uint32_t* bm, int w, int words, int pool_pages) {
   if (w >= words) return 0u;
   uint32_t valid = 0xffffffffu;
@@ -134,7 +136,8 @@ __global__ void __launch_bounds__(256) append_alloc_bulk_kernel(AppendBatch in, 
                                                                 Entry* entries_all, uint32_t* bm_main,
                                                                 uint32_t* bm_alt, int words, int pool_pages,
                                                                 int n_pages, int T, int H, int row_bytes, int P,
-                                                                int owner, int* err, long long src_tok_bytes) {
+                                                                int owner, int* err, long long src_tok_bytes,
+                                                                int n_frames) {
   griddep_wait();
   griddep_launch_dependents();
   extern __shared__ __align__(128) uint8_t sm[];
@@ -145,9 +148,15 @@ __global__ void __launch_bounds__(256) append_alloc_bulk_kernel(AppendBatch in, 
   const int page_bytes = P * H * row_bytes;
   uint4* src_s = reinterpret_cast<uint4*>(sm);                 // [slot][head][chunk]
   uint4* dst_s = reinterpret_cast<uint4*>(sm + page_bytes);    // [head][slot][chunk]
+  // CTA (layer of the batch, frame of the batch, tensor, page of the frame); the frame's
+  // page g is the (f * n_pages + g)-th lowest free page of its layer
   const int g = blockIdx.x % n_pages;
   const int tensor = (blockIdx.x / n_pages) & 1;
-  const int bl = blockIdx.x / (2 * n_pages);
+  const int fb_idx = blockIdx.x / (2 * n_pages);
+  const int f = fb_idx % n_frames;
+  const int bl = fb_idx / n_frames;
+  const int rank = f * n_pages + g;
+  const int total_pages = n_frames * n_pages;
   const int ntok = min(P, T - g * P);
   const long long layer = starts.first_layer + bl;
   const bool on_alt = (alt_mask >> bl) & 1ull;
@@ -157,7 +166,7 @@ __global__ void __launch_bounds__(256) append_alloc_bulk_kernel(AppendBatch in, 
   // H rows when the cache holds a range of the caller's heads)
   const int tok_bytes = H * row_bytes;
   const uint8_t* src = static_cast<const uint8_t*>(tensor ? in.v[bl] : in.k[bl]) +
-                       static_cast<long long>(g) * P * src_tok_bytes;
+                       (static_cast<long long>(f) * T + static_cast<long long>(g) * P) * src_tok_bytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     abort_flag = 0;
@@ -177,7 +186,7 @@ __global__ void __launch_bounds__(256) append_alloc_bulk_kernel(AppendBatch in, 
     }
   }
   if (warp == 0) {
-    // the g-th free page: word popcounts scanned 32 words at a time
+    // the rank-th free page: word popcounts scanned 32 words at a time
     int found = 0;
     for (int w0 = 0; w0 < words; w0 += 32) {
       const uint32_t fb = free_bits(cur, w0 + lane, words, pool_pages);
@@ -189,16 +198,16 @@ __global__ void __launch_bounds__(256) append_alloc_bulk_kernel(AppendBatch in, 
         if (lane >= o) x += y;
       }
       const int before = found + x - cnt;
-      const unsigned hit = __ballot_sync(0xffffffffu, g >= before && g < found + x);
+      const unsigned hit = __ballot_sync(0xffffffffu, rank >= before && rank < found + x);
       if (hit) {
-        if (lane == __ffs(hit) - 1) s_phys = (w0 + lane) * 32 + static_cast<int>(__fns(fb, 0, g - before + 1));
+        if (lane == __ffs(hit) - 1) s_phys = (w0 + lane) * 32 + static_cast<int>(__fns(fb, 0, rank - before + 1));
         break;
       }
       found += __shfl_sync(0xffffffffu, x, 31);
     }
   }
-  if (tensor == 0 && g == 0) {
-    // the next bitmap: the n_pages lowest free pages marked used
+  if (tensor == 0 && rank == 0) {
+    // the next bitmap: the n_frames * n_pages lowest free pages marked used
     int found = 0;
     for (int w0 = 0; w0 < words; w0 += 256) {
       const int w = w0 + threadIdx.x;
@@ -220,7 +229,7 @@ __global__ void __launch_bounds__(256) append_alloc_bulk_kernel(AppendBatch in, 
       }
       int r = found + wbase + x - cnt;
       uint32_t m = fb, taken = 0;
-      while (m && r < n_pages) {
+      while (m && r < total_pages) {
         const uint32_t bit = m & (0u - m);
         taken |= bit;
         m ^= bit;
@@ -230,7 +239,7 @@ __global__ void __launch_bounds__(256) append_alloc_bulk_kernel(AppendBatch in, 
       found += total;
       __syncthreads();
     }
-    if (threadIdx.x == 0 && found < n_pages) latch_error(err, DERR_POOL);
+    if (threadIdx.x == 0 && found < total_pages) latch_error(err, DERR_POOL);
   }
   __syncthreads();
   const int phys = s_phys;
@@ -241,7 +250,7 @@ __global__ void __launch_bounds__(256) append_alloc_bulk_kernel(AppendBatch in, 
   }
   if (tensor == 0 && threadIdx.x == 0) {
     const int valid = g == n_pages - 1 ? T - (n_pages - 1) * P : P;
-    entries_all[layer * pool_pages + starts.start[bl] + g] = make_int4(phys, owner, g, valid);
+    entries_all[layer * pool_pages + starts.start[bl] + rank] = make_int4(phys, owner + f, g, valid);
   }
   uint8_t* dst = (tensor ? v_pool_all : k_pool_all) + (layer * pool_pages + phys) * static_cast<long long>(page_bytes);
   if (!mbar_wait_bounded(&bar, 0, &abort_flag, err)) return;
@@ -450,8 +459,8 @@ cudaError_t launch_append_alloc_layers(cudaStream_t s, int elem_bytes, const App
                                        const LayerStarts& starts, unsigned long long alt_mask, int n_layers,
                                        void* k_pool_all, void* v_pool_all, Entry* entries_all, uint32_t* bm_main,
                                        uint32_t* bm_alt, int words, int pool_pages, int n_pages, int T, int H, int D,
-                                       int P, int owner, int* err, long long src_tok_bytes) {
-  if (!append_alloc_fusable(elem_bytes, H, D, P)) return cudaErrorInvalidValue;
+                                       int P, int owner, int* err, long long src_tok_bytes, int n_frames) {
+  if (!append_alloc_fusable(elem_bytes, H, D, P) || n_frames < 1) return cudaErrorInvalidValue;
   if (src_tok_bytes == 0) src_tok_bytes = static_cast<long long>(H) * D * elem_bytes;
   if (src_tok_bytes % 16) return cudaErrorInvalidValue;
   static PerDeviceOnce attr;
@@ -461,10 +470,10 @@ cudaError_t launch_append_alloc_layers(cudaStream_t s, int elem_bytes, const App
   });
   if (e != cudaSuccess) return e;
   const int page_bytes = P * H * D * elem_bytes;
-  return launch_pdl(append_alloc_bulk_kernel, dim3(2 * n_layers * n_pages), dim3(256),
+  return launch_pdl(append_alloc_bulk_kernel, dim3(2 * n_layers * n_frames * n_pages), dim3(256),
                     static_cast<size_t>(2 * page_bytes), s, in, starts, alt_mask, n_layers,
                     static_cast<uint8_t*>(k_pool_all), static_cast<uint8_t*>(v_pool_all), entries_all, bm_main, bm_alt,
-                    words, pool_pages, n_pages, T, H, D * elem_bytes, P, owner, err, src_tok_bytes);
+                    words, pool_pages, n_pages, T, H, D * elem_bytes, P, owner, err, src_tok_bytes, n_frames);
 }
 
 cudaError_t launch_append(cudaStream_t s, int elem_bytes, const void* k, const void* v, void* k_pool,

@@ -195,11 +195,14 @@ cudaError_t launch_append_layers(cudaStream_t s, int elem_bytes, const AppendBat
 bool append_alloc_fusable(int elem_bytes, int H, int D, int P);
 // src_tok_bytes: bytes between consecutive tokens of the sources (0: H * D * elem_bytes,
 // the cache holds every head); the source pointers then point at the first held head.
+// n_frames > 1 (one layer's joint phase): frames owner .. owner + n_frames - 1, their
+// sources T tokens apart, entries from starts.start[b] on in frame order.
 cudaError_t launch_append_alloc_layers(cudaStream_t s, int elem_bytes, const AppendBatch& in,
                                        const LayerStarts& starts, unsigned long long alt_mask, int n_layers,
                                        void* k_pool_all, void* v_pool_all, Entry* entries_all, uint32_t* bm_main,
                                        uint32_t* bm_alt, int words, int pool_pages, int n_pages, int T, int H, int D,
-                                       int P, int owner, int* err, long long src_tok_bytes = 0);
+                                       int P, int owner, int* err, long long src_tok_bytes = 0,
+                                       int n_frames = 1);
 cudaError_t launch_append_fp8_layers(cudaStream_t s, const AppendBatch& in, const LayerStarts& starts, int n_layers,
                                      uint8_t* k_pool_all, uint8_t* v_pool_all, float* k_scale_all,
                                      float* v_scale_all, const Entry* entries_all, int pool_pages, int n_pages, int T,
