@@ -16,31 +16,36 @@
 //
 // Roles of a CTA (384 threads, one CTA per SM, all 512 TMEM columns; warpgroup 0 gives up
 // registers to the two softmax warpgroups with setmaxnreg):
-//   warp 0 (one lane)   TMA producer: the pair's two query tiles (128-byte swizzled, the
-//                       A operand of S) once per piece, then per KV tile the 8 page-head
-//                       blocks of K and of V into a 4-stage ring. Pages past the end of the
+//   warp 0 (one lane)   TMA producer: per KV tile the 8 page-head blocks of K and of V
+//                       (128-byte swizzled) into a 5-stage ring. Pages past the end of the
 //                       list are read past the end of the pool, which TMA fills with zeros.
-//   warp 1              MMA issuer (the warp waits, one elected lane issues):
-//                       S_i = Q_i K^T (tcgen05.mma kind::f16, M=128, N=128, both operands
-//                       in shared memory) into TMEM, and O'_i += P_i [V | 1] (M=128, N=80,
-//                       A = P_i read from TMEM, B = the V tile as an MN-major operand
-//                       followed by a constant block of ones), so accumulator column 64
-//                       carries the exact row sum of the same bf16 P the product used.
-//   warps 4-7, 8-11     softmax of query tile 0 and 1 (thread = query row = TMEM lane).
-//                       Per KV tile: the 128 scores from TMEM, P = 2^(s*c - m) for 96
-//                       columns on the MUFU and for 32 on the FMA pipe (a cubic in the
-//                       fraction, the integer part added to the exponent field), truncated
-//                       to bf16 pairs and written back over the first 64 columns of S.
+//   warps 1, 2          MMA issuers of query tile 0 and 1 (the warp waits, one elected lane
+//                       issues), per 64-slot half of a KV tile: S = Q K^T (tcgen05.mma
+//                       kind::f16, M=128, N=64, A = Q read from TMEM, B = the K half in
+//                       shared memory) and O' += P [V | 1] (M=128, N=80, A = P from TMEM,
+//                       B = the V half as an MN-major operand followed by a block of
+//                       ones), so column 64 of O' is the exact row sum of the bf16 P used.
+//   warps 4-7, 8-11     softmax of query tile 0 and 1 (thread = query row = TMEM lane):
+//                       first the row of Q into TMEM, then per half the 64 scores from
+//                       TMEM, P = 2^(s*c - m) for 5 of every 8 column pairs on the MUFU
+//                       and for 3 on the FMA pipe (a cubic in the fraction, the integer
+//                       part added to the exponent field), interleaved, rounded to bf16
+//                       pairs and written over the first 32 columns of the half's own S
+//                       buffer.
 //
-// P overwrites S, so S_i of the next tile is issued after the P.V product of this one; the
-// two query tiles alternate (while one tile's softmax runs, the tensor core does the other
-// tile's P.V and next S), which keeps the MUFU and the tensor core busy together.
+// TMEM per query tile (240 of 256 columns): Q (32: bf16 pairs), two S buffers (64 each;
+// half u uses buffer u & 1, and its P goes over the buffer's first 32 columns once its S is
+// in registers), O' (80). The issuer keeps S one half ahead of the softmax: after the P.V
+// product of half u it issues S of half u + 2 into the same buffer (one issuer's MMAs run
+// in order, so the product has read P before S overwrites it). A softmax warp then finds
+// the next S computed when it finishes a half, and each half costs it one wait (S ready)
+// and one arrive (P ready).
 //
 // Online softmax with lazy rescaling: the reference max m of a row only moves when a
-// tile's P would exceed 2^8 (the exact fp32 tile max, from 3-input max instructions, is
-// compared with m + 8). When a row's reference moves (the first tile of a piece, or a new
-// maximum), O' (with its row-sum column) is rescaled in TMEM; the P.V product of the
-// previous tile has completed by then because it was issued before this tile's S.
+// half's P would exceed 2^8 (the exact fp32 max of the half, from 3-input max
+// instructions, is compared with m + 8). When a row's reference moves (the first half of a
+// piece, or a new maximum), O' (with its row-sum column) is rescaled by 2^(m_old - m_new)
+// after the previous half's P.V has completed.
 //
 // Partial pages: slots past a page's valid count hold K = V = 0 (the append and compaction
 // kernels write zeros there) and their scores are set to -inf before the softmax, in the
@@ -60,27 +65,33 @@ namespace kvc {
 namespace tc {
 constexpr int kBM = 128;                      // query rows per query tile
 constexpr int kQT = 2;                        // query tiles per CTA
-constexpr int kBN = 128;                      // KV slots per tile
+constexpr int kBN = 128;                      // KV slots per TMA stage
+constexpr int kBH = 64;                       // KV slots per S tile (half a stage)
 constexpr int kHD = 64;                       // head dim (one 128-byte swizzle row)
+constexpr int kStages = 5;
 constexpr int kON = kHD + 16;                 // O' columns: O plus the row-sum block
-constexpr int kStages = 4;
 constexpr int kTileBytes = kBN * kHD * 2;     // 16 KB (K or V tile)
-constexpr int kQBytes = kBM * kHD * 2;        // 16 KB per query tile
-constexpr int kOnesBytes = kBN * kHD * 2;     // 16 KB block of bf16 ones
+constexpr int kHalfBytes = kBH * kHD * 2;     // 8 KB: rows of one half (a multiple of the 1 KB swizzle atom)
+constexpr int kOnesBytes = kHalfBytes;        // bf16 ones: the row-sum block of the B operand of P.V
 constexpr int kThreads = 384;                 // 3 warpgroups
-constexpr int kRegsLow = 48, kRegsHigh = 224;  // after the split: 128 x 48 + 256 x 224 <= 384 x 168
+constexpr int kRegsLow = 56, kRegsHigh = 224;  // after the split: 128 x 56 + 256 x 224 <= 384 x 168
 constexpr int kTmemCols = 512;
-constexpr int kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 336;
-constexpr int kPolyCols = 32;                 // columns of a tile whose 2^x runs on the FMA pipe
+// TMEM columns of query tile i, from 256 i: Q (bf16 pairs), S buffers 0 and 1 (fp32; P as
+// bf16 pairs over the first 32 columns of its buffer), O' (fp32)
+constexpr int kColQ = 0, kColS = 32, kColO = 160;
+__host__ __device__ constexpr int col_base(int i) { return 256 * i; }
 constexpr float kLog2PMax = 8.0f;             // a P above 2^8 moves the row's reference max
-constexpr size_t kSmemBytes = 1024 + kQT * kQBytes + 2 * kStages * kTileBytes + kOnesBytes + 512;
+constexpr int kPolyPer8 = 3;                  // of every 8 column pairs, the 2^x on the FMA pipe
+constexpr size_t kSmemBytes = 1024 + 2 * kStages * kTileBytes + kOnesBytes + 512;
 }  // namespace tc
 
 // ---- the FMA-pipe exponential
-// 2^x for a pair: x clamped to [-126, 127], x = n + f with n = rint(x) (the 1.5 * 2^23 shift)
+// 2^x for a pair: x clamped below at -126, x = n + f with n = rint(x) (the 1.5 * 2^23 shift)
 // and f in [-0.5, 0.5]; 2^f = 1 + f (c1 + f (c2 + f c3)), a cubic fitted for this kernel by
 // iteratively reweighted least squares on the relative error (at most 1.02e-4, against the
-// 2^-8 of the bf16 truncation P takes next); 2^n is added to the exponent field.
+// 2^-9 of the bf16 rounding P takes next); 2^n is added to the exponent field. No upper
+// clamp: the softmax only evaluates x = s*c - m <= 8 (the reference max m is at most 8
+// below any score it weights).
 __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
@@ -96,9 +107,11 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
   return r;
 }
-__device__ __forceinline__ void exp2_fma_pair(float x0, float x1, float& y0, float& y1) {
+__device__ __forceinline__ uint64_t exp2_fma_pair(uint64_t x2) {
   constexpr float kShift = 12582912.0f;       // 1.5 * 2^23
-  const uint64_t xc = pk2(fminf(fmaxf(x0, -126.f), 127.f), fminf(fmaxf(x1, -126.f), 127.f));
+  float x0, x1;
+  up2(x2, x0, x1);
+  const uint64_t xc = pk2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
   const uint64_t t = add2(xc, pk2(kShift, kShift));
   const uint64_t fr = sub2(xc, sub2(t, pk2(kShift, kShift)));
   uint64_t q = fma2(pk2(0.05500858277082443f, 0.05500858277082443f), fr,
@@ -108,37 +121,33 @@ __device__ __forceinline__ void exp2_fma_pair(float x0, float x1, float& y0, flo
   float q0, q1, t0, t1;
   up2(q, q0, q1);
   up2(t, t0, t1);
-  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+  return pk2(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+             __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
 }
 
-// One tile of P for a row: pb[i] = bf16 pair of 2^(s*c - m) for columns 2i, 2i+1 (the last
-// kPolyCols columns on the FMA pipe, the others on the MUFU). Written in three stages over
-// the score registers (exponents in place, then every 2^x, then the packing) so that all
-// of a row's MUFU instructions are independent and can issue back to back.
-__device__ __forceinline__ void tile_p(uint32_t (&s)[tc::kBN], float c, float m, uint32_t (&pb)[tc::kBN / 2]) {
+// One S tile of P for a row: pb[i] = bf16 pair of 2^(s*c - m) for columns 2i, 2i+1, rounded
+// to nearest. Of every 8 pairs the last kPoly go to the FMA pipe and the others to the
+// MUFU, and every pair is finished (exponent, packing) in one pass, so MUFU instructions
+// are spread through the row's FMA and ALU work instead of queueing behind one another.
+template <int N>
+__device__ __forceinline__ void tile_p(const uint32_t (&s)[N], float c, float m, uint32_t (&pb)[N / 2]) {
+  constexpr int kPoly = tc::kPolyPer8;
   const uint64_t c2 = pk2(c, c), nm2 = pk2(-m, -m);
 #pragma unroll
-  for (int i = 0; i < tc::kBN / 2; ++i) {
-    float x0, x1;
-    up2(fma2_pair(s[2 * i], s[2 * i + 1], c2, nm2), x0, x1);
-    s[2 * i] = __float_as_uint(x0);
-    s[2 * i + 1] = __float_as_uint(x1);
-  }
-#pragma unroll
-  for (int i = 0; i < tc::kBN / 2; ++i) {
-    float y0, y1;
-    if (2 * i >= tc::kBN - tc::kPolyCols) {
-      exp2_fma_pair(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]), y0, y1);
+  for (int i = 0; i < N / 2; ++i) {
+    const uint64_t x2 = fma2_pair(s[2 * i], s[2 * i + 1], c2, nm2);
+    uint64_t y2;
+    if ((i & 7) >= 8 - kPoly) {
+      y2 = exp2_fma_pair(x2);
     } else {
-      y0 = ex2(__uint_as_float(s[2 * i]));
-      y1 = ex2(__uint_as_float(s[2 * i + 1]));
+      float x0, x1;
+      up2(x2, x0, x1);
+      y2 = pk2(ex2(x0), ex2(x1));
     }
-    s[2 * i] = __float_as_uint(y0);
-    s[2 * i + 1] = __float_as_uint(y1);
+    float y0, y1;
+    up2(y2, y0, y1);
+    pb[i] = pack_bf16(y0, y1);
   }
-#pragma unroll
-  for (int i = 0; i < tc::kBN / 2; ++i) pb[i] = bf16x2_trunc(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]));
 }
 
 // Register split between warpgroups (every warp of a warpgroup executes the same one).
@@ -270,30 +279,34 @@ __device__ __forceinline__ void store_piece(const TcParams& p, int wg, int wq, i
 
 template <int P, bool kPerHead>
 __global__ void __launch_bounds__(tc::kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-                   const __grid_constant__ CUtensorMap tmap_v, const TcParams p) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                   const TcParams p) {
   griddep_wait();
   griddep_launch_dependents();
   using namespace tc;
-  constexpr int kPPT = kBN / P;               // pages per KV tile
+  constexpr int kPPT = kBN / P;               // pages per KV tile (TMA stage)
+  constexpr int kPPH = kBH / P;               // pages per half (S tile)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_s = smem;                                   // [2][128 rows][128 B]
-  uint8_t* k_s = q_s + kQT * kQBytes;
+  uint8_t* k_s = smem;                                   // [stage][128 rows][128 B]
   uint8_t* v_s = k_s + kStages * kTileBytes;
-  uint8_t* ones_s = v_s + kStages * kTileBytes;
+  uint8_t* ones_s = v_s + kStages * kTileBytes;          // after every V stage: a positive offset
   uint64_t* bars = reinterpret_cast<uint64_t*>(ones_s + kOnesBytes);
-  uint64_t* q_full = bars;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;
+  uint64_t* k_full = bars;
   uint64_t* v_full = k_full + kStages;
-  uint64_t* kv_empty = v_full + kStages;
-  uint64_t* s_full = kv_empty + kStages;      // [2] one per query tile
-  uint64_t* p_full = s_full + 2;              // [2]
-  uint64_t* o_full = p_full + 2;
-  uint64_t* o_free = o_full + 1;
-  uint64_t* mma_final = o_free + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 1);
+  uint64_t* kv_empty = v_full + kStages;      // both issuers done with the stage
+  // Per query tile i ([i], or [2 i + b] for S buffer b). Every wait is on a phase at most
+  // one ahead of the last one the waiter saw complete (a parity wait cannot tell two
+  // phases apart), which is why P and the piece's end have their own barriers:
+  uint64_t* q_ready = kv_empty + kStages;     // Q in TMEM (the 4 softmax warps)
+  uint64_t* s_full = q_ready + 2;             // S buffer computed
+  uint64_t* p_full = s_full + 4;              // P in S buffer b (the 4 softmax warps)
+  uint64_t* pv_done = p_full + 4;             // a P.V product complete (rescale: S of half u
+                                              // complete implies P.V of half u - 2 complete)
+  uint64_t* o_full = pv_done + 2;             // the piece's last P.V complete
+  uint64_t* o_free = o_full + 2;              // O' read by the epilogue (the 4 softmax warps)
+  uint64_t* mma_final = o_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -305,20 +318,22 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   const Sweep sweep0{min(g * R, HT), min(g * R + R, HT)};
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&kv_empty[i], kQT);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
+    for (int i = 0; i < kQT; ++i) {
+      mbar_init(&q_ready[i], 4);
+      mbar_init(&s_full[2 * i], 1);
+      mbar_init(&s_full[2 * i + 1], 1);
+      mbar_init(&p_full[2 * i], 4);
+      mbar_init(&p_full[2 * i + 1], 4);
+      mbar_init(&pv_done[i], 1);
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_free[i], 4);
+      mbar_init(&mma_final[i], 1);
     }
-    mbar_init(o_full, 1);
-    mbar_init(o_free, 8);
-    mbar_init(mma_final, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -339,22 +354,16 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     reg_dealloc<kRegsLow>();
     if (lane == 0) {
       // ------------------------------------------------------------------ TMA producer
-      tma_prefetch_desc(&tmap_q);
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_v);
       int last[kStages];
 #pragma unroll
       for (int i = 0; i < kStages; ++i) last[i] = -1;
-      int jg = 0, pc = 0;
+      int jg = 0;
       bool ok = true;
       Sweep sw = sweep0;
       int h, t0, t1;
       while (ok && next_piece(sw, n_tiles, h, t0, t1)) {
-        if (pc > 0 && !mbar_wait_bounded(q_empty, (pc - 1) & 1, abort_flag, p.err)) break;
-        mbar_arrive_expect_tx(q_full, kQT * kQBytes);
-#pragma unroll
-        for (int i = 0; i < kQT; ++i)
-          tma_load_3d(q_s + i * kQBytes, &tmap_q, q_full, 0, p.head0 + h, (2 * qp + i) * kBM);
         const long long hp = kPerHead ? static_cast<long long>(h) * p.head_pages : 0;
         const Entry* ent = kPerHead ? p.entries + hp : p.entries;
         int phys_next[kPPT];
@@ -392,10 +401,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           for (int q = 0; q < kPPT; ++q) tma_load_2d(v_s + st * kTileBytes + q * P * 128, &tmap_v, &v_full[st], 0, row[q]);
           last[st] = jg;
         }
-        ++pc;
       }
       // drain: every copy this CTA issued has landed before shared memory is released
-      if (pc > 0) mbar_wait_drain(q_full, (pc - 1) & 1, p.err);
 #pragma unroll
       for (int i = 0; i < kStages; ++i) {
         if (last[i] >= 0) {
@@ -404,200 +411,218 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
     reg_dealloc<kRegsLow>();
-    // ------------------------------------------------------------------ MMA issuer
-    const uint32_t idesc_s = idesc_f16kind(1, kBM, kBN, 0, 0);
+    // ------------------------------------------------------------------ MMA issuer of query tile i
+    // Halves are numbered globally (uu = 2 * KV tile + half); half uu uses S buffer uu & 1.
+    const int i = warp - 1;
+    const uint32_t idesc_s = idesc_f16kind(1, kBM, kBH, 0, 0);
     const uint32_t idesc_o = idesc_f16kind(1, kBM, kON, 0, 1);
-    const uint32_t tS[2] = {tmem + kColS0, tmem + kColS1};
-    const uint32_t tO[2] = {tmem + kColO0, tmem + kColO1};
-    const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
-    const uint32_t ones_addr = smem_u32(ones_s);
+    const uint32_t tb = tmem + col_base(i);
+    const uint32_t k_addr = smem_u32(k_s), v_addr = smem_u32(v_s), ones_addr = smem_u32(ones_s);
     const bool leader = elect_one();
-    auto issue_s = [&](int i, int st) {
-      const uint32_t qa = q_addr + i * kQBytes, kb = k_addr + st * kTileBytes;
+    int ub = 0, pc = 0;                           // first half of the piece; pieces done
+    // S of half uu (u: its index in the piece) into buffer uu & 1. Issued after the P.V
+    // product of half uu - 2 (which read its P from this buffer): this issuer's MMAs run in
+    // order, so that product has read P before S overwrites it.
+    auto issue_s = [&](int uu, int u) -> bool {
+      const int jj = uu >> 1, hb = uu & 1, st = jj % kStages;
+      bool w = true;
+      if (hb == 0) w = mbar_wait_bounded(&k_full[st], (jj / kStages) & 1, abort_flag, p.err);
+      if (u == 0) w = w && mbar_wait_bounded(&q_ready[i], pc & 1, abort_flag, p.err);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      if (leader) {
+        const uint32_t kb = k_addr + st * kTileBytes + hb * kHalfBytes;
 #pragma unroll
-      for (int kk = 0; kk < kHD / 16; ++kk)
-        mma_ss(tS[i], sw128_desc(qa + kk * 32, 16, 1024), sw128_desc(kb + kk * 32, 16, 1024), idesc_s, kk > 0);
-      mma_commit(&s_full[i]);
+        for (int kk = 0; kk < kHD / 16; ++kk)
+          mma_ts(tb + kColS + hb * kBH, tb + kColQ + kk * 8, sw128_desc(kb + kk * 32, 16, 1024), idesc_s,
+                 kk > 0 ? 1u : 0u);
+        mma_commit(&s_full[2 * i + hb]);
+      }
+      __syncwarp();
+      return true;
     };
-    int jg = 0, pc = 0;
+    // O' += P [V | 1] for half uu; the first half of a piece overwrites O' once the previous
+    // piece's epilogue has read it
+    auto issue_pv = [&](int uu, int u, bool last) -> bool {
+      const int jj = uu >> 1, hb = uu & 1, st = jj % kStages;
+      bool w = mbar_wait_bounded(&p_full[2 * i + hb], jj & 1, abort_flag, p.err);
+      if (hb == 0) w = w && mbar_wait_bounded(&v_full[st], (jj / kStages) & 1, abort_flag, p.err);
+      if (u == 0 && pc > 0) w = w && mbar_wait_bounded(&o_free[i], (pc - 1) & 1, abort_flag, p.err);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      if (leader) {
+        const uint32_t vb = v_addr + st * kTileBytes + hb * kHalfBytes;
+        const uint32_t lbo = ones_addr - vb;      // the N block after V: the ones
+#pragma unroll
+        for (int kk = 0; kk < kBH / 16; ++kk)
+          mma_ts(tb + kColO, tb + kColS + hb * kBH + kk * 8, sw128_desc(vb + kk * 2048, lbo, 1024), idesc_o,
+                 (u > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&pv_done[i]);
+        if (hb == 1) mma_commit(&kv_empty[st]);
+        if (last) mma_commit(&o_full[i]);
+      }
+      __syncwarp();
+      return true;
+    };
     bool ok = true;
     Sweep sw = sweep0;
     int h, t0, t1;
     while (ok && next_piece(sw, n_tiles, h, t0, t1)) {
-      const int n = t1 - t0;
-      {
-        const int st = jg % kStages;
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(q_full, pc & 1, abort_flag, p.err) &&
-                                         mbar_wait_bounded(&k_full[st], (jg / kStages) & 1, abort_flag, p.err)))
-          break;
-        tc_fence_after();
-        if (leader) {
-          issue_s(0, st);
-          issue_s(1, st);
-          if (n == 1) mma_commit(q_empty);
-        }
-        __syncwarp();
+      const int nh = 2 * (t1 - t0);
+      ok = issue_s(ub, 0) && issue_s(ub + 1, 1);
+      for (int u = 0; ok && u < nh; ++u) {
+        if (!issue_pv(ub + u, u, u + 1 == nh)) ok = false;
+        else if (u + 2 < nh && !issue_s(ub + u + 2, u + 2)) ok = false;
       }
-      for (int j = 0; j < n; ++j) {
-        const int jj = jg + j;
-        const int st = jj % kStages;
-        const uint32_t ph = (jj / kStages) & 1;
-        const int st1 = (jj + 1) % kStages;
-        const uint32_t ph1 = ((jj + 1) / kStages) & 1;
-        for (int i = 0; i < kQT; ++i) {
-          bool w = mbar_wait_bounded(&p_full[i], jj & 1, abort_flag, p.err);
-          if (i == 0) {
-            w = w && mbar_wait_bounded(&v_full[st], ph, abort_flag, p.err);
-            if (j == 0 && pc > 0) w = w && mbar_wait_bounded(o_free, (pc - 1) & 1, abort_flag, p.err);
-            if (j + 1 < n) w = w && mbar_wait_bounded(&k_full[st1], ph1, abort_flag, p.err);
-          }
-          if (!__all_sync(0xffffffffu, w)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (leader) {
-            const uint32_t vb = v_addr + st * kTileBytes;
-            const uint32_t lbo = ones_addr - vb;
-#pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk)
-              mma_ts(tO[i], tS[i] + kk * 8, sw128_desc(vb + kk * 2048, lbo, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-            if (j + 1 < n) {
-              issue_s(i, st1);
-              if (i == 1 && j + 2 == n) mma_commit(q_empty);
-            }
-          }
-          __syncwarp();
-        }
-        if (!ok) break;
-        if (leader) mma_commit(&kv_empty[st]);
-        __syncwarp();
-      }
-      if (!ok) break;
-      if (leader) mma_commit(o_full);
-      __syncwarp();
-      jg += n;
+      ub += nh;
       ++pc;
     }
-    if (leader) mma_commit(mma_final);
+    if (leader) mma_commit(&mma_final[i]);
     __syncwarp();
-    mbar_wait_drain(mma_final, 0, p.err);
+    mbar_wait_drain(&mma_final[i], 0, p.err);
   } else if (warp < 4) {
-    reg_dealloc<kRegsLow>();                       // warps 2 and 3 only give up registers
+    reg_dealloc<kRegsLow>();                       // warp 3 only gives up registers
   } else {
     reg_alloc<kRegsHigh>();
     // ------------------------------------------------------------------ softmax warps
     const int wg = (warp - 4) >> 2;               // query tile of the pair
     const int wq = warp & 3;                      // TMEM lane quadrant this warp may access
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + (wg ? kColS1 : kColS0) + lane_off;
-    const uint32_t tO = tmem + (wg ? kColO1 : kColO0) + lane_off;
+    const uint32_t tb = tmem + col_base(wg) + (static_cast<uint32_t>(wq * 32) << 16);
     const float c = p.scale_log2;
-    int jg = 0, pc = 0;
+    const int row = (2 * qp + wg) * kBM + wq * 32 + lane;
+    int ub = 0, pc = 0;
     bool ok = true;
     Sweep sw = sweep0;
     int h, t0, t1;
     while (ok && next_piece(sw, n_tiles, h, t0, t1)) {
-      const int n = t1 - t0;
+      const int nh = 2 * (t1 - t0);
       const Entry* ent = kPerHead ? p.entries + static_cast<long long>(h) * p.head_pages : p.entries;
-      float m = -INFINITY;       // reference max (log2 domain) of the row
-      int vnext[kPPT];
+      {
+        // this row of Q (zeros past the last query) into TMEM, the A operand of S; the S
+        // products of the previous piece, its only readers, have completed (their S was read)
+        uint32_t qv[32];
+        if (row < p.T) {
+          const uint4* src =
+              reinterpret_cast<const uint4*>(p.q + (static_cast<long long>(row) * p.out_heads + p.head0 + h) * kHD);
 #pragma unroll
-      for (int q = 0; q < kPPT; ++q) {
+          for (int v = 0; v < 8; ++v) {
+            const uint4 w = __ldg(src + v);
+            qv[4 * v] = w.x;
+            qv[4 * v + 1] = w.y;
+            qv[4 * v + 2] = w.z;
+            qv[4 * v + 3] = w.w;
+          }
+        } else {
+#pragma unroll
+          for (int v = 0; v < 32; ++v) qv[v] = 0u;
+        }
+        tmem_st32(tb + kColQ, qv);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_ready[wg]);
+      }
+      float m = -INFINITY;       // reference max (log2 domain) of the row
+      int vnext[kPPH];
+#pragma unroll
+      for (int q = 0; q < kPPH; ++q) {
         const int idx = t0 * kPPT + q;
         vnext[q] = idx < p.n_pages ? __ldg(&ent[idx].w) : 0;
       }
-      for (int j = 0; j < n; ++j) {
-        const int jj = jg + j;
-        int vcur[kPPT];
+      for (int u = 0; u < nh; ++u) {
+        const int uu = ub + u, hb = uu & 1, jj = uu >> 1;
+        int vcur[kPPH];
         bool partial = false;
 #pragma unroll
-        for (int q = 0; q < kPPT; ++q) {
+        for (int q = 0; q < kPPH; ++q) {
           vcur[q] = vnext[q];
           partial |= vcur[q] < P;
         }
-        if (j + 1 < n) {
+        if (u + 1 < nh) {
 #pragma unroll
-          for (int q = 0; q < kPPT; ++q) {
-            const int idx = (t0 + j + 1) * kPPT + q;
+          for (int q = 0; q < kPPH; ++q) {
+            const int idx = t0 * kPPT + (u + 1) * kPPH + q;
             vnext[q] = idx < p.n_pages ? __ldg(&ent[idx].w) : 0;
           }
         }
-        uint32_t s[kBN];
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s_full[wg], jj & 1, abort_flag, p.err))) {
+        uint32_t s[kBH];
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s_full[2 * wg + hb], jj & 1, abort_flag, p.err))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+        tmem_ld32(tb + kColS + hb * kBH, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_ld32(tb + kColS + hb * kBH + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
         tmem_ld_wait();
         if (partial) {
           // slots past a page's valid count (and pages past the list end) take no weight
 #pragma unroll
-          for (int cc = 0; cc < kBN; ++cc)
+          for (int cc = 0; cc < kBH; ++cc)
             if ((cc % P) >= vcur[cc / P]) s[cc] = __float_as_uint(-INFINITY);
         }
-        // exact fp32 tile max; the row's reference max moves when some P would exceed 2^8
-        // (or on the first tile of a piece), and O' is then rescaled by 2^(m_old - m_new):
-        // the previous tile's P.V was issued before this tile's S and has completed
-        float ta = -INFINITY, tb = -INFINITY;
+        // exact fp32 max of the half; the row's reference max moves when some P would exceed
+        // 2^8 (or on the first half of a piece); O' is then rescaled by 2^(m_old - m_new)
+        // once the previous half's P.V has completed
+        float ma = -INFINITY, mb = -INFINITY;
 #pragma unroll
-        for (int cc = 0; cc < kBN; cc += 4) {
-          ta = max3(ta, __uint_as_float(s[cc]), __uint_as_float(s[cc + 1]));
-          tb = max3(tb, __uint_as_float(s[cc + 2]), __uint_as_float(s[cc + 3]));
+        for (int cc = 0; cc < kBH; cc += 4) {
+          ma = max3(ma, __uint_as_float(s[cc]), __uint_as_float(s[cc + 1]));
+          mb = max3(mb, __uint_as_float(s[cc + 2]), __uint_as_float(s[cc + 3]));
         }
-        const float tm = fmaxf(ta, tb) * c;
-        const bool move = (j == 0) || tm > m + kLog2PMax;
+        const float tm = fmaxf(ma, mb) * c;
+        const bool move = (u == 0) || tm > m + kLog2PMax;
         if (__any_sync(0xffffffffu, move)) {
           const float m_new = move ? (tm == -INFINITY ? (m == -INFINITY ? 0.f : m) : tm) : m;
-          const bool resc = move && j > 0 && m_new != m;
+          const bool resc = move && u > 0 && m_new != m;
           if (__any_sync(0xffffffffu, resc)) {
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&pv_done[wg], (uu - 1) & 1, abort_flag, p.err))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
             const float f = resc ? ex2(m - m_new) : 1.0f;
 #pragma unroll
             for (int q4 = 0; q4 < kON / 16; ++q4) {
               uint32_t oc[16];
-              tmem_ld16(tO + q4 * 16, oc);
+              tmem_ld16(tb + kColO + q4 * 16, oc);
               tmem_ld_wait();
 #pragma unroll
               for (int d = 0; d < 16; ++d) oc[d] = __float_as_uint(__uint_as_float(oc[d]) * f);
-              tmem_st16(tO + q4 * 16, oc);
+              tmem_st16(tb + kColO + q4 * 16, oc);
             }
           }
           m = m_new;
         }
-        uint32_t pb[kBN / 2];
+        uint32_t pb[kBH / 2];
         tile_p(s, c, m, pb);
-        // P over the first 64 columns of S (tcgen05.ld/st are .sync.aligned: every branch
-        // around them is warp-uniform)
-        tmem_st32(tS + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pb[0]));
-        tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pb[32]));
+        // P over the first 32 columns of this half's S buffer, whose S is in registers; the
+        // buffer is not written again before this P's product has read it (tcgen05.ld/st are
+        // .sync.aligned: every branch around them is warp-uniform)
+        tmem_st32(tb + kColS + hb * kBH, pb);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[wg]);
+        if (lane == 0) mbar_arrive(&p_full[2 * wg + hb]);
       }
       if (!ok) break;
       // ---------------------------------------------------------------- epilogue
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(o_full, pc & 1, abort_flag, p.err))) {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&o_full[wg], pc & 1, abort_flag, p.err))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t o0[32], o1[32], ls[16];
-      tmem_ld32(tO, o0);
-      tmem_ld32(tO + 32, o1);
-      tmem_ld16(tO + 64, ls);
+      uint32_t o0[32], o1[32];
+      tmem_ld32(tb + kColO, o0);
+      tmem_ld32(tb + kColO + 32, o1);
+      const uint32_t lsum = tmem_ld1(tb + kColO + 64);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(o_free);
-      store_piece(p, wg, wq, lane, h, qp, g, o0, o1, __uint_as_float(ls[0]), m);
-      jg += n;
+      if (lane == 0) mbar_arrive(&o_free[wg]);
+      store_piece(p, wg, wq, lane, h, qp, g, o0, o1, __uint_as_float(lsum), m);
+      ub += nh;
       ++pc;
     }
   }
@@ -769,9 +794,9 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   if (a.P != 16 || (a.fp8 && a.head_pages)) return cudaErrorInvalidValue;
   const int qh = a.q_heads > 0 ? a.q_heads : a.H;
   if (a.head0 < 0 || a.head0 + a.H > qh || (a.fp8 && qh != a.H)) return cudaErrorInvalidValue;
-  CUtensorMap tq;
-  if (!encode_q_tmap(&tq, a.q, a.T, qh)) return cudaErrorInvalidValue;
   if (!a.fp8) {
+    // the softmax warps read Q rows with 16-byte loads
+    if (reinterpret_cast<uintptr_t>(a.q) & 15) return cudaErrorInvalidValue;
     static PerDeviceOnce attr;
     cudaError_t e = attr.run([] {
       cudaError_t r = cudaFuncSetAttribute(attn_tc_kernel<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -809,10 +834,10 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
     prm.out_heads = qh;
     prm.head0 = a.head0;
     if (a.head_pages)
-      e = launch_pdl(attn_tc_kernel<16, true>, dim3(pl.grid), dim3(tc::kThreads), tc::kSmemBytes, s, tq, *a.tmap_k,
+      e = launch_pdl(attn_tc_kernel<16, true>, dim3(pl.grid), dim3(tc::kThreads), tc::kSmemBytes, s, *a.tmap_k,
                      *a.tmap_v, prm);
     else
-      e = launch_pdl(attn_tc_kernel<16, false>, dim3(pl.grid), dim3(tc::kThreads), tc::kSmemBytes, s, tq, *a.tmap_k,
+      e = launch_pdl(attn_tc_kernel<16, false>, dim3(pl.grid), dim3(tc::kThreads), tc::kSmemBytes, s, *a.tmap_k,
                      *a.tmap_v, prm);
     if (e != cudaSuccess) return e;
     if (launched) *launched = 1;
@@ -821,6 +846,8 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   }
   // FP8 storage: one CTA per SM takes two 128-row query tiles of a head and a range of
   // 64-slot KV tiles; more than one split goes through the combine kernel
+  CUtensorMap tq;
+  if (!encode_q_tmap(&tq, a.q, a.T, qh)) return cudaErrorInvalidValue;
   const int q_tiles = (a.T + 127) / 128;
   const int total_tiles = (a.n_pages * a.P + 63) / 64;
   const int units = ((q_tiles + 1) / 2) * a.H;
