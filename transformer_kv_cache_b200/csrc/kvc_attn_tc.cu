@@ -150,6 +150,21 @@ __device__ __forceinline__ void tile_p(const uint32_t (&s)[N], float c, float m,
   }
 }
 
+// Largest of a row's 64 scores as a tree of 3-input max instructions (depth 4), so the
+// row's maximum does not wait on one long dependent chain.
+__device__ __forceinline__ float row_max64(const uint32_t (&s)[tc::kBH]) {
+  float a[22];
+#pragma unroll
+  for (int i = 0; i < 21; ++i)
+    a[i] = max3(__uint_as_float(s[3 * i]), __uint_as_float(s[3 * i + 1]), __uint_as_float(s[3 * i + 2]));
+  a[21] = __uint_as_float(s[63]);
+  float b[8];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) b[i] = max3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+  b[7] = a[21];
+  return max3(max3(b[0], b[1], b[2]), max3(b[3], b[4], b[5]), fmaxf(b[6], b[7]));
+}
+
 // Register split between warpgroups (every warp of a warpgroup executes the same one).
 template <int N>
 __device__ __forceinline__ void reg_dealloc() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
@@ -460,11 +475,16 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           mma_ts(tb + kColO, tb + kColS + hb * kBH + kk * 8, sw128_desc(vb + kk * 2048, lbo, 1024), idesc_o,
                  (u > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&pv_done[i]);
-        if (hb == 1) mma_commit(&kv_empty[st]);
         if (last) mma_commit(&o_full[i]);
       }
       __syncwarp();
       return true;
+    };
+    // the stage of half uu's KV tile is released after its second half's P.V (committed
+    // after the next S, off the path from P.V to that S)
+    auto release = [&](int uu) {
+      if (leader && (uu & 1)) mma_commit(&kv_empty[(uu >> 1) % kStages]);
+      __syncwarp();
     };
     bool ok = true;
     Sweep sw = sweep0;
@@ -475,6 +495,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       for (int u = 0; ok && u < nh; ++u) {
         if (!issue_pv(ub + u, u, u + 1 == nh)) ok = false;
         else if (u + 2 < nh && !issue_s(ub + u + 2, u + 2)) ok = false;
+        else release(ub + u);
       }
       ub += nh;
       ++pc;
@@ -565,13 +586,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         // exact fp32 max of the half; the row's reference max moves when some P would exceed
         // 2^8 (or on the first half of a piece); O' is then rescaled by 2^(m_old - m_new)
         // once the previous half's P.V has completed
-        float ma = -INFINITY, mb = -INFINITY;
-#pragma unroll
-        for (int cc = 0; cc < kBH; cc += 4) {
-          ma = max3(ma, __uint_as_float(s[cc]), __uint_as_float(s[cc + 1]));
-          mb = max3(mb, __uint_as_float(s[cc + 2]), __uint_as_float(s[cc + 3]));
-        }
-        const float tm = fmaxf(ma, mb) * c;
+        const float tm = row_max64(s) * c;
         const bool move = (u == 0) || tm > m + kLog2PMax;
         if (__any_sync(0xffffffffu, move)) {
           const float m_new = move ? (tm == -INFINITY ? (m == -INFINITY ? 0.f : m) : tm) : m;
