@@ -179,6 +179,18 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ clocks during the timed region
 
+def sync_polling(stream) -> None:
+    """Wait for the stream by polling an event with short sleeps, so the clock sampler's
+    thread keeps running while the GPU works (a blocking synchronize can hold the
+    interpreter for the whole wait)."""
+    import torch
+    done = torch.cuda.Event()
+    done.record(stream)
+    while not done.query():
+        time.sleep(0.0002)
+    stream.synchronize()
+
+
 class ClockSampler:
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting", 0x10: "sync_boost"}
@@ -357,7 +369,7 @@ def run_ours(args):
                 kvc.kvc_attend(h, 0, q, out)
                 ev[i][2].record(stream)
             e1.record(stream)
-            stream.synchronize()
+            sync_polling(stream)
         barrier()
         elapsed_ms = e0.elapsed_time(e1)
         log(f"timed region {elapsed_ms:.2f} ms")
@@ -573,7 +585,7 @@ def run_workload(args):
                 key, fired = step(t, evs[i])
                 keys += key
                 fires += fired
-            stream.synchronize()
+            sync_polling(stream)
         _, info1 = kvc.kvc_page_table(h, 0)
         assert info1["device_error"] == 0
         kvc.kvc_destroy(h)
@@ -673,7 +685,7 @@ def run_joint(args):
         with ClockSampler(local) as clk:
             for i in range(steps):
                 step(evs[i])
-            stream.synchronize()
+            sync_polling(stream)
         _, info = kvc.kvc_page_table(h, 0)
         assert info["device_error"] == 0
         kvc.kvc_destroy(h)
