@@ -330,7 +330,7 @@ def run_ours(args):
     T, H, D, P = wl.tokens_per_frame, wl.num_heads, wl.head_dim, wl.page_size
     S, W = wl.scale_frames, wl.window_frames
     fill, warm, steps = S + W, args.warmup, args.steps
-    n_frames = fill + warm + steps
+    n_frames = fill + warm + steps + 3              # + the end-to-end leg's 3 warm-up steps
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(device=dev)
     peaks, peak_kind = load_peaks()
@@ -425,13 +425,28 @@ def run_ours(args):
         log("end-to-end leg")
         kvc.kvc_reset(h)
         n_e2e = min(args.e2e_steps, steps)
+        e2e_warm = 3
         with torch.cuda.stream(stream):
             for t in range(fill):
                 q, k, v = frames[t]
                 kvc.kvc_append_frame(h, 0, t, k, v, True)
                 kvc.kvc_attend(h, 0, q, out)
-            host = [tuple(x.cpu().pin_memory() for x in frames[fill + i]) for i in range(n_e2e)]
+            host = [tuple(x.cpu().pin_memory() for x in frames[fill + i]) for i in range(e2e_warm + n_e2e)]
             oh = torch.empty((T, H, D), dtype=torch.bfloat16).pin_memory()
+            # untimed warm-up: every pinned buffer crosses the bus once (its first transfer is
+            # slower), and e2e_warm host-buffer steps run before the timed ones
+            scratch = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+            for x in host:
+                for y in x:
+                    scratch.copy_(y, non_blocking=True)
+            oh.copy_(scratch, non_blocking=True)
+            for i in range(e2e_warm):
+                qh, kh, vh = host[i]
+                kvc.kvc_step_host_async(h, 0, fill + i, True, qh, kh, vh, oh)
+            kvc.kvc_synchronize(h)
+            stream.synchronize()
+            host = host[e2e_warm:]
+            fill += e2e_warm
             barrier()
             f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             f0.record(stream)
@@ -448,7 +463,8 @@ def run_ours(args):
         e_ms = max_over_ranks(f0.elapsed_time(f1), world, dev)
         fb = T * H * D * 2
         e2e = {"value": job_rate(world, n_e2e, e_ms), "unit": UNIT, "h2d_bytes_per_step": 3 * fb,
-               "d2h_bytes_per_step": fb, "steps": n_e2e, "api": "kvc_step_host_async + kvc_synchronize"}
+               "d2h_bytes_per_step": fb, "steps": n_e2e, "warmup": e2e_warm,
+               "api": "kvc_step_host_async + kvc_synchronize"}
     kvc.kvc_destroy(h)
 
     if rank == 0:
