@@ -558,7 +558,7 @@ def run_workload(args):
         st = FrameStream(wl, seed=2000, device=dev)
         pool = [[st.frame(l, t) for t in range(distinct)] for l in range(L)]
         res = [[st.residual(l, t) for t in range(distinct)] for l in range(L)] if budget else None
-        out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+        outs = [torch.empty((T, H, D), dtype=torch.bfloat16, device=dev) for _ in range(L)]
         h = kvc.kvc_create(kvc.config_from_workload(wl, kv_splits=args.kv_splits), stream)
 
         def step(t, ev=None):
@@ -574,12 +574,10 @@ def run_workload(args):
                         kvc.kvc_prune(h, l)
                     fired = L
                 if ev: ev[2].record(stream)
-                for l in range(L):
-                    kvc.kvc_attend(h, l, pool[l][i][0], out)
+                kvc.kvc_attend_all(h, [pool[l][i][0] for l in range(L)], outs)
                 if ev: ev[3].record(stream)
                 return key, fired
-            for l in range(L):
-                kvc.kvc_attend(h, l, pool[l][i][0], out)
+            kvc.kvc_attend_all(h, [pool[l][i][0] for l in range(L)], outs)
             if ev: ev[2].record(stream)
             if budget:
                 for l in range(L):

@@ -202,6 +202,17 @@ KVC_API kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const v
  * Errors: KVC_ERR_STATE if nothing is pending. */
 KVC_API kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_dev);
 
+/* kvc_attend on every layer, in layer order: q_devs[l] and o_devs[l] are layer l's
+ * [T, H, D] queries and outputs (each 16-byte aligned), and every layer must have a
+ * pending frame. The results, page tables and counters are those of the per-layer
+ * calls. With bf16 storage on the tensor cores, when every layer is small (fewer than 16
+ * (head, 128-slot KV tile) steps per group of CTAs, as in the rolling memory), the layers'
+ * attention runs in one launch per 32 layers (after the rolling memory's pruning of every
+ * layer); otherwise the call is the per-layer loop.
+ * Errors: KVC_ERR_ARG (NULL or misaligned pointers), KVC_ERR_STATE (a layer without a
+ * pending frame; nothing is attended then). */
+KVC_API kvc_status kvc_attend_all(kvc_cache* c, const void* const* q_devs, void* const* o_devs);
+
 /* The joint scale-frame phase ([GCT] Scale-Frame Phase): the first n_frames frames of a
  * stream, processed together with bidirectional attention. q_dev, k_dev, v_dev and o_dev
  * are [n_frames * T, H, D] (frame-major, io dtype). Frames 0 .. n_frames-1 are appended
@@ -370,10 +381,14 @@ KVC_API int32_t kvc_version(void);
  * valid_tokens must hold zeros in both K and V, as kvc_append_frame writes them). head_dim must be 64 and page_size 16; kv_splits >= 1 splits
  * the KV sequence across CTAs. Enqueued on `stream`; nothing is allocated or freed.
  *
- * Split partials live in one file-scope device array of 480 partial tiles (128 query
- * rows x 64 dims fp32 + one log-sum-exp per row, 15.97 MB) that every GPU loading the
- * library holds until the process exits. Calls with (ceil(tokens/128) * num_heads *
- * effective splits) > 480 and kv_splits > 1 are rejected with KVC_ERR_ARG. The first
+ * Split partials live in one file-scope device array of 544 partial tiles (128 query
+ * rows x 64 dims fp32 + one log-sum-exp per row) and 16,384 counters (18.17 MB in all)
+ * that every GPU loading the library holds until the process exits. With kv_splits = s
+ * the kernel runs G = ceil(num_heads * n / R) groups of Q = ceil(ceil(tokens / 128) / 2)
+ * CTAs, n = ceil(n_pages / 8) KV tiles and R = ceil(n / s); when a head's tiles fall into
+ * more than one group, the call needs 4 * G * Q partial tiles, and calls needing more
+ * than 544 (or more than 16,384 counters: num_heads * ceil(tokens / 128) * 4) are
+ * rejected with KVC_ERR_ARG. The first
  * call on a device looks the array's device address up (cudaGetSymbolAddress); make
  * that first call before any stream capture. All calls share the array: calls whose
  * kernels overlap on the GPU race on it. Nothing in it needs to start at zero. A wait in

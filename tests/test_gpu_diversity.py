@@ -24,6 +24,7 @@ def kvc():
 
 
 def run_rolling(kvc, wl, frames, rows=None, budgets_at=None, check_ids=True, seed=11, prune_first=False,
+                attend_all=False,
                 append_all=False, adapt_at=None):
     dev = torch.device("cuda")
     L, H, D, T = wl.num_layers, wl.num_heads, wl.head_dim, wl.tokens_per_frame
@@ -58,14 +59,20 @@ def run_rolling(kvc, wl, frames, rows=None, budgets_at=None, check_ids=True, see
             qkv = [st.frame(l, t) for l in range(L)]
             if append_all:                              # every layer's frame in one call
                 kvc.kvc_append_frame_all(h, t, [x[1] for x in qkv], [x[2] for x in qkv], True)
+            if attend_all:                              # every layer pruned and attended in one call
+                outs = [torch.empty_like(o) for _ in range(L)]
+                kvc.kvc_attend_all(h, [x[0] for x in qkv], outs)
             for l in range(L):
                 q, k, v = qkv[l]
                 if not append_all:
                     kvc.kvc_append_frame(h, l, t, k, v, True)
-                if prune_first and t > 0:
-                    kvc.kvc_prune(h, l)                 # the pruning step on its own; twice prunes once
-                    kvc.kvc_prune(h, l)
-                kvc.kvc_attend(h, l, q, o)
+                if attend_all:
+                    o = outs[l]
+                else:
+                    if prune_first and t > 0:
+                        kvc.kvc_prune(h, l)             # the pruning step on its own; twice prunes once
+                        kvc.kvc_prune(h, l)
+                    kvc.kvc_attend(h, l, q, o)
                 orc.append(l, t, np64(k), np64(v))
                 orc.prune(l)
                 if t >= 1:
@@ -119,6 +126,15 @@ def test_rolling_memory_append_all_layers(kvc):
     wl = WORKLOADS["vggt_infinite_12l"].replace(num_layers=3, tokens_per_frame=150, num_heads=4,
                                                 diversity_budget=200)
     run_rolling(kvc, wl, 6, append_all=True)
+
+
+def test_rolling_memory_attend_all_layers(kvc):
+    """kvc_attend_all: every layer pruned, then every layer attended in one launch (the
+    layers are small), with kept sets, layer averages and outputs checked per layer; the
+    layers' budgets differ, so their page counts do too."""
+    wl = WORKLOADS["vggt_infinite_12l"].replace(num_layers=3, tokens_per_frame=150, num_heads=4,
+                                                diversity_budget=200)
+    run_rolling(kvc, wl, 7, append_all=True, attend_all=True, budgets_at={3: [200, 60, 131]})
 
 
 def test_layer_budgets_between_frames(kvc):

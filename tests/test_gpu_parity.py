@@ -41,6 +41,41 @@ def test_bf16_tensor_core_small(kvc, T, H, W, S, frames, splits):
     run_parity(kvc, wl, frames, kv_splits=splits, check_pages=True)
 
 
+def test_attend_all_layers_one_launch(kvc):
+    """kvc_attend_all on a 4-layer window cache whose layers are small (one launch for every
+    layer): every layer's output against the oracle, page tables equal, keyframe interval
+    2 past the window, and the library's launch count shows one attention launch per frame."""
+    wl = WORKLOADS["vggt_24layer_k4"].replace(num_layers=4, tokens_per_frame=200, num_heads=4, window_frames=3,
+                                              scale_frames=1, keyframe_interval=2, num_special_tokens=5)
+    L, T, H, D = wl.num_layers, wl.tokens_per_frame, wl.num_heads, wl.head_dim
+    dev = torch.device("cuda")
+    h = kvc.kvc_create(kvc.config_from_workload(wl))
+    try:
+        st = FrameStream(wl, seed=19, device=dev)
+        orc = StreamOracle(OracleConfig.from_workload(wl))
+        outs = [torch.empty((T, H, D), dtype=torch.bfloat16, device=dev) for _ in range(L)]
+        for t in range(11):
+            key = keyframe_schedule(t, wl.scale_frames, wl.keyframe_interval)
+            qkv = [st.frame(l, t) for l in range(L)]
+            kvc.kvc_append_frame_all(h, t, [x[1] for x in qkv], [x[2] for x in qkv], key)
+            _, before = kvc.kvc_page_table(h, 0)
+            kvc.kvc_attend_all(h, [x[0] for x in qkv], outs)
+            _, after = kvc.kvc_page_table(h, 0)
+            attn = after["kernel_launches"] - before["kernel_launches"]
+            assert attn <= 1 + L, (t, attn)              # one attention launch, at most one eviction per layer
+            torch.cuda.synchronize()
+            for l in range(L):
+                q, k, v = qkv[l]
+                orc.append(l, t, np64(k), np64(v), key)
+                ref = orc.attend(l, np64(q))
+                compare_out(np64(outs[l]), ref, "bf16", f"frame {t} layer {l}")
+                pt, info = kvc.kvc_page_table(h, l)
+                assert np.array_equal(pt, orc.page_table(l)), f"page table differs at frame {t} layer {l}"
+                assert info["device_error"] == 0
+    finally:
+        kvc.kvc_destroy(h)
+
+
 def test_bf16_keyframes_two_layers(kvc):
     wl = WORKLOADS["vggt_24layer_k4"].replace(num_layers=2, tokens_per_frame=200, num_heads=4,
                                                window_frames=4, scale_frames=2)

@@ -25,6 +25,7 @@ STATUS = ["KVC_OK", "KVC_ERR_ARG", "KVC_ERR_OOM", "KVC_ERR_CUDA", "KVC_ERR_STATE
 
 # every symbol include/kvc.h declares
 EXPORTS = ["kvc_create", "kvc_destroy", "kvc_set_stream", "kvc_reset", "kvc_append_frame", "kvc_attend",
+           "kvc_attend_all",
            "kvc_compress", "kvc_page_table", "kvc_token_meta", "kvc_last_merge", "kvc_export_pages",
            "kvc_step_host", "kvc_synchronize", "kvc_last_error", "kvc_status_string", "kvc_version",
            "kvc_debug_fail_allocs", "kvc_debug_bounded_wait", "kvc_attend_paged_noalloc", "kvc_append_frame_all",
@@ -78,6 +79,7 @@ def _load():
         "kvc_append_frame": ([vp, i32, i32, vp, vp, i32], i32),
         "kvc_attend": ([vp, i32, vp, vp], i32),
         "kvc_append_frame_all": ([vp, i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32], i32),
+        "kvc_attend_all": ([vp, ctypes.POINTER(vp), ctypes.POINTER(vp)], i32),
         "kvc_compress": ([vp, i32, vp, i32p], i32),
         "kvc_page_table": ([vp, i32, i32p, i32, i32p, ctypes.POINTER(kvc_info)], i32),
         "kvc_token_meta": ([vp, i32, i64p, i32p, fp, i32, i32p], i32),
@@ -214,6 +216,14 @@ def kvc_append_frame_all(handle, frame_idx: int, ks, vs, is_keyframe: bool = Tru
 
 def kvc_attend(handle, layer: int, q, o) -> None:
     _check(handle, _lib.kvc_attend(handle, layer, _ptr(q), _ptr(o)))
+
+
+def kvc_attend_all(handle, qs, os) -> None:
+    """qs, os: per-layer device tensors (or pointers), one per layer of the cache."""
+    n = len(qs)
+    qa = (ctypes.c_void_p * n)(*[_ptr(q) for q in qs])
+    oa = (ctypes.c_void_p * n)(*[_ptr(o) for o in os])
+    _check(handle, _lib.kvc_attend_all(handle, qa, oa))
 
 
 def kvc_compress(handle, layer: int, residual) -> bool:

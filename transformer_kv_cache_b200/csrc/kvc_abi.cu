@@ -36,10 +36,10 @@ cudaError_t dev_alloc_t(T** p, size_t bytes) {
 }
 
 // Piece counters of the attention kernel, for the largest query count (a frame, or the
-// joint phase's S frames).
+// joint phase's S frames) and the heads of the most layers one launch takes.
 size_t split_cnt_count(const kvc_config& g) {
   const long long rows = static_cast<long long>(g.tokens_per_frame) * std::max(1, g.scale_frames);
-  return attn_counter_count(rows, g.num_heads);
+  return attn_counter_count(rows, g.num_heads * std::min(g.num_layers, kMaxAttnLayers));
 }
 
 void free_all(kvc_cache* c) {
@@ -291,7 +291,9 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   const size_t frame_bytes = static_cast<size_t>(T) * H * D * c->elem_io;
   c->tc_path = g.io_dtype == KVC_BF16 && (g.kv_dtype == KVC_BF16 || g.kv_dtype == KVC_FP8_E4M3) && D == 64 && P == 16;
   const int q_tiles = (T + 127) / 128;
-  c->part_rows = static_cast<size_t>(q_tiles) * H * 16;
+  // partial tiles: 16 per (query tile, head), and at least 8 per SM (a split unit's pieces
+  // take 4 per CTA of the groups that cut it)
+  c->part_rows = std::max(static_cast<size_t>(q_tiles) * H * 16, static_cast<size_t>(8) * std::max(1, c->sm_count));
 
   cudaError_t e = cudaSuccess;
   auto A = [&](cudaError_t r) {
@@ -765,6 +767,8 @@ kvc_status attend_layer(kvc_cache* c, int layer, const void* q_dev, void* o_dev,
   return KVC_OK;
 }
 
+kvc_status commit_layer(kvc_cache* c, int layer);
+
 kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_dev) {
   if (!c) return KVC_ERR_ARG;
   if (!valid_layer(c, layer) || !q_dev || !o_dev) return fail(c, KVC_ERR_ARG, "kvc_attend: bad layer or pointer");
@@ -773,11 +777,17 @@ kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_de
   LayerHost& L = c->L[layer];
   if (!L.has_pending) return fail(c, KVC_ERR_STATE, "kvc_attend: no frame pending on this layer");
   if (c->per_head) return div_attend(c, layer, q_dev, o_dev);
+  kvc_status ast = attend_layer(c, layer, q_dev, o_dev, c->cfg.tokens_per_frame);
+  if (ast != KVC_OK) return ast;
+  return commit_layer(c, layer);
+}
+
+// After a layer's attention: commit the pending frame and evict past the window, or
+// release a skipped frame.
+kvc_status commit_layer(kvc_cache* c, int layer) {
   const kvc_config& g = c->cfg;
   const int T = g.tokens_per_frame;
-  kvc_status ast = attend_layer(c, layer, q_dev, o_dev, T);
-  if (ast != KVC_OK) return ast;
-  // commit / evict, or release the skipped frame
+  LayerHost& L = c->L[layer];
   if (L.pending_key) {
     L.frames.push_back(L.pending);
     L.tokens += T;
@@ -802,6 +812,100 @@ kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_de
     L.skipped++;
   }
   L.has_pending = false;
+  return KVC_OK;
+}
+
+// Every layer's pending frame attended, as kvc_attend on each layer in order. On the bf16
+// tensor-core path, layers too small to fill the GPU alone (fewer than
+// kLayerBatchStepsPerGroup (head, KV tile) steps per CTA group) go through one launch
+// per kMaxAttnLayers layers; the commits follow, layer by layer.
+kvc_status kvc_attend_all(kvc_cache* c, const void* const* q_devs, void* const* o_devs) {
+  if (!c) return KVC_ERR_ARG;
+  const kvc_config& g = c->cfg;
+  if (!q_devs || !o_devs) return fail(c, KVC_ERR_ARG, "kvc_attend_all: NULL pointer array");
+  for (int l = 0; l < g.num_layers; ++l) {
+    if (!q_devs[l] || !o_devs[l] ||
+        ((reinterpret_cast<uintptr_t>(q_devs[l]) | reinterpret_cast<uintptr_t>(o_devs[l])) & 15))
+      return fail(c, KVC_ERR_ARG, "kvc_attend_all: Q and O must be non-null and 16-byte aligned");
+    if (!c->L[l].has_pending) return fail(c, KVC_ERR_STATE, "kvc_attend_all: a layer has no pending frame");
+  }
+  bool batch = c->tc_path && g.kv_dtype != KVC_FP8_E4M3 && g.num_layers > 1;
+  if (batch) {
+    if (c->per_head) {
+      // the pruning comes first: the page counts the attention sees are the pruned ones
+      for (int l = 0; l < g.num_layers; ++l) {
+        kvc_status st = div_prune(c, l);
+        if (st != KVC_OK) return st;
+      }
+    }
+    const int q_pairs = ((g.tokens_per_frame + 127) / 128 + 1) / 2;
+    const long long groups = std::max(1, c->sm_count / q_pairs);
+    for (int l = 0; l < g.num_layers && batch; ++l) {
+      const long long steps = static_cast<long long>(g.num_heads) * ((c->L[l].n_entries * g.page_size + 127) / 128);
+      if (steps >= kLayerBatchStepsPerGroup * groups) batch = false;
+    }
+  }
+  if (!batch) {
+    for (int l = 0; l < g.num_layers; ++l) {
+      kvc_status st = kvc_attend(c, l, q_devs[l], o_devs[l]);
+      if (st != KVC_OK) return st;
+    }
+    return KVC_OK;
+  }
+  const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads;
+  TcAttnArgs a{};
+  a.T = T;
+  a.H = H;
+  a.P = P;
+  a.pool_rows = static_cast<long long>(g.num_layers) * c->pool_pages * H * P;
+  a.softmax_scale = g.softmax_scale;
+  a.splits = g.kv_splits;
+  a.tmap_k = &c->tmap_k[0];
+  a.tmap_v = &c->tmap_v[0];
+  a.fp8 = false;
+  a.q_heads = c->model_heads;
+  a.head0 = c->head0;
+  a.part_o = c->part_o;
+  a.part_lse = c->part_lse;
+  a.part_rows = c->part_rows;
+  a.split_cnt = c->split_cnt;
+  a.sm_count = c->sm_count;
+  a.err = c->d_err;
+  a.head_pages = c->per_head ? c->pool_pages : 0;
+  for (int l0 = 0; l0 < g.num_layers; l0 += kMaxAttnLayers) {
+    const int n = std::min(kMaxAttnLayers, g.num_layers - l0);
+    LayerAttn la[kMaxAttnLayers];
+    for (int b = 0; b < n; ++b) {
+      const int l = l0 + b;
+      la[b] = LayerAttn{};
+      la[b].q = q_devs[l];
+      la[b].o = o_devs[l];
+      la[b].n_pages = c->L[l].n_entries;
+      if (c->per_head) {
+        const size_t sub0 = static_cast<size_t>(l) * H * c->pool_pages;
+        la[b].entries = c->entries + sub0;
+        la[b].page_base = static_cast<long long>(sub0);
+      } else {
+        la[b].entries = layer_entries(c, l);
+        la[b].page_base = static_cast<long long>(l) * c->pool_pages;
+      }
+    }
+    int launched = 0;
+    cudaError_t e = launch_attn_tc_layers(c->stream, a, la, n, &launched);
+    c->launches += launched;
+    if (e != cudaSuccess) return cuda_fail(c, e, "attention launch (layers)");
+  }
+  for (int l = 0; l < g.num_layers; ++l) {
+    LayerHost& L = c->L[l];
+    if (c->per_head) {
+      L.has_pending = false;
+      L.committed++;
+      L.tokens = static_cast<int64_t>(T) + L.mut_tokens;
+    } else {
+      kvc_status st = commit_layer(c, l);
+      if (st != KVC_OK) return st;
+    }
+  }
   return KVC_OK;
 }
 

@@ -171,39 +171,50 @@ __device__ __forceinline__ void reg_dealloc() { asm volatile("setmaxnreg.dec.syn
 template <int N>
 __device__ __forceinline__ void reg_alloc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
 
-// The schedule of one CTA: group g sweeps [g*R, min((g+1)*R, H*n_tiles)) of the flattened
-// (head, KV tile) sequence for query-tile pair qp. next_piece() cuts the range at head
-// boundaries.
+// The schedule of one CTA: group g sweeps [g*R, min((g+1)*R, steps)) of the flattened
+// (layer, head, KV tile) sequence (layer l's steps start at lt.l[l].pos0) for query-tile
+// pair qp. next_piece() cuts the range at head (and so layer) boundaries.
 struct Sweep {
-  int pos, end;
+  int pos, end, l;
 };
-__device__ __forceinline__ bool next_piece(Sweep& sw, int n_tiles, int& h, int& t0, int& t1) {
+__device__ __forceinline__ bool next_piece(Sweep& sw, const AttnLayers& lt, int H, int& l, int& h, int& t0,
+                                           int& t1) {
   if (sw.pos >= sw.end) return false;
-  h = sw.pos / n_tiles;
-  t0 = sw.pos - h * n_tiles;
-  t1 = min(n_tiles, t0 + (sw.end - sw.pos));
+  while (sw.l + 1 < lt.n && sw.pos >= lt.l[sw.l + 1].pos0) ++sw.l;
+  const int nt = lt.l[sw.l].n_tiles;
+  const int rel = sw.pos - lt.l[sw.l].pos0;
+  l = sw.l;
+  h = rel / nt;
+  t0 = rel - h * nt;
+  t1 = min(nt, t0 + (sw.end - sw.pos));
   sw.pos += t1 - t0;
   return true;
 }
 
 // Epilogue of one warp's 32 query rows of a piece. Single-piece units store bf16 O
 // directly; otherwise every piece stores its normalised partial and log2-sum-exp, counts
-// itself on the warp's counter, and the piece that counts last merges:
+// itself on the warp's counter, and the piece that counts last merges. Only a group's
+// first and last piece can belong to a unit of several pieces (the pieces between them are
+// whole heads), so a partial lives in the slot of (its group, first or last piece of the
+// group): a piece that starts where its group starts takes the first slot. The merge is
 // O = sum_k 2^(lse_k - M) O_k / sum_k 2^(lse_k - M), M the largest lse, over the unit's
 // pieces in order (its own from registers, the others through L2). Only warp-level
 // synchronisation is used, so a warp that gave up on a wait cannot hold another here.
-__device__ __forceinline__ void store_piece(const TcParams& p, int wg, int wq, int lane, int h, int qp, int g,
-                                            const uint32_t (&o0)[32], const uint32_t (&o1)[32], float l, float m) {
+__device__ __forceinline__ void store_piece(const TcParams& p, const LayerAttn& la, int lay, int wg, int wq, int lane,
+                                            int h, int qp, int g, const uint32_t (&o0)[32], const uint32_t (&o1)[32],
+                                            float l, float m) {
   using namespace tc;
   const int r = wq * 32 + lane;
   const int qtile = 2 * qp + wg;
   const int row = qtile * kBM + r;
   const float inv = 1.f / l;
-  const int n_tiles = p.total_tiles, R = p.tiles_per_split;
-  const int g_first = (h * n_tiles) / R;
-  const int g_last = (h * n_tiles + n_tiles - 1) / R;
+  const int n_tiles = la.n_tiles, R = p.tiles_per_split;
+  const int g_first = (la.pos0 + h * n_tiles) / R;
+  const int g_last = (la.pos0 + h * n_tiles + n_tiles - 1) / R;
   const int npieces = g_last - g_first + 1;
-  uint4* out = reinterpret_cast<uint4*>(p.out + (static_cast<long long>(row) * p.out_heads + p.head0 + h) * kHD);
+  const int hh = lay * p.H + h;                 // the unit's head among all layers' heads
+  uint4* out = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(la.o) +
+                                        (static_cast<long long>(row) * p.out_heads + p.head0 + h) * kHD);
   if (npieces == 1) {
     if (row < p.T) {
 #pragma unroll
@@ -220,8 +231,12 @@ __device__ __forceinline__ void store_piece(const TcParams& p, int wg, int wq, i
     return;
   }
   if (qtile >= p.q_tiles) return;           // the pair's second tile is past the queries
-  const int unit = h * p.q_pairs + qp;
-  auto slot_row = [&](int k) { return (static_cast<long long>(unit) * p.splits + k) * (kQT * kBM) + wg * kBM + r; };
+  // piece k of the unit is in group g_first + k; only the first can start inside its group
+  const bool starts_inside = la.pos0 + h * n_tiles > g_first * R;
+  auto slot_row = [&](int k) {
+    const long long slot = 2LL * (g_first + k) + (k == 0 && starts_inside ? 1 : 0);
+    return (slot * p.q_pairs + qp) * (kQT * kBM) + wg * kBM + r;
+  };
   const int me = g - g_first;
   const float lse_me = m + __log2f(l);
   {
@@ -239,7 +254,7 @@ __device__ __forceinline__ void store_piece(const TcParams& p, int wg, int wq, i
   // threadfence-then-count: each partial is visible before its count
   __threadfence();
   __syncwarp();
-  const int cidx = ((h * p.q_tiles + qtile) << 2) + wq;
+  const int cidx = ((hh * p.q_tiles + qtile) << 2) + wq;
   int last = 0;
   if (lane == 0) last = atomicAdd(&p.split_cnt[cidx], 1) == npieces - 1;
   last = __shfl_sync(0xffffffffu, last, 0);
@@ -295,7 +310,7 @@ __device__ __forceinline__ void store_piece(const TcParams& p, int wg, int wq, i
 template <int P, bool kPerHead>
 __global__ void __launch_bounds__(tc::kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
-                   const TcParams p) {
+                   const TcParams p, const __grid_constant__ AttnLayers lt) {
   griddep_wait();
   griddep_launch_dependents();
   using namespace tc;
@@ -327,10 +342,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qp = blockIdx.x % p.q_pairs;
   const int g = blockIdx.x / p.q_pairs;
-  const int n_tiles = p.total_tiles;
-  const int HT = p.H * n_tiles;
+  const int HT = p.total_tiles;                 // steps of all layers
   const int R = p.tiles_per_split;
-  const Sweep sweep0{min(g * R, HT), min(g * R + R, HT)};
+  const Sweep sweep0{min(g * R, HT), min(g * R + R, HT), 0};
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -377,15 +391,18 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       int jg = 0;
       bool ok = true;
       Sweep sw = sweep0;
-      int h, t0, t1;
-      while (ok && next_piece(sw, n_tiles, h, t0, t1)) {
+      int lay, h, t0, t1;
+      while (ok && next_piece(sw, lt, p.H, lay, h, t0, t1)) {
+        const LayerAttn& la = lt.l[lay];
         const long long hp = kPerHead ? static_cast<long long>(h) * p.head_pages : 0;
-        const Entry* ent = kPerHead ? p.entries + hp : p.entries;
+        const Entry* ent = kPerHead ? la.entries + hp : la.entries;
+        const int n_pages = la.n_pages;
+        const long long page_base = la.page_base;
         int phys_next[kPPT];
 #pragma unroll
         for (int q = 0; q < kPPT; ++q) {
           const int idx = t0 * kPPT + q;
-          phys_next[q] = idx < p.n_pages ? __ldg(&ent[idx].x) : -1;
+          phys_next[q] = idx < n_pages ? __ldg(&ent[idx].x) : -1;
         }
         for (int t = t0; t < t1; ++t, ++jg) {
           const int st = jg % kStages;
@@ -393,15 +410,15 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 #pragma unroll
           for (int q = 0; q < kPPT; ++q) {
             if (kPerHead)
-              row[q] = phys_next[q] >= 0 ? static_cast<int>((p.page_base + hp + phys_next[q]) * P) : p.pool_rows;
+              row[q] = phys_next[q] >= 0 ? static_cast<int>((page_base + hp + phys_next[q]) * P) : p.pool_rows;
             else
-              row[q] = phys_next[q] >= 0 ? static_cast<int>(((p.page_base + phys_next[q]) * p.H + h) * P) : p.pool_rows;
+              row[q] = phys_next[q] >= 0 ? static_cast<int>(((page_base + phys_next[q]) * p.H + h) * P) : p.pool_rows;
           }
           if (t + 1 < t1) {
 #pragma unroll
             for (int q = 0; q < kPPT; ++q) {
               const int idx = (t + 1) * kPPT + q;
-              phys_next[q] = idx < p.n_pages ? __ldg(&ent[idx].x) : -1;
+              phys_next[q] = idx < n_pages ? __ldg(&ent[idx].x) : -1;
             }
           }
           if (jg >= kStages && !mbar_wait_bounded(&kv_empty[st], ((jg / kStages) - 1) & 1, abort_flag, p.err)) {
@@ -488,8 +505,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     };
     bool ok = true;
     Sweep sw = sweep0;
-    int h, t0, t1;
-    while (ok && next_piece(sw, n_tiles, h, t0, t1)) {
+    int lay, h, t0, t1;
+    while (ok && next_piece(sw, lt, p.H, lay, h, t0, t1)) {
       const int nh = 2 * (t1 - t0);
       ok = issue_s(ub, 0) && issue_s(ub + 1, 1);
       for (int u = 0; ok && u < nh; ++u) {
@@ -516,17 +533,20 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     int ub = 0, pc = 0;
     bool ok = true;
     Sweep sw = sweep0;
-    int h, t0, t1;
-    while (ok && next_piece(sw, n_tiles, h, t0, t1)) {
+    int lay, h, t0, t1;
+    while (ok && next_piece(sw, lt, p.H, lay, h, t0, t1)) {
       const int nh = 2 * (t1 - t0);
-      const Entry* ent = kPerHead ? p.entries + static_cast<long long>(h) * p.head_pages : p.entries;
+      const LayerAttn& la = lt.l[lay];
+      const Entry* ent = kPerHead ? la.entries + static_cast<long long>(h) * p.head_pages : la.entries;
+      const int n_pages = la.n_pages;
       {
         // this row of Q (zeros past the last query) into TMEM, the A operand of S; the S
         // products of the previous piece, its only readers, have completed (their S was read)
         uint32_t qv[32];
         if (row < p.T) {
           const uint4* src =
-              reinterpret_cast<const uint4*>(p.q + (static_cast<long long>(row) * p.out_heads + p.head0 + h) * kHD);
+              reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(la.q) +
+                                             (static_cast<long long>(row) * p.out_heads + p.head0 + h) * kHD);
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
             const uint4 w = __ldg(src + v);
@@ -550,7 +570,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 #pragma unroll
       for (int q = 0; q < kPPH; ++q) {
         const int idx = t0 * kPPT + q;
-        vnext[q] = idx < p.n_pages ? __ldg(&ent[idx].w) : 0;
+        vnext[q] = idx < n_pages ? __ldg(&ent[idx].w) : 0;
       }
       for (int u = 0; u < nh; ++u) {
         const int uu = ub + u, hb = uu & 1, jj = uu >> 1;
@@ -565,7 +585,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 #pragma unroll
           for (int q = 0; q < kPPH; ++q) {
             const int idx = t0 * kPPT + (u + 1) * kPPH + q;
-            vnext[q] = idx < p.n_pages ? __ldg(&ent[idx].w) : 0;
+            vnext[q] = idx < n_pages ? __ldg(&ent[idx].w) : 0;
           }
         }
         uint32_t s[kBH];
@@ -636,7 +656,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_free[wg]);
-      store_piece(p, wg, wq, lane, h, qp, g, o0, o1, __uint_as_float(lsum), m);
+      store_piece(p, la, lay, wg, wq, lane, h, qp, g, o0, o1, __uint_as_float(lsum), m);
       ub += nh;
       ++pc;
     }
@@ -759,37 +779,47 @@ int choose_splits(int units, int tiles, int slots, bool fp8) {
   return 1;
 }
 
-// Schedule of the bf16 kernel. R = KV tiles per group; groups of q_pairs CTAs. Automatic:
-// as many groups as fill the SMs (one CTA each); with kv_splits = s > 0, about s pieces per
-// head. If the partial scratch (part_tiles 128-row tiles) cannot hold every unit's pieces,
-// R grows until it can (R a multiple of the head's tiles leaves one piece per unit), unless
-// `strict`, in which case a split count that does not fit fails.
-bool plan_attn_bf16(int T, int H, int n_pages, int P, int sm_count, int kv_splits, size_t part_tiles, bool strict,
-                    AttnPlan* out) {
-  if (T < 1 || H < 1 || n_pages < 1 || P < 1 || sm_count < 1) return false;
+// Schedule of the bf16 kernel over one or more layers. R = steps per group; groups of
+// q_pairs CTAs. Automatic: as many groups as fill the SMs (one CTA each); with
+// kv_splits = s > 0, about s pieces per head of the largest layer. Split units need
+// 2 x groups x q_pairs x 2 partial tiles (a group's first and last piece); when more than
+// part_tiles, R doubles (fewer groups) until they fit, unless `strict`, in which case the
+// plan fails.
+bool plan_attn_bf16(int T, int H, const int* n_pages, int n_layers, int P, int sm_count, int kv_splits,
+                    size_t part_tiles, bool strict, AttnPlan* out, int* n_tiles, int* pos0) {
+  if (T < 1 || H < 1 || n_layers < 1 || P < 1 || sm_count < 1) return false;
   AttnPlan a{};
   a.q_tiles = (T + tc::kBM - 1) / tc::kBM;
   a.q_pairs = (a.q_tiles + 1) / 2;
-  a.n_tiles = static_cast<int>((static_cast<long long>(n_pages) * P + tc::kBN - 1) / tc::kBN);
-  const long long HT = static_cast<long long>(H) * a.n_tiles;
+  long long steps = 0;
+  int max_nt = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    if (n_pages[l] < 1) return false;
+    n_tiles[l] = static_cast<int>((static_cast<long long>(n_pages[l]) * P + tc::kBN - 1) / tc::kBN);
+    pos0[l] = static_cast<int>(steps);
+    steps += static_cast<long long>(H) * n_tiles[l];
+    max_nt = std::max(max_nt, n_tiles[l]);
+    if (steps > (1LL << 30)) return false;
+  }
+  a.steps = steps;
   long long R;
   if (kv_splits > 0) {
-    R = (a.n_tiles + kv_splits - 1) / kv_splits;
+    R = (max_nt + kv_splits - 1) / kv_splits;
   } else {
     const long long groups = std::max(1, sm_count / a.q_pairs);
-    R = (HT + groups - 1) / groups;
+    R = (steps + groups - 1) / groups;
   }
   if (R < 1) R = 1;
   for (;;) {
-    const long long groups = (HT + R - 1) / R;
+    const long long groups = (steps + R - 1) / R;
     int max_pieces = 1;
-    for (int h = 0; h < H; ++h) {
-      const long long gf = (static_cast<long long>(h) * a.n_tiles) / R;
-      const long long gl = (static_cast<long long>(h) * a.n_tiles + a.n_tiles - 1) / R;
-      max_pieces = std::max(max_pieces, static_cast<int>(gl - gf + 1));
-    }
-    const long long need = max_pieces > 1 ? static_cast<long long>(H) * a.q_pairs * max_pieces * tc::kQT : 0;
-    if (need <= static_cast<long long>(part_tiles) || R % a.n_tiles == 0 || strict) {
+    for (int l = 0; l < n_layers; ++l)
+      for (int h = 0; h < H; ++h) {
+        const long long s0 = pos0[l] + static_cast<long long>(h) * n_tiles[l];
+        max_pieces = std::max(max_pieces, static_cast<int>((s0 + n_tiles[l] - 1) / R - s0 / R + 1));
+      }
+    const long long need = max_pieces > 1 ? 2 * groups * a.q_pairs * tc::kQT : 0;
+    if (need <= static_cast<long long>(part_tiles) || strict) {
       if (need > static_cast<long long>(part_tiles)) return false;
       a.R = static_cast<int>(R);
       a.groups = static_cast<int>(groups);
@@ -799,9 +829,80 @@ bool plan_attn_bf16(int T, int H, int n_pages, int P, int sm_count, int kv_split
       *out = a;
       return true;
     }
-    // grow R to the next multiple of the head's tiles, or double it below that
-    R = R * 2 >= a.n_tiles ? ((R / a.n_tiles) + 1) * a.n_tiles : R * 2;
+    R *= 2;
   }
+}
+
+namespace {
+cudaError_t launch_bf16_layers(cudaStream_t s, const TcAttnArgs& a, const LayerAttn* layers, int n,
+                               int* splits_used, int* launched) {
+  if (n < 1 || n > kMaxAttnLayers) return cudaErrorInvalidValue;
+  const int qh = a.q_heads > 0 ? a.q_heads : a.H;
+  static PerDeviceOnce attr;
+  cudaError_t e = attr.run([] {
+    cudaError_t r = cudaFuncSetAttribute(attn_tc_kernel<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(tc::kSmemBytes));
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(attn_tc_kernel<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(tc::kSmemBytes));
+    return r;
+  });
+  if (e != cudaSuccess) return e;
+  AttnLayers lt{};
+  lt.n = n;
+  int np[kMaxAttnLayers], nt[kMaxAttnLayers], p0[kMaxAttnLayers];
+  for (int l = 0; l < n; ++l) {
+    // the softmax warps read Q rows and write O rows with 16-byte accesses
+    if ((reinterpret_cast<uintptr_t>(layers[l].q) | reinterpret_cast<uintptr_t>(layers[l].o)) & 15)
+      return cudaErrorInvalidValue;
+    np[l] = layers[l].n_pages;
+  }
+  AttnPlan pl;
+  if (!plan_attn_bf16(a.T, a.H, np, n, a.P, a.sm_count, a.splits, a.part_rows, a.strict_splits, &pl, nt, p0))
+    return cudaErrorInvalidValue;
+  if (pl.max_pieces > 1 && !a.split_cnt) return cudaErrorInvalidValue;
+  for (int l = 0; l < n; ++l) {
+    lt.l[l] = layers[l];
+    lt.l[l].n_tiles = nt[l];
+    lt.l[l].pos0 = p0[l];
+  }
+  TcParams prm{};
+  prm.T = a.T;
+  prm.H = a.H;
+  prm.q_tiles = pl.q_tiles;
+  prm.q_pairs = pl.q_pairs;
+  prm.splits = pl.max_pieces;
+  prm.tiles_per_split = pl.R;
+  prm.total_tiles = static_cast<int>(pl.steps);
+  prm.pool_rows = static_cast<int>(a.pool_rows);
+  prm.scale_log2 = static_cast<float>(static_cast<double>(a.softmax_scale) * 1.4426950408889634);
+  prm.part_o = a.part_o;
+  prm.part_lse = a.part_lse;
+  prm.err = a.err;
+  prm.head_pages = a.head_pages;
+  prm.split_cnt = a.split_cnt;
+  prm.out_heads = qh;
+  prm.head0 = a.head0;
+  if (a.head_pages)
+    e = launch_pdl(attn_tc_kernel<16, true>, dim3(pl.grid), dim3(tc::kThreads), tc::kSmemBytes, s, *a.tmap_k,
+                   *a.tmap_v, prm, lt);
+  else
+    e = launch_pdl(attn_tc_kernel<16, false>, dim3(pl.grid), dim3(tc::kThreads), tc::kSmemBytes, s, *a.tmap_k,
+                   *a.tmap_v, prm, lt);
+  if (e != cudaSuccess) return e;
+  if (launched) *launched = 1;
+  if (splits_used) *splits_used = pl.max_pieces;
+  return cudaSuccess;
+}
+}  // namespace
+
+cudaError_t launch_attn_tc_layers(cudaStream_t s, const TcAttnArgs& base, const LayerAttn* layers, int n,
+                                  int* launched) {
+  if (launched) *launched = 0;
+  if (base.P != 16 || base.fp8) return cudaErrorInvalidValue;
+  const int qh = base.q_heads > 0 ? base.q_heads : base.H;
+  if (base.head0 < 0 || base.head0 + base.H > qh) return cudaErrorInvalidValue;
+  return launch_bf16_layers(s, base, layers, n, nullptr, launched);
 }
 
 cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used, int* launched) {
@@ -810,54 +911,13 @@ cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used
   const int qh = a.q_heads > 0 ? a.q_heads : a.H;
   if (a.head0 < 0 || a.head0 + a.H > qh || (a.fp8 && qh != a.H)) return cudaErrorInvalidValue;
   if (!a.fp8) {
-    // the softmax warps read Q rows with 16-byte loads
-    if (reinterpret_cast<uintptr_t>(a.q) & 15) return cudaErrorInvalidValue;
-    static PerDeviceOnce attr;
-    cudaError_t e = attr.run([] {
-      cudaError_t r = cudaFuncSetAttribute(attn_tc_kernel<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(tc::kSmemBytes));
-      if (r == cudaSuccess)
-        r = cudaFuncSetAttribute(attn_tc_kernel<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(tc::kSmemBytes));
-      return r;
-    });
-    if (e != cudaSuccess) return e;
-    AttnPlan pl;
-    if (!plan_attn_bf16(a.T, a.H, a.n_pages, a.P, a.sm_count, a.splits, a.part_rows, a.strict_splits, &pl))
-      return cudaErrorInvalidValue;
-    if (pl.max_pieces > 1 && !a.split_cnt) return cudaErrorInvalidValue;
-    TcParams prm{};
-    prm.q = static_cast<const __nv_bfloat16*>(a.q);
-    prm.entries = a.entries;
-    prm.n_pages = a.n_pages;
-    prm.T = a.T;
-    prm.H = a.H;
-    prm.q_tiles = pl.q_tiles;
-    prm.q_pairs = pl.q_pairs;
-    prm.splits = pl.max_pieces;
-    prm.tiles_per_split = pl.R;
-    prm.total_tiles = pl.n_tiles;
-    prm.page_base = a.page_base;
-    prm.pool_rows = static_cast<int>(a.pool_rows);
-    prm.scale_log2 = static_cast<float>(static_cast<double>(a.softmax_scale) * 1.4426950408889634);
-    prm.out = static_cast<__nv_bfloat16*>(a.o);
-    prm.part_o = a.part_o;
-    prm.part_lse = a.part_lse;
-    prm.err = a.err;
-    prm.head_pages = a.head_pages;
-    prm.split_cnt = a.split_cnt;
-    prm.out_heads = qh;
-    prm.head0 = a.head0;
-    if (a.head_pages)
-      e = launch_pdl(attn_tc_kernel<16, true>, dim3(pl.grid), dim3(tc::kThreads), tc::kSmemBytes, s, *a.tmap_k,
-                     *a.tmap_v, prm);
-    else
-      e = launch_pdl(attn_tc_kernel<16, false>, dim3(pl.grid), dim3(tc::kThreads), tc::kSmemBytes, s, *a.tmap_k,
-                     *a.tmap_v, prm);
-    if (e != cudaSuccess) return e;
-    if (launched) *launched = 1;
-    if (splits_used) *splits_used = pl.max_pieces;
-    return cudaSuccess;
+    LayerAttn one{};
+    one.q = a.q;
+    one.o = a.o;
+    one.entries = a.entries;
+    one.page_base = a.page_base;
+    one.n_pages = a.n_pages;
+    return launch_bf16_layers(s, a, &one, 1, splits_used, launched);
   }
   // FP8 storage: one CTA per SM takes two 128-row query tiles of a head and a range of
   // 64-slot KV tiles; more than one split goes through the combine kernel

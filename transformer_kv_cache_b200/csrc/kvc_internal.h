@@ -252,18 +252,46 @@ struct TcAttnArgs {
 };
 // Returns the number of kernels launched through *launched.
 cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used, int* launched);
+
+// Several layers in one launch of the bf16 tensor-core kernel: base carries what the layers
+// share (T, H, P, the pool tensor maps, scratch, counters for n x H heads, head_pages); each
+// layer its queries, outputs, page list and first pool page. At most kMaxAttnLayers layers.
+constexpr int kMaxAttnLayers = 32;
+struct LayerAttn {
+  const void* q;
+  void* o;
+  const Entry* entries;
+  long long page_base;
+  int n_pages;
+  int n_tiles;                      // set by the launcher
+  int pos0;                         // first step of the layer in the flattened sweep (launcher)
+  int pad;
+};
+struct AttnLayers {
+  int n;
+  int pad;
+  LayerAttn l[kMaxAttnLayers];
+};
+cudaError_t launch_attn_tc_layers(cudaStream_t s, const TcAttnArgs& base, const LayerAttn* layers, int n,
+                                  int* launched);
 int choose_splits(int units, int tiles, int slots, bool fp8);
 
-// Schedule of the bf16 tensor-core attention (kvc_attn_tc.cu): units are (head, pair of
-// 128-row query tiles); groups of q_pairs CTAs sweep R consecutive (head, 128-slot KV tile)
-// steps each; a unit's pieces (at most max_pieces) are merged in the kernel through
-// part_tiles 128-row partial tiles and [H][q_tiles][4] counters.
+// Schedule of the bf16 tensor-core attention (kvc_attn_tc.cu): units are (layer, head,
+// pair of 128-row query tiles); groups of q_pairs CTAs sweep R consecutive (layer, head,
+// 128-slot KV tile) steps each; a unit's pieces (at most max_pieces) are merged in the
+// kernel through part_tiles 128-row partial tiles and [layers x H][q_tiles][4] counters.
+// n_pages[l] are the layers' page counts (per head for per-head page lists); n_tiles[l]
+// and pos0[l] (the layer's first step) are written for each layer.
 struct AttnPlan {
-  int q_tiles, q_pairs, n_tiles, R, groups, grid, max_pieces;
+  int q_tiles, q_pairs, R, groups, grid, max_pieces;
+  long long steps;                  // layers x H x their KV tiles
   size_t part_tiles;
 };
-bool plan_attn_bf16(int T, int H, int n_pages, int P, int sm_count, int kv_splits, size_t part_tiles, bool strict,
-                    AttnPlan* out);
+bool plan_attn_bf16(int T, int H, const int* n_pages, int n_layers, int P, int sm_count, int kv_splits,
+                    size_t part_tiles, bool strict, AttnPlan* out, int* n_tiles, int* pos0);
+// Steps per CTA group below which a layer is too small to fill the GPU on its own and
+// several layers are better attended in one launch.
+constexpr int kLayerBatchStepsPerGroup = 16;
 // Split counters the bf16 kernel needs for T query rows and H heads.
 inline size_t attn_counter_count(long long T, int H) { return static_cast<size_t>(H) * ((T + 127) / 128) * 4; }
 

@@ -94,7 +94,9 @@ extern "C" kvc_status kvc_attend_paged_noalloc(const void* q_dev, void* o_dev, c
   // the requested split count as the kernel runs it; one whose partials exceed the array
   // is rejected
   AttnPlan plan;
-  if (!plan_attn_bf16(tokens, num_heads, n_pages, page_size, sms, kv_splits, kNoAllocTiles, true, &plan))
+  int n_tiles = 0, pos0 = 0;
+  if (!plan_attn_bf16(tokens, num_heads, &n_pages, 1, page_size, sms, kv_splits, kNoAllocTiles, true, &plan,
+                      &n_tiles, &pos0))
     return KVC_ERR_ARG;
   CUtensorMap tk, tv;
   const size_t rows = static_cast<size_t>(pool_pages) * num_heads * page_size;
