@@ -570,8 +570,7 @@ def run_workload(args):
             fired = 0
             if rolling:                               # prune every layer, then attend every layer
                 if t > 0:
-                    for l in range(L):
-                        kvc.kvc_prune(h, l)
+                    kvc.kvc_prune_all(h)
                     fired = L
                 if ev: ev[2].record(stream)
                 kvc.kvc_attend_all(h, [pool[l][i][0] for l in range(L)], outs)

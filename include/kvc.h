@@ -343,6 +343,11 @@ KVC_API kvc_status kvc_adapt_layer_budgets(kvc_cache* c, double tau, int32_t k_a
  * no frame pending); calling it twice prunes once. */
 KVC_API kvc_status kvc_prune(kvc_cache* c, int32_t layer);
 
+/* kvc_prune on every layer that has a pending frame, in one launch per run of up to 32
+ * consecutive such layers (the layers' candidate sets and budgets may differ); layers
+ * without a pending frame are left alone. Errors: KVC_ERR_STATE (not a rolling cache). */
+KVC_API kvc_status kvc_prune_all(kvc_cache* c);
+
 /* Mean diversity score of the layer's last pruning over all heads' candidates (fp64:
  * per head the scores summed in blocks of 32 consecutive candidates in ascending token
  * id, then the block sums in order; then the heads in order, divided by H * candidates).

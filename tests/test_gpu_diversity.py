@@ -60,6 +60,9 @@ def run_rolling(kvc, wl, frames, rows=None, budgets_at=None, check_ids=True, see
             if append_all:                              # every layer's frame in one call
                 kvc.kvc_append_frame_all(h, t, [x[1] for x in qkv], [x[2] for x in qkv], True)
             if attend_all:                              # every layer pruned and attended in one call
+                if prune_first and t > 0:
+                    kvc.kvc_prune_all(h)                # the pruning of every layer on its own; twice prunes once
+                    kvc.kvc_prune_all(h)
                 outs = [torch.empty_like(o) for _ in range(L)]
                 kvc.kvc_attend_all(h, [x[0] for x in qkv], outs)
             for l in range(L):
@@ -129,12 +132,14 @@ def test_rolling_memory_append_all_layers(kvc):
 
 
 def test_rolling_memory_attend_all_layers(kvc):
-    """kvc_attend_all: every layer pruned, then every layer attended in one launch (the
-    layers are small), with kept sets, layer averages and outputs checked per layer; the
-    layers' budgets differ, so their page counts do too."""
+    """kvc_attend_all: every layer pruned (one launch), then every layer attended (one
+    launch; the layers are small), with kept sets, layer averages and outputs checked per
+    layer; the layers' budgets differ, so their page counts do too. Then kvc_prune_all
+    before kvc_attend_all."""
     wl = WORKLOADS["vggt_infinite_12l"].replace(num_layers=3, tokens_per_frame=150, num_heads=4,
                                                 diversity_budget=200)
     run_rolling(kvc, wl, 7, append_all=True, attend_all=True, budgets_at={3: [200, 60, 131]})
+    run_rolling(kvc, wl, 5, append_all=True, attend_all=True, prune_first=True)
 
 
 def test_layer_budgets_between_frames(kvc):

@@ -25,7 +25,7 @@ STATUS = ["KVC_OK", "KVC_ERR_ARG", "KVC_ERR_OOM", "KVC_ERR_CUDA", "KVC_ERR_STATE
 
 # every symbol include/kvc.h declares
 EXPORTS = ["kvc_create", "kvc_destroy", "kvc_set_stream", "kvc_reset", "kvc_append_frame", "kvc_attend",
-           "kvc_attend_all",
+           "kvc_attend_all", "kvc_prune_all",
            "kvc_compress", "kvc_page_table", "kvc_token_meta", "kvc_last_merge", "kvc_export_pages",
            "kvc_step_host", "kvc_synchronize", "kvc_last_error", "kvc_status_string", "kvc_version",
            "kvc_debug_fail_allocs", "kvc_debug_bounded_wait", "kvc_attend_paged_noalloc", "kvc_append_frame_all",
@@ -91,6 +91,7 @@ def _load():
         "kvc_set_layer_budgets": ([vp, vp, i32], i32),
         "kvc_adapt_layer_budgets": ([vp, ctypes.c_double, i32, vp], i32),
         "kvc_prune": ([vp, i32], i32),
+        "kvc_prune_all": ([vp], i32),
         "kvc_scale_phase": ([vp, i32, i32, vp, vp, vp, vp], i32),
         "kvc_export_fp8_group_scales": ([vp, i32, i32, i32, vp, vp], i32),
         "kvc_layer_diversity": ([vp, i32, vp], i32),
@@ -323,6 +324,10 @@ def kvc_export_fp8_group_scales(handle, layer: int, first_row: int, n_rows: int,
 def kvc_prune(handle, layer: int) -> None:
     """Prune every head of `layer` to its Top-K candidates (the step before kvc_attend)."""
     _check(handle, _lib.kvc_prune(handle, layer))
+
+
+def kvc_prune_all(handle) -> None:
+    _check(handle, _lib.kvc_prune_all(handle))
 
 
 def kvc_adapt_layer_budgets(handle, num_layers: int, tau: float, k_avg: int) -> np.ndarray:

@@ -480,34 +480,52 @@ kvc_status div_append_layers(kvc_cache* c, int l0, int nl, int frame_idx, const 
   return KVC_OK;
 }
 
-// Scores every head's candidates and keeps its Top-K (no-op without a pending frame).
-kvc_status div_prune(kvc_cache* c, int layer) {
-  LayerHost& L = c->L[layer];
+// Scores every head's candidates and keeps its Top-K, for the layers [l0, l0 + n) that
+// have a pending frame: each run of consecutive such layers (up to kMaxPruneLayers) in one
+// launch.
+kvc_status div_prune_layers(kvc_cache* c, int l0, int n) {
   const kvc_config& g = c->cfg;
   const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads;
-  if (L.pend_pages == 0) return KVC_OK;
-  const size_t sub0 = static_cast<size_t>(layer) * H * c->pool_pages;
-  const int64_t cand = L.mut_tokens + T;
-  const int keep = static_cast<int>(std::min<int64_t>(c->layer_budget[layer], cand));
-  const int n_new = (keep + P - 1) / P;
-  // the kept tokens are compacted in place into the first n_new candidate pages; the
-  // other candidate pages are freed by the kernel
-  cudaError_t e = launch_diversity_prune(c->stream, c->entries + sub0, c->k_pool + sub0 * c->page_bytes_kv,
-                                         c->v_pool + sub0 * c->page_bytes_kv,
-                                         c->bitmap + static_cast<size_t>(layer) * H * c->bitmap_words,
-                                         c->bitmap_words, c->tok_id + sub0 * P, c->pool_pages, L.anchor_pages,
-                                         L.mut_pages + L.pend_pages, keep, H, g.head_dim, P,
-                                         c->div_sums + static_cast<size_t>(layer) * H, c->d_err);
-  if (e != cudaSuccess) return cuda_fail(c, e, "diversity pruning");
-  c->launches++;
-  L.n_entries = L.anchor_pages + n_new;
-  L.mut_pages = n_new;
-  L.mut_tokens = keep;
-  L.pend_pages = 0;
-  L.cand_count = cand;
-  L.compressions++;
+  for (int l = l0; l < l0 + n;) {
+    if (c->L[l].pend_pages == 0) {
+      ++l;
+      continue;
+    }
+    PruneLayerArgs args[kMaxPruneLayers];
+    int m = 0;
+    while (l + m < l0 + n && m < kMaxPruneLayers && c->L[l + m].pend_pages > 0) {
+      const LayerHost& L = c->L[l + m];
+      const int64_t cand = L.mut_tokens + T;
+      args[m].first_cand_entry = L.anchor_pages;
+      args[m].n_cand_entries = L.mut_pages + L.pend_pages;
+      args[m].keep = static_cast<int>(std::min<int64_t>(c->layer_budget[l + m], cand));
+      ++m;
+    }
+    // the kept tokens are compacted in place into the first ceil(keep / P) candidate
+    // pages; the other candidate pages are freed by the kernel
+    const size_t sub0 = static_cast<size_t>(l) * H * c->pool_pages;
+    cudaError_t e = launch_diversity_prune_layers(
+        c->stream, c->entries + sub0, c->k_pool + sub0 * c->page_bytes_kv, c->v_pool + sub0 * c->page_bytes_kv,
+        c->bitmap + static_cast<size_t>(l) * H * c->bitmap_words, c->bitmap_words, c->tok_id + sub0 * P,
+        c->pool_pages, args, m, H, g.head_dim, P, c->div_sums + static_cast<size_t>(l) * H, c->d_err);
+    if (e != cudaSuccess) return cuda_fail(c, e, "diversity pruning");
+    c->launches++;
+    for (int b = 0; b < m; ++b) {
+      LayerHost& L = c->L[l + b];
+      const int keep = args[b].keep;
+      L.n_entries = L.anchor_pages + (keep + P - 1) / P;
+      L.mut_pages = (keep + P - 1) / P;
+      L.cand_count = L.mut_tokens + T;
+      L.mut_tokens = keep;
+      L.pend_pages = 0;
+      L.compressions++;
+    }
+    l += m;
+  }
   return KVC_OK;
 }
+
+kvc_status div_prune(kvc_cache* c, int layer) { return div_prune_layers(c, layer, 1); }
 
 kvc_status div_attend(kvc_cache* c, int layer, const void* q_dev, void* o_dev) {
   kvc_status st = div_prune(c, layer);
@@ -833,10 +851,8 @@ kvc_status kvc_attend_all(kvc_cache* c, const void* const* q_devs, void* const* 
   if (batch) {
     if (c->per_head) {
       // the pruning comes first: the page counts the attention sees are the pruned ones
-      for (int l = 0; l < g.num_layers; ++l) {
-        kvc_status st = div_prune(c, l);
-        if (st != KVC_OK) return st;
-      }
+      kvc_status st = div_prune_layers(c, 0, g.num_layers);
+      if (st != KVC_OK) return st;
     }
     const int q_pairs = ((g.tokens_per_frame + 127) / 128 + 1) / 2;
     const long long groups = std::max(1, c->sm_count / q_pairs);
@@ -1181,6 +1197,12 @@ kvc_status kvc_prune(kvc_cache* c, int32_t layer) {
   if (!valid_layer(c, layer)) return fail(c, KVC_ERR_ARG, "kvc_prune: bad layer");
   if (!c->L[layer].has_pending) return fail(c, KVC_ERR_STATE, "kvc_prune: no frame pending on this layer");
   return div_prune(c, layer);
+}
+
+kvc_status kvc_prune_all(kvc_cache* c) {
+  if (!c) return KVC_ERR_ARG;
+  if (!c->per_head) return fail(c, KVC_ERR_STATE, "kvc_prune_all: not a diversity-pruned cache");
+  return div_prune_layers(c, 0, c->cfg.num_layers);
 }
 
 kvc_status kvc_adapt_layer_budgets(kvc_cache* c, double tau, int32_t k_avg, int32_t* budgets_out) {

@@ -196,12 +196,22 @@ __device__ int cta_scan_excl(int x, int* s_warp, int* total) {
   return r;
 }
 
+// Layers of one launch: blockIdx.y selects the layer, whose bases are the launch's plus
+// blockIdx.y strides, and whose candidate entries, budget and per-CTA candidate count
+// (B) are its row of the table.
 __global__ void __cluster_dims__(kPruneCluster, 1, 1) __launch_bounds__(kPruneThreads, 2) diversity_prune_kernel(
-    Entry* entries_layer, __nv_bfloat16* k_pool, __nv_bfloat16* v_pool, uint32_t* bitmap_layer, int words,
-    int64_t* tok_id_layer, int pool_pages, int first, int n_entries, int keep, int P, int B, double* sums_layer,
-    int* err) {
+    Entry* entries_base, __nv_bfloat16* k_base, __nv_bfloat16* v_base, uint32_t* bitmap_base, int words,
+    int64_t* tok_base, int pool_pages, int P, double* sums_base, int* err, const __grid_constant__ PruneBatch pb) {
   griddep_wait();
   griddep_launch_dependents();
+  const long long y = blockIdx.y;
+  Entry* entries_layer = entries_base + y * pb.entries_stride;
+  __nv_bfloat16* k_pool = k_base + y * pb.pool_stride;
+  __nv_bfloat16* v_pool = v_base + y * pb.pool_stride;
+  uint32_t* bitmap_layer = bitmap_base + y * pb.bitmap_stride;
+  int64_t* tok_id_layer = tok_base + y * pb.tok_stride;
+  double* sums_layer = sums_base + y * pb.sums_stride;
+  const int first = pb.l[y].first, n_entries = pb.l[y].n_entries, keep = pb.l[y].keep, B = pb.l[y].B;
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ int s_warp[32];
   __shared__ double s_mu[kDivD];
@@ -545,17 +555,31 @@ cudaError_t launch_append_heads(cudaStream_t s, const AppendBatch& in, int first
 
 int diversity_prune_max_candidates() { return kPruneCluster * kPruneMaxB; }
 
-cudaError_t launch_diversity_prune(cudaStream_t s, Entry* entries_layer, void* k_pool, void* v_pool,
-                                   uint32_t* bitmap_layer, int words, int64_t* tok_id_layer, int pool_pages,
-                                   int first_cand_entry, int n_cand_entries, int keep, int H, int D, int P,
-                                   double* sums_layer, int* err) {
-  const int n_max = n_cand_entries * P;
-  if (D != kDivD || n_cand_entries < 1 || n_cand_entries > kPruneThreads || keep < 1 ||
-      n_max > kPruneCluster * kPruneMaxB)
-    return cudaErrorInvalidValue;
-  int B = (n_max + kPruneCluster - 1) / kPruneCluster;
-  B = (B + kCandBlock - 1) / kCandBlock * kCandBlock;
-  const size_t smem = prune_layout(n_max, B, n_cand_entries).total;
+cudaError_t launch_diversity_prune_layers(cudaStream_t s, Entry* entries_base, void* k_base, void* v_base,
+                                          uint32_t* bitmap_base, int words, int64_t* tok_base, int pool_pages,
+                                          const PruneLayerArgs* layers, int n, int H, int D, int P,
+                                          double* sums_base, int* err) {
+  if (D != kDivD || n < 1 || n > kMaxPruneLayers) return cudaErrorInvalidValue;
+  PruneBatch pb{};
+  pb.entries_stride = static_cast<long long>(H) * pool_pages;
+  pb.pool_stride = static_cast<long long>(H) * pool_pages * P * kDivD;
+  pb.tok_stride = static_cast<long long>(H) * pool_pages * P;
+  pb.bitmap_stride = static_cast<long long>(H) * words;
+  pb.sums_stride = H;
+  size_t smem = 0;
+  for (int l = 0; l < n; ++l) {
+    const int n_max = layers[l].n_cand_entries * P;
+    if (layers[l].n_cand_entries < 1 || layers[l].n_cand_entries > kPruneThreads || layers[l].keep < 1 ||
+        n_max > kPruneCluster * kPruneMaxB)
+      return cudaErrorInvalidValue;
+    int B = (n_max + kPruneCluster - 1) / kPruneCluster;
+    B = (B + kCandBlock - 1) / kCandBlock * kCandBlock;
+    pb.l[l].first = layers[l].first_cand_entry;
+    pb.l[l].n_entries = layers[l].n_cand_entries;
+    pb.l[l].keep = layers[l].keep;
+    pb.l[l].B = B;
+    smem = std::max(smem, static_cast<size_t>(prune_layout(n_max, B, layers[l].n_cand_entries).total));
+  }
   // opt in once per device for the largest layout any call can need
   static PerDeviceOnce attr;
   cudaError_t e = attr.run([] {
@@ -564,10 +588,9 @@ cudaError_t launch_diversity_prune(cudaStream_t s, Entry* entries_layer, void* k
                                 static_cast<int>(most));
   });
   if (e != cudaSuccess) return e;
-  return launch_pdl(diversity_prune_kernel, dim3(H * kPruneCluster), dim3(kPruneThreads), smem, s,
-                    entries_layer, static_cast<__nv_bfloat16*>(k_pool), static_cast<__nv_bfloat16*>(v_pool),
-                    bitmap_layer, words, tok_id_layer, pool_pages, first_cand_entry, n_cand_entries, keep, P, B,
-                    sums_layer, err);
+  return launch_pdl(diversity_prune_kernel, dim3(H * kPruneCluster, n), dim3(kPruneThreads), smem, s, entries_base,
+                    static_cast<__nv_bfloat16*>(k_base), static_cast<__nv_bfloat16*>(v_base), bitmap_base, words,
+                    tok_base, pool_pages, P, sums_base, err, pb);
 }
 
 // Layer-wise adaptive budgets ("InfiniteVGGT" explainer, Layer-wise adaptive budgets): from

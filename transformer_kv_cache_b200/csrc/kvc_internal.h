@@ -332,10 +332,26 @@ cudaError_t launch_append_heads(cudaStream_t s, const AppendBatch& in, int first
                                 int64_t* tok_id_all, int pool_pages, int n_pages, int T, int H, int D, int P,
                                 int frame);
 int diversity_prune_max_candidates();
-cudaError_t launch_diversity_prune(cudaStream_t s, Entry* entries_layer, void* k_pool, void* v_pool,
-                                   uint32_t* bitmap_layer, int words, int64_t* tok_id_layer, int pool_pages,
-                                   int first_cand_entry, int n_cand_entries, int keep, int H, int D, int P,
-                                   double* sums_layer, int* err);
+// Pruning of n consecutive layers of a rolling memory in one launch (blockIdx.y = layer):
+// the bases are layer 0's (entries, pools, free bitmaps, token ids, score sums of its
+// sub-layers); each layer's candidates are the entries [first_cand_entry,
+// first_cand_entry + n_cand_entries) of every head's list, of which keep are kept.
+constexpr int kMaxPruneLayers = 32;
+struct PruneLayerArgs {
+  int first_cand_entry, n_cand_entries, keep;
+};
+struct PruneLayer {
+  int first, n_entries, keep, B;
+};
+struct PruneBatch {
+  long long entries_stride, pool_stride, tok_stride, bitmap_stride;
+  int sums_stride, pad;
+  PruneLayer l[kMaxPruneLayers];
+};
+cudaError_t launch_diversity_prune_layers(cudaStream_t s, Entry* entries_base, void* k_base, void* v_base,
+                                          uint32_t* bitmap_base, int words, int64_t* tok_base, int pool_pages,
+                                          const PruneLayerArgs* layers, int n, int H, int D, int P,
+                                          double* sums_base, int* err);
 
 // Layer-wise adaptive budgets of the rolling memory: budget_l = clamp(floor(L * k *
 // softmax(mean_l / tau)), 1, cap) from the layers' per-head score sums and candidate counts.
