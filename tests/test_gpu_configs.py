@@ -3,9 +3,10 @@ against the fp64 oracle:
 
 * 24 layers of the 518x378 shape with keyframe interval 4, streamed past the sliding
   window ("How GCTStream ...", Selective Frame Caching with Skip Append and Sliding
-  Window Eviction): every layer's page table against the closed-form retained set at
-  every step, three layers mirrored by the oracle in full (page tables bit for bit,
-  outputs on sampled rows of late frames).
+  Window Eviction), every layer attended in one launch per frame (kvc_attend_all): every
+  layer's page table against the closed-form retained set at every step, three layers
+  mirrored by the oracle in full (page tables bit for bit, outputs on sampled rows of late
+  frames).
 * 24 layers with a 16,384-token budget through two compression events per layer
   (StreamCacheVGGT page, 2.1.1-2.1.4 and 2): the rank window of 5 layers rolls over all
   24; four layers are mirrored in full, every layer is scored.
@@ -64,16 +65,17 @@ def test_config_24_layers_keyframe_interval_4_past_the_window(kvc):
     try:
         st = FrameStream(wl, seed=31, device=dev)
         orc = StreamOracle(OracleConfig.from_workload(wl))
-        o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+        outs = [torch.empty((T, H, D), dtype=torch.bfloat16, device=dev) for _ in range(L)]
         evicted = 0
         for t in range(frames):
             key = keyframe_schedule(t, S, k)
             qkv = [st.frame(l, t) for l in range(L)]
             kvc.kvc_append_frame_all(h, t, [x[1] for x in qkv], [x[2] for x in qkv], key)
+            kvc.kvc_attend_all(h, [x[0] for x in qkv], outs)   # every layer in one attention launch
             want = retained(t, S, W, k)
             for l in range(L):
                 q, kk, vv = qkv[l]
-                kvc.kvc_attend(h, l, q, o)
+                o = outs[l]
                 if l in mirror:
                     orc.append(l, t, np64(kk), np64(vv), key)
                     if t in check:

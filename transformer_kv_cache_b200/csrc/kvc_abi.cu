@@ -834,9 +834,9 @@ kvc_status commit_layer(kvc_cache* c, int layer) {
 }
 
 // Every layer's pending frame attended, as kvc_attend on each layer in order. On the bf16
-// tensor-core path, layers too small to fill the GPU alone (fewer than
-// kLayerBatchStepsPerGroup (head, KV tile) steps per CTA group) go through one launch
-// per kMaxAttnLayers layers; the commits follow, layer by layer.
+// tensor-core path the layers go through one launch per kMaxAttnLayers layers (one sweep
+// over every layer's (head, KV tile) steps: no per-layer launch cost or tail); the
+// commits follow, layer by layer.
 kvc_status kvc_attend_all(kvc_cache* c, const void* const* q_devs, void* const* o_devs) {
   if (!c) return KVC_ERR_ARG;
   const kvc_config& g = c->cfg;
@@ -847,18 +847,12 @@ kvc_status kvc_attend_all(kvc_cache* c, const void* const* q_devs, void* const* 
       return fail(c, KVC_ERR_ARG, "kvc_attend_all: Q and O must be non-null and 16-byte aligned");
     if (!c->L[l].has_pending) return fail(c, KVC_ERR_STATE, "kvc_attend_all: a layer has no pending frame");
   }
-  bool batch = c->tc_path && g.kv_dtype != KVC_FP8_E4M3 && g.num_layers > 1;
+  const bool batch = c->tc_path && g.kv_dtype != KVC_FP8_E4M3 && g.num_layers > 1;
   if (batch) {
     if (c->per_head) {
       // the pruning comes first: the page counts the attention sees are the pruned ones
       kvc_status st = div_prune_layers(c, 0, g.num_layers);
       if (st != KVC_OK) return st;
-    }
-    const int q_pairs = ((g.tokens_per_frame + 127) / 128 + 1) / 2;
-    const long long groups = std::max(1, c->sm_count / q_pairs);
-    for (int l = 0; l < g.num_layers && batch; ++l) {
-      const long long steps = static_cast<long long>(g.num_heads) * ((c->L[l].n_entries * g.page_size + 127) / 128);
-      if (steps >= kLayerBatchStepsPerGroup * groups) batch = false;
     }
   }
   if (!batch) {

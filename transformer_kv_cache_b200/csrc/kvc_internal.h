@@ -289,9 +289,7 @@ struct AttnPlan {
 };
 bool plan_attn_bf16(int T, int H, const int* n_pages, int n_layers, int P, int sm_count, int kv_splits,
                     size_t part_tiles, bool strict, AttnPlan* out, int* n_tiles, int* pos0);
-// Steps per CTA group below which a layer is too small to fill the GPU on its own and
-// several layers are better attended in one launch.
-constexpr int kLayerBatchStepsPerGroup = 16;
+
 // Split counters the bf16 kernel needs for T query rows and H heads.
 inline size_t attn_counter_count(long long T, int H) { return static_cast<size_t>(H) * ((T + 127) / 128) * 4; }
 
