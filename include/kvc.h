@@ -205,9 +205,10 @@ KVC_API kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, vo
 /* kvc_attend on every layer, in layer order: q_devs[l] and o_devs[l] are layer l's
  * [T, H, D] queries and outputs (each 16-byte aligned), and every layer must have a
  * pending frame. The results, page tables and counters are those of the per-layer
- * calls. With bf16 storage on the tensor cores the layers' attention runs in one launch
- * per 32 layers (after the rolling memory's pruning of every layer, itself one launch);
- * otherwise (FP8, fp32, other head dims or page sizes) the call is the per-layer loop.
+ * calls. On the tensor cores (bf16 or FP8 storage, D = 64, P = 16) the layers'
+ * attention runs in one launch per 32 layers (after the rolling memory's pruning of
+ * every layer, itself one launch); otherwise (fp32, other head dims or page sizes) the
+ * call is the per-layer loop.
  * Errors: KVC_ERR_ARG (NULL or misaligned pointers), KVC_ERR_STATE (a layer without a
  * pending frame; nothing is attended then). */
 KVC_API kvc_status kvc_attend_all(kvc_cache* c, const void* const* q_devs, void* const* o_devs);

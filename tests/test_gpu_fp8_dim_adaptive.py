@@ -20,7 +20,7 @@ def kvc():
 
 @pytest.mark.parametrize("T,H,W,S,frames,splits", [
     (300, 4, 6, 2, 10, 0),     # ragged last page, eviction, automatic splits
-    (300, 2, 4, 1, 8, 3),      # three KV splits and the combine
+    (300, 2, 4, 1, 8, 3),      # about three pieces per head, merged in the kernel
     (37, 2, 3, 1, 8, 0),       # one ragged query tile, last page 5 valid
 ])
 def test_dimension_adaptive_fp8(kvc, T, H, W, S, frames, splits):

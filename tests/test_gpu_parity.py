@@ -41,12 +41,15 @@ def test_bf16_tensor_core_small(kvc, T, H, W, S, frames, splits):
     run_parity(kvc, wl, frames, kv_splits=splits, check_pages=True)
 
 
-def test_attend_all_layers_one_launch(kvc):
+@pytest.mark.parametrize("kv_dtype,dim_adaptive", [("bf16", 0), ("fp8_e4m3", 0), ("fp8_e4m3", 1)])
+def test_attend_all_layers_one_launch(kvc, kv_dtype, dim_adaptive):
     """kvc_attend_all on a 4-layer window cache whose layers are small (one launch for every
     layer): every layer's output against the oracle, page tables equal, keyframe interval
-    2 past the window, and the library's launch count shows one attention launch per frame."""
+    2 past the window, and the library's launch count shows one attention launch per frame;
+    bf16 and FP8 E4M3 storage (page scales, and dimension-adaptive scales)."""
     wl = WORKLOADS["vggt_24layer_k4"].replace(num_layers=4, tokens_per_frame=200, num_heads=4, window_frames=3,
-                                              scale_frames=1, keyframe_interval=2, num_special_tokens=5)
+                                              scale_frames=1, keyframe_interval=2, num_special_tokens=5,
+                                              kv_dtype=kv_dtype, fp8_dim_adaptive=dim_adaptive)
     L, T, H, D = wl.num_layers, wl.tokens_per_frame, wl.num_heads, wl.head_dim
     dev = torch.device("cuda")
     h = kvc.kvc_create(kvc.config_from_workload(wl))
@@ -99,8 +102,8 @@ def test_fp8_small_codes_and_outputs(kvc):
 
 
 @pytest.mark.parametrize("T,H,splits", [
-    (300, 3, 1),     # one CTA per (q tile, head): every KV tile in one softmax pass
-    (300, 3, 3),     # three KV splits and the combine
+    (300, 3, 1),     # one piece per head: every KV tile in one softmax pass
+    (300, 3, 3),     # about three pieces per head, merged in the kernel
     (37, 2, 0),      # ragged q tile, partial last page of every frame
 ])
 def test_fp8_tensor_core(kvc, T, H, splits):

@@ -833,10 +833,10 @@ kvc_status commit_layer(kvc_cache* c, int layer) {
   return KVC_OK;
 }
 
-// Every layer's pending frame attended, as kvc_attend on each layer in order. On the bf16
-// tensor-core path the layers go through one launch per kMaxAttnLayers layers (one sweep
-// over every layer's (head, KV tile) steps: no per-layer launch cost or tail); the
-// commits follow, layer by layer.
+// Every layer's pending frame attended, as kvc_attend on each layer in order. On the
+// tensor-core path (bf16 or E4M3 storage) the layers go through one launch per
+// kMaxAttnLayers layers (one sweep over every layer's (head, KV tile) steps: no per-layer
+// launch cost or tail); the commits follow, layer by layer.
 kvc_status kvc_attend_all(kvc_cache* c, const void* const* q_devs, void* const* o_devs) {
   if (!c) return KVC_ERR_ARG;
   const kvc_config& g = c->cfg;
@@ -847,7 +847,8 @@ kvc_status kvc_attend_all(kvc_cache* c, const void* const* q_devs, void* const* 
       return fail(c, KVC_ERR_ARG, "kvc_attend_all: Q and O must be non-null and 16-byte aligned");
     if (!c->L[l].has_pending) return fail(c, KVC_ERR_STATE, "kvc_attend_all: a layer has no pending frame");
   }
-  const bool batch = c->tc_path && g.kv_dtype != KVC_FP8_E4M3 && g.num_layers > 1;
+  const bool fp8 = g.kv_dtype == KVC_FP8_E4M3;
+  const bool batch = c->tc_path && g.num_layers > 1 && !(fp8 && c->per_head);
   if (batch) {
     if (c->per_head) {
       // the pruning comes first: the page counts the attention sees are the pruned ones
@@ -872,7 +873,11 @@ kvc_status kvc_attend_all(kvc_cache* c, const void* const* q_devs, void* const* 
   a.splits = g.kv_splits;
   a.tmap_k = &c->tmap_k[0];
   a.tmap_v = &c->tmap_v[0];
-  a.fp8 = false;
+  a.fp8 = fp8;
+  a.k_scale = c->k_scale;
+  a.v_scale = c->v_scale;
+  a.k_chan = c->k_chan;
+  a.v_tok = c->v_tok;
   a.q_heads = c->model_heads;
   a.head0 = c->head0;
   a.part_o = c->part_o;

@@ -1,5 +1,5 @@
-// kvc_attn_common.cuh -- parameters and device helpers shared by the tensor-core attention
-// kernels (bf16 and FP8 storage).
+// kvc_attn_common.cuh -- parameters and device helpers of the tensor-core attention kernel
+// (bf16 and FP8 E4M3 storage).
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -10,25 +10,24 @@
 namespace kvc {
 
 struct TcParams {
-  const __nv_bfloat16* q;       // [T][H][D] queries
-  const float* k_scale;         // FP8 storage only: per (pool page, head) scales
+  const float* k_scale;         // E4M3 storage: [pool page][head] K and V scales
   const float* v_scale;
-  const Entry* entries;
-  int n_pages, T, H;
-  int q_tiles, splits, tiles_per_split, total_tiles;
-  int q_pairs;                  // bf16 kernel: query-tile pairs (one per CTA of a group)
-  int out_heads, head0;         // bf16 kernel: heads of Q and O; the cache's head h is head0 + h
-  long long page_base;          // layer * pool_pages: first pool page of the layer
+  int T, H;
+  int q_tiles;                  // 128-row query tiles
+  int splits;                   // most pieces of one unit (head, query-tile pair)
+  int tiles_per_split;          // R: steps (128-slot KV tiles) per group of CTAs
+  int total_tiles;              // steps of all layers
+  int q_pairs;                  // query-tile pairs (one per CTA of a group)
+  int out_heads, head0;         // heads of Q and O; the cache's head h is head0 + h
   int pool_rows;                // rows of the pool tensor maps (a row index past the end reads zeros)
   float scale_log2;
-  __nv_bfloat16* out;
   float* part_o;
   float* part_lse;
   int* err;
   int head_pages;               // > 0: per-head page lists (see TcAttnArgs)
-  int* split_cnt;               // [H][q_tiles][4] zeroed counters: the piece that counts last merges (bf16 kernel)
-  const float* k_chan;          // dimension-adaptive FP8: [pool page][head][64] K channel scales
-  const float* v_tok;           // dimension-adaptive FP8: [pool page][head][16] V token scales
+  int* split_cnt;               // [layer x H][q_tiles][4] zeroed counters: the piece that counts last merges
+  const float* k_chan;          // dimension-adaptive E4M3: [pool page][head][64] K channel scales
+  const float* v_tok;           // dimension-adaptive E4M3: [pool page][head][16] V token scales
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -86,11 +85,5 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
-
-
-// FP8 E4M3 storage variant (kvc_attn_fp8.cu): same parameters, the query map of the bf16
-// kernel, pool maps over the code bytes (box 64 B x P rows, no swizzle).
-cudaError_t launch_attn_fp8_kernel(cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                   const TcParams& prm, int grid);
 
 }  // namespace kvc

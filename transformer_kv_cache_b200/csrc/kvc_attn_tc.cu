@@ -83,6 +83,18 @@ __host__ __device__ constexpr int col_base(int i) { return 256 * i; }
 constexpr float kLog2PMax = 8.0f;             // a P above 2^8 moves the row's reference max
 constexpr int kPolyPer8 = 3;                  // of every 8 column pairs, the 2^x on the FMA pipe
 constexpr size_t kSmemBytes = 1024 + 2 * kStages * kTileBytes + kOnesBytes + 512;
+// E4M3 storage: a fourth warpgroup widens the codes of each KV tile into the f16 operand
+// ring; the codes land by TMA in a ring of their own
+constexpr int kThreads8 = 512;
+constexpr int kStages8 = 4;                   // f16 operand stages
+constexpr int kCodeStages = 3;                // code stages (K and V codes of one KV tile)
+constexpr int kCodeTileBytes = kBN * kHD;     // 8 KB: one tensor's codes of a KV tile
+constexpr int kRegsConv = 96, kRegsHigh8 = 176;  // 128 x 56 + 256 x 176 + 128 x 96 <= 512 x 128
+constexpr int kMetaBytes = kStages8 * (8 + 8 + 1) * 4;   // per operand stage: the tile's page metadata
+constexpr size_t kSmemBytes8 =
+    1024 + 2 * kStages8 * kTileBytes + kOnesBytes + 2 * kCodeStages * kCodeTileBytes + kMetaBytes + 512;
+// storage modes of the kernel
+constexpr int kBf16 = 0, kE4m3 = 1, kE4m3Da = 2;   // bf16; E4M3 + page scales; + dimension-adaptive
 }  // namespace tc
 
 // ---- the FMA-pipe exponential
@@ -125,16 +137,39 @@ __device__ __forceinline__ uint64_t exp2_fma_pair(uint64_t x2) {
              __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
 }
 
-// One S tile of P for a row: pb[i] = bf16 pair of 2^(s*c - m) for columns 2i, 2i+1, rounded
-// to nearest. Of every 8 pairs the last kPoly go to the FMA pipe and the others to the
-// MUFU, and every pair is finished (exponent, packing) in one pass, so MUFU instructions
-// are spread through the row's FMA and ALU work instead of queueing behind one another.
-template <int N>
-__device__ __forceinline__ void tile_p(const uint32_t (&s)[N], float c, float m, uint32_t (&pb)[N / 2]) {
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// ---- E4M3 codes
+// Two E4M3 codes (low byte first) as an f16 pair, exactly (every E4M3 value is an f16 value).
+__device__ __forceinline__ uint32_t f16x2_of_e4m3x2(uint32_t code_pair) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(static_cast<uint16_t>(code_pair)));
+  return r;
+}
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// One S tile of P for a row: pb[i] = pair of 2^(s*c - m) for columns 2i, 2i+1, rounded to
+// nearest bf16 (or f16). c is the logit factor of the pair's group of N / 2 / NQ pairs
+// (NQ = 1: one factor; for E4M3 storage one per page, which carries the page's K scale).
+// Of every 8 pairs the last kPoly go to the FMA pipe and the others to the MUFU, and every
+// pair is finished (exponent, packing) in one pass, so MUFU instructions are spread through
+// the row's FMA and ALU work instead of queueing behind one another.
+template <bool kF16, int N, int NQ>
+__device__ __forceinline__ void tile_p(const uint32_t (&s)[N], const float (&cq)[NQ], float m,
+                                       uint32_t (&pb)[N / 2]) {
   constexpr int kPoly = tc::kPolyPer8;
-  const uint64_t c2 = pk2(c, c), nm2 = pk2(-m, -m);
+  constexpr int kPairsPerQ = N / 2 / NQ;
+  const uint64_t nm2 = pk2(-m, -m);
 #pragma unroll
   for (int i = 0; i < N / 2; ++i) {
+    const uint64_t c2 = pk2(cq[i / kPairsPerQ], cq[i / kPairsPerQ]);
     const uint64_t x2 = fma2_pair(s[2 * i], s[2 * i + 1], c2, nm2);
     uint64_t y2;
     if ((i & 7) >= 8 - kPoly) {
@@ -146,7 +181,7 @@ __device__ __forceinline__ void tile_p(const uint32_t (&s)[N], float c, float m,
     }
     float y0, y1;
     up2(y2, y0, y1);
-    pb[i] = pack_bf16(y0, y1);
+    pb[i] = kF16 ? pack_f16(y0, y1) : pack_bf16(y0, y1);
   }
 }
 
@@ -163,6 +198,23 @@ __device__ __forceinline__ float row_max64(const uint32_t (&s)[tc::kBH]) {
   for (int i = 0; i < 7; ++i) b[i] = max3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
   b[7] = a[21];
   return max3(max3(b[0], b[1], b[2]), max3(b[3], b[4], b[5]), fmaxf(b[6], b[7]));
+}
+// Largest scaled score of a row with one logit factor per 16-slot page (E4M3 storage): the
+// page's largest raw score times its factor (factors are positive).
+__device__ __forceinline__ float row_max64_pages(const uint32_t (&s)[tc::kBH], const float (&cq)[4]) {
+  float r = -INFINITY;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t* t = &s[16 * q];
+    const float a = max3(__uint_as_float(t[0]), __uint_as_float(t[1]), __uint_as_float(t[2]));
+    const float b = max3(__uint_as_float(t[3]), __uint_as_float(t[4]), __uint_as_float(t[5]));
+    const float c = max3(__uint_as_float(t[6]), __uint_as_float(t[7]), __uint_as_float(t[8]));
+    const float d = max3(__uint_as_float(t[9]), __uint_as_float(t[10]), __uint_as_float(t[11]));
+    const float e = max3(__uint_as_float(t[12]), __uint_as_float(t[13]), __uint_as_float(t[14]));
+    const float pm = max3(max3(a, b, c), max3(d, e, __uint_as_float(t[15])), -INFINITY);
+    r = fmaxf(r, pm * cq[q]);
+  }
+  return r;
 }
 
 // Register split between warpgroups (every warp of a warpgroup executes the same one).
@@ -191,8 +243,8 @@ __device__ __forceinline__ bool next_piece(Sweep& sw, const AttnLayers& lt, int 
   return true;
 }
 
-// Epilogue of one warp's 32 query rows of a piece. Single-piece units store bf16 O
-// directly; otherwise every piece stores its normalised partial and log2-sum-exp, counts
+// Epilogue of one warp's 32 query rows of a piece (O = oscale O' / l, oscale the V reference
+// scale of E4M3 storage, else 1). Single-piece units store bf16 O directly; otherwise every piece stores its normalised partial and log2-sum-exp, counts
 // itself on the warp's counter, and the piece that counts last merges. Only a group's
 // first and last piece can belong to a unit of several pieces (the pieces between them are
 // whole heads), so a partial lives in the slot of (its group, first or last piece of the
@@ -202,12 +254,12 @@ __device__ __forceinline__ bool next_piece(Sweep& sw, const AttnLayers& lt, int 
 // synchronisation is used, so a warp that gave up on a wait cannot hold another here.
 __device__ __forceinline__ void store_piece(const TcParams& p, const LayerAttn& la, int lay, int wg, int wq, int lane,
                                             int h, int qp, int g, const uint32_t (&o0)[32], const uint32_t (&o1)[32],
-                                            float l, float m) {
+                                            float l, float m, float oscale) {
   using namespace tc;
   const int r = wq * 32 + lane;
   const int qtile = 2 * qp + wg;
   const int row = qtile * kBM + r;
-  const float inv = 1.f / l;
+  const float inv = oscale / l;
   const int n_tiles = la.n_tiles, R = p.tiles_per_split;
   const int g_first = (la.pos0 + h * n_tiles) / R;
   const int g_last = (la.pos0 + h * n_tiles + n_tiles - 1) / R;
@@ -307,28 +359,39 @@ __device__ __forceinline__ void store_piece(const TcParams& p, const LayerAttn& 
   if (lane == 0) p.split_cnt[cidx] = 0;   // ready for the next launch
 }
 
-template <int P, bool kPerHead>
-__global__ void __launch_bounds__(tc::kThreads, 1)
+template <int P, bool kPerHead, int kMode>
+__global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThreads8, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                    const TcParams p, const __grid_constant__ AttnLayers lt) {
   griddep_wait();
   griddep_launch_dependents();
   using namespace tc;
+  constexpr bool kF8 = kMode != kBf16;        // E4M3 codes, widened to f16 operands
+  constexpr bool kDA = kMode == kE4m3Da;
+  constexpr int kS = kF8 ? kStages8 : kStages;   // operand stages
   constexpr int kPPT = kBN / P;               // pages per KV tile (TMA stage)
   constexpr int kPPH = kBH / P;               // pages per half (S tile)
+  static_assert(P == 16, "16-slot pages: a 64-slot half holds 4 of them");
+  static_assert(!kF8 || !kPerHead, "E4M3 storage: one page list per layer");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* k_s = smem;                                   // [stage][128 rows][128 B]
-  uint8_t* v_s = k_s + kStages * kTileBytes;
-  uint8_t* ones_s = v_s + kStages * kTileBytes;          // after every V stage: a positive offset
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ones_s + kOnesBytes);
+  uint8_t* v_s = k_s + kS * kTileBytes;
+  uint8_t* ones_s = v_s + kS * kTileBytes;               // after every V stage: a positive offset
+  uint8_t* codes = ones_s + kOnesBytes;                  // E4M3: [code stage][K, V][128 rows][64 B]
+  // E4M3, per operand stage (written by the converters with the tile's K, read by the
+  // softmax): the valid slots and K scales of the tile's 8 pages, the piece's V reference
+  int* meta_valid = reinterpret_cast<int*>(codes + (kF8 ? 2 * kCodeStages * kCodeTileBytes : 0));   // [kS][8]
+  float* meta_ks = reinterpret_cast<float*>(meta_valid + (kF8 ? kS * 8 : 0));                       // [kS][8]
+  float* meta_vref = meta_ks + (kF8 ? kS * 8 : 0);                                                  // [kS]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(meta_vref + (kF8 ? kS : 0));
   uint64_t* k_full = bars;
-  uint64_t* v_full = k_full + kStages;
-  uint64_t* kv_empty = v_full + kStages;      // both issuers done with the stage
+  uint64_t* v_full = k_full + kS;
+  uint64_t* kv_empty = v_full + kS;           // both issuers done with the stage
   // Per query tile i ([i], or [2 i + b] for S buffer b). Every wait is on a phase at most
   // one ahead of the last one the waiter saw complete (a parity wait cannot tell two
   // phases apart), which is why P and the piece's end have their own barriers:
-  uint64_t* q_ready = kv_empty + kStages;     // Q in TMEM (the 4 softmax warps)
+  uint64_t* q_ready = kv_empty + kS;          // Q in TMEM (the 4 softmax warps)
   uint64_t* s_full = q_ready + 2;             // S buffer computed
   uint64_t* p_full = s_full + 4;              // P in S buffer b (the 4 softmax warps)
   uint64_t* pv_done = p_full + 4;             // a P.V product complete (rescale: S of half u
@@ -336,7 +399,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   uint64_t* o_full = pv_done + 2;             // the piece's last P.V complete
   uint64_t* o_free = o_full + 2;              // O' read by the epilogue (the 4 softmax warps)
   uint64_t* mma_final = o_free + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_final + 2);
+  uint64_t* code_full = mma_final + 2;        // E4M3: a code stage landed
+  uint64_t* code_empty = code_full + kCodeStages;   // E4M3: a code stage read (the 4 converters)
+  uint64_t* vref_bar = code_empty + kCodeStages;    // E4M3: [piece & 1] partial V maxima written
+  float* vref_part = reinterpret_cast<float*>(vref_bar + 2);   // [piece & 1][converter]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(vref_part + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -347,9 +414,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   const Sweep sweep0{min(g * R, HT), min(g * R + R, HT), 0};
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&v_full[i], 1);
+    for (int i = 0; i < kS; ++i) {
+      mbar_init(&k_full[i], kF8 ? 4 : 1);       // E4M3: the 4 converter warps
+      mbar_init(&v_full[i], kF8 ? 4 : 1);
       mbar_init(&kv_empty[i], kQT);
     }
     for (int i = 0; i < kQT; ++i) {
@@ -363,13 +430,22 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       mbar_init(&o_free[i], 4);
       mbar_init(&mma_final[i], 1);
     }
+    if (kF8) {
+      for (int i = 0; i < kCodeStages; ++i) {
+        mbar_init(&code_full[i], 1);
+        mbar_init(&code_empty[i], 4);
+      }
+      mbar_init(&vref_bar[0], 4);
+      mbar_init(&vref_bar[1], 4);
+    }
     *abort_flag = 0;
     mbar_fence_init();
   }
   // the constant ones block (every element 1.0, so the swizzle does not matter), made
   // visible to the tensor core's operand reads
-  for (int i = threadIdx.x; i < kOnesBytes / 16; i += kThreads)
-    reinterpret_cast<uint4*>(ones_s)[i] = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
+  const uint32_t one2 = kF8 ? 0x3c003c00u : 0x3f803f80u;
+  for (int i = threadIdx.x; i < kOnesBytes / 16; i += (kF8 ? kThreads8 : kThreads))
+    reinterpret_cast<uint4*>(ones_s)[i] = make_uint4(one2, one2, one2, one2);
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -383,11 +459,13 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     reg_dealloc<kRegsLow>();
     if (lane == 0) {
       // ------------------------------------------------------------------ TMA producer
+      // bf16: the K and V tiles into the operand ring; E4M3: their codes into the code ring
+      constexpr int kRing = kF8 ? kCodeStages : kS;
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_v);
-      int last[kStages];
+      int last[kRing];
 #pragma unroll
-      for (int i = 0; i < kStages; ++i) last[i] = -1;
+      for (int i = 0; i < kRing; ++i) last[i] = -1;
       int jg = 0;
       bool ok = true;
       Sweep sw = sweep0;
@@ -405,7 +483,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           phys_next[q] = idx < n_pages ? __ldg(&ent[idx].x) : -1;
         }
         for (int t = t0; t < t1; ++t, ++jg) {
-          const int st = jg % kStages;
+          const int st = jg % kRing;
           int row[kPPT];
 #pragma unroll
           for (int q = 0; q < kPPT; ++q) {
@@ -421,25 +499,42 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
               phys_next[q] = idx < n_pages ? __ldg(&ent[idx].x) : -1;
             }
           }
-          if (jg >= kStages && !mbar_wait_bounded(&kv_empty[st], ((jg / kStages) - 1) & 1, abort_flag, p.err)) {
+          uint64_t* free_bar = kF8 ? &code_empty[st] : &kv_empty[st];
+          if (jg >= kRing && !mbar_wait_bounded(free_bar, ((jg / kRing) - 1) & 1, abort_flag, p.err)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+          if (kF8) {
+            uint8_t* cb = codes + st * 2 * kCodeTileBytes;
+            mbar_arrive_expect_tx(&code_full[st], 2 * kCodeTileBytes);
 #pragma unroll
-          for (int q = 0; q < kPPT; ++q) tma_load_2d(k_s + st * kTileBytes + q * P * 128, &tmap_k, &k_full[st], 0, row[q]);
-          mbar_arrive_expect_tx(&v_full[st], kTileBytes);
+            for (int q = 0; q < kPPT; ++q) tma_load_2d(cb + q * P * kHD, &tmap_k, &code_full[st], 0, row[q]);
 #pragma unroll
-          for (int q = 0; q < kPPT; ++q) tma_load_2d(v_s + st * kTileBytes + q * P * 128, &tmap_v, &v_full[st], 0, row[q]);
+            for (int q = 0; q < kPPT; ++q)
+              tma_load_2d(cb + kCodeTileBytes + q * P * kHD, &tmap_v, &code_full[st], 0, row[q]);
+          } else {
+            mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+#pragma unroll
+            for (int q = 0; q < kPPT; ++q)
+              tma_load_2d(k_s + st * kTileBytes + q * P * 128, &tmap_k, &k_full[st], 0, row[q]);
+            mbar_arrive_expect_tx(&v_full[st], kTileBytes);
+#pragma unroll
+            for (int q = 0; q < kPPT; ++q)
+              tma_load_2d(v_s + st * kTileBytes + q * P * 128, &tmap_v, &v_full[st], 0, row[q]);
+          }
           last[st] = jg;
         }
       }
       // drain: every copy this CTA issued has landed before shared memory is released
 #pragma unroll
-      for (int i = 0; i < kStages; ++i) {
+      for (int i = 0; i < kRing; ++i) {
         if (last[i] >= 0) {
-          mbar_wait_drain(&k_full[i], (last[i] / kStages) & 1, p.err);
-          mbar_wait_drain(&v_full[i], (last[i] / kStages) & 1, p.err);
+          if (kF8) {
+            mbar_wait_drain(&code_full[i], (last[i] / kRing) & 1, p.err);
+          } else {
+            mbar_wait_drain(&k_full[i], (last[i] / kRing) & 1, p.err);
+            mbar_wait_drain(&v_full[i], (last[i] / kRing) & 1, p.err);
+          }
         }
       }
     }
@@ -448,8 +543,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     // ------------------------------------------------------------------ MMA issuer of query tile i
     // Halves are numbered globally (uu = 2 * KV tile + half); half uu uses S buffer uu & 1.
     const int i = warp - 1;
-    const uint32_t idesc_s = idesc_f16kind(1, kBM, kBH, 0, 0);
-    const uint32_t idesc_o = idesc_f16kind(1, kBM, kON, 0, 1);
+    const uint32_t fmt = kF8 ? 0u : 1u;         // operand type: f16 or bf16
+    const uint32_t idesc_s = idesc_f16kind(fmt, kBM, kBH, 0, 0);
+    const uint32_t idesc_o = idesc_f16kind(fmt, kBM, kON, 0, 1);
     const uint32_t tb = tmem + col_base(i);
     const uint32_t k_addr = smem_u32(k_s), v_addr = smem_u32(v_s), ones_addr = smem_u32(ones_s);
     const bool leader = elect_one();
@@ -458,9 +554,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     // product of half uu - 2 (which read its P from this buffer): this issuer's MMAs run in
     // order, so that product has read P before S overwrites it.
     auto issue_s = [&](int uu, int u) -> bool {
-      const int jj = uu >> 1, hb = uu & 1, st = jj % kStages;
+      const int jj = uu >> 1, hb = uu & 1, st = jj % kS;
       bool w = true;
-      if (hb == 0) w = mbar_wait_bounded(&k_full[st], (jj / kStages) & 1, abort_flag, p.err);
+      if (hb == 0) w = mbar_wait_bounded(&k_full[st], (jj / kS) & 1, abort_flag, p.err);
       if (u == 0) w = w && mbar_wait_bounded(&q_ready[i], pc & 1, abort_flag, p.err);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
@@ -478,9 +574,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     // O' += P [V | 1] for half uu; the first half of a piece overwrites O' once the previous
     // piece's epilogue has read it
     auto issue_pv = [&](int uu, int u, bool last) -> bool {
-      const int jj = uu >> 1, hb = uu & 1, st = jj % kStages;
+      const int jj = uu >> 1, hb = uu & 1, st = jj % kS;
       bool w = mbar_wait_bounded(&p_full[2 * i + hb], jj & 1, abort_flag, p.err);
-      if (hb == 0) w = w && mbar_wait_bounded(&v_full[st], (jj / kStages) & 1, abort_flag, p.err);
+      if (hb == 0) w = w && mbar_wait_bounded(&v_full[st], (jj / kS) & 1, abort_flag, p.err);
       if (u == 0 && pc > 0) w = w && mbar_wait_bounded(&o_free[i], (pc - 1) & 1, abort_flag, p.err);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
@@ -500,7 +596,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     // the stage of half uu's KV tile is released after its second half's P.V (committed
     // after the next S, off the path from P.V to that S)
     auto release = [&](int uu) {
-      if (leader && (uu & 1)) mma_commit(&kv_empty[(uu >> 1) % kStages]);
+      if (leader && (uu & 1)) mma_commit(&kv_empty[(uu >> 1) % kS]);
       __syncwarp();
     };
     bool ok = true;
@@ -522,8 +618,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     mbar_wait_drain(&mma_final[i], 0, p.err);
   } else if (warp < 4) {
     reg_dealloc<kRegsLow>();                       // warp 3 only gives up registers
-  } else {
-    reg_alloc<kRegsHigh>();
+  } else if (!kF8 || warp < 12) {
+    reg_alloc<kF8 ? kRegsHigh8 : kRegsHigh>();
     // ------------------------------------------------------------------ softmax warps
     const int wg = (warp - 4) >> 2;               // query tile of the pair
     const int wq = warp & 3;                      // TMEM lane quadrant this warp may access
@@ -539,6 +635,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       const LayerAttn& la = lt.l[lay];
       const Entry* ent = kPerHead ? la.entries + static_cast<long long>(h) * p.head_pages : la.entries;
       const int n_pages = la.n_pages;
+      float row_fac = 1.f;       // E4M3: 2^-e of the query row's scaling into f16
       {
         // this row of Q (zeros past the last query) into TMEM, the A operand of S; the S
         // products of the previous piece, its only readers, have completed (their S was read)
@@ -555,6 +652,24 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             qv[4 * v + 2] = w.z;
             qv[4 * v + 3] = w.w;
           }
+          if (kF8) {
+            // f16 operands: the row is scaled by the power of two 2^e that brings its largest
+            // magnitude into [2^14, 2^15), so no finite bf16 query overflows f16 and small
+            // rows keep their bits; the row's logit factor carries 2^-e, which makes the
+            // scaling exact (e is clamped to [-120, 100] so that factor stays a normal float)
+            float qmax = 0.f;
+#pragma unroll
+            for (int v = 0; v < 32; ++v) qmax = max3(qmax, fabsf(bf16lo(qv[v])), fabsf(bf16hi(qv[v])));
+            int e = 0;
+            if (qmax > 0.f) {
+              int ex;
+              frexpf(qmax, &ex);                  // qmax in [2^(ex-1), 2^ex)
+              e = min(100, max(-120, 15 - ex));
+            }
+            row_fac = ldexpf(1.f, -e);
+#pragma unroll
+            for (int v = 0; v < 32; ++v) qv[v] = pack_f16(ldexpf(bf16lo(qv[v]), e), ldexpf(bf16hi(qv[v]), e));
+          }
         } else {
 #pragma unroll
           for (int v = 0; v < 32; ++v) qv[v] = 0u;
@@ -566,26 +681,59 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         if (lane == 0) mbar_arrive(&q_ready[wg]);
       }
       float m = -INFINITY;       // reference max (log2 domain) of the row
+      float vref = 1.f;          // E4M3: the piece's V reference
+      // bf16: valid slots of the pages of the next half (every lane loads all of them)
       int vnext[kPPH];
+      if (!kF8) {
 #pragma unroll
-      for (int q = 0; q < kPPH; ++q) {
-        const int idx = t0 * kPPT + q;
-        vnext[q] = idx < n_pages ? __ldg(&ent[idx].w) : 0;
+        for (int q = 0; q < kPPH; ++q) {
+          const int idx = t0 * kPPT + q;
+          vnext[q] = idx < n_pages ? __ldg(&ent[idx].w) : 0;
+        }
       }
       for (int u = 0; u < nh; ++u) {
         const int uu = ub + u, hb = uu & 1, jj = uu >> 1;
         int vcur[kPPH];
+        float cq[kF8 ? kPPH : 1];                 // logit factor (per page for E4M3)
         bool partial = false;
-#pragma unroll
-        for (int q = 0; q < kPPH; ++q) {
-          vcur[q] = vnext[q];
-          partial |= vcur[q] < P;
-        }
-        if (u + 1 < nh) {
+        if constexpr (kF8) {
+          // the half's 4 pages from the stage's metadata, which the converters wrote before
+          // they released the tile's K (the wait makes their writes visible; the stage is
+          // not refilled before this tile's P.V products, which need this half's P)
+          const int st = jj % kS;
+          if (hb == 0 &&
+              !__all_sync(0xffffffffu, mbar_wait_bounded(&k_full[st], (jj / kS) & 1, abort_flag, p.err))) {
+            ok = false;
+            break;
+          }
+          const int4 v4 = *reinterpret_cast<const int4*>(&meta_valid[st * 8 + 4 * hb]);
+          const float4 ks4 = *reinterpret_cast<const float4*>(&meta_ks[st * 8 + 4 * hb]);
+          vref = meta_vref[st];
+          vcur[0] = v4.x;
+          vcur[1] = v4.y;
+          vcur[2] = v4.z;
+          vcur[3] = v4.w;
+          partial = min(min(v4.x, v4.y), min(v4.z, v4.w)) < P;
+          // a zero-scale page (all-zero K, or past the list) gets a tiny positive factor:
+          // its valid scores are 0 either way, and its masked -inf scores stay -inf
+          const float crow = c * row_fac;
+          cq[0] = fmaxf(crow * ks4.x, 1e-30f);
+          cq[1] = fmaxf(crow * ks4.y, 1e-30f);
+          cq[2] = fmaxf(crow * ks4.z, 1e-30f);
+          cq[3] = fmaxf(crow * ks4.w, 1e-30f);
+        } else {
+          cq[0] = c;
 #pragma unroll
           for (int q = 0; q < kPPH; ++q) {
-            const int idx = t0 * kPPT + (u + 1) * kPPH + q;
-            vnext[q] = idx < n_pages ? __ldg(&ent[idx].w) : 0;
+            vcur[q] = vnext[q];
+            partial |= vcur[q] < P;
+          }
+          if (u + 1 < nh) {
+#pragma unroll
+            for (int q = 0; q < kPPH; ++q) {
+              const int idx = t0 * kPPT + (u + 1) * kPPH + q;
+              vnext[q] = idx < n_pages ? __ldg(&ent[idx].w) : 0;
+            }
           }
         }
         uint32_t s[kBH];
@@ -606,7 +754,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         // exact fp32 max of the half; the row's reference max moves when some P would exceed
         // 2^8 (or on the first half of a piece); O' is then rescaled by 2^(m_old - m_new)
         // once the previous half's P.V has completed
-        const float tm = row_max64(s) * c;
+        float tm;
+        if constexpr (kF8) tm = row_max64_pages(s, cq);
+        else tm = row_max64(s) * c;
         const bool move = (u == 0) || tm > m + kLog2PMax;
         if (__any_sync(0xffffffffu, move)) {
           const float m_new = move ? (tm == -INFINITY ? (m == -INFINITY ? 0.f : m) : tm) : m;
@@ -631,7 +781,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           m = m_new;
         }
         uint32_t pb[kBH / 2];
-        tile_p(s, c, m, pb);
+        tile_p<kF8>(s, cq, m, pb);
         // P over the first 32 columns of this half's S buffer, whose S is in registers; the
         // buffer is not written again before this P's product has read it (tcgen05.ld/st are
         // .sync.aligned: every branch around them is warp-uniform)
@@ -656,8 +806,177 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_free[wg]);
-      store_piece(p, la, lay, wg, wq, lane, h, qp, g, o0, o1, __uint_as_float(lsum), m);
+      // E4M3: V was divided by the piece's V reference
+      store_piece(p, la, lay, wg, wq, lane, h, qp, g, o0, o1, __uint_as_float(lsum), m, kF8 ? vref : 1.f);
       ub += nh;
+      ++pc;
+    }
+  } else if constexpr (kF8) {
+    reg_dealloc<kRegsConv>();
+    // ------------------------------------------------------------------ E4M3 converters
+    // Converter cw widens rows [32 cw, 32 cw + 32) of every KV tile (pages 2 cw and 2 cw + 1):
+    // lane (r0, c0) = (lane >> 3, lane & 7) takes rows 32 cw + r0 + 4 i (i < 8), 8-code chunk
+    // c0, stored at chunk c0 ^ (row & 7) of the 128-byte-swizzled f16 row. K codes stay
+    // unscaled (the page's K scale is in the softmax's logit factor); V codes are multiplied
+    // by the page's V scale over the piece's V reference (the largest V scale of its pages).
+    // Dimension-adaptive scales: K also by its channel scale over the page's K scale, V by its
+    // token scale instead of the page's.
+    const int cw = warp - 12;
+    const int r0 = lane >> 3, c0 = lane & 7;
+    const int src_off = (32 * cw + r0) * kHD + 8 * c0;
+    const int dst_even = (32 * cw + r0) * 128 + ((c0 ^ r0) << 4);
+    const int dst_odd = (32 * cw + r0) * 128 + ((c0 ^ r0 ^ 4) << 4);
+    int jg = 0, pc = 0;
+    bool ok = true;
+    Sweep sw = sweep0;
+    int lay, h, t0, t1;
+    while (ok && next_piece(sw, lt, p.H, lay, h, t0, t1)) {
+      const LayerAttn& la = lt.l[lay];
+      const Entry* ent = la.entries;
+      const int n_pages = la.n_pages;
+      const long long page_base = la.page_base;
+      // V reference of the piece: each converter takes a quarter of its pages, 16 loads in
+      // flight per lane, and the four partial maxima meet in shared memory
+      float mv = 0.f;
+      {
+        const int i0 = t0 * kPPT, i1 = min(t1 * kPPT, n_pages);
+        const int span = (i1 - i0 + 3) / 4;
+        const int a0 = i0 + cw * span, a1 = min(i1, a0 + span);
+        for (int base = a0; base < a1; base += 32 * 16) {
+          int ph[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const int idx = base + 32 * k + lane;
+            ph[k] = idx < a1 ? __ldg(&ent[idx].x) : -1;
+          }
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            if (ph[k] >= 0) mv = fmaxf(mv, __ldg(&p.v_scale[(page_base + ph[k]) * p.H + h]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, o));
+        const int b = pc & 1;
+        if (lane == 0) {
+          vref_part[4 * b + cw] = mv;
+          mbar_arrive(&vref_bar[b]);
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&vref_bar[b], (pc >> 1) & 1, abort_flag, p.err))) {
+          ok = false;
+          break;
+        }
+        mv = fmaxf(fmaxf(vref_part[4 * b], vref_part[4 * b + 1]), fmaxf(vref_part[4 * b + 2], vref_part[4 * b + 3]));
+        if (mv == 0.f) mv = 1.f;                  // all-zero pages: any reference works
+      }
+      const float iv = 1.f / mv;
+      // this converter's two pages of tile t (every lane loads both): physical page and
+      // valid slots, one tile ahead
+      auto entry_of = [&](int t, int gg) -> int2 {
+        const int idx = t * kPPT + 2 * cw + gg;
+        if (t < t1 && idx < n_pages) {
+          const int4 e = __ldg(&ent[idx]);
+          return make_int2(e.x, e.w);
+        }
+        return make_int2(-1, 0);
+      };
+      int2 en_next[2] = {entry_of(t0, 0), entry_of(t0, 1)};
+      for (int t = t0; ok && t < t1; ++t, ++jg) {
+        const int st = jg % kS, cs = jg % kCodeStages;
+        const int ph[2] = {en_next[0].x, en_next[1].x};
+        const int nv[2] = {en_next[0].y, en_next[1].y};
+        en_next[0] = entry_of(t + 1, 0);
+        en_next[1] = entry_of(t + 1, 1);
+        // f16 factors of this tile: vr[gg] per page, or per row (and per K chunk) for the
+        // dimension-adaptive scales; the pages' K scales for the softmax
+        uint32_t vr[kDA ? 8 : 2];
+        uint32_t kf[kDA ? 2 : 1][4];
+        float ksp[2];
+#pragma unroll
+        for (int gg = 0; gg < 2; ++gg) {
+          const long long base = (page_base + ph[gg]) * p.H + h;
+          ksp[gg] = ph[gg] >= 0 ? __ldg(&p.k_scale[base]) : 0.f;
+          if (!kDA) {
+            const float vs = ph[gg] >= 0 ? __ldg(&p.v_scale[base]) : 0.f;
+            vr[gg] = pack_f16(vs * iv, vs * iv);
+          } else {
+            float kc[8], vt[4];
+            const float ks = ksp[gg];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) kc[e] = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) vt[e] = 0.f;
+            if (ph[gg] >= 0) {
+              const float4 a = __ldg(reinterpret_cast<const float4*>(p.k_chan + base * kHD + 8 * c0));
+              const float4 b = __ldg(reinterpret_cast<const float4*>(p.k_chan + base * kHD + 8 * c0) + 1);
+              kc[0] = a.x; kc[1] = a.y; kc[2] = a.z; kc[3] = a.w;
+              kc[4] = b.x; kc[5] = b.y; kc[6] = b.z; kc[7] = b.w;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) vt[e] = __ldg(&p.v_tok[base * P + r0 + 4 * e]);
+            }
+            const float inv = ks > 0.f ? 1.f / ks : 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) kf[kDA ? gg : 0][e] = pack_f16(kc[2 * e] * inv, kc[2 * e + 1] * inv);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) vr[kDA ? 4 * gg + e : 0] = pack_f16(vt[e] * iv, vt[e] * iv);
+          }
+        }
+        // the operand stage is free once both query tiles' products of tile jg - kS are done
+        if (jg >= kS &&
+            !__all_sync(0xffffffffu, mbar_wait_bounded(&kv_empty[st], ((jg / kS) - 1) & 1, abort_flag, p.err))) {
+          ok = false;
+          break;
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&code_full[cs], (jg / kCodeStages) & 1, abort_flag, p.err))) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          meta_ks[st * 8 + 2 * cw] = ksp[0];
+          meta_ks[st * 8 + 2 * cw + 1] = ksp[1];
+          meta_valid[st * 8 + 2 * cw] = nv[0];
+          meta_valid[st * 8 + 2 * cw + 1] = nv[1];
+          if (cw == 0) meta_vref[st] = mv;
+        }
+        const uint8_t* ksrc = codes + cs * 2 * kCodeTileBytes + src_off;
+        const uint8_t* vsrc = ksrc + kCodeTileBytes;
+        uint8_t* kdst = k_s + st * kTileBytes;
+        uint8_t* vdst = v_s + st * kTileBytes;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {             // row 32 cw + r0 + 4 i: page i / 4 of the two
+          const uint2 kc = *reinterpret_cast<const uint2*>(ksrc + i * 4 * kHD);
+          uint4 ko;
+          ko.x = f16x2_of_e4m3x2(kc.x);
+          ko.y = f16x2_of_e4m3x2(kc.x >> 16);
+          ko.z = f16x2_of_e4m3x2(kc.y);
+          ko.w = f16x2_of_e4m3x2(kc.y >> 16);
+          if (kDA) {
+            ko.x = hmul2(ko.x, kf[kDA ? i >> 2 : 0][0]);
+            ko.y = hmul2(ko.y, kf[kDA ? i >> 2 : 0][1]);
+            ko.z = hmul2(ko.z, kf[kDA ? i >> 2 : 0][2]);
+            ko.w = hmul2(ko.w, kf[kDA ? i >> 2 : 0][3]);
+          }
+          *reinterpret_cast<uint4*>(kdst + i * 512 + ((i & 1) ? dst_odd : dst_even)) = ko;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&k_full[st]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint2 vc = *reinterpret_cast<const uint2*>(vsrc + i * 4 * kHD);
+          const uint32_t f = vr[kDA ? i : i >> 2];
+          uint4 vo;
+          vo.x = hmul2(f16x2_of_e4m3x2(vc.x), f);
+          vo.y = hmul2(f16x2_of_e4m3x2(vc.x >> 16), f);
+          vo.z = hmul2(f16x2_of_e4m3x2(vc.y), f);
+          vo.w = hmul2(f16x2_of_e4m3x2(vc.y >> 16), f);
+          *reinterpret_cast<uint4*>(vdst + i * 512 + ((i & 1) ? dst_odd : dst_even)) = vo;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&v_full[st]);
+          mbar_arrive(&code_empty[cs]);
+        }
+      }
       ++pc;
     }
   }
@@ -670,47 +989,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   }
 }
 
-// Merge split partials of the FP8 kernel: O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M).
-// One warp per (row, head): lane s (and s + 32) loads split s's log-sum-exp, so the maximum
-// and the weights take one round of loads and warp shuffles; then each lane accumulates two
-// of the 64 dims over the splits (up to 64 splits). Partials are [head][split][query tile]
-// tiles of 128 rows.
-__global__ void combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
-                               __nv_bfloat16* __restrict__ out, int T, int H, int q_tiles, int splits) {
-  griddep_wait();
-  griddep_launch_dependents();
-  constexpr int kRows = 128, kD = 64;
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (gw >= T * H) return;
-  const int t = gw / H, h = gw % H;
-  const int qt = t / kRows, r = t % kRows;
-  const long long pi0 = static_cast<long long>(h) * splits * q_tiles + qt;
-  auto row_of = [&](int s) { return (pi0 + static_cast<long long>(s) * q_tiles) * kRows + r; };
-  const float l0 = lane < splits ? __ldg(&part_lse[row_of(lane)]) : -INFINITY;
-  const float l1 = lane + 32 < splits ? __ldg(&part_lse[row_of(lane + 32)]) : -INFINITY;
-  float M = fmaxf(l0, l1);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float w0 = lane < splits ? exp2f(l0 - M) : 0.f;
-  const float w1 = lane + 32 < splits ? exp2f(l1 - M) : 0.f;
-  float ws = w0 + w1;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
-  float a0 = 0.f, a1 = 0.f;
-#pragma unroll 4
-  for (int s = 0; s < splits; ++s) {
-    const float w = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
-    const float2 o = __ldg(reinterpret_cast<const float2*>(part_o + row_of(s) * kD) + lane);
-    a0 = fmaf(w, o.x, a0);
-    a1 = fmaf(w, o.y, a1);
-  }
-  const float inv = 1.f / ws;
-  reinterpret_cast<__nv_bfloat162*>(out + (static_cast<long long>(t) * H + h) * kD)[lane] =
-      __floats2bfloat162_rn(a0 * inv, a1 * inv);
-}
-
 // ------------------------------------------------------------------ host side
+
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -740,45 +1020,6 @@ bool encode_pool_tmap(CUtensorMap* map, void* base, size_t rows, int D, int P, i
 
 // Queries [T][H][64] bf16 as a 3-D map; one box is 128 rows of one head (128-byte swizzle),
 // rows past T read as zeros.
-static bool encode_q_tmap(CUtensorMap* map, const void* q, int T, int H) {
-  auto fn = get_encode_fn();
-  if (!fn) return false;
-  constexpr int kD = 64, kRows = 128;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * 2, static_cast<cuuint64_t>(H) * kD * 2};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(kD), 1, static_cast<cuuint32_t>(kRows)};
-  cuuint32_t es[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-// Pick the number of KV splits of the FP8 kernel (one CTA per SM, two query tiles per CTA).
-// Cost of a split count, in units of one 64-slot KV tile: waves x (fixed cost of a CTA +
-// tiles per CTA) + a cost per split (the partials written and combined): 4 and
-// 0.5 + 0.25 s tiles, measured. Among counts within 1% of the best cost the fewest win.
-int choose_splits(int units, int tiles, int slots, bool fp8) {
-  (void)fp8;
-  const double cta_cost = 4.0;
-  const int max_s = tiles < 64 ? tiles : 64;
-  double cost[65];
-  double best_cost = 1e30;
-  for (int s = 1; s <= max_s; ++s) {
-    cost[s] = 1e30;
-    const int tps = (tiles + s - 1) / s;
-    if ((tiles + tps - 1) / tps != s) continue;        // the same as a smaller split count
-    const long long ctas = static_cast<long long>(units) * s;
-    const long long waves = (ctas + slots - 1) / slots;
-    const double split_cost = s == 1 ? 0.0 : 0.5 + 0.25 * s;
-    cost[s] = static_cast<double>(waves) * (cta_cost + tps) + split_cost;
-    if (cost[s] < best_cost) best_cost = cost[s];
-  }
-  for (int s = 1; s <= max_s; ++s)
-    if (cost[s] <= best_cost * 1.01) return s;
-  return 1;
-}
-
 // Schedule of the bf16 kernel over one or more layers. R = steps per group; groups of
 // q_pairs CTAs. Automatic: as many groups as fill the SMs (one CTA each); with
 // kv_splits = s > 0, about s pieces per head of the largest layer. Split units need
@@ -834,17 +1075,35 @@ bool plan_attn_bf16(int T, int H, const int* n_pages, int n_layers, int P, int s
 }
 
 namespace {
-cudaError_t launch_bf16_layers(cudaStream_t s, const TcAttnArgs& a, const LayerAttn* layers, int n,
-                               int* splits_used, int* launched) {
+template <int kMode>
+cudaError_t launch_mode(cudaStream_t s, bool per_head, dim3 grid, const TcParams& prm, const TcAttnArgs& a,
+                        const AttnLayers& lt) {
+  constexpr bool kF8 = kMode != tc::kBf16;
+  const int threads = kF8 ? tc::kThreads8 : tc::kThreads;
+  const size_t smem = kF8 ? tc::kSmemBytes8 : tc::kSmemBytes;
+  if (per_head) {
+    if constexpr (kF8) return cudaErrorInvalidValue;
+    else return launch_pdl(attn_tc_kernel<16, true, kMode>, grid, dim3(threads), smem, s, *a.tmap_k, *a.tmap_v, prm, lt);
+  }
+  return launch_pdl(attn_tc_kernel<16, false, kMode>, grid, dim3(threads), smem, s, *a.tmap_k, *a.tmap_v, prm, lt);
+}
+
+cudaError_t launch_layers(cudaStream_t s, const TcAttnArgs& a, const LayerAttn* layers, int n, int* splits_used,
+                          int* launched) {
   if (n < 1 || n > kMaxAttnLayers) return cudaErrorInvalidValue;
+  if (a.P != 16 || (a.fp8 && a.head_pages)) return cudaErrorInvalidValue;
+  if (a.fp8 && (!a.k_scale || !a.v_scale || (a.k_chan != nullptr) != (a.v_tok != nullptr)))
+    return cudaErrorInvalidValue;
   const int qh = a.q_heads > 0 ? a.q_heads : a.H;
+  if (a.head0 < 0 || a.head0 + a.H > qh) return cudaErrorInvalidValue;
   static PerDeviceOnce attr;
   cudaError_t e = attr.run([] {
-    cudaError_t r = cudaFuncSetAttribute(attn_tc_kernel<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(tc::kSmemBytes));
-    if (r == cudaSuccess)
-      r = cudaFuncSetAttribute(attn_tc_kernel<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(tc::kSmemBytes));
+    const int b = static_cast<int>(tc::kSmemBytes), f = static_cast<int>(tc::kSmemBytes8);
+    const cudaFuncAttribute at = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    cudaError_t r = cudaFuncSetAttribute(attn_tc_kernel<16, false, tc::kBf16>, at, b);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(attn_tc_kernel<16, true, tc::kBf16>, at, b);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(attn_tc_kernel<16, false, tc::kE4m3>, at, f);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(attn_tc_kernel<16, false, tc::kE4m3Da>, at, f);
     return r;
   });
   if (e != cudaSuccess) return e;
@@ -883,12 +1142,14 @@ cudaError_t launch_bf16_layers(cudaStream_t s, const TcAttnArgs& a, const LayerA
   prm.split_cnt = a.split_cnt;
   prm.out_heads = qh;
   prm.head0 = a.head0;
-  if (a.head_pages)
-    e = launch_pdl(attn_tc_kernel<16, true>, dim3(pl.grid), dim3(tc::kThreads), tc::kSmemBytes, s, *a.tmap_k,
-                   *a.tmap_v, prm, lt);
-  else
-    e = launch_pdl(attn_tc_kernel<16, false>, dim3(pl.grid), dim3(tc::kThreads), tc::kSmemBytes, s, *a.tmap_k,
-                   *a.tmap_v, prm, lt);
+  prm.k_scale = a.k_scale;
+  prm.v_scale = a.v_scale;
+  prm.k_chan = a.k_chan;
+  prm.v_tok = a.v_tok;
+  const dim3 grid(pl.grid);
+  if (!a.fp8) e = launch_mode<tc::kBf16>(s, a.head_pages > 0, grid, prm, a, lt);
+  else if (a.k_chan) e = launch_mode<tc::kE4m3Da>(s, false, grid, prm, a, lt);
+  else e = launch_mode<tc::kE4m3>(s, false, grid, prm, a, lt);
   if (e != cudaSuccess) return e;
   if (launched) *launched = 1;
   if (splits_used) *splits_used = pl.max_pieces;
@@ -899,79 +1160,18 @@ cudaError_t launch_bf16_layers(cudaStream_t s, const TcAttnArgs& a, const LayerA
 cudaError_t launch_attn_tc_layers(cudaStream_t s, const TcAttnArgs& base, const LayerAttn* layers, int n,
                                   int* launched) {
   if (launched) *launched = 0;
-  if (base.P != 16 || base.fp8) return cudaErrorInvalidValue;
-  const int qh = base.q_heads > 0 ? base.q_heads : base.H;
-  if (base.head0 < 0 || base.head0 + base.H > qh) return cudaErrorInvalidValue;
-  return launch_bf16_layers(s, base, layers, n, nullptr, launched);
+  return launch_layers(s, base, layers, n, nullptr, launched);
 }
 
 cudaError_t launch_attn_tc(cudaStream_t s, const TcAttnArgs& a, int* splits_used, int* launched) {
   if (launched) *launched = 0;
-  if (a.P != 16 || (a.fp8 && a.head_pages)) return cudaErrorInvalidValue;
-  const int qh = a.q_heads > 0 ? a.q_heads : a.H;
-  if (a.head0 < 0 || a.head0 + a.H > qh || (a.fp8 && qh != a.H)) return cudaErrorInvalidValue;
-  if (!a.fp8) {
-    LayerAttn one{};
-    one.q = a.q;
-    one.o = a.o;
-    one.entries = a.entries;
-    one.page_base = a.page_base;
-    one.n_pages = a.n_pages;
-    return launch_bf16_layers(s, a, &one, 1, splits_used, launched);
-  }
-  // FP8 storage: one CTA per SM takes two 128-row query tiles of a head and a range of
-  // 64-slot KV tiles; more than one split goes through the combine kernel
-  CUtensorMap tq;
-  if (!encode_q_tmap(&tq, a.q, a.T, qh)) return cudaErrorInvalidValue;
-  const int q_tiles = (a.T + 127) / 128;
-  const int total_tiles = (a.n_pages * a.P + 63) / 64;
-  const int units = ((q_tiles + 1) / 2) * a.H;
-  const int part_units = q_tiles * a.H;       // 128-row partial tiles per split
-  int splits = a.splits > 0 ? a.splits : choose_splits(units, total_tiles, a.sm_count, true);
-  if (splits > total_tiles) splits = total_tiles;
-  if (splits > 64) splits = 64;                  // the combine takes up to 64 partials per row
-  int tps = (total_tiles + splits - 1) / splits;
-  splits = (total_tiles + tps - 1) / tps;
-  if (splits > 1 && static_cast<size_t>(part_units) * splits > a.part_rows) {
-    // not enough partial scratch: fall back to as many splits as fit
-    splits = static_cast<int>(a.part_rows / part_units);
-    if (splits < 1) splits = 1;
-    tps = (total_tiles + splits - 1) / splits;
-    splits = (total_tiles + tps - 1) / tps;
-  }
-  TcParams prm{};
-  prm.q = static_cast<const __nv_bfloat16*>(a.q);
-  prm.k_scale = a.k_scale;
-  prm.v_scale = a.v_scale;
-  prm.entries = a.entries;
-  prm.n_pages = a.n_pages;
-  prm.T = a.T;
-  prm.H = a.H;
-  prm.q_tiles = q_tiles;
-  prm.splits = splits;
-  prm.tiles_per_split = tps;
-  prm.total_tiles = total_tiles;
-  prm.page_base = a.page_base;
-  prm.pool_rows = static_cast<int>(a.pool_rows);
-  prm.scale_log2 = static_cast<float>(static_cast<double>(a.softmax_scale) * 1.4426950408889634);
-  prm.out = static_cast<__nv_bfloat16*>(a.o);
-  prm.part_o = a.part_o;
-  prm.part_lse = a.part_lse;
-  prm.err = a.err;
-  prm.k_chan = a.k_chan;
-  prm.v_tok = a.v_tok;
-  cudaError_t e = launch_attn_fp8_kernel(s, tq, *a.tmap_k, *a.tmap_v, prm, units * splits);
-  if (e != cudaSuccess) return e;
-  if (launched) *launched = 1;
-  if (splits > 1) {
-    const long long warps = static_cast<long long>(a.T) * a.H;
-    const int threads = 256;
-    e = launch_pdl(combine_kernel, dim3(static_cast<int>((warps * 32 + threads - 1) / threads)), dim3(threads), 0, s,
-                   a.part_o, a.part_lse, static_cast<__nv_bfloat16*>(a.o), a.T, a.H, q_tiles, splits);
-    if (launched) *launched = 2;
-  }
-  if (splits_used) *splits_used = splits;
-  return e;
+  LayerAttn one{};
+  one.q = a.q;
+  one.o = a.o;
+  one.entries = a.entries;
+  one.page_base = a.page_base;
+  one.n_pages = a.n_pages;
+  return launch_layers(s, a, &one, 1, splits_used, launched);
 }
 
 }  // namespace kvc

@@ -274,7 +274,6 @@ struct AttnLayers {
 };
 cudaError_t launch_attn_tc_layers(cudaStream_t s, const TcAttnArgs& base, const LayerAttn* layers, int n,
                                   int* launched);
-int choose_splits(int units, int tiles, int slots, bool fp8);
 
 // Schedule of the bf16 tensor-core attention (kvc_attn_tc.cu): units are (layer, head,
 // pair of 128-row query tiles); groups of q_pairs CTAs sweep R consecutive (layer, head,
