@@ -99,8 +99,9 @@ typedef struct {
   int32_t residual_dim;         /* R, columns of the residual given to kvc_compress */
   int32_t protect_first_frame;  /* 1: every token of frame 0 is always kept */
   int32_t max_frames;           /* cap on cached frames when W <= 0 and B == 0 */
-  int32_t kv_splits;            /* KV splits per query tile in attention (at most 64 are
-                                   used); 0 = automatic */
+  int32_t kv_splits;            /* s > 0: the tensor-core attention cuts each head's KV
+                                   sequence into about s pieces (merged in the kernel);
+                                   0 = automatic (the pieces that fill the SMs) */
   int32_t diversity_budget;     /* K > 0: rolling diversity-pruned memory, K kept tokens per
                                    head per layer besides the first frame (see kvc_attend) */
   int32_t special_frames;       /* > 0 (window mode only): cross-frame special tokens, see

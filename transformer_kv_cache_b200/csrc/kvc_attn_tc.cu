@@ -1,4 +1,5 @@
-// kvc_attn_tc.cu -- frame attention over the paged bf16 cache on sm_100a tensor cores.
+// kvc_attn_tc.cu -- frame attention over the paged cache (bf16 or FP8 E4M3 storage) on
+// sm_100a tensor cores.
 //
 // Computes O[i, h] = sum_j softmax_j(scale * q_i . k_j) v_j for the T queries of the new
 // frame over every valid slot of the layer's page list ("How GCTStream ...",
@@ -14,8 +15,8 @@
 // pieces of a unit are merged by the piece that finishes last (partial outputs carry their
 // log2-sum-exp), so no separate combine launch is needed.
 //
-// Roles of a CTA (384 threads, one CTA per SM, all 512 TMEM columns; warpgroup 0 gives up
-// registers to the two softmax warpgroups with setmaxnreg):
+// Roles of a CTA (384 threads for bf16 storage, one CTA per SM, all 512 TMEM columns;
+// warpgroup 0 gives up registers to the two softmax warpgroups with setmaxnreg):
 //   warp 0 (one lane)   TMA producer: per KV tile the 8 page-head blocks of K and of V
 //                       (128-byte swizzled) into a 5-stage ring. Pages past the end of the
 //                       list are read past the end of the pool, which TMA fills with zeros.
@@ -50,6 +51,22 @@
 // Partial pages: slots past a page's valid count hold K = V = 0 (the append and compaction
 // kernels write zeros there) and their scores are set to -inf before the softmax, in the
 // tiles that have such slots; pages past the end of the list are masked the same way.
+//
+// E4M3 storage ("XStreamVGGT" abstract: KV cache quantisation; codes with one absmax scale
+// per (page, head), or per K channel and V token with the dimension-adaptive scales). The
+// tensor cores multiply f16 operands (kind::f16 takes one type for A and B), so the CTA has a
+// fourth warpgroup (512 threads): the TMA producer loads each KV tile's codes into a 3-stage
+// code ring, and warps 12-15, one per sub-partition, each widen a quarter of the tile (32
+// rows of K and V) into the 4-stage f16 operand ring with the exact E4M3 -> f16 conversion.
+// K codes stay unscaled: the page's K scale multiplies the logit factor of the page's 16
+// columns in the softmax. V codes are multiplied by the page's V scale over the piece's V
+// reference (the largest V scale of its pages, which keeps every product in f16 range) and
+// the epilogue multiplies O by that reference; this rounding of V to f16 (relative 2^-11)
+// is the only extra rounding of an operand. Each Q row is scaled into f16 by the power of
+// two that brings its largest magnitude into [2^14, 2^15), the row's logit factor carrying
+// the inverse. P is rounded to f16. The converters also write each tile's page metadata
+// (valid slots, K scales, V reference) next to the stage, which the softmax reads after the
+// stage's K barrier.
 //
 // Every barrier wait is bounded: on timeout the CTA records KVC_ERR_TIMEOUT in the error
 // word, drains its own copies and MMAs, frees TMEM and returns.
