@@ -5,10 +5,12 @@
 // The decision is taken in fp64, as the definition is written; the tensor cores only
 // narrow the search:
 //
-//   screen  one CTA per 128 sources x 128 targets: the bf16 keys (stored values, exact)
-//           of both sides go through tcgen05 (K = H*D, fp32 accumulation in TMEM); the
-//           epilogue scales each dot product by the two fp32 inverse norms and keeps the
-//           four largest approximate cosines of the tile per source.
+//   screen  one CTA per 256 sources x 256 targets (two M=128, N=256 accumulators filling
+//           TMEM, so each key byte brought from L2 feeds 128 multiply-adds): the bf16 keys
+//           (stored values, exact) of both sides go through tcgen05 (K = H*D, fp32
+//           accumulation in TMEM); the epilogue scales each dot product by the two fp32
+//           inverse norms and keeps the four largest approximate cosines of the tile per
+//           source.
 //   refine  one warp per source: M = the largest screened value over all tiles; every
 //           target whose screened value is within kMargin of M is re-evaluated in fp64,
 //           and where a tile's fourth value is itself within the margin, all targets of
@@ -27,27 +29,33 @@
 
 namespace kvc {
 namespace cs {
-constexpr int kBM = 128, kBN = 128, kBK = 64;      // sources x targets x key dims per stage
+constexpr int kBM = 128;                           // sources per accumulator (MMA M)
+constexpr int kMT = 2;                             // accumulators per CTA: 256 sources
+constexpr int kBN = 256;                           // targets per CTA (MMA N)
+constexpr int kBK = 64;                            // key dims per stage
 constexpr int kStages = 3;
-constexpr int kTileBytes = kBM * kBK * 2;          // 16 KB per operand per stage
-constexpr int kThreads = 192;
-constexpr int kTmemCols = 128;
-constexpr size_t kSmemBytes = 1024 + 2 * kStages * kTileBytes + kBN * 4 + 256;
+constexpr int kBoxBytes = 128 * kBK * 2;           // one TMA box: 128 rows x 64 dims (16 KB)
+constexpr int kATileBytes = kMT * kBoxBytes;       // 256 source rows
+constexpr int kBTileBytes = 2 * kBoxBytes;         // 256 target rows
+constexpr int kThreads = 384;                      // TMA, MMA, 2 idle, 8 epilogue warps
+constexpr int kTmemCols = 512;
+constexpr size_t kSmemBytes = 1024 + kStages * (kATileBytes + kBTileBytes) + kBN * 4 + 256;
 constexpr float kMargin = 0.0009765625f;           // 2^-10
 }  // namespace cs
 
 // Screened cosines: warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues the MMAs, warps
-// 2..5 run the epilogue (one source row per thread).
-__global__ void __launch_bounds__(cs::kThreads, 2)
+// 4..11 run the epilogue (one source row per thread; warps 4..7 the first accumulator,
+// 8..11 the second).
+__global__ void __launch_bounds__(cs::kThreads, 1)
     cos_screen_kernel(const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_e,
                       const float* __restrict__ inv_ns, const float* __restrict__ inv_ne, int n_src, int n_elig,
                       int HD, float* __restrict__ top_v, int32_t* __restrict__ top_j, int tiles_n, int* err) {
   using namespace cs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* a_s = smem;                                   // sources [kStages]
-  uint8_t* b_s = smem + kStages * kTileBytes;            // targets [kStages]
-  float* inv_e_s = reinterpret_cast<float*>(b_s + kStages * kTileBytes);
+  uint8_t* a_s = smem;                                   // sources [kStages][256 rows]
+  uint8_t* b_s = smem + kStages * kATileBytes;           // targets [kStages][256 rows]
+  float* inv_e_s = reinterpret_cast<float*>(b_s + kStages * kBTileBytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(inv_e_s + kBN);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
@@ -55,7 +63,7 @@ __global__ void __launch_bounds__(cs::kThreads, 2)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e0 = blockIdx.x * kBN, s0 = blockIdx.y * kBM;
+  const int e0 = blockIdx.x * kBN, s0 = blockIdx.y * (kMT * kBM);
   const int nk = (HD + kBK - 1) / kBK;                  // dims past HD read as zeros
 
   if (threadIdx.x == 0) {
@@ -84,9 +92,11 @@ __global__ void __launch_bounds__(cs::kThreads, 2)
       for (int kb = 0; kb < nk; ++kb) {
         const int st = kb % kStages;
         if (kb >= kStages && !mbar_wait_bounded(&empty[st], ((kb / kStages) - 1) & 1, abort_flag, err)) break;
-        mbar_arrive_expect_tx(&full[st], 2 * kTileBytes);
-        tma_load_2d(a_s + st * kTileBytes, &tmap_s, &full[st], kb * kBK, s0);
-        tma_load_2d(b_s + st * kTileBytes, &tmap_e, &full[st], kb * kBK, e0);
+        mbar_arrive_expect_tx(&full[st], kATileBytes + kBTileBytes);
+        tma_load_2d(a_s + st * kATileBytes, &tmap_s, &full[st], kb * kBK, s0);
+        tma_load_2d(a_s + st * kATileBytes + kBoxBytes, &tmap_s, &full[st], kb * kBK, s0 + 128);
+        tma_load_2d(b_s + st * kBTileBytes, &tmap_e, &full[st], kb * kBK, e0);
+        tma_load_2d(b_s + st * kBTileBytes + kBoxBytes, &tmap_e, &full[st], kb * kBK, e0 + 128);
         issued = kb + 1;
       }
       // the last load issued into each stage has landed before the CTA exits
@@ -107,28 +117,31 @@ __global__ void __launch_bounds__(cs::kThreads, 2)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk)
-          mma_ss(tmem, sw128_desc(a_addr + st * kTileBytes + kk * 32, 16, 1024),
-                 sw128_desc(b_addr + st * kTileBytes + kk * 32, 16, 1024), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int mt = 0; mt < kMT; ++mt)
+            mma_ss(tmem + mt * kBN, sw128_desc(a_addr + st * kATileBytes + mt * kBoxBytes + kk * 32, 16, 1024),
+                   sw128_desc(b_addr + st * kBTileBytes + kk * 32, 16, 1024), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&empty[st]);
       }
       mma_commit(acc_full);
       volatile int never = 0;
       mbar_wait_bounded(acc_full, 0, &never, err);
     }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------------ epilogue
-    const int et = threadIdx.x - 64;                    // 0..127
+    const int et = threadIdx.x - 128;                   // 0..255
     inv_e_s[et] = e0 + et < n_elig ? inv_ne[e0 + et] : 0.f;
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    const int wq = warp & 3;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    const int mt = (warp - 4) >> 2;                     // accumulator of this warp
+    const int wq = warp & 3;                            // its TMEM lane quadrant
     const int row = wq * 32 + lane;
-    const int i = s0 + row;
+    const int i = s0 + mt * kBM + row;
     const float inv_s = i < n_src ? inv_ns[i] : 0.f;
     float t0 = -INFINITY, t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY;
     int j0 = 0x7fffffff, j1 = 0x7fffffff, j2 = 0x7fffffff, j3 = 0x7fffffff;
     if (__all_sync(0xffffffffu, mbar_wait_bounded(acc_full, 0, abort_flag, err))) {
       tc_fence_after();
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+      const uint32_t taddr = tmem + mt * kBN + (static_cast<uint32_t>(wq * 32) << 16);
 #pragma unroll 1
       for (int q = 0; q < kBN / 32; ++q) {
         uint32_t v[32];
@@ -305,7 +318,7 @@ cudaError_t launch_merge_targets(cudaStream_t s, const __nv_bfloat16* ks, const 
   if (ea != cudaSuccess) return ea;
   CUtensorMap ts, te;
   if (!encode_keys_tmap(&ts, ks, n_src, HD) || !encode_keys_tmap(&te, ke, n_elig, HD)) return cudaErrorInvalidValue;
-  dim3 grid((n_elig + cs::kBN - 1) / cs::kBN, (n_src + cs::kBM - 1) / cs::kBM);
+  dim3 grid((n_elig + cs::kBN - 1) / cs::kBN, (n_src + cs::kMT * cs::kBM - 1) / (cs::kMT * cs::kBM));
   cos_screen_kernel<<<grid, cs::kThreads, cs::kSmemBytes, s>>>(ts, te, inv_ns, inv_ne, n_src, n_elig, HD, top_v,
                                                                top_j, tiles_n, err);
   cudaError_t e = cudaGetLastError();
