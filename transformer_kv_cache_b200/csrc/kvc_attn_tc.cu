@@ -93,13 +93,18 @@ constexpr int kOnesBytes = kHalfBytes;        // bf16 ones: the row-sum block of
 constexpr int kThreads = 384;                 // 3 warpgroups
 constexpr int kRegsLow = 56, kRegsHigh = 224;  // after the split: 128 x 56 + 256 x 224 <= 384 x 168
 constexpr int kTmemCols = 512;
-// TMEM columns of query tile i, from 256 i: Q (bf16 pairs), S buffers 0 and 1 (fp32; P as
-// bf16 pairs over the first 32 columns of its buffer), O' (fp32)
-constexpr int kColQ = 0, kColS = 32, kColO = 160;
+// TMEM columns of query tile i, from 256 i: Q (bf16 pairs), the A operand of the mask
+// product (8 columns: 1 in each row's first element), S buffers 0 and 1 (fp32; P as bf16
+// pairs over the first 32 columns of its buffer), O' (fp32)
+constexpr int kColQ = 0, kColQb = 32, kColS = 40, kColO = 168;
 __host__ __device__ constexpr int col_base(int i) { return 256 * i; }
 constexpr float kLog2PMax = 8.0f;             // a P above 2^8 moves the row's reference max
 constexpr int kPolyPer8 = 3;                  // of every 8 column pairs, the 2^x on the FMA pipe
-constexpr size_t kSmemBytes = 1024 + 2 * kStages * kTileBytes + kOnesBytes + 512;
+// bf16 storage: per stage and half, the B operand of the mask product (64 slots x 16 bf16,
+// 32-byte rows: the slot's bias in its first element, 0 or kMaskBias)
+constexpr int kBiasHalfBytes = kBH * 32;
+constexpr uint16_t kMaskBias = 0xF180;        // bf16 -2^100
+constexpr size_t kSmemBytes = 1024 + 2 * kStages * kTileBytes + kOnesBytes + kStages * 2 * kBiasHalfBytes + 512;
 // E4M3 storage: a fourth warpgroup widens the codes of each KV tile into the f16 operand
 // ring; the codes land by TMA in a ring of their own
 constexpr int kThreads8 = 512;
@@ -395,7 +400,8 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
   uint8_t* k_s = smem;                                   // [stage][128 rows][128 B]
   uint8_t* v_s = k_s + kS * kTileBytes;
   uint8_t* ones_s = v_s + kS * kTileBytes;               // after every V stage: a positive offset
-  uint8_t* codes = ones_s + kOnesBytes;                  // E4M3: [code stage][K, V][128 rows][64 B]
+  uint8_t* bias_s = ones_s + kOnesBytes;                 // bf16: [stage][half][64 slots][32 B]
+  uint8_t* codes = bias_s + (kF8 ? 0 : kS * 2 * kBiasHalfBytes);   // E4M3: [code stage][K, V][128 rows][64 B]
   // E4M3, per operand stage (written by the converters with the tile's K, read by the
   // softmax): the valid slots and K scales of the tile's 8 pages, the piece's V reference
   int* meta_valid = reinterpret_cast<int*>(codes + (kF8 ? 2 * kCodeStages * kCodeTileBytes : 0));   // [kS][8]
@@ -420,7 +426,8 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
   uint64_t* code_empty = code_full + kCodeStages;   // E4M3: a code stage read (the 4 converters)
   uint64_t* vref_bar = code_empty + kCodeStages;    // E4M3: [piece & 1] partial V maxima written
   float* vref_part = reinterpret_cast<float*>(vref_bar + 2);   // [piece & 1][converter]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(vref_part + 8);
+  uint64_t* bias_pack = reinterpret_cast<uint64_t*>(vref_part + 8);   // bf16: [stage] valid slots its mask rows hold
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bias_pack + kS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -463,6 +470,16 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
   const uint32_t one2 = kF8 ? 0x3c003c00u : 0x3f803f80u;
   for (int i = threadIdx.x; i < kOnesBytes / 16; i += (kF8 ? kThreads8 : kThreads))
     reinterpret_cast<uint4*>(ones_s)[i] = make_uint4(one2, one2, one2, one2);
+  if (!kF8) {
+    // every slot of every stage starts unmasked (all pages full)
+    for (int i = threadIdx.x; i < kS * 2 * kBiasHalfBytes / 16; i += kThreads)
+      reinterpret_cast<uint4*>(bias_s)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = threadIdx.x; i < kS; i += kThreads) {
+      uint64_t full = 0;                          // every page P valid slots, packed 5 bits a page
+      for (int q = 0; q < kPPT; ++q) full |= static_cast<uint64_t>(P) << (5 * q);
+      bias_pack[i] = full;
+    }
+  }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -493,15 +510,21 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
         const Entry* ent = kPerHead ? la.entries + hp : la.entries;
         const int n_pages = la.n_pages;
         const long long page_base = la.page_base;
+        // physical page of each page of the next tile (past the list: -1) and, packed 5 bits
+        // a page, their valid slots (past the list: 0)
         int phys_next[kPPT];
+        uint64_t vpack_next = 0;
 #pragma unroll
         for (int q = 0; q < kPPT; ++q) {
           const int idx = t0 * kPPT + q;
-          phys_next[q] = idx < n_pages ? __ldg(&ent[idx].x) : -1;
+          const int4 en = idx < n_pages ? __ldg(&ent[idx]) : make_int4(-1, 0, 0, 0);
+          phys_next[q] = en.x;
+          vpack_next |= static_cast<uint64_t>(min(max(en.w, 0), P)) << (5 * q);
         }
         for (int t = t0; t < t1; ++t, ++jg) {
           const int st = jg % kRing;
           int row[kPPT];
+          const uint64_t vpack = vpack_next;
 #pragma unroll
           for (int q = 0; q < kPPT; ++q) {
             if (kPerHead)
@@ -510,10 +533,13 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
               row[q] = phys_next[q] >= 0 ? static_cast<int>(((page_base + phys_next[q]) * p.H + h) * P) : p.pool_rows;
           }
           if (t + 1 < t1) {
+            vpack_next = 0;
 #pragma unroll
             for (int q = 0; q < kPPT; ++q) {
               const int idx = (t + 1) * kPPT + q;
-              phys_next[q] = idx < n_pages ? __ldg(&ent[idx].x) : -1;
+              const int4 en = idx < n_pages ? __ldg(&ent[idx]) : make_int4(-1, 0, 0, 0);
+              phys_next[q] = en.x;
+              vpack_next |= static_cast<uint64_t>(min(max(en.w, 0), P)) << (5 * q);
             }
           }
           uint64_t* free_bar = kF8 ? &code_empty[st] : &kv_empty[st];
@@ -530,6 +556,28 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
             for (int q = 0; q < kPPT; ++q)
               tma_load_2d(cb + kCodeTileBytes + q * P * kHD, &tmap_v, &code_full[st], 0, row[q]);
           } else {
+            // the stage's mask rows: slot j of page q is masked (bias kMaskBias) iff j >= its
+            // valid count. The stage remembers the counts its rows hold (packed as the tile's
+            // are), and only rows whose state changes are written: nothing for a full tile
+            // after a full tile. Both 16-byte halves of a row start with the bias, so the
+            // 32-byte swizzle cannot move it out of the element the product reads.
+            const uint64_t held = bias_pack[st];
+            if (vpack != held) {
+              for (int q = 0; q < kPPT; ++q) {
+                const int vo = static_cast<int>((held >> (5 * q)) & 31u);
+                const int vn = static_cast<int>((vpack >> (5 * q)) & 31u);
+                if (vo != vn) {
+                  uint8_t* rows = bias_s + (st * 2 + q / kPPH) * kBiasHalfBytes + (q % kPPH) * P * 32;
+                  const uint16_t val = vn < vo ? kMaskBias : 0;
+                  for (int j = min(vo, vn); j < max(vo, vn); ++j) {
+                    *reinterpret_cast<uint16_t*>(rows + j * 32) = val;
+                    *reinterpret_cast<uint16_t*>(rows + j * 32 + 16) = val;
+                  }
+                }
+              }
+              bias_pack[st] = vpack;
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            }
             mbar_arrive_expect_tx(&k_full[st], kTileBytes);
 #pragma unroll
             for (int q = 0; q < kPPT; ++q)
@@ -565,6 +613,7 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
     const uint32_t idesc_o = idesc_f16kind(fmt, kBM, kON, 0, 1);
     const uint32_t tb = tmem + col_base(i);
     const uint32_t k_addr = smem_u32(k_s), v_addr = smem_u32(v_s), ones_addr = smem_u32(ones_s);
+    const uint32_t bias_addr = smem_u32(bias_s);
     const bool leader = elect_one();
     int ub = 0, pc = 0;                           // first half of the piece; pieces done
     // S of half uu (u: its index in the piece) into buffer uu & 1. Issued after the P.V
@@ -583,6 +632,9 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
         for (int kk = 0; kk < kHD / 16; ++kk)
           mma_ts(tb + kColS + hb * kBH, tb + kColQ + kk * 8, sw128_desc(kb + kk * 32, 16, 1024), idesc_s,
                  kk > 0 ? 1u : 0u);
+        // bf16: + 1 x the slots' bias (0, or -2^100 for slots past a page's valid count)
+        if (!kF8) mma_ts(tb + kColS + hb * kBH, tb + kColQb, sw32_desc(bias_addr + (st * 2 + hb) * kBiasHalfBytes, 256),
+                         idesc_s, 1u);
         mma_commit(&s_full[2 * i + hb]);
       }
       __syncwarp();
@@ -650,8 +702,6 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
     while (ok && next_piece(sw, lt, p.H, lay, h, t0, t1)) {
       const int nh = 2 * (t1 - t0);
       const LayerAttn& la = lt.l[lay];
-      const Entry* ent = kPerHead ? la.entries + static_cast<long long>(h) * p.head_pages : la.entries;
-      const int n_pages = la.n_pages;
       float row_fac = 1.f;       // E4M3: 2^-e of the query row's scaling into f16
       {
         // this row of Q (zeros past the last query) into TMEM, the A operand of S; the S
@@ -692,6 +742,11 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
           for (int v = 0; v < 32; ++v) qv[v] = 0u;
         }
         tmem_st32(tb + kColQ, qv);
+        if (!kF8) {
+          // A operand of the mask product: 1 in the row's first element
+          const uint32_t qb[8] = {0x3f80u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+          tmem_st8(tb + kColQb, qb);
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -699,15 +754,6 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
       }
       float m = -INFINITY;       // reference max (log2 domain) of the row
       float vref = 1.f;          // E4M3: the piece's V reference
-      // bf16: valid slots of the pages of the next half (every lane loads all of them)
-      int vnext[kPPH];
-      if (!kF8) {
-#pragma unroll
-        for (int q = 0; q < kPPH; ++q) {
-          const int idx = t0 * kPPT + q;
-          vnext[q] = idx < n_pages ? __ldg(&ent[idx].w) : 0;
-        }
-      }
       for (int u = 0; u < nh; ++u) {
         const int uu = ub + u, hb = uu & 1, jj = uu >> 1;
         int vcur[kPPH];
@@ -739,19 +785,8 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
           cq[2] = fmaxf(crow * ks4.z, 1e-30f);
           cq[3] = fmaxf(crow * ks4.w, 1e-30f);
         } else {
+          // bf16: slots past a page's valid count were masked inside S by the mask product
           cq[0] = c;
-#pragma unroll
-          for (int q = 0; q < kPPH; ++q) {
-            vcur[q] = vnext[q];
-            partial |= vcur[q] < P;
-          }
-          if (u + 1 < nh) {
-#pragma unroll
-            for (int q = 0; q < kPPH; ++q) {
-              const int idx = t0 * kPPT + (u + 1) * kPPH + q;
-              vnext[q] = idx < n_pages ? __ldg(&ent[idx].w) : 0;
-            }
-          }
         }
         uint32_t s[kBH];
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s_full[2 * wg + hb], jj & 1, abort_flag, p.err))) {
@@ -762,8 +797,8 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
         tmem_ld32(tb + kColS + hb * kBH, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
         tmem_ld32(tb + kColS + hb * kBH + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
         tmem_ld_wait();
-        if (partial) {
-          // slots past a page's valid count (and pages past the list end) take no weight
+        if (kF8 && partial) {
+          // E4M3: slots past a page's valid count (and pages past the list end) take no weight
 #pragma unroll
           for (int cc = 0; cc < kBH; ++cc)
             if ((cc % P) >= vcur[cc / P]) s[cc] = __float_as_uint(-INFINITY);

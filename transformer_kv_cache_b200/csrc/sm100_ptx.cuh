@@ -192,6 +192,10 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
       KVC_W8(0), KVC_W8(8)
       : "memory");
 }
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), KVC_W8(0)
+               : "memory");
+}
 #undef KVC_R8
 #undef KVC_W8
 
@@ -205,6 +209,20 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1) << 46;
   d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+// Shared-memory matrix descriptor for a K-major operand 16 elements (32 bytes) wide with the
+// 32-byte swizzle: rows 32 bytes apart, 8-row groups sbo_bytes apart (the leading offset is
+// unused), version 1, base offset 0, layout type SWIZZLE_32B (6). The swizzle moves a row's
+// two 16-byte halves only within the row's 32 bytes.
+__device__ __forceinline__ uint64_t sw32_desc(uint32_t saddr, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(6) << 61;
   return d;
 }
 
