@@ -34,7 +34,8 @@
 //                       pairs and written over the first 32 columns of the half's own S
 //                       buffer.
 //
-// TMEM per query tile (240 of 256 columns): Q (32: bf16 pairs), two S buffers (64 each;
+// TMEM per query tile (248 of 256 columns): Q (32: bf16 pairs), the mask product's A
+// operand (8), two S buffers (64 each;
 // half u uses buffer u & 1, and its P goes over the buffer's first 32 columns once its S is
 // in registers), O' (80). The issuer keeps S one half ahead of the softmax: after the P.V
 // product of half u it issues S of half u + 2 into the same buffer (one issuer's MMAs run
@@ -49,8 +50,16 @@
 // after the previous half's P.V has completed.
 //
 // Partial pages: slots past a page's valid count hold K = V = 0 (the append and compaction
-// kernels write zeros there) and their scores are set to -inf before the softmax, in the
-// tiles that have such slots; pages past the end of the list are masked the same way.
+// kernels write zeros there); pages past the end of the list are read as zeros. Such slots
+// must take no weight. With bf16 storage S carries the mask itself: one more K=16 MMA per
+// S tile adds 1 x bias, where the A operand is a TMEM block holding 1 in each row's first
+// element and the B operand a per-stage, per-half shared-memory block (64 slots x 16 bf16,
+// 32-byte swizzle) holding -2^100 for masked slots and 0 elsewhere. The TMA producer keeps
+// these blocks current from the page entries it already loads, rewriting only the rows
+// whose state changes (none between two full tiles). A masked score is then about
+// -2^100 x the logit factor and its P rounds to 0 (2^-126 on the FMA-pipe path, as for a
+// -inf score), so the softmax needs no page metadata. With E4M3 storage the per-page logit
+// factors can be tiny, so the softmax sets those scores to -inf from the stage metadata.
 //
 // E4M3 storage ("XStreamVGGT" abstract: KV cache quantisation; codes with one absmax scale
 // per (page, head), or per K channel and V token with the dimension-adaptive scales). The
