@@ -579,8 +579,7 @@ def run_workload(args):
             kvc.kvc_attend_all(h, [pool[l][i][0] for l in range(L)], outs)
             if ev: ev[2].record(stream)
             if budget:
-                for l in range(L):
-                    fired += kvc.kvc_compress(h, l, res[l][i])
+                fired += sum(kvc.kvc_compress_all(h, [res[l][i] for l in range(L)]))
             if ev: ev[3].record(stream)
             return key, fired
 

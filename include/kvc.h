@@ -247,6 +247,17 @@ KVC_API kvc_status kvc_scale_phase(kvc_cache* c, int32_t layer, int32_t n_frames
  * KVC_ERR_BUDGET (protected tokens exceed the keep tier). */
 KVC_API kvc_status kvc_compress(kvc_cache* c, int32_t layer, const float* residual_dev, int32_t* fired_out);
 
+/* kvc_compress on every layer of the frame just attended: residual_devs[l] is layer l's
+ * [T, R] fp32 residual (device); fired_out (host, num_layers int32, may be NULL) receives
+ * per layer 1 when a compression ran. Results, page tables and metadata are those of
+ * kvc_compress on layers 0, 1, ... in order. Every layer is scored first, in order (the
+ * CLCES rank window spans layers); the layers over budget are then compressed side by side
+ * on the cache's side streams (each with its own scratch), joined back into the cache's
+ * stream before the call returns. kvc_last_raw_scores afterwards gives the last layer's
+ * raw scores. Errors: those of kvc_compress (the first one met); KVC_ERR_ARG for a NULL
+ * array or residual. */
+KVC_API kvc_status kvc_compress_all(kvc_cache* c, const float* const* residual_devs, int32_t* fired_out);
+
 /* Synchronise and copy the page table of `layer` to host: rows of 4 int32
  * (owner, page_in_owner, phys_page, valid_tokens) in cache order; owner is the
  * frame index, or -1 for pages written by compaction. Writes at most

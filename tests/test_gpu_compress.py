@@ -158,3 +158,67 @@ def test_budget_call_order_errors(kvc):
         kvc.kvc_compress(h, 0, st.residual(0, 0))        # layer 0 after layer 1 in the same frame
     assert e.value.status_name == "KVC_ERR_STATE"
     kvc.kvc_destroy(h)
+
+
+def run_pair(kvc, wl, frames, full_shape_rows=None):
+    """Two caches fed the same stream: one compresses with kvc_compress on each layer in
+    order, the other with kvc_compress_all (layers scored in order, then compressed side by
+    side on the side streams). Their state must agree bit for bit after every frame: token
+    ids, merge counts, s_hat, page tables, merge pairs and the stored K and V. Returns the
+    number of compression events."""
+    dev = torch.device("cuda")
+    L, T, H, D, P = wl.num_layers, wl.tokens_per_frame, wl.num_heads, wl.head_dim, wl.page_size
+    ha = kvc.kvc_create(kvc.config_from_workload(wl))
+    hb = kvc.kvc_create(kvc.config_from_workload(wl))
+    events = 0
+    try:
+        st = FrameStream(wl, seed=5, device=dev)
+        oa = [torch.empty((T, H, D), dtype=torch.bfloat16, device=dev) for _ in range(L)]
+        ob = [torch.empty((T, H, D), dtype=torch.bfloat16, device=dev) for _ in range(L)]
+        for t in range(frames):
+            qkv = [st.frame(l, t) for l in range(L)]
+            res = [st.residual(l, t) for l in range(L)]
+            for h, outs in ((ha, oa), (hb, ob)):
+                kvc.kvc_append_frame_all(h, t, [x[1] for x in qkv], [x[2] for x in qkv], True)
+                kvc.kvc_attend_all(h, [x[0] for x in qkv], outs)
+            fired_a = [kvc.kvc_compress(ha, l, res[l]) for l in range(L)]
+            fired_b = kvc.kvc_compress_all(hb, res)
+            assert fired_a == fired_b, (t, fired_a, fired_b)
+            events += sum(fired_b)
+            torch.cuda.synchronize()
+            for l in range(L):
+                assert torch.equal(oa[l], ob[l]), f"outputs differ at frame {t} layer {l}"
+                for a, b, what in zip(kvc.kvc_token_meta(ha, l, 1 << 16), kvc.kvc_token_meta(hb, l, 1 << 16),
+                                      ("ids", "counts", "s_hat")):
+                    assert np.array_equal(a, b), f"{what} differ at frame {t} layer {l}"
+                pa, ia = kvc.kvc_page_table(ha, l)
+                pb, ib = kvc.kvc_page_table(hb, l)
+                assert np.array_equal(pa, pb), f"page table differs at frame {t} layer {l}"
+                assert ia["device_error"] == 0 and ib["device_error"] == 0
+                if fired_b[l]:
+                    sa, da = kvc.kvc_last_merge(ha, l, 1 << 15)
+                    sb, db = kvc.kvc_last_merge(hb, l, 1 << 15)
+                    assert np.array_equal(sa, sb) and np.array_equal(da, db), f"merges differ at frame {t} layer {l}"
+                    n = len(pa)
+                    ka, va, _, _ = kvc.kvc_export_pages(ha, l, 0, n, H * P * D * 2, H)
+                    kb, vb, _, _ = kvc.kvc_export_pages(hb, l, 0, n, H * P * D * 2, H)
+                    assert np.array_equal(ka, kb) and np.array_equal(va, vb), f"pages differ at frame {t} layer {l}"
+        return events
+    finally:
+        kvc.kvc_destroy(ha)
+        kvc.kvc_destroy(hb)
+
+
+def test_compress_all_matches_per_layer_calls(kvc):
+    """Six layers (more than the four side streams, so two layers share a stream and its
+    scratch in one call), ragged pages, special tokens, several events per layer."""
+    wl = WORKLOADS["vggt_budget_16k"].replace(tokens_per_frame=45, num_heads=4, budget_tokens=300, num_layers=6,
+                                               residual_dim=64, num_special_tokens=3)
+    assert run_pair(kvc, wl, 16) >= 18
+
+
+def test_compress_all_matches_per_layer_calls_full_shape(kvc):
+    """Full 1004-token / 16-head / B = 16384 layers, 5 of them, through one compression event
+    each."""
+    wl = WORKLOADS["vggt_budget_16k"].replace(num_layers=5)
+    assert run_pair(kvc, wl, 18) >= 5

@@ -26,7 +26,7 @@ STATUS = ["KVC_OK", "KVC_ERR_ARG", "KVC_ERR_OOM", "KVC_ERR_CUDA", "KVC_ERR_STATE
 # every symbol include/kvc.h declares
 EXPORTS = ["kvc_create", "kvc_destroy", "kvc_set_stream", "kvc_reset", "kvc_append_frame", "kvc_attend",
            "kvc_attend_all", "kvc_prune_all",
-           "kvc_compress", "kvc_page_table", "kvc_token_meta", "kvc_last_merge", "kvc_export_pages",
+           "kvc_compress", "kvc_compress_all", "kvc_page_table", "kvc_token_meta", "kvc_last_merge", "kvc_export_pages",
            "kvc_step_host", "kvc_synchronize", "kvc_last_error", "kvc_status_string", "kvc_version",
            "kvc_debug_fail_allocs", "kvc_debug_bounded_wait", "kvc_attend_paged_noalloc", "kvc_append_frame_all",
            "kvc_step_host_async", "kvc_set_layer_budgets", "kvc_prune", "kvc_layer_diversity",
@@ -81,6 +81,7 @@ def _load():
         "kvc_append_frame_all": ([vp, i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32], i32),
         "kvc_attend_all": ([vp, ctypes.POINTER(vp), ctypes.POINTER(vp)], i32),
         "kvc_compress": ([vp, i32, vp, i32p], i32),
+        "kvc_compress_all": ([vp, ctypes.POINTER(vp), i32p], i32),
         "kvc_page_table": ([vp, i32, i32p, i32, i32p, ctypes.POINTER(kvc_info)], i32),
         "kvc_token_meta": ([vp, i32, i64p, i32p, fp, i32, i32p], i32),
         "kvc_last_merge": ([vp, i32, i64p, i64p, i32, i32p], i32),
@@ -231,6 +232,16 @@ def kvc_compress(handle, layer: int, residual) -> bool:
     fired = ctypes.c_int32(0)
     _check(handle, _lib.kvc_compress(handle, layer, _ptr(residual), ctypes.byref(fired)))
     return bool(fired.value)
+
+
+def kvc_compress_all(handle, residuals) -> list:
+    """residuals: per-layer device fp32 tensors (or pointers), one per layer of the cache.
+    Returns, per layer, whether a compression ran."""
+    n = len(residuals)
+    ra = (ctypes.c_void_p * n)(*[_ptr(r) for r in residuals])
+    fired = (ctypes.c_int32 * n)()
+    _check(handle, _lib.kvc_compress_all(handle, ra, fired))
+    return [bool(f) for f in fired]
 
 
 def kvc_page_table(handle, layer: int):

@@ -57,6 +57,11 @@ void free_all(kvc_cache* c) {
   }
   if (c->copy_up) cudaStreamDestroy(c->copy_up);
   if (c->copy_down) cudaStreamDestroy(c->copy_down);
+  for (int i = 0; i < kvc_cache::kCmpSets; ++i) {
+    if (c->cmp_stream[i]) cudaStreamDestroy(c->cmp_stream[i]);
+    if (c->cmp_join[i]) cudaEventDestroy(c->cmp_join[i]);
+  }
+  if (c->cmp_fork) cudaEventDestroy(c->cmp_fork);
 }
 
 kvc_status fail(kvc_cache* c, kvc_status s, const char* msg) {
@@ -171,6 +176,7 @@ kvc_status evict_frame(kvc_cache* c, int layer, const FrameRec& f) {
 namespace kvc {
 // Budget-mode helpers live in kvc_compress.cu.
 kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_t* fired);
+kvc_status compress_all_layers(kvc_cache* c, const float* const* residuals, int32_t* fired);
 kvc_status init_token_meta(kvc_cache* c, int layer, int first_entry, int n_pages, int frame);
 size_t compress_scratch_bytes(const kvc_config& cfg, int pool_pages);
 }  // namespace kvc
@@ -344,7 +350,12 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
     A(dev_alloc_t(&c->tok_shat, slots * sizeof(float)));
     A(dev_alloc_t(&c->rank_hist, static_cast<size_t>(g.rank_window) * T * sizeof(int32_t)));
     c->cmp_scratch_bytes = compress_scratch_bytes(g, c->pool_pages);
-    A(dev_alloc(&c->cmp_scratch, c->cmp_scratch_bytes));
+    A(dev_alloc(&c->cmp_scratch, c->cmp_scratch_bytes * kvc_cache::kCmpSets));
+    for (int i = 0; i < kvc_cache::kCmpSets; ++i) {
+      A(cudaStreamCreateWithFlags(&c->cmp_stream[i], cudaStreamNonBlocking));
+      A(cudaEventCreateWithFlags(&c->cmp_join[i], cudaEventDisableTiming));
+    }
+    A(cudaEventCreateWithFlags(&c->cmp_fork, cudaEventDisableTiming));
   }
   if (e != cudaSuccess) {
     free_all(c);
@@ -997,6 +1008,18 @@ kvc_status kvc_compress(kvc_cache* c, int32_t layer, const float* residual_dev, 
   if (c->cfg.budget_tokens <= 0) return fail(c, KVC_ERR_ARG, "kvc_compress: budget_tokens is 0");
   if (!residual_dev) return fail(c, KVC_ERR_ARG, "kvc_compress: residual is NULL");
   return compress_layer(c, layer, residual_dev, fired_out);
+}
+
+kvc_status kvc_compress_all(kvc_cache* c, const float* const* residual_devs, int32_t* fired_out) {
+  if (!c) return KVC_ERR_ARG;
+  const kvc_config& g = c->cfg;
+  if (g.budget_tokens <= 0) return fail(c, KVC_ERR_ARG, "kvc_compress_all: budget_tokens is 0");
+  if (!residual_devs) return fail(c, KVC_ERR_ARG, "kvc_compress_all: NULL residual array");
+  for (int l = 0; l < g.num_layers; ++l) {
+    if (fired_out) fired_out[l] = 0;
+    if (!residual_devs[l]) return fail(c, KVC_ERR_ARG, "kvc_compress_all: a residual is NULL");
+  }
+  return compress_all_layers(c, residual_devs, fired_out);
 }
 
 kvc_status kvc_page_table(kvc_cache* c, int32_t layer, int32_t* rows_host, int32_t capacity, int32_t* n_rows,

@@ -932,7 +932,21 @@ kvc_status init_token_meta(kvc_cache* c, int layer, int first_entry, int n_pages
   return KVC_OK;
 }
 
-kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_t* fired) {
+// Scratch set i (of kCmpSets); the raw scores and the merge records always live in set 0.
+Scratch scratch_set(kvc_cache* c, int i) {
+  Scratch s0, si;
+  uint8_t* base = static_cast<uint8_t*>(c->cmp_scratch);
+  carve(c->cfg, base, &s0);
+  carve(c->cfg, base + static_cast<size_t>(i) * c->cmp_scratch_bytes, &si);
+  si.s_raw = s0.s_raw;
+  si.last_src = s0.last_src;
+  si.last_dst = s0.last_dst;
+  return si;
+}
+
+// Scoring of the frame just committed on `layer` (raw score, CLCES rank, s_hat), on the
+// cache's stream with scratch set 0. Layers of a frame come in ascending order.
+kvc_status score_layer(kvc_cache* c, int layer, const float* residual) {
   const kvc_config& g = c->cfg;
   LayerHost& L = c->L[layer];
   if (L.has_pending || L.frames.empty() || L.frames.back().frame != L.last_frame) {
@@ -954,10 +968,8 @@ kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_
     c->last_error = "kvc_compress: layers of a frame must be scored in ascending order";
     return KVC_ERR_STATE;
   }
-  Scratch sc;
-  carve(g, static_cast<uint8_t*>(c->cmp_scratch), &sc);
-  const Caps cp = caps_of(g);
-  const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads, D = g.head_dim;
+  const Scratch sc = scratch_set(c, 0);
+  const int T = g.tokens_per_frame, P = g.page_size;
   const int RW = g.rank_window;
   const size_t lay_slots = static_cast<size_t>(layer) * c->pool_pages * P;
   Entry* E = c->entries + static_cast<size_t>(layer) * c->pool_pages;
@@ -990,10 +1002,25 @@ kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_
     c->last_error = std::string("kvc_compress scoring: ") + cudaGetErrorString(e);
     return KVC_ERR_CUDA;
   }
-  const int B = g.budget_tokens;
-  if (L.tokens <= B) return KVC_OK;
+  return KVC_OK;
+}
 
-  // ---- compression
+// Compression of a layer over its budget, on stream s with scratch set sc (no other
+// compression may use sc meanwhile). Host checks come before any launch.
+kvc_status compress_body(kvc_cache* c, int layer, cudaStream_t s, const Scratch& sc, int32_t* fired) {
+  const kvc_config& g = c->cfg;
+  LayerHost& L = c->L[layer];
+  const Caps cp = caps_of(g);
+  const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads, D = g.head_dim;
+  const size_t lay_slots = static_cast<size_t>(layer) * c->pool_pages * P;
+  Entry* E = c->entries + static_cast<size_t>(layer) * c->pool_pages;
+  cudaError_t e = cudaSuccess;
+  auto ok = [&]() {
+    cudaError_t r = cudaGetLastError();
+    if (r != cudaSuccess && e == cudaSuccess) e = r;
+    c->launches++;
+  };
+  const int B = g.budget_tokens;
   const int N = static_cast<int>(L.tokens);
   const int n_keep = static_cast<int>(cp.n_keep);
   const int n_merge_cap = B - n_keep;
@@ -1098,6 +1125,56 @@ kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_
   L.high_water = std::max<int64_t>(L.high_water, n_old + n_new);
   if (fired) *fired = 1;
   return KVC_OK;
+}
+
+kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_t* fired) {
+  kvc_status st = score_layer(c, layer, residual);
+  if (st != KVC_OK) return st;
+  if (c->L[layer].tokens <= c->cfg.budget_tokens) return KVC_OK;
+  return compress_body(c, layer, c->stream, scratch_set(c, 0), fired);
+}
+
+// Every layer scored in ascending order on the cache's stream (the CLCES rank window
+// spans layers), then the layers over budget compressed side by side: layer k of them on
+// side stream k mod kCmpSets with scratch set k mod kCmpSets, forked from and joined back
+// into the cache's stream. A layer's compression reads and writes only that layer's pages,
+// page table, token metadata and free bitmap, so the layers are independent.
+kvc_status compress_all_layers(kvc_cache* c, const float* const* residuals, int32_t* fired) {
+  const kvc_config& g = c->cfg;
+  for (int l = 0; l < g.num_layers; ++l) {
+    if (fired) fired[l] = 0;
+    kvc_status st = score_layer(c, l, residuals[l]);
+    if (st != KVC_OK) return st;
+  }
+  int todo[64];
+  int n = 0;
+  for (int l = 0; l < g.num_layers && n < 64; ++l)
+    if (c->L[l].tokens > g.budget_tokens) todo[n++] = l;
+  if (n == 0) return KVC_OK;
+  const int sets = std::min(n, static_cast<int>(kvc_cache::kCmpSets));
+  cudaError_t e = cudaEventRecord(c->cmp_fork, c->stream);
+  for (int i = 0; i < sets && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(c->cmp_stream[i], c->cmp_fork, 0);
+  if (e != cudaSuccess) {
+    c->last_error = std::string("kvc_compress_all fork: ") + cudaGetErrorString(e);
+    return KVC_ERR_CUDA;
+  }
+  kvc_status first = KVC_OK;
+  for (int k = 0; k < n; ++k) {
+    const int i = k % sets;
+    kvc_status st = compress_body(c, todo[k], c->cmp_stream[i], scratch_set(c, i), fired ? &fired[todo[k]] : nullptr);
+    if (st != KVC_OK && first == KVC_OK) first = st;
+  }
+  // join every side stream back, whatever happened above
+  for (int i = 0; i < sets; ++i) {
+    cudaError_t r = cudaEventRecord(c->cmp_join[i], c->cmp_stream[i]);
+    if (r == cudaSuccess) r = cudaStreamWaitEvent(c->stream, c->cmp_join[i], 0);
+    if (r != cudaSuccess && e == cudaSuccess) e = r;
+  }
+  if (e != cudaSuccess && first == KVC_OK) {
+    c->last_error = std::string("kvc_compress_all join: ") + cudaGetErrorString(e);
+    first = KVC_ERR_CUDA;
+  }
+  return first;
 }
 
 }  // namespace kvc

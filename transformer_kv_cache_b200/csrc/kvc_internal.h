@@ -95,9 +95,15 @@ struct Cache {
   int64_t* tok_id = nullptr;
   int32_t* tok_cnt = nullptr;
   float* tok_shat = nullptr;
-  // compression scratch
+  // compression scratch: kCmpSets sets of cmp_scratch_bytes each; set 0 also holds the
+  // raw scores and the merge records that kvc_last_raw_scores and kvc_last_merge read.
+  // kvc_compress_all compresses layers on the side streams, set i on stream i.
+  static constexpr int kCmpSets = 4;
   void* cmp_scratch = nullptr;
   size_t cmp_scratch_bytes = 0;
+  cudaStream_t cmp_stream[kCmpSets] = {nullptr, nullptr, nullptr, nullptr};
+  cudaEvent_t cmp_fork = nullptr;
+  cudaEvent_t cmp_join[kCmpSets] = {nullptr, nullptr, nullptr, nullptr};
   // attention split scratch (partial O and log-sum-exp)
   float* k_chan = nullptr;          // dimension-adaptive FP8: [layer][page][head][D] K channel scales
   float* v_tok = nullptr;           // dimension-adaptive FP8: [layer][page][head][P] V token scales
