@@ -28,8 +28,8 @@
 //                       ones), so column 64 of O' is the exact row sum of the bf16 P used.
 //   warps 4-7, 8-11     softmax of query tile 0 and 1 (thread = query row = TMEM lane):
 //                       first the row of Q into TMEM, then per half the 64 scores from
-//                       TMEM, P = 2^(s*c - m) for 5 of every 8 column pairs on the MUFU
-//                       and for 3 on the FMA pipe (a cubic in the fraction, the integer
+//                       TMEM, P = 2^(s*c - m) for 6 of every 8 column pairs on the MUFU
+//                       and for 2 on the FMA pipe (a cubic in the fraction, the integer
 //                       part added to the exponent field), interleaved, rounded to bf16
 //                       pairs and written over the first 32 columns of the half's own S
 //                       buffer.
@@ -108,7 +108,7 @@ constexpr int kTmemCols = 512;
 constexpr int kColQ = 0, kColQb = 32, kColS = 40, kColO = 168;
 __host__ __device__ constexpr int col_base(int i) { return 256 * i; }
 constexpr float kLog2PMax = 8.0f;             // a P above 2^8 moves the row's reference max
-constexpr int kPolyPer8 = 3;                  // of every 8 column pairs, the 2^x on the FMA pipe
+constexpr int kPolyPer8 = 2;                  // of every 8 column pairs, the 2^x on the FMA pipe
 // bf16 storage: per stage and half, the B operand of the mask product (64 slots x 16 bf16,
 // 32-byte rows: the slot's bias in its first element, 0 or kMaskBias)
 constexpr int kBiasHalfBytes = kBH * 32;
