@@ -29,10 +29,11 @@ namespace {
 
 constexpr int kDivD = 64;
 
-// One frame into the per-head pages of a batch of layers: one thread per (layer, slot,
-// head) row of 64 dims, heads fastest (the source rows of a slot are contiguous). A slot
-// past T gets zeros and token id -1. The page-table entries [start, start + n_pages) of
-// every head were just written by the allocator.
+// One frame into the per-head pages of a batch of layers: eight lanes per (layer, slot,
+// head) row of 64 dims, one 16-byte chunk each, heads next (so a warp loads four heads of a
+// slot, 512 contiguous bytes, and writes four whole 128-byte rows). A slot past T gets zeros
+// and token id -1. The page-table entries [start, start + n_pages) of every head were just
+// written by the allocator.
 __global__ void __launch_bounds__(256) append_heads_kernel(AppendBatch in, int first_layer, LayerStarts starts,
                                                            int n_layers, uint4* k_pool, uint4* v_pool,
                                                            const Entry* __restrict__ entries_all,
@@ -40,36 +41,29 @@ __global__ void __launch_bounds__(256) append_heads_kernel(AppendBatch in, int f
                                                            int H, int P, long long frame_base) {
   griddep_wait();
   griddep_launch_dependents();
+  constexpr int kChunks = kDivD / 8;              // 16-byte chunks per row
   const int slots = n_pages * P;
-  const long long total = static_cast<long long>(n_layers) * slots * H;
+  const long long total = static_cast<long long>(n_layers) * slots * H * kChunks;
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int h = static_cast<int>(idx % H);
-    const long long rt = idx / H;
+    const int q = static_cast<int>(idx % kChunks);
+    const long long r = idx / kChunks;
+    const int h = static_cast<int>(r % H);
+    const long long rt = r / H;
     const int t = static_cast<int>(rt % slots);
     const int b = static_cast<int>(rt / slots);
     const long long sub = (static_cast<long long>(first_layer + b) * H + h) * pool_pages;
     const int phys = __ldg(&entries_all[sub + starts.start[b] + t / P].x);
-    const long long dst = ((sub + phys) * P + t % P) * (kDivD / 8);
-    uint4 kv[2][kDivD / 8];
+    const long long dst = ((sub + phys) * P + t % P) * kChunks + q;
+    uint4 kc = make_uint4(0, 0, 0, 0), vc = make_uint4(0, 0, 0, 0);
     if (t < T) {
-      const uint4* ks = static_cast<const uint4*>(in.k[b]) + (static_cast<long long>(t) * H + h) * (kDivD / 8);
-      const uint4* vs = static_cast<const uint4*>(in.v[b]) + (static_cast<long long>(t) * H + h) * (kDivD / 8);
-#pragma unroll
-      for (int q = 0; q < kDivD / 8; ++q) {
-        kv[0][q] = __ldg(ks + q);
-        kv[1][q] = __ldg(vs + q);
-      }
-    } else {
-#pragma unroll
-      for (int q = 0; q < kDivD / 8; ++q) kv[0][q] = kv[1][q] = make_uint4(0, 0, 0, 0);
+      const long long src = (static_cast<long long>(t) * H + h) * kChunks + q;
+      kc = __ldg(static_cast<const uint4*>(in.k[b]) + src);
+      vc = __ldg(static_cast<const uint4*>(in.v[b]) + src);
     }
-#pragma unroll
-    for (int q = 0; q < kDivD / 8; ++q) {
-      k_pool[dst + q] = kv[0][q];
-      v_pool[dst + q] = kv[1][q];
-    }
-    tok_id_all[(sub + phys) * P + t % P] = t < T ? frame_base + t : -1;
+    k_pool[dst] = kc;
+    v_pool[dst] = vc;
+    if (q == 0) tok_id_all[(sub + phys) * P + t % P] = t < T ? frame_base + t : -1;
   }
 }
 
@@ -544,10 +538,10 @@ cudaError_t launch_append_heads(cudaStream_t s, const AppendBatch& in, int first
                                 int64_t* tok_id_all, int pool_pages, int n_pages, int T, int H, int D, int P,
                                 int frame) {
   if (D != kDivD) return cudaErrorInvalidValue;
-  const long long total = static_cast<long long>(n_layers) * n_pages * P * H;
+  const long long total = static_cast<long long>(n_layers) * n_pages * P * H * (kDivD / 8);
   const int threads = 256;
   long long blocks = (total + threads - 1) / threads;
-  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks > 148 * 32) blocks = 148 * 32;
   return launch_pdl(append_heads_kernel, dim3(static_cast<int>(blocks)), dim3(threads), 0, s,
                     in, first_layer, starts, n_layers, static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool),
                     entries_all, tok_id_all, pool_pages, n_pages, T, H, P, static_cast<long long>(frame) * T);
