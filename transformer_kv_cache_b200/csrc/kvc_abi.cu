@@ -178,6 +178,7 @@ namespace kvc {
 kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_t* fired);
 kvc_status compress_all_layers(kvc_cache* c, const float* const* residuals, int32_t* fired);
 kvc_status init_token_meta(kvc_cache* c, int layer, int first_entry, int n_pages, int frame);
+kvc_status init_token_meta_layers(kvc_cache* c, const LayerStarts& st, int n_layers, int n_pages, int frame);
 size_t compress_scratch_bytes(const kvc_config& cfg, int pool_pages);
 }  // namespace kvc
 
@@ -712,6 +713,10 @@ kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const void* con
       if (e != cudaSuccess) return cuda_fail(c, e, "append (all layers)");
       c->launches++;
       for (int b = 0; b < nl; ++b) c->L[l0 + b].bm_alt = !c->L[l0 + b].bm_alt;
+      if (g.budget_tokens > 0) {
+        kvc_status ms = init_token_meta_layers(c, st, nl, n, frame_idx);
+        if (ms != KVC_OK) return ms;
+      }
       continue;
     }
     // FP8 storage or pages too large for the fused kernel: never on the fused path, so every
@@ -728,13 +733,13 @@ kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const void* con
                                c->pool_pages, n, T, g.num_heads, g.head_dim, P, c->d_err);
     if (e != cudaSuccess) return cuda_fail(c, e, "append (all layers)");
     c->launches++;
+    if (g.budget_tokens > 0) {
+      kvc_status ms = init_token_meta_layers(c, st, nl, n, frame_idx);
+      if (ms != KVC_OK) return ms;
+    }
   }
   for (int l = 0; l < g.num_layers; ++l) {
     LayerHost& L = c->L[l];
-    if (g.budget_tokens > 0) {
-      kvc_status st = init_token_meta(c, l, L.n_entries, n, frame_idx);
-      if (st != KVC_OK) return st;
-    }
     L.pending.frame = frame_idx;
     L.pending.first_entry = L.n_entries;
     L.pending.n_entries = n;

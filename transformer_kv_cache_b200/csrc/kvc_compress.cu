@@ -256,6 +256,24 @@ __global__ void meta_init_kernel(int64_t* tok_id, int32_t* tok_cnt, float* tok_s
   tok_shat[k] = 0.f;
 }
 
+// The same for a batch of layers, blockIdx.y the layer of the batch (st.first_layer + y),
+// its new entries starting at st.start[y].
+__global__ void meta_init_layers_kernel(int64_t* tok_id_all, int32_t* tok_cnt_all, float* tok_shat_all,
+                                        const Entry* entries_all, LayerStarts st, int pool_pages, int n_pages, int P,
+                                        int T, int frame) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n_pages * P) return;
+  const int layer = st.first_layer + static_cast<int>(blockIdx.y);
+  const size_t base = static_cast<size_t>(layer) * pool_pages * P;
+  const Entry* pages = entries_all + static_cast<size_t>(layer) * pool_pages + st.start[blockIdx.y];
+  const int g = idx / P, s = idx % P;
+  const int tok = g * P + s;
+  const size_t k = base + static_cast<size_t>(pages[g].x) * P + s;
+  tok_id_all[k] = tok < T ? static_cast<int64_t>(frame) * T + tok : -1;
+  tok_cnt_all[k] = tok < T ? 1 : 0;
+  tok_shat_all[k] = 0.f;
+}
+
 // Exclusive scan of v over the CTA (blockDim.x a multiple of 32, at most 1024); *total
 // receives the CTA-wide sum. s_warp holds 32 ints.
 __device__ __forceinline__ int cta_exclusive_scan(int v, int* s_warp, int* total) {
@@ -923,6 +941,20 @@ kvc_status init_token_meta(kvc_cache* c, int layer, int first_entry, int n_pages
   const int n = n_pages * P;
   meta_init_kernel<<<(n + 255) / 256, 256, 0, c->stream>>>(c->tok_id + base, c->tok_cnt + base, c->tok_shat + base,
                                                            pages, n_pages, P, c->cfg.tokens_per_frame, frame);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    c->last_error = std::string("token metadata: ") + cudaGetErrorString(e);
+    return KVC_ERR_CUDA;
+  }
+  c->launches++;
+  return KVC_OK;
+}
+
+kvc_status init_token_meta_layers(kvc_cache* c, const LayerStarts& st, int n_layers, int n_pages, int frame) {
+  const int P = c->cfg.page_size;
+  const int n = n_pages * P;
+  meta_init_layers_kernel<<<dim3((n + 255) / 256, n_layers), 256, 0, c->stream>>>(
+      c->tok_id, c->tok_cnt, c->tok_shat, c->entries, st, c->pool_pages, n_pages, P, c->cfg.tokens_per_frame, frame);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     c->last_error = std::string("token metadata: ") + cudaGetErrorString(e);
