@@ -162,10 +162,10 @@ def test_budget_call_order_errors(kvc):
 
 def run_pair(kvc, wl, frames, full_shape_rows=None):
     """Two caches fed the same stream: one compresses with kvc_compress on each layer in
-    order, the other with kvc_compress_all (layers scored in order, then compressed side by
-    side on the side streams). Their state must agree bit for bit after every frame: token
-    ids, merge counts, s_hat, page tables, merge pairs and the stored K and V. Returns the
-    number of compression events."""
+    order, the other with kvc_compress_all (every layer scored in two launches, then the
+    layers compressed side by side on the side streams). Their state must agree bit for
+    bit after every frame: raw scores, token ids, merge counts, s_hat, page tables, merge
+    pairs and the stored K and V. Returns the number of compression events."""
     dev = torch.device("cuda")
     L, T, H, D, P = wl.num_layers, wl.tokens_per_frame, wl.num_heads, wl.head_dim, wl.page_size
     ha = kvc.kvc_create(kvc.config_from_workload(wl))
@@ -184,6 +184,8 @@ def run_pair(kvc, wl, frames, full_shape_rows=None):
             fired_a = [kvc.kvc_compress(ha, l, res[l]) for l in range(L)]
             fired_b = kvc.kvc_compress_all(hb, res)
             assert fired_a == fired_b, (t, fired_a, fired_b)
+            # the last layer's raw scores
+            assert np.array_equal(kvc.kvc_last_raw_scores(ha), kvc.kvc_last_raw_scores(hb)), t
             events += sum(fired_b)
             torch.cuda.synchronize()
             for l in range(L):

@@ -58,6 +58,7 @@ struct Scratch {
   float* top_v;        // four best screened cosines per (source, target tile)
   int32_t* top_j;
   float* s_raw;        // raw scores of the frame being scored [T]
+  float* s_raw_all;    // raw scores of every layer of the frame [layers][T] (kvc_compress_all)
   int64_t* last_src;   // [layers][merge cap]
   int64_t* last_dst;
 };
@@ -115,6 +116,7 @@ size_t carve(const kvc_config& g, uint8_t* base, Scratch* s) {
   t.top_v = reinterpret_cast<float*>(take(c.n_merge * c.tiles * 16));
   t.top_j = reinterpret_cast<int32_t*>(take(c.n_merge * c.tiles * 16));
   t.s_raw = reinterpret_cast<float*>(take(static_cast<size_t>(g.tokens_per_frame) * 4));
+  t.s_raw_all = reinterpret_cast<float*>(take(static_cast<size_t>(g.num_layers) * g.tokens_per_frame * 4));
   t.last_src = reinterpret_cast<int64_t*>(take(static_cast<size_t>(g.num_layers) * c.n_merge * 8));
   t.last_dst = reinterpret_cast<int64_t*>(take(static_cast<size_t>(g.num_layers) * c.n_merge * 8));
   if (s) *s = t;
@@ -147,7 +149,7 @@ __device__ __forceinline__ __nv_bfloat16 f64_to_bf16_rne(double x) {
 // consecutive channels in ascending c, then the block sums in ascending block order. One
 // warp per token: lane b sums block b (its 32 channels are 8 float4 loads), lane 0 adds
 // the block sums in order; for more than 32 blocks the warp repeats per 32 blocks.
-__global__ void residual_norm_kernel(const float* __restrict__ r, int T, int R, float* __restrict__ s_out) {
+__device__ __forceinline__ void residual_norm_rows(const float* __restrict__ r, int T, int R, float* __restrict__ s_out) {
   const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= T) return;
@@ -188,6 +190,17 @@ __global__ void residual_norm_kernel(const float* __restrict__ r, int T, int R, 
     }
   }
   if (lane == 0) s_out[row] = __double2float_rn(__dsqrt_rn(acc));
+}
+__global__ void residual_norm_kernel(const float* __restrict__ r, int T, int R, float* __restrict__ s_out) {
+  residual_norm_rows(r, T, R, s_out);
+}
+// Every layer of a frame in one launch, blockIdx.y the layer.
+struct ResidualBatch {
+  const float* r[kMaxBatchLayers];
+};
+__global__ void residual_norm_layers_kernel(const __grid_constant__ ResidualBatch rb, int T, int R,
+                                            float* __restrict__ s_all) {
+  residual_norm_rows(rb.r[blockIdx.y], T, R, s_all + static_cast<long long>(blockIdx.y) * T);
 }
 
 // Ranks of the frame's T tokens (s descending, ties to the lower slot), stored in the
@@ -239,6 +252,60 @@ __global__ void __launch_bounds__(128) clces_kernel(const float* __restrict__ s,
     const int g = i / P;
     const int phys = frame_pages[g].x;
     tok_shat_layer[static_cast<long long>(phys) * P + (i % P)] = __double2float_rn(w);
+  }
+}
+
+// CLCES of every layer of a frame in one launch (layers scored in order in one call): a
+// CTA carries its kClcesTokens tokens through the layers in order, keeping their ranks of
+// the last RW layers in shared memory, since a token's Cons needs only its own ranks. The
+// arithmetic per (layer, token) is clces_kernel's (ranks by counting, integer window sums,
+// the same fp64 operations).
+__global__ void __launch_bounds__(128) clces_layers_kernel(const float* __restrict__ s_all, int T, int n_layers,
+                                                            int RW, float lam, const Entry* __restrict__ entries_all,
+                                                            LayerStarts fr, int pool_pages, int P,
+                                                            float* __restrict__ tok_shat_all) {
+  extern __shared__ float s_sm[];
+  __shared__ int rk[32][kClcesTokens];          // [layer % RW][token of the CTA]
+  const int sub = threadIdx.x & 7, tl = static_cast<int>(threadIdx.x >> 3);
+  const int i = blockIdx.x * kClcesTokens + tl;
+  const double sqrt12 = __dsqrt_rn(12.0);
+  const double lamd = static_cast<double>(lam);
+  for (int l = 0; l < n_layers; ++l) {
+    __syncthreads();                            // the previous layer's scores are no longer read
+    const float* s = s_all + static_cast<long long>(l) * T;
+    for (int j = threadIdx.x; j < T; j += blockDim.x) s_sm[j] = s[j];
+    __syncthreads();
+    int r = 0;
+    if (i < T) {
+      const float si = s_sm[i];
+      for (int j = sub; j < T; j += 8) {
+        const float sj = s_sm[j];
+        r += (sj > si) || (sj == si && j < i);
+      }
+    }
+    r += __shfl_xor_sync(0xffffffffu, r, 1);
+    r += __shfl_xor_sync(0xffffffffu, r, 2);
+    r += __shfl_xor_sync(0xffffffffu, r, 4);
+    if (i < T && sub == 0) {
+      rk[l % RW][tl] = r;
+      const int w0 = max(0, l - RW + 1);
+      const int n_win = l - w0 + 1;
+      long long sr = 0, sr2 = 0;
+      for (int k = w0; k <= l; ++k) {
+        const long long v = rk[k % RW][tl];
+        sr += v;
+        sr2 += v * v;
+      }
+      const long long Dv = static_cast<long long>(n_win) * sr2 - sr * sr;
+      const double sigma = __ddiv_rn(__dsqrt_rn(static_cast<double>(Dv)),
+                                     __dmul_rn(static_cast<double>(n_win), static_cast<double>(T - 1)));
+      double cons = __dsub_rn(1.0, __dmul_rn(sigma, sqrt12));
+      if (cons < 0.0) cons = 0.0;
+      const double w = __dmul_rn(static_cast<double>(s_sm[i]), __dadd_rn(1.0, __dmul_rn(lamd, cons)));
+      const long long lay = static_cast<long long>(l) * pool_pages;
+      const int phys = entries_all[lay + fr.start[l] + i / P].x;
+      tok_shat_all[(lay + phys) * P + (i % P)] = __double2float_rn(w);
+    }
   }
 }
 
@@ -1159,6 +1226,62 @@ kvc_status compress_body(kvc_cache* c, int layer, cudaStream_t s, const Scratch&
   return KVC_OK;
 }
 
+// Every layer of the frame scored in two launches (raw scores, then CLCES of all layers),
+// with the results of score_layer on layers 0, 1, ... in order; kvc_last_raw_scores then
+// gives the last layer's raw scores. Used when every layer is at the same frame and none of
+// its layers has been scored yet; otherwise the layers are scored one by one.
+kvc_status score_all_layers(kvc_cache* c, const float* const* residuals) {
+  const kvc_config& g = c->cfg;
+  const int nl = g.num_layers;
+  const int t = c->L[0].last_frame;
+  bool batch = nl <= kMaxBatchLayers && g.rank_window <= 32 && !(c->hist_frame == t && c->hist_next_layer > 0);
+  for (int l = 0; l < nl && batch; ++l) {
+    const LayerHost& L = c->L[l];
+    if (L.last_frame != t || L.has_pending || L.frames.empty() || L.frames.back().frame != t || L.scored_frame == t)
+      batch = false;
+  }
+  if (!batch) {
+    for (int l = 0; l < nl; ++l) {
+      kvc_status st = score_layer(c, l, residuals[l]);
+      if (st != KVC_OK) return st;
+    }
+    return KVC_OK;
+  }
+  const Scratch sc = scratch_set(c, 0);
+  const int T = g.tokens_per_frame, P = g.page_size;
+  ResidualBatch rb{};
+  LayerStarts fr{};
+  for (int l = 0; l < nl; ++l) {
+    rb.r[l] = residuals[l];
+    fr.start[l] = c->L[l].frames.back().first_entry;
+  }
+  cudaStream_t s = c->stream;
+  residual_norm_layers_kernel<<<dim3((T * 32 + 255) / 256, nl), 256, 0, s>>>(rb, T, g.residual_dim, sc.s_raw_all);
+  cudaError_t e = cudaGetLastError();
+  c->launches++;
+  if (e == cudaSuccess) {
+    clces_layers_kernel<<<(T + kClcesTokens - 1) / kClcesTokens, 128, T * sizeof(float), s>>>(
+        sc.s_raw_all, T, nl, g.rank_window, g.lambda_, c->entries, fr, c->pool_pages, P, c->tok_shat);
+    e = cudaGetLastError();
+    c->launches++;
+  }
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(sc.s_raw, sc.s_raw_all + static_cast<size_t>(nl - 1) * T, static_cast<size_t>(T) * sizeof(float),
+                        cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) {
+    c->last_error = std::string("kvc_compress_all scoring: ") + cudaGetErrorString(e);
+    return KVC_ERR_CUDA;
+  }
+  c->hist_frame = t;
+  c->hist_layers.clear();
+  for (int l = 0; l < nl; ++l) {
+    c->hist_layers.push_back(l);
+    c->L[l].scored_frame = t;
+  }
+  c->hist_next_layer = nl;
+  return KVC_OK;
+}
+
 kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_t* fired) {
   kvc_status st = score_layer(c, layer, residual);
   if (st != KVC_OK) return st;
@@ -1173,11 +1296,10 @@ kvc_status compress_layer(kvc_cache* c, int layer, const float* residual, int32_
 // page table, token metadata and free bitmap, so the layers are independent.
 kvc_status compress_all_layers(kvc_cache* c, const float* const* residuals, int32_t* fired) {
   const kvc_config& g = c->cfg;
-  for (int l = 0; l < g.num_layers; ++l) {
+  for (int l = 0; l < g.num_layers; ++l)
     if (fired) fired[l] = 0;
-    kvc_status st = score_layer(c, l, residuals[l]);
-    if (st != KVC_OK) return st;
-  }
+  kvc_status sst = score_all_layers(c, residuals);
+  if (sst != KVC_OK) return sst;
   int todo[64];
   int n = 0;
   for (int l = 0; l < g.num_layers && n < 64; ++l)
