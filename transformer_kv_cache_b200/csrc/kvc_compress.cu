@@ -260,26 +260,42 @@ __global__ void __launch_bounds__(128) clces_kernel(const float* __restrict__ s,
 // the last RW layers in shared memory, since a token's Cons needs only its own ranks. The
 // arithmetic per (layer, token) is clces_kernel's (ranks by counting, integer window sums,
 // the same fp64 operations).
+// kStaged: every layer's scores are staged in shared memory at once (n_layers * T floats),
+// with kClcesStagedTokens tokens per 64-thread CTA (twice the CTAs); otherwise one layer's
+// scores at a time.
+constexpr int kClcesStagedTokens = 8;
+template <bool kStaged>
 __global__ void __launch_bounds__(128) clces_layers_kernel(const float* __restrict__ s_all, int T, int n_layers,
                                                             int RW, float lam, const Entry* __restrict__ entries_all,
                                                             LayerStarts fr, int pool_pages, int P,
                                                             float* __restrict__ tok_shat_all) {
   extern __shared__ float s_sm[];
-  __shared__ int rk[32][kClcesTokens];          // [layer % RW][token of the CTA]
+  constexpr int kTok = kStaged ? kClcesStagedTokens : kClcesTokens;
+  __shared__ int rk[32][kTok];                  // [layer % RW][token of the CTA]
   const int sub = threadIdx.x & 7, tl = static_cast<int>(threadIdx.x >> 3);
-  const int i = blockIdx.x * kClcesTokens + tl;
+  const int i = blockIdx.x * kTok + tl;
   const double sqrt12 = __dsqrt_rn(12.0);
   const double lamd = static_cast<double>(lam);
-  for (int l = 0; l < n_layers; ++l) {
-    __syncthreads();                            // the previous layer's scores are no longer read
-    const float* s = s_all + static_cast<long long>(l) * T;
-    for (int j = threadIdx.x; j < T; j += blockDim.x) s_sm[j] = s[j];
+  if (kStaged) {
+    const long long n = static_cast<long long>(n_layers) * T;
+    for (long long j = threadIdx.x; j < n; j += blockDim.x) s_sm[j] = s_all[j];
     __syncthreads();
+  }
+  for (int l = 0; l < n_layers; ++l) {
+    const float* s_l = s_sm;
+    if (kStaged) {
+      s_l = s_sm + static_cast<long long>(l) * T;
+    } else {
+      __syncthreads();                          // the previous layer's scores are no longer read
+      const float* s = s_all + static_cast<long long>(l) * T;
+      for (int j = threadIdx.x; j < T; j += blockDim.x) s_sm[j] = s[j];
+      __syncthreads();
+    }
     int r = 0;
     if (i < T) {
-      const float si = s_sm[i];
+      const float si = s_l[i];
       for (int j = sub; j < T; j += 8) {
-        const float sj = s_sm[j];
+        const float sj = s_l[j];
         r += (sj > si) || (sj == si && j < i);
       }
     }
@@ -301,7 +317,7 @@ __global__ void __launch_bounds__(128) clces_layers_kernel(const float* __restri
                                      __dmul_rn(static_cast<double>(n_win), static_cast<double>(T - 1)));
       double cons = __dsub_rn(1.0, __dmul_rn(sigma, sqrt12));
       if (cons < 0.0) cons = 0.0;
-      const double w = __dmul_rn(static_cast<double>(s_sm[i]), __dadd_rn(1.0, __dmul_rn(lamd, cons)));
+      const double w = __dmul_rn(static_cast<double>(s_l[i]), __dadd_rn(1.0, __dmul_rn(lamd, cons)));
       const long long lay = static_cast<long long>(l) * pool_pages;
       const int phys = entries_all[lay + fr.start[l] + i / P].x;
       tok_shat_all[(lay + phys) * P + (i % P)] = __double2float_rn(w);
@@ -1260,9 +1276,23 @@ kvc_status score_all_layers(kvc_cache* c, const float* const* residuals) {
   cudaError_t e = cudaGetLastError();
   c->launches++;
   if (e == cudaSuccess) {
-    clces_layers_kernel<<<(T + kClcesTokens - 1) / kClcesTokens, 128, T * sizeof(float), s>>>(
-        sc.s_raw_all, T, nl, g.rank_window, g.lambda_, c->entries, fr, c->pool_pages, P, c->tok_shat);
-    e = cudaGetLastError();
+    const size_t staged = static_cast<size_t>(nl) * T * sizeof(float);
+    constexpr size_t kStagedMax = 200 * 1024;
+    if (staged <= kStagedMax) {
+      static PerDeviceOnce attr;
+      e = attr.run([] {
+        return cudaFuncSetAttribute(clces_layers_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(kStagedMax));
+      });
+      if (e == cudaSuccess)
+        clces_layers_kernel<true><<<(T + kClcesStagedTokens - 1) / kClcesStagedTokens, 8 * kClcesStagedTokens, staged,
+                                    s>>>(sc.s_raw_all, T, nl, g.rank_window, g.lambda_, c->entries, fr,
+                                         c->pool_pages, P, c->tok_shat);
+    } else {
+      clces_layers_kernel<false><<<(T + kClcesTokens - 1) / kClcesTokens, 8 * kClcesTokens, T * sizeof(float), s>>>(
+          sc.s_raw_all, T, nl, g.rank_window, g.lambda_, c->entries, fr, c->pool_pages, P, c->tok_shat);
+    }
+    if (e == cudaSuccess) e = cudaGetLastError();
     c->launches++;
   }
   if (e == cudaSuccess)
