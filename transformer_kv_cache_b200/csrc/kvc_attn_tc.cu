@@ -390,7 +390,10 @@ __device__ __forceinline__ void store_piece(const TcParams& p, const LayerAttn& 
   if (lane == 0) p.split_cnt[cidx] = 0;   // ready for the next launch
 }
 
-template <int P, bool kPerHead, int kMode>
+// kPrefetch (bf16 only): each piece's epilogue loads the next piece's Q rows before its
+// last wait and stores them in TMEM right after reading O', so the next piece's S starts
+// while this piece's outputs are stored; chosen for launches with many pieces per CTA.
+template <int P, bool kPerHead, int kMode, bool kPrefetch = false>
 __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThreads8, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                    const TcParams p, const __grid_constant__ AttnLayers lt) {
@@ -706,13 +709,16 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
     const int row = (2 * qp + wg) * kBM + wq * 32 + lane;
     int ub = 0, pc = 0;
     bool ok = true;
+    [[maybe_unused]] bool q_stored = false;   // kPrefetch: this piece's Q is already in TMEM
     Sweep sw = sweep0;
     int lay, h, t0, t1;
     while (ok && next_piece(sw, lt, p.H, lay, h, t0, t1)) {
       const int nh = 2 * (t1 - t0);
       const LayerAttn& la = lt.l[lay];
       float row_fac = 1.f;       // E4M3: 2^-e of the query row's scaling into f16
-      {
+      bool have_q = false;
+      if constexpr (kPrefetch) have_q = q_stored;
+      if (!have_q) {
         // this row of Q (zeros past the last query) into TMEM, the A operand of S; the S
         // products of the previous piece, its only readers, have completed (their S was read)
         uint32_t qv[32];
@@ -761,6 +767,7 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
         __syncwarp();
         if (lane == 0) mbar_arrive(&q_ready[wg]);
       }
+      if constexpr (kPrefetch) q_stored = false;
       float m = -INFINITY;       // reference max (log2 domain) of the row
       float vref = 1.f;          // E4M3: the piece's V reference
       for (int u = 0; u < nh; ++u) {
@@ -854,6 +861,30 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
       }
       if (!ok) break;
       // ---------------------------------------------------------------- epilogue
+      [[maybe_unused]] bool has_next = false;
+      [[maybe_unused]] uint32_t qn[32];
+      if constexpr (kPrefetch && !kF8) {
+        Sweep swn = sw;
+        int layn, hn, t0n, t1n;
+        has_next = next_piece(swn, lt, p.H, layn, hn, t0n, t1n);
+        if (has_next) {
+          if (row < p.T) {
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(lt.l[layn].q) +
+                                                              (static_cast<long long>(row) * p.out_heads + p.head0 + hn) * kHD);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const uint4 w = __ldg(src + v);
+              qn[4 * v] = w.x;
+              qn[4 * v + 1] = w.y;
+              qn[4 * v + 2] = w.z;
+              qn[4 * v + 3] = w.w;
+            }
+          } else {
+#pragma unroll
+            for (int v = 0; v < 32; ++v) qn[v] = 0u;
+          }
+        }
+      }
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(&o_full[wg], pc & 1, abort_flag, p.err))) {
         ok = false;
         break;
@@ -867,6 +898,19 @@ __global__ void __launch_bounds__(kMode == tc::kBf16 ? tc::kThreads : tc::kThrea
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_free[wg]);
+      if constexpr (kPrefetch && !kF8) {
+        if (has_next) {
+          // the next piece's Q: every S product of this piece has completed (its S was read)
+          tmem_st32(tb + kColQ, qn);
+          const uint32_t qb[8] = {0x3f80u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+          tmem_st8(tb + kColQb, qb);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&q_ready[wg]);
+          q_stored = true;
+        }
+      }
       // E4M3: V was divided by the piece's V reference
       store_piece(p, la, lay, wg, wq, lane, h, qp, g, o0, o1, __uint_as_float(lsum), m, kF8 ? vref : 1.f);
       ub += nh;
@@ -1137,14 +1181,22 @@ bool plan_attn_bf16(int T, int H, const int* n_pages, int n_layers, int P, int s
 
 namespace {
 template <int kMode>
-cudaError_t launch_mode(cudaStream_t s, bool per_head, dim3 grid, const TcParams& prm, const TcAttnArgs& a,
-                        const AttnLayers& lt) {
+cudaError_t launch_mode(cudaStream_t s, bool per_head, bool prefetch, dim3 grid, const TcParams& prm,
+                        const TcAttnArgs& a, const AttnLayers& lt) {
   constexpr bool kF8 = kMode != tc::kBf16;
   const int threads = kF8 ? tc::kThreads8 : tc::kThreads;
   const size_t smem = kF8 ? tc::kSmemBytes8 : tc::kSmemBytes;
-  if (per_head) {
-    if constexpr (kF8) return cudaErrorInvalidValue;
-    else return launch_pdl(attn_tc_kernel<16, true, kMode>, grid, dim3(threads), smem, s, *a.tmap_k, *a.tmap_v, prm, lt);
+  if constexpr (kF8) {
+    if (per_head) return cudaErrorInvalidValue;
+  } else {
+    if (per_head && prefetch)
+      return launch_pdl(attn_tc_kernel<16, true, kMode, true>, grid, dim3(threads), smem, s, *a.tmap_k, *a.tmap_v,
+                        prm, lt);
+    if (per_head)
+      return launch_pdl(attn_tc_kernel<16, true, kMode>, grid, dim3(threads), smem, s, *a.tmap_k, *a.tmap_v, prm, lt);
+    if (prefetch)
+      return launch_pdl(attn_tc_kernel<16, false, kMode, true>, grid, dim3(threads), smem, s, *a.tmap_k, *a.tmap_v,
+                        prm, lt);
   }
   return launch_pdl(attn_tc_kernel<16, false, kMode>, grid, dim3(threads), smem, s, *a.tmap_k, *a.tmap_v, prm, lt);
 }
@@ -1163,6 +1215,8 @@ cudaError_t launch_layers(cudaStream_t s, const TcAttnArgs& a, const LayerAttn* 
     const cudaFuncAttribute at = cudaFuncAttributeMaxDynamicSharedMemorySize;
     cudaError_t r = cudaFuncSetAttribute(attn_tc_kernel<16, false, tc::kBf16>, at, b);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(attn_tc_kernel<16, true, tc::kBf16>, at, b);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(attn_tc_kernel<16, false, tc::kBf16, true>, at, b);
+    if (r == cudaSuccess) r = cudaFuncSetAttribute(attn_tc_kernel<16, true, tc::kBf16, true>, at, b);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(attn_tc_kernel<16, false, tc::kE4m3>, at, f);
     if (r == cudaSuccess) r = cudaFuncSetAttribute(attn_tc_kernel<16, false, tc::kE4m3Da>, at, f);
     return r;
@@ -1208,9 +1262,11 @@ cudaError_t launch_layers(cudaStream_t s, const TcAttnArgs& a, const LayerAttn* 
   prm.k_chan = a.k_chan;
   prm.v_tok = a.v_tok;
   const dim3 grid(pl.grid);
-  if (!a.fp8) e = launch_mode<tc::kBf16>(s, a.head_pages > 0, grid, prm, a, lt);
-  else if (a.k_chan) e = launch_mode<tc::kE4m3Da>(s, false, grid, prm, a, lt);
-  else e = launch_mode<tc::kE4m3>(s, false, grid, prm, a, lt);
+  // the Q prefetch pays where a CTA sweeps many pieces: several layers or per-head lists
+  const bool prefetch = n > 1 || a.head_pages > 0;
+  if (!a.fp8) e = launch_mode<tc::kBf16>(s, a.head_pages > 0, prefetch, grid, prm, a, lt);
+  else if (a.k_chan) e = launch_mode<tc::kE4m3Da>(s, false, false, grid, prm, a, lt);
+  else e = launch_mode<tc::kE4m3>(s, false, false, grid, prm, a, lt);
   if (e != cudaSuccess) return e;
   if (launched) *launched = 1;
   if (splits_used) *splits_used = pl.max_pieces;
