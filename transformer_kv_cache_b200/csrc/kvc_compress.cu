@@ -1135,6 +1135,12 @@ kvc_status compress_body(kvc_cache* c, int layer, cudaStream_t s, const Scratch&
     if (r != cudaSuccess && e == cudaSuccess) e = r;
     c->launches++;
   };
+  // a failed launch stops the sequence: later kernels index by the tier lists and the page
+  // entries that the failed one was to write
+  auto fail = [&]() {
+    c->last_error = std::string("kvc_compress: ") + cudaGetErrorString(e);
+    return KVC_ERR_CUDA;
+  };
   const int B = g.budget_tokens;
   const int N = static_cast<int>(L.tokens);
   const int n_keep = static_cast<int>(cp.n_keep);
@@ -1172,6 +1178,7 @@ kvc_status compress_body(kvc_cache* c, int layer, cudaStream_t s, const Scratch&
   }
   check_counts_kernel<<<1, 1, 0, s>>>(sc.counts, N, n_keep, n_keep_other, n_merge, c->d_err);
   ok();
+  if (e != cudaSuccess) return fail();
   const int HD = H * D;
   int64_t* lsrc = sc.last_src + static_cast<size_t>(layer) * cp.n_merge;
   int64_t* ldst = sc.last_dst + static_cast<size_t>(layer) * cp.n_merge;
@@ -1208,6 +1215,7 @@ kvc_status compress_body(kvc_cache* c, int layer, cudaStream_t s, const Scratch&
     record_merges_kernel<<<(n_merge + 255) / 256, 256, 0, s>>>(sc, static_cast<int>(cp.n_merge), lsrc, ldst);
     ok();
   }
+  if (e != cudaSuccess) return fail();
   // compaction into the lowest free pages, then release every old page
   const int n_old = L.n_entries;
   const int n_new = (n_keep + P - 1) / P;
@@ -1215,21 +1223,18 @@ kvc_status compress_body(kvc_cache* c, int layer, cudaStream_t s, const Scratch&
     c->last_error = "kvc_compress: page pool too small for compaction";
     return KVC_ERR_STATE;
   }
-  e = e != cudaSuccess ? e : launch_mgr_alloc(s, E, layer_free_bitmap(c, layer),
-                                              c->bitmap_words, c->pool_pages, n_old, n_new, -1, P,
-                                              n_keep - (n_new - 1) * P, c->d_err);
+  e = launch_mgr_alloc(s, E, layer_free_bitmap(c, layer), c->bitmap_words, c->pool_pages, n_old, n_new, -1, P,
+                       n_keep - (n_new - 1) * P, c->d_err);
   c->launches++;
+  if (e != cudaSuccess) return fail();
   compact_kernel<<<(n_new * P * 32 + 255) / 256, 256, 0, s>>>(sc, static_cast<int>(cp.n_keep), E + n_old, n_new, kp, vp,
                                                               c->tok_id + lay_slots, c->tok_cnt + lay_slots,
                                                               c->tok_shat + lay_slots, H, P, D);
   ok();
-  e = e != cudaSuccess ? e : launch_mgr_remove(s, E, layer_free_bitmap(c, layer),
-                                               n_old + n_new, 0, n_old, c->d_err);
+  if (e != cudaSuccess) return fail();
+  e = launch_mgr_remove(s, E, layer_free_bitmap(c, layer), n_old + n_new, 0, n_old, c->d_err);
   c->launches++;
-  if (e != cudaSuccess) {
-    c->last_error = std::string("kvc_compress: ") + cudaGetErrorString(e);
-    return KVC_ERR_CUDA;
-  }
+  if (e != cudaSuccess) return fail();
   L.n_entries = n_new;
   L.frames.clear();
   L.block_entries = n_new;
@@ -1330,10 +1335,10 @@ kvc_status compress_all_layers(kvc_cache* c, const float* const* residuals, int3
     if (fired) fired[l] = 0;
   kvc_status sst = score_all_layers(c, residuals);
   if (sst != KVC_OK) return sst;
-  int todo[64];
-  int n = 0;
-  for (int l = 0; l < g.num_layers && n < 64; ++l)
-    if (c->L[l].tokens > g.budget_tokens) todo[n++] = l;
+  std::vector<int> todo;
+  for (int l = 0; l < g.num_layers; ++l)
+    if (c->L[l].tokens > g.budget_tokens) todo.push_back(l);
+  const int n = static_cast<int>(todo.size());
   if (n == 0) return KVC_OK;
   const int sets = std::min(n, static_cast<int>(kvc_cache::kCmpSets));
   cudaError_t e = cudaEventRecord(c->cmp_fork, c->stream);
