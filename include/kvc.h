@@ -141,7 +141,11 @@ typedef struct kvc_cache kvc_cache;
  * page pools sized for the configuration (window: (S + W + 1) frames of pages
  * per layer; budget: 2*ceil(B/P) + (ceil(B/T) + 2) frames of pages), page
  * tables and scratch, and zero-fills them. On success *out owns everything;
- * release with kvc_destroy. Errors: KVC_ERR_ARG (bad config), KVC_ERR_OOM. */
+ * release with kvc_destroy. Errors: KVC_ERR_ARG (bad config; also sizes past
+ * the index range: more than 2^30 pages per layer, more than 2^31 - 1 pool
+ * rows of P slots per head over all layers on the tensor-core path, or a
+ * field above its cap: 65,536 layers, heads or page size, 2^24 tokens per
+ * frame or frames of window, scale or max_frames), KVC_ERR_OOM. */
 KVC_API kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out);
 
 /* Synchronise the stream and free everything the cache owns. NULL is a no-op. */

@@ -95,6 +95,12 @@ CONFIG_RULES = [
     ("vggt_infinite_12l", dict(diversity_budget=1100), "more candidates than the pruning cluster holds"),
     ("vggt_infinite_12l", dict(diversity_budget=-1), "negative diversity budget"),
     ("vggt_infinite_12l", dict(window_frames=64), "rolling memory with a window"),
+    ("vggt_518x378", dict(window_frames=(1 << 24) + 1), "window past its cap"),
+    ("vggt_518x378", dict(window_frames=0, max_frames=(1 << 24) + 1), "frame cap past its cap"),
+    ("vggt_518x378", dict(window_frames=0, max_frames=200_000), "pool rows past the int row index"),
+    ("vggt_518x378", dict(tokens_per_frame=(1 << 24) + 1), "frame past the token cap"),
+    ("vggt_518x378", dict(head_begin=2**31 - 2), "head range overflowing int"),
+    ("vggt_infinite_12l", dict(diversity_budget=2**31 - 1), "diversity budget overflowing int"),
 ]
 
 

@@ -216,7 +216,9 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
     if (g.reserved[i] != 0) return KVC_ERR_ARG;
   // a head range of the caller's tensors: bf16 window caches on the tensor-core path
   const int mh = g.model_heads > 0 ? g.model_heads : g.num_heads;
-  if (g.model_heads < 0 || g.head_begin < 0 || g.num_heads < 1 || g.head_begin + g.num_heads > mh) return KVC_ERR_ARG;
+  if (g.model_heads < 0 || g.model_heads > (1 << 16) || g.head_begin < 0 || g.num_heads < 1 ||
+      g.head_begin > mh - g.num_heads)
+    return KVC_ERR_ARG;
   if (mh != g.num_heads &&
       (g.io_dtype != KVC_BF16 || g.kv_dtype != KVC_BF16 || g.head_dim != 64 || g.page_size != 16 ||
        g.window_frames <= 0 || g.budget_tokens > 0 || g.diversity_budget > 0))
@@ -227,7 +229,11 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   if (g.special_frames < 0 || g.special_frames > (1 << 20) ||
       (g.special_frames > 0 && (g.window_frames <= 0 || g.budget_tokens > 0 || g.diversity_budget > 0)))
     return KVC_ERR_ARG;
+  // the size caps keep every page count and row index below in range of int
   const bool dims_ok = g.num_layers >= 1 && g.num_heads >= 1 && g.tokens_per_frame >= 1 && g.page_size >= 1 &&
+                       g.num_layers <= (1 << 16) && g.num_heads <= (1 << 16) && g.tokens_per_frame <= (1 << 24) &&
+                       g.page_size <= (1 << 16) && g.window_frames <= (1 << 24) && g.scale_frames <= (1 << 24) &&
+                       g.max_frames <= (1 << 24) &&
                        g.num_special_tokens >= 0 && g.num_special_tokens <= g.tokens_per_frame &&
                        g.scale_frames >= 0 && g.budget_tokens >= 0 &&
                        (g.head_dim == 16 || g.head_dim == 32 || g.head_dim == 64 || g.head_dim == 128);
@@ -247,16 +253,41 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   if (g.diversity_budget > 0) {
     // rolling diversity-pruned memory: bf16 tensor-core path, no window, no token budget;
     // a head's candidates (kept pages + one frame) fit the pruning kernel's shared memory
-    const int ppf = (g.tokens_per_frame + g.page_size - 1) / g.page_size;
+    const long long frame_pages = (g.tokens_per_frame + g.page_size - 1) / g.page_size;
+    const long long kept_pages = (static_cast<long long>(g.diversity_budget) + g.page_size - 1) / g.page_size;
     if (g.io_dtype != KVC_BF16 || g.kv_dtype != KVC_BF16 || g.head_dim != 64 || g.page_size != 16 ||
         g.num_heads > kMaxBatchLayers ||
         g.window_frames > 0 || g.budget_tokens > 0 ||
-        ((g.diversity_budget + g.page_size - 1) / g.page_size + ppf) * g.page_size > diversity_prune_max_candidates())
+        (kept_pages + frame_pages) * g.page_size > diversity_prune_max_candidates())
       return KVC_ERR_ARG;
   } else if (g.window_frames <= 0 && g.budget_tokens == 0 && g.max_frames < 1) {
     return KVC_ERR_ARG;
   }
   if (g.kv_splits < 0) return KVC_ERR_ARG;
+
+  const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads, D = g.head_dim;
+  const int ppf = (T + P - 1) / P;
+  long long pool_pages;
+  if (g.diversity_budget > 0) {
+    // per head: the anchor frame, the kept pages and one pending frame (pruning compacts
+    // the kept tokens in place)
+    const long long kp = (static_cast<long long>(g.diversity_budget) + P - 1) / P;
+    pool_pages = 2LL * ppf + kp + 1;
+  } else if (g.window_frames > 0) {
+    pool_pages = (static_cast<long long>(g.scale_frames) + g.window_frames + 1) * ppf +
+                 static_cast<long long>(g.special_frames) * special_pages(g);
+  } else if (g.budget_tokens > 0) {
+    const long long B = g.budget_tokens;
+    pool_pages = 2 * ((B + P - 1) / P) + ((B + T - 1) / T + 2) * ppf;
+  } else {
+    pool_pages = (static_cast<long long>(g.max_frames) + 1) * ppf;
+  }
+  // page counts are ints on the device; the tensor-core path addresses the pools by an int
+  // row index (pages x heads x P rows over all layers)
+  const long long pool_rows_all = static_cast<long long>(g.num_layers) * pool_pages * H * P;
+  const bool tc_shape = g.io_dtype == KVC_BF16 && (g.kv_dtype == KVC_BF16 || g.kv_dtype == KVC_FP8_E4M3) &&
+                        D == 64 && P == 16;
+  if (pool_pages > (1LL << 30) || (tc_shape && pool_rows_all > INT_MAX)) return KVC_ERR_ARG;
 
   kvc_cache* c = new (std::nothrow) kvc_cache();
   if (!c) return KVC_ERR_OOM;
@@ -264,25 +295,12 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   c->stream = static_cast<cudaStream_t>(stream);
   cudaGetDevice(&c->device);
   cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device);
-  const int T = g.tokens_per_frame, P = g.page_size, H = g.num_heads, D = g.head_dim;
-  c->ppf = (T + P - 1) / P;
+  c->ppf = ppf;
   c->model_heads = g.model_heads > 0 ? g.model_heads : H;
   c->head0 = g.head_begin;
   c->per_head = g.diversity_budget > 0;
-  if (c->per_head) {
-    // per head: the anchor frame, the kept pages and one pending frame (pruning compacts
-    // the kept tokens in place)
-    const int kp = (g.diversity_budget + P - 1) / P;
-    c->pool_pages = 2 * c->ppf + kp + 1;
-    c->layer_budget.assign(g.num_layers, g.diversity_budget);
-  } else if (g.window_frames > 0) {
-    c->pool_pages = (g.scale_frames + g.window_frames + 1) * c->ppf + g.special_frames * special_pages(g);
-  } else if (g.budget_tokens > 0) {
-    const int B = g.budget_tokens;
-    c->pool_pages = 2 * ((B + P - 1) / P) + ((B + T - 1) / T + 2) * c->ppf;
-  } else {
-    c->pool_pages = (g.max_frames + 1) * c->ppf;
-  }
+  if (c->per_head) c->layer_budget.assign(g.num_layers, g.diversity_budget);
+  c->pool_pages = static_cast<int>(pool_pages);
   c->bitmap_words = (c->pool_pages + 31) / 32;
   c->elem_io = dtype_bytes(g.io_dtype);
   c->elem_kv = dtype_bytes(g.kv_dtype);
@@ -296,7 +314,7 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   const size_t L = g.num_layers;
   const size_t NS = c->per_head ? L * H : L;   // page lists (sub-layers)
   const size_t frame_bytes = static_cast<size_t>(T) * H * D * c->elem_io;
-  c->tc_path = g.io_dtype == KVC_BF16 && (g.kv_dtype == KVC_BF16 || g.kv_dtype == KVC_FP8_E4M3) && D == 64 && P == 16;
+  c->tc_path = tc_shape;
   const int q_tiles = (T + 127) / 128;
   // partial tiles: 16 per (query tile, head), and at least 8 per SM (a split unit's pieces
   // take 4 per CTA of the groups that cut it)

@@ -7,6 +7,7 @@
 
 #include <mutex>
 #include <string>
+#include <climits>
 #include <vector>
 
 #include "kvc.h"
