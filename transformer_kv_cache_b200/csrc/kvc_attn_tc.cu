@@ -1231,8 +1231,6 @@ cudaError_t launch_layers(cudaStream_t s, const TcAttnArgs& a, const LayerAttn* 
       return cudaErrorInvalidValue;
     np[l] = layers[l].n_pages;
   }
-  // TMA row coordinates are ints; the row one past the end reads zeros
-  if (a.pool_rows < 1 || a.pool_rows > INT_MAX) return cudaErrorInvalidValue;
   AttnPlan pl;
   if (!plan_attn_bf16(a.T, a.H, np, n, a.P, a.sm_count, a.splits, a.part_rows, a.strict_splits, &pl, nt, p0))
     return cudaErrorInvalidValue;
