@@ -414,7 +414,9 @@ KVC_API int32_t kvc_version(void);
  * that first call before any stream capture. All calls share the array: calls whose
  * kernels overlap on the GPU race on it. Nothing in it needs to start at zero. A wait in
  * the kernel that gives up (bounded) ends the kernel without an error report here.
- * Errors: KVC_ERR_ARG (shapes, alignment, sizes beyond the array), KVC_ERR_CUDA. */
+ * Errors: KVC_ERR_ARG (shapes, alignment, sizes beyond the array, a softmax_scale
+ * that is not positive and finite, pools of more than 2^31 - 1 rows of 16 slots per
+ * head), KVC_ERR_CUDA. */
 KVC_API kvc_status kvc_attend_paged_noalloc(const void* q_dev, void* o_dev, const void* k_pool_dev,
                                             const void* v_pool_dev, int64_t pool_pages,
                                             const int32_t* page_table_dev, int32_t n_pages, int32_t tokens,

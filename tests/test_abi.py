@@ -165,6 +165,49 @@ def test_null_handle_is_rejected_by_every_entry_point():
     assert fn(*zero_args(fn)) == 1
 
 
+# The allocation-free entry point's host checks, one rule at a time, with fake 16-byte
+# aligned device addresses. Run only where no GPU is present: a rule that stopped
+# rejecting then ends at the first CUDA call (KVC_ERR_CUDA) instead of launching over
+# addresses that do not exist.
+NOALLOC_BASE = dict(q=0x10000, o=0x20000, k_pool=0x30000, v_pool=0x40000, pool_pages=64, page_table=0x50000,
+                    n_pages=8, tokens=300, num_heads=4, head_dim=64, page_size=16, softmax_scale=0.125,
+                    kv_splits=1)
+NOALLOC_RULES = [
+    (dict(head_dim=32), "head dim other than 64"),
+    (dict(page_size=8), "page size other than 16"),
+    (dict(tokens=0), "no query rows"),
+    (dict(num_heads=0), "no heads"),
+    (dict(n_pages=0), "no pages"),
+    (dict(pool_pages=0), "empty pool"),
+    (dict(softmax_scale=0.0), "scale not positive"),
+    (dict(softmax_scale=float("nan")), "scale NaN"),
+    (dict(softmax_scale=float("inf")), "scale infinite"),
+    (dict(kv_splits=0), "no KV split"),
+    (dict(q=0x10008), "Q not 16-byte aligned"),
+    (dict(page_table=0x50004), "page table not 16-byte aligned"),
+    (dict(pool_pages=2**31 // (4 * 16) + 1), "pool rows past the int row index"),
+    (dict(tokens=1025 * 128), "more piece counters than the array holds"),
+]
+
+
+@pytest.mark.parametrize("change,why", NOALLOC_RULES, ids=[r[1] for r in NOALLOC_RULES])
+def test_noalloc_rule_rejected_before_any_cuda_call(change, why):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("fake device addresses: host checks only, on a host without a GPU")
+    import transformer_kv_cache_b200 as kvc
+    fn = kvc._lib.kvc_attend_paged_noalloc
+
+    def call(**over):
+        a = dict(NOALLOC_BASE, **over)
+        return fn(a["q"], a["o"], a["k_pool"], a["v_pool"], a["pool_pages"], a["page_table"], a["n_pages"],
+                  a["tokens"], a["num_heads"], a["head_dim"], a["page_size"], a["softmax_scale"],
+                  a["kv_splits"], None)
+
+    assert call() == 3, "the base call passes the host checks and stops at the first CUDA call"
+    assert call(**change) == 1, why             # KVC_ERR_ARG
+
+
 def test_plain_c_program_links_and_calls_the_library():
     """A C99 program compiled against include/kvc.h and linked with libkvc.so: the host-only
     calls work without Python (version, status strings, argument rejection, NULL handles)."""

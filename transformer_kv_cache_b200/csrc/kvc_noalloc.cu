@@ -19,6 +19,7 @@
 #include <cuda_bf16.h>
 
 #include <climits>
+#include <cmath>
 #include <mutex>
 
 #include "kvc_internal.h"
@@ -78,7 +79,7 @@ extern "C" kvc_status kvc_attend_paged_noalloc(const void* q_dev, void* o_dev, c
   using namespace kvc;
   if (!q_dev || !o_dev || !k_pool_dev || !v_pool_dev || !page_table_dev) return KVC_ERR_ARG;
   if (head_dim != 64 || page_size != 16 || tokens < 1 || num_heads < 1 || n_pages < 1 || pool_pages < 1 ||
-      !(softmax_scale > 0.f) || kv_splits < 1)
+      !(softmax_scale > 0.f) || !std::isfinite(softmax_scale) || kv_splits < 1)
     return KVC_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(q_dev) | reinterpret_cast<uintptr_t>(o_dev) |
        reinterpret_cast<uintptr_t>(k_pool_dev) | reinterpret_cast<uintptr_t>(v_pool_dev) |
