@@ -1104,11 +1104,15 @@ kvc_status kvc_token_meta(kvc_cache* c, int32_t layer, int64_t* ids_host, int32_
   std::vector<int64_t> ids(static_cast<size_t>(c->pool_pages) * P);
   std::vector<int32_t> cnt(ids.size());
   std::vector<float> sh(ids.size());
-  cudaMemcpy(ids.data(), c->tok_id + base, ids.size() * sizeof(int64_t), cudaMemcpyDeviceToHost);
-  cudaMemcpy(cnt.data(), c->tok_cnt + base, cnt.size() * sizeof(int32_t), cudaMemcpyDeviceToHost);
-  cudaMemcpy(sh.data(), c->tok_shat + base, sh.size() * sizeof(float), cudaMemcpyDeviceToHost);
+  cudaError_t e = cudaMemcpy(ids.data(), c->tok_id + base, ids.size() * sizeof(int64_t), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(cnt.data(), c->tok_cnt + base, cnt.size() * sizeof(int32_t), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(sh.data(), c->tok_shat + base, sh.size() * sizeof(float), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(c, e, "kvc_token_meta copy");
   int k = 0;
   for (int i = 0; i < n; ++i) {
+    if (ent[i].x < 0 || ent[i].x >= c->pool_pages || ent[i].w < 0 || ent[i].w > P)
+      return fail(c, KVC_ERR_DEVICE, "kvc_token_meta: page-table row outside the pool");
     for (int s = 0; s < ent[i].w; ++s, ++k) {
       if (k >= capacity) continue;
       const size_t slot = static_cast<size_t>(ent[i].x) * P + s;
@@ -1129,7 +1133,7 @@ kvc_status kvc_export_pages(kvc_cache* c, int32_t layer, int32_t first_row, int3
   kvc_status st = sync_and_check(c);
   if (st != KVC_OK) return st;
   LayerHost& L = c->L[layer];
-  if (first_row < 0 || n_rows < 0 || first_row + n_rows > L.n_entries)
+  if (first_row < 0 || n_rows < 0 || first_row > L.n_entries || n_rows > L.n_entries - first_row)
     return fail(c, KVC_ERR_ARG, "kvc_export_pages: row range outside the page table");
   std::vector<Entry> ent(n_rows);
   if (n_rows > 0 && cudaMemcpy(ent.data(), layer_entries(c, layer) + first_row, n_rows * sizeof(Entry),
@@ -1166,7 +1170,7 @@ kvc_status kvc_export_fp8_group_scales(kvc_cache* c, int32_t layer, int32_t firs
   kvc_status st = sync_and_check(c);
   if (st != KVC_OK) return st;
   LayerHost& L = c->L[layer];
-  if (first_row < 0 || n_rows < 0 || first_row + n_rows > L.n_entries)
+  if (first_row < 0 || n_rows < 0 || first_row > L.n_entries || n_rows > L.n_entries - first_row)
     return fail(c, KVC_ERR_ARG, "kvc_export_fp8_group_scales: row range outside the page table");
   std::vector<Entry> ent(n_rows);
   if (n_rows > 0 && cudaMemcpy(ent.data(), layer_entries(c, layer) + first_row, n_rows * sizeof(Entry),
@@ -1314,11 +1318,14 @@ kvc_status kvc_head_tokens(kvc_cache* c, int32_t layer, int32_t head, int64_t* i
     e = cudaMemcpy(ids.data(), c->tok_id + sub * P, ids.size() * sizeof(int64_t), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(c, e, "kvc_head_tokens copy");
   int m = 0;
-  for (int i = 0; i < n; ++i)
+  for (int i = 0; i < n; ++i) {
+    if (ent[i].x < 0 || ent[i].x >= c->pool_pages || ent[i].w < 0 || ent[i].w > P)
+      return fail(c, KVC_ERR_DEVICE, "kvc_head_tokens: page-table row outside the pool");
     for (int s = 0; s < ent[i].w; ++s) {
       if (m >= capacity) return fail(c, KVC_ERR_ARG, "kvc_head_tokens: capacity too small");
       ids_out[m++] = ids[static_cast<size_t>(ent[i].x) * P + s];
     }
+  }
   *n_out = m;
   return KVC_OK;
 }
