@@ -125,3 +125,19 @@ def test_head_sharded_step_reassembles_the_full_output():
     import bench
     with pytest.raises(ValueError):
         bench.head_range(0, 3, 4)
+
+
+def test_profile_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
+    """The bench's roofline `traffic` comes from the committed ncu summary of the attention
+    kernel, and only while the kernel source hashes to the one that summary names."""
+    sys.path.insert(0, ROOT)
+    import bench
+    txt = open(bench.PROFILE_ATTN).read()
+    assert "source_sha256:" in txt and "traffic_bytes_per_launch:" in txt
+    t = bench.profile_traffic()
+    assert t is not None, "the attention source changed since its ncu summary was taken"
+    assert 2.9e8 < t < 3.5e8                 # about the 298.7 MB algorithmic bytes of a launch
+    changed = tmp_path / "kvc_attn_tc.cu"
+    changed.write_bytes(open(bench.ATTN_SRC, "rb").read() + b"\n")
+    monkeypatch.setattr(bench, "ATTN_SRC", str(changed))
+    assert bench.profile_traffic() is None
