@@ -143,9 +143,10 @@ typedef struct kvc_cache kvc_cache;
  * tables and scratch, and zero-fills them. On success *out owns everything;
  * release with kvc_destroy. Errors: KVC_ERR_ARG (bad config; also sizes past
  * the index range: more than 2^30 pages per layer, more than 2^31 - 1 pool
- * rows of P slots per head over all layers on the tensor-core path, or a
- * field above its cap: 65,536 layers, heads or page size, 2^24 tokens per
- * frame or frames of window, scale or max_frames), KVC_ERR_OOM. */
+ * rows of P slots per head over all layers on the tensor-core path, a frame
+ * (tokens x model heads x head_dim) or a page (P x heads x head_dim) of 2^29 elements
+ * or more, or a field above its cap: 65,536 layers, heads or page size,
+ * 2^24 tokens per frame or frames of window, scale or max_frames), KVC_ERR_OOM. */
 KVC_API kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out);
 
 /* Synchronise the stream and free everything the cache owns. NULL is a no-op. */
@@ -224,8 +225,8 @@ KVC_API kvc_status kvc_attend_all(kvc_cache* c, const void* const* q_devs, void*
  * and committed (as kvc_append_frame with is_keyframe = 1), then all n_frames * T
  * queries attend over all of their tokens with no mask; the causal frame-by-frame phase
  * continues with frame n_frames. 1 <= n_frames <= max(1, scale_frames). Errors:
- * KVC_ERR_ARG (pointers, alignment, frame count), KVC_ERR_STATE (the layer is not empty,
- * a token budget or per-head page lists). */
+ * KVC_ERR_ARG (pointers, alignment, frame count, more than 2^31 - 1 elements in Q),
+ * KVC_ERR_STATE (the layer is not empty, a token budget or per-head page lists). */
 KVC_API kvc_status kvc_scale_phase(kvc_cache* c, int32_t layer, int32_t n_frames, const void* q_dev,
                                    const void* k_dev, const void* v_dev, void* o_dev);
 

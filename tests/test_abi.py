@@ -100,6 +100,10 @@ CONFIG_RULES = [
     ("vggt_518x378", dict(window_frames=0, max_frames=200_000), "pool rows past the int row index"),
     ("vggt_518x378", dict(tokens_per_frame=(1 << 24) + 1), "frame past the token cap"),
     ("vggt_518x378", dict(head_begin=2**31 - 2), "head range overflowing int"),
+    ("vggt_518x378", dict(io_dtype="f32", kv_dtype="f32", tokens_per_frame=1 << 22),
+     "frame past the int element index"),
+    ("vggt_518x378", dict(io_dtype="f32", kv_dtype="f32", page_size=1 << 16, num_heads=1 << 10),
+     "page past the int element index"),
     ("vggt_infinite_12l", dict(diversity_budget=2**31 - 1), "diversity budget overflowing int"),
 ]
 

@@ -288,6 +288,13 @@ kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** out) {
   const bool tc_shape = g.io_dtype == KVC_BF16 && (g.kv_dtype == KVC_BF16 || g.kv_dtype == KVC_FP8_E4M3) &&
                         D == 64 && P == 16;
   if (pool_pages > (1LL << 30) || (tc_shape && pool_rows_all > INT_MAX)) return KVC_ERR_ARG;
+  // a frame's and a page's elements, and the append kernels' work items (2 per page and
+  // head of every layer, up to 64 threads each), are ints
+  const long long model_heads = g.model_heads > 0 ? g.model_heads : H;
+  if (static_cast<long long>(T) * model_heads * D * 4 > INT_MAX ||
+      static_cast<long long>(P) * H * D * 4 > INT_MAX ||
+      static_cast<long long>(g.num_layers) * ppf * H * 2 * 64 > INT_MAX)
+    return KVC_ERR_ARG;
 
   kvc_cache* c = new (std::nothrow) kvc_cache();
   if (!c) return KVC_ERR_OOM;
@@ -970,6 +977,9 @@ kvc_status kvc_scale_phase(kvc_cache* c, int32_t layer, int32_t n_frames, const 
     return fail(c, KVC_ERR_ARG, "kvc_scale_phase: Q, K, V and O must be 16-byte aligned");
   if (c->per_head || g.budget_tokens > 0)
     return fail(c, KVC_ERR_STATE, "kvc_scale_phase: not with a token budget or per-head page lists");
+  // the kernels index the n*T query rows' elements with ints
+  if (static_cast<long long>(n_frames) * g.tokens_per_frame * c->model_heads * g.head_dim > INT_MAX)
+    return fail(c, KVC_ERR_ARG, "kvc_scale_phase: more than 2^31 - 1 query elements");
   LayerHost& L = c->L[layer];
   if (L.n_entries != 0 || L.has_pending || L.last_frame >= 0)
     return fail(c, KVC_ERR_STATE, "kvc_scale_phase: the joint phase starts an empty layer");
