@@ -241,3 +241,23 @@ int main(void) {
                         "-L", lib_dir, "-lkvc", "-Wl,-rpath," + lib_dir], check=True)
         out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()
     assert out == ["1", "1", "KVC_ERR_ARG", "1", "1", "null", "cache"]
+
+
+def test_binding_refuses_host_buffers_for_device_arguments():
+    """The binding hands the library only CUDA tensors (or explicit addresses) where a
+    kernel reads or writes: a CPU tensor or numpy array raises before any C call."""
+    import numpy as np
+    import torch
+    import transformer_kv_cache_b200 as kvc
+    host_t, host_np = torch.zeros(16), np.zeros(16, np.float32)
+    for bad in (host_t, host_np):
+        with pytest.raises(TypeError):
+            kvc.kvc_attend(0, 0, bad, bad)
+        with pytest.raises(TypeError):
+            kvc.kvc_append_frame(0, 0, 0, bad, bad)
+        with pytest.raises(TypeError):
+            kvc.kvc_attend_all(0, [bad], [bad])
+        with pytest.raises(TypeError):
+            kvc.kvc_compress(0, 0, bad)
+        with pytest.raises(TypeError):
+            kvc.kvc_attend_paged_noalloc(bad, bad, bad, bad, 1, bad, 1, 1, 1, 64, 16, 0.125)

@@ -127,6 +127,16 @@ def _ptr(x) -> Optional[int]:
     return x.data_ptr()
 
 
+def _dptr(x) -> Optional[int]:
+    """Device pointer of a CUDA tensor, or an int taken as a device address. A host buffer
+    (numpy array or CPU tensor) is refused here, before a kernel could read it."""
+    if x is None or isinstance(x, int):
+        return x
+    if isinstance(x, np.ndarray) or not getattr(x, "is_cuda", False):
+        raise TypeError("a CUDA tensor (or a device address) is expected here, not a host buffer")
+    return x.data_ptr()
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         import torch
@@ -205,32 +215,32 @@ def kvc_reset(handle) -> None:
 
 
 def kvc_append_frame(handle, layer: int, frame_idx: int, k, v, is_keyframe: bool = True) -> None:
-    _check(handle, _lib.kvc_append_frame(handle, layer, frame_idx, _ptr(k), _ptr(v), int(bool(is_keyframe))))
+    _check(handle, _lib.kvc_append_frame(handle, layer, frame_idx, _dptr(k), _dptr(v), int(bool(is_keyframe))))
 
 
 def kvc_append_frame_all(handle, frame_idx: int, ks, vs, is_keyframe: bool = True) -> None:
     """ks, vs: per-layer device tensors (or pointers), one per layer."""
     n = len(ks)
-    ka = (ctypes.c_void_p * n)(*[_ptr(k) for k in ks])
-    va = (ctypes.c_void_p * n)(*[_ptr(v) for v in vs])
+    ka = (ctypes.c_void_p * n)(*[_dptr(k) for k in ks])
+    va = (ctypes.c_void_p * n)(*[_dptr(v) for v in vs])
     _check(handle, _lib.kvc_append_frame_all(handle, frame_idx, ka, va, int(bool(is_keyframe))))
 
 
 def kvc_attend(handle, layer: int, q, o) -> None:
-    _check(handle, _lib.kvc_attend(handle, layer, _ptr(q), _ptr(o)))
+    _check(handle, _lib.kvc_attend(handle, layer, _dptr(q), _dptr(o)))
 
 
 def kvc_attend_all(handle, qs, os) -> None:
     """qs, os: per-layer device tensors (or pointers), one per layer of the cache."""
     n = len(qs)
-    qa = (ctypes.c_void_p * n)(*[_ptr(q) for q in qs])
-    oa = (ctypes.c_void_p * n)(*[_ptr(o) for o in os])
+    qa = (ctypes.c_void_p * n)(*[_dptr(q) for q in qs])
+    oa = (ctypes.c_void_p * n)(*[_dptr(o) for o in os])
     _check(handle, _lib.kvc_attend_all(handle, qa, oa))
 
 
 def kvc_compress(handle, layer: int, residual) -> bool:
     fired = ctypes.c_int32(0)
-    _check(handle, _lib.kvc_compress(handle, layer, _ptr(residual), ctypes.byref(fired)))
+    _check(handle, _lib.kvc_compress(handle, layer, _dptr(residual), ctypes.byref(fired)))
     return bool(fired.value)
 
 
@@ -238,7 +248,7 @@ def kvc_compress_all(handle, residuals) -> list:
     """residuals: per-layer device fp32 tensors (or pointers), one per layer of the cache.
     Returns, per layer, whether a compression ran."""
     n = len(residuals)
-    ra = (ctypes.c_void_p * n)(*[_ptr(r) for r in residuals])
+    ra = (ctypes.c_void_p * n)(*[_dptr(r) for r in residuals])
     fired = (ctypes.c_int32 * n)()
     _check(handle, _lib.kvc_compress_all(handle, ra, fired))
     return [bool(f) for f in fired]
@@ -320,7 +330,7 @@ def kvc_set_layer_budgets(handle, budgets) -> None:
 def kvc_scale_phase(handle, layer: int, n_frames: int, q, k, v, o) -> None:
     """The joint scale-frame phase: frames 0..n_frames-1 ([n_frames*T, H, D] tensors)
     appended, committed, and attended bidirectionally."""
-    _check(handle, _lib.kvc_scale_phase(handle, layer, n_frames, _ptr(q), _ptr(k), _ptr(v), _ptr(o)))
+    _check(handle, _lib.kvc_scale_phase(handle, layer, n_frames, _dptr(q), _dptr(k), _dptr(v), _dptr(o)))
 
 
 def kvc_export_fp8_group_scales(handle, layer: int, first_row: int, n_rows: int, H: int, D: int, P: int):
@@ -387,7 +397,7 @@ def kvc_attend_paged_noalloc(q, o, k_pool, v_pool, pool_pages: int, page_table, 
                              num_heads: int, head_dim: int, page_size: int, softmax_scale: float,
                              kv_splits: int = 1, stream=None) -> None:
     """Attention over caller-owned pools with no device allocation (see include/kvc.h)."""
-    st = _lib.kvc_attend_paged_noalloc(_ptr(q), _ptr(o), _ptr(k_pool), _ptr(v_pool), pool_pages, _ptr(page_table),
+    st = _lib.kvc_attend_paged_noalloc(_dptr(q), _dptr(o), _dptr(k_pool), _dptr(v_pool), pool_pages, _dptr(page_table),
                                        n_pages, tokens, num_heads, head_dim, page_size, softmax_scale, kv_splits,
                                        _stream(stream))
     if st != 0:
