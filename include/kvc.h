@@ -260,7 +260,9 @@ KVC_API kvc_status kvc_compress(kvc_cache* c, int32_t layer, const float* residu
  * on the cache's side streams (each with its own scratch), joined back into the cache's
  * stream before the call returns. kvc_last_raw_scores afterwards gives the last layer's
  * raw scores. Errors: those of kvc_compress (the first one met); KVC_ERR_ARG for a NULL
- * array or residual. */
+ * array or residual. An error in the scoring leaves every layer uncompressed; an error in
+ * one layer's compression (e.g. KVC_ERR_BUDGET) does not stop the other layers over
+ * budget, which are compressed as usual: fired_out tells which were. */
 KVC_API kvc_status kvc_compress_all(kvc_cache* c, const float* const* residual_devs, int32_t* fired_out);
 
 /* Synchronise and copy the page table of `layer` to host: rows of 4 int32
