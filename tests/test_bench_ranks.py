@@ -141,3 +141,24 @@ def test_profile_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     changed.write_bytes(open(bench.ATTN_SRC, "rb").read() + b"\n")
     monkeypatch.setattr(bench, "ATTN_SRC", str(changed))
     assert bench.profile_traffic() is None
+
+
+@pytest.mark.parametrize("text,kind,hbm,bf16", [
+    ('{"hbm_gbs": 7000.5, "bf16_tflops": 1650, "bf16_tflops_sustained": 1420}', "measured", 7000.5, 1650.0),
+    ('{"hbm": {"hbm_gbs": 7001}, "gemm": {"bf16_tflops": {"value": 1640.0}}}', "measured", 7001.0, 1640.0),
+    ('{"hbm_gbs": 7002, "bf16_tflops": 1630}', "measured", 7002.0, 1630.0),
+    ('{"hbm_gbs": 7003}', "fallback", 6650.0, 1590.0),
+    ('{"hbm_gbs": "fast", "bf16_tflops": -1}', "fallback", 6650.0, 1590.0),
+    ("not json", "fallback", 6650.0, 1590.0),
+])
+def test_peaks_file_read_or_fallback(tmp_path, text, kind, hbm, bf16):
+    """The roofline denominators come from the peaks file when it holds the HBM and bf16
+    figures (flat, in sections, or as {"value": x}); otherwise every figure falls back."""
+    sys.path.insert(0, ROOT)
+    import bench
+    f = tmp_path / "peaks.json"
+    f.write_text(text)
+    peaks, k = bench.load_peaks(str(f))
+    assert (k, peaks["hbm_gbs"], peaks["bf16_tflops"]) == (kind, hbm, bf16)
+    assert peaks["bf16_tflops_sustained"] > 0
+    assert bench.load_peaks(str(tmp_path / "absent.json"))[1] == "fallback"
