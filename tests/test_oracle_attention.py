@@ -3,6 +3,7 @@ frames, the retained-set closed form, constant memory, and attention special cas
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings, strategies as st
 
 import brute
 from kvc_streams import WORKLOADS, FrameStream, keyframe_schedule
@@ -75,6 +76,22 @@ def test_random_small_configs_match_brute_force(T, P, S, W, k):
     wl = WORKLOADS["tiny_f32"].replace(tokens_per_frame=T, page_size=P, scale_frames=S,
                                         window_frames=W, keyframe_interval=k, num_heads=3, head_dim=8)
     _run_and_check(wl, 14, seed=T * 100 + P)
+
+
+@settings(max_examples=30, deadline=None, derandomize=True)
+@given(T=st.integers(1, 40), P=st.sampled_from([1, 2, 4, 8, 16]), S=st.integers(0, 3), W=st.integers(0, 4),
+       k=st.integers(1, 4), H=st.integers(1, 3), D=st.sampled_from([16, 32]),
+       kv=st.sampled_from(["f32", "bf16", "fp8_e4m3"]), frames=st.integers(1, 12))
+def test_swept_small_configs_match_brute_force(T, P, S, W, k, H, D, kv, frames):
+    """Seeded sweep over frame sizes (ragged and exact page fits, T < P), windows with and
+    without scale frames, keyframe intervals, head counts and storage formats: every step's
+    output and page table against brute force over the concatenated retained frames."""
+    io = "bf16" if kv != "f32" else "f32"
+    if kv == "fp8_e4m3" and P * D > 2048:
+        P = 2048 // D
+    wl = WORKLOADS["tiny_f32"].replace(tokens_per_frame=T, page_size=P, scale_frames=S, window_frames=W,
+                                        keyframe_interval=k, num_heads=H, head_dim=D, io_dtype=io, kv_dtype=kv)
+    _run_and_check(wl, frames, seed=T * 1000 + P * 10 + H)
 
 
 def test_fp8_small_matches_brute_force():
