@@ -5,6 +5,7 @@ import math
 import numpy as np
 import pytest
 import torch
+from hypothesis import assume, given, settings, strategies as st
 from scipy.spatial.distance import cdist
 
 from kvc_streams import WORKLOADS, FrameStream
@@ -43,8 +44,8 @@ def _drive(wl, frames, seed=0, on_event=None):
     return orc, events
 
 
-def _compression_check():
-    wl = _small_wl()
+def _compression_check(frames=9, min_events=4, **kw):
+    wl = _small_wl(**kw)
     n_keep = math.floor(float(np.float32(wl.keep_frac)) * wl.budget_tokens)
     n_merge = wl.budget_tokens - n_keep
     seen = []
@@ -113,12 +114,28 @@ def _compression_check():
         assert np.all(pt[:, 0] == -1)
         assert pt[:, 3].sum() == n_keep and np.all(pt[:-1, 3] == wl.page_size)
 
-    orc, events = _drive(wl, 9, on_event=check)
-    assert events >= 4 and len(seen) == events
+    orc, events = _drive(wl, frames, on_event=check)
+    assert events >= min_events and len(seen) == events
 
 
 def test_compression_properties():
     _compression_check()
+
+
+@settings(max_examples=20, deadline=None, derandomize=True)
+@given(T=st.integers(5, 12), P=st.sampled_from([2, 4, 8]), B=st.integers(24, 64),
+       keep_frac=st.sampled_from([0.5, 0.6, 0.75]), specials=st.integers(0, 2), H=st.integers(1, 3))
+def test_compression_properties_swept(T, P, B, keep_frac, specials, H):
+    """The same properties over frame sizes, page sizes, budgets, keep fractions, special
+    token counts and head counts; the stream runs while the protected tokens (frame 0 and
+    every frame's specials) still fit the keep tier."""
+    n_keep = math.floor(float(np.float32(keep_frac)) * B)
+    frames = 1
+    while frames < 14 and T + specials * frames <= n_keep:
+        frames += 1
+    assume(frames * T > B + T)            # at least one compression event
+    _compression_check(frames=frames, min_events=1, tokens_per_frame=T, page_size=P, budget_tokens=B,
+                       keep_frac=keep_frac, num_special_tokens=specials, num_heads=H)
 
 
 def test_full_protected_keep_tier_drops_merge_tier():
