@@ -3,6 +3,7 @@ scipy's cosine distance and softmax, brute-force Top-K, the page's worked number
 closed-form cases, and a planted mistake that the pins must catch."""
 import numpy as np
 import pytest
+from hypothesis import given, settings, strategies as st
 from scipy.spatial.distance import cosine
 from scipy.special import softmax
 
@@ -114,11 +115,10 @@ def test_anchor_immutable_and_memory_bounded():
             assert np.all(mut >= T) and np.all(np.diff(mut) > 0)
 
 
-def _kept_set_check():
+def _kept_set_check(T=20, H=3, D=16, K=30, frames=7, seed=3):
     # brute force on one head: candidates = previous kept + new frame, scored by scipy
-    T, H, D, K = 20, 3, 16, 30
     prev = {h: (np.zeros(0, int), np.zeros((0, D))) for h in range(H)}
-    for t, orc, (q, k, v), _ in _stream(T=T, H=H, D=D, K=K):
+    for t, orc, (q, k, v), _ in _stream(T=T, H=H, D=D, K=K, frames=frames, seed=seed):
         if t == 0:
             continue
         for h in range(H):
@@ -133,6 +133,15 @@ def _kept_set_check():
 
 def test_kept_set_is_top_k_of_candidates_each_frame():
     _kept_set_check()
+
+
+@settings(max_examples=20, deadline=None, derandomize=True)
+@given(T=st.integers(1, 24), H=st.integers(1, 3), D=st.sampled_from([4, 8, 16]), K=st.integers(1, 60),
+       frames=st.integers(2, 8), seed=st.integers(0, 1000))
+def test_kept_set_is_top_k_swept(T, H, D, K, frames, seed):
+    """The kept set against brute-force Top-K by scipy cosine over frame sizes (a frame
+    smaller and larger than K), head counts, head dims, budgets and stream lengths."""
+    _kept_set_check(T=T, H=H, D=D, K=K, frames=frames, seed=seed)
 
 
 def _ties_check():
