@@ -6,6 +6,7 @@ from fractions import Fraction
 
 import numpy as np
 import pytest
+from hypothesis import given, settings, strategies as st
 
 from kvc_streams import WORKLOADS
 from oracle import OracleConfig, StreamOracle, to_f32
@@ -72,11 +73,23 @@ def test_opposite_ranks_over_two_layers_give_cons_zero():
 
 
 def test_sigma_matches_library_population_variance():
-    rng = np.random.default_rng(1)
-    T = 40
-    orc = _orc(T, lam=0.5, window=5)
+    _sigma_check(T=40, window=5, lam=0.5, layers=8, seed=1)
+
+
+@settings(max_examples=25, deadline=None, derandomize=True)
+@given(T=st.integers(2, 60), window=st.integers(1, 8), lam=st.sampled_from([0.0, 0.25, 0.5, 1.0]),
+       layers=st.integers(1, 10), seed=st.integers(0, 1000))
+def test_sigma_matches_library_population_variance_swept(T, window, lam, layers, seed):
+    """The same check over frame sizes, rank windows (shorter and longer than the layer
+    count), consistency weights and seeds."""
+    _sigma_check(T=T, window=window, lam=lam, layers=layers, seed=seed)
+
+
+def _sigma_check(T, window, lam, layers, seed):
+    rng = np.random.default_rng(seed)
+    orc = _orc(T, lam=lam, window=window, layers=max(layers, 1))
     ranks = []
-    for l in range(8):
+    for l in range(layers):
         r = rng.standard_normal((T, 8))
         s = to_f32(np.sqrt((r * r).sum(axis=1)))
         # library ranking: stable argsort of -s gives ties to the lower index
@@ -84,13 +97,13 @@ def test_sigma_matches_library_population_variance():
         R = np.empty(T, int); R[order] = np.arange(T)
         ranks.append(R)
         sh = orc.score(l, 0, r)
-        win = ranks[max(0, l - 4): l + 1]
+        win = ranks[max(0, l - window + 1): l + 1]
         for i in range(T):
             vals = [Fraction(int(w[i]), T - 1) for w in win]
             var = statistics.pvariance(vals)                       # exact rational variance
             sigma = math.sqrt(var)
             cons = max(0.0, 1.0 - sigma * math.sqrt(12.0))
-            want = float(s[i]) * (1.0 + 0.5 * cons)
+            want = float(s[i]) * (1.0 + lam * cons)
             # the oracle evaluates sigma from the exact integer D in its own order;
             # agree to fp32 rounding of nearly equal fp64 values
             assert abs(sh[i] - want) <= 2 ** -22 * abs(want), (l, i, sh[i], want)
