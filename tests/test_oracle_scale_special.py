@@ -3,6 +3,7 @@
 explicitly concatenated tokens rebuilt from the definitions, not from the oracle's pages."""
 import numpy as np
 import pytest
+from hypothesis import given, settings, strategies as st
 
 import brute
 from oracle import OracleConfig, StreamOracle
@@ -105,6 +106,16 @@ def _special_tokens_check(T, P, ns, cap, S, W):
 
 @pytest.mark.parametrize("T,P,ns,cap,S,W", SPECIAL_CASES)
 def test_special_tokens_outlive_their_frames(T, P, ns, cap, S, W):
+    _special_tokens_check(T, P, ns, cap, S, W)
+
+
+@settings(max_examples=25, deadline=None, derandomize=True)
+@given(T=st.integers(1, 40), P=st.sampled_from([1, 2, 4, 8, 16]), ns_frac=st.floats(0.0, 1.0),
+       cap=st.integers(1, 6), S=st.integers(0, 3), W=st.integers(1, 5))
+def test_special_tokens_outlive_their_frames_swept(T, P, ns_frac, cap, S, W):
+    """The same check over frame and page sizes (special tokens within one page, across
+    pages, the whole frame), FIFO caps, scale frames and windows."""
+    ns = max(1, min(T, round(ns_frac * T)))
     _special_tokens_check(T, P, ns, cap, S, W)
 
 
