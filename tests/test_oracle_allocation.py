@@ -10,6 +10,7 @@ written into page-aligned storage); "How GCTStream ...", Sliding Window Eviction
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings, strategies as st
 
 from kvc_streams import WORKLOADS, FrameStream
 from oracle import OracleConfig, StreamOracle
@@ -138,3 +139,45 @@ def test_planted_never_reuse_is_caught_by_compaction(monkeypatch):
     monkeypatch.setattr(StreamOracle, "_alloc", _never_reuse)
     with pytest.raises(AssertionError):
         _budget_check()
+
+
+def _window_model(T, P, S, W, keys):
+    """Page tables of a window stream by a direct model of the reading: a frame takes the
+    ppf lowest free ids; a committed keyframe keeps the first S and last W committed
+    frames and frees the others' pages; a non-keyframe frees its own after attending."""
+    ppf = -(-T // P)
+    valid = [P] * (ppf - 1) + [T - (ppf - 1) * P]
+    free, committed, tables = set(range(10 ** 4)), [], []
+    for t, key in enumerate(keys):
+        phys = sorted(free)[:ppf]
+        free -= set(phys)
+        if key:
+            committed.append((t, phys))
+            keep = committed[:S] + [c for c in committed[-W:] if c not in committed[:S]]
+            for c in committed:
+                if c not in keep:
+                    free |= set(c[1])
+            committed = [c for c in committed if c in keep]
+        else:
+            free |= set(phys)
+        tables.append([[f, g, ph[g], valid[g]] for f, ph in sorted(committed) for g in range(ppf)])
+    return tables
+
+
+@settings(max_examples=25, deadline=None, derandomize=True)
+@given(T=st.integers(1, 30), P=st.sampled_from([1, 2, 4, 8, 16]), S=st.integers(0, 3), W=st.integers(1, 4),
+       keys=st.lists(st.booleans(), min_size=1, max_size=14))
+def test_window_stream_pages_match_a_direct_model(T, P, S, W, keys):
+    """The oracle's page tables over window streams with random keyframe flags (frames
+    that evict, free pages that are reused, skip-append frames) against the direct model
+    of the lowest-free reading."""
+    wl = WORKLOADS["tiny_f32"].replace(tokens_per_frame=T, page_size=P, window_frames=W, scale_frames=S,
+                                       num_heads=1, head_dim=4)
+    st_ = FrameStream(wl, seed=T + 100 * P, device="cpu")
+    orc = StreamOracle(OracleConfig.from_workload(wl))
+    want = _window_model(T, P, S, W, keys)
+    for t, key in enumerate(keys):
+        q, k, v = (_np(x) for x in st_.frame(0, t))
+        orc.append(0, t, k, v, key)
+        orc.attend(0, q)
+        assert orc.page_table(0).tolist() == want[t], t
