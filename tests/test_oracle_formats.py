@@ -7,6 +7,7 @@ import struct
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings, strategies as st
 
 from oracle import bf16_round, e4m3_encode, e4m3_decode, fp8_quantise_block, to_f32
 
@@ -95,6 +96,21 @@ def test_fp8_block_error_bound():
     # subnormal floor of half of 2^-9 * scale
     bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * scale) * (1 + 1e-6)
     assert np.all(np.abs(deq - x) <= bound)
+
+
+@settings(max_examples=30, deadline=None, derandomize=True)
+@given(rows=st.integers(1, 16), cols=st.integers(1, 128), log2_mag=st.integers(-40, 40),
+       outlier=st.floats(1.0, 1e4), seed=st.integers(0, 10 ** 6))
+def test_fp8_block_matches_torch_float8_swept(rows, cols, log2_mag, outlier, seed):
+    """Per-block absmax E4M3 quantisation against torch's float8 cast with an fp32 scale,
+    over block shapes, magnitudes from 2^-40 to 2^40 (bf16 cache inputs) and outliers."""
+    import brute
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows, cols)) * 2.0 ** log2_mag
+    x.flat[rng.integers(x.size)] *= outlier
+    x = bf16_round(x)
+    _, _, deq = fp8_quantise_block(x)
+    np.testing.assert_array_equal(deq, brute.fp8_dequant_torch(x))
 
 
 # ---- dimension-adaptive FP8 ("XStreamVGGT" abstract; K per channel, V per token)
