@@ -205,7 +205,8 @@ KVC_API kvc_status kvc_append_frame_all(kvc_cache* c, int32_t frame_idx, const v
  * while |softmax_scale * q . k| stays far below 2^20 the softmax keeps its full
  * resolution; logits of 2^24 and beyond (where fp32 cannot tell logits one unit apart)
  * are outside the supported range and may give non-finite outputs.
- * Errors: KVC_ERR_STATE if nothing is pending. */
+ * Errors: KVC_ERR_ARG (bad layer, NULL or non-16-byte-aligned Q or O), KVC_ERR_STATE
+ * (nothing pending on the layer), KVC_ERR_CUDA (a launch failed). */
 KVC_API kvc_status kvc_attend(kvc_cache* c, int32_t layer, const void* q_dev, void* o_dev);
 
 /* kvc_attend on every layer, in layer order: q_devs[l] and o_devs[l] are layer l's
@@ -269,13 +270,17 @@ KVC_API kvc_status kvc_compress_all(kvc_cache* c, const float* const* residual_d
  * (owner, page_in_owner, phys_page, valid_tokens) in cache order; owner is the
  * frame index, or -1 for pages written by compaction. Writes at most
  * `capacity` rows; *n_rows receives the full count. `info` (may be NULL)
- * receives the layer's statistics. */
+ * receives the layer's statistics. Errors: KVC_ERR_ARG (bad layer), KVC_ERR_CUDA,
+ * and a device-side failure latched earlier (KVC_ERR_TIMEOUT, KVC_ERR_DEVICE). */
 KVC_API kvc_status kvc_page_table(kvc_cache* c, int32_t layer, int32_t* rows_host, int32_t capacity,
                           int32_t* n_rows, kvc_info* info);
 
 /* Synchronise and copy per-token metadata of `layer` in cache order: token id
  * (frame * T + slot), merge count, and enhanced score s_hat. Any output pointer
- * may be NULL. */
+ * may be NULL; at most `capacity` tokens are written and *n_out receives the full count.
+ * Errors: KVC_ERR_ARG (bad layer), KVC_ERR_UNSUPPORTED (no token budget: no metadata),
+ * KVC_ERR_STATE (per-head page lists), KVC_ERR_DEVICE (a page-table row outside the
+ * pool), KVC_ERR_CUDA, and a device-side failure latched earlier. */
 KVC_API kvc_status kvc_token_meta(kvc_cache* c, int32_t layer, int64_t* ids_host, int32_t* counts_host,
                           float* shat_host, int32_t capacity, int32_t* n_out);
 
@@ -287,14 +292,18 @@ KVC_API kvc_status kvc_token_meta(kvc_cache* c, int32_t layer, int64_t* ids_host
 KVC_API kvc_status kvc_last_raw_scores(kvc_cache* c, float* s_host, int32_t capacity, int32_t* n_out);
 
 /* Synchronise and copy the (source id, target id) pairs of the last
- * compression of `layer`, in ascending source id. */
+ * compression of `layer`, in ascending source id. At most `capacity` pairs are written;
+ * *n_out receives the full count. Errors: KVC_ERR_ARG (bad layer, budget_tokens is 0),
+ * KVC_ERR_CUDA. */
 KVC_API kvc_status kvc_last_merge(kvc_cache* c, int32_t layer, int64_t* src_host, int64_t* dst_host,
                           int32_t capacity, int32_t* n_out);
 
 /* Synchronise and copy the raw pool contents of page-table rows
  * [first_row, first_row + n_rows) of `layer`: K and V pages as stored
  * ([H][P][D] per page, storage dtype; FP8: codes), and for FP8 the per-(page,
- * head) scales [n_rows][H] fp32 (scale pointers may be NULL otherwise). */
+ * head) scales [n_rows][H] fp32 (scale pointers may be NULL otherwise). Errors:
+ * KVC_ERR_ARG (bad layer, rows outside the page table), KVC_ERR_STATE (per-head page
+ * lists), KVC_ERR_CUDA, and a device-side failure latched earlier. */
 KVC_API kvc_status kvc_export_pages(kvc_cache* c, int32_t layer, int32_t first_row, int32_t n_rows,
                             void* k_host, void* v_host, float* k_scale_host, float* v_scale_host);
 
@@ -308,7 +317,9 @@ KVC_API kvc_status kvc_export_fp8_group_scales(kvc_cache* c, int32_t layer, int3
 /* One whole frame step of `layer` from HOST buffers: copy q, k, v [T, H, D]
  * host -> device, append, attend (+ commit/evict), copy O device -> host,
  * and wait for the copy. Pinned host memory gives full copy bandwidth. Caches that hold
- * a head range (model_heads > num_heads) are refused with KVC_ERR_ARG. */
+ * a head range (model_heads > num_heads) are refused with KVC_ERR_ARG. Errors: those of
+ * kvc_append_frame and kvc_attend, KVC_ERR_ARG (a NULL host buffer), KVC_ERR_CUDA (a
+ * copy), and a device-side failure latched by this or an earlier step. */
 KVC_API kvc_status kvc_step_host(kvc_cache* c, int32_t layer, int32_t frame_idx, int32_t is_keyframe,
                          const void* q_host, const void* k_host, const void* v_host, void* o_host);
 

@@ -1391,8 +1391,14 @@ extern "C" kvc_status kvc_last_merge(kvc_cache* c, int32_t layer, int64_t* src_h
   const int n = c->L[layer].last_merge_n;
   const int m = std::min(n, capacity);
   if (m > 0) {
-    if (src_host) cudaMemcpy(src_host, sc.last_src + static_cast<size_t>(layer) * cp.n_merge, m * 8, cudaMemcpyDeviceToHost);
-    if (dst_host) cudaMemcpy(dst_host, sc.last_dst + static_cast<size_t>(layer) * cp.n_merge, m * 8, cudaMemcpyDeviceToHost);
+    if (src_host)
+      e = cudaMemcpy(src_host, sc.last_src + static_cast<size_t>(layer) * cp.n_merge, m * 8, cudaMemcpyDeviceToHost);
+    if (dst_host && e == cudaSuccess)
+      e = cudaMemcpy(dst_host, sc.last_dst + static_cast<size_t>(layer) * cp.n_merge, m * 8, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) {
+      c->last_error = std::string("kvc_last_merge copy: ") + cudaGetErrorString(e);
+      return KVC_ERR_CUDA;
+    }
   }
   if (n_out) *n_out = n;
   return KVC_OK;
