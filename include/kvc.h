@@ -152,12 +152,13 @@ KVC_API kvc_status kvc_create(const kvc_config* cfg, void* stream, kvc_cache** o
 /* Synchronise the stream and free everything the cache owns. NULL is a no-op. */
 KVC_API kvc_status kvc_destroy(kvc_cache* c);
 
-/* Change the stream used by later calls. */
+/* Change the stream used by later calls (work already enqueued stays on the old one:
+ * synchronise it first if later work must follow it). Errors: KVC_ERR_ARG (NULL cache). */
 KVC_API kvc_status kvc_set_stream(kvc_cache* c, void* stream);
 
 /* Empty every layer (page tables, free lists, rank history, counters) between
  * videos, keeping the pool memory ([GCT] Cache Initialization and Cleanup,
- * clean_kv_cache). Stream-ordered. */
+ * clean_kv_cache). Stream-ordered. Errors: KVC_ERR_ARG (NULL cache), KVC_ERR_CUDA. */
 KVC_API kvc_status kvc_reset(kvc_cache* c);
 
 /* Page-aligned append of frame `frame_idx` to `layer` ([LBM] Page-Aligned
