@@ -261,3 +261,14 @@ def test_binding_refuses_host_buffers_for_device_arguments():
             kvc.kvc_compress(0, 0, bad)
         with pytest.raises(TypeError):
             kvc.kvc_attend_paged_noalloc(bad, bad, bad, bad, 1, bad, 1, 1, 1, 64, 16, 0.125)
+
+
+@pytest.mark.parametrize("compiler,std,ext", [("gcc", "c99", "c"), ("g++", "c++17", "cpp")])
+def test_header_compiles_without_warnings(compiler, std, ext):
+    """include/kvc.h is plain C: it compiles warning-free under strict C99 and C++17."""
+    src = '#include "kvc.h"\nint main(void) { kvc_config c; (void)c; return (int)kvc_version(); }\n'
+    with tempfile.TemporaryDirectory() as d:
+        f = os.path.join(d, "hdr." + ext)
+        open(f, "w").write(src)
+        subprocess.run([compiler, "-std=" + std, "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-I", os.path.join(ROOT, "include"), "-c", f, "-o", os.path.join(d, "hdr.o")], check=True)
